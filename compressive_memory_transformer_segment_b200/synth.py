@@ -1,0 +1,111 @@
+"""Seeded synthetic inputs for the Infini-attention layer forward.
+
+This module is shared by the tests, the bench and the CPU oracle's callers.  It
+holds none of the method's arithmetic: it draws i.i.d. values from a seeded
+counter-based generator (NumPy's Philox) and rounds them to bf16 where the
+workload asks for bf16.
+
+Streams.  Every (tensor, batch, head) slice has its own Philox key
+(seed, stream id), so any slice can be regenerated alone (large workloads are
+checked on sampled heads) and generation parallelises over threads without
+changing the values.
+"""
+
+from concurrent.futures import ThreadPoolExecutor
+import os
+
+import numpy as np
+
+_T_Q, _T_K, _T_V, _T_BETA, _T_PAIR = 1, 2, 3, 4, 5
+
+
+def _stream(seed, tensor, b=0, h=0):
+    return np.random.Generator(
+        np.random.Philox(key=[int(seed), (tensor << 40) | (b << 20) | h]))
+
+
+def round_bf16_bits(x):
+    """Round float32 values to bf16 (round to nearest even); return uint16 bits.
+
+    NaN is not produced by the generators, so no NaN handling is needed.
+    """
+    u = np.ascontiguousarray(x, dtype=np.float32).view(np.uint32)
+    bias = ((u >> 16) & 1) + np.uint32(0x7FFF)
+    return ((u + bias) >> 16).astype(np.uint16)
+
+
+def bf16_bits_to_f32(bits):
+    """Exact float32 values of bf16 bit patterns."""
+    return (np.asarray(bits, dtype=np.uint16).astype(np.uint32) << 16).view(np.float32)
+
+
+def _normal_slice(seed, tensor, b, h, n, d, bf16):
+    x = _stream(seed, tensor, b, h).standard_normal((n, d), dtype=np.float32)
+    if bf16:
+        return round_bf16_bits(x)
+    return x
+
+
+def normal_tensor(seed, tensor, B, H, L, d, bf16, threads=None, heads=None):
+    """[B, H, L, d] i.i.d. N(0, 1): uint16 bf16 bits if ``bf16`` else float32.
+
+    ``heads`` limits generation to the listed head indices (others stay 0).
+    """
+    out = np.zeros((B, H, L, d), dtype=np.uint16 if bf16 else np.float32)
+    jobs = [(b, h) for b in range(B) for h in range(H)
+            if heads is None or h in heads]
+
+    def work(bh):
+        b, h = bh
+        out[b, h] = _normal_slice(seed, tensor, b, h, L, d, bf16)
+
+    n = threads or min(32, os.cpu_count() or 1)
+    with ThreadPoolExecutor(max_workers=n) as ex:
+        list(ex.map(work, jobs))
+    return out
+
+
+def make_inputs(cfg, seed=None, heads_q=None, heads_kv=None):
+    """Inputs for one workload configuration (see ``configs.py``).
+
+    Returns a dict with
+      q, k, v : uint16 bf16 bits [B,H,L,d] when cfg.dtype == 'bf16', else float32
+      beta    : float32 [H_q], U(-beta_range, beta_range)
+      M_in    : float32 [B,H_kv,d_k,d_v] zeros;  z_in: float32 [B,H_kv,d_k] zeros
+    and, for workloads with an inserted key/value pair, 'pair_pos'.
+    ``heads_q`` / ``heads_kv`` restrict which head slices are drawn.
+    """
+    seed = cfg.seed if seed is None else seed
+    bf16 = cfg.dtype == "bf16"
+    q = normal_tensor(seed, _T_Q, cfg.B, cfg.H_q, cfg.L, cfg.d_k, bf16, heads=heads_q)
+    k = normal_tensor(seed, _T_K, cfg.B, cfg.H_kv, cfg.L, cfg.d_k, bf16, heads=heads_kv)
+    v = normal_tensor(seed, _T_V, cfg.B, cfg.H_kv, cfg.L, cfg.d_v, bf16, heads=heads_kv)
+    beta = _stream(seed, _T_BETA).uniform(-cfg.beta_range, cfg.beta_range,
+                                          size=cfg.H_q).astype(np.float32)
+    res = dict(q=q, k=k, v=v, beta=beta,
+               M_in=np.zeros((cfg.B, cfg.H_kv, cfg.d_k, cfg.d_v), np.float32),
+               z_in=np.zeros((cfg.B, cfg.H_kv, cfg.d_k), np.float32))
+    if cfg.insert_pair:
+        # One fixed key/value pair, drawn from its own stream, placed at token
+        # 2*S + 1000 (inside the third segment) of every (batch, KV head); the
+        # query at the last position of every query head is set to that key.
+        g = _stream(seed, _T_PAIR)
+        ks = g.standard_normal(cfg.d_k, dtype=np.float32)
+        vs = g.standard_normal(cfg.d_v, dtype=np.float32)
+        if bf16:
+            ks, vs = round_bf16_bits(ks), round_bf16_bits(vs)
+        p = 2 * cfg.seg_len + 1000
+        if p >= cfg.L:
+            raise ValueError("inserted pair lies beyond the sequence")
+        k[:, :, p, :] = ks
+        v[:, :, p, :] = vs
+        q[:, :, cfg.L - 1, :] = ks
+        res["pair_pos"] = p
+    return res
+
+
+def as_float64(x, dtype):
+    """Exact float64 values of a generated tensor (bf16 bits or float32)."""
+    if dtype == "bf16":
+        return bf16_bits_to_f32(x).astype(np.float64)
+    return np.asarray(x, dtype=np.float64)

@@ -1,0 +1,30 @@
+"""Float64 CPU oracle for the Infini-attention layer forward pass.
+
+TEST INFRASTRUCTURE ONLY.  Nothing in the product path (the CUDA library, its
+Python binding, the package) imports, calls or links anything in this folder.
+Only ``tests/``, ``__graft_entry__.smoke()`` and the ``cpu_baseline`` /
+``--impl reference`` legs of ``bench.py`` may use it.
+
+The oracle shares no code with the CUDA path.  Both sides consume the same
+seeded inputs, produced by ``compressive_memory_transformer_segment_b200.synth``,
+which holds none of the method's arithmetic.
+
+Pinned functions (each is checked in ``tests/test_oracle_pins.py`` against a
+library routine, a closed form, brute force or an invariant):
+  elu_plus_one, gate_sigmoid, local_causal_attention, memory_retrieval,
+  memory_update (linear and delta), infini_attention_forward, scan_states,
+  segment_output.
+No function here is "parity unpinned".
+"""
+
+from .infini_oracle import (  # noqa: F401
+    elu_plus_one,
+    gate_sigmoid,
+    local_causal_attention,
+    memory_retrieval,
+    memory_update,
+    segment_bounds,
+    scan_states,
+    segment_output,
+    infini_attention_forward,
+)
