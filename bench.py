@@ -1,0 +1,395 @@
+"""Benchmark of the Infini-attention layer forward on B200.
+
+One step = one infini_attn_forward over one batch of the workload (local
+attention, retrieval, gate and memory update for every segment), inputs
+resident in HBM.  Prints one JSON line on rank 0.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--config NAME] [--impl reference]
+
+Multi-GPU (launched by torchrun, one process per GPU): the work shards over
+independent (batch, KV head) chains with no data-path collective, so every
+rank runs its own full batch of the workload (weak scaling) and the value is
+all ranks' tokens over the slowest rank's device time.
+
+``--impl reference`` times the float64 CPU oracle on a bounded sample of the
+same workload, on the host cores.
+"""
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from compressive_memory_transformer_segment_b200 import configs, synth  # noqa: E402
+
+METRIC = "Infini-attention fwd tokens/s on 1 B200; % of bf16 tensor-core peak"
+DEFAULT_CONFIG = "8b-delta"
+L2_BYTES = 126 * 1024 * 1024
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return p, "measured"
+    except (OSError, ValueError):
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+def host_cores():
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count() or 1
+
+
+# ---------------------------------------------------------------- oracle timing
+
+def oracle_sample(w, budget_s):
+    """Time the float64 oracle on whole KV chains (each with all query heads of
+    its group), segment by segment, until about ``budget_s`` seconds have passed.
+
+    Returns (token-equivalents/s, description, seconds).  One token of the
+    workload needs all H_kv chains, so r rows of one chain count as r/H_kv tokens.
+    """
+    import oracle  # the CPU baseline is the only product-adjacent use of the oracle
+
+    g = w.H_q // w.H_kv
+    beta = synth.make_beta(w)
+    chains = [(b, j) for b in range(w.B) for j in range(w.H_kv)]
+    rows = 0
+    nseg = 0
+    used = []
+    elapsed = 0.0
+    for b, j in chains:
+        kc = synth.as_float64(synth.make_head(w, "k", b, j), w.dtype)
+        vc = synth.as_float64(synth.make_head(w, "v", b, j), w.dtype)
+        heads = range(j * g, (j + 1) * g)
+        qs = {h: synth.as_float64(synth.make_head(w, "q", b, h), w.dtype) for h in heads}
+        used.append((b, j))
+        t0 = time.perf_counter()
+        scan = oracle.scan_states(kc, vc, np.zeros((w.d_k, w.d_v)), np.zeros(w.d_k),
+                                  w.seg_len, w.rule)
+        for s, r0, r1, M, z in scan:
+            if r0 == r1:
+                break
+            for h in heads:
+                oracle.segment_output(qs[h][r0:r1], kc[r0:r1], vc[r0:r1], M, z, float(beta[h]))
+            rows += r1 - r0
+            nseg += 1
+            if elapsed + time.perf_counter() - t0 >= budget_s:
+                next(scan)  # the generator applies this segment's memory update on resume
+                break
+        elapsed += time.perf_counter() - t0
+        if elapsed >= budget_s:
+            break
+    tokens = rows / w.H_kv
+    desc = (f"oracle (NumPy float64), {len(used)} (batch, KV head) chain(s) from {used[0]}, "
+            f"each with its {g} query head(s): {nseg} segment(s) of up to {w.seg_len} rows "
+            f"({rows} rows) in {elapsed:.2f} s of compute (input generation untimed); "
+            f"token-equivalents = rows / H_kv")
+    return tokens / elapsed, desc, elapsed
+
+
+def run_reference(args, w):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    budget = max(1.0, args.reference_budget / max(1, args.steps + args.warmup))
+    for _ in range(args.warmup):
+        oracle_sample(w, budget)
+    vals, descs, times = [], [], []
+    for _ in range(args.steps):
+        v, d, dt = oracle_sample(w, budget)
+        vals.append(v)
+        descs.append(d)
+        times.append(dt)
+    value = statistics.median(vals)
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1000.0 * statistics.median(times), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": config_dict(w, args.gpus, None),
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": host_cores(),
+                         "kind": "oracle", "sample": descs[-1]},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ---------------------------------------------------------------- GPU arm
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_rank{gpu_index}.csv")
+
+    def __enter__(self):
+        try:
+            os.makedirs(os.path.dirname(self.path), exist_ok=True)
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=self.f, stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+            self.f.close()
+
+    def summary(self):
+        if self.proc is None or not os.path.exists(self.path):
+            return None
+        sm, smax, reasons = [], [], set()
+        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+        for line in open(self.path):
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax.append(float(parts[2]))
+            except ValueError:
+                continue
+            for name, flag in zip(names, parts[5:9]):
+                if flag.lower().startswith("active"):
+                    reasons.add(name)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(smax),
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def config_dict(w, n_gpus, l2_note):
+    d = {"workload": w.name, "B": w.B, "H_q": w.H_q, "H_kv": w.H_kv, "L": w.L,
+         "d_k": w.d_k, "d_v": w.d_v, "seg_len": w.seg_len, "T": w.T, "rule": w.rule,
+         "io_dtype": w.dtype, "state_dtype": "f32", "tokens_per_step_per_gpu": w.tokens,
+         "parallelism": f"dp{n_gpus} (independent (batch, KV head) chains, no collective)"}
+    if l2_note:
+        d["l2"] = l2_note
+    return d
+
+
+def run_gpu(args, w):
+    import torch
+    import torch.distributed as dist
+
+    from compressive_memory_transformer_segment_b200 import api
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    api.load_library()
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    # Inputs: seeded, generated on the host, copied once to HBM.
+    wr = w.with_(seed=w.seed + 7919 * rank)
+    inp = synth.make_inputs(wr)
+    tdt = torch.bfloat16 if w.dtype == "bf16" else torch.float32
+
+    def host_tensor(x):
+        if w.dtype == "bf16":
+            return torch.from_numpy(np.ascontiguousarray(x).view(np.int16)).view(torch.bfloat16)
+        return torch.from_numpy(np.ascontiguousarray(x, dtype=np.float32))
+
+    hq, hk, hv = (host_tensor(inp[n]) for n in ("q", "k", "v"))
+    q, k, v = (t.to(dev) for t in (hq, hk, hv))
+    beta = torch.from_numpy(inp["beta"]).to(dev)
+    M0, z0 = api.init_state(w.B, w.H_kv, w.d_k, w.d_v, device=dev)
+    out = torch.empty((w.B, w.H_q, w.L, w.d_v), dtype=tdt, device=dev)
+    M1 = torch.empty_like(M0)
+    z1 = torch.empty_like(z0)
+    dims = api.make_dims(w.B, w.H_q, w.H_kv, w.L, w.d_k, w.d_v, tdt)
+    plan = api.plan(dims, w.seg_len, w.rule)
+    ws = torch.empty(plan["workspace_bytes"], dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    in_bytes = sum(t.numel() * t.element_size() for t in (q, k, v))
+    flush = None
+    if in_bytes < 2 * L2_BYTES:
+        flush = torch.empty(2 * L2_BYTES, dtype=torch.uint8, device=dev)
+        l2_note = "L2 flushed (256 MiB write) between timed steps; each step timed alone"
+    else:
+        l2_note = f"inputs ({in_bytes / 2**20:.0f} MiB) larger than L2; steps timed back to back"
+
+    def step():
+        api.forward(q, k, v, beta, M0, z0, w.seg_len, w.rule, out=out, M_out=M1, z_out=z1,
+                    workspace=ws, stream=stream)
+
+    for _ in range(args.warmup):
+        step()
+    api.sync_status(stream)
+
+    api.set_kernel_timing(True)
+    api.kernel_times(reset=True)
+    barrier()
+    torch.cuda.synchronize(dev)
+    with ClockSampler(local) as clocks:
+        if flush is None:
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            for _ in range(args.steps):
+                step()
+            e1.record(stream)
+            torch.cuda.synchronize(dev)
+            elapsed_ms = e0.elapsed_time(e1)
+        else:
+            elapsed_ms = 0.0
+            for _ in range(args.steps):
+                flush.fill_(1)
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                e0.record(stream)
+                step()
+                e1.record(stream)
+                torch.cuda.synchronize(dev)
+                elapsed_ms += e0.elapsed_time(e1)
+    barrier()
+    torch.cuda.synchronize(dev)
+    api.set_kernel_timing(False)
+    ktimes = api.kernel_times(reset=True)
+    api.sync_status(stream)
+
+    t = torch.tensor([elapsed_ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    max_ms = float(t.item())
+    tokens = w.tokens * args.steps * world
+    value = tokens / (max_ms / 1000.0)
+
+    # End to end through the C ABI with host buffers (pinned), copies inside.
+    hq_p, hk_p, hv_p = (x.pin_memory() for x in (hq, hk, hv))
+    hbeta = torch.from_numpy(inp["beta"]).pin_memory()
+    hM0 = torch.zeros(M0.shape, dtype=torch.float32).pin_memory()
+    hz0 = torch.zeros(z0.shape, dtype=torch.float32).pin_memory()
+    hout = torch.empty(out.shape, dtype=tdt).pin_memory()
+    hM1 = torch.empty(M0.shape, dtype=torch.float32).pin_memory()
+    hz1 = torch.empty(z0.shape, dtype=torch.float32).pin_memory()
+    arena = torch.empty(api.host_arena_bytes(dims, w.seg_len, w.rule), dtype=torch.uint8, device=dev)
+    del ws
+    e2e_steps = max(1, min(args.steps, 5))
+
+    def e2e_step():
+        api.forward_host(hq_p, hk_p, hv_p, hbeta, hM0, hz0, w.seg_len, w.rule, hout, hM1, hz1,
+                         arena, stream=stream)
+
+    e2e_step()
+    torch.cuda.synchronize(dev)
+    barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    te = torch.tensor([e0.elapsed_time(e1)], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(te, op=dist.ReduceOp.MAX)
+    e2e_value = w.tokens * e2e_steps * world / (float(te.item()) / 1000.0)
+    h2d = sum(x.numel() * x.element_size() for x in (hq_p, hk_p, hv_p, hbeta, hM0, hz0))
+    d2h = sum(x.numel() * x.element_size() for x in (hout, hM1, hz1))
+
+    if world > 1:
+        dist.destroy_process_group()
+    if rank != 0:
+        return 0
+
+    peaks, peak_src = load_peaks()
+    flops = configs.algorithmic_flops(w)
+    att_ms, att_n = ktimes["attention"]
+    scan_ms, scan_n = ktimes["state_scan"]
+    # Dominant kernel: the segment attention kernel (local attention, retrieval,
+    # gate).  Its algorithmic flops: every flop of the step except the update.
+    upd = w.B * w.H_kv * w.L * (2 * w.d_k * w.d_v + w.d_k)
+    if w.rule == "delta":
+        upd += w.B * w.H_kv * w.L * (2 * w.d_k * w.d_v + 2 * w.d_k)
+    att_flops = flops - upd
+    att_avg_s = (att_ms / max(att_n, 1)) / 1000.0
+    achieved = att_flops / att_avg_s / 1e12 if att_avg_s > 0 else 0.0
+    peak = peaks["bf16_tflops"]
+    step_ms = max_ms / args.steps
+    line = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": step_ms,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": w.dtype, "data": "synthetic (seeded Philox N(0,1) q/k/v, U(-r,r) beta)",
+        "config": config_dict(w, world, l2_note),
+        "path": plan["path"],
+        "tc_peak_frac_step": (flops / (step_ms / 1000.0)) / (peak * 1e12),
+        "clocks": clocks.summary(),
+        "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h, "steps": e2e_steps},
+        "gpu_launches": plan["launches"] * args.steps,
+        "roofline": {"bound": "tensor", "kernel": "segment attention", "achieved": achieved,
+                     "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
+                     "peak_source": f"{peak_src} bf16 burst", "traffic": None,
+                     "algorithmic_flops_per_launch": att_flops,
+                     "avg_launch_ms": att_avg_s * 1000.0},
+        "kernel_ms": {"attention": att_ms / max(att_n, 1), "state_scan": scan_ms / max(scan_n, 1)},
+    }
+    if args.cpu_baseline:
+        v, desc, _ = oracle_sample(w, args.cpu_budget)
+        line["cpu_baseline"] = {"value": v, "unit": "tokens/s", "cores": host_cores(),
+                                "kind": "oracle", "sample": desc}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--config", default=DEFAULT_CONFIG, choices=sorted(configs.WORKLOADS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", dest="cpu_baseline", action="store_false")
+    ap.add_argument("--cpu-budget", type=float, default=15.0,
+                    help="seconds of oracle work for the cpu_baseline sample")
+    ap.add_argument("--reference-budget", type=float, default=60.0,
+                    help="total seconds of oracle work for --impl reference")
+    args = ap.parse_args()
+    if args.warmup < 3 and args.impl == "ours":
+        args.warmup = 3
+    w = configs.WORKLOADS[args.config]
+    if args.impl == "reference":
+        return run_reference(args, w)
+    return run_gpu(args, w)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

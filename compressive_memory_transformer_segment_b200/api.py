@@ -1,0 +1,249 @@
+"""Thin Python binding of libinfini_attn.so (argument marshalling only).
+
+Every step of the layer runs in the library's CUDA kernels; this module only
+checks tensor metadata, builds the C structs and passes raw pointers and the
+current CUDA stream.  PyTorch provides device memory and streams.  There is no
+fallback: if the library is missing, every call raises.
+
+Names follow the C ABI in include/infini_attn.h.
+"""
+
+import ctypes
+import os
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libinfini_attn.so")
+
+RULES = {"linear": 0, "delta": 1}
+DTYPES = {torch.bfloat16: 0, torch.float32: 1}
+PATHS = {0: "simt", 1: "tcgen05"}
+
+OK = 0
+ERR_ARG, ERR_UNSUPPORTED, ERR_ALIAS, ERR_CUDA, ERR_TIMEOUT, ERR_WORKSPACE, ERR_ALIGN = (
+    -1, -2, -3, -4, -5, -6, -7)
+
+
+class Dims(ctypes.Structure):
+    _fields_ = [("B", ctypes.c_int), ("H_q", ctypes.c_int), ("H_kv", ctypes.c_int),
+                ("L", ctypes.c_int), ("d_k", ctypes.c_int), ("d_v", ctypes.c_int),
+                ("dtype", ctypes.c_int)]
+
+
+class Plan(ctypes.Structure):
+    _fields_ = [("path", ctypes.c_int), ("launches", ctypes.c_int),
+                ("num_segments", ctypes.c_int), ("workspace_bytes", ctypes.c_size_t)]
+
+
+class InfiniError(RuntimeError):
+    def __init__(self, status, message):
+        super().__init__(f"infini_attn status {status}: {message}")
+        self.status = status
+
+
+_lib = None
+
+# (name, restype, argtypes) for every entry point of include/infini_attn.h.
+_P = ctypes.c_void_p
+_SIGNATURES = [
+    ("infini_attn_version", ctypes.c_int, []),
+    ("infini_attn_status_string", ctypes.c_char_p, [ctypes.c_int]),
+    ("infini_attn_init_state", ctypes.c_int, [_P, _P, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                              ctypes.c_int, _P]),
+    ("infini_attn_workspace_bytes", ctypes.c_size_t, [ctypes.POINTER(Dims), ctypes.c_int, ctypes.c_int]),
+    ("infini_attn_plan", ctypes.c_int, [ctypes.POINTER(Dims), ctypes.c_int, ctypes.c_int,
+                                        ctypes.POINTER(Plan)]),
+    ("infini_attn_forward", ctypes.c_int, [_P, _P, _P, _P, _P, _P, ctypes.c_int, ctypes.c_int,
+                                           ctypes.POINTER(Dims), _P, _P, _P, _P, ctypes.c_size_t, _P]),
+    ("infini_attn_host_arena_bytes", ctypes.c_size_t, [ctypes.POINTER(Dims), ctypes.c_int, ctypes.c_int]),
+    ("infini_attn_forward_host", ctypes.c_int, [_P, _P, _P, _P, _P, _P, ctypes.c_int, ctypes.c_int,
+                                                ctypes.POINTER(Dims), _P, _P, _P, _P,
+                                                ctypes.c_size_t, _P]),
+    ("infini_attn_sync_status", ctypes.c_int, [_P]),
+    ("infini_attn_set_kernel_timing", ctypes.c_int, [ctypes.c_int]),
+    ("infini_attn_kernel_times", ctypes.c_int, [ctypes.POINTER(ctypes.c_double),
+                                                ctypes.POINTER(ctypes.c_int), ctypes.c_int,
+                                                ctypes.c_int]),
+]
+
+
+def load_library(path=None):
+    """Load the in-tree CUDA library (raises if it was not built)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    path = path or LIB_PATH
+    if not os.path.exists(path):
+        raise FileNotFoundError(
+            f"{path} is missing: build it with "
+            "`python -m compressive_memory_transformer_segment_b200.build`")
+    lib = ctypes.CDLL(path)
+    for name, res, args in _SIGNATURES:
+        fn = getattr(lib, name)
+        fn.restype = res
+        fn.argtypes = args
+    _lib = lib
+    return lib
+
+
+def exported_symbols():
+    return [name for name, _, _ in _SIGNATURES]
+
+
+def status_string(status):
+    return load_library().infini_attn_status_string(int(status)).decode()
+
+
+def _check(rc):
+    if rc != OK:
+        raise InfiniError(rc, status_string(rc))
+
+
+def _stream_handle(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def make_dims(B, H_q, H_kv, L, d_k, d_v, dtype):
+    return Dims(B, H_q, H_kv, L, d_k, d_v, DTYPES[dtype] if isinstance(dtype, torch.dtype) else dtype)
+
+
+def _dims_from(q, k, v):
+    if q.dim() != 4 or k.dim() != 4 or v.dim() != 4:
+        raise ValueError("q, k, v must be [B, H, L, d]")
+    B, H_q, L, d_k = q.shape
+    H_kv, d_v = k.shape[1], v.shape[-1]
+    if tuple(k.shape) != (B, H_kv, L, d_k) or tuple(v.shape) != (B, H_kv, L, d_v):
+        raise ValueError("k must be [B, H_kv, L, d_k] and v [B, H_kv, L, d_v]")
+    if q.dtype not in DTYPES or k.dtype != q.dtype or v.dtype != q.dtype:
+        raise ValueError("q, k, v must share one dtype, bfloat16 or float32")
+    return make_dims(B, H_q, H_kv, L, d_k, d_v, q.dtype)
+
+
+def _rule(rule):
+    return RULES[rule] if isinstance(rule, str) else int(rule)
+
+
+def workspace_bytes(dims, seg_len, rule):
+    return load_library().infini_attn_workspace_bytes(ctypes.byref(dims), int(seg_len), _rule(rule))
+
+
+def plan(dims, seg_len, rule):
+    p = Plan()
+    _check(load_library().infini_attn_plan(ctypes.byref(dims), int(seg_len), _rule(rule),
+                                           ctypes.byref(p)))
+    return {"path": PATHS.get(p.path, p.path), "launches": p.launches,
+            "num_segments": p.num_segments, "workspace_bytes": p.workspace_bytes}
+
+
+def init_state(B, H_kv, d_k, d_v, device=None, stream=None):
+    """Allocate and zero (M, z) on the GPU through infini_attn_init_state."""
+    device = device or torch.device("cuda", torch.cuda.current_device())
+    M = torch.empty((B, H_kv, d_k, d_v), dtype=torch.float32, device=device)
+    z = torch.empty((B, H_kv, d_k), dtype=torch.float32, device=device)
+    _check(load_library().infini_attn_init_state(
+        ctypes.c_void_p(M.data_ptr()), ctypes.c_void_p(z.data_ptr()), B, H_kv, d_k, d_v,
+        _stream_handle(stream)))
+    return M, z
+
+
+def _dev(t, name, dtype=None, shape=None):
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if dtype is not None and t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def forward(q, k, v, beta, M_in, z_in, seg_len, rule, out=None, M_out=None, z_out=None,
+            workspace=None, stream=None):
+    """infini_attn_forward on CUDA tensors; returns (out, M_out, z_out).
+
+    Outputs are allocated when not given.  ``workspace`` is an optional uint8
+    CUDA tensor of at least workspace_bytes(...) bytes; without it the library
+    takes stream-ordered scratch itself.
+    """
+    lib = load_library()
+    dims = _dims_from(q, k, v)
+    B, H_q, L, H_kv, d_k, d_v = dims.B, dims.H_q, dims.L, dims.H_kv, dims.d_k, dims.d_v
+    if out is None:
+        out = torch.empty((B, H_q, L, d_v), dtype=q.dtype, device=q.device)
+    if M_out is None:
+        M_out = torch.empty((B, H_kv, d_k, d_v), dtype=torch.float32, device=q.device)
+    if z_out is None:
+        z_out = torch.empty((B, H_kv, d_k), dtype=torch.float32, device=q.device)
+    args = [_dev(q, "q"), _dev(k, "k"), _dev(v, "v"),
+            _dev(beta, "beta", torch.float32, (H_q,)),
+            _dev(M_in, "M_in", torch.float32, (B, H_kv, d_k, d_v)),
+            _dev(z_in, "z_in", torch.float32, (B, H_kv, d_k))]
+    outs = [_dev(out, "out", q.dtype, (B, H_q, L, d_v)),
+            _dev(M_out, "M_out", torch.float32, (B, H_kv, d_k, d_v)),
+            _dev(z_out, "z_out", torch.float32, (B, H_kv, d_k))]
+    if workspace is not None:
+        ws_ptr, ws_n = _dev(workspace, "workspace", torch.uint8), workspace.numel()
+    else:
+        ws_ptr, ws_n = ctypes.c_void_p(0), 0
+    _check(lib.infini_attn_forward(*args, int(seg_len), _rule(rule), ctypes.byref(dims), *outs,
+                                   ws_ptr, ws_n, _stream_handle(stream)))
+    return out, M_out, z_out
+
+
+def host_arena_bytes(dims, seg_len, rule):
+    return load_library().infini_attn_host_arena_bytes(ctypes.byref(dims), int(seg_len), _rule(rule))
+
+
+def _host(t, name, dtype=None, shape=None):
+    if not isinstance(t, torch.Tensor) or t.is_cuda or not t.is_contiguous():
+        raise ValueError(f"{name} must be a contiguous CPU tensor")
+    if dtype is not None and t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def forward_host(q, k, v, beta, M_in, z_in, seg_len, rule, out, M_out, z_out, arena,
+                 stream=None):
+    """infini_attn_forward_host: host tensors in and out (pinned for async
+    copies), device ``arena`` (uint8 CUDA tensor of host_arena_bytes(...))."""
+    lib = load_library()
+    dims = _dims_from(q, k, v)
+    B, H_q, L, H_kv, d_k, d_v = dims.B, dims.H_q, dims.L, dims.H_kv, dims.d_k, dims.d_v
+    args = [_host(q, "q"), _host(k, "k"), _host(v, "v"),
+            _host(beta, "beta", torch.float32, (H_q,)),
+            _host(M_in, "M_in", torch.float32, (B, H_kv, d_k, d_v)),
+            _host(z_in, "z_in", torch.float32, (B, H_kv, d_k))]
+    outs = [_host(out, "out", q.dtype, (B, H_q, L, d_v)),
+            _host(M_out, "M_out", torch.float32, (B, H_kv, d_k, d_v)),
+            _host(z_out, "z_out", torch.float32, (B, H_kv, d_k))]
+    _check(lib.infini_attn_forward_host(*args, int(seg_len), _rule(rule), ctypes.byref(dims), *outs,
+                                        _dev(arena, "arena", torch.uint8), arena.numel(),
+                                        _stream_handle(stream)))
+    return out, M_out, z_out
+
+
+def sync_status(stream=None):
+    """Wait for the stream; raise InfiniError(ERR_TIMEOUT) if a kernel gave up."""
+    _check(load_library().infini_attn_sync_status(_stream_handle(stream)))
+
+
+KERNEL_KINDS = ("state_scan", "attention")
+
+
+def set_kernel_timing(enable):
+    _check(load_library().infini_attn_set_kernel_timing(1 if enable else 0))
+
+
+def kernel_times(reset=True):
+    """{kind: (total ms, launches)} of the kernels timed since the last reset."""
+    n = len(KERNEL_KINDS)
+    ms = (ctypes.c_double * n)()
+    cnt = (ctypes.c_int * n)()
+    _check(load_library().infini_attn_kernel_times(ms, cnt, n, 1 if reset else 0))
+    return {KERNEL_KINDS[i]: (ms[i], cnt[i]) for i in range(n)}

@@ -1,0 +1,341 @@
+// C ABI of libinfini_attn.so: argument checks, workspace layout, kernel
+// dispatch.  The operation and every entry point are documented in
+// include/infini_attn.h.
+#include <cuda_runtime.h>
+#include <stdint.h>
+#include <string.h>
+
+#include <mutex>
+#include <vector>
+
+#include "infini_attn.h"
+#include "kernels.h"
+
+namespace infini {
+
+// Device status word: kernels OR in a bit when a bounded wait runs out.
+__device__ unsigned int g_status;
+
+namespace {
+
+constexpr size_t kAlign = 256;
+constexpr size_t kHeader = 256;
+
+size_t align_up(size_t x) { return (x + kAlign - 1) & ~(kAlign - 1); }
+
+bool head_dim_ok(int d) { return d == 32 || d == 64 || d == 128; }
+
+struct Shape {
+  int B, H_q, H_kv, L, d_k, d_v, S, T;
+  bool bf16, delta;
+  size_t elem;
+  size_t q_bytes, k_bytes, v_bytes, out_bytes, beta_bytes, M_bytes, z_bytes;
+  int path;
+  int launches;
+  // workspace layout
+  size_t ws_zpref, ws_mpref, ws_total;
+};
+
+int check_shape(const infini_dims_t* d, int seg_len, int rule, Shape* s) {
+  if (!d || !s) return INFINI_ERR_ARG;
+  if (d->B < 1 || d->H_q < 1 || d->H_kv < 1 || d->L < 1 || seg_len < 1) return INFINI_ERR_ARG;
+  if (d->H_q % d->H_kv != 0) return INFINI_ERR_ARG;
+  if (rule != INFINI_RULE_LINEAR && rule != INFINI_RULE_DELTA) return INFINI_ERR_ARG;
+  if (d->dtype != INFINI_DTYPE_BF16 && d->dtype != INFINI_DTYPE_F32) return INFINI_ERR_ARG;
+  if (!head_dim_ok(d->d_k) || !head_dim_ok(d->d_v)) return INFINI_ERR_UNSUPPORTED;
+  // Grid limits: (b, head) pairs index gridDim.y.
+  if ((long long)d->B * d->H_q > 65535) return INFINI_ERR_UNSUPPORTED;
+  s->B = d->B; s->H_q = d->H_q; s->H_kv = d->H_kv; s->L = d->L;
+  s->d_k = d->d_k; s->d_v = d->d_v;
+  s->S = seg_len;  // the last segment is simply shorter
+  s->T = (int)(((long long)d->L + seg_len - 1) / seg_len);
+  s->bf16 = d->dtype == INFINI_DTYPE_BF16;
+  s->delta = rule == INFINI_RULE_DELTA;
+  s->elem = s->bf16 ? 2 : 4;
+  const size_t BHq = (size_t)d->B * d->H_q, BHkv = (size_t)d->B * d->H_kv;
+  s->q_bytes = BHq * d->L * d->d_k * s->elem;
+  s->k_bytes = BHkv * d->L * d->d_k * s->elem;
+  s->v_bytes = BHkv * d->L * d->d_v * s->elem;
+  s->out_bytes = BHq * d->L * d->d_v * s->elem;
+  s->beta_bytes = (size_t)d->H_q * 4;
+  s->M_bytes = BHkv * d->d_k * d->d_v * 4;
+  s->z_bytes = BHkv * d->d_k * 4;
+  s->path = INFINI_PATH_SIMT;
+  s->launches = 2;
+  const size_t mpref_elem = 4;
+  s->ws_zpref = kHeader;
+  s->ws_mpref = align_up(s->ws_zpref + (size_t)s->T * BHkv * d->d_k * 4);
+  s->ws_total = align_up(s->ws_mpref + (size_t)s->T * BHkv * d->d_k * d->d_v * mpref_elem);
+  return INFINI_OK;
+}
+
+bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }
+
+struct Range {
+  uintptr_t lo, hi;
+};
+bool overlap(Range a, Range b) { return a.lo < b.hi && b.lo < a.hi; }
+Range rng(const void* p, size_t n) { return Range{(uintptr_t)p, (uintptr_t)p + n}; }
+
+// Optional per-kernel event timing (benchmarks only).
+constexpr int kKinds = 2;  // 0 = state scan, 1 = attention
+struct TimedLaunch {
+  int kind;
+  cudaEvent_t a, b;
+};
+std::mutex g_timing_mu;
+bool g_timing = false;
+std::vector<TimedLaunch> g_pending;
+std::vector<cudaEvent_t> g_event_pool;
+double g_ms[kKinds];
+int g_launches[kKinds];
+
+cudaEvent_t pooled_event() {
+  if (!g_event_pool.empty()) {
+    cudaEvent_t e = g_event_pool.back();
+    g_event_pool.pop_back();
+    return e;
+  }
+  cudaEvent_t e = nullptr;
+  if (cudaEventCreate(&e) != cudaSuccess) return nullptr;
+  return e;
+}
+
+// Runs `launch` on `st`, bracketed by events when timing is enabled.
+template <typename F>
+cudaError_t timed(int kind, cudaStream_t st, F&& launch) {
+  std::unique_lock<std::mutex> lock(g_timing_mu);
+  if (!g_timing) {
+    lock.unlock();
+    return launch();
+  }
+  cudaEvent_t a = pooled_event(), b = pooled_event();
+  if (!a || !b) return cudaErrorMemoryAllocation;
+  cudaError_t e = cudaEventRecord(a, st);
+  if (e == cudaSuccess) e = launch();
+  if (e == cudaSuccess) e = cudaEventRecord(b, st);
+  if (e == cudaSuccess) {
+    g_pending.push_back({kind, a, b});
+  } else {
+    g_event_pool.push_back(a);
+    g_event_pool.push_back(b);
+  }
+  return e;
+}
+
+unsigned int* status_ptr() {
+  void* p = nullptr;
+  if (cudaGetSymbolAddress(&p, g_status) != cudaSuccess) return nullptr;
+  return static_cast<unsigned int*>(p);
+}
+
+}  // namespace
+}  // namespace infini
+
+using namespace infini;
+
+extern "C" {
+
+int infini_attn_version(void) { return (1 << 16) | 0; }
+
+const char* infini_attn_status_string(int status) {
+  switch (status) {
+    case INFINI_OK: return "ok";
+    case INFINI_ERR_ARG: return "invalid argument (NULL pointer, size < 1, bad enum, H_q % H_kv != 0)";
+    case INFINI_ERR_UNSUPPORTED: return "unsupported shape (head dims must be 32, 64 or 128; B*H_q <= 65535)";
+    case INFINI_ERR_ALIAS: return "an output overlaps an input, another output or the workspace";
+    case INFINI_ERR_CUDA: return "a CUDA runtime call failed";
+    case INFINI_ERR_TIMEOUT: return "a kernel gave up a bounded wait (device status word set)";
+    case INFINI_ERR_WORKSPACE: return "workspace too small or not 256-byte aligned";
+    case INFINI_ERR_ALIGN: return "a pointer is not 16-byte aligned";
+    default: return "unknown status";
+  }
+}
+
+int infini_attn_init_state(float* M, float* z, int B, int H_kv, int d_k, int d_v, void* stream) {
+  if (!M || !z || B < 1 || H_kv < 1 || d_k < 1 || d_v < 1) return INFINI_ERR_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const size_t nM = (size_t)B * H_kv * d_k * d_v * sizeof(float);
+  const size_t nz = (size_t)B * H_kv * d_k * sizeof(float);
+  if (cudaMemsetAsync(M, 0, nM, st) != cudaSuccess) return INFINI_ERR_CUDA;
+  if (cudaMemsetAsync(z, 0, nz, st) != cudaSuccess) return INFINI_ERR_CUDA;
+  return INFINI_OK;
+}
+
+size_t infini_attn_workspace_bytes(const infini_dims_t* dims, int seg_len, int rule) {
+  Shape s;
+  if (check_shape(dims, seg_len, rule, &s) != INFINI_OK) return 0;
+  return s.ws_total;
+}
+
+int infini_attn_plan(const infini_dims_t* dims, int seg_len, int rule, infini_plan_t* plan) {
+  Shape s;
+  int rc = check_shape(dims, seg_len, rule, &s);
+  if (rc != INFINI_OK) return rc;
+  if (!plan) return INFINI_ERR_ARG;
+  plan->path = s.path;
+  plan->launches = s.launches;
+  plan->num_segments = s.T;
+  plan->workspace_bytes = s.ws_total;
+  return INFINI_OK;
+}
+
+int infini_attn_forward(const void* q, const void* k, const void* v, const float* beta,
+                        const float* M_in, const float* z_in, int seg_len, int rule,
+                        const infini_dims_t* dims, void* out, float* M_out, float* z_out,
+                        void* workspace, size_t workspace_bytes, void* stream) {
+  Shape s;
+  int rc = check_shape(dims, seg_len, rule, &s);
+  if (rc != INFINI_OK) return rc;
+  if (!q || !k || !v || !beta || !M_in || !z_in || !out || !M_out || !z_out) return INFINI_ERR_ARG;
+  const void* ptrs[] = {q, k, v, beta, M_in, z_in, out, M_out, z_out};
+  for (const void* p : ptrs)
+    if (!aligned16(p)) return INFINI_ERR_ALIGN;
+  if (workspace == nullptr && workspace_bytes != 0) return INFINI_ERR_ARG;
+  if (workspace != nullptr) {
+    if (workspace_bytes < s.ws_total || ((uintptr_t)workspace & (kAlign - 1)) != 0)
+      return INFINI_ERR_WORKSPACE;
+  }
+  // Aliasing: outputs may not overlap inputs or each other, except the
+  // in-place state (M_out == M_in, z_out == z_in exactly).
+  const Range r_out = rng(out, s.out_bytes), r_M = rng(M_out, s.M_bytes), r_z = rng(z_out, s.z_bytes);
+  const Range ins[] = {rng(q, s.q_bytes), rng(k, s.k_bytes), rng(v, s.v_bytes),
+                       rng(beta, s.beta_bytes), rng(M_in, s.M_bytes), rng(z_in, s.z_bytes)};
+  for (int i = 0; i < 6; ++i) {
+    if (overlap(r_out, ins[i])) return INFINI_ERR_ALIAS;
+    if (overlap(r_M, ins[i]) && !(i == 4 && M_out == M_in)) return INFINI_ERR_ALIAS;
+    if (overlap(r_z, ins[i]) && !(i == 5 && z_out == z_in)) return INFINI_ERR_ALIAS;
+  }
+  if (overlap(r_out, r_M) || overlap(r_out, r_z) || overlap(r_M, r_z)) return INFINI_ERR_ALIAS;
+  if (workspace) {
+    const Range r_ws = rng(workspace, s.ws_total);
+    if (overlap(r_ws, r_out) || overlap(r_ws, r_M) || overlap(r_ws, r_z)) return INFINI_ERR_ALIAS;
+    for (int i = 0; i < 6; ++i)
+      if (overlap(r_ws, ins[i])) return INFINI_ERR_ALIAS;
+  }
+
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  unsigned int* status = status_ptr();
+  if (!status) return INFINI_ERR_CUDA;
+  char* ws = static_cast<char*>(workspace);
+  bool owned = false;
+  if (!ws) {
+    if (cudaMallocAsync(reinterpret_cast<void**>(&ws), s.ws_total, st) != cudaSuccess)
+      return INFINI_ERR_CUDA;
+    owned = true;
+  }
+  Problem p;
+  p.q = q; p.k = k; p.v = v; p.beta = beta; p.M_in = M_in;
+  p.out = out; p.M_out = M_out; p.z_out = z_out;
+  p.B = s.B; p.H_q = s.H_q; p.H_kv = s.H_kv; p.L = s.L; p.d_k = s.d_k; p.d_v = s.d_v;
+  p.S = s.S; p.T = s.T; p.bf16 = s.bf16; p.delta = s.delta;
+  p.z_pref = reinterpret_cast<float*>(ws + s.ws_zpref);
+  p.M_pref = ws + s.ws_mpref;
+  p.status = status;
+
+  cudaError_t e = cudaMemcpyAsync(p.z_pref, z_in, s.z_bytes, cudaMemcpyDeviceToDevice, st);
+  if (e == cudaSuccess) e = timed(0, st, [&] { return launch_simt_state_scan(p, st); });
+  if (e == cudaSuccess) e = timed(1, st, [&] { return launch_simt_attention(p, st); });
+  if (owned) {
+    cudaError_t f = cudaFreeAsync(ws, st);
+    if (e == cudaSuccess) e = f;
+  }
+  return e == cudaSuccess ? INFINI_OK : INFINI_ERR_CUDA;
+}
+
+size_t infini_attn_host_arena_bytes(const infini_dims_t* dims, int seg_len, int rule) {
+  Shape s;
+  if (check_shape(dims, seg_len, rule, &s) != INFINI_OK) return 0;
+  return align_up(s.q_bytes) + align_up(s.k_bytes) + align_up(s.v_bytes) + align_up(s.beta_bytes) +
+         2 * align_up(s.M_bytes) + 2 * align_up(s.z_bytes) + align_up(s.out_bytes) + s.ws_total;
+}
+
+int infini_attn_forward_host(const void* q_h, const void* k_h, const void* v_h,
+                             const float* beta_h, const float* M_in_h, const float* z_in_h,
+                             int seg_len, int rule, const infini_dims_t* dims,
+                             void* out_h, float* M_out_h, float* z_out_h,
+                             void* arena, size_t arena_bytes, void* stream) {
+  Shape s;
+  int rc = check_shape(dims, seg_len, rule, &s);
+  if (rc != INFINI_OK) return rc;
+  if (!q_h || !k_h || !v_h || !beta_h || !M_in_h || !z_in_h || !out_h || !M_out_h || !z_out_h ||
+      !arena)
+    return INFINI_ERR_ARG;
+  if (arena_bytes < infini_attn_host_arena_bytes(dims, seg_len, rule) ||
+      ((uintptr_t)arena & (kAlign - 1)) != 0)
+    return INFINI_ERR_WORKSPACE;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  char* a = static_cast<char*>(arena);
+  size_t off = 0;
+  auto take = [&](size_t n) { char* p = a + off; off += align_up(n); return p; };
+  char* q = take(s.q_bytes);
+  char* k = take(s.k_bytes);
+  char* v = take(s.v_bytes);
+  float* beta = reinterpret_cast<float*>(take(s.beta_bytes));
+  float* M = reinterpret_cast<float*>(take(s.M_bytes));
+  float* z = reinterpret_cast<float*>(take(s.z_bytes));
+  float* M2 = reinterpret_cast<float*>(take(s.M_bytes));
+  float* z2 = reinterpret_cast<float*>(take(s.z_bytes));
+  char* out = take(s.out_bytes);
+  char* ws = a + off;
+  const struct { void* dst; const void* src; size_t n; } h2d[] = {
+      {q, q_h, s.q_bytes}, {k, k_h, s.k_bytes}, {v, v_h, s.v_bytes},
+      {beta, beta_h, s.beta_bytes}, {M, M_in_h, s.M_bytes}, {z, z_in_h, s.z_bytes}};
+  for (const auto& c : h2d)
+    if (cudaMemcpyAsync(c.dst, c.src, c.n, cudaMemcpyHostToDevice, st) != cudaSuccess)
+      return INFINI_ERR_CUDA;
+  rc = infini_attn_forward(q, k, v, beta, M, z, seg_len, rule, dims, out, M2, z2, ws, s.ws_total,
+                           stream);
+  if (rc != INFINI_OK) return rc;
+  if (cudaMemcpyAsync(out_h, out, s.out_bytes, cudaMemcpyDeviceToHost, st) != cudaSuccess ||
+      cudaMemcpyAsync(M_out_h, M2, s.M_bytes, cudaMemcpyDeviceToHost, st) != cudaSuccess ||
+      cudaMemcpyAsync(z_out_h, z2, s.z_bytes, cudaMemcpyDeviceToHost, st) != cudaSuccess)
+    return INFINI_ERR_CUDA;
+  return INFINI_OK;
+}
+
+int infini_attn_set_kernel_timing(int enable) {
+  std::lock_guard<std::mutex> lock(g_timing_mu);
+  g_timing = enable != 0;
+  return INFINI_OK;
+}
+
+int infini_attn_kernel_times(double* ms, int* launches, int n_kinds, int reset) {
+  if (!ms || !launches || n_kinds < 1) return INFINI_ERR_ARG;
+  std::lock_guard<std::mutex> lock(g_timing_mu);
+  for (const TimedLaunch& t : g_pending) {
+    float el = 0.f;
+    if (cudaEventSynchronize(t.b) != cudaSuccess) return INFINI_ERR_CUDA;
+    if (cudaEventElapsedTime(&el, t.a, t.b) != cudaSuccess) return INFINI_ERR_CUDA;
+    g_ms[t.kind] += el;
+    g_launches[t.kind] += 1;
+    g_event_pool.push_back(t.a);
+    g_event_pool.push_back(t.b);
+  }
+  g_pending.clear();
+  for (int k = 0; k < n_kinds; ++k) {
+    ms[k] = k < kKinds ? g_ms[k] : 0.0;
+    launches[k] = k < kKinds ? g_launches[k] : 0;
+  }
+  if (reset)
+    for (int k = 0; k < kKinds; ++k) {
+      g_ms[k] = 0.0;
+      g_launches[k] = 0;
+    }
+  return INFINI_OK;
+}
+
+int infini_attn_sync_status(void* stream) {
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (cudaStreamSynchronize(st) != cudaSuccess) return INFINI_ERR_CUDA;
+  unsigned int word = 0;
+  if (cudaMemcpyFromSymbol(&word, g_status, sizeof(word)) != cudaSuccess) return INFINI_ERR_CUDA;
+  if (word != 0) {
+    const unsigned int zero = 0;
+    if (cudaMemcpyToSymbol(g_status, &zero, sizeof(zero)) != cudaSuccess) return INFINI_ERR_CUDA;
+    return INFINI_ERR_TIMEOUT;
+  }
+  return INFINI_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,33 @@
+// Internal launcher declarations shared by the C-ABI layer and the kernels.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+namespace infini {
+
+// Problem description handed from the C-ABI layer to the launchers.
+struct Problem {
+  const void* q;
+  const void* k;
+  const void* v;
+  const float* beta;
+  const float* M_in;
+  void* out;
+  float* M_out;
+  float* z_out;
+  int B, H_q, H_kv, L, d_k, d_v, S, T;
+  bool bf16;
+  bool delta;
+  // Workspace views.
+  float* z_pref;       // [T][B*H_kv][d_k] f32: z_{s-1} read by segment s (slot 0 = z_in)
+  void* M_pref;        // [T][B*H_kv][d_k][d_v]: M_{s-1} (f32 on the SIMT path, bf16 on tcgen05)
+  unsigned int* status;  // device status word
+};
+
+// fp32 CUDA-core path (any S, any supported d, f32 or bf16 I/O).
+cudaError_t launch_simt_state_scan(const Problem& p, cudaStream_t stream);
+cudaError_t launch_simt_attention(const Problem& p, cudaStream_t stream);
+
+}  // namespace infini

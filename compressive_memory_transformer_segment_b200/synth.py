@@ -65,6 +65,42 @@ def normal_tensor(seed, tensor, B, H, L, d, bf16, threads=None, heads=None):
     return out
 
 
+_TENSOR_CODES = {"q": _T_Q, "k": _T_K, "v": _T_V}
+
+
+def _pair(cfg, seed):
+    g = _stream(seed, _T_PAIR)
+    ks = g.standard_normal(cfg.d_k, dtype=np.float32)
+    vs = g.standard_normal(cfg.d_v, dtype=np.float32)
+    if cfg.dtype == "bf16":
+        ks, vs = round_bf16_bits(ks), round_bf16_bits(vs)
+    p = 2 * cfg.seg_len + 1000
+    if p >= cfg.L:
+        raise ValueError("inserted pair lies beyond the sequence")
+    return p, {"k": ks, "v": vs, "q": ks}
+
+
+def make_head(cfg, name, b, h, seed=None):
+    """The [L, d] slice of tensor ``name`` ('q', 'k' or 'v') for batch row b
+    and head h, exactly as make_inputs would place it."""
+    seed = cfg.seed if seed is None else seed
+    d = cfg.d_v if name == "v" else cfg.d_k
+    x = _normal_slice(seed, _TENSOR_CODES[name], b, h, cfg.L, d, cfg.dtype == "bf16")
+    if cfg.insert_pair:
+        p, pair = _pair(cfg, seed)
+        if name == "q":
+            x[cfg.L - 1] = pair["q"]
+        else:
+            x[p] = pair[name]
+    return x
+
+
+def make_beta(cfg, seed=None):
+    seed = cfg.seed if seed is None else seed
+    return _stream(seed, _T_BETA).uniform(-cfg.beta_range, cfg.beta_range,
+                                          size=cfg.H_q).astype(np.float32)
+
+
 def make_inputs(cfg, seed=None, heads_q=None, heads_kv=None):
     """Inputs for one workload configuration (see ``configs.py``).
 
@@ -73,33 +109,29 @@ def make_inputs(cfg, seed=None, heads_q=None, heads_kv=None):
       beta    : float32 [H_q], U(-beta_range, beta_range)
       M_in    : float32 [B,H_kv,d_k,d_v] zeros;  z_in: float32 [B,H_kv,d_k] zeros
     and, for workloads with an inserted key/value pair, 'pair_pos'.
-    ``heads_q`` / ``heads_kv`` restrict which head slices are drawn.
+    ``heads_q`` / ``heads_kv`` restrict which head slices are drawn (others 0).
+
+    Inserted pair: one fixed key/value pair, drawn from its own stream, sits at
+    token 2*S + 1000 (inside the third segment) of every (batch, KV head), and
+    the query at the last position of every query head is set to that key.
     """
     seed = cfg.seed if seed is None else seed
     bf16 = cfg.dtype == "bf16"
     q = normal_tensor(seed, _T_Q, cfg.B, cfg.H_q, cfg.L, cfg.d_k, bf16, heads=heads_q)
     k = normal_tensor(seed, _T_K, cfg.B, cfg.H_kv, cfg.L, cfg.d_k, bf16, heads=heads_kv)
     v = normal_tensor(seed, _T_V, cfg.B, cfg.H_kv, cfg.L, cfg.d_v, bf16, heads=heads_kv)
-    beta = _stream(seed, _T_BETA).uniform(-cfg.beta_range, cfg.beta_range,
-                                          size=cfg.H_q).astype(np.float32)
-    res = dict(q=q, k=k, v=v, beta=beta,
+    res = dict(q=q, k=k, v=v, beta=make_beta(cfg, seed),
                M_in=np.zeros((cfg.B, cfg.H_kv, cfg.d_k, cfg.d_v), np.float32),
                z_in=np.zeros((cfg.B, cfg.H_kv, cfg.d_k), np.float32))
     if cfg.insert_pair:
-        # One fixed key/value pair, drawn from its own stream, placed at token
-        # 2*S + 1000 (inside the third segment) of every (batch, KV head); the
-        # query at the last position of every query head is set to that key.
-        g = _stream(seed, _T_PAIR)
-        ks = g.standard_normal(cfg.d_k, dtype=np.float32)
-        vs = g.standard_normal(cfg.d_v, dtype=np.float32)
-        if bf16:
-            ks, vs = round_bf16_bits(ks), round_bf16_bits(vs)
-        p = 2 * cfg.seg_len + 1000
-        if p >= cfg.L:
-            raise ValueError("inserted pair lies beyond the sequence")
-        k[:, :, p, :] = ks
-        v[:, :, p, :] = vs
-        q[:, :, cfg.L - 1, :] = ks
+        p, pair = _pair(cfg, seed)
+        hq = range(cfg.H_q) if heads_q is None else sorted(heads_q)
+        hk = range(cfg.H_kv) if heads_kv is None else sorted(heads_kv)
+        for h in hk:
+            k[:, h, p, :] = pair["k"]
+            v[:, h, p, :] = pair["v"]
+        for h in hq:
+            q[:, h, cfg.L - 1, :] = pair["q"]
         res["pair_pos"] = p
     return res
 

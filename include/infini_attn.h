@@ -1,0 +1,195 @@
+/*
+ * infini_attn.h -- C ABI of libinfini_attn.so, a B200 (sm_100a) implementation
+ * of the Infini-attention layer forward pass.
+ *
+ * The operation.  For every batch row b and query head h (KV head
+ * kv = floor(h / (H_q / H_kv))), the sequence of length L is cut into
+ * T = ceil(L / S) segments of S rows (the last may be shorter), scanned in
+ * order s = 1..T.  In segment s, with Q, K, V the segment's rows:
+ *   A_dot = softmax(Q K^T / sqrt(d_k) + causal mask (key j <= query i)) V
+ *   A_mem = sigma(Q) M_{s-1} / (sigma(Q) z_{s-1})  row-wise, 0 where the
+ *           denominator is exactly 0; sigma(x) = ELU(x) + 1
+ *   out   = sg(beta_h) A_mem + (1 - sg(beta_h)) A_dot,  sg = logistic
+ * and then the KV head's memory is updated with the segment's keys/values:
+ *   linear: M_s = M_{s-1} + sigma(K)^T V
+ *   delta : M_s = M_{s-1} + sigma(K)^T (V - sigma(K) M_{s-1} / (sigma(K) z_{s-1}))
+ *           (retrieval term 0 on rows whose denominator is 0)
+ *   both  : z_s = z_{s-1} + sum over the segment's rows of sigma(K)
+ * Only (M, z) pass from one segment to the next; after segment T they are
+ * returned as (M_out, z_out).
+ *
+ * Where this is defined:
+ *   "Hugging Face Infini-Attention 再現分析", section "Infini-Attention
+ *   メカニズム": Segmentation, Local Attention, Memory Retrieval (ELU + 1),
+ *   Integration (sigmoid of a learned per-head beta), Memory Update, State
+ *   Transfer.
+ *   "Leave No Context Behind" explainer, sections "メモリ構造" (one associative
+ *   matrix per head, the attention's own Q/K/V), "メモリの読み出し"
+ *   (normalised by the sum of past keys), "メモリの更新" (outer-product
+ *   accumulation; the delta rule writes only the difference),
+ *   "長期情報と短期情報の統合" (per-head gate), "実装上の流れ" (read, mix,
+ *   then update with the current K/V).
+ *   "Как работает Infini-attention", section 3, equation 1: the 1/sqrt(d)
+ *   softmax scale.
+ *
+ * Conventions for every entry point below:
+ *   - Device pointers point to memory of the current CUDA device; host
+ *     pointers are marked as such.  The caller owns every buffer; the library
+ *     keeps no pointer after a call returns.
+ *   - `stream` is a cudaStream_t (NULL = the legacy default stream).  Work is
+ *     enqueued on it and the call returns without waiting for the GPU.
+ *   - Return value: an infini_status_t (0 = success, negative = error).
+ *     Argument errors are detected before anything is enqueued.
+ */
+#ifndef INFINI_ATTN_H
+#define INFINI_ATTN_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define INFINI_API __attribute__((visibility("default")))
+#else
+#define INFINI_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  INFINI_RULE_LINEAR = 0,   /* M_s = M_{s-1} + sigma(K)^T V               */
+  INFINI_RULE_DELTA = 1     /* M_s = M_{s-1} + sigma(K)^T (V - retrieved)  */
+} infini_rule_t;
+
+typedef enum {
+  INFINI_DTYPE_BF16 = 0,    /* q, k, v, out in bfloat16; fp32 arithmetic   */
+  INFINI_DTYPE_F32 = 1      /* q, k, v, out in float32; fp32 arithmetic    */
+} infini_dtype_t;
+
+typedef enum {
+  INFINI_OK = 0,
+  INFINI_ERR_ARG = -1,          /* bad size, NULL pointer, bad enum value   */
+  INFINI_ERR_UNSUPPORTED = -2,  /* valid but unsupported shape (head dims)  */
+  INFINI_ERR_ALIAS = -3,        /* an output overlaps an input or another output */
+  INFINI_ERR_CUDA = -4,         /* a CUDA runtime call failed               */
+  INFINI_ERR_TIMEOUT = -5,      /* a kernel gave up waiting (device-side)   */
+  INFINI_ERR_WORKSPACE = -6,    /* workspace too small or misaligned        */
+  INFINI_ERR_ALIGN = -7         /* a pointer is not 16-byte aligned         */
+} infini_status_t;
+
+/* Problem sizes.  Layouts (all contiguous, row-major):
+ *   q   [B, H_q,  L, d_k]   dtype          k [B, H_kv, L, d_k]   dtype
+ *   v   [B, H_kv, L, d_v]   dtype        out [B, H_q,  L, d_v]   dtype
+ *   beta[H_q] float32 (raw logit; sg is applied inside)
+ *   M   [B, H_kv, d_k, d_v] float32        z [B, H_kv, d_k]      float32
+ * Supported: B, H_q, H_kv, L >= 1; H_q % H_kv == 0; d_k, d_v in {32, 64, 128}.
+ */
+typedef struct {
+  int B, H_q, H_kv, L, d_k, d_v;
+  int dtype;                    /* an infini_dtype_t */
+} infini_dims_t;
+
+/* Which kernels a call will run (reported by infini_attn_plan). */
+typedef enum {
+  INFINI_PATH_SIMT = 0,         /* fp32 CUDA-core kernels (any S, fp32 I/O)  */
+  INFINI_PATH_TCGEN05 = 1       /* tcgen05/TMEM tensor-core kernels (bf16)   */
+} infini_path_t;
+
+typedef struct {
+  int path;                     /* an infini_path_t                          */
+  int launches;                 /* kernels enqueued by one infini_attn_forward */
+  int num_segments;             /* T = ceil(L / seg_len)                     */
+  size_t workspace_bytes;       /* = infini_attn_workspace_bytes(...)        */
+} infini_plan_t;
+
+/* Library version, (major << 16) | minor. */
+INFINI_API int infini_attn_version(void);
+
+/* Static, NUL-terminated description of a status code. Never NULL. */
+INFINI_API const char* infini_attn_status_string(int status);
+
+/* Zero a memory state: M_0 = 0, z_0 = 0 (the empty memory every stream starts
+ * from; "Hugging Face Infini-Attention 再現分析", Memory Update starts from an
+ * empty buffer).  M: device [B, H_kv, d_k, d_v] f32; z: device [B, H_kv, d_k]
+ * f32.  Enqueued on `stream`.  Errors: INFINI_ERR_ARG (NULL or sizes < 1),
+ * INFINI_ERR_CUDA. */
+INFINI_API int infini_attn_init_state(float* M, float* z, int B, int H_kv, int d_k, int d_v,
+                           void* stream);
+
+/* Bytes of device workspace infini_attn_forward needs for these sizes (the
+ * memory read by each segment, kept for all T segments, plus a 256-byte
+ * header).  0 if the arguments are invalid. */
+INFINI_API size_t infini_attn_workspace_bytes(const infini_dims_t* dims, int seg_len, int rule);
+
+/* Fill *plan for these sizes.  Returns INFINI_OK or the error that
+ * infini_attn_forward would return for them (before touching the GPU). */
+INFINI_API int infini_attn_plan(const infini_dims_t* dims, int seg_len, int rule, infini_plan_t* plan);
+
+/* The layer forward (see the top of this file).
+ *   q, k, v          device, layouts above, element type dims->dtype
+ *   beta             device float32 [H_q]
+ *   M_in, z_in       device float32 state read by the first segment
+ *   seg_len          S >= 1
+ *   rule             an infini_rule_t
+ *   out              device [B, H_q, L, d_v], element type dims->dtype
+ *   M_out, z_out     device float32 state after the last segment.  M_out may
+ *                    equal M_in and z_out may equal z_in (in-place streaming:
+ *                    feed the next call the state this call returns); any other
+ *                    overlap between an output and an input, another output or
+ *                    the workspace is INFINI_ERR_ALIAS.
+ *   workspace        device scratch of `workspace_bytes` >= the size
+ *                    infini_attn_workspace_bytes reports, 256-byte aligned;
+ *                    or NULL with workspace_bytes == 0, in which case the call
+ *                    takes it with cudaMallocAsync on `stream` and frees it
+ *                    with cudaFreeAsync after the last kernel.
+ *   stream           cudaStream_t.
+ * All pointers must be 16-byte aligned (INFINI_ERR_ALIGN).  Device-side
+ * failures (a kernel that gave up a bounded wait) are reported by
+ * infini_attn_sync_status.  The result does not depend on the workspace's
+ * previous contents, and repeated calls on the same inputs give bitwise
+ * identical outputs. */
+INFINI_API int infini_attn_forward(const void* q, const void* k, const void* v, const float* beta,
+                        const float* M_in, const float* z_in, int seg_len, int rule,
+                        const infini_dims_t* dims, void* out, float* M_out, float* z_out,
+                        void* workspace, size_t workspace_bytes, void* stream);
+
+/* Bytes of device arena infini_attn_forward_host needs: room for q, k, v,
+ * beta, M, z, out and the workspace, each 256-byte aligned.  0 if invalid. */
+INFINI_API size_t infini_attn_host_arena_bytes(const infini_dims_t* dims, int seg_len, int rule);
+
+/* The same forward on HOST buffers.  q_h, k_h, v_h, beta_h, M_in_h, z_in_h,
+ * out_h, M_out_h, z_out_h are host pointers with the layouts above (pinned
+ * memory makes the copies asynchronous; pageable memory works but the copies
+ * then synchronise).  `arena` is a device buffer of arena_bytes >=
+ * infini_attn_host_arena_bytes(...), 256-byte aligned.  The call enqueues the
+ * host-to-device copies, the forward and the device-to-host copies on
+ * `stream`; the host results are valid once the stream has finished. */
+INFINI_API int infini_attn_forward_host(const void* q_h, const void* k_h, const void* v_h,
+                             const float* beta_h, const float* M_in_h, const float* z_in_h,
+                             int seg_len, int rule, const infini_dims_t* dims,
+                             void* out_h, float* M_out_h, float* z_out_h,
+                             void* arena, size_t arena_bytes, void* stream);
+
+/* Wait for `stream` to finish, then report and clear the device status word
+ * the kernels set when one of their bounded waits ran out:
+ * INFINI_OK, INFINI_ERR_TIMEOUT, or INFINI_ERR_CUDA if the stream itself
+ * reported an error. */
+INFINI_API int infini_attn_sync_status(void* stream);
+
+/* Benchmark support: per-kernel device timing.  While enabled, every
+ * infini_attn_forward records a CUDA event on its stream before and after each
+ * kernel it enqueues.  infini_attn_kernel_times waits for those events and
+ * writes, for each kernel kind k < n_kinds, the summed milliseconds ms[k] and
+ * the launch count launches[k] since the last reset (reset != 0 clears them).
+ * Kinds: 0 = memory-state scan, 1 = segment attention.  The timing state is
+ * process-wide; do not run forwards on other threads while reading it.
+ * Errors: INFINI_ERR_ARG (NULL arrays, n_kinds < 1), INFINI_ERR_CUDA. */
+INFINI_API int infini_attn_set_kernel_timing(int enable);
+INFINI_API int infini_attn_kernel_times(double* ms, int* launches, int n_kinds, int reset);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* INFINI_ATTN_H */

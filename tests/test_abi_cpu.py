@@ -1,0 +1,119 @@
+"""The C-ABI library on a machine without a GPU: it loads, exports every
+symbol include/infini_attn.h declares, and rejects bad arguments on the host
+before any CUDA call (no compute is launched here)."""
+
+import ctypes
+import os
+import re
+
+import pytest
+
+from compressive_memory_transformer_segment_b200 import api, configs
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def header_symbols():
+    names = set()
+    for fn in os.listdir(os.path.join(ROOT, "include")):
+        if fn.endswith(".h"):
+            text = open(os.path.join(ROOT, "include", fn)).read()
+            names |= set(re.findall(r"INFINI_API\s+[\w\s\*]*?\b(infini_attn_\w+)\s*\(", text))
+    return names
+
+
+@pytest.fixture(scope="module")
+def lib():
+    return api.load_library()
+
+
+def test_library_exports_every_declared_symbol(lib):
+    declared = header_symbols()
+    assert {"infini_attn_init_state", "infini_attn_forward"} <= declared
+    for name in declared:
+        assert hasattr(lib, name), name
+    assert declared == set(api.exported_symbols())
+    assert lib.infini_attn_version() >> 16 == 1
+
+
+def test_status_strings(lib):
+    for code in (0, -1, -2, -3, -4, -5, -6, -7, 12345):
+        assert api.status_string(code)
+
+
+def dims_of(w):
+    return api.make_dims(w.B, w.H_q, w.H_kv, w.L, w.d_k, w.d_v, 0 if w.dtype == "bf16" else 1)
+
+
+@pytest.mark.parametrize("name", sorted(configs.WORKLOADS))
+def test_plan_and_workspace_for_every_workload(name):
+    w = configs.WORKLOADS[name]
+    d = dims_of(w)
+    p = api.plan(d, w.seg_len, w.rule)
+    assert p["num_segments"] == w.T
+    assert p["workspace_bytes"] == api.workspace_bytes(d, w.seg_len, w.rule) > 0
+    # The workspace holds at least the z read by every segment.
+    assert p["workspace_bytes"] >= w.T * w.B * w.H_kv * w.d_k * 4
+    assert api.host_arena_bytes(d, w.seg_len, w.rule) > p["workspace_bytes"]
+
+
+@pytest.mark.parametrize("bad", [
+    dict(B=0), dict(H_q=3, H_kv=2), dict(L=0), dict(d_k=48), dict(d_v=256), dict(dtype=7),
+])
+def test_plan_rejects_bad_sizes(bad):
+    base = dict(B=1, H_q=4, H_kv=2, L=128, d_k=64, d_v=64, dtype=0)
+    base.update(bad)
+    d = api.Dims(**base)
+    with pytest.raises(api.InfiniError) as e:
+        api.plan(d, 64, "linear")
+    assert e.value.status in (api.ERR_ARG, api.ERR_UNSUPPORTED)
+    assert api.workspace_bytes(d, 64, "linear") == 0
+
+
+def test_plan_rejects_bad_rule_and_segment():
+    d = api.Dims(1, 2, 2, 64, 32, 32, 1)
+    for seg, rule in ((0, 0), (-3, 1), (16, 2)):
+        with pytest.raises(api.InfiniError):
+            api.plan(d, seg, rule)
+
+
+def _fwd(lib, ptrs, dims, seg=64, rule=0, ws=0, ws_n=0):
+    P = ctypes.c_void_p
+    q, k, v, beta, M, z, out, Mo, zo = (P(x) for x in ptrs)
+    return lib.infini_attn_forward(q, k, v, beta, M, z, seg, rule, ctypes.byref(dims), out, Mo, zo,
+                                   P(ws), ws_n, P(0))
+
+
+def test_forward_validates_on_host_before_any_cuda_call(lib):
+    """Fake, never-dereferenced addresses: every case below must be rejected
+    by the host checks, so no CUDA call happens (this machine has no GPU)."""
+    d = api.Dims(1, 2, 2, 128, 32, 32, 1)  # f32: q = k = v = out = 32 KiB
+    MB = 1 << 20
+    good = [1 * MB, 2 * MB, 3 * MB, 4 * MB, 5 * MB, 6 * MB, 7 * MB, 8 * MB, 9 * MB]
+    bad = list(good)
+    bad[0] = 0
+    assert _fwd(lib, bad, d) == api.ERR_ARG
+    bad = list(good)
+    bad[2] += 4
+    assert _fwd(lib, bad, d) == api.ERR_ALIGN
+    bad = list(good)
+    bad[6] = good[0] + 1024  # out inside q
+    assert _fwd(lib, bad, d) == api.ERR_ALIAS
+    bad = list(good)
+    bad[7] = good[6]  # M_out == out
+    assert _fwd(lib, bad, d) == api.ERR_ALIAS
+    bad = list(good)
+    bad[8] = good[4] + 16  # z_out overlaps M_in (not the permitted in-place pair)
+    assert _fwd(lib, bad, d) == api.ERR_ALIAS
+    assert _fwd(lib, good, d, ws=10 * MB, ws_n=16) == api.ERR_WORKSPACE
+    assert _fwd(lib, good, d, ws=10 * MB + 16, ws_n=1 << 30) == api.ERR_WORKSPACE
+    assert _fwd(lib, good, d, ws=0, ws_n=64) == api.ERR_ARG
+    assert _fwd(lib, good, d, ws=good[0], ws_n=1 << 20) == api.ERR_ALIAS
+    d_bad = api.Dims(1, 2, 2, 128, 40, 32, 1)
+    assert _fwd(lib, good, d_bad) == api.ERR_UNSUPPORTED
+
+
+def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
+    monkeypatch.setattr(api, "_lib", None)
+    with pytest.raises(FileNotFoundError):
+        api.load_library(str(tmp_path / "missing.so"))

@@ -1,0 +1,249 @@
+"""GPU parity: the CUDA library (through the C ABI) against the float64 oracle
+on identical seeded inputs.
+
+Small cases are compared element by element in full; the workloads too large
+for the oracle are run at full size, in the same launch configuration the
+bench times, and compared on sampled heads and segments (heads are independent
+of one another, so the other heads only need to exist).
+
+Tolerances: max |out - oracle| <= 2e-2 for bf16 I/O, <= 1e-4 for fp32 I/O;
+relative error of M (Frobenius, per KV head) and of z (per entry) <= 1e-3.
+"""
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from compressive_memory_transformer_segment_b200 import configs, synth
+from helpers import (TOL_OUT, TOL_STATE, gpu_forward, oracle_forward, state_rel_errors,
+                     to_torch)
+
+pytestmark = pytest.mark.gpu
+
+W = configs.WORKLOADS
+
+
+def check_full(api, w, inp=None, M_in=None, z_in=None):
+    inp = synth.make_inputs(w) if inp is None else inp
+    out, M, z = gpu_forward(api, inp, w, M_in=M_in, z_in=z_in)
+    ro, rM, rz = oracle_forward(inp, w, M_in=M_in, z_in=z_in)
+    err = float(np.max(np.abs(out - ro)))
+    em, ez = state_rel_errors(M, z, rM, rz)
+    assert np.all(np.isfinite(out))
+    assert err <= TOL_OUT[w.dtype], (w.name, err)
+    assert em <= TOL_STATE and ez <= TOL_STATE, (w.name, em, ez)
+    return err, em, ez
+
+
+# ------------------------------------------------------------ configurations
+
+@pytest.mark.parametrize("name", ["tiny", "200m-linear", "200m-delta"])
+def test_workload_full_parity(cuda_lib, name):
+    check_full(cuda_lib, W[name])
+
+
+def test_tiny_delta(cuda_lib):
+    check_full(cuda_lib, W["tiny"].with_(rule="delta"))
+
+
+CASES = [
+    # name, overrides
+    ("ragged_tail_f32", dict(L=200)),
+    ("seg1", dict(L=16, seg_len=1)),
+    ("seg63", dict(L=300, seg_len=63)),
+    ("seg65_delta", dict(L=300, seg_len=65, rule="delta")),
+    ("L_lt_S", dict(L=50, seg_len=64)),
+    ("gqa_b2", dict(B=2, H_q=8, H_kv=2, L=192, rule="delta")),
+    ("dk64_dv32", dict(d_k=64, d_v=32, L=160)),
+    ("dk32_dv128", dict(d_k=32, d_v=128, L=160, rule="delta")),
+    ("bf16_d128_S256", dict(dtype="bf16", d_k=128, d_v=128, L=700, seg_len=256, H_q=4, H_kv=2)),
+    ("bf16_d64_S128_delta", dict(dtype="bf16", d_k=64, d_v=64, L=512 + 77, seg_len=128, rule="delta")),
+    ("bf16_d128_S2048_ragged", dict(dtype="bf16", d_k=128, d_v=128, L=4096 + 300, seg_len=2048,
+                                    H_q=4, H_kv=1, rule="delta")),
+    ("bf16_S64_odd_L", dict(dtype="bf16", d_k=64, d_v=64, L=64 * 5 + 17, seg_len=64, H_q=2, H_kv=2)),
+]
+
+
+@pytest.mark.parametrize("name,over", CASES, ids=[c[0] for c in CASES])
+def test_edge_cases(cuda_lib, name, over):
+    check_full(cuda_lib, W["tiny"].with_(name=name, **over))
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_gate_extremes(cuda_lib, dtype):
+    w = W["tiny"].with_(dtype=dtype, H_q=4, H_kv=2, L=256, seg_len=64)
+    inp = synth.make_inputs(w)
+    inp["beta"] = np.array([-np.inf, np.inf, -80.0, 80.0], np.float32)
+    check_full(cuda_lib, w, inp)
+    # beta = +inf: the first segment retrieves from an empty memory -> exactly 0.
+    out, _, _ = gpu_forward(cuda_lib, inp, w)
+    assert np.all(out[:, 1, :64] == 0.0)
+
+
+@pytest.mark.parametrize("rule", ["linear", "delta"])
+def test_nonzero_initial_state(cuda_lib, rule):
+    w = W["tiny"].with_(rule=rule, B=2, H_q=4, H_kv=2, L=192)
+    prev = synth.make_inputs(w.with_(seed=77))
+    _, M0, z0 = oracle_forward(prev, w)
+    check_full(cuda_lib, w, M_in=M0.astype(np.float32), z_in=z0.astype(np.float32))
+
+
+@pytest.mark.parametrize("dtype,rule", [("f32", "linear"), ("bf16", "delta")])
+def test_split_stream_in_place_state(cuda_lib, dtype, rule):
+    """forward(L1) then forward(L2) with the state updated in place equals
+    forward(L1 + L2) when L1 is a whole number of segments."""
+    api = cuda_lib
+    w = W["tiny"].with_(dtype=dtype, rule=rule, B=2, H_q=4, H_kv=2, L=320, seg_len=64)
+    inp = synth.make_inputs(w)
+    q, k, v = (to_torch(inp[n], dtype) for n in ("q", "k", "v"))
+    beta = torch.from_numpy(inp["beta"]).cuda()
+    M, z = api.init_state(2, 2, 32, 32)
+    out_full, M_full, z_full = api.forward(q, k, v, beta, M, z, 64, rule)
+    L1 = 128
+    o1, _, _ = api.forward(q[:, :, :L1].contiguous(), k[:, :, :L1].contiguous(),
+                           v[:, :, :L1].contiguous(), beta, M, z, 64, rule, M_out=M, z_out=z)
+    o2, _, _ = api.forward(q[:, :, L1:].contiguous(), k[:, :, L1:].contiguous(),
+                           v[:, :, L1:].contiguous(), beta, M, z, 64, rule, M_out=M, z_out=z)
+    api.sync_status()
+    tol = TOL_OUT[dtype]
+    assert torch.max(torch.abs(torch.cat([o1, o2], 2).float() - out_full.float())) <= tol
+    assert torch.allclose(M, M_full, rtol=1e-5, atol=1e-4)
+    assert torch.allclose(z, z_full, rtol=1e-6, atol=1e-5)
+
+
+def test_gqa_equals_repeated_kv_mha(cuda_lib):
+    api = cuda_lib
+    w = W["tiny"].with_(dtype="bf16", B=2, H_q=8, H_kv=2, L=256, seg_len=64, rule="delta")
+    inp = synth.make_inputs(w)
+    q, k, v = (to_torch(inp[n], "bf16") for n in ("q", "k", "v"))
+    beta = torch.from_numpy(inp["beta"]).cuda()
+    M0, z0 = api.init_state(2, 2, 32, 32)
+    out, M, z = api.forward(q, k, v, beta, M0, z0, 64, "delta")
+    kr, vr = k.repeat_interleave(4, 1).contiguous(), v.repeat_interleave(4, 1).contiguous()
+    M1, z1 = api.init_state(2, 8, 32, 32)
+    out2, M2, z2 = api.forward(q, kr, vr, beta, M1, z1, 64, "delta")
+    api.sync_status()
+    assert torch.equal(out, out2)
+    assert torch.equal(M2, M.repeat_interleave(4, 1))
+    assert torch.equal(z2, z.repeat_interleave(4, 1))
+
+
+def test_repeat_calls_bitwise_identical(cuda_lib):
+    api = cuda_lib
+    w = W["200m-delta"]
+    inp = synth.make_inputs(w)
+    a = gpu_forward(api, inp, w)
+    b = gpu_forward(api, inp, w)
+    for x, y in zip(a, b):
+        np.testing.assert_array_equal(x, y)
+
+
+def test_workspace_given_or_taken_agree(cuda_lib):
+    api = cuda_lib
+    w = W["200m-linear"]
+    inp = synth.make_inputs(w)
+    dims = api.make_dims(w.B, w.H_q, w.H_kv, w.L, w.d_k, w.d_v, torch.bfloat16)
+    n = api.workspace_bytes(dims, w.seg_len, w.rule)
+    ws = torch.full((n,), 0xAB, dtype=torch.uint8, device="cuda")  # garbage contents
+    a = gpu_forward(api, inp, w, workspace=ws)
+    b = gpu_forward(api, inp, w)
+    for x, y in zip(a, b):
+        np.testing.assert_array_equal(x, y)
+
+
+def test_host_buffer_entry_point_matches_device(cuda_lib):
+    api = cuda_lib
+    w = W["200m-delta"]
+    inp = synth.make_inputs(w)
+    dev = gpu_forward(api, inp, w)
+    q, k, v = (to_torch(inp[n], "bf16", "cpu").pin_memory() for n in ("q", "k", "v"))
+    beta = torch.from_numpy(inp["beta"]).pin_memory()
+    M0 = torch.from_numpy(inp["M_in"]).pin_memory()
+    z0 = torch.from_numpy(inp["z_in"]).pin_memory()
+    out = torch.empty((w.B, w.H_q, w.L, w.d_v), dtype=torch.bfloat16).pin_memory()
+    M = torch.empty_like(M0).pin_memory()
+    z = torch.empty_like(z0).pin_memory()
+    dims = api.make_dims(w.B, w.H_q, w.H_kv, w.L, w.d_k, w.d_v, torch.bfloat16)
+    arena = torch.empty(api.host_arena_bytes(dims, w.seg_len, w.rule), dtype=torch.uint8,
+                        device="cuda")
+    api.forward_host(q, k, v, beta, M0, z0, w.seg_len, w.rule, out, M, z, arena)
+    api.sync_status()
+    np.testing.assert_array_equal(out.float().numpy(), dev[0])
+    np.testing.assert_array_equal(M.numpy(), dev[1])
+    np.testing.assert_array_equal(z.numpy(), dev[2])
+
+
+def test_gpu_argument_errors(cuda_lib):
+    api = cuda_lib
+    q = torch.zeros((1, 2, 64, 32), device="cuda")
+    k = torch.zeros((1, 2, 64, 32), device="cuda")
+    beta = torch.zeros(2, device="cuda")
+    M, z = api.init_state(1, 2, 32, 32)
+    with pytest.raises(api.InfiniError) as e:
+        api.forward(q, k, k, beta, M, z, 64, "linear", out=q)  # out aliases q
+    assert e.value.status == api.ERR_ALIAS
+    with pytest.raises(api.InfiniError) as e:
+        api.forward(q, k, k, beta, M, z, 0, "linear")
+    assert e.value.status == api.ERR_ARG
+    # In-place state is allowed.
+    api.forward(q, k, k, beta, M, z, 64, "linear", M_out=M, z_out=z)
+    api.sync_status()
+
+
+# ------------------------------------------------------------ full size, sampled
+
+SAMPLED = {
+    # name: (batch row, KV head, query heads of that group to check, segments)
+    "300m-linear": (3, 5, [5], [0, 1, 7]),
+    "300m-delta": (1, 15, [15], [0, 4, 7]),
+    "8b-delta": (1, 6, [24, 27], [0, 8, 15]),
+    "1m-linear": (0, 13, [13], [0, 2, 255, 511]),
+}
+
+
+def sampled_inputs(w, b, j, heads):
+    """Full-size GPU tensors whose sampled slices hold the seeded values."""
+    t = torch.bfloat16 if w.dtype == "bf16" else torch.float32
+    q = torch.zeros((w.B, w.H_q, w.L, w.d_k), dtype=t, device="cuda")
+    k = torch.zeros((w.B, w.H_kv, w.L, w.d_k), dtype=t, device="cuda")
+    v = torch.zeros((w.B, w.H_kv, w.L, w.d_v), dtype=t, device="cuda")
+    host = {}
+    for h in heads:
+        host[("q", h)] = synth.make_head(w, "q", b, h)
+        q[b, h] = to_torch(host[("q", h)], w.dtype)
+    for name, dst in (("k", k), ("v", v)):
+        host[(name, j)] = synth.make_head(w, name, b, j)
+        dst[b, j] = to_torch(host[(name, j)], w.dtype)
+    return q, k, v, host
+
+
+@pytest.mark.parametrize("name", list(SAMPLED))
+def test_full_size_sampled(cuda_lib, name):
+    api = cuda_lib
+    w = W[name]
+    b, j, heads, segs = SAMPLED[name]
+    q, k, v, host = sampled_inputs(w, b, j, heads)
+    beta_np = synth.make_beta(w)
+    beta = torch.from_numpy(beta_np).cuda()
+    M0, z0 = api.init_state(w.B, w.H_kv, w.d_k, w.d_v)
+    out, M, z = api.forward(q, k, v, beta, M0, z0, w.seg_len, w.rule)
+    api.sync_status()
+    del q, k, v
+    kc = synth.as_float64(host[("k", j)], w.dtype)
+    vc = synth.as_float64(host[("v", j)], w.dtype)
+    worst = 0.0
+    for s, r0, r1, Mp, zp in oracle.scan_states(kc, vc, np.zeros((w.d_k, w.d_v)), np.zeros(w.d_k),
+                                                w.seg_len, w.rule):
+        if r0 == r1:
+            em, ez = state_rel_errors(M[b, j].cpu().numpy(), z[b, j].cpu().numpy(), Mp, zp)
+            assert em <= TOL_STATE and ez <= TOL_STATE, (em, ez)
+            break
+        if s not in segs:
+            continue
+        for h in heads:
+            qs = synth.as_float64(host[("q", h)][r0:r1], w.dtype)
+            ref = oracle.segment_output(qs, kc[r0:r1], vc[r0:r1], Mp, zp, float(beta_np[h]))
+            got = out[b, h, r0:r1].float().cpu().numpy()
+            worst = max(worst, float(np.max(np.abs(got - ref))))
+    assert worst <= TOL_OUT[w.dtype], worst

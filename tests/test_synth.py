@@ -44,3 +44,14 @@ def test_algorithmic_counts_8b():
     w = configs.WORKLOADS["8b-delta"]
     assert abs(configs.algorithmic_flops(w) / 1.204e12 - 1) < 2e-3
     assert abs(configs.algorithmic_bytes(w) / 1.344e9 - 1) < 2e-3
+
+
+def test_make_head_matches_make_inputs():
+    w = configs.WORKLOADS["tiny"].with_(B=2, H_q=4, H_kv=2, L=2 * 64 + 1000 + 8,
+                                        insert_pair=True, dtype="bf16")
+    x = synth.make_inputs(w)
+    for name, H in (("q", 4), ("k", 2), ("v", 2)):
+        for b in range(2):
+            for h in range(H):
+                np.testing.assert_array_equal(synth.make_head(w, name, b, h), x[name][b, h])
+    np.testing.assert_array_equal(synth.make_beta(w), x["beta"])
