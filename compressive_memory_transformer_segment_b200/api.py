@@ -23,6 +23,7 @@ PATHS = {0: "simt", 1: "tcgen05"}
 OK = 0
 ERR_ARG, ERR_UNSUPPORTED, ERR_ALIAS, ERR_CUDA, ERR_TIMEOUT, ERR_WORKSPACE, ERR_ALIGN = (
     -1, -2, -3, -4, -5, -6, -7)
+ERR_SCRATCH_LIMIT = -8
 
 
 class Dims(ctypes.Structure):
@@ -65,6 +66,10 @@ _SIGNATURES = [
     ("infini_attn_kernel_times", ctypes.c_int, [ctypes.POINTER(ctypes.c_double),
                                                 ctypes.POINTER(ctypes.c_int), ctypes.c_int,
                                                 ctypes.c_int]),
+    ("infini_attn_forward_noalloc", ctypes.c_int, [_P, _P, _P, _P, _P, _P, ctypes.c_int,
+                                                   ctypes.c_int, ctypes.POINTER(Dims), _P, _P, _P,
+                                                   _P]),
+    ("infini_attn_noalloc_scratch_limit", ctypes.c_size_t, []),
 ]
 
 
@@ -247,3 +252,27 @@ def kernel_times(reset=True):
     cnt = (ctypes.c_int * n)()
     _check(load_library().infini_attn_kernel_times(ms, cnt, n, 1 if reset else 0))
     return {KERNEL_KINDS[i]: (ms[i], cnt[i]) for i in range(n)}
+
+
+def noalloc_scratch_limit():
+    return load_library().infini_attn_noalloc_scratch_limit()
+
+
+def forward_noalloc(q, k, v, beta, M_in, z_in, seg_len, rule, out, M_out, z_out, stream=None):
+    """infini_attn_forward_noalloc: the forward for callers that cannot allocate
+    GPU memory while they run.  All outputs must be given (this wrapper
+    allocates nothing either); scratch comes from the library's static array.
+    """
+    lib = load_library()
+    dims = _dims_from(q, k, v)
+    B, H_q, L, H_kv, d_k, d_v = dims.B, dims.H_q, dims.L, dims.H_kv, dims.d_k, dims.d_v
+    args = [_dev(q, "q"), _dev(k, "k"), _dev(v, "v"),
+            _dev(beta, "beta", torch.float32, (H_q,)),
+            _dev(M_in, "M_in", torch.float32, (B, H_kv, d_k, d_v)),
+            _dev(z_in, "z_in", torch.float32, (B, H_kv, d_k))]
+    outs = [_dev(out, "out", q.dtype, (B, H_q, L, d_v)),
+            _dev(M_out, "M_out", torch.float32, (B, H_kv, d_k, d_v)),
+            _dev(z_out, "z_out", torch.float32, (B, H_kv, d_k))]
+    _check(lib.infini_attn_forward_noalloc(*args, int(seg_len), _rule(rule), ctypes.byref(dims),
+                                           *outs, _stream_handle(stream)))
+    return out, M_out, z_out

@@ -148,6 +148,9 @@ const char* infini_attn_status_string(int status) {
     case INFINI_ERR_TIMEOUT: return "a kernel gave up a bounded wait (device status word set)";
     case INFINI_ERR_WORKSPACE: return "workspace too small or not 256-byte aligned";
     case INFINI_ERR_ALIGN: return "a pointer is not 16-byte aligned";
+    case INFINI_ERR_SCRATCH_LIMIT:
+      return "problem needs more scratch than the no-allocation entry point's static array "
+             "holds; use infini_attn_forward with a workspace";
     default: return "unknown status";
   }
 }

@@ -1,0 +1,80 @@
+// infini_attn_forward_noalloc: the layer forward for callers that cannot
+// allocate GPU memory at call time.
+//
+// Who needs it.  Some callers may not call cudaMalloc / cudaMallocAsync (or an
+// allocator that ends in them) while they run: code that executes inside a
+// region where allocation is forbidden or would deadlock (a custom allocator's
+// own callback, a real-time or interrupt-like loop that must not block on the
+// driver's allocator, an embedding that owns all device memory through a
+// fixed arena and does not expose it).  Such a caller still owns and passes its
+// inputs and outputs, but it cannot hand this library a workspace.
+//
+// How.  The scratch the forward needs (the memory every segment reads, for
+// all segments) lives in one file-scope device array of fixed size,
+// kNoAllocScratchBytes.  Host code cannot use the array's name as a device
+// address, so the first call on each device looks its address up with
+// cudaGetSymbolAddress (with that device current) and keeps it; later calls
+// on that device reuse it.  The call then runs the regular forward with that
+// address as its workspace.  Nothing here allocates.
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include <mutex>
+
+#include "infini_attn.h"
+
+namespace {
+
+// 32 MiB: enough for the tiny, 200M-, 300M- and 8B-shaped workloads; a
+// 1M-token stream needs about 1 GiB and is rejected.
+constexpr size_t kNoAllocScratchBytes = size_t(32) << 20;
+constexpr int kMaxDevices = 64;
+
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
+std::mutex g_mu;
+void* g_scratch_addr[kMaxDevices];  // device address of g_noalloc_scratch, per device
+
+// Looks up (once per device) the device address of the static scratch array.
+cudaError_t scratch_address(void** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> lock(g_mu);
+  if (!g_scratch_addr[dev]) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    if (e != cudaSuccess) return e;
+    g_scratch_addr[dev] = p;
+  }
+  *out = g_scratch_addr[dev];
+  return cudaSuccess;
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t infini_attn_noalloc_scratch_limit(void) { return kNoAllocScratchBytes; }
+
+int infini_attn_forward_noalloc(const void* q, const void* k, const void* v, const float* beta,
+                                const float* M_in, const float* z_in, int seg_len, int rule,
+                                const infini_dims_t* dims, void* out, float* M_out, float* z_out,
+                                void* stream) {
+  const size_t need = infini_attn_workspace_bytes(dims, seg_len, rule);
+  if (need == 0) {
+    infini_plan_t plan;
+    const int rc = infini_attn_plan(dims, seg_len, rule, &plan);
+    return rc != INFINI_OK ? rc : INFINI_ERR_ARG;
+  }
+  if (need > kNoAllocScratchBytes) return INFINI_ERR_SCRATCH_LIMIT;
+  void* scratch = nullptr;
+  if (scratch_address(&scratch) != cudaSuccess) return INFINI_ERR_CUDA;
+  // Every byte of scratch the kernels read is written earlier in the same
+  // call, so nothing has to be cleared between calls.
+  return infini_attn_forward(q, k, v, beta, M_in, z_in, seg_len, rule, dims, out, M_out, z_out,
+                             scratch, kNoAllocScratchBytes, stream);
+}
+
+}  // extern "C"

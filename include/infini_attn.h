@@ -75,7 +75,8 @@ typedef enum {
   INFINI_ERR_CUDA = -4,         /* a CUDA runtime call failed               */
   INFINI_ERR_TIMEOUT = -5,      /* a kernel gave up waiting (device-side)   */
   INFINI_ERR_WORKSPACE = -6,    /* workspace too small or misaligned        */
-  INFINI_ERR_ALIGN = -7         /* a pointer is not 16-byte aligned         */
+  INFINI_ERR_ALIGN = -7,        /* a pointer is not 16-byte aligned         */
+  INFINI_ERR_SCRATCH_LIMIT = -8 /* problem too large for infini_attn_forward_noalloc */
 } infini_status_t;
 
 /* Problem sizes.  Layouts (all contiguous, row-major):
@@ -187,6 +188,40 @@ INFINI_API int infini_attn_sync_status(void* stream);
  * Errors: INFINI_ERR_ARG (NULL arrays, n_kinds < 1), INFINI_ERR_CUDA. */
 INFINI_API int infini_attn_set_kernel_timing(int enable);
 INFINI_API int infini_attn_kernel_times(double* ms, int* launches, int n_kinds, int reset);
+
+/* No-allocation variant of infini_attn_forward.  The paper has no
+ * counterpart: this is a deployment facility of this library.
+ *
+ * For callers that cannot allocate GPU memory while they run (code inside an
+ * allocator callback, a loop that must never block on the driver's allocator,
+ * an embedding that owns all device memory and cannot lend a workspace).
+ * Arguments and results are those of infini_attn_forward without the
+ * workspace: the scratch comes from one static device array of
+ * infini_attn_noalloc_scratch_limit() bytes (32 MiB), which every GPU that
+ * loads this part of the library holds until the process exits.
+ *   - Problems whose workspace (infini_attn_workspace_bytes) exceeds that
+ *     limit return INFINI_ERR_SCRATCH_LIMIT before anything is enqueued
+ *     (a 1M-token stream does; the tiny, 200M-, 300M- and 8B-shaped
+ *     workloads fit).
+ *   - The call allocates nothing: no cudaMalloc, cudaMallocAsync or
+ *     allocating library routine.
+ *   - The first call on each device looks up the array's device address
+ *     (cudaGetSymbolAddress, with that device current); make that first call
+ *     before any stream capture.
+ *   - All calls on a device share the one array and it keeps the last call's
+ *     contents; nothing in it needs clearing (every byte read is written
+ *     earlier in the same call).  Calls whose GPU work overlaps -- on two
+ *     streams, or from two threads -- race on the array and corrupt each
+ *     other's results: serialise them.
+ * Errors: those of infini_attn_forward, plus INFINI_ERR_SCRATCH_LIMIT. */
+INFINI_API int infini_attn_forward_noalloc(const void* q, const void* k, const void* v,
+                                           const float* beta, const float* M_in,
+                                           const float* z_in, int seg_len, int rule,
+                                           const infini_dims_t* dims, void* out, float* M_out,
+                                           float* z_out, void* stream);
+
+/* Bytes of the static scratch array infini_attn_forward_noalloc uses. */
+INFINI_API size_t infini_attn_noalloc_scratch_limit(void);
 
 #ifdef __cplusplus
 }
