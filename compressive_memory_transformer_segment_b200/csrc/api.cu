@@ -60,9 +60,10 @@ int check_shape(const infini_dims_t* d, int seg_len, int rule, Shape* s) {
   s->beta_bytes = (size_t)d->H_q * 4;
   s->M_bytes = BHkv * d->d_k * d->d_v * 4;
   s->z_bytes = BHkv * d->d_k * 4;
-  s->path = INFINI_PATH_SIMT;
+  const bool tc = tc_attention_supported(d->d_k, d->d_v, seg_len, s->bf16);
+  s->path = tc ? INFINI_PATH_TCGEN05 : INFINI_PATH_SIMT;
   s->launches = 2;
-  const size_t mpref_elem = 4;
+  const size_t mpref_elem = tc ? 2 : 4;
   s->ws_zpref = kHeader;
   s->ws_mpref = align_up(s->ws_zpref + (size_t)s->T * BHkv * d->d_k * 4);
   s->ws_total = align_up(s->ws_mpref + (size_t)s->T * BHkv * d->d_k * d->d_v * mpref_elem);
@@ -234,11 +235,15 @@ int infini_attn_forward(const void* q, const void* k, const void* v, const float
   p.S = s.S; p.T = s.T; p.bf16 = s.bf16; p.delta = s.delta;
   p.z_pref = reinterpret_cast<float*>(ws + s.ws_zpref);
   p.M_pref = ws + s.ws_mpref;
+  p.M_pref_bf16 = s.path == INFINI_PATH_TCGEN05;
   p.status = status;
 
   cudaError_t e = cudaMemcpyAsync(p.z_pref, z_in, s.z_bytes, cudaMemcpyDeviceToDevice, st);
   if (e == cudaSuccess) e = timed(0, st, [&] { return launch_simt_state_scan(p, st); });
-  if (e == cudaSuccess) e = timed(1, st, [&] { return launch_simt_attention(p, st); });
+  if (e == cudaSuccess)
+    e = timed(1, st, [&] {
+      return s.path == INFINI_PATH_TCGEN05 ? launch_tc_attention(p, st) : launch_simt_attention(p, st);
+    });
   if (owned) {
     cudaError_t f = cudaFreeAsync(ws, st);
     if (e == cudaSuccess) e = f;

@@ -23,11 +23,17 @@ struct Problem {
   // Workspace views.
   float* z_pref;       // [T][B*H_kv][d_k] f32: z_{s-1} read by segment s (slot 0 = z_in)
   void* M_pref;        // [T][B*H_kv][d_k][d_v]: M_{s-1} (f32 on the SIMT path, bf16 on tcgen05)
+  bool M_pref_bf16;    // element type of M_pref
   unsigned int* status;  // device status word
 };
 
 // fp32 CUDA-core path (any S, any supported d, f32 or bf16 I/O).
 cudaError_t launch_simt_state_scan(const Problem& p, cudaStream_t stream);
 cudaError_t launch_simt_attention(const Problem& p, cudaStream_t stream);
+
+// Tensor-core (tcgen05 / TMEM / TMA) segment attention: bf16 I/O,
+// d_k == d_v in {64, 128}, S a multiple of 128.  Reads bf16 M_pref.
+bool tc_attention_supported(int d_k, int d_v, int S, bool bf16);
+cudaError_t launch_tc_attention(const Problem& p, cudaStream_t stream);
 
 }  // namespace infini

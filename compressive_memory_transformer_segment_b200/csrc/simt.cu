@@ -43,12 +43,12 @@ struct ScanSmem {
 // of the chain's M for the whole scan; the delta rule's column j depends only
 // on column j of M and on the shared denominator sigma(K) z, so the column
 // blocks are independent.  Thread (warp w, lane c) holds M[w + 8 i][c].
-template <typename T, int DK, int DV, bool DELTA>
+template <typename T, typename MP, int DK, int DV, bool DELTA>
 __global__ void __launch_bounds__(kScanThreads)
 simt_state_scan(const T* __restrict__ kx, const T* __restrict__ vx,
                 const float* __restrict__ M_in, float* __restrict__ M_out,
                 float* __restrict__ z_out, float* __restrict__ z_pref,
-                float* __restrict__ M_pref, int L, int S, int nseg, int BH) {
+                MP* __restrict__ M_pref, int L, int S, int nseg, int BH) {
   using SM = ScanSmem<DK>;
   extern __shared__ float smem[];
   float* sK = smem;
@@ -77,10 +77,10 @@ simt_state_scan(const T* __restrict__ kx, const T* __restrict__ vx,
     const int r0 = s * S;
     const int r1 = min(r0 + S, L);
     // The memory segment s reads: M_{s-1}, z_{s-1}.
-    float* Mp = M_pref + ((size_t)s * BH + bh) * DK * DV;
+    MP* Mp = M_pref + ((size_t)s * BH + bh) * DK * DV;
 #pragma unroll
     for (int i = 0; i < kRows; ++i) {
-      Mp[(size_t)(warp + 8 * i) * DV + c0 + lane] = Mreg[i];
+      Mp[(size_t)(warp + 8 * i) * DV + c0 + lane] = from_f32<MP>(Mreg[i]);
       dM[i] = 0.f;
       if (DELTA) Ms[(warp + 8 * i) * kScanCols + lane] = Mreg[i];
     }
@@ -309,7 +309,17 @@ template <typename T, int DK, int DV>
 cudaError_t scan_dispatch_rule(const Problem& p, cudaStream_t stream) {
   const size_t smem = ScanSmem<DK>::kTotal * sizeof(float);
   dim3 grid(DV / kScanCols, p.B * p.H_kv);
-  auto kern = p.delta ? simt_state_scan<T, DK, DV, true> : simt_state_scan<T, DK, DV, false>;
+  if (p.M_pref_bf16) {
+    auto kern = p.delta ? simt_state_scan<T, __nv_bfloat16, DK, DV, true>
+                        : simt_state_scan<T, __nv_bfloat16, DK, DV, false>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    kern<<<grid, kScanThreads, smem, stream>>>(
+        static_cast<const T*>(p.k), static_cast<const T*>(p.v), p.M_in, p.M_out, p.z_out,
+        p.z_pref, static_cast<__nv_bfloat16*>(p.M_pref), p.L, p.S, p.T, p.B * p.H_kv);
+    return cudaGetLastError();
+  }
+  auto kern = p.delta ? simt_state_scan<T, float, DK, DV, true> : simt_state_scan<T, float, DK, DV, false>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   kern<<<grid, kScanThreads, smem, stream>>>(

@@ -247,3 +247,75 @@ def test_full_size_sampled(cuda_lib, name):
             got = out[b, h, r0:r1].float().cpu().numpy()
             worst = max(worst, float(np.max(np.abs(got - ref))))
     assert worst <= TOL_OUT[w.dtype], worst
+
+
+# ------------------------------------------------------------ path selection
+
+TC_CASES = [
+    ("tc_d128_S128_linear", dict(dtype="bf16", d_k=128, d_v=128, L=384, seg_len=128, H_q=2, H_kv=2)),
+    ("tc_d128_S256_gqa_delta", dict(dtype="bf16", d_k=128, d_v=128, L=1024, seg_len=256, B=2,
+                                    H_q=8, H_kv=2, rule="delta")),
+    ("tc_d64_S512_ragged", dict(dtype="bf16", d_k=64, d_v=64, L=1500, seg_len=512, H_q=3, H_kv=3)),
+    ("tc_d128_L_lt_S", dict(dtype="bf16", d_k=128, d_v=128, L=200, seg_len=256)),
+]
+
+
+def test_path_selection(cuda_lib):
+    api = cuda_lib
+    for name, over, path in [("8b-delta", {}, "tcgen05"), ("1m-linear", {}, "tcgen05"),
+                             ("300m-delta", {}, "tcgen05"), ("tiny", {}, "simt"),
+                             ("200m-linear", {}, "simt")]:
+        w = W[name].with_(**over)
+        dims = api.make_dims(w.B, w.H_q, w.H_kv, w.L, w.d_k, w.d_v, 0 if w.dtype == "bf16" else 1)
+        assert api.plan(dims, w.seg_len, w.rule)["path"] == path, name
+    for name, over in TC_CASES:
+        w = W["tiny"].with_(**over)
+        dims = api.make_dims(w.B, w.H_q, w.H_kv, w.L, w.d_k, w.d_v, 0)
+        assert api.plan(dims, w.seg_len, w.rule)["path"] == "tcgen05", name
+
+
+@pytest.mark.parametrize("name,over", TC_CASES, ids=[c[0] for c in TC_CASES])
+def test_tensor_core_path_cases(cuda_lib, name, over):
+    check_full(cuda_lib, W["tiny"].with_(name=name, **over))
+
+
+def test_tensor_core_path_deterministic_and_workspace_independent(cuda_lib):
+    api = cuda_lib
+    w = W["tiny"].with_(dtype="bf16", d_k=128, d_v=128, L=1024, seg_len=256, B=2, H_q=4, H_kv=2,
+                        rule="delta")
+    inp = synth.make_inputs(w)
+    dims = api.make_dims(w.B, w.H_q, w.H_kv, w.L, w.d_k, w.d_v, torch.bfloat16)
+    n = api.workspace_bytes(dims, w.seg_len, w.rule)
+    ws = torch.full((n,), 0x7F, dtype=torch.uint8, device="cuda")
+    a = gpu_forward(api, inp, w, workspace=ws)
+    b = gpu_forward(api, inp, w)
+    for x, y in zip(a, b):
+        np.testing.assert_array_equal(x, y)
+
+
+def test_tensor_core_path_gate_extremes(cuda_lib):
+    w = W["tiny"].with_(dtype="bf16", d_k=64, d_v=64, H_q=4, H_kv=2, L=512, seg_len=128)
+    inp = synth.make_inputs(w)
+    inp["beta"] = np.array([-np.inf, np.inf, -80.0, 80.0], np.float32)
+    check_full(cuda_lib, w, inp)
+    out, _, _ = gpu_forward(cuda_lib, inp, w)
+    assert np.all(out[:, 1, :128] == 0.0)
+
+
+def test_tensor_core_path_split_stream(cuda_lib):
+    api = cuda_lib
+    w = W["tiny"].with_(dtype="bf16", rule="delta", B=1, H_q=4, H_kv=2, L=1024, seg_len=256,
+                        d_k=128, d_v=128)
+    inp = synth.make_inputs(w)
+    q, k, v = (to_torch(inp[n], "bf16") for n in ("q", "k", "v"))
+    beta = torch.from_numpy(inp["beta"]).cuda()
+    M, z = api.init_state(1, 2, 128, 128)
+    out_full, M_full, z_full = api.forward(q, k, v, beta, M, z, 256, "delta")
+    L1 = 512
+    o1, _, _ = api.forward(q[:, :, :L1].contiguous(), k[:, :, :L1].contiguous(),
+                           v[:, :, :L1].contiguous(), beta, M, z, 256, "delta", M_out=M, z_out=z)
+    o2, _, _ = api.forward(q[:, :, L1:].contiguous(), k[:, :, L1:].contiguous(),
+                           v[:, :, L1:].contiguous(), beta, M, z, 256, "delta", M_out=M, z_out=z)
+    api.sync_status()
+    assert torch.max(torch.abs(torch.cat([o1, o2], 2).float() - out_full.float())) <= 2e-2
+    assert torch.allclose(M, M_full, rtol=1e-5, atol=1e-4)
