@@ -60,7 +60,8 @@ int check_shape(const infini_dims_t* d, int seg_len, int rule, Shape* s) {
   s->beta_bytes = (size_t)d->H_q * 4;
   s->M_bytes = BHkv * d->d_k * d->d_v * 4;
   s->z_bytes = BHkv * d->d_k * 4;
-  const bool tc = tc_attention_supported(d->d_k, d->d_v, seg_len, s->bf16);
+  const bool tc = tc_attention_supported(d->d_k, d->d_v, seg_len, s->bf16) &&
+                  tc_scan_supported(d->d_k, d->d_v, s->bf16);
   s->path = tc ? INFINI_PATH_TCGEN05 : INFINI_PATH_SIMT;
   s->launches = 2;
   const size_t mpref_elem = tc ? 2 : 4;
@@ -239,7 +240,10 @@ int infini_attn_forward(const void* q, const void* k, const void* v, const float
   p.status = status;
 
   cudaError_t e = cudaMemcpyAsync(p.z_pref, z_in, s.z_bytes, cudaMemcpyDeviceToDevice, st);
-  if (e == cudaSuccess) e = timed(0, st, [&] { return launch_simt_state_scan(p, st); });
+  if (e == cudaSuccess)
+    e = timed(0, st, [&] {
+      return s.path == INFINI_PATH_TCGEN05 ? launch_tc_state_scan(p, st) : launch_simt_state_scan(p, st);
+    });
   if (e == cudaSuccess)
     e = timed(1, st, [&] {
       return s.path == INFINI_PATH_TCGEN05 ? launch_tc_attention(p, st) : launch_simt_attention(p, st);

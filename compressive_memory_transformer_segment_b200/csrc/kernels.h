@@ -36,4 +36,9 @@ cudaError_t launch_simt_attention(const Problem& p, cudaStream_t stream);
 bool tc_attention_supported(int d_k, int d_v, int S, bool bf16);
 cudaError_t launch_tc_attention(const Problem& p, cudaStream_t stream);
 
+// Tensor-core memory-state scan (both rules): bf16 I/O, d_k == d_v in
+// {64, 128}, any S.  Writes bf16 M_pref and fp32 z_pref.
+bool tc_scan_supported(int d_k, int d_v, bool bf16);
+cudaError_t launch_tc_state_scan(const Problem& p, cudaStream_t stream);
+
 }  // namespace infini
