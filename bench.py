@@ -133,28 +133,70 @@ def run_reference(args, w):
 # ---------------------------------------------------------------- GPU arm
 
 class ClockSampler:
-    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    """Samples SM clock and throttle reasons while the timed region runs.
+
+    Uses NVML in a background thread (every 10 ms); falls back to an
+    nvidia-smi subprocess.  Only reads GPU state."""
+
+    NAMES = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
 
     def __init__(self, gpu_index):
         self.gpu = gpu_index
+        self.samples = []
+        self.thread = None
         self.proc = None
         self.path = os.path.join(ROOT, "gpurun_out", f"clocks_rank{gpu_index}.csv")
 
+    def _nvml_loop(self, pynvml, h):
+        bits = {"hw_slowdown": 0x8, "hw_thermal_slowdown": 0x40, "sw_thermal_slowdown": 0x20,
+                "sw_power_cap": 0x4}
+        while not self.stop:
+            try:
+                sm = pynvml.nvmlDeviceGetClockInfo(h, pynvml.NVML_CLOCK_SM)
+                smax = pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM)
+                r = pynvml.nvmlDeviceGetCurrentClocksEventReasons(h)
+                self.samples.append((sm, smax, [n for n, b in bits.items() if r & b]))
+            except Exception:
+                pass
+            time.sleep(0.01)
+
     def __enter__(self):
+        self.stop = False
+        try:
+            import threading
+            import pynvml
+            pynvml.nvmlInit()
+            idx = self.gpu
+            vis = os.environ.get("CUDA_VISIBLE_DEVICES")
+            if vis:
+                try:
+                    idx = int(vis.split(",")[self.gpu])
+                except (ValueError, IndexError):
+                    pass
+            h = pynvml.nvmlDeviceGetHandleByIndex(idx)
+            self.thread = threading.Thread(target=self._nvml_loop, args=(pynvml, h), daemon=True)
+            self.thread.start()
+            return self
+        except Exception:
+            self.thread = None
         try:
             os.makedirs(os.path.dirname(self.path), exist_ok=True)
             self.f = open(self.path, "w")
             self.proc = subprocess.Popen(
-                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
-                 "--format=csv,noheader,nounits", "-lms", "200"],
+                ["nvidia-smi", "-i", str(self.gpu),
+                 "--query-gpu=index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+                 "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+                 "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap",
+                 "--format=csv,noheader,nounits", "-lms", "50"],
                 stdout=self.f, stderr=subprocess.DEVNULL)
         except OSError:
             self.proc = None
         return self
 
     def __exit__(self, *exc):
+        self.stop = True
+        if self.thread is not None:
+            self.thread.join(timeout=2)
         if self.proc is not None:
             self.proc.terminate()
             try:
@@ -162,28 +204,25 @@ class ClockSampler:
             except subprocess.TimeoutExpired:
                 self.proc.kill()
             self.f.close()
+            for line in open(self.path):
+                parts = [x.strip() for x in line.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    sm, smax = float(parts[1]), float(parts[2])
+                except ValueError:
+                    continue
+                rs = [n for n, flag in zip(self.NAMES, parts[5:9]) if flag.lower().startswith("active")]
+                self.samples.append((sm, smax, rs))
 
     def summary(self):
-        if self.proc is None or not os.path.exists(self.path):
+        if not self.samples:
             return None
-        sm, smax, reasons = [], [], set()
-        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
-        for line in open(self.path):
-            parts = [x.strip() for x in line.split(",")]
-            if len(parts) < 9:
-                continue
-            try:
-                sm.append(float(parts[1]))
-                smax.append(float(parts[2]))
-            except ValueError:
-                continue
-            for name, flag in zip(names, parts[5:9]):
-                if flag.lower().startswith("active"):
-                    reasons.add(name)
-        if not sm:
-            return None
-        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(smax),
-                "reasons": sorted(reasons), "samples": len(sm)}
+        sm = [x[0] for x in self.samples]
+        reasons = sorted({r for x in self.samples for r in x[2]})
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(x[1] for x in self.samples),
+                "reasons": reasons, "samples": len(sm),
+                "source": "nvml" if self.thread is not None else "nvidia-smi"}
 
 
 def config_dict(w, n_gpus, l2_note):
@@ -293,6 +332,15 @@ def run_gpu(args, w):
     value = tokens / (max_ms / 1000.0)
 
     # End to end through the C ABI with host buffers (pinned), copies inside.
+    if not args.e2e:
+        if world > 1:
+            dist.destroy_process_group()
+        if rank == 0:
+            print(json.dumps({"metric": METRIC, "value": value, "unit": "tokens/s",
+                              "ms_per_step": max_ms / args.steps,
+                              "kernel_ms": {k: v[0] / max(v[1], 1) for k, v in ktimes.items()},
+                              "config": config_dict(w, world, l2_note), "note": "profiling run"}))
+        return 0
     hq_p, hk_p, hv_p = (x.pin_memory() for x in (hq, hk, hv))
     hbeta = torch.from_numpy(inp["beta"]).pin_memory()
     hM0 = torch.zeros(M0.shape, dtype=torch.float32).pin_memory()
@@ -378,6 +426,10 @@ def main():
     ap.add_argument("--config", default=DEFAULT_CONFIG, choices=sorted(configs.WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", dest="cpu_baseline", action="store_false")
+    ap.add_argument("--no-e2e", dest="e2e", action="store_false",
+                    help="skip the host-buffer end-to-end measurement (profiling runs)")
+    ap.add_argument("--batch", type=int, default=None,
+                    help="override the workload's batch size (smaller profiling captures)")
     ap.add_argument("--cpu-budget", type=float, default=15.0,
                     help="seconds of oracle work for the cpu_baseline sample")
     ap.add_argument("--reference-budget", type=float, default=60.0,
@@ -386,6 +438,8 @@ def main():
     if args.warmup < 3 and args.impl == "ours":
         args.warmup = 3
     w = configs.WORKLOADS[args.config]
+    if args.batch is not None:
+        w = w.with_(B=args.batch, name=f"{w.name}-B{args.batch}")
     if args.impl == "reference":
         return run_reference(args, w)
     return run_gpu(args, w)
