@@ -33,7 +33,7 @@ struct Shape {
   int path;
   int launches;
   // workspace layout
-  size_t ws_zpref, ws_mpref, ws_total;
+  size_t ws_zpref, ws_mpref, ws_g, ws_b, ws_dz, ws_total;
 };
 
 int check_shape(const infini_dims_t* d, int seg_len, int rule, Shape* s) {
@@ -63,11 +63,21 @@ int check_shape(const infini_dims_t* d, int seg_len, int rule, Shape* s) {
   const bool tc = tc_attention_supported(d->d_k, d->d_v, seg_len, s->bf16) &&
                   tc_scan_supported(d->d_k, d->d_v, s->bf16);
   s->path = tc ? INFINI_PATH_TCGEN05 : INFINI_PATH_SIMT;
-  s->launches = 2;
+  s->launches = tc ? 1 + tc_scan_launches(s->delta) : 2;
   const size_t mpref_elem = tc ? 2 : 4;
   s->ws_zpref = kHeader;
   s->ws_mpref = align_up(s->ws_zpref + (size_t)s->T * BHkv * d->d_k * 4);
-  s->ws_total = align_up(s->ws_mpref + (size_t)s->T * BHkv * d->d_k * d->d_v * mpref_elem);
+  size_t end = align_up(s->ws_mpref + (size_t)s->T * BHkv * d->d_k * d->d_v * mpref_elem);
+  s->ws_g = s->ws_b = s->ws_dz = end;
+  if (tc) {
+    size_t g = 0, b = 0, z = 0;
+    tc_scan_workspace(d->B, d->H_kv, s->T, d->d_k, s->delta, &g, &b, &z);
+    s->ws_g = end;
+    s->ws_b = align_up(s->ws_g + g);
+    s->ws_dz = align_up(s->ws_b + b);
+    end = align_up(s->ws_dz + z);
+  }
+  s->ws_total = end;
   return INFINI_OK;
 }
 
@@ -237,6 +247,9 @@ int infini_attn_forward(const void* q, const void* k, const void* v, const float
   p.z_pref = reinterpret_cast<float*>(ws + s.ws_zpref);
   p.M_pref = ws + s.ws_mpref;
   p.M_pref_bf16 = s.path == INFINI_PATH_TCGEN05;
+  p.Gbuf = reinterpret_cast<float*>(ws + s.ws_g);
+  p.Bbuf = reinterpret_cast<float*>(ws + s.ws_b);
+  p.dz = reinterpret_cast<float*>(ws + s.ws_dz);
   p.status = status;
 
   cudaError_t e = cudaMemcpyAsync(p.z_pref, z_in, s.z_bytes, cudaMemcpyDeviceToDevice, st);

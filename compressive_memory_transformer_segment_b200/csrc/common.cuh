@@ -28,6 +28,15 @@ template <> __device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(flo
 // ("Hugging Face Infini-Attention 再現分析", Memory Retrieval).
 __device__ __forceinline__ float elu1(float x) { return x > 0.f ? x + 1.f : expf(x); }
 
+// sigma with the hardware 2^x approximation (relative error ~2^-22), for
+// operands that are rounded to bf16 right after.
+__device__ __forceinline__ float elu1_fast(float x) {
+  if (x > 0.f) return x + 1.f;
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x * 1.4426950408889634f));
+  return y;
+}
+
 // Logistic gate sg(beta); exact 0 / 1 at -inf / +inf.
 __device__ __forceinline__ float gate_sigmoid(float b) { return 1.f / (1.f + expf(-b)); }
 

@@ -24,6 +24,10 @@ struct Problem {
   float* z_pref;       // [T][B*H_kv][d_k] f32: z_{s-1} read by segment s (slot 0 = z_in)
   void* M_pref;        // [T][B*H_kv][d_k][d_v]: M_{s-1} (f32 on the SIMT path, bf16 on tcgen05)
   bool M_pref_bf16;    // element type of M_pref
+  // Tensor-core scan only: per (segment, KV head) products and column sums.
+  float* Gbuf;         // [T][B*H_kv][d][d] f32 (delta rule)
+  float* Bbuf;         // [T][B*H_kv][d][d] f32
+  float* dz;           // [T][B*H_kv][d] f32
   unsigned int* status;  // device status word
 };
 
@@ -37,8 +41,12 @@ bool tc_attention_supported(int d_k, int d_v, int S, bool bf16);
 cudaError_t launch_tc_attention(const Problem& p, cudaStream_t stream);
 
 // Tensor-core memory-state scan (both rules): bf16 I/O, d_k == d_v in
-// {64, 128}, any S.  Writes bf16 M_pref and fp32 z_pref.
+// {64, 128}, any S.  Writes bf16 M_pref and fp32 z_pref; needs the Gbuf,
+// Bbuf and dz workspace regions sized by tc_scan_workspace.
 bool tc_scan_supported(int d_k, int d_v, bool bf16);
+int tc_scan_launches(bool delta);
+void tc_scan_workspace(int B, int H_kv, int T, int d, bool delta, size_t* g_bytes, size_t* b_bytes,
+                       size_t* dz_bytes);
 cudaError_t launch_tc_state_scan(const Problem& p, cudaStream_t stream);
 
 }  // namespace infini

@@ -25,9 +25,9 @@
 
 namespace {
 
-// 32 MiB: enough for the tiny, 200M-, 300M- and 8B-shaped workloads; a
-// 1M-token stream needs about 1 GiB and is rejected.
-constexpr size_t kNoAllocScratchBytes = size_t(32) << 20;
+// 64 MiB: enough for the tiny, 200M-, 300M- and 8B-shaped workloads; a
+// 1M-token stream needs about 1.7 GiB and is rejected.
+constexpr size_t kNoAllocScratchBytes = size_t(64) << 20;
 constexpr int kMaxDevices = 64;
 
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];

@@ -270,6 +270,35 @@ __device__ __forceinline__ float ex2_approx(float x) {
   return y;
 }
 
+// 2^x on the FMA pipe, to share the work of 2^x with the MUFU unit.
+// Cody-Waite range reduction x = n + f with n = rint(x), |f| <= 1/2 (the
+// rounding is done by adding 1.5 * 2^23, which leaves n in the low mantissa
+// bits), a degree-3 polynomial for 2^f (least-squares fit on [-1/2, 1/2]
+// weighted to the relative error; max relative error 7.6e-5), and the scale
+// by 2^n as an integer add of n << 23 to the exponent bits.  Inputs are
+// clamped to >= -125 so the exponent never underflows; results below 2^-125
+// matter to nothing here.
+__device__ __forceinline__ float exp2_poly(float x) {
+  x = fmaxf(x, -125.f);
+  const float kRound = 12582912.f;
+  const float t = x + kRound;
+  const float f = x - (t - kRound);
+  const float p = fmaf(fmaf(fmaf(0.055186376f, f, 0.24261236f), f, 0.69325829f), f, 0.99992794f);
+  return __uint_as_float(__float_as_uint(p) + (__float_as_uint(t) << 23));
+}
+
+// Two non-negative finite floats to a bf16 pair (round half up), using
+// integer ops only (keeps the conversion off the XU pipe that computes 2^x).
+__device__ __forceinline__ uint32_t pack_bf16x2_pos(float lo, float hi) {
+  const uint32_t a = __float_as_uint(lo) + 0x8000u;
+  const uint32_t b = __float_as_uint(hi) + 0x8000u;
+  return __byte_perm(a, b, 0x7632);
+}
+
+// bf16 pair -> two floats (exact).
+__device__ __forceinline__ float bf16lo_to_f32(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf16hi_to_f32(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
+
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&v);

@@ -1,34 +1,31 @@
-// Tensor-core memory-state scan for the Infini-attention forward (sm_100a).
+// Memory-state scan for the Infini-attention forward on the tensor-core path
+// (sm_100a): segment-parallel products, then a short sequential combine.
 //
-// For one (batch, KV head) chain and one 64-column block of M, the CTA scans
-// the segments in order ("Hugging Face Infini-Attention 再現分析", Memory
-// Update and State Transfer; "Leave No Context Behind" explainer,
-// "メモリの更新" with the delta rule):
-//   at the start of segment s it publishes M_{s-1} (bf16, for the attention
-//   kernel's retrieval) and z_{s-1} (fp32), then applies the segment's update
-//     linear: M += sigma(K)^T V
-//     delta : M += sigma(K)^T (V - sigma(K) M_{s-1} / (sigma(K) z_{s-1}))
-//     both  : z += sum_t sigma(K_t)
-//   and after the last segment writes M_T, z_T (fp32).
-//
-// Precision.  The update's operands are split into bf16 pairs, x = hi + lo
-// with hi = bf16(x) and lo = bf16(x - hi), so the products carry ~16
-// significant bits:
-//   dM = hi(sK)^T [hi(U) | 1] + lo(sK)^T [hi(U) | 1] + hi(sK)^T lo(U),
-// where the constant column of ones yields dz in the same TMEM tile.  TMEM
-// accumulates only the current segment's (dM, dz), restarted from zero each
-// segment: adding small products into a large running sum inside the tensor
-// core loses about one unit in the last place per instruction, which over a
-// 1M-token stream exceeds the state tolerance.  The running M and z are fp32
-// registers of the math threads (thread t holds row t of M[:, cols] and z[t])
-// and take one IEEE fp32 add of (dM, dz) per segment.
-// The delta rule's retrieval term R = sigma(K) M_{s-1} uses hi(sK) and a bf16
-// snapshot of M_{s-1}; its denominator sigma(K).z_{s-1} is fp32.
-//
-// Roles (192 threads): warp 0 = TMA producer (K and V blocks of 128 tokens),
-// warp 1 = TMEM allocation + the single MMA-issuing thread, warps 2..5 = one
-// thread per token (and per row of M).
-// TMEM columns: dM|dz accumulator [0, 80) (dM in 0..63, dz in 64), R [128, 192).
+// The update of one KV head's memory over segment s ("Hugging Face
+// Infini-Attention 再現分析", Memory Update; "Leave No Context Behind"
+// explainer, "メモリの更新" incl. the delta rule) is affine in M_{s-1}:
+//   linear: M_s = M_{s-1} + B_s
+//   delta : M_s = M_{s-1} + sigma(K)^T (V - D^-1 sigma(K) M_{s-1})
+//               = M_{s-1} - G_s M_{s-1} + B_s
+//   with B_s = sigma(K)^T V, G_s = sigma(K)^T D^-1 sigma(K),
+//   D = diag(r), r_t = sigma(k_t) . z_{s-1} (rows with r_t = 0 take no
+//   retrieval term, i.e. a zero row of D^-1), and z_s = z_{s-1} + sum_t sigma(k_t).
+// z does not depend on M, so every segment's (G_s, B_s) can be formed at once:
+//   zsum / zprefix (delta only): dz_s = column sums of sigma(K_s), then the
+//       prefix z_{s-1} for every segment and z_T;
+//   tc_segment_products (tcgen05): one CTA per (segment, KV head) forms
+//       B_s (and dz_s through a constant ones column, linear rule) and, for
+//       the delta rule, G_s = Y^T sigma(K) with Y = D^-1 sigma(K);
+//   combine_delta / combine_linear (fp32): walks the segments in order,
+//       publishing M_{s-1} (bf16, read by the attention kernel's retrieval)
+//       and z_{s-1}, and writes M_T, z_T.
+// Precision.  The products' operands are bf16 pairs x = hi + lo
+// (hi = bf16(x), lo = bf16(x - hi)), carrying ~16 significant bits:
+//   B = hi(sK)^T V + lo(sK)^T V (V is exact in bf16),
+//   G = hi(Y)^T hi(sK) + lo(Y)^T hi(sK) + hi(Y)^T lo(sK).
+// TMEM accumulates one segment only; the running state is combined in fp32
+// on CUDA cores (accumulating a long stream inside the tensor core drifts by
+// about one unit in the last place per instruction).
 #include <cuda.h>
 
 #include "kernels.h"
@@ -40,43 +37,81 @@ namespace {
 
 using namespace tc;
 
-constexpr int kTok = 128;       // tokens per block
-constexpr int kNB = 64;         // columns of M per CTA
-constexpr int kNExt = kNB + 16;  // + the z column (padded to an MMA N multiple of 16)
+// ---------------------------------------------------------------- dz and z prefix
+
+// dz[s][bh][c] = sum over the segment's rows t of sigma(k[bh][t][c]).
+// Grid (T, B*H_kv), block D threads (one per column).
+template <int D>
+__global__ void __launch_bounds__(128) zsum(const __nv_bfloat16* __restrict__ k,
+                                            float* __restrict__ dz, int L, int S) {
+  const int s = blockIdx.x, bh = blockIdx.y, c = threadIdx.x;
+  const int r0 = s * S, r1 = min(r0 + S, L);
+  const __nv_bfloat16* kc = k + (size_t)bh * L * D + c;
+  float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
+  int t = r0;
+  for (; t + 4 <= r1; t += 4) {
+    a0 += elu1(__bfloat162float(kc[(size_t)t * D]));
+    a1 += elu1(__bfloat162float(kc[(size_t)(t + 1) * D]));
+    a2 += elu1(__bfloat162float(kc[(size_t)(t + 2) * D]));
+    a3 += elu1(__bfloat162float(kc[(size_t)(t + 3) * D]));
+  }
+  for (; t < r1; ++t) a0 += elu1(__bfloat162float(kc[(size_t)t * D]));
+  dz[((size_t)s * gridDim.y + bh) * D + c] = (a0 + a1) + (a2 + a3);
+}
+
+// z_{s-1} for s = 1..T-1 into z_pref (slot 0 already holds z_in) and z_T.
+// Grid (B*H_kv), block D threads.
+template <int D>
+__global__ void __launch_bounds__(128) zprefix(const float* __restrict__ dz, float* __restrict__ z_pref,
+                                               float* __restrict__ z_out, int T) {
+  const int bh = blockIdx.x, c = threadIdx.x, BH = gridDim.x;
+  float z = z_pref[(size_t)bh * D + c];
+  for (int s = 1; s < T; ++s) {
+    z += dz[((size_t)(s - 1) * BH + bh) * D + c];
+    z_pref[((size_t)s * BH + bh) * D + c] = z;
+  }
+  z_out[(size_t)bh * D + c] = z + dz[((size_t)(T - 1) * BH + bh) * D + c];
+}
+
+// ---------------------------------------------------------------- segment products
+
+constexpr int kTok = 128;  // tokens per block
 constexpr int kThreads = 192;
 constexpr uint32_t kTmemCols = 256;
-constexpr uint32_t kColR = 128;
 
-template <int D>
-struct ScanSmem {
-  static constexpr int kK = 0;                       // K block [128][D] (D/64 panels)
-  static constexpr int kV = kK + kTok * D * 2;       // V block [128][64]
-  static constexpr int kSkHi = kV + kTok * 64 * 2;   // sigma(K) hi [128][128] (2 panels)
+template <int D, bool DELTA>
+struct ProdSmem {
+  static constexpr int kK = 0;                                      // K block [128][D]
+  static constexpr int kV = kK + kTok * D * 2;                      // V block [128][D] (+ ones)
+  static constexpr int kVBytes = kTok * D * 2 + (DELTA ? 0 : kTok * 64 * 2);
+  static constexpr int kSkHi = kV + kVBytes;                        // [128 tok][128] (2 panels)
   static constexpr int kSkLo = kSkHi + kTok * 128 * 2;
-  static constexpr int kUHi = kSkLo + kTok * 128 * 2;  // [U_hi | ones] (2 panels)
-  static constexpr int kULo = kUHi + kTok * 128 * 2;   // U_lo (1 panel)
-  static constexpr int kMb = kULo + kTok * 64 * 2;     // bf16 M_{s-1}[:, cols] [D][64]
-  static constexpr int kZ = kMb + D * 64 * 2;          // fp32 z_{s-1} [128]
+  static constexpr int kYHi = kSkLo + kTok * 128 * 2;               // delta only
+  static constexpr int kYLo = kYHi + (DELTA ? kTok * 128 * 2 : 0);
+  static constexpr int kZ = kYLo + (DELTA ? kTok * 128 * 2 : 0);    // fp32 z_{s-1}
   static constexpr int kBar = kZ + 128 * 4;
-  // k_full, k_empty, v_full, v_empty, sk_ready, r_ready, u_ready, sk_free,
-  // mb_ready, drain
-  static constexpr int kNumBars = 10;
+  // k_full k_empty v_full v_empty op_ready op_free done
+  static constexpr int kNumBars = 7;
   static constexpr int kTmemSlot = kBar + kNumBars * 8;
   static constexpr int kAbort = kTmemSlot + 4;
   static constexpr int kAlloc = kAbort + 4 + 1024;
 };
 
+// Grid (T, B*H_kv).  Roles: warp 0 TMA producer (K, V blocks), warp 1 TMEM
+// allocation + MMA issue, warps 2..5 one thread per token of the block (and,
+// at the end, per row of the products).
+// TMEM: delta G [0, D), B [128, 128 + D); linear [B | dz] [0, D + 16).
 template <int D, bool DELTA>
 __global__ void __launch_bounds__(kThreads, 1)
-tc_state_scan(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
-              const float* __restrict__ M_in, float* __restrict__ M_out, float* __restrict__ z_out,
-              float* __restrict__ z_pref, __nv_bfloat16* __restrict__ M_pref,
-              unsigned int* __restrict__ status, int L, int S, int T) {
-  using SM = ScanSmem<D>;
-  const int cb = blockIdx.x;  // column block
-  const int c0 = cb * kNB;
-  const int bh = blockIdx.y;
-  const int BH = gridDim.y;
+tc_segment_products(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
+                    const float* __restrict__ z_pref, float* __restrict__ Gbuf,
+                    float* __restrict__ Bbuf, float* __restrict__ dz,
+                    unsigned int* __restrict__ status, int L, int S) {
+  using SM = ProdSmem<D, DELTA>;
+  const int s = blockIdx.x, bh = blockIdx.y, BH = gridDim.y;
+  const int seg0 = s * S, seg_len = min(S, L - seg0);
+  const int nblk = (seg_len + kTok - 1) / kTok;
+  const size_t slice = (size_t)s * BH + bh;
 
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   unsigned char* smem = reinterpret_cast<unsigned char*>(
@@ -85,21 +120,17 @@ tc_state_scan(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ 
   unsigned char* sV = smem + SM::kV;
   unsigned char* sSkHi = smem + SM::kSkHi;
   unsigned char* sSkLo = smem + SM::kSkLo;
-  unsigned char* sUHi = smem + SM::kUHi;
-  unsigned char* sULo = smem + SM::kULo;
-  unsigned char* sMb = smem + SM::kMb;
+  unsigned char* sYHi = smem + SM::kYHi;
+  unsigned char* sYLo = smem + SM::kYLo;
   float* zs = reinterpret_cast<float*>(smem + SM::kZ);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + SM::kBar);
   uint64_t* k_full = bars + 0;
   uint64_t* k_empty = bars + 1;
   uint64_t* v_full = bars + 2;
   uint64_t* v_empty = bars + 3;
-  uint64_t* sk_ready = bars + 4;
-  uint64_t* r_ready = bars + 5;
-  uint64_t* u_ready = bars + 6;
-  uint64_t* sk_free = bars + 7;
-  uint64_t* mb_ready = bars + 8;
-  uint64_t* drain = bars + 9;
+  uint64_t* op_ready = bars + 4;
+  uint64_t* op_free = bars + 5;
+  uint64_t* done = bars + 6;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + SM::kTmemSlot);
   volatile int* abort = reinterpret_cast<volatile int*>(smem + SM::kAbort);
 
@@ -109,13 +140,10 @@ tc_state_scan(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ 
     mbar_init(k_full, 1);
     mbar_init(k_empty, 128);
     mbar_init(v_full, 1);
-    mbar_init(v_empty, 128);
-    mbar_init(sk_ready, 128);
-    mbar_init(r_ready, 1);
-    mbar_init(u_ready, 128);
-    mbar_init(sk_free, 1);
-    mbar_init(mb_ready, 128);
-    mbar_init(drain, 1);
+    mbar_init(v_empty, 1);
+    mbar_init(op_ready, 128);
+    mbar_init(op_free, 1);
+    mbar_init(done, 1);
     *abort = 0;
     fence_mbar_init();
   }
@@ -124,233 +152,193 @@ tc_state_scan(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ 
     tmem_relinquish();
     tc_fence_before();
   }
-  // Constant parts of the operand buffers: the ones column of [U_hi | ones]
-  // (panel 1, column 0) and, for D = 64, the zero upper half of sigma(K).
+  // Constant operand parts: the ones column after V (linear rule) and, for
+  // D = 64, the zero upper halves of sigma(K) and Y (the products' M = 128).
   for (int i = threadIdx.x; i < kTok * 64 * 2 / 16; i += kThreads) {
     const int row = i / 8, chunk = i % 8;
-    uint4 v = make_uint4(0, 0, 0, 0);
-    if (chunk == (row & 7)) v.x = 0x3F80u;  // element (row, 0) = bf16(1.0)
-    *reinterpret_cast<uint4*>(sUHi + kTok * 128 + i * 16) = v;
+    if (!DELTA) {
+      uint4 v = make_uint4(0, 0, 0, 0);
+      if (chunk == (row & 7)) v.x = 0x3F80u;  // element (row, 0) = bf16(1.0)
+      *reinterpret_cast<uint4*>(sV + kTok * D * 2 + i * 16) = v;
+    }
     if (D == 64) {
-      *reinterpret_cast<uint4*>(sSkHi + kTok * 128 + i * 16) = make_uint4(0, 0, 0, 0);
-      *reinterpret_cast<uint4*>(sSkLo + kTok * 128 + i * 16) = make_uint4(0, 0, 0, 0);
+      const uint4 zero = make_uint4(0, 0, 0, 0);
+      *reinterpret_cast<uint4*>(sSkHi + kTok * 128 + i * 16) = zero;
+      *reinterpret_cast<uint4*>(sSkLo + kTok * 128 + i * 16) = zero;
+      if (DELTA) {
+        *reinterpret_cast<uint4*>(sYHi + kTok * 128 + i * 16) = zero;
+        *reinterpret_cast<uint4*>(sYLo + kTok * 128 + i * 16) = zero;
+      }
     }
   }
+  if (DELTA)
+    for (int i = threadIdx.x; i < 128; i += kThreads) zs[i] = i < D ? z_pref[slice * D + i] : 0.f;
   fence_proxy_async();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  const uint32_t tM = tmem;
-  const uint32_t tR = tmem + kColR;
 
   if (warp == 0) {
     if (lane == 0) {
       // ------------------------------------------------ TMA producer
-      int gb = 0, issued_k = 0, issued_v = 0;
-      bool ok = true;
-      for (int s = 0; ok && s < T; ++s) {
-        const int seg0 = s * S, seg_len = min(S, L - seg0);
-        const int nblk = (seg_len + kTok - 1) / kTok;
-        for (int tb = 0; tb < nblk; ++tb, ++gb) {
-          const uint32_t par = (gb & 1) ^ 1;
-          if (!(ok = mbar_wait(k_empty, par, abort, status))) break;
-          mbar_arrive_expect_tx(k_full, kTok * D * 2);
-          for (int p = 0; p < D / 64; ++p)
-            tma_load_3d(sK + p * kTok * 128, &tm_k, k_full, p * 64, seg0 + tb * kTok, bh);
-          issued_k = gb + 1;
-          if (!(ok = mbar_wait(v_empty, par, abort, status))) break;
-          mbar_arrive_expect_tx(v_full, kTok * 64 * 2);
-          tma_load_3d(sV, &tm_v, v_full, c0, seg0 + tb * kTok, bh);
-          issued_v = gb + 1;
-        }
+      int issued_k = 0, issued_v = 0;
+      for (int blk = 0; blk < nblk; ++blk) {
+        const uint32_t par = (blk & 1) ^ 1;
+        if (!mbar_wait(k_empty, par, abort, status)) break;
+        mbar_arrive_expect_tx(k_full, kTok * D * 2);
+        for (int p = 0; p < D / 64; ++p)
+          tma_load_3d(sK + p * kTok * 128, &tm_k, k_full, p * 64, seg0 + blk * kTok, bh);
+        issued_k = blk + 1;
+        if (!mbar_wait(v_empty, par, abort, status)) break;
+        mbar_arrive_expect_tx(v_full, kTok * D * 2);
+        for (int p = 0; p < D / 64; ++p)
+          tma_load_3d(sV + p * kTok * 128, &tm_v, v_full, p * 64, seg0 + blk * kTok, bh);
+        issued_v = blk + 1;
       }
-      // Drain: the last copies must have landed before the CTA exits.
       if (issued_k > 0) mbar_wait(k_full, (issued_k - 1) & 1, abort, status, false);
       if (issued_v > 0) mbar_wait(v_full, (issued_v - 1) & 1, abort, status, false);
     }
   } else if (warp == 1) {
     if (lane == 0) {
       // ------------------------------------------------ MMA issuer
-      constexpr uint32_t idesc_r = idesc_bf16_f32(128, kNB, false, true);
-      constexpr uint32_t idesc_ext = idesc_bf16_f32(128, kNExt, true, true);
-      constexpr uint32_t idesc_lo = idesc_bf16_f32(128, kNB, true, true);
-      const uint32_t skhi = smem_u32(sSkHi), sklo = smem_u32(sSkLo);
-      const uint32_t uhi = smem_u32(sUHi), ulo = smem_u32(sULo), mb = smem_u32(sMb);
-      int gb = 0;
+      // All operands are MN-major [tokens][128] tiles (panels of 64 columns,
+      // 16 KiB apart); one 16-token K step = 2048 bytes.
+      const uint64_t skhi = sw128_desc(smem_u32(sSkHi), kTok * 128, 1024);
+      const uint64_t sklo = sw128_desc(smem_u32(sSkLo), kTok * 128, 1024);
+      const uint64_t yhi = sw128_desc(smem_u32(sYHi), kTok * 128, 1024);
+      const uint64_t ylo = sw128_desc(smem_u32(sYLo), kTok * 128, 1024);
+      const uint64_t vv = sw128_desc(smem_u32(sV), kTok * 128, 1024);
+      constexpr uint32_t idesc_d = idesc_bf16_f32(128, D, true, true);
+      constexpr uint32_t idesc_ext = idesc_bf16_f32(128, D + 16, true, true);
+      const uint32_t tG = tmem, tB = DELTA ? tmem + 128 : tmem;
       bool ok = true;
-      for (int s = 0; ok && s < T; ++s) {
-        const int seg_len = min(S, L - s * S);
-        const int nblk = (seg_len + kTok - 1) / kTok;
-        if (!(ok = mbar_wait(mb_ready, s & 1, abort, status))) break;
-        for (int tb = 0; tb < nblk; ++tb, ++gb) {
-          if (!(ok = mbar_wait(sk_ready, gb & 1, abort, status))) break;
-          tc_fence_after();
+      for (int blk = 0; ok && blk < nblk; ++blk) {
+        if (!(ok = mbar_wait(op_ready, blk & 1, abort, status))) break;
+        if (!(ok = mbar_wait(v_full, blk & 1, abort, status))) break;
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < kTok / 16; ++kk) {
+          const uint32_t st = mnmajor_step(kk);
+          const uint32_t acc = (blk > 0 || kk > 0) ? 1u : 0u;
           if (DELTA) {
-            // R = hi(sigma(K)) M_{s-1}: tokens x columns, K = D.
-#pragma unroll
-            for (int kk = 0; kk < D / 16; ++kk) {
-              const uint32_t off = (kk >> 2) * (kTok * 128) + (kk & 3) * 32;
-              mma_ss(tR, sw128_desc(skhi + off, 16, 1024), sw128_desc(mb + kk * 2048, D * 128, 1024),
-                     idesc_r, kk > 0 ? 1u : 0u);
-            }
-            tc_commit(r_ready);
+            mma_ss(tG, yhi + st, skhi + st, idesc_d, acc);
+            mma_ss(tG, ylo + st, skhi + st, idesc_d, 1u);
+            mma_ss(tG, yhi + st, sklo + st, idesc_d, 1u);
+            mma_ss(tB, skhi + st, vv + st, idesc_d, acc);
+            mma_ss(tB, sklo + st, vv + st, idesc_d, 1u);
+          } else {
+            mma_ss(tB, skhi + st, vv + st, idesc_ext, acc);
+            mma_ss(tB, sklo + st, vv + st, idesc_ext, 1u);
           }
-          if (!(ok = mbar_wait(u_ready, gb & 1, abort, status))) break;
-          tc_fence_after();
-          // dM|dz += sigma(K)^T [U | 1], over the block's 128 tokens.
-#pragma unroll
-          for (int kk = 0; kk < kTok / 16; ++kk) {
-            const uint64_t a_hi = sw128_desc(skhi + kk * 2048, kTok * 128, 1024);
-            const uint64_t a_lo = sw128_desc(sklo + kk * 2048, kTok * 128, 1024);
-            const uint64_t b_hi = sw128_desc(uhi + kk * 2048, kTok * 128, 1024);
-            // The segment's first product restarts the accumulator at zero.
-            mma_ss(tM, a_hi, b_hi, idesc_ext, (tb > 0 || kk > 0) ? 1u : 0u);
-            mma_ss(tM, a_lo, b_hi, idesc_ext, 1u);
-            if (DELTA) mma_ss(tM, a_hi, sw128_desc(ulo + kk * 2048, kTok * 128, 1024), idesc_lo, 1u);
-          }
-          tc_commit(sk_free);
         }
+        tc_commit(op_free);
+        tc_commit(v_empty);
       }
-      tc_commit(drain);
-      mbar_wait(drain, 0, abort, status, false);
+      tc_commit(done);
+      mbar_wait(done, 0, abort, status, false);
     }
   } else {
     // -------------------------------------------------- math threads
-    const int t = 32 * (warp & 3) + lane;  // token within the block = TMEM lane = row of M
+    const int t = 32 * (warp & 3) + lane;  // token of the block; later, row of the products
     const uint32_t lane_off = (uint32_t)(32 * (warp & 3)) << 16;
     bool ok = true;
-    // Running state, fp32: row t of M[:, c0..c0+63] and z[t] (rows >= D stay 0).
-    float macc[kNB];
-    float zacc = 0.f;
-#pragma unroll
-    for (int i = 0; i < kNB; ++i) macc[i] = t < D ? M_in[((size_t)bh * D + t) * D + c0 + i] : 0.f;
-    // z_in was copied to slot 0 of z_pref before this kernel.
-    if (t < D) zacc = z_pref[(size_t)bh * D + t];
-    int gb = 0;
-    for (int s = 0; s <= T && ok; ++s) {
-      if (gb > 0) {
-        // The previous segment's products are complete: fold (dM, dz) into
-        // the running state (this also frees Mb, sigma(K) and U).
-        ok = __all_sync(0xffffffffu, mbar_wait(sk_free, (gb - 1) & 1, abort, status));
+    for (int blk = 0; blk < nblk; ++blk) {
+      if (blk > 0) {
+        ok = __all_sync(0xffffffffu, mbar_wait(op_free, (blk - 1) & 1, abort, status));
         if (!ok) break;
-        tc_fence_after();
-        uint32_t drow[64], dz[32];
-        tmem_ld32(tM + lane_off, drow);
-        tmem_ld32(tM + lane_off + 32, drow + 32);
-        tmem_ld32(tM + lane_off + 64, dz);
-        tmem_wait_ld();
-#pragma unroll
-        for (int i = 0; i < kNB; ++i) macc[i] += __uint_as_float(drow[i]);
-        zacc += __uint_as_float(dz[0]);
       }
-      if (s == T) {  // final state
-        if (t < D) {
-          float4* dst = reinterpret_cast<float4*>(M_out + ((size_t)bh * D + t) * D + c0);
-#pragma unroll
-          for (int i = 0; i < 16; ++i)
-            dst[i] = make_float4(macc[4 * i], macc[4 * i + 1], macc[4 * i + 2], macc[4 * i + 3]);
-          if (cb == 0) z_out[(size_t)bh * D + t] = zacc;
-        }
-        break;
-      }
-      const float zt = zacc;
-      if (t < D) {
-        uint4* gdst = reinterpret_cast<uint4*>(M_pref + (((size_t)s * BH + bh) * D + t) * D + c0);
-#pragma unroll
-        for (int c8 = 0; c8 < 8; ++c8) {
-          uint4 v;
-          v.x = pack_bf16x2(macc[8 * c8 + 0], macc[8 * c8 + 1]);
-          v.y = pack_bf16x2(macc[8 * c8 + 2], macc[8 * c8 + 3]);
-          v.z = pack_bf16x2(macc[8 * c8 + 4], macc[8 * c8 + 5]);
-          v.w = pack_bf16x2(macc[8 * c8 + 6], macc[8 * c8 + 7]);
-          *reinterpret_cast<uint4*>(sMb + sw128_offset(t, 8 * c8, D)) = v;
-          gdst[c8] = v;
-        }
-        if (cb == 0) z_pref[((size_t)s * BH + bh) * D + t] = zt;
-      }
-      zs[t] = t < D ? zt : 0.f;
-      fence_proxy_async();
-      mbar_arrive(mb_ready);
-      // Every math thread's z entry is in zs before any thread reads it.
-      ok = __all_sync(0xffffffffu, mbar_wait(mb_ready, s & 1, abort, status));
+      ok = __all_sync(0xffffffffu, mbar_wait(k_full, blk & 1, abort, status));
       if (!ok) break;
-
-      const int seg0 = s * S, seg_len = min(S, L - seg0);
-      const int nblk = (seg_len + kTok - 1) / kTok;
-      for (int tb = 0; tb < nblk; ++tb, ++gb) {
-        if (tb > 0) {
-          ok = __all_sync(0xffffffffu, mbar_wait(sk_free, (gb - 1) & 1, abort, status));
-          if (!ok) break;
+      const bool valid = blk * kTok + t < seg_len;
+      // sigma(K) row t as hi/lo pairs (rows past the segment are 0), and
+      // r_t = sigma(k_t) . z_{s-1} (delta).
+      float r = 0.f;
+#pragma unroll 4
+      for (int c8 = 0; c8 < D / 8; ++c8) {
+        const uint32_t off = sw128_offset(t, 8 * c8, kTok);
+        const uint4 kv = *reinterpret_cast<const uint4*>(sK + off);
+        const uint32_t kw[4] = {kv.x, kv.y, kv.z, kv.w};
+        uint32_t hw[4], lw[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const float a = valid ? elu1_fast(bf16lo_to_f32(kw[i])) : 0.f;
+          const float b = valid ? elu1_fast(bf16hi_to_f32(kw[i])) : 0.f;
+          if (DELTA) {
+            r = fmaf(a, zs[8 * c8 + 2 * i], r);
+            r = fmaf(b, zs[8 * c8 + 2 * i + 1], r);
+          }
+          hw[i] = pack_bf16x2(a, b);
+          lw[i] = pack_bf16x2(a - bf16lo_to_f32(hw[i]), b - bf16hi_to_f32(hw[i]));
         }
-        const bool valid = tb * kTok + t < seg_len;
-        // sigma(K) row t as hi/lo bf16 pairs, and r_t = sigma(k_t) . z_{s-1}.
-        ok = __all_sync(0xffffffffu, mbar_wait(k_full, gb & 1, abort, status));
-        if (!ok) break;
-        float r = 0.f;
+        *reinterpret_cast<uint4*>(sSkHi + off) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+        *reinterpret_cast<uint4*>(sSkLo + off) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
+      }
+      mbar_arrive(k_empty);
+      if (DELTA) {
+        // Y = sigma(K) / r (0 where r = 0), from the pair just written.
+        const float w = r != 0.f ? 1.f / r : 0.f;
 #pragma unroll 4
         for (int c8 = 0; c8 < D / 8; ++c8) {
           const uint32_t off = sw128_offset(t, 8 * c8, kTok);
-          const uint4 kv = *reinterpret_cast<const uint4*>(sK + off);
-          const uint32_t kw[4] = {kv.x, kv.y, kv.z, kv.w};
+          const uint4 hv = *reinterpret_cast<const uint4*>(sSkHi + off);
+          const uint4 lv = *reinterpret_cast<const uint4*>(sSkLo + off);
+          const uint32_t hh[4] = {hv.x, hv.y, hv.z, hv.w}, ll[4] = {lv.x, lv.y, lv.z, lv.w};
           uint32_t hw[4], lw[4];
 #pragma unroll
           for (int i = 0; i < 4; ++i) {
-            const __nv_bfloat162 pr = *reinterpret_cast<const __nv_bfloat162*>(&kw[i]);
-            const float a = valid ? elu1(__low2float(pr)) : 0.f;
-            const float b = valid ? elu1(__high2float(pr)) : 0.f;
-            r = fmaf(a, zs[8 * c8 + 2 * i], r);
-            r = fmaf(b, zs[8 * c8 + 2 * i + 1], r);
-            const __nv_bfloat162 hi = __floats2bfloat162_rn(a, b);
-            hw[i] = *reinterpret_cast<const uint32_t*>(&hi);
-            lw[i] = pack_bf16x2(a - __low2float(hi), b - __high2float(hi));
+            const float a = w * (bf16lo_to_f32(hh[i]) + bf16lo_to_f32(ll[i]));
+            const float b = w * (bf16hi_to_f32(hh[i]) + bf16hi_to_f32(ll[i]));
+            hw[i] = pack_bf16x2(a, b);
+            lw[i] = pack_bf16x2(a - bf16lo_to_f32(hw[i]), b - bf16hi_to_f32(hw[i]));
           }
-          *reinterpret_cast<uint4*>(sSkHi + off) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
-          *reinterpret_cast<uint4*>(sSkLo + off) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
+          *reinterpret_cast<uint4*>(sYHi + off) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+          *reinterpret_cast<uint4*>(sYLo + off) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
         }
-        mbar_arrive(k_empty);
-        fence_proxy_async();
-        mbar_arrive(sk_ready);
-        // U = V - R / r (delta) or V (linear), as hi/lo pairs, row t.
-        uint32_t rrow[64];
-        const float inv_r = r != 0.f ? 1.f / r : 0.f;
-        if (DELTA) {
-          ok = __all_sync(0xffffffffu, mbar_wait(r_ready, gb & 1, abort, status));
-          if (!ok) break;
-          tc_fence_after();
-          tmem_ld32(tR + lane_off, rrow);
-          tmem_ld32(tR + lane_off + 32, rrow + 32);
+      }
+      fence_proxy_async();
+      mbar_arrive(op_ready);
+    }
+    // The segment's products, row t (t < D), to the workspace in fp32.
+    if (ok) ok = __all_sync(0xffffffffu, mbar_wait(done, 0, abort, status));
+    if (ok) {
+      tc_fence_after();
+      if (DELTA) {
+#pragma unroll
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t g[32], bb[32];
+          tmem_ld32(tmem + lane_off + c * 32, g);
+          tmem_ld32(tmem + 128 + lane_off + c * 32, bb);
           tmem_wait_ld();
-        }
-        ok = __all_sync(0xffffffffu, mbar_wait(v_full, gb & 1, abort, status));
-        if (!ok) break;
+          if (t < D) {
+            float4* gd = reinterpret_cast<float4*>(Gbuf + (slice * D + t) * D + c * 32);
+            float4* bd = reinterpret_cast<float4*>(Bbuf + (slice * D + t) * D + c * 32);
 #pragma unroll
-        for (int c8 = 0; c8 < 8; ++c8) {
-          const uint32_t off = sw128_offset(t, 8 * c8, kTok);
-          const uint4 vv = *reinterpret_cast<const uint4*>(sV + off);
-          if (!DELTA) {
-            *reinterpret_cast<uint4*>(sUHi + off) = valid ? vv : make_uint4(0, 0, 0, 0);
-            continue;
+            for (int i = 0; i < 8; ++i) {
+              gd[i] = make_float4(__uint_as_float(g[4 * i]), __uint_as_float(g[4 * i + 1]),
+                                  __uint_as_float(g[4 * i + 2]), __uint_as_float(g[4 * i + 3]));
+              bd[i] = make_float4(__uint_as_float(bb[4 * i]), __uint_as_float(bb[4 * i + 1]),
+                                  __uint_as_float(bb[4 * i + 2]), __uint_as_float(bb[4 * i + 3]));
+            }
           }
-          const uint32_t vw[4] = {vv.x, vv.y, vv.z, vv.w};
-          uint32_t hw[4], lw[4];
-#pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            const __nv_bfloat162 pr = *reinterpret_cast<const __nv_bfloat162*>(&vw[i]);
-            const int c = 8 * c8 + 2 * i;
-            float u0 = __low2float(pr) - __uint_as_float(rrow[c]) * inv_r;
-            float u1 = __high2float(pr) - __uint_as_float(rrow[c + 1]) * inv_r;
-            if (!valid) u0 = u1 = 0.f;
-            const __nv_bfloat162 hi = __floats2bfloat162_rn(u0, u1);
-            hw[i] = *reinterpret_cast<const uint32_t*>(&hi);
-            lw[i] = pack_bf16x2(u0 - __low2float(hi), u1 - __high2float(hi));
-          }
-          *reinterpret_cast<uint4*>(sUHi + off) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
-          *reinterpret_cast<uint4*>(sULo + off) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
         }
-        mbar_arrive(v_empty);
-        fence_proxy_async();
-        tc_fence_before();
-        mbar_arrive(u_ready);
+      } else {
+#pragma unroll
+        for (int c = 0; c < D / 32 + 1; ++c) {
+          uint32_t bb[32];
+          tmem_ld32(tmem + lane_off + c * 32, bb);
+          tmem_wait_ld();
+          if (t < D) {
+            if (c < D / 32) {
+              float4* bd = reinterpret_cast<float4*>(Bbuf + (slice * D + t) * D + c * 32);
+#pragma unroll
+              for (int i = 0; i < 8; ++i)
+                bd[i] = make_float4(__uint_as_float(bb[4 * i]), __uint_as_float(bb[4 * i + 1]),
+                                    __uint_as_float(bb[4 * i + 2]), __uint_as_float(bb[4 * i + 3]));
+            } else {
+              dz[slice * D + t] = __uint_as_float(bb[0]);
+            }
+          }
+        }
       }
     }
   }
@@ -361,6 +349,115 @@ tc_state_scan(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ 
     tmem_dealloc(tmem, kTmemCols);
   }
 }
+
+// ---------------------------------------------------------------- sequential combine
+
+constexpr int kCB = 16;  // columns of M per combine CTA (delta)
+
+// Delta rule: M_s = M_{s-1} - G_s M_{s-1} + B_s on columns [16 cb, 16 cb + 16).
+// Grid (B*H_kv, D/16), block 256 threads: thread -> (row k = tid % 128,
+// 8 columns); rows >= D idle for D = 64.  Plain (non-spinning) block barriers.
+template <int D>
+__global__ void __launch_bounds__(256) combine_delta(const float* __restrict__ M_in,
+                                                     const float* __restrict__ Gbuf,
+                                                     const float* __restrict__ Bbuf,
+                                                     __nv_bfloat16* __restrict__ M_pref,
+                                                     float* __restrict__ M_out, int T) {
+  extern __shared__ float csm[];
+  float* sG = csm;                  // G_s, rows padded to D + 1 floats
+  float* sM = csm + D * (D + 1);    // M_{s-1}[:, 16 columns]
+  const int bh = blockIdx.x, c0 = blockIdx.y * kCB, BH = gridDim.x;
+  const int tid = threadIdx.x, k = tid & 127, cg = (tid >> 7) * 8;
+  const bool active = k < D;
+  float m[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) m[i] = active ? M_in[((size_t)bh * D + k) * D + c0 + cg + i] : 0.f;
+  for (int s = 0; s < T; ++s) {
+    const size_t slice = (size_t)s * BH + bh;
+    // Publish M_{s-1} (bf16) for segment s's retrieval.
+    if (active) {
+      uint4 w;
+      w.x = pack_bf16x2(m[0], m[1]);
+      w.y = pack_bf16x2(m[2], m[3]);
+      w.z = pack_bf16x2(m[4], m[5]);
+      w.w = pack_bf16x2(m[6], m[7]);
+      *reinterpret_cast<uint4*>(M_pref + (slice * D + k) * D + c0 + cg) = w;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) sM[k * kCB + cg + i] = m[i];
+    }
+    const float* G = Gbuf + slice * D * D;
+    for (int e = tid; e < D * D; e += 256) sG[(e / D) * (D + 1) + (e % D)] = G[e];
+    __syncthreads();
+    if (active) {
+      float acc[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) acc[i] = 0.f;
+#pragma unroll 4
+      for (int kk = 0; kk < D; ++kk) {
+        const float gv = sG[k * (D + 1) + kk];
+        const float4 ma = *reinterpret_cast<const float4*>(sM + kk * kCB + cg);
+        const float4 mb = *reinterpret_cast<const float4*>(sM + kk * kCB + cg + 4);
+        acc[0] = fmaf(gv, ma.x, acc[0]);
+        acc[1] = fmaf(gv, ma.y, acc[1]);
+        acc[2] = fmaf(gv, ma.z, acc[2]);
+        acc[3] = fmaf(gv, ma.w, acc[3]);
+        acc[4] = fmaf(gv, mb.x, acc[4]);
+        acc[5] = fmaf(gv, mb.y, acc[5]);
+        acc[6] = fmaf(gv, mb.z, acc[6]);
+        acc[7] = fmaf(gv, mb.w, acc[7]);
+      }
+      const float* Bk = Bbuf + (slice * D + k) * D + c0 + cg;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) m[i] = (m[i] - acc[i]) + Bk[i];
+    }
+    __syncthreads();
+  }
+  if (active)
+#pragma unroll
+    for (int i = 0; i < 8; ++i) M_out[((size_t)bh * D + k) * D + c0 + cg + i] = m[i];
+}
+
+// Linear rule: M_s = M_{s-1} + B_s, z_s = z_{s-1} + dz_s, element-parallel.
+// Grid (B*H_kv, ceil(D*D / 1024)), block 256 threads x 4 elements; block
+// (bh, 0) also carries z.
+template <int D>
+__global__ void __launch_bounds__(256) combine_linear(const float* __restrict__ M_in,
+                                                      const float* __restrict__ Bbuf,
+                                                      const float* __restrict__ dz,
+                                                      __nv_bfloat16* __restrict__ M_pref,
+                                                      float* __restrict__ z_pref,
+                                                      float* __restrict__ M_out,
+                                                      float* __restrict__ z_out, int T) {
+  const int bh = blockIdx.x, BH = gridDim.x;
+  const int e = (blockIdx.y * 256 + threadIdx.x) * 4;  // element of the D x D matrix
+  if (e < D * D) {
+    float4 m = *reinterpret_cast<const float4*>(M_in + (size_t)bh * D * D + e);
+    for (int s = 0; s < T; ++s) {
+      const size_t slice = (size_t)s * BH + bh;
+      uint2 w;
+      w.x = pack_bf16x2(m.x, m.y);
+      w.y = pack_bf16x2(m.z, m.w);
+      *reinterpret_cast<uint2*>(M_pref + slice * D * D + e) = w;
+      const float4 b = *reinterpret_cast<const float4*>(Bbuf + slice * D * D + e);
+      m.x += b.x;
+      m.y += b.y;
+      m.z += b.z;
+      m.w += b.w;
+    }
+    *reinterpret_cast<float4*>(M_out + (size_t)bh * D * D + e) = m;
+  }
+  if (blockIdx.y == 0 && threadIdx.x < D) {
+    const int c = threadIdx.x;
+    float z = z_pref[(size_t)bh * D + c];  // slot 0 = z_in
+    for (int s = 1; s < T; ++s) {
+      z += dz[((size_t)(s - 1) * BH + bh) * D + c];
+      z_pref[((size_t)s * BH + bh) * D + c] = z;
+    }
+    z_out[(size_t)bh * D + c] = z + dz[((size_t)(T - 1) * BH + bh) * D + c];
+  }
+}
+
+// ---------------------------------------------------------------- host side
 
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
@@ -393,20 +490,43 @@ bool make_map(CUtensorMap* m, const void* base, uint64_t cols, uint64_t rows, ui
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+template <int D, bool DELTA>
+cudaError_t launch_products(const Problem& p, const CUtensorMap& tk, const CUtensorMap& tv,
+                            cudaStream_t stream) {
+  const int smem = ProdSmem<D, DELTA>::kAlloc;
+  auto kern = tc_segment_products<D, DELTA>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return e;
+  kern<<<dim3(p.T, p.B * p.H_kv), kThreads, smem, stream>>>(tk, tv, p.z_pref, p.Gbuf, p.Bbuf, p.dz,
+                                                           p.status, p.L, p.S);
+  return cudaGetLastError();
+}
+
 template <int D>
 cudaError_t launch(const Problem& p, cudaStream_t stream) {
   CUtensorMap tk, tv;
   const uint64_t BHkv = (uint64_t)p.B * p.H_kv;
   if (!make_map(&tk, p.k, D, p.L, BHkv, kTok) || !make_map(&tv, p.v, D, p.L, BHkv, kTok))
     return cudaErrorInvalidValue;
-  const int smem = ScanSmem<D>::kAlloc;
-  dim3 grid(D / kNB, (unsigned)BHkv);
-  auto kern = p.delta ? tc_state_scan<D, true> : tc_state_scan<D, false>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-  if (e != cudaSuccess) return e;
-  kern<<<grid, kThreads, smem, stream>>>(tk, tv, p.M_in, p.M_out, p.z_out, p.z_pref,
-                                         static_cast<__nv_bfloat16*>(p.M_pref), p.status, p.L,
-                                         p.S, p.T);
+  const unsigned BH = (unsigned)BHkv;
+  __nv_bfloat16* Mp = static_cast<__nv_bfloat16*>(p.M_pref);
+  cudaError_t e;
+  if (p.delta) {
+    zsum<D><<<dim3(p.T, BH), D, 0, stream>>>(static_cast<const __nv_bfloat16*>(p.k), p.dz, p.L, p.S);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    zprefix<D><<<BH, D, 0, stream>>>(p.dz, p.z_pref, p.z_out, p.T);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    if ((e = launch_products<D, true>(p, tk, tv, stream)) != cudaSuccess) return e;
+    const int csmem = (D * (D + 1) + D * kCB) * (int)sizeof(float);
+    e = cudaFuncSetAttribute(combine_delta<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, csmem);
+    if (e != cudaSuccess) return e;
+    combine_delta<D><<<dim3(BH, D / kCB), 256, csmem, stream>>>(p.M_in, p.Gbuf, p.Bbuf, Mp, p.M_out,
+                                                                 p.T);
+    return cudaGetLastError();
+  }
+  if ((e = launch_products<D, false>(p, tk, tv, stream)) != cudaSuccess) return e;
+  combine_linear<D><<<dim3(BH, (D * D + 1023) / 1024), 256, 0, stream>>>(
+      p.M_in, p.Bbuf, p.dz, Mp, p.z_pref, p.M_out, p.z_out, p.T);
   return cudaGetLastError();
 }
 
@@ -414,6 +534,16 @@ cudaError_t launch(const Problem& p, cudaStream_t stream) {
 
 bool tc_scan_supported(int d_k, int d_v, bool bf16) {
   return bf16 && d_k == d_v && (d_k == 64 || d_k == 128);
+}
+
+int tc_scan_launches(bool delta) { return delta ? 4 : 2; }
+
+void tc_scan_workspace(int B, int H_kv, int T, int d, bool delta, size_t* g_bytes, size_t* b_bytes,
+                       size_t* dz_bytes) {
+  const size_t slices = (size_t)T * B * H_kv;
+  *g_bytes = delta ? slices * d * d * 4 : 0;
+  *b_bytes = slices * d * d * 4;
+  *dz_bytes = slices * d * 4;
 }
 
 cudaError_t launch_tc_state_scan(const Problem& p, cudaStream_t stream) {

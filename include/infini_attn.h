@@ -197,7 +197,7 @@ INFINI_API int infini_attn_kernel_times(double* ms, int* launches, int n_kinds, 
  * an embedding that owns all device memory and cannot lend a workspace).
  * Arguments and results are those of infini_attn_forward without the
  * workspace: the scratch comes from one static device array of
- * infini_attn_noalloc_scratch_limit() bytes (32 MiB), which every GPU that
+ * infini_attn_noalloc_scratch_limit() bytes (64 MiB), which every GPU that
  * loads this part of the library holds until the process exits.
  *   - Problems whose workspace (infini_attn_workspace_bytes) exceeds that
  *     limit return INFINI_ERR_SCRATCH_LIMIT before anything is enqueued
