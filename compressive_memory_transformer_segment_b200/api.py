@@ -66,6 +66,7 @@ _SIGNATURES = [
     ("infini_attn_kernel_times", ctypes.c_int, [ctypes.POINTER(ctypes.c_double),
                                                 ctypes.POINTER(ctypes.c_int), ctypes.c_int,
                                                 ctypes.c_int]),
+    ("infini_attn_selftest_approx", ctypes.c_int, [_P, _P, _P, _P, ctypes.c_int, _P]),
     ("infini_attn_forward_noalloc", ctypes.c_int, [_P, _P, _P, _P, _P, _P, ctypes.c_int,
                                                    ctypes.c_int, ctypes.POINTER(Dims), _P, _P, _P,
                                                    _P]),
@@ -276,3 +277,15 @@ def forward_noalloc(q, k, v, beta, M_in, z_in, seg_len, rule, out, M_out, z_out,
     _check(lib.infini_attn_forward_noalloc(*args, int(seg_len), _rule(rule), ctypes.byref(dims),
                                            *outs, _stream_handle(stream)))
     return out, M_out, z_out
+
+
+def selftest_approx(x, stream=None):
+    """(poly 2^x, hardware 2^x, bf16 bits of |x|) computed on the GPU for the
+    CUDA float32 tensor ``x`` by the kernel-side approximations."""
+    x = x.contiguous()
+    y_poly, y_mufu = torch.empty_like(x), torch.empty_like(x)
+    bits = torch.empty(x.shape, dtype=torch.int32, device=x.device)
+    _check(load_library().infini_attn_selftest_approx(
+        _dev(x, "x", torch.float32), _dev(y_poly, "y_poly"), _dev(y_mufu, "y_mufu"),
+        _dev(bits, "bits"), x.numel(), _stream_handle(stream)))
+    return y_poly, y_mufu, bits

@@ -267,11 +267,13 @@ tc_attention(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
       ok = __all_sync(0xffffffffu, mbar_wait(s_full, j & 1, abort, status));
       if (!ok) break;
       tc_fence_after();
-      // One pass per 64-column half: load, max, exponentiate against the
-      // running max m_run, pack P (bf16) over the scores already read.  The
-      // running max only moves when a half's max exceeds it by more than 2^8
-      // (always on the first half of the first tile): then O, the row sum
-      // and any P half already written for this tile are rescaled.
+      // One pass per 64-column half: load the scores, exponentiate against
+      // the running max m_run, pack P (bf16) over the scores already read.
+      // On the first tile the half's max is taken first (m_run is still
+      // -inf); afterwards the max is tracked alongside the exponentials and
+      // only checked at the end of the half: if it exceeds m_run by more than
+      // 2^8 (rare), the half is recomputed against the new max and O, the row
+      // sum and the P half already written are rescaled.
       const bool diag = j == qt;  // key c is visible to row r iff c <= r
       float lsum = 0.f;
 #pragma unroll
@@ -280,22 +282,49 @@ tc_attention(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
         tmem_ld32(tS + hf * 64, sv);
         tmem_ld32(tS + hf * 64 + 32, sv + 32);
         tmem_wait_ld();
-        float m8[8];
-#pragma unroll
-        for (int i = 0; i < 8; ++i) m8[i] = -INFINITY;
         if (diag) {
 #pragma unroll
           for (int i = 0; i < 64; ++i)
-            if (hf * 64 + i <= r) m8[i & 7] = fmaxf(m8[i & 7], __uint_as_float(sv[i]));
-        } else {
+            if (hf * 64 + i > r) sv[i] = __float_as_uint(-INFINITY);
+        }
+        float mxs;
+        if (j == 0 && hf == 0) {
+          float m8[8];
+#pragma unroll
+          for (int i = 0; i < 8; ++i) m8[i] = -INFINITY;
 #pragma unroll
           for (int i = 0; i < 64; ++i) m8[i & 7] = fmaxf(m8[i & 7], __uint_as_float(sv[i]));
+          mxs = sl2 * fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
+                            fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
+          m_run = mxs;
         }
-        const float mxs = sl2 * fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
-                                      fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
+        uint32_t packed[32];
+        float2 acc2[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+        float m8[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) m8[i] = -INFINITY;
+        {
+          const float2 sc = make_float2(sl2, sl2), nm2 = make_float2(-m_run, -m_run);
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            const float s0 = __uint_as_float(sv[2 * i]), s1 = __uint_as_float(sv[2 * i + 1]);
+            m8[(2 * i) & 7] = fmaxf(m8[(2 * i) & 7], s0);
+            m8[(2 * i + 1) & 7] = fmaxf(m8[(2 * i + 1) & 7], s1);
+            const float2 x = __ffma2_rn(make_float2(s0, s1), sc, nm2);
+            // One pair in four goes to the FMA pipe (exp2_poly), the rest to MUFU.
+            const float p0 = (i & 3) == 3 ? exp2_poly(x.x) : ex2_approx(x.x);
+            const float p1 = (i & 3) == 3 ? exp2_poly(x.y) : ex2_approx(x.y);
+            acc2[i & 1] = __fadd2_rn(acc2[i & 1], make_float2(p0, p1));
+            packed[i] = pack_bf16x2_pos(p0, p1);
+          }
+        }
+        mxs = sl2 * fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
+                          fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
         const bool need = mxs > m_run + 8.f;
         if (__any_sync(0xffffffffu, need)) {
-          const float f = need ? ex2_approx(m_run - mxs) : 1.f;  // 0 while m_run = -inf
+          // Rare: the max jumped.  Rescale what was accumulated against the
+          // old max and redo this half against the new one.
+          const float f = need ? ex2_approx(m_run - mxs) : 1.f;
           if (j > 0) {
             // O holds P.V through tile j-1 (complete: the scores of tile j
             // were produced after it).
@@ -310,7 +339,6 @@ tc_attention(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
             }
           }
           if (hf > 0) {
-            // The first half's P of this tile was written against the old max.
             uint32_t pw[32];
             tmem_ld32(tS, pw);
             tmem_wait_ld();
@@ -325,33 +353,17 @@ tc_attention(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
             lsum *= f;
             m_run = mxs;
           }
-        }
-        const float nm = -m_run;
-        float ls[4] = {0.f, 0.f, 0.f, 0.f};
-        uint32_t packed[32];
-        if (diag) {
+          const float nm = -m_run;
+          acc2[0] = acc2[1] = make_float2(0.f, 0.f);
 #pragma unroll
           for (int i = 0; i < 32; ++i) {
-            const int c0 = hf * 64 + 2 * i;
-            const float p0 = c0 <= r ? ex2_approx(fmaf(__uint_as_float(sv[2 * i]), sl2, nm)) : 0.f;
-            const float p1 =
-                c0 + 1 <= r ? ex2_approx(fmaf(__uint_as_float(sv[2 * i + 1]), sl2, nm)) : 0.f;
-            ls[i & 3] += p0 + p1;
-            packed[i] = pack_bf16x2_pos(p0, p1);
-          }
-        } else {
-#pragma unroll
-          for (int i = 0; i < 32; ++i) {
-            // One pair in four goes to the FMA pipe (exp2_poly), the rest to MUFU.
-            const float x0 = fmaf(__uint_as_float(sv[2 * i]), sl2, nm);
-            const float x1 = fmaf(__uint_as_float(sv[2 * i + 1]), sl2, nm);
-            const float p0 = (i & 3) == 3 ? exp2_poly(x0) : ex2_approx(x0);
-            const float p1 = (i & 3) == 3 ? exp2_poly(x1) : ex2_approx(x1);
-            ls[i & 3] += p0 + p1;
+            const float p0 = ex2_approx(fmaf(__uint_as_float(sv[2 * i]), sl2, nm));
+            const float p1 = ex2_approx(fmaf(__uint_as_float(sv[2 * i + 1]), sl2, nm));
+            acc2[i & 1] = __fadd2_rn(acc2[i & 1], make_float2(p0, p1));
             packed[i] = pack_bf16x2_pos(p0, p1);
           }
         }
-        lsum += (ls[0] + ls[1]) + (ls[2] + ls[3]);
+        lsum += (acc2[0].x + acc2[0].y) + (acc2[1].x + acc2[1].y);
         // P columns 32*hf .. 32*hf+31 lie inside score columns already read.
         tmem_st32(tS + hf * 32, packed);
       }

@@ -40,23 +40,41 @@ using namespace tc;
 // ---------------------------------------------------------------- dz and z prefix
 
 // dz[s][bh][c] = sum over the segment's rows t of sigma(k[bh][t][c]).
-// Grid (T, B*H_kv), block D threads (one per column).
+// Grid (T, B*H_kv), block 256 threads: thread (token lane tg, 8-column group
+// cg) reads 16-byte pieces of rows tg, tg + NT, ...; the NT partial sums of
+// each column are then added in shared memory.
 template <int D>
-__global__ void __launch_bounds__(128) zsum(const __nv_bfloat16* __restrict__ k,
+__global__ void __launch_bounds__(256) zsum(const __nv_bfloat16* __restrict__ k,
                                             float* __restrict__ dz, int L, int S) {
-  const int s = blockIdx.x, bh = blockIdx.y, c = threadIdx.x;
+  constexpr int kCG = D / 8;      // 16-byte column groups per row
+  constexpr int kNT = 256 / kCG;  // token lanes
+  __shared__ float part[kNT * D];
+  const int s = blockIdx.x, bh = blockIdx.y, tid = threadIdx.x;
+  const int cg = tid % kCG, tg = tid / kCG;
   const int r0 = s * S, r1 = min(r0 + S, L);
-  const __nv_bfloat16* kc = k + (size_t)bh * L * D + c;
-  float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
-  int t = r0;
-  for (; t + 4 <= r1; t += 4) {
-    a0 += elu1(__bfloat162float(kc[(size_t)t * D]));
-    a1 += elu1(__bfloat162float(kc[(size_t)(t + 1) * D]));
-    a2 += elu1(__bfloat162float(kc[(size_t)(t + 2) * D]));
-    a3 += elu1(__bfloat162float(kc[(size_t)(t + 3) * D]));
+  const uint4* base = reinterpret_cast<const uint4*>(k + (size_t)bh * L * D) + cg;
+  float acc[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) acc[i] = 0.f;
+#pragma unroll 4
+  for (int t = r0 + tg; t < r1; t += kNT) {
+    const uint4 v = __ldg(base + (size_t)t * kCG);
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      acc[2 * i] += elu1_fast(__uint_as_float(w[i] << 16));
+      acc[2 * i + 1] += elu1_fast(__uint_as_float(w[i] & 0xFFFF0000u));
+    }
   }
-  for (; t < r1; ++t) a0 += elu1(__bfloat162float(kc[(size_t)t * D]));
-  dz[((size_t)s * gridDim.y + bh) * D + c] = (a0 + a1) + (a2 + a3);
+#pragma unroll
+  for (int i = 0; i < 8; ++i) part[tg * D + cg * 8 + i] = acc[i];
+  __syncthreads();
+  if (tid < D) {
+    float sum = 0.f;
+#pragma unroll 8
+    for (int j = 0; j < kNT; ++j) sum += part[j * D + tid];
+    dz[((size_t)s * gridDim.y + bh) * D + tid] = sum;
+  }
 }
 
 // z_{s-1} for s = 1..T-1 into z_pref (slot 0 already holds z_in) and z_T.
@@ -258,14 +276,21 @@ tc_segment_products(const __grid_constant__ CUtensorMap tm_k, const __grid_const
         const uint32_t off = sw128_offset(t, 8 * c8, kTok);
         const uint4 kv = *reinterpret_cast<const uint4*>(sK + off);
         const uint32_t kw[4] = {kv.x, kv.y, kv.z, kv.w};
+        float zc[8];
+        if (DELTA) {
+          const float4 za = *reinterpret_cast<const float4*>(zs + 8 * c8);
+          const float4 zb = *reinterpret_cast<const float4*>(zs + 8 * c8 + 4);
+          zc[0] = za.x; zc[1] = za.y; zc[2] = za.z; zc[3] = za.w;
+          zc[4] = zb.x; zc[5] = zb.y; zc[6] = zb.z; zc[7] = zb.w;
+        }
         uint32_t hw[4], lw[4];
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
           const float a = valid ? elu1_fast(bf16lo_to_f32(kw[i])) : 0.f;
           const float b = valid ? elu1_fast(bf16hi_to_f32(kw[i])) : 0.f;
           if (DELTA) {
-            r = fmaf(a, zs[8 * c8 + 2 * i], r);
-            r = fmaf(b, zs[8 * c8 + 2 * i + 1], r);
+            r = fmaf(a, zc[2 * i], r);
+            r = fmaf(b, zc[2 * i + 1], r);
           }
           hw[i] = pack_bf16x2(a, b);
           lw[i] = pack_bf16x2(a - bf16lo_to_f32(hw[i]), b - bf16hi_to_f32(hw[i]));
@@ -352,69 +377,86 @@ tc_segment_products(const __grid_constant__ CUtensorMap tm_k, const __grid_const
 
 // ---------------------------------------------------------------- sequential combine
 
-constexpr int kCB = 16;  // columns of M per combine CTA (delta)
+constexpr int kCB = 8;  // columns of M per combine CTA (delta)
 
-// Delta rule: M_s = M_{s-1} - G_s M_{s-1} + B_s on columns [16 cb, 16 cb + 16).
-// Grid (B*H_kv, D/16), block 256 threads: thread -> (row k = tid % 128,
-// 8 columns); rows >= D idle for D = 64.  Plain (non-spinning) block barriers.
+__device__ __forceinline__ void cp_async16(void* smem_dst, const void* gmem_src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(smem_dst)), "l"(gmem_src)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+
+// Delta rule: M_s = M_{s-1} - G_s M_{s-1} + B_s on columns [8 cb, 8 cb + 8).
+// Grid (B*H_kv, D/8), block 256 threads: thread -> (row k = tid % 128,
+// 4 columns); rows >= D idle for D = 64.  G_s is symmetric up to the
+// rounding of its bf16 pair products (the dropped lo*lo term, ~2^-16
+// relative), so row k of G_s M is read from column k of G_s, which makes
+// the shared-memory reads conflict-free; G_{s+1} streams in (cp.async)
+// while G_s is used.  Plain block barriers only.
 template <int D>
 __global__ void __launch_bounds__(256) combine_delta(const float* __restrict__ M_in,
                                                      const float* __restrict__ Gbuf,
                                                      const float* __restrict__ Bbuf,
                                                      __nv_bfloat16* __restrict__ M_pref,
                                                      float* __restrict__ M_out, int T) {
-  extern __shared__ float csm[];
-  float* sG = csm;                  // G_s, rows padded to D + 1 floats
-  float* sM = csm + D * (D + 1);    // M_{s-1}[:, 16 columns]
+  extern __shared__ __align__(16) float csm[];
+  float* sG = csm;               // two G_s buffers [D][D]
+  float* sM = csm + 2 * D * D;   // M_{s-1}[:, 8 columns]
   const int bh = blockIdx.x, c0 = blockIdx.y * kCB, BH = gridDim.x;
-  const int tid = threadIdx.x, k = tid & 127, cg = (tid >> 7) * 8;
+  const int tid = threadIdx.x, k = tid & 127, cg = (tid >> 7) * 4;
   const bool active = k < D;
-  float m[8];
+  auto load_g = [&](int s, float* dst) {
+    const float4* src = reinterpret_cast<const float4*>(Gbuf + ((size_t)s * BH + bh) * D * D);
+    for (int e = tid; e < D * D / 4; e += 256) cp_async16(dst + 4 * e, src + e);
+    cp_async_commit();
+  };
+  float m[4];
 #pragma unroll
-  for (int i = 0; i < 8; ++i) m[i] = active ? M_in[((size_t)bh * D + k) * D + c0 + cg + i] : 0.f;
+  for (int i = 0; i < 4; ++i) m[i] = active ? M_in[((size_t)bh * D + k) * D + c0 + cg + i] : 0.f;
+  load_g(0, sG);
   for (int s = 0; s < T; ++s) {
     const size_t slice = (size_t)s * BH + bh;
+    float* G = sG + (s & 1) * D * D;
+    if (s + 1 < T) {
+      load_g(s + 1, sG + ((s + 1) & 1) * D * D);
+      cp_async_wait<1>();
+    } else {
+      cp_async_wait<0>();
+    }
     // Publish M_{s-1} (bf16) for segment s's retrieval.
     if (active) {
-      uint4 w;
+      uint2 w;
       w.x = pack_bf16x2(m[0], m[1]);
       w.y = pack_bf16x2(m[2], m[3]);
-      w.z = pack_bf16x2(m[4], m[5]);
-      w.w = pack_bf16x2(m[6], m[7]);
-      *reinterpret_cast<uint4*>(M_pref + (slice * D + k) * D + c0 + cg) = w;
-#pragma unroll
-      for (int i = 0; i < 8; ++i) sM[k * kCB + cg + i] = m[i];
+      *reinterpret_cast<uint2*>(M_pref + (slice * D + k) * D + c0 + cg) = w;
+      *reinterpret_cast<float4*>(sM + k * kCB + cg) = make_float4(m[0], m[1], m[2], m[3]);
     }
-    const float* G = Gbuf + slice * D * D;
-    for (int e = tid; e < D * D; e += 256) sG[(e / D) * (D + 1) + (e % D)] = G[e];
     __syncthreads();
     if (active) {
-      float acc[8];
-#pragma unroll
-      for (int i = 0; i < 8; ++i) acc[i] = 0.f;
-#pragma unroll 4
+      float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll 8
       for (int kk = 0; kk < D; ++kk) {
-        const float gv = sG[k * (D + 1) + kk];
-        const float4 ma = *reinterpret_cast<const float4*>(sM + kk * kCB + cg);
-        const float4 mb = *reinterpret_cast<const float4*>(sM + kk * kCB + cg + 4);
-        acc[0] = fmaf(gv, ma.x, acc[0]);
-        acc[1] = fmaf(gv, ma.y, acc[1]);
-        acc[2] = fmaf(gv, ma.z, acc[2]);
-        acc[3] = fmaf(gv, ma.w, acc[3]);
-        acc[4] = fmaf(gv, mb.x, acc[4]);
-        acc[5] = fmaf(gv, mb.y, acc[5]);
-        acc[6] = fmaf(gv, mb.z, acc[6]);
-        acc[7] = fmaf(gv, mb.w, acc[7]);
+        const float gv = G[kk * D + k];
+        const float4 mv = *reinterpret_cast<const float4*>(sM + kk * kCB + cg);
+        acc[0] = fmaf(gv, mv.x, acc[0]);
+        acc[1] = fmaf(gv, mv.y, acc[1]);
+        acc[2] = fmaf(gv, mv.z, acc[2]);
+        acc[3] = fmaf(gv, mv.w, acc[3]);
       }
-      const float* Bk = Bbuf + (slice * D + k) * D + c0 + cg;
-#pragma unroll
-      for (int i = 0; i < 8; ++i) m[i] = (m[i] - acc[i]) + Bk[i];
+      const float4 bk = *reinterpret_cast<const float4*>(Bbuf + (slice * D + k) * D + c0 + cg);
+      m[0] = (m[0] - acc[0]) + bk.x;
+      m[1] = (m[1] - acc[1]) + bk.y;
+      m[2] = (m[2] - acc[2]) + bk.z;
+      m[3] = (m[3] - acc[3]) + bk.w;
     }
     __syncthreads();
   }
   if (active)
 #pragma unroll
-    for (int i = 0; i < 8; ++i) M_out[((size_t)bh * D + k) * D + c0 + cg + i] = m[i];
+    for (int i = 0; i < 4; ++i) M_out[((size_t)bh * D + k) * D + c0 + cg + i] = m[i];
 }
 
 // Linear rule: M_s = M_{s-1} + B_s, z_s = z_{s-1} + dz_s, element-parallel.
@@ -512,12 +554,12 @@ cudaError_t launch(const Problem& p, cudaStream_t stream) {
   __nv_bfloat16* Mp = static_cast<__nv_bfloat16*>(p.M_pref);
   cudaError_t e;
   if (p.delta) {
-    zsum<D><<<dim3(p.T, BH), D, 0, stream>>>(static_cast<const __nv_bfloat16*>(p.k), p.dz, p.L, p.S);
+    zsum<D><<<dim3(p.T, BH), 256, 0, stream>>>(static_cast<const __nv_bfloat16*>(p.k), p.dz, p.L, p.S);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     zprefix<D><<<BH, D, 0, stream>>>(p.dz, p.z_pref, p.z_out, p.T);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     if ((e = launch_products<D, true>(p, tk, tv, stream)) != cudaSuccess) return e;
-    const int csmem = (D * (D + 1) + D * kCB) * (int)sizeof(float);
+    const int csmem = (2 * D * D + D * kCB) * (int)sizeof(float);
     e = cudaFuncSetAttribute(combine_delta<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, csmem);
     if (e != cudaSuccess) return e;
     combine_delta<D><<<dim3(BH, D / kCB), 256, csmem, stream>>>(p.M_in, p.Gbuf, p.Bbuf, Mp, p.M_out,

@@ -223,6 +223,19 @@ INFINI_API int infini_attn_forward_noalloc(const void* q, const void* k, const v
 /* Bytes of the static scratch array infini_attn_forward_noalloc uses. */
 INFINI_API size_t infini_attn_noalloc_scratch_limit(void);
 
+/* Self-check of device approximations (a testing aid; the method has no
+ * counterpart).  For i < n, with x, y_poly, y_mufu device float arrays and
+ * bf16_bits a device uint32 array:
+ *   y_poly[i]    = the FMA-pipe 2^x the attention kernel uses for part of its
+ *                  probabilities (range reduction + degree-3 polynomial; inputs
+ *                  below -125 are clamped to -125),
+ *   y_mufu[i]    = the hardware 2^x approximation (subnormal results -> 0),
+ *   bf16_bits[i] = bf16 bits of |x[i]| as the kernel packs probabilities
+ *                  (round half up; ties differ from round-to-nearest-even).
+ * Enqueued on `stream`.  Errors: INFINI_ERR_ARG, INFINI_ERR_CUDA. */
+INFINI_API int infini_attn_selftest_approx(const float* x, float* y_poly, float* y_mufu,
+                                           unsigned int* bf16_bits, int n, void* stream);
+
 #ifdef __cplusplus
 }
 #endif
