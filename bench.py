@@ -35,6 +35,32 @@ DEFAULT_CONFIG = "8b-delta"
 L2_BYTES = 126 * 1024 * 1024
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
+# DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) of one attention
+# launch, from an ncu capture summarised under profiles/, valid only while the
+# kernel sources hash to what they were at capture time.
+ATTENTION_TRAFFIC = {
+    "8b-delta": {"bytes": 2 * (406.998272e6 + 240.843776e6),
+                 "note": "ncu capture at batch 1, scaled x2 to the batch-2 launch",
+                 "profile": "profiles/tc_attention_8b-delta.md",
+                 "sha1": {"tc_attention.cu": "ab5a21d4ba3d1ccaf1dd1683fbbe86b1ab6bf640",
+                          "tc_common.cuh": "c82269991654d8b1f3bb1c0290a5eadbf9d329db"}},
+}
+
+
+def attention_traffic(name):
+    """Recorded per-launch traffic for this workload, or None if the kernel
+    changed since the counters were taken (or none were taken)."""
+    import hashlib
+    rec = ATTENTION_TRAFFIC.get(name)
+    if rec is None:
+        return None
+    csrc = os.path.join(ROOT, "compressive_memory_transformer_segment_b200", "csrc")
+    for fn, sha in rec["sha1"].items():
+        with open(os.path.join(csrc, fn), "rb") as f:
+            if hashlib.sha1(f.read()).hexdigest() != sha:
+                return None
+    return rec
+
 
 def load_peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
@@ -239,7 +265,7 @@ def run_gpu(args, w):
     import torch
     import torch.distributed as dist
 
-    from compressive_memory_transformer_segment_b200 import api
+    from compressive_memory_transformer_segment_b200 import api, shard
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -324,10 +350,7 @@ def run_gpu(args, w):
     ktimes = api.kernel_times(reset=True)
     api.sync_status(stream)
 
-    t = torch.tensor([elapsed_ms], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    max_ms = float(t.item())
+    max_ms = shard.max_over_ranks(elapsed_ms, device=dev)
     tokens = w.tokens * args.steps * world
     value = tokens / (max_ms / 1000.0)
 
@@ -365,10 +388,8 @@ def run_gpu(args, w):
         e2e_step()
     e1.record(stream)
     torch.cuda.synchronize(dev)
-    te = torch.tensor([e0.elapsed_time(e1)], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(te, op=dist.ReduceOp.MAX)
-    e2e_value = w.tokens * e2e_steps * world / (float(te.item()) / 1000.0)
+    e2e_ms = shard.max_over_ranks(e0.elapsed_time(e1), device=dev)
+    e2e_value = w.tokens * e2e_steps * world / (e2e_ms / 1000.0)
     h2d = sum(x.numel() * x.element_size() for x in (hq_p, hk_p, hv_p, hbeta, hM0, hz0))
     d2h = sum(x.numel() * x.element_size() for x in (hout, hM1, hz1))
 
@@ -405,7 +426,9 @@ def run_gpu(args, w):
         "gpu_launches": plan["launches"] * args.steps,
         "roofline": {"bound": "tensor", "kernel": "segment attention", "achieved": achieved,
                      "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
-                     "peak_source": f"{peak_src} bf16 burst", "traffic": None,
+                     "peak_source": f"{peak_src} bf16 burst",
+                     "traffic": (attention_traffic(w.name) or {}).get("bytes"),
+                     "traffic_note": (attention_traffic(w.name) or {}).get("note"),
                      "algorithmic_flops_per_launch": att_flops,
                      "avg_launch_ms": att_avg_s * 1000.0},
         "kernel_ms": {"attention": att_ms / max(att_n, 1), "state_scan": scan_ms / max(scan_n, 1)},
