@@ -1,6 +1,7 @@
 // Self-check of the device approximations the tensor-core attention kernel
-// uses in place of library functions: the FMA-pipe 2^x (exp2_poly), the
-// hardware 2^x (ex2.approx), and the integer bf16 packing of probabilities.
+// uses in place of library functions: the FMA-pipe 2^x (exp2_poly2, both of
+// its lanes), the hardware 2^x (ex2.approx), and the bf16 packing of
+// probabilities.
 #include <cuda_runtime.h>
 
 #include "infini_attn.h"
@@ -14,10 +15,11 @@ __global__ void selftest_kernel(const float* __restrict__ x, float* __restrict__
   const int i = blockIdx.x * blockDim.x + threadIdx.x;
   if (i >= n) return;
   const float v = x[i];
-  y_poly[i] = infini::tc::exp2_poly(v);
+  const float2 p2 = infini::tc::exp2_poly2(make_float2(v, v));
+  y_poly[i] = (i & 1) ? p2.y : p2.x;
   y_mufu[i] = infini::tc::ex2_approx(v);
   const float a = fabsf(v);
-  bf16_bits[i] = infini::tc::pack_bf16x2_pos(a, a) & 0xFFFFu;
+  bf16_bits[i] = infini::tc::pack_bf16x2(a, a) & 0xFFFFu;
 }
 
 }  // namespace

@@ -114,6 +114,13 @@ __device__ __forceinline__ void tma_store_wait_read() {
   asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
 }
 
+// Pulls a tile into L2 ahead of its load (no shared memory, no barrier).
+__device__ __forceinline__ void tma_prefetch_l2_3d(const CUtensorMap* map, int x, int y, int z) {
+  asm volatile("cp.async.bulk.prefetch.tensor.3d.L2.global.tile [%0, {%1, %2, %3}];" ::"l"(map),
+               "r"(x), "r"(y), "r"(z)
+               : "memory");
+}
+
 __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(map) : "memory");
 }
@@ -205,6 +212,17 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t* r) {
       : "r"(taddr));
 }
 
+// 16 consecutive 32-bit columns of this thread's TMEM lane (r[0..15]).
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t* r) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+      "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+        "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr));
+}
+
 __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t* r) {
   asm volatile(
       "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
@@ -270,35 +288,43 @@ __device__ __forceinline__ float ex2_approx(float x) {
   return y;
 }
 
-// 2^x on the FMA pipe, to share the work of 2^x with the MUFU unit.
-// Cody-Waite range reduction x = n + f with n = rint(x), |f| <= 1/2 (the
-// rounding is done by adding 1.5 * 2^23, which leaves n in the low mantissa
-// bits), a degree-3 polynomial for 2^f (least-squares fit on [-1/2, 1/2]
-// weighted to the relative error; max relative error 7.6e-5), and the scale
-// by 2^n as an integer add of n << 23 to the exponent bits.  Inputs are
-// clamped to >= -125 so the exponent never underflows; results below 2^-125
-// matter to nothing here.
-__device__ __forceinline__ float exp2_poly(float x) {
-  x = fmaxf(x, -125.f);
+// 2^x on the FMA pipe for two values at once (the paired fp32 instructions
+// take one issue slot for two lanes' worth of work), to share the work of 2^x
+// with the MUFU unit.  Cody-Waite range reduction x = n + f with n = rint(x),
+// |f| <= 1/2 (the rounding is done by adding 1.5 * 2^23, which leaves n in the
+// low mantissa bits), a degree-3 polynomial for 2^f (least-squares fit on
+// [-1/2, 1/2] weighted to the relative error; max relative error 7.6e-5), and
+// the scale by 2^n as an integer add of n << 23 to the exponent bits.  Inputs
+// are clamped to >= -125 so the exponent never underflows; results below
+// 2^-125 matter to nothing here.
+__device__ __forceinline__ float2 exp2_poly2(float2 x) {
+  x.x = fmaxf(x.x, -125.f);
+  x.y = fmaxf(x.y, -125.f);
   const float kRound = 12582912.f;
-  const float t = x + kRound;
-  const float f = x - (t - kRound);
-  const float p = fmaf(fmaf(fmaf(0.055186376f, f, 0.24261236f), f, 0.69325829f), f, 0.99992794f);
-  return __uint_as_float(__float_as_uint(p) + (__float_as_uint(t) << 23));
+  const float2 t = __fadd2_rn(x, make_float2(kRound, kRound));
+  const float2 n = __fadd2_rn(t, make_float2(-kRound, -kRound));
+  const float2 f = __ffma2_rn(n, make_float2(-1.f, -1.f), x);
+  float2 p = __ffma2_rn(make_float2(0.055186376f, 0.055186376f), f,
+                        make_float2(0.24261236f, 0.24261236f));
+  p = __ffma2_rn(p, f, make_float2(0.69325829f, 0.69325829f));
+  p = __ffma2_rn(p, f, make_float2(0.99992794f, 0.99992794f));
+  return make_float2(__uint_as_float(__float_as_uint(p.x) + (__float_as_uint(t.x) << 23)),
+                     __uint_as_float(__float_as_uint(p.y) + (__float_as_uint(t.y) << 23)));
 }
 
-// Two non-negative finite floats to a bf16 pair (round half up), using
-// integer ops only (keeps the conversion off the XU pipe that computes 2^x).
-__device__ __forceinline__ uint32_t pack_bf16x2_pos(float lo, float hi) {
-  const uint32_t a = __float_as_uint(lo) + 0x8000u;
-  const uint32_t b = __float_as_uint(hi) + 0x8000u;
-  return __byte_perm(a, b, 0x7632);
+// max(a, b, c) in one instruction (three-input fp32 max, sm_100).
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
 }
 
 // bf16 pair -> two floats (exact).
 __device__ __forceinline__ float bf16lo_to_f32(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf16hi_to_f32(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
 
+// Two floats to a bf16 pair, round to nearest even (one cvt.rn.bf16x2.f32,
+// which runs on the ALU pipe, not on the MUFU unit that computes 2^x).
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&v);

@@ -156,10 +156,10 @@ tc_segment_products(const __grid_constant__ CUtensorMap tm_k, const __grid_const
 
   if (threadIdx.x == 0) {
     mbar_init(k_full, 1);
-    mbar_init(k_empty, 128);
+    mbar_init(k_empty, 4);   // one arrival per math warp
     mbar_init(v_full, 1);
     mbar_init(v_empty, 1);
-    mbar_init(op_ready, 128);
+    mbar_init(op_ready, 4);
     mbar_init(op_free, 1);
     mbar_init(done, 1);
     *abort = 0;
@@ -197,28 +197,36 @@ tc_segment_products(const __grid_constant__ CUtensorMap tm_k, const __grid_const
   const uint32_t tmem = *tmem_slot;
 
   if (warp == 0) {
-    if (lane == 0) {
+    {
       // ------------------------------------------------ TMA producer
+      // The whole warp runs the loop and every wait (kept warp-uniform);
+      // lane 0 issues the copies.
       int issued_k = 0, issued_v = 0;
       for (int blk = 0; blk < nblk; ++blk) {
         const uint32_t par = (blk & 1) ^ 1;
-        if (!mbar_wait(k_empty, par, abort, status)) break;
-        mbar_arrive_expect_tx(k_full, kTok * D * 2);
-        for (int p = 0; p < D / 64; ++p)
-          tma_load_3d(sK + p * kTok * 128, &tm_k, k_full, p * 64, seg0 + blk * kTok, bh);
+        if (!__all_sync(0xffffffffu, mbar_wait(k_empty, par, abort, status))) break;
+        if (lane == 0) {
+          mbar_arrive_expect_tx(k_full, kTok * D * 2);
+          for (int p = 0; p < D / 64; ++p)
+            tma_load_3d(sK + p * kTok * 128, &tm_k, k_full, p * 64, seg0 + blk * kTok, bh);
+        }
         issued_k = blk + 1;
-        if (!mbar_wait(v_empty, par, abort, status)) break;
-        mbar_arrive_expect_tx(v_full, kTok * D * 2);
-        for (int p = 0; p < D / 64; ++p)
-          tma_load_3d(sV + p * kTok * 128, &tm_v, v_full, p * 64, seg0 + blk * kTok, bh);
+        if (!__all_sync(0xffffffffu, mbar_wait(v_empty, par, abort, status))) break;
+        if (lane == 0) {
+          mbar_arrive_expect_tx(v_full, kTok * D * 2);
+          for (int p = 0; p < D / 64; ++p)
+            tma_load_3d(sV + p * kTok * 128, &tm_v, v_full, p * 64, seg0 + blk * kTok, bh);
+        }
         issued_v = blk + 1;
       }
       if (issued_k > 0) mbar_wait(k_full, (issued_k - 1) & 1, abort, status, false);
       if (issued_v > 0) mbar_wait(v_full, (issued_v - 1) & 1, abort, status, false);
+      __syncwarp();
     }
   } else if (warp == 1) {
-    if (lane == 0) {
+    {
       // ------------------------------------------------ MMA issuer
+      // The whole warp runs the loop and every wait; lane 0 issues.
       // All operands are MN-major [tokens][128] tiles (panels of 64 columns,
       // 16 KiB apart); one 16-token K step = 2048 bytes.
       const uint64_t skhi = sw128_desc(smem_u32(sSkHi), kTok * 128, 1024);
@@ -231,9 +239,10 @@ tc_segment_products(const __grid_constant__ CUtensorMap tm_k, const __grid_const
       const uint32_t tG = tmem, tB = DELTA ? tmem + 128 : tmem;
       bool ok = true;
       for (int blk = 0; ok && blk < nblk; ++blk) {
-        if (!(ok = mbar_wait(op_ready, blk & 1, abort, status))) break;
-        if (!(ok = mbar_wait(v_full, blk & 1, abort, status))) break;
+        if (!(ok = __all_sync(0xffffffffu, mbar_wait(op_ready, blk & 1, abort, status)))) break;
+        if (!(ok = __all_sync(0xffffffffu, mbar_wait(v_full, blk & 1, abort, status)))) break;
         tc_fence_after();
+        if (lane != 0) continue;
 #pragma unroll
         for (int kk = 0; kk < kTok / 16; ++kk) {
           const uint32_t st = mnmajor_step(kk);
@@ -252,8 +261,10 @@ tc_segment_products(const __grid_constant__ CUtensorMap tm_k, const __grid_const
         tc_commit(op_free);
         tc_commit(v_empty);
       }
-      tc_commit(done);
+      if (lane == 0) tc_commit(done);
+      __syncwarp();
       mbar_wait(done, 0, abort, status, false);
+      __syncwarp();
     }
   } else {
     // -------------------------------------------------- math threads
@@ -298,7 +309,8 @@ tc_segment_products(const __grid_constant__ CUtensorMap tm_k, const __grid_const
         *reinterpret_cast<uint4*>(sSkHi + off) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
         *reinterpret_cast<uint4*>(sSkLo + off) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
       }
-      mbar_arrive(k_empty);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(k_empty);
       if (DELTA) {
         // Y = sigma(K) / r (0 where r = 0), from the pair just written.
         const float w = r != 0.f ? 1.f / r : 0.f;
@@ -321,7 +333,8 @@ tc_segment_products(const __grid_constant__ CUtensorMap tm_k, const __grid_const
         }
       }
       fence_proxy_async();
-      mbar_arrive(op_ready);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(op_ready);
     }
     // The segment's products, row t (t < D), to the workspace in fp32.
     if (ok) ok = __all_sync(0xffffffffu, mbar_wait(done, 0, abort, status));

@@ -1,7 +1,7 @@
 """The attention kernel's own device approximations, checked against float64
 references: the FMA-pipe 2^x (range reduction + a degree-3 polynomial fitted
-on [-1/2, 1/2], stated relative error 7.6e-5), the hardware 2^x, and the
-integer bf16 packing of non-negative probabilities."""
+on [-1/2, 1/2], stated relative error 7.6e-5; both lanes of the paired
+version), the hardware 2^x, and the bf16 packing of probabilities."""
 
 import numpy as np
 import pytest
@@ -28,16 +28,17 @@ def test_exp2_approximations(cuda_lib):
 
 
 def test_probability_packing_is_bf16_rounding(cuda_lib):
+    """The packing of P is round-to-nearest-even bf16 (what torch does)."""
     api = cuda_lib
     rng = np.random.default_rng(0)
     x = np.concatenate([rng.uniform(0, 300, 200000), 2.0 ** rng.uniform(-40, 8, 200000), [0.0, 1.0, 256.0]])
     xt = torch.from_numpy(x.astype(np.float32))
     _, _, bits = api.selftest_approx(xt.cuda())
     got = bits.cpu().numpy().astype(np.uint32)
-    u = xt.numpy().view(np.uint32)
-    half_up = ((u + 0x8000) >> 16).astype(np.uint32)
-    np.testing.assert_array_equal(got, half_up)
-    # Against round-to-nearest-even it differs only on exact ties.
     rne = xt.to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16).astype(np.uint32)
-    diff = got != rne
-    assert np.all((u[diff] & 0xFFFF) == 0x8000)
+    np.testing.assert_array_equal(got, rne)
+    # Exact ties go to the even neighbour: 1 + 2^-8 -> 1, 1 + 3 * 2^-8 -> 1 + 2^-6.
+    ties = torch.tensor([1 + 2.0 ** -8, 1 + 3 * 2.0 ** -8], dtype=torch.float32)
+    _, _, tb = api.selftest_approx(ties.cuda())
+    got_t = tb.cpu().numpy().astype(np.uint32) << 16
+    np.testing.assert_array_equal(got_t.view(np.float32), np.array([1.0, 1 + 2.0 ** -6], np.float32))

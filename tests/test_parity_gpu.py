@@ -257,6 +257,12 @@ TC_CASES = [
                                     H_q=8, H_kv=2, rule="delta")),
     ("tc_d64_S512_ragged", dict(dtype="bf16", d_k=64, d_v=64, L=1500, seg_len=512, H_q=3, H_kv=3)),
     ("tc_d128_L_lt_S", dict(dtype="bf16", d_k=128, d_v=128, L=200, seg_len=256)),
+    # Three query heads per KV head and an odd number of query tiles per group:
+    # work items pair tiles of different positions, one item has a single tile.
+    ("tc_d64_gqa3_S384_ragged", dict(dtype="bf16", d_k=64, d_v=64, L=900, seg_len=384, H_q=6,
+                                     H_kv=2, rule="delta")),
+    ("tc_d128_gqa2_S256_ragged", dict(dtype="bf16", d_k=128, d_v=128, L=700, seg_len=256, B=2,
+                                      H_q=4, H_kv=2)),
 ]
 
 
