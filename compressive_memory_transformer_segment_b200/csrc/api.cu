@@ -9,6 +9,7 @@
 #include <vector>
 
 #include "infini_attn.h"
+#include "common.cuh"
 #include "kernels.h"
 
 namespace infini {
@@ -358,7 +359,7 @@ int infini_attn_sync_status(void* stream) {
   if (word != 0) {
     const unsigned int zero = 0;
     if (cudaMemcpyToSymbol(g_status, &zero, sizeof(zero)) != cudaSuccess) return INFINI_ERR_CUDA;
-    return INFINI_ERR_TIMEOUT;
+    return (word & infini::kStatusLayout) ? INFINI_ERR_UNSUPPORTED : INFINI_ERR_TIMEOUT;
   }
   return INFINI_OK;
 }

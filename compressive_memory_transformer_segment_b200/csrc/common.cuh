@@ -10,6 +10,7 @@ namespace infini {
 // Bits of the device status word (reported by infini_attn_sync_status).
 enum : unsigned int {
   kStatusTimeout = 1u,  // a bounded wait ran out
+  kStatusLayout = 2u,   // a kernel found its shared memory not laid out as it requires
 };
 
 template <typename T> __device__ __forceinline__ float to_f32(T x);

@@ -53,41 +53,40 @@ using namespace tc;
 constexpr int kBM = 128;  // query rows per tile
 constexpr int kBN = 128;  // keys per K/V tile
 constexpr int kThreads = 384;
-constexpr int kRegsRoles = 104;   // per thread, warpgroup 0 (producer, MMA)
-constexpr int kRegsSoftmax = 200; // per thread, warpgroups 1 and 2
+constexpr int kRegsRoles = 120;   // per thread, warpgroup 0 (producer, MMA)
+constexpr int kRegsSoftmax = 192; // per thread, warpgroups 1 and 2
 constexpr uint32_t kTmemCols = 512;
 constexpr int kSmemLimit = 232448;  // opt-in dynamic shared memory per block
 
 template <int D>
 struct Smem {
   static constexpr int kTile = kBM * D * 2;  // bytes of a 128 x D bf16 tile (>= D x D for M)
-  static constexpr int kRing = (kSmemLimit - 8192 - 2 * kTile) / kTile;
-  static constexpr int kQ = 0;  // Q of slot A, Q of slot B
-  static constexpr int kRingOff = 2 * kTile;
+  // Q tiles: [slot][item parity] (the next item's Q loads during this one).
+  static constexpr int kRing = (kSmemLimit - 3072 - 4 * kTile) / kTile;
+  static constexpr int kQ = 0;
+  static constexpr int kRingOff = 4 * kTile;
   static constexpr int kBar = kRingOff + kRing * kTile;
-  // ring full[kRing], ring empty[kRing], then two (one per slot) of each of
-  // q_full q_empty s_full p_ready sq_ready r_full tmem_free, then z_ready,
-  // xbar[4] (one per row quarter) and drain.
+  // ring full[kRing], ring empty[kRing], q_full[4] q_empty[4] (per Q
+  // tile), then two (one per slot) of each of s_full p_ready sq_ready r_full
+  // tmem_free z_ready, then drain.
   static constexpr int kFull = 0;
   static constexpr int kEmpty = kRing;
   static constexpr int kQFull = 2 * kRing;
-  static constexpr int kQEmpty = kQFull + 2;
-  static constexpr int kSFull = kQEmpty + 2;
+  static constexpr int kQEmpty = kQFull + 4;
+  static constexpr int kSFull = kQEmpty + 4;
   static constexpr int kPReady = kSFull + 2;
   static constexpr int kSqReady = kPReady + 2;
   static constexpr int kRFull = kSqReady + 2;
   static constexpr int kTFree = kRFull + 2;
   static constexpr int kZReady = kTFree + 2;
-  static constexpr int kXBar = kZReady + 1;
-  static constexpr int kDrain = kXBar + 4;
+  static constexpr int kDrain = kZReady + 2;
   static constexpr int kNumBars = kDrain + 1;
-  // z_{s-1} of the item's group, fp32 [D], read as float4: 128-byte aligned.
+  // z_{s-1} per slot, fp32 [2][D], read as float4: 128-byte aligned.
   static constexpr int kZ = (kBar + kNumBars * 8 + 127) / 128 * 128;
-  // Row exchange between the two column halves: fp32 [2 parity][2 half][128 row][2].
-  static constexpr int kX = kZ + D * 4;
-  static constexpr int kTmemSlot = kX + 2 * 2 * 128 * 2 * 4;
+  static constexpr int kTmemSlot = kZ + 2 * D * 4;
   static constexpr int kAbort = kTmemSlot + 4;
-  static constexpr int kAlloc = kAbort + 4 + 1024;  // + slack to align the base to 1024
+  // The dynamic shared memory base is 1024-byte aligned (checked at entry).
+  static constexpr int kAlloc = kAbort + 4;
   static_assert(kRing >= 3, "ring too small");
   static_assert(kZ % 16 == 0 && kBar % 8 == 0 && kTmemSlot % 4 == 0, "alignment");
   static_assert(kAlloc <= kSmemLimit, "shared memory");
@@ -142,22 +141,25 @@ __device__ __forceinline__ void warp_arrive(uint64_t* bar) {
   if ((threadIdx.x & 31) == 0) mbar_arrive(bar);
 }
 
-// Max of 128 floats (bit patterns in a[64], b[64]) as a shallow tree of
-// three-input maxima: 43 + 15 + 5 + 2 + 1 operations, depth 5.
+// Max of 128 floats (bit patterns in a[64], b[64]) with three-input maxima:
+// 16 independent accumulators over 8 values each (depth 4), then a short
+// tree; few values live at once.
 __device__ __forceinline__ float row_max128(const uint32_t* a, const uint32_t* b) {
   auto v = [&](int k) { return __uint_as_float(k < 64 ? a[k] : b[k - 64]); };
-  float l1[43];
+  float acc[16];
 #pragma unroll
-  for (int i = 0; i < 42; ++i) l1[i] = fmax3(v(3 * i), v(3 * i + 1), v(3 * i + 2));
-  l1[42] = fmaxf(v(126), v(127));
-  float l2[15];
+  for (int k = 0; k < 16; ++k) acc[k] = fmax3(v(k), v(16 + k), v(32 + k));
 #pragma unroll
-  for (int i = 0; i < 14; ++i) l2[i] = fmax3(l1[3 * i], l1[3 * i + 1], l1[3 * i + 2]);
-  l2[14] = l1[42];
-  float l3[5];
+  for (int k = 0; k < 16; ++k) acc[k] = fmax3(acc[k], v(48 + k), v(64 + k));
 #pragma unroll
-  for (int i = 0; i < 5; ++i) l3[i] = fmax3(l2[3 * i], l2[3 * i + 1], l2[3 * i + 2]);
-  return fmaxf(fmax3(l3[0], l3[1], l3[2]), fmaxf(l3[3], l3[4]));
+  for (int k = 0; k < 16; ++k) acc[k] = fmax3(acc[k], v(80 + k), v(96 + k));
+#pragma unroll
+  for (int k = 0; k < 16; ++k) acc[k] = fmaxf(acc[k], v(112 + k));
+  float t[6];
+#pragma unroll
+  for (int i = 0; i < 5; ++i) t[i] = fmax3(acc[3 * i], acc[3 * i + 1], acc[3 * i + 2]);
+  t[5] = acc[15];
+  return fmaxf(fmax3(t[0], t[1], t[2]), fmax3(t[3], t[4], t[5]));
 }
 
 // P = 2^(s * sl2 - m) for 64 scores (fp32 bit patterns), as 32 bf16 pairs;
@@ -194,8 +196,14 @@ tc_attention(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
   constexpr int kRing = SM::kRing;
 
   extern __shared__ __align__(1024) unsigned char smem_raw[];
-  unsigned char* smem = reinterpret_cast<unsigned char*>(
-      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  // The swizzled tiles need 1024-byte aligned addresses; the layout fills
+  // the opt-in maximum, leaving no room to realign.  (Every thread takes
+  // the same branch, before any barrier.)
+  if ((smem_u32(smem_raw) & 1023u) != 0) {
+    if (threadIdx.x == 0) atomicOr(status, kStatusLayout);
+    return;
+  }
+  unsigned char* smem = smem_raw;
   unsigned char* ring = smem + SM::kRingOff;
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + SM::kBar);
   uint64_t* full = bars + SM::kFull;
@@ -208,7 +216,6 @@ tc_attention(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
   uint64_t* r_full = bars + SM::kRFull;
   uint64_t* tmem_free = bars + SM::kTFree;
   uint64_t* z_ready = bars + SM::kZReady;
-  uint64_t* xbars = bars + SM::kXBar;
   uint64_t* drain = bars + SM::kDrain;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + SM::kTmemSlot);
   volatile int* abort = reinterpret_cast<volatile int*>(smem + SM::kAbort);
@@ -220,17 +227,18 @@ tc_attention(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
       mbar_init(full + i, 1);
       mbar_init(empty + i, 1);
     }
-    for (int x = 0; x < 2; ++x) {
-      mbar_init(q_full + x, 1);
-      mbar_init(q_empty + x, 1);
-      mbar_init(s_full + x, 1);
-      mbar_init(p_ready + x, 8);  // one arrival per softmax warp
-      mbar_init(sq_ready + x, 8);
-      mbar_init(r_full + x, 1);
-      mbar_init(tmem_free + x, 8);
+    for (int b = 0; b < 4; ++b) {
+      mbar_init(q_full + b, 1);
+      mbar_init(q_empty + b, 1);
     }
-    mbar_init(z_ready, 8);
-    for (int q = 0; q < 4; ++q) mbar_init(xbars + q, 2);
+    for (int x = 0; x < 2; ++x) {
+      mbar_init(s_full + x, 1);
+      mbar_init(p_ready + x, 4);  // one arrival per softmax warp of the slot
+      mbar_init(sq_ready + x, 4);
+      mbar_init(r_full + x, 1);
+      mbar_init(tmem_free + x, 4);
+      mbar_init(z_ready + x, 4);
+    }
     mbar_init(drain, 1);
     *abort = 0;
     fence_mbar_init();
@@ -251,7 +259,7 @@ tc_attention(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
   const uint32_t tmem = *tmem_slot;
   const int BHkv = sh.B * sh.H_kv;
 
-  // 384 threads x 168 registers at launch = 4 x 32 x 104 + 8 x 32 x 200; each
+  // 384 threads x 168 registers at launch = 4 x 32 x 120 + 8 x 32 x 192; each
   // role's code sits under its own setmaxnreg.
   if (warp < 4) {
     asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsRoles));
@@ -261,7 +269,7 @@ tc_attention(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
       // The whole warp runs the loop and every wait (kept warp-uniform);
       // lane 0 issues the copies.
       uint32_t rc = 0;                // ring loads issued
-      uint32_t qi[2] = {0u, 0u};      // Q loads issued per slot
+      uint32_t qi[2] = {0u, 0u};      // Q loads issued per slot (tile = 2 * slot + count % 2)
       bool ok = true;
       auto ring_load = [&](const CUtensorMap* map, int rows_box, int row0, int plane) -> bool {
         const uint32_t slot = rc % kRing, ph = (rc / kRing) & 1u;
@@ -275,37 +283,40 @@ tc_attention(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
         ++rc;
         return true;
       };
+      // Query tiles of an item into the slots' next Q tiles (a tile is free
+      // once the retrieval two items back has read it).
+      auto q_load = [&](const Item& nx) -> bool {
+        for (int x = 0; x < 2; ++x) {
+          if (nx.n[x] == 0) continue;
+          const uint32_t b = 2 * x + (qi[x] & 1u);
+          if (!__all_sync(0xffffffffu, mbar_wait(q_empty + b, ((qi[x] >> 1) & 1u) ^ 1u, abort, status)))
+            return false;
+          if (lane == 0) {
+            unsigned char* dst = smem + SM::kQ + b * kTileBytes;
+            mbar_arrive_expect_tx(q_full + b, kTileBytes);
+            for (int p = 0; p < kPanels; ++p)
+              tma_load_3d(dst + p * kBM * 128, &tm_q, q_full + b, p * 64, nx.seg0 + nx.qt[x] * kBM,
+                          nx.b * sh.H_q + nx.h[x]);
+          }
+          ++qi[x];
+        }
+        return true;
+      };
+      if (blockIdx.x < sh.items) ok = q_load(decode_item(blockIdx.x, sh));
       for (int idx = blockIdx.x; ok && idx < sh.items; idx += gridDim.x) {
         const Item it = decode_item(idx, sh);
-        if (it.n_max == 0) continue;
+        if (it.n_max == 0) {
+          // An empty item (past the end of a short last segment) still hands
+          // on the next item's query tiles.
+          if (idx + (int)gridDim.x < sh.items) ok = q_load(decode_item(idx + gridDim.x, sh));
+          continue;
+        }
         const int bh_kv = it.b * sh.H_kv + it.h_kv;
         for (int j = 0; ok && j < it.n_max; ++j) {
           ok = ring_load(&tm_k, kBN, it.seg0 + j * kBN, bh_kv) &&
                ring_load(&tm_v, kBN, it.seg0 + j * kBN, bh_kv);
-          if (ok && j == 0) {
-            for (int x = 0; ok && x < 2; ++x) {
-              if (it.n[x] == 0) continue;
-              if (!(ok = __all_sync(0xffffffffu, mbar_wait(q_empty + x, (qi[x] & 1u) ^ 1u, abort, status))))
-                break;
-              if (lane == 0) {
-                unsigned char* dst = smem + SM::kQ + x * kTileBytes;
-                mbar_arrive_expect_tx(q_full + x, kTileBytes);
-                for (int p = 0; p < kPanels; ++p)
-                  tma_load_3d(dst + p * kBM * 128, &tm_q, q_full + x, p * 64, it.seg0 + it.qt[x] * kBM,
-                              it.b * sh.H_q + it.h[x]);
-              }
-              ++qi[x];
-            }
-          }
-        }
-        // The next item's query tiles into L2 (the producer runs a few tiles
-        // ahead of the tensor core, so they arrive before they are loaded).
-        if (ok && lane == 0 && idx + (int)gridDim.x < sh.items) {
-          const Item nx = decode_item(idx + gridDim.x, sh);
-          for (int x = 0; x < 2; ++x)
-            if (nx.n[x] > 0)
-              for (int p = 0; p < kPanels; ++p)
-                tma_prefetch_l2_3d(&tm_q, p * 64, nx.seg0 + nx.qt[x] * kBM, nx.b * sh.H_q + nx.h[x]);
+          // The next item's query tiles, early in this item.
+          if (ok && j == 0 && idx + (int)gridDim.x < sh.items) ok = q_load(decode_item(idx + gridDim.x, sh));
         }
         // M_{s-1} (D x D, panels of D rows).
         if (ok) ok = ring_load(&tm_m, D, 0, it.s * BHkv + bh_kv);
@@ -317,7 +328,10 @@ tc_attention(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
         mbar_wait(full + u % kRing, (u / kRing) & 1u, abort, status, false);
       }
       for (int x = 0; x < 2; ++x)
-        if (qi[x] > 0) mbar_wait(q_full + x, (qi[x] - 1) & 1u, abort, status, false);
+        for (int p = 0; p < 2; ++p) {
+          const uint32_t uses = (qi[x] + 1u - p) / 2u;  // loads into tile 2x + p
+          if (uses > 0) mbar_wait(q_full + 2 * x + p, (uses - 1) & 1u, abort, status, false);
+        }
       __syncwarp();
     }
   } else if (warp == 1) {
@@ -327,8 +341,7 @@ tc_attention(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
       // lane 0 issues the MMAs and commits.
       constexpr uint32_t idesc_qk = idesc_bf16_f32(kBM, kBN, false, false);
       constexpr uint32_t idesc_pv = idesc_bf16_f32(kBM, D, false, true);
-      const uint64_t dq[2] = {sw128_desc(smem_u32(smem + SM::kQ), 16, 1024),
-                              sw128_desc(smem_u32(smem + SM::kQ + kTileBytes), 16, 1024)};
+      const uint64_t dq0 = sw128_desc(smem_u32(smem + SM::kQ), 16, 1024);
       const uint64_t dk0 = sw128_desc(smem_u32(ring), 16, 1024);
       const uint64_t dv0 = sw128_desc(smem_u32(ring), kBN * 128, 1024);
       const uint64_t dm0 = sw128_desc(smem_u32(ring), D * 128, 1024);
@@ -377,15 +390,18 @@ tc_attention(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
               if (j == 0) {
                 // The previous item's epilogue has read this slot's TMEM.
                 if (!(ok = __all_sync(0xffffffffu, mbar_wait(tmem_free + x, (ic[x] & 1u) ^ 1u, abort, status)))) break;
-                if (!(ok = __all_sync(0xffffffffu, mbar_wait(q_full + x, ic[x] & 1u, abort, status)))) break;
+                if (!(ok = __all_sync(0xffffffffu, mbar_wait(q_full + 2 * x + (ic[x] & 1u), (ic[x] >> 1) & 1u,
+                                                             abort, status))))
+                  break;
               }
+              const uint64_t dq = dq0 + (((2 * x + (ic[x] & 1u)) * kTileBytes) >> 4);
               if (!k_ready && !(ok = __all_sync(0xffffffffu, mbar_wait(full + ks, kph, abort, status)))) break;
               k_ready = true;
               tc_fence_after();
               if (lane == 0) {
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk)
-                  mma_ss(tS, dq[x] + kmajor_step(kk, kBM), dk + kmajor_step(kk, kBN), idesc_qk,
+                  mma_ss(tS, dq + kmajor_step(kk, kBM), dk + kmajor_step(kk, kBN), idesc_qk,
                          kk > 0 ? 1u : 0u);
                 tc_commit(s_full + x);
               }
@@ -412,11 +428,13 @@ tc_attention(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
           tc_fence_after();
           if (lane == 0) {
             const uint32_t tS = tmem + x * 256;
+            const uint32_t qb = 2 * x + (ic[x] & 1u);
+            const uint64_t dq = dq0 + ((qb * kTileBytes) >> 4);
 #pragma unroll
             for (int kk = 0; kk < D / 16; ++kk)
-              mma_ss(tS, dq[x] + kmajor_step(kk, kBM), dm + mnmajor_step(kk), idesc_pv, kk > 0 ? 1u : 0u);
+              mma_ss(tS, dq + kmajor_step(kk, kBM), dm + mnmajor_step(kk), idesc_pv, kk > 0 ? 1u : 0u);
             tc_commit(r_full + x);
-            tc_commit(q_empty + x);
+            tc_commit(q_empty + qb);
           }
         }
         if (!ok) break;
@@ -434,206 +452,163 @@ tc_attention(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
   } else {
     asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegsSoftmax));
     // -------------------------------------------------- softmax / epilogue
-    // Warps 4..11 work on every tile of both slots together: warp w owns the
-    // rows 32*(w%4) .. +31 (its TMEM lanes) and the column half hc = (w-4)/4
-    // (keys 64*hc .. +63 of a score tile, features D/2*hc .. of O and R).
-    // The two threads of a row swap their half's tile max (and, at the end
-    // of an item, row sum and retrieval denominator) through shared memory,
-    // paired by an mbarrier per row quarter.  Waits are made warp-uniform
-    // (__all_sync) so that the .sync.aligned TMEM instructions are always
-    // executed by full warps.
-    const int hc = (warp - 4) >> 2;
-    const int qr = warp & 3;
-    const int r = 32 * qr + lane;
-    const uint32_t lane_off = (uint32_t)(32 * qr) << 16;
+    // Warpgroup 1 serves slot A, warpgroup 2 slot B: one thread per query row
+    // (its TMEM lane).  While one slot's softmax runs, the tensor core works
+    // on the other slot.  Waits are made warp-uniform (__all_sync) so that
+    // the .sync.aligned TMEM instructions are always executed by full warps.
+    const int x = (warp - 4) >> 2;
+    const int r = 32 * (warp & 3) + lane;
+    const uint32_t lane_off = (uint32_t)(32 * (warp & 3)) << 16;
+    const uint32_t tS = tmem + x * 256 + lane_off;
+    const uint32_t tO = tS + 128;
+    float* zs = reinterpret_cast<float*>(smem + SM::kZ) + x * D;
     const float sl2 = rsqrtf((float)D) * 1.4426950408889634f;
-    float* zs = reinterpret_cast<float*>(smem + SM::kZ);
-    float* xb = reinterpret_cast<float*>(smem + SM::kX);
-    uint64_t* xbar = xbars + qr;
-    // Per-slot state lives in scalars selected by the slot index (the slot
-    // loops are not unrolled: one copy of the tile code keeps the hot loop
-    // small enough for the instruction cache).
-    uint32_t sc0 = 0u, sc1 = 0u, ic0 = 0u, ic1 = 0u, xc = 0u, iz = 0u;
+    uint32_t sc = 0u, ic = 0u;
     bool ok = true;
-    // Row exchange: post this half's pair of values, later fetch the other's.
-    // Slots alternate with the exchange count so that a new post never
-    // overwrites a value the partner has not read yet.
-    auto xpost = [&](float a, float b) {
-      float* mine = xb + (((xc & 1u) * 2 + hc) * 128 + r) * 2;
-      mine[0] = a;
-      mine[1] = b;
-      warp_arrive(xbar);
-    };
-    auto xget = [&](float& a, float& b) -> bool {
-      const bool w_ok = __all_sync(0xffffffffu, mbar_wait(xbar, xc & 1u, abort, status));
-      const float* other = xb + (((xc & 1u) * 2 + (hc ^ 1)) * 128 + r) * 2;
-      a = other[0];
-      b = other[1];
-      ++xc;
-      return w_ok;
-    };
     for (int idx = blockIdx.x; ok && idx < sh.items; idx += gridDim.x) {
       const Item it = decode_item(idx, sh);
-      if (it.n_max == 0) continue;
+      const int n = it.n[x];
+      if (n == 0) continue;
+      const int qt = it.qt[x], h = it.h[x];
       const int mslice = it.s * BHkv + it.b * sh.H_kv + it.h_kv;
-      // z_{s-1} of the group to shared memory (every read of the previous
-      // item's copy finished before any thread could get here: those reads
-      // precede sq_ready, which the retrieval MMA waited for before r_full).
-      {
-        const int t = hc * 128 + r;
-        if (t < D) zs[t] = __ldg(z_pref + (size_t)mslice * D + t);
-        warp_arrive(z_ready);
-      }
-      float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
-#pragma unroll 1
-      for (int step = 0; step < 2 * it.n_max; ++step) {
-        const int j = step >> 1, x = step & 1;
-        if (j >= (x ? it.n[1] : it.n[0])) continue;
-        float m_run = x ? m1 : m0, l_run = x ? l1 : l0;
-        const uint32_t scx = x ? sc1 : sc0;
-        const uint32_t tS = tmem + x * 256 + lane_off;
-        ok = __all_sync(0xffffffffu, mbar_wait(s_full + x, scx & 1u, abort, status));
-        if (x) sc1 = scx + 1; else sc0 = scx + 1;
+      // z_{s-1} to this slot's shared copy (every read of the previous
+      // item's copy precedes sq_ready, which the retrieval MMA waited for
+      // before r_full, which this warpgroup waited for before getting here).
+      if (r < D) zs[r] = __ldg(z_pref + (size_t)mslice * D + r);
+      warp_arrive(z_ready + x);
+      float m_run = -INFINITY, l_run = 0.f;
+      for (int j = 0; j < n; ++j) {
+        ok = __all_sync(0xffffffffu, mbar_wait(s_full + x, sc & 1u, abort, status));
+        ++sc;
         if (!ok) break;
         tc_fence_after();
-        // The whole score row (both halves): the tile max is then known to
-        // both threads of the row without any exchange; each exponentiates
-        // only its own 64 keys.
-        uint32_t sv[64], so[64];
-        tmem_ld32(tS + 64 * hc, sv);
-        tmem_ld32(tS + 64 * hc + 32, sv + 32);
-        tmem_ld32(tS + 64 * (hc ^ 1), so);
-        tmem_ld32(tS + 64 * (hc ^ 1) + 32, so + 32);
+        uint32_t sv[128];
+#pragma unroll
+        for (int c = 0; c < 4; ++c) tmem_ld32(tS + c * 32, sv + c * 32);
         tmem_wait_ld();
-        if (j == (x ? it.qt[1] : it.qt[0])) {
+        if (j == qt) {
           // Diagonal tile: key c is visible to row r iff c <= r.
-          const int lim = r - 64 * hc, limo = r - 64 * (hc ^ 1);
 #pragma unroll
-          for (int i = 0; i < 64; ++i) {
-            if (i > lim) sv[i] = __float_as_uint(-INFINITY);
-            if (i > limo) so[i] = __float_as_uint(-INFINITY);
-          }
+          for (int i = 0; i < 128; ++i)
+            if (i > r) sv[i] = __float_as_uint(-INFINITY);
         }
-        const float mt = sl2 * row_max128(sv, so);
-        if (j == 0) m_run = mt;
-        // Exponentials against the running max; after the first tile, if the
-        // row's tile max exceeds it by more than 2^8 (rare), rescale this
-        // half of O (complete through tile j-1: the scores of tile j were
-        // produced after it) and the sum, then take them.  Both threads of
-        // the row see the same tile max and decide alike.
-        if (j > 0) {
-          const bool need = mt > m_run + 8.f;
-          if (__any_sync(0xffffffffu, need)) {
-            const float f = need ? ex2_approx(m_run - mt) : 1.f;
-            const uint32_t tO = tS + 128 + hc * (D / 2);
-#pragma unroll 1
-            for (int c = 0; c < D / 32; ++c) {
-              uint32_t raw[16];
-              tmem_ld16(tO + c * 16, raw);
-              tmem_wait_ld();
-#pragma unroll
-              for (int i = 0; i < 16; ++i) raw[i] = __float_as_uint(__uint_as_float(raw[i]) * f);
-              tmem_st16(tO + c * 16, raw);
-            }
-            tmem_wait_st();
-            if (need) {
-              l_run *= f;
-              m_run = mt;
-            }
-          }
-        }
+        // The reference max: the row max of the item's first tile; later
+        // tiles are exponentiated against it directly, and only if a row's
+        // tile sum exceeds 2^16 (its max grew by more than 2^16 / 128, or
+        // overflowed) is the true tile max taken, O and the sum rescaled and
+        // the tile redone.  P stays below 2^16 and the reference never falls.
+        if (j == 0) m_run = sl2 * row_max128(sv, sv + 64);
+        // P (bf16 pairs) over the scores already read: keys 0..63 -> columns
+        // 0..31, keys 64..127 -> columns 64..95.
         uint32_t packed[32];
-        const float lsum = exp_pack64(sv, sl2, m_run, packed);
-        // P of this half's 64 keys into 32 columns inside its own score
-        // columns (keys 0..63 -> columns 0..31, keys 64..127 -> 64..95).
-        tmem_st32(tS + 64 * hc, packed);
+        float lsum = exp_pack64(sv, sl2, m_run, packed);
+        tmem_st32(tS, packed);
+        lsum += exp_pack64(sv + 64, sl2, m_run, packed);
+        tmem_st32(tS + 64, packed);
+        const bool need = !(lsum <= 65536.f);
+        if (__any_sync(0xffffffffu, need)) {
+          const float mt = need ? sl2 * row_max128(sv, sv + 64) : m_run;
+          const float f = need ? ex2_approx(m_run - mt) : 1.f;
+#pragma unroll 1
+          for (int c = 0; c < D / 16; ++c) {
+            uint32_t raw[16];
+            tmem_ld16(tO + c * 16, raw);
+            tmem_wait_ld();
+#pragma unroll
+            for (int i = 0; i < 16; ++i) raw[i] = __float_as_uint(__uint_as_float(raw[i]) * f);
+            tmem_st16(tO + c * 16, raw);
+          }
+          if (need) {
+            l_run *= f;
+            m_run = mt;
+          }
+          // Redo P against the (possibly new) reference (unchanged rows get
+          // the same values again).
+          lsum = exp_pack64(sv, sl2, m_run, packed);
+          tmem_st32(tS, packed);
+          lsum += exp_pack64(sv + 64, sl2, m_run, packed);
+          tmem_st32(tS + 64, packed);
+        }
         l_run += lsum;
-        if (x) { m1 = m_run; l1 = l_run; } else { m0 = m_run; l0 = l_run; }
         tmem_wait_st();
         tc_fence_before();
         warp_arrive(p_ready + x);
       }
       if (!ok) break;
-      // sigma(Q) in place of Q for this half's features (every QK^T product
-      // of the item is complete once its last score tiles arrived) and the
-      // partial retrieval denominator sigma(q_r) . z_{s-1} in fp32.
-      ok = __all_sync(0xffffffffu, mbar_wait(z_ready, iz & 1u, abort, status));
-      ++iz;
+      // sigma(Q) in place of Q (every QK^T product of this slot is complete
+      // once its last score tile arrived) and the retrieval denominator
+      // sigma(q_r) . z_{s-1} in fp32 from the unrounded sigma.
+      ok = __all_sync(0xffffffffu, mbar_wait(z_ready + x, ic & 1u, abort, status));
       if (!ok) break;
-      float den0 = 0.f, den1 = 0.f;
-#pragma unroll 1
-      for (int x = 0; x < 2; ++x) {
-        if ((x ? it.n[1] : it.n[0]) == 0) continue;
-        unsigned char* sQ = smem + SM::kQ + x * kTileBytes;
-        float den = 0.f;
+      unsigned char* sQ = smem + SM::kQ + (2 * x + (ic & 1u)) * kTileBytes;
+      float den = 0.f;
 #pragma unroll 2
-        for (int c8 = hc * (D / 16); c8 < (hc + 1) * (D / 16); ++c8) {
-          const uint32_t off = sw128_offset(r, c8 * 8, kBM);
-          const uint4 v = *reinterpret_cast<const uint4*>(sQ + off);
-          const float4 za = reinterpret_cast<const float4*>(zs)[2 * c8];
-          const float4 zb = reinterpret_cast<const float4*>(zs)[2 * c8 + 1];
-          const float zz[8] = {za.x, za.y, za.z, za.w, zb.x, zb.y, zb.z, zb.w};
-          const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-          uint32_t o[4];
+      for (int c8 = 0; c8 < D / 8; ++c8) {
+        const uint32_t off = sw128_offset(r, c8 * 8, kBM);
+        const uint4 v = *reinterpret_cast<const uint4*>(sQ + off);
+        const float4 za = reinterpret_cast<const float4*>(zs)[2 * c8];
+        const float4 zb = reinterpret_cast<const float4*>(zs)[2 * c8 + 1];
+        const float zz[8] = {za.x, za.y, za.z, za.w, zb.x, zb.y, zb.z, zb.w};
+        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+        uint32_t o[4];
 #pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            const float a = elu1_fast(bf16lo_to_f32(w[i]));
-            const float b = elu1_fast(bf16hi_to_f32(w[i]));
-            den = fmaf(a, zz[2 * i], den);
-            den = fmaf(b, zz[2 * i + 1], den);
-            o[i] = pack_bf16x2(a, b);
+        for (int i = 0; i < 4; ++i) {
+          // sigma = x + 1 for x > 0, e^x otherwise; half of the 2^x on the
+          // FMA pipe (both are exact to well below bf16 rounding).
+          const float2 xv = make_float2(bf16lo_to_f32(w[i]), bf16hi_to_f32(w[i]));
+          const float2 xe = make_float2(xv.x * 1.4426950408889634f, xv.y * 1.4426950408889634f);
+          float2 e;
+          if (i & 1) {
+            e = exp2_poly2(xe);
+          } else {
+            e.x = ex2_approx(xe.x);
+            e.y = ex2_approx(xe.y);
           }
-          *reinterpret_cast<uint4*>(sQ + off) = make_uint4(o[0], o[1], o[2], o[3]);
+          const float a = xv.x > 0.f ? xv.x + 1.f : e.x;
+          const float b = xv.y > 0.f ? xv.y + 1.f : e.y;
+          den = fmaf(a, zz[2 * i], den);
+          den = fmaf(b, zz[2 * i + 1], den);
+          o[i] = pack_bf16x2(a, b);
         }
-        if (x) den1 = den; else den0 = den;
-        fence_proxy_async();
-        warp_arrive(sq_ready + x);
+        *reinterpret_cast<uint4*>(sQ + off) = make_uint4(o[0], o[1], o[2], o[3]);
       }
-      // out = (1 - g)/l * O + g/den * R for this half's features: TMEM read
-      // out first (then the next item may use the slot's columns), stored
-      // from registers.
-#pragma unroll 1
-      for (int x = 0; x < 2; ++x) {
-        if ((x ? it.n[1] : it.n[0]) == 0) continue;
-        float lo, dno;
-        const float lh = x ? l1 : l0, dh = x ? den1 : den0;
-        xpost(lh, dh);
-        if (!(ok = xget(lo, dno))) break;
-        const float l = lh + lo, dn = dh + dno;
-        const uint32_t icx = x ? ic1 : ic0;
-        if (!(ok = __all_sync(0xffffffffu, mbar_wait(r_full + x, icx & 1u, abort, status)))) break;
-        if (x) ic1 = icx + 1; else ic0 = icx + 1;
-        tc_fence_after();
-        const int hx = x ? it.h[1] : it.h[0], qt = x ? it.qt[1] : it.qt[0];
-        const float gm = gate_sigmoid(__ldg(beta + hx));
-        const uint32_t tS = tmem + x * 256 + lane_off + hc * (D / 2);
-        const uint32_t tO = tmem + x * 256 + lane_off + 128 + hc * (D / 2);
-        const float wo = (1.f - gm) / l;
-        const float wm = dn != 0.f ? gm / dn : 0.f;
-        const float2 wo2 = make_float2(wo, wo), wm2 = make_float2(wm, wm);
-        uint32_t w[D / 4];
+      fence_proxy_async();
+      warp_arrive(sq_ready + x);
+      ok = __all_sync(0xffffffffu, mbar_wait(r_full + x, ic & 1u, abort, status));
+      ++ic;
+      if (!ok) break;
+      tc_fence_after();
+      // out = (1 - g)/l * O + g/den * R: TMEM read out first (then the next
+      // item may use this slot's columns), stored row by row from registers.
+      const float gm = gate_sigmoid(__ldg(beta + h));
+      const float wo = (1.f - gm) / l_run;
+      const float wm = den != 0.f ? gm / den : 0.f;
+      const float2 wo2 = make_float2(wo, wo), wm2 = make_float2(wm, wm);
+      uint32_t w[D / 2];
 #pragma unroll
-        for (int c = 0; c < D / 64; ++c) {
-          uint32_t o_raw[32], r_raw[32];
-          tmem_ld32(tO + c * 32, o_raw);
-          tmem_ld32(tS + c * 32, r_raw);
-          tmem_wait_ld();
+      for (int c = 0; c < D / 32; c += 2) {
+        // Two 32-column chunks of O and R per TMEM wait.
+        uint32_t o_raw[64], r_raw[64];
+        tmem_ld32(tO + c * 32, o_raw);
+        tmem_ld32(tS + c * 32, r_raw);
+        tmem_ld32(tO + c * 32 + 32, o_raw + 32);
+        tmem_ld32(tS + c * 32 + 32, r_raw + 32);
+        tmem_wait_ld();
 #pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            const float2 a = make_float2(__uint_as_float(o_raw[2 * i]), __uint_as_float(o_raw[2 * i + 1]));
-            const float2 m = make_float2(__uint_as_float(r_raw[2 * i]), __uint_as_float(r_raw[2 * i + 1]));
-            const float2 y = __ffma2_rn(m, wm2, __fmul2_rn(a, wo2));
-            w[c * 16 + i] = pack_bf16x2(y.x, y.y);
-          }
+        for (int i = 0; i < 32; ++i) {
+          const float2 a = make_float2(__uint_as_float(o_raw[2 * i]), __uint_as_float(o_raw[2 * i + 1]));
+          const float2 m = make_float2(__uint_as_float(r_raw[2 * i]), __uint_as_float(r_raw[2 * i + 1]));
+          const float2 y = __ffma2_rn(m, wm2, __fmul2_rn(a, wo2));
+          w[c * 16 + i] = pack_bf16x2(y.x, y.y);
         }
-        tc_fence_before();
-        warp_arrive(tmem_free + x);
-        if (qt * kBM + r < it.seg_len) {
-          uint4* dst = reinterpret_cast<uint4*>(
-              out + ((size_t)(it.b * sh.H_q + hx) * sh.L + it.seg0 + qt * kBM + r) * D + hc * (D / 2));
+      }
+      tc_fence_before();
+      warp_arrive(tmem_free + x);
+      if (qt * kBM + r < it.seg_len) {
+        uint4* dst = reinterpret_cast<uint4*>(
+            out + ((size_t)(it.b * sh.H_q + h) * sh.L + it.seg0 + qt * kBM + r) * D);
 #pragma unroll
-          for (int i = 0; i < D / 16; ++i) dst[i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
-        }
+        for (int i = 0; i < D / 8; ++i) dst[i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
       }
     }
   }

@@ -174,8 +174,10 @@ INFINI_API int infini_attn_forward_host(const void* q_h, const void* k_h, const 
 
 /* Wait for `stream` to finish, then report and clear the device status word
  * the kernels set when one of their bounded waits ran out:
- * INFINI_OK, INFINI_ERR_TIMEOUT, or INFINI_ERR_CUDA if the stream itself
- * reported an error. */
+ * INFINI_OK, INFINI_ERR_TIMEOUT, INFINI_ERR_UNSUPPORTED if a kernel found
+ * its dynamic shared memory placed where its layout cannot use it (it then
+ * computes nothing), or INFINI_ERR_CUDA if the stream itself reported an
+ * error. */
 INFINI_API int infini_attn_sync_status(void* stream);
 
 /* Benchmark support: per-kernel device timing.  While enabled, every
