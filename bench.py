@@ -39,11 +39,11 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # launch, from an ncu capture summarised under profiles/, valid only while the
 # kernel sources hash to what they were at capture time.
 ATTENTION_TRAFFIC = {
-    "8b-delta": {"bytes": 2 * (406.998272e6 + 240.843776e6),
+    "8b-delta": {"bytes": 2 * (409.577728e6 + 230.632448e6),
                  "note": "ncu capture at batch 1, scaled x2 to the batch-2 launch",
                  "profile": "profiles/tc_attention_8b-delta.md",
-                 "sha1": {"tc_attention.cu": "ab5a21d4ba3d1ccaf1dd1683fbbe86b1ab6bf640",
-                          "tc_common.cuh": "c82269991654d8b1f3bb1c0290a5eadbf9d329db"}},
+                 "sha1": {"tc_attention.cu": "4fbaf38e7f176796e2c0d07111a6b28486e54282",
+                          "tc_common.cuh": "a2612deb59163975e015c94465b32bea6a1a4f2d"}},
 }
 
 

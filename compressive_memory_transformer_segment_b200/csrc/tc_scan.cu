@@ -388,6 +388,225 @@ tc_segment_products(const __grid_constant__ CUtensorMap tm_k, const __grid_const
   }
 }
 
+// ---------------------------------------------------------------- linear-rule products (d = 128)
+
+// B_s = sigma(K_s)^T V_s and dz_s = column sums of sigma(K_s) for one
+// (segment, KV head), streamed in 64-token blocks: a 4-stage TMA ring of
+// (K, V) blocks, sigma(K) as bf16 hi/lo pairs in two alternating operand
+// buffers (the math warps build block b+1 while the tensor core multiplies
+// block b), dz summed by the math threads.  HBM-bound: each block brings
+// 32 KiB of K and V.
+constexpr int kLTok = 64;      // tokens per block
+constexpr int kLStages = 4;    // K/V ring depth
+constexpr int kLMath = 8;      // math warps
+constexpr int kLThreads = 64 + 32 * kLMath;
+
+struct LinSmem {
+  static constexpr int kD = 128;
+  static constexpr int kPanel = kLTok * 128;          // 64 rows x 128 B
+  static constexpr int kHalf = kLTok * kD * 2;        // one 64 x 128 bf16 block (K, V, hi or lo)
+  static constexpr int kStage = 2 * kHalf;            // K then V
+  static constexpr int kRing = 0;
+  static constexpr int kOp = kRing + kLStages * kStage;  // [2][hi, lo]
+  static constexpr int kRed = kOp + 2 * 2 * kHalf;       // dz partials fp32 [16 lanes][128]
+  static constexpr int kBar = kRed + 16 * kD * 4;
+  // full[kLStages] empty[kLStages] op_full[2] op_empty[2] acc_full red_ready
+  static constexpr int kNumBars = 2 * kLStages + 6;
+  static constexpr int kTmemSlot = kBar + kNumBars * 8;
+  static constexpr int kAbort = kTmemSlot + 4;
+  static constexpr int kAlloc = kAbort + 4 + 1024;
+};
+
+__global__ void __launch_bounds__(kLThreads, 1)
+tc_linear_products(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
+                   float* __restrict__ Bbuf, float* __restrict__ dz, unsigned int* __restrict__ status,
+                   int L, int S) {
+  using SM = LinSmem;
+  constexpr int D = SM::kD;
+  const int s = blockIdx.x, bh = blockIdx.y, BH = gridDim.y;
+  const int seg0 = s * S, seg_len = min(S, L - seg0);
+  const int nblk = (seg_len + kLTok - 1) / kLTok;
+  const size_t slice = (size_t)s * BH + bh;
+
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
+  unsigned char* smem = reinterpret_cast<unsigned char*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  unsigned char* ring = smem + SM::kRing;
+  unsigned char* op = smem + SM::kOp;
+  float* red = reinterpret_cast<float*>(smem + SM::kRed);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + SM::kBar);
+  uint64_t* full = bars;
+  uint64_t* empty = bars + kLStages;
+  uint64_t* op_full = bars + 2 * kLStages;
+  uint64_t* op_empty = op_full + 2;
+  uint64_t* acc_full = op_empty + 2;
+  uint64_t* red_ready = acc_full + 1;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + SM::kTmemSlot);
+  volatile int* abort = reinterpret_cast<volatile int*>(smem + SM::kAbort);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < kLStages; ++i) {
+      mbar_init(full + i, 1);
+      mbar_init(empty + i, kLMath + 1);  // math warps (K read) + the MMA commit (V read)
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(op_full + i, kLMath);
+      mbar_init(op_empty + i, 1);
+    }
+    mbar_init(acc_full, 1);
+    mbar_init(red_ready, kLMath);
+    *abort = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, 128);
+    tmem_relinquish();
+    tc_fence_before();
+  }
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    // ---------------------------------------------- TMA producer (whole warp waits, lane 0 issues)
+    int issued = 0;
+    for (int b = 0; b < nblk; ++b) {
+      const int st = b % kLStages;
+      const uint32_t ph = (uint32_t)(b / kLStages) & 1u;
+      if (!__all_sync(0xffffffffu, mbar_wait(empty + st, ph ^ 1u, abort, status))) break;
+      if (lane == 0) {
+        unsigned char* dst = ring + st * SM::kStage;
+        mbar_arrive_expect_tx(full + st, SM::kStage);
+        for (int p = 0; p < D / 64; ++p) {
+          tma_load_3d(dst + p * SM::kPanel, &tm_k, full + st, p * 64, seg0 + b * kLTok, bh);
+          tma_load_3d(dst + SM::kHalf + p * SM::kPanel, &tm_v, full + st, p * 64, seg0 + b * kLTok, bh);
+        }
+      }
+      issued = b + 1;
+    }
+    // Every copy issued must land before the CTA exits.
+    for (int b = max(0, issued - kLStages); b < issued; ++b)
+      mbar_wait(full + b % kLStages, (uint32_t)(b / kLStages) & 1u, abort, status, false);
+    __syncwarp();
+  } else if (warp == 1) {
+    // ---------------------------------------------- MMA issuer (whole warp waits, lane 0 issues)
+    constexpr uint32_t idesc = idesc_bf16_f32(128, D, true, true);
+    const uint64_t dop = sw128_desc(smem_u32(op), SM::kPanel, 1024);
+    const uint64_t dring = sw128_desc(smem_u32(ring + SM::kHalf), SM::kPanel, 1024);
+    bool ok = true;
+    for (int b = 0; ok && b < nblk; ++b) {
+      const int st = b % kLStages, ob = b & 1;
+      if (!(ok = __all_sync(0xffffffffu, mbar_wait(op_full + ob, (uint32_t)(b >> 1) & 1u, abort, status)))) break;
+      if (!(ok = __all_sync(0xffffffffu, mbar_wait(full + st, (uint32_t)(b / kLStages) & 1u, abort, status)))) break;
+      tc_fence_after();
+      if (lane == 0) {
+        const uint64_t hi = dop + ((ob * 2 * SM::kHalf) >> 4);
+        const uint64_t lo = hi + (SM::kHalf >> 4);
+        const uint64_t vv = dring + ((st * SM::kStage) >> 4);
+#pragma unroll
+        for (int kk = 0; kk < kLTok / 16; ++kk) {
+          const uint32_t stp = mnmajor_step(kk);
+          mma_ss(tmem, hi + stp, vv + stp, idesc, (b > 0 || kk > 0) ? 1u : 0u);
+          mma_ss(tmem, lo + stp, vv + stp, idesc, 1u);
+        }
+        tc_commit(op_empty + ob);
+        tc_commit(empty + st);
+      }
+    }
+    if (lane == 0) tc_commit(acc_full);
+    __syncwarp();
+    mbar_wait(acc_full, 0, abort, status, false);
+    __syncwarp();
+  } else {
+    // ---------------------------------------------- math warps
+    // Thread (column chunk cg of 8 columns, token lane tl): tokens tl, tl+16, ...
+    const int mt = threadIdx.x - 64;
+    const int cg = mt & 15, tl = mt >> 4;
+    float acc[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) acc[i] = 0.f;
+    bool ok = true;
+    for (int b = 0; b < nblk; ++b) {
+      const int st = b % kLStages, ob = b & 1;
+      ok = __all_sync(0xffffffffu, mbar_wait(full + st, (uint32_t)(b / kLStages) & 1u, abort, status));
+      if (!ok) break;
+      const unsigned char* kb = ring + st * SM::kStage;
+      uint4 hi4[kLTok / 16], lo4[kLTok / 16];
+#pragma unroll
+      for (int i = 0; i < kLTok / 16; ++i) {
+        const int t = tl + 16 * i;
+        const bool valid = b * kLTok + t < seg_len;
+        const uint32_t off = sw128_offset(t, 8 * cg, kLTok);
+        const uint4 kv = *reinterpret_cast<const uint4*>(kb + off);
+        const uint32_t kw[4] = {kv.x, kv.y, kv.z, kv.w};
+        uint32_t hw[4], lw[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float a = valid ? elu1_fast(bf16lo_to_f32(kw[e])) : 0.f;
+          const float c = valid ? elu1_fast(bf16hi_to_f32(kw[e])) : 0.f;
+          acc[2 * e] += a;
+          acc[2 * e + 1] += c;
+          hw[e] = pack_bf16x2(a, c);
+          lw[e] = pack_bf16x2(a - bf16lo_to_f32(hw[e]), c - bf16hi_to_f32(hw[e]));
+        }
+        hi4[i] = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+        lo4[i] = make_uint4(lw[0], lw[1], lw[2], lw[3]);
+      }
+      // K of this block has been read.
+      __syncwarp();
+      if (lane == 0) mbar_arrive(empty + st);
+      // The operand buffer is free once the MMAs of block b - 2 are done.
+      ok = __all_sync(0xffffffffu, mbar_wait(op_empty + ob, ((uint32_t)(b >> 1) & 1u) ^ 1u, abort, status));
+      if (!ok) break;
+      unsigned char* hb = op + ob * 2 * SM::kHalf;
+#pragma unroll
+      for (int i = 0; i < kLTok / 16; ++i) {
+        const uint32_t off = sw128_offset(tl + 16 * i, 8 * cg, kLTok);
+        *reinterpret_cast<uint4*>(hb + off) = hi4[i];
+        *reinterpret_cast<uint4*>(hb + SM::kHalf + off) = lo4[i];
+      }
+      fence_proxy_async();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(op_full + ob);
+    }
+    // dz: the 16 token lanes' partial column sums, reduced in shared memory.
+#pragma unroll
+    for (int i = 0; i < 8; ++i) red[tl * D + 8 * cg + i] = acc[i];
+    __syncwarp();
+    if (lane == 0) mbar_arrive(red_ready);
+    if (ok) ok = __all_sync(0xffffffffu, mbar_wait(red_ready, 0, abort, status));
+    if (ok && mt < D) {
+      float sum = 0.f;
+#pragma unroll
+      for (int j = 0; j < 16; ++j) sum += red[j * D + mt];
+      dz[slice * D + mt] = sum;
+    }
+    // B_s: TMEM lane k = row k; the two warps of a lane quarter take 64 columns each.
+    if (ok) ok = __all_sync(0xffffffffu, mbar_wait(acc_full, 0, abort, status));
+    if (ok) {
+      tc_fence_after();
+      const int k = 32 * (warp & 3) + lane, half = (warp - 2) >> 2;
+      const uint32_t ta = tmem + ((uint32_t)(32 * (warp & 3)) << 16) + 64 * half;
+      uint32_t v[64];
+      tmem_ld32(ta, v);
+      tmem_ld32(ta + 32, v + 32);
+      tmem_wait_ld();
+      float4* dst = reinterpret_cast<float4*>(Bbuf + (slice * D + k) * D + 64 * half);
+#pragma unroll
+      for (int i = 0; i < 16; ++i)
+        dst[i] = make_float4(__uint_as_float(v[4 * i]), __uint_as_float(v[4 * i + 1]),
+                             __uint_as_float(v[4 * i + 2]), __uint_as_float(v[4 * i + 3]));
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 128);
+  }
+}
+
 // ---------------------------------------------------------------- sequential combine
 
 constexpr int kCB = 8;  // columns of M per combine CTA (delta)
@@ -579,7 +798,18 @@ cudaError_t launch(const Problem& p, cudaStream_t stream) {
                                                                  p.T);
     return cudaGetLastError();
   }
-  if ((e = launch_products<D, false>(p, tk, tv, stream)) != cudaSuccess) return e;
+  if (D == 128) {
+    CUtensorMap lk, lv;
+    if (!make_map(&lk, p.k, D, p.L, BHkv, kLTok) || !make_map(&lv, p.v, D, p.L, BHkv, kLTok))
+      return cudaErrorInvalidValue;
+    const int smem = LinSmem::kAlloc;
+    e = cudaFuncSetAttribute(tc_linear_products, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    tc_linear_products<<<dim3(p.T, BH), kLThreads, smem, stream>>>(lk, lv, p.Bbuf, p.dz, p.status, p.L, p.S);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  } else if ((e = launch_products<D, false>(p, tk, tv, stream)) != cudaSuccess) {
+    return e;
+  }
   combine_linear<D><<<dim3(BH, (D * D + 1023) / 1024), 256, 0, stream>>>(
       p.M_in, p.Bbuf, p.dz, Mp, p.z_pref, p.M_out, p.z_out, p.T);
   return cudaGetLastError();
