@@ -39,19 +39,22 @@ using namespace tc;
 
 // ---------------------------------------------------------------- dz and z prefix
 
-// dz[s][bh][c] = sum over the segment's rows t of sigma(k[bh][t][c]).
-// Grid (T, B*H_kv), block 256 threads: thread (token lane tg, 8-column group
-// cg) reads 16-byte pieces of rows tg, tg + NT, ...; the NT partial sums of
-// each column are then added in shared memory.
+// Partial column sums of sigma(K): dz[s * C + c][bh][col] = sum over rows t
+// of chunk c (of C equal row chunks of segment s) of sigma(k[bh][t][col]).
+// Grid (T * C, B*H_kv), block 256 threads: thread (token lane tg, 8-column
+// group cg) reads 16-byte pieces of rows tg, tg + NT, ...; the NT partial
+// sums of each column are then added in shared memory.  Splitting segments
+// into chunks gives the read of K enough CTAs to run at HBM speed.
 template <int D>
 __global__ void __launch_bounds__(256) zsum(const __nv_bfloat16* __restrict__ k,
-                                            float* __restrict__ dz, int L, int S) {
+                                            float* __restrict__ dz, int L, int S, int C) {
   constexpr int kCG = D / 8;      // 16-byte column groups per row
   constexpr int kNT = 256 / kCG;  // token lanes
   __shared__ float part[kNT * D];
-  const int s = blockIdx.x, bh = blockIdx.y, tid = threadIdx.x;
+  const int s = blockIdx.x / C, c = blockIdx.x % C, bh = blockIdx.y, tid = threadIdx.x;
   const int cg = tid % kCG, tg = tid / kCG;
-  const int r0 = s * S, r1 = min(r0 + S, L);
+  const int chunk = (S + C - 1) / C;
+  const int r0 = s * S + c * chunk, r1 = min(min(r0 + chunk, s * S + S), L);
   const uint4* base = reinterpret_cast<const uint4*>(k + (size_t)bh * L * D) + cg;
   float acc[8];
 #pragma unroll
@@ -73,23 +76,30 @@ __global__ void __launch_bounds__(256) zsum(const __nv_bfloat16* __restrict__ k,
     float sum = 0.f;
 #pragma unroll 8
     for (int j = 0; j < kNT; ++j) sum += part[j * D + tid];
-    dz[((size_t)s * gridDim.y + bh) * D + tid] = sum;
+    dz[((size_t)blockIdx.x * gridDim.y + bh) * D + tid] = sum;
   }
 }
 
-// z_{s-1} for s = 1..T-1 into z_pref (slot 0 already holds z_in) and z_T.
-// Grid (B*H_kv), block D threads.
+// z_{s-1} for s = 1..T-1 into z_pref (slot 0 already holds z_in) and z_T,
+// from the C chunk partials of every segment.  Grid (B*H_kv), block D threads.
 template <int D>
 __global__ void __launch_bounds__(128) zprefix(const float* __restrict__ dz, float* __restrict__ z_pref,
-                                               float* __restrict__ z_out, int T) {
+                                               float* __restrict__ z_out, int T, int C) {
   const int bh = blockIdx.x, c = threadIdx.x, BH = gridDim.x;
   float z = z_pref[(size_t)bh * D + c];
-  for (int s = 1; s < T; ++s) {
-    z += dz[((size_t)(s - 1) * BH + bh) * D + c];
-    z_pref[((size_t)s * BH + bh) * D + c] = z;
+  for (int s = 0; s < T; ++s) {
+    if (s > 0) z_pref[((size_t)s * BH + bh) * D + c] = z;
+    float seg = 0.f;
+    for (int j = 0; j < C; ++j) seg += dz[((size_t)(s * C + j) * BH + bh) * D + c];
+    z += seg;
   }
-  z_out[(size_t)bh * D + c] = z + dz[((size_t)(T - 1) * BH + bh) * D + c];
+  z_out[(size_t)bh * D + c] = z;
 }
+
+constexpr int kZChunksMax = 8;
+
+// Row chunks per segment for zsum: about 256 rows each, at most kZChunksMax.
+int zsum_chunks(int S) { return S >= 256 * kZChunksMax ? kZChunksMax : (S >= 512 ? S / 256 : 1); }
 
 // ---------------------------------------------------------------- segment products
 
@@ -388,41 +398,50 @@ tc_segment_products(const __grid_constant__ CUtensorMap tm_k, const __grid_const
   }
 }
 
-// ---------------------------------------------------------------- linear-rule products (d = 128)
+// ---------------------------------------------------------------- pipelined products (d = 128)
 
-// B_s = sigma(K_s)^T V_s and dz_s = column sums of sigma(K_s) for one
-// (segment, KV head), streamed in 64-token blocks: a 4-stage TMA ring of
-// (K, V) blocks, sigma(K) as bf16 hi/lo pairs in two alternating operand
-// buffers (the math warps build block b+1 while the tensor core multiplies
-// block b), dz summed by the math threads.  HBM-bound: each block brings
-// 32 KiB of K and V.
+// Per (segment, KV head), streamed in 64-token blocks:
+//   linear: B_s = sigma(K_s)^T V_s and dz_s = column sums of sigma(K_s);
+//   delta : B_s as above and G_s = Y^T sigma(K_s), Y = D^-1 sigma(K_s),
+//           D = diag(sigma(K_s) z_{s-1}) (rows with r_t = 0 give zero rows).
+// A TMA ring of (K, V) blocks; sigma(K) (and Y) as bf16 hi/lo pairs in two
+// alternating operand buffers, so the math warps build block b+1 while the
+// tensor core multiplies block b; dz (linear) summed by the math threads.
+// The linear rule is HBM-bound (each block brings 32 KiB of K and V); the
+// delta rule does 20 MMAs (128 x 128 x 16) per block.
 constexpr int kLTok = 64;      // tokens per block
-constexpr int kLStages = 4;    // K/V ring depth
 constexpr int kLMath = 8;      // math warps
 constexpr int kLThreads = 64 + 32 * kLMath;
 
-struct LinSmem {
+template <bool DELTA>
+struct PipeSmem {
   static constexpr int kD = 128;
-  static constexpr int kPanel = kLTok * 128;          // 64 rows x 128 B
-  static constexpr int kHalf = kLTok * kD * 2;        // one 64 x 128 bf16 block (K, V, hi or lo)
-  static constexpr int kStage = 2 * kHalf;            // K then V
+  static constexpr int kStages = DELTA ? 2 : 4;          // K/V ring depth
+  static constexpr int kPanel = kLTok * 128;              // 64 rows x 128 B
+  static constexpr int kHalf = kLTok * kD * 2;            // one 64 x 128 bf16 block
+  static constexpr int kStage = 2 * kHalf;                // K then V
+  static constexpr int kOpParts = DELTA ? 4 : 2;          // sigma hi, lo (, Y hi, lo)
   static constexpr int kRing = 0;
-  static constexpr int kOp = kRing + kLStages * kStage;  // [2][hi, lo]
-  static constexpr int kRed = kOp + 2 * 2 * kHalf;       // dz partials fp32 [16 lanes][128]
-  static constexpr int kBar = kRed + 16 * kD * 4;
-  // full[kLStages] empty[kLStages] op_full[2] op_empty[2] acc_full red_ready
-  static constexpr int kNumBars = 2 * kLStages + 6;
+  static constexpr int kOp = kRing + kStages * kStage;    // [2][parts]
+  static constexpr int kRed = kOp + 2 * kOpParts * kHalf; // dz partials fp32 [16][128]
+  static constexpr int kZ = kRed + (DELTA ? 0 : 16 * kD * 4);  // z_{s-1} fp32 [128] (delta)
+  static constexpr int kBar = kZ + (DELTA ? kD * 4 : 0);
+  // full[kStages] empty[kStages] op_full[2] op_empty[2] acc_full red_ready
+  static constexpr int kNumBars = 2 * kStages + 6;
   static constexpr int kTmemSlot = kBar + kNumBars * 8;
   static constexpr int kAbort = kTmemSlot + 4;
   static constexpr int kAlloc = kAbort + 4 + 1024;
+  static constexpr uint32_t kTmemCols = DELTA ? 256 : 128;  // [G |] B
 };
 
+template <bool DELTA>
 __global__ void __launch_bounds__(kLThreads, 1)
-tc_linear_products(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
-                   float* __restrict__ Bbuf, float* __restrict__ dz, unsigned int* __restrict__ status,
-                   int L, int S) {
-  using SM = LinSmem;
+tc_pipe_products(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
+                 const float* __restrict__ z_pref, float* __restrict__ Gbuf, float* __restrict__ Bbuf,
+                 float* __restrict__ dz, unsigned int* __restrict__ status, int L, int S) {
+  using SM = PipeSmem<DELTA>;
   constexpr int D = SM::kD;
+  constexpr int kStages = SM::kStages;
   const int s = blockIdx.x, bh = blockIdx.y, BH = gridDim.y;
   const int seg0 = s * S, seg_len = min(S, L - seg0);
   const int nblk = (seg_len + kLTok - 1) / kLTok;
@@ -434,10 +453,11 @@ tc_linear_products(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
   unsigned char* ring = smem + SM::kRing;
   unsigned char* op = smem + SM::kOp;
   float* red = reinterpret_cast<float*>(smem + SM::kRed);
+  float* zs = reinterpret_cast<float*>(smem + SM::kZ);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + SM::kBar);
   uint64_t* full = bars;
-  uint64_t* empty = bars + kLStages;
-  uint64_t* op_full = bars + 2 * kLStages;
+  uint64_t* empty = bars + kStages;
+  uint64_t* op_full = bars + 2 * kStages;
   uint64_t* op_empty = op_full + 2;
   uint64_t* acc_full = op_empty + 2;
   uint64_t* red_ready = acc_full + 1;
@@ -446,7 +466,7 @@ tc_linear_products(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i < kLStages; ++i) {
+    for (int i = 0; i < kStages; ++i) {
       mbar_init(full + i, 1);
       mbar_init(empty + i, kLMath + 1);  // math warps (K read) + the MMA commit (V read)
     }
@@ -459,21 +479,24 @@ tc_linear_products(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
     *abort = 0;
     fence_mbar_init();
   }
+  if (DELTA)
+    for (int i = threadIdx.x; i < D; i += kLThreads) zs[i] = z_pref[slice * D + i];
   if (warp == 1) {
-    tmem_alloc(tmem_slot, 128);
+    tmem_alloc(tmem_slot, SM::kTmemCols);
     tmem_relinquish();
     tc_fence_before();
   }
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  const uint32_t tG = tmem, tB = DELTA ? tmem + 128 : tmem;
 
   if (warp == 0) {
     // ---------------------------------------------- TMA producer (whole warp waits, lane 0 issues)
     int issued = 0;
     for (int b = 0; b < nblk; ++b) {
-      const int st = b % kLStages;
-      const uint32_t ph = (uint32_t)(b / kLStages) & 1u;
+      const int st = b % kStages;
+      const uint32_t ph = (uint32_t)(b / kStages) & 1u;
       if (!__all_sync(0xffffffffu, mbar_wait(empty + st, ph ^ 1u, abort, status))) break;
       if (lane == 0) {
         unsigned char* dst = ring + st * SM::kStage;
@@ -486,8 +509,8 @@ tc_linear_products(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
       issued = b + 1;
     }
     // Every copy issued must land before the CTA exits.
-    for (int b = max(0, issued - kLStages); b < issued; ++b)
-      mbar_wait(full + b % kLStages, (uint32_t)(b / kLStages) & 1u, abort, status, false);
+    for (int b = max(0, issued - kStages); b < issued; ++b)
+      mbar_wait(full + b % kStages, (uint32_t)(b / kStages) & 1u, abort, status, false);
     __syncwarp();
   } else if (warp == 1) {
     // ---------------------------------------------- MMA issuer (whole warp waits, lane 0 issues)
@@ -496,19 +519,28 @@ tc_linear_products(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
     const uint64_t dring = sw128_desc(smem_u32(ring + SM::kHalf), SM::kPanel, 1024);
     bool ok = true;
     for (int b = 0; ok && b < nblk; ++b) {
-      const int st = b % kLStages, ob = b & 1;
+      const int st = b % kStages, ob = b & 1;
       if (!(ok = __all_sync(0xffffffffu, mbar_wait(op_full + ob, (uint32_t)(b >> 1) & 1u, abort, status)))) break;
-      if (!(ok = __all_sync(0xffffffffu, mbar_wait(full + st, (uint32_t)(b / kLStages) & 1u, abort, status)))) break;
+      if (!(ok = __all_sync(0xffffffffu, mbar_wait(full + st, (uint32_t)(b / kStages) & 1u, abort, status)))) break;
       tc_fence_after();
       if (lane == 0) {
-        const uint64_t hi = dop + ((ob * 2 * SM::kHalf) >> 4);
-        const uint64_t lo = hi + (SM::kHalf >> 4);
+        // Operand parts: sigma hi, sigma lo, (Y hi, Y lo).
+        const uint64_t shi = dop + ((ob * SM::kOpParts * SM::kHalf) >> 4);
+        const uint64_t slo = shi + (SM::kHalf >> 4);
+        const uint64_t yhi = shi + ((2 * SM::kHalf) >> 4);
+        const uint64_t ylo = shi + ((3 * SM::kHalf) >> 4);
         const uint64_t vv = dring + ((st * SM::kStage) >> 4);
 #pragma unroll
         for (int kk = 0; kk < kLTok / 16; ++kk) {
           const uint32_t stp = mnmajor_step(kk);
-          mma_ss(tmem, hi + stp, vv + stp, idesc, (b > 0 || kk > 0) ? 1u : 0u);
-          mma_ss(tmem, lo + stp, vv + stp, idesc, 1u);
+          const uint32_t acc = (b > 0 || kk > 0) ? 1u : 0u;
+          if (DELTA) {
+            mma_ss(tG, yhi + stp, shi + stp, idesc, acc);
+            mma_ss(tG, ylo + stp, shi + stp, idesc, 1u);
+            mma_ss(tG, yhi + stp, slo + stp, idesc, 1u);
+          }
+          mma_ss(tB, shi + stp, vv + stp, idesc, acc);
+          mma_ss(tB, slo + stp, vv + stp, idesc, 1u);
         }
         tc_commit(op_empty + ob);
         tc_commit(empty + st);
@@ -520,19 +552,25 @@ tc_linear_products(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
     __syncwarp();
   } else {
     // ---------------------------------------------- math warps
-    // Thread (column chunk cg of 8 columns, token lane tl): tokens tl, tl+16, ...
+    // Thread (column chunk cg of 8 columns, token lane tl): tokens tl, tl+16,
+    // ...; the 16 threads of a token are lanes 0..15 or 16..31 of one warp.
     const int mt = threadIdx.x - 64;
     const int cg = mt & 15, tl = mt >> 4;
     float acc[8];
 #pragma unroll
     for (int i = 0; i < 8; ++i) acc[i] = 0.f;
+    float zc[8];
+    if (DELTA) {
+#pragma unroll
+      for (int i = 0; i < 8; ++i) zc[i] = zs[8 * cg + i];
+    }
     bool ok = true;
     for (int b = 0; b < nblk; ++b) {
-      const int st = b % kLStages, ob = b & 1;
-      ok = __all_sync(0xffffffffu, mbar_wait(full + st, (uint32_t)(b / kLStages) & 1u, abort, status));
+      const int st = b % kStages, ob = b & 1;
+      ok = __all_sync(0xffffffffu, mbar_wait(full + st, (uint32_t)(b / kStages) & 1u, abort, status));
       if (!ok) break;
       const unsigned char* kb = ring + st * SM::kStage;
-      uint4 hi4[kLTok / 16], lo4[kLTok / 16];
+      uint4 hi4[kLTok / 16], lo4[kLTok / 16], yh4[kLTok / 16], yl4[kLTok / 16];
 #pragma unroll
       for (int i = 0; i < kLTok / 16; ++i) {
         const int t = tl + 16 * i;
@@ -540,18 +578,38 @@ tc_linear_products(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
         const uint32_t off = sw128_offset(t, 8 * cg, kLTok);
         const uint4 kv = *reinterpret_cast<const uint4*>(kb + off);
         const uint32_t kw[4] = {kv.x, kv.y, kv.z, kv.w};
+        float sg[8];
         uint32_t hw[4], lw[4];
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
-          const float a = valid ? elu1_fast(bf16lo_to_f32(kw[e])) : 0.f;
-          const float c = valid ? elu1_fast(bf16hi_to_f32(kw[e])) : 0.f;
-          acc[2 * e] += a;
-          acc[2 * e + 1] += c;
-          hw[e] = pack_bf16x2(a, c);
-          lw[e] = pack_bf16x2(a - bf16lo_to_f32(hw[e]), c - bf16hi_to_f32(hw[e]));
+          sg[2 * e] = valid ? elu1_fast(bf16lo_to_f32(kw[e])) : 0.f;
+          sg[2 * e + 1] = valid ? elu1_fast(bf16hi_to_f32(kw[e])) : 0.f;
+          hw[e] = pack_bf16x2(sg[2 * e], sg[2 * e + 1]);
+          lw[e] = pack_bf16x2(sg[2 * e] - bf16lo_to_f32(hw[e]), sg[2 * e + 1] - bf16hi_to_f32(hw[e]));
         }
         hi4[i] = make_uint4(hw[0], hw[1], hw[2], hw[3]);
         lo4[i] = make_uint4(lw[0], lw[1], lw[2], lw[3]);
+        if (DELTA) {
+          // r_t = sigma(k_t) . z_{s-1} over the token's 16 threads; Y = sigma / r.
+          float r = 0.f;
+#pragma unroll
+          for (int e = 0; e < 8; ++e) r = fmaf(sg[e], zc[e], r);
+#pragma unroll
+          for (int o = 8; o > 0; o >>= 1) r += __shfl_xor_sync(0xffffffffu, r, o);
+          const float w = r != 0.f ? 1.f / r : 0.f;
+          uint32_t yh[4], yl[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const float a = w * sg[2 * e], c = w * sg[2 * e + 1];
+            yh[e] = pack_bf16x2(a, c);
+            yl[e] = pack_bf16x2(a - bf16lo_to_f32(yh[e]), c - bf16hi_to_f32(yh[e]));
+          }
+          yh4[i] = make_uint4(yh[0], yh[1], yh[2], yh[3]);
+          yl4[i] = make_uint4(yl[0], yl[1], yl[2], yl[3]);
+        } else {
+#pragma unroll
+          for (int e = 0; e < 8; ++e) acc[e] += sg[e];
+        }
       }
       // K of this block has been read.
       __syncwarp();
@@ -559,51 +617,76 @@ tc_linear_products(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
       // The operand buffer is free once the MMAs of block b - 2 are done.
       ok = __all_sync(0xffffffffu, mbar_wait(op_empty + ob, ((uint32_t)(b >> 1) & 1u) ^ 1u, abort, status));
       if (!ok) break;
-      unsigned char* hb = op + ob * 2 * SM::kHalf;
+      unsigned char* hb = op + ob * SM::kOpParts * SM::kHalf;
 #pragma unroll
       for (int i = 0; i < kLTok / 16; ++i) {
         const uint32_t off = sw128_offset(tl + 16 * i, 8 * cg, kLTok);
         *reinterpret_cast<uint4*>(hb + off) = hi4[i];
         *reinterpret_cast<uint4*>(hb + SM::kHalf + off) = lo4[i];
+        if (DELTA) {
+          *reinterpret_cast<uint4*>(hb + 2 * SM::kHalf + off) = yh4[i];
+          *reinterpret_cast<uint4*>(hb + 3 * SM::kHalf + off) = yl4[i];
+        }
       }
       fence_proxy_async();
       __syncwarp();
       if (lane == 0) mbar_arrive(op_full + ob);
     }
-    // dz: the 16 token lanes' partial column sums, reduced in shared memory.
+    if (!DELTA) {
+      // dz: the 16 token lanes' partial column sums, reduced in shared memory.
 #pragma unroll
-    for (int i = 0; i < 8; ++i) red[tl * D + 8 * cg + i] = acc[i];
-    __syncwarp();
-    if (lane == 0) mbar_arrive(red_ready);
-    if (ok) ok = __all_sync(0xffffffffu, mbar_wait(red_ready, 0, abort, status));
-    if (ok && mt < D) {
-      float sum = 0.f;
+      for (int i = 0; i < 8; ++i) red[tl * D + 8 * cg + i] = acc[i];
+      __syncwarp();
+      if (lane == 0) mbar_arrive(red_ready);
+      if (ok) ok = __all_sync(0xffffffffu, mbar_wait(red_ready, 0, abort, status));
+      if (ok && mt < D) {
+        float sum = 0.f;
 #pragma unroll
-      for (int j = 0; j < 16; ++j) sum += red[j * D + mt];
-      dz[slice * D + mt] = sum;
+        for (int j = 0; j < 16; ++j) sum += red[j * D + mt];
+        dz[slice * D + mt] = sum;
+      }
     }
-    // B_s: TMEM lane k = row k; the two warps of a lane quarter take 64 columns each.
+    // The products: TMEM lane k = row k.  Linear: the two warps of a lane
+    // quarter take 64 columns of B each; delta: one takes G, the other B.
     if (ok) ok = __all_sync(0xffffffffu, mbar_wait(acc_full, 0, abort, status));
     if (ok) {
       tc_fence_after();
       const int k = 32 * (warp & 3) + lane, half = (warp - 2) >> 2;
-      const uint32_t ta = tmem + ((uint32_t)(32 * (warp & 3)) << 16) + 64 * half;
-      uint32_t v[64];
-      tmem_ld32(ta, v);
-      tmem_ld32(ta + 32, v + 32);
-      tmem_wait_ld();
-      float4* dst = reinterpret_cast<float4*>(Bbuf + (slice * D + k) * D + 64 * half);
+      const uint32_t lq = (uint32_t)(32 * (warp & 3)) << 16;
+      if (DELTA) {
+        float* rowp = (half ? Bbuf : Gbuf) + (slice * D + k) * D;
+        const uint32_t ta = (half ? tB : tG) + lq;
 #pragma unroll
-      for (int i = 0; i < 16; ++i)
-        dst[i] = make_float4(__uint_as_float(v[4 * i]), __uint_as_float(v[4 * i + 1]),
-                             __uint_as_float(v[4 * i + 2]), __uint_as_float(v[4 * i + 3]));
+        for (int c = 0; c < D / 64; ++c) {
+          uint32_t v[64];
+          tmem_ld32(ta + 64 * c, v);
+          tmem_ld32(ta + 64 * c + 32, v + 32);
+          tmem_wait_ld();
+          float4* dst = reinterpret_cast<float4*>(rowp + 64 * c);
+#pragma unroll
+          for (int i = 0; i < 16; ++i)
+            dst[i] = make_float4(__uint_as_float(v[4 * i]), __uint_as_float(v[4 * i + 1]),
+                                 __uint_as_float(v[4 * i + 2]), __uint_as_float(v[4 * i + 3]));
+        }
+      } else {
+        const uint32_t ta = tB + lq + 64 * half;
+        uint32_t v[64];
+        tmem_ld32(ta, v);
+        tmem_ld32(ta + 32, v + 32);
+        tmem_wait_ld();
+        float4* dst = reinterpret_cast<float4*>(Bbuf + (slice * D + k) * D + 64 * half);
+#pragma unroll
+        for (int i = 0; i < 16; ++i)
+          dst[i] = make_float4(__uint_as_float(v[4 * i]), __uint_as_float(v[4 * i + 1]),
+                               __uint_as_float(v[4 * i + 2]), __uint_as_float(v[4 * i + 3]));
+      }
     }
   }
   tc_fence_before();
   __syncthreads();
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem, 128);
+    tmem_dealloc(tmem, SM::kTmemCols);
   }
 }
 
@@ -776,6 +859,21 @@ cudaError_t launch_products(const Problem& p, const CUtensorMap& tk, const CUten
   return cudaGetLastError();
 }
 
+template <bool DELTA>
+cudaError_t launch_pipe_products(const Problem& p, cudaStream_t stream) {
+  CUtensorMap lk, lv;
+  const uint64_t BHkv = (uint64_t)p.B * p.H_kv;
+  if (!make_map(&lk, p.k, 128, p.L, BHkv, kLTok) || !make_map(&lv, p.v, 128, p.L, BHkv, kLTok))
+    return cudaErrorInvalidValue;
+  const int smem = PipeSmem<DELTA>::kAlloc;
+  auto kern = tc_pipe_products<DELTA>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return e;
+  kern<<<dim3(p.T, (unsigned)BHkv), kLThreads, smem, stream>>>(lk, lv, p.z_pref, p.Gbuf, p.Bbuf, p.dz,
+                                                               p.status, p.L, p.S);
+  return cudaGetLastError();
+}
+
 template <int D>
 cudaError_t launch(const Problem& p, cudaStream_t stream) {
   CUtensorMap tk, tv;
@@ -786,11 +884,17 @@ cudaError_t launch(const Problem& p, cudaStream_t stream) {
   __nv_bfloat16* Mp = static_cast<__nv_bfloat16*>(p.M_pref);
   cudaError_t e;
   if (p.delta) {
-    zsum<D><<<dim3(p.T, BH), 256, 0, stream>>>(static_cast<const __nv_bfloat16*>(p.k), p.dz, p.L, p.S);
+    const int C = zsum_chunks(p.S);
+    zsum<D><<<dim3(p.T * C, BH), 256, 0, stream>>>(static_cast<const __nv_bfloat16*>(p.k), p.dz, p.L,
+                                                   p.S, C);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    zprefix<D><<<BH, D, 0, stream>>>(p.dz, p.z_pref, p.z_out, p.T);
+    zprefix<D><<<BH, D, 0, stream>>>(p.dz, p.z_pref, p.z_out, p.T, C);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    if ((e = launch_products<D, true>(p, tk, tv, stream)) != cudaSuccess) return e;
+    if (D == 128)
+      e = launch_pipe_products<true>(p, stream);
+    else
+      e = launch_products<D, true>(p, tk, tv, stream);
+    if (e != cudaSuccess) return e;
     const int csmem = (2 * D * D + D * kCB) * (int)sizeof(float);
     e = cudaFuncSetAttribute(combine_delta<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, csmem);
     if (e != cudaSuccess) return e;
@@ -798,18 +902,11 @@ cudaError_t launch(const Problem& p, cudaStream_t stream) {
                                                                  p.T);
     return cudaGetLastError();
   }
-  if (D == 128) {
-    CUtensorMap lk, lv;
-    if (!make_map(&lk, p.k, D, p.L, BHkv, kLTok) || !make_map(&lv, p.v, D, p.L, BHkv, kLTok))
-      return cudaErrorInvalidValue;
-    const int smem = LinSmem::kAlloc;
-    e = cudaFuncSetAttribute(tc_linear_products, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-    if (e != cudaSuccess) return e;
-    tc_linear_products<<<dim3(p.T, BH), kLThreads, smem, stream>>>(lk, lv, p.Bbuf, p.dz, p.status, p.L, p.S);
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  } else if ((e = launch_products<D, false>(p, tk, tv, stream)) != cudaSuccess) {
-    return e;
-  }
+  if (D == 128)
+    e = launch_pipe_products<false>(p, stream);
+  else
+    e = launch_products<D, false>(p, tk, tv, stream);
+  if (e != cudaSuccess) return e;
   combine_linear<D><<<dim3(BH, (D * D + 1023) / 1024), 256, 0, stream>>>(
       p.M_in, p.Bbuf, p.dz, Mp, p.z_pref, p.M_out, p.z_out, p.T);
   return cudaGetLastError();
@@ -828,7 +925,8 @@ void tc_scan_workspace(int B, int H_kv, int T, int d, bool delta, size_t* g_byte
   const size_t slices = (size_t)T * B * H_kv;
   *g_bytes = delta ? slices * d * d * 4 : 0;
   *b_bytes = slices * d * d * 4;
-  *dz_bytes = slices * d * 4;
+  // The delta rule's column sums come in up to kZChunksMax chunk partials.
+  *dz_bytes = slices * d * 4 * (delta ? kZChunksMax : 1);
 }
 
 cudaError_t launch_tc_state_scan(const Problem& p, cudaStream_t stream) {
