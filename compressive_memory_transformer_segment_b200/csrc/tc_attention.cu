@@ -697,6 +697,10 @@ bool tc_attention_supported(int d_k, int d_v, int S, bool bf16) {
 }
 
 cudaError_t launch_tc_attention(const Problem& p, cudaStream_t stream) {
+  // With one query head per KV head, a work item would pair tiles qt and
+  // qt - 1 of one head and one slot would idle for a tile of every item; the
+  // one-tile-per-CTA kernel (two CTAs per SM) is faster there.
+  if (p.H_q == p.H_kv) return launch_tc_attention_single(p, stream);
   if (p.d_k == 128) return launch<128>(p, stream);
   if (p.d_k == 64) return launch<64>(p, stream);
   return cudaErrorInvalidValue;
