@@ -67,6 +67,7 @@ _SIGNATURES = [
                                                 ctypes.POINTER(ctypes.c_int), ctypes.c_int,
                                                 ctypes.c_int]),
     ("infini_attn_selftest_approx", ctypes.c_int, [_P, _P, _P, _P, ctypes.c_int, _P]),
+    ("infini_attn_selftest_timeout", ctypes.c_int, [_P]),
     ("infini_attn_forward_noalloc", ctypes.c_int, [_P, _P, _P, _P, _P, _P, ctypes.c_int,
                                                    ctypes.c_int, ctypes.POINTER(Dims), _P, _P, _P,
                                                    _P]),
@@ -289,3 +290,10 @@ def selftest_approx(x, stream=None):
         _dev(x, "x", torch.float32), _dev(y_poly, "y_poly"), _dev(y_mufu, "y_mufu"),
         _dev(bits, "bits"), x.numel(), _stream_handle(stream)))
     return y_poly, y_mufu, bits
+
+
+def selftest_timeout(stream=None):
+    """Enqueue the bounded-wait failure-path self-check (one warp whose wait
+    on a barrier nothing arrives at gives up after ~2 s and sets the device
+    status word); a following sync_status raises InfiniError(ERR_TIMEOUT)."""
+    _check(load_library().infini_attn_selftest_timeout(_stream_handle(stream)))

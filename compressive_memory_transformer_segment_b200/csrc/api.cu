@@ -143,6 +143,9 @@ unsigned int* status_ptr() {
 }
 
 }  // namespace
+
+unsigned int* device_status_word() { return status_ptr(); }
+
 }  // namespace infini
 
 using namespace infini;

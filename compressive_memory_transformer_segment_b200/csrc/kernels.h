@@ -38,6 +38,9 @@ cudaError_t launch_simt_attention(const Problem& p, cudaStream_t stream);
 // Tensor-core (tcgen05 / TMEM / TMA) segment attention: bf16 I/O,
 // d_k == d_v in {64, 128}, S a multiple of 128.  Reads bf16 M_pref.
 bool tc_attention_supported(int d_k, int d_v, int S, bool bf16);
+// Device address of the status word the kernels set (see common.cuh).
+unsigned int* device_status_word();
+
 cudaError_t launch_tc_attention(const Problem& p, cudaStream_t stream);
 // The one-query-tile-per-CTA variant (used when H_q == H_kv).
 cudaError_t launch_tc_attention_single(const Problem& p, cudaStream_t stream);

@@ -233,10 +233,20 @@ INFINI_API size_t infini_attn_noalloc_scratch_limit(void);
  *                  below -125 are clamped to -125),
  *   y_mufu[i]    = the hardware 2^x approximation (subnormal results -> 0),
  *   bf16_bits[i] = bf16 bits of |x[i]| as the kernel packs probabilities
- *                  (round half up; ties differ from round-to-nearest-even).
+ *                  (round to nearest even).
  * Enqueued on `stream`.  Errors: INFINI_ERR_ARG, INFINI_ERR_CUDA. */
 INFINI_API int infini_attn_selftest_approx(const float* x, float* y_poly, float* y_mufu,
                                            unsigned int* bf16_bits, int n, void* stream);
+
+/* Self-check of the failure path of the tensor-core kernels' bounded waits (a
+ * testing aid; the method has no counterpart).  Enqueues on `stream` one warp
+ * that waits, through the same bounded mbarrier wait the kernels use, on a
+ * barrier nothing ever arrives at: the wait gives up after its time limit
+ * (2 s of %globaltimer), sets the timeout bit of the device status word and
+ * the kernel returns normally -- no fault, the context stays usable.  A
+ * following infini_attn_sync_status(stream) reports INFINI_ERR_TIMEOUT and
+ * clears the word.  Errors: INFINI_ERR_CUDA (launch failed). */
+INFINI_API int infini_attn_selftest_timeout(void* stream);
 
 #ifdef __cplusplus
 }

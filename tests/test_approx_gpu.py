@@ -42,3 +42,18 @@ def test_probability_packing_is_bf16_rounding(cuda_lib):
     _, _, tb = api.selftest_approx(ties.cuda())
     got_t = tb.cpu().numpy().astype(np.uint32) << 16
     np.testing.assert_array_equal(got_t.view(np.float32), np.array([1.0, 1 + 2.0 ** -6], np.float32))
+
+
+def test_bounded_wait_timeout_sets_status_and_context_survives(cuda_lib):
+    """The kernels' bounded mbarrier wait, made to run out on purpose (a
+    barrier nothing arrives at): the kernel returns, the status word reports
+    the timeout once, and the context keeps working."""
+    api = cuda_lib
+    api.sync_status()  # start clean
+    api.selftest_timeout()
+    with pytest.raises(api.InfiniError) as e:
+        api.sync_status()
+    assert e.value.status == api.ERR_TIMEOUT
+    api.sync_status()  # the word was cleared
+    y, _, _ = api.selftest_approx(torch.tensor([0.0, 1.0, -1.0], device="cuda"))
+    assert torch.allclose(y.cpu(), torch.tensor([1.0, 2.0, 0.5]), rtol=1e-4)
