@@ -410,12 +410,17 @@ tc_segment_products(const __grid_constant__ CUtensorMap tm_k, const __grid_const
 // The linear rule is HBM-bound (each block brings 32 KiB of K and V); the
 // delta rule does 20 MMAs (128 x 128 x 16) per block.
 constexpr int kLTok = 64;      // tokens per block
-constexpr int kLMath = 8;      // math warps
-constexpr int kLThreads = 64 + 32 * kLMath;
 
 template <bool DELTA>
 struct PipeSmem {
   static constexpr int kD = 128;
+  // Math warps: 16 for the linear rule (2 tokens per thread and block, to
+  // hide the latency of the sigma chain), 8 for the delta rule (its thread
+  // state needs the registers).
+  static constexpr int kMath = DELTA ? 8 : 16;
+  static constexpr int kThreads = 64 + 32 * kMath;
+  static constexpr int kTL = 2 * kMath;                   // token lanes
+  static constexpr int kTokPerThread = kLTok / kTL;
   static constexpr int kStages = DELTA ? 2 : 4;          // K/V ring depth
   static constexpr int kPanel = kLTok * 128;              // 64 rows x 128 B
   static constexpr int kHalf = kLTok * kD * 2;            // one 64 x 128 bf16 block
@@ -423,8 +428,8 @@ struct PipeSmem {
   static constexpr int kOpParts = DELTA ? 4 : 2;          // sigma hi, lo (, Y hi, lo)
   static constexpr int kRing = 0;
   static constexpr int kOp = kRing + kStages * kStage;    // [2][parts]
-  static constexpr int kRed = kOp + 2 * kOpParts * kHalf; // dz partials fp32 [16][128]
-  static constexpr int kZ = kRed + (DELTA ? 0 : 16 * kD * 4);  // z_{s-1} fp32 [128] (delta)
+  static constexpr int kRed = kOp + 2 * kOpParts * kHalf; // dz partials fp32 [kTL][128]
+  static constexpr int kZ = kRed + (DELTA ? 0 : kTL * kD * 4);  // z_{s-1} fp32 [128] (delta)
   static constexpr int kBar = kZ + (DELTA ? kD * 4 : 0);
   // full[kStages] empty[kStages] op_full[2] op_empty[2] acc_full red_ready
   static constexpr int kNumBars = 2 * kStages + 6;
@@ -435,13 +440,17 @@ struct PipeSmem {
 };
 
 template <bool DELTA>
-__global__ void __launch_bounds__(kLThreads, 1)
+__global__ void __launch_bounds__(PipeSmem<DELTA>::kThreads, 1)
 tc_pipe_products(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                  const float* __restrict__ z_pref, float* __restrict__ Gbuf, float* __restrict__ Bbuf,
                  float* __restrict__ dz, unsigned int* __restrict__ status, int L, int S) {
   using SM = PipeSmem<DELTA>;
   constexpr int D = SM::kD;
   constexpr int kStages = SM::kStages;
+  constexpr int kLMath = SM::kMath;
+  constexpr int kLThreads = SM::kThreads;
+  constexpr int kTL = SM::kTL;
+  constexpr int kTPT = SM::kTokPerThread;
   const int s = blockIdx.x, bh = blockIdx.y, BH = gridDim.y;
   const int seg0 = s * S, seg_len = min(S, L - seg0);
   const int nblk = (seg_len + kLTok - 1) / kLTok;
@@ -552,8 +561,9 @@ tc_pipe_products(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
     __syncwarp();
   } else {
     // ---------------------------------------------- math warps
-    // Thread (column chunk cg of 8 columns, token lane tl): tokens tl, tl+16,
-    // ...; the 16 threads of a token are lanes 0..15 or 16..31 of one warp.
+    // Thread (column chunk cg of 8 columns, token lane tl): tokens tl,
+    // tl + kTL, ...; the 16 threads of a token are lanes 0..15 or 16..31 of
+    // one warp.
     const int mt = threadIdx.x - 64;
     const int cg = mt & 15, tl = mt >> 4;
     float acc[8];
@@ -570,10 +580,10 @@ tc_pipe_products(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
       ok = __all_sync(0xffffffffu, mbar_wait(full + st, (uint32_t)(b / kStages) & 1u, abort, status));
       if (!ok) break;
       const unsigned char* kb = ring + st * SM::kStage;
-      uint4 hi4[kLTok / 16], lo4[kLTok / 16], yh4[kLTok / 16], yl4[kLTok / 16];
+      uint4 hi4[kTPT], lo4[kTPT], yh4[kTPT], yl4[kTPT];
 #pragma unroll
-      for (int i = 0; i < kLTok / 16; ++i) {
-        const int t = tl + 16 * i;
+      for (int i = 0; i < kTPT; ++i) {
+        const int t = tl + kTL * i;
         const bool valid = b * kLTok + t < seg_len;
         const uint32_t off = sw128_offset(t, 8 * cg, kLTok);
         const uint4 kv = *reinterpret_cast<const uint4*>(kb + off);
@@ -619,8 +629,8 @@ tc_pipe_products(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
       if (!ok) break;
       unsigned char* hb = op + ob * SM::kOpParts * SM::kHalf;
 #pragma unroll
-      for (int i = 0; i < kLTok / 16; ++i) {
-        const uint32_t off = sw128_offset(tl + 16 * i, 8 * cg, kLTok);
+      for (int i = 0; i < kTPT; ++i) {
+        const uint32_t off = sw128_offset(tl + kTL * i, 8 * cg, kLTok);
         *reinterpret_cast<uint4*>(hb + off) = hi4[i];
         *reinterpret_cast<uint4*>(hb + SM::kHalf + off) = lo4[i];
         if (DELTA) {
@@ -633,7 +643,7 @@ tc_pipe_products(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
       if (lane == 0) mbar_arrive(op_full + ob);
     }
     if (!DELTA) {
-      // dz: the 16 token lanes' partial column sums, reduced in shared memory.
+      // dz: the token lanes' partial column sums, reduced in shared memory.
 #pragma unroll
       for (int i = 0; i < 8; ++i) red[tl * D + 8 * cg + i] = acc[i];
       __syncwarp();
@@ -642,12 +652,13 @@ tc_pipe_products(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
       if (ok && mt < D) {
         float sum = 0.f;
 #pragma unroll
-        for (int j = 0; j < 16; ++j) sum += red[j * D + mt];
+        for (int j = 0; j < kTL; ++j) sum += red[j * D + mt];
         dz[slice * D + mt] = sum;
       }
     }
-    // The products: TMEM lane k = row k.  Linear: the two warps of a lane
-    // quarter take 64 columns of B each; delta: one takes G, the other B.
+    // The products: TMEM lane k = row k.  Linear: the kMath / 4 warps of a
+    // lane quarter share the 128 columns of B; delta: one takes G, the
+    // other B.
     if (ok) ok = __all_sync(0xffffffffu, mbar_wait(acc_full, 0, abort, status));
     if (ok) {
       tc_fence_after();
@@ -669,16 +680,19 @@ tc_pipe_products(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
                                  __uint_as_float(v[4 * i + 2]), __uint_as_float(v[4 * i + 3]));
         }
       } else {
-        const uint32_t ta = tB + lq + 64 * half;
-        uint32_t v[64];
-        tmem_ld32(ta, v);
-        tmem_ld32(ta + 32, v + 32);
-        tmem_wait_ld();
-        float4* dst = reinterpret_cast<float4*>(Bbuf + (slice * D + k) * D + 64 * half);
+        constexpr int kCols = 4 * D / kLMath;  // columns per warp
+        const uint32_t ta = tB + lq + kCols * half;
+        float4* dst = reinterpret_cast<float4*>(Bbuf + (slice * D + k) * D + kCols * half);
 #pragma unroll
-        for (int i = 0; i < 16; ++i)
-          dst[i] = make_float4(__uint_as_float(v[4 * i]), __uint_as_float(v[4 * i + 1]),
-                               __uint_as_float(v[4 * i + 2]), __uint_as_float(v[4 * i + 3]));
+        for (int c = 0; c < kCols / 32; ++c) {
+          uint32_t v[32];
+          tmem_ld32(ta + 32 * c, v);
+          tmem_wait_ld();
+#pragma unroll
+          for (int i = 0; i < 8; ++i)
+            dst[8 * c + i] = make_float4(__uint_as_float(v[4 * i]), __uint_as_float(v[4 * i + 1]),
+                                         __uint_as_float(v[4 * i + 2]), __uint_as_float(v[4 * i + 3]));
+        }
       }
     }
   }
@@ -869,8 +883,8 @@ cudaError_t launch_pipe_products(const Problem& p, cudaStream_t stream) {
   auto kern = tc_pipe_products<DELTA>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
-  kern<<<dim3(p.T, (unsigned)BHkv), kLThreads, smem, stream>>>(lk, lv, p.z_pref, p.Gbuf, p.Bbuf, p.dz,
-                                                               p.status, p.L, p.S);
+  kern<<<dim3(p.T, (unsigned)BHkv), PipeSmem<DELTA>::kThreads, smem, stream>>>(
+      lk, lv, p.z_pref, p.Gbuf, p.Bbuf, p.dz, p.status, p.L, p.S);
   return cudaGetLastError();
 }
 
