@@ -420,6 +420,9 @@ def run_gpu(args, w):
         "config": config_dict(w, world, l2_note),
         "path": plan["path"],
         "tc_peak_frac_step": (flops / (step_ms / 1000.0)) / (peak * 1e12),
+        # The step's algorithmic bytes (q, k, v read once, out written once,
+        # M/z in and out) against the measured HBM copy bandwidth.
+        "hbm_frac_step": (configs.algorithmic_bytes(w) / (step_ms / 1000.0)) / (peaks["hbm_gbs"] * 1e9),
         "clocks": clocks.summary(),
         "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "steps": e2e_steps},

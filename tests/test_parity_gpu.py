@@ -325,3 +325,36 @@ def test_tensor_core_path_split_stream(cuda_lib):
     api.sync_status()
     assert torch.max(torch.abs(torch.cat([o1, o2], 2).float() - out_full.float())) <= 2e-2
     assert torch.allclose(M, M_full, rtol=1e-5, atol=1e-4)
+
+
+def test_linear_rule_tokens_per_second_does_not_fall_with_length(cuda_lib):
+    """The per-token cost is O(S) at fixed S and d: at the 1M-token shape
+    (32 heads, d = 128, S = 2048, linear rule) a 1M-token forward keeps at least
+    the throughput of a 64K-token slice (device time, CUDA events)."""
+    api = cuda_lib
+    dev = torch.device("cuda", 0)
+    g = torch.Generator(device=dev).manual_seed(7)
+
+    def tokens_per_s(L, reps):
+        q = torch.randn(1, 32, L, 128, device=dev, generator=g).to(torch.bfloat16)
+        k = torch.randn(1, 32, L, 128, device=dev, generator=g).to(torch.bfloat16)
+        v = torch.randn(1, 32, L, 128, device=dev, generator=g).to(torch.bfloat16)
+        beta = torch.zeros(32, device=dev)
+        M, z = api.init_state(1, 32, 128, 128)
+        dims = api.make_dims(1, 32, 32, L, 128, 128, torch.bfloat16)
+        ws = torch.empty(api.workspace_bytes(dims, 2048, "linear"), dtype=torch.uint8, device=dev)
+        out = torch.empty_like(q)
+        Mo, zo = torch.empty_like(M), torch.empty_like(z)
+        for _ in range(2):
+            api.forward(q, k, v, beta, M, z, 2048, "linear", out, Mo, zo, ws)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(reps):
+            api.forward(q, k, v, beta, M, z, 2048, "linear", out, Mo, zo, ws)
+        e1.record()
+        api.sync_status()
+        return L * reps / (e0.elapsed_time(e1) / 1e3)
+
+    small = tokens_per_s(65536, 8)
+    large = tokens_per_s(1 << 20, 2)
+    assert large >= 0.8 * small, (small, large)
