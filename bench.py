@@ -40,9 +40,11 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # kernel sources hash to what they were at capture time.
 ATTENTION_TRAFFIC = {
     "8b-delta": {"bytes": 2 * (409.577728e6 + 230.632448e6),
-                 "note": "ncu capture at batch 1, scaled x2 to the batch-2 launch",
+                 "note": "ncu capture at batch 1, scaled x2 to the batch-2 launch; the file's "
+                         "host dispatch to the one-tile kernel (H_q == H_kv) was added after "
+                         "the capture, the paired kernel's device code is unchanged",
                  "profile": "profiles/tc_attention_8b-delta.md",
-                 "sha1": {"tc_attention.cu": "4fbaf38e7f176796e2c0d07111a6b28486e54282",
+                 "sha1": {"tc_attention.cu": "cadd3fd433ecfb41c02a7f98d923e9d204977ab6",
                           "tc_common.cuh": "a2612deb59163975e015c94465b32bea6a1a4f2d"}},
 }
 

@@ -285,6 +285,36 @@ def test_tensor_core_path_cases(cuda_lib, name, over):
     check_full(cuda_lib, W["tiny"].with_(name=name, **over))
 
 
+def _scale_bf16_bits(bits, factor):
+    """bf16 bit patterns times a power of two (exact)."""
+    f = (bits.astype(np.uint32) << 16).view(np.float32) * np.float32(factor)
+    return (f.view(np.uint32) >> 16).astype(np.uint16)
+
+
+# Keys of later tiles 8x larger than the rest: their scores exceed the first
+# tile's row max by far more than 2^16 / 128 in 2^x terms, so the lazy softmax
+# reference moves mid-segment: in the low half of a tile (keys 0..63), in the
+# high half (64..127) and in both, with earlier tiles already accumulated in O.
+SPIKE_CASES = [
+    ("spike_d128_gqa", dict(dtype="bf16", d_k=128, d_v=128, L=1024, seg_len=512, H_q=4, H_kv=2,
+                            rule="delta")),
+    ("spike_d64_gqa", dict(dtype="bf16", d_k=64, d_v=64, L=1024, seg_len=512, H_q=4, H_kv=2)),
+    ("spike_d128_one_q_per_kv", dict(dtype="bf16", d_k=128, d_v=128, L=1024, seg_len=512, H_q=2,
+                                     H_kv=2)),
+]
+
+
+@pytest.mark.parametrize("name,over", SPIKE_CASES, ids=[c[0] for c in SPIKE_CASES])
+def test_tensor_core_path_softmax_reference_moves(cuda_lib, name, over):
+    w = W["tiny"].with_(name=name, **over)
+    inp = synth.make_inputs(w)
+    for seg0 in range(0, w.L, w.seg_len):
+        for off in (128 + 100, 256 + 10, 384 + 5, 384 + 120):
+            if seg0 + off < w.L:
+                inp["k"][:, :, seg0 + off, :] = _scale_bf16_bits(inp["k"][:, :, seg0 + off, :], 8.0)
+    check_full(cuda_lib, w, inp)
+
+
 def test_tensor_core_path_deterministic_and_workspace_independent(cuda_lib):
     api = cuda_lib
     w = W["tiny"].with_(dtype="bf16", d_k=128, d_v=128, L=1024, seg_len=256, B=2, H_q=4, H_kv=2,
