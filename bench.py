@@ -42,9 +42,10 @@ ATTENTION_TRAFFIC = {
     "8b-delta": {"bytes": 2 * (409.577728e6 + 230.632448e6),
                  "note": "ncu capture at batch 1, scaled x2 to the batch-2 launch; the file's "
                          "host dispatch to the one-tile kernel (H_q == H_kv) was added after "
-                         "the capture, the paired kernel's device code is unchanged",
+                         "the capture and the header comment rewritten; the paired kernel's "
+                         "device code is unchanged",
                  "profile": "profiles/tc_attention_8b-delta.md",
-                 "sha1": {"tc_attention.cu": "cadd3fd433ecfb41c02a7f98d923e9d204977ab6",
+                 "sha1": {"tc_attention.cu": "8054f13e63ddfd60411415ae0c937af5bf12fe6f",
                           "tc_common.cuh": "a2612deb59163975e015c94465b32bea6a1a4f2d"}},
 }
 

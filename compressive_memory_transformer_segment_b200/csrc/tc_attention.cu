@@ -22,21 +22,22 @@
 //
 // Roles (384 threads, three warpgroups; the first gives registers to the
 // other two with setmaxnreg):
-//   warp 0      TMA producer: per item K_0, V_0, the two Q tiles, K_1, V_1,
-//               ..., then M_{s-1}, through a ring of shared-memory slots; an
-//               L2 prefetch of the next item's Q tiles.
+//   warp 0      TMA producer: per item K_0, V_0, the next item's two Q
+//               tiles (double-buffered), K_1, V_1, ..., then M_{s-1}, through
+//               a ring of shared-memory slots.
 //   warp 1      allocates TMEM; one thread issues every tcgen05.mma with the
 //               operand descriptors precomputed per group of MMAs:
 //               S_j = Q K_j^T, O += P_j V_j (P read from TMEM), and at the end
-//               of the item R = sigma(Q) M_{s-1} into the score columns.
+//               of the item R = sigma(Q) M_{s-1} into the score columns.  A
+//               slot's P.V and next QK^T go back to back (16 MMAs at d = 128).
 //   warps 2, 3  idle.
 //   warps 4..7  slot A, warps 8..11 slot B: one thread per query row.  Online
-//               softmax in base 2 on the scores in TMEM (row max first, with a
-//               three-input max; the running max moves, and O is rescaled,
-//               only when the tile max exceeds it by more than 2^8); P (bf16)
-//               written over the scores; then sigma(Q) in place of Q with the
-//               fp32 retrieval denominator sigma(q).z, and the gated output
-//               stored from registers.
+//               softmax in base 2 on the scores in TMEM (the first tile's row
+//               max is the reference; it moves, and O is rescaled, only when
+//               a tile's sum exceeds 2^16); P (bf16) written over the scores;
+//               then sigma(Q) in place of Q with the fp32 retrieval
+//               denominator sigma(q).z, and the gated output stored from
+//               registers.
 // TMEM (512 columns): slot A S = [0, 128), O = [128, 128 + D);
 //                     slot B S = [256, 384), O = [384, 384 + D).
 #include <cuda.h>
