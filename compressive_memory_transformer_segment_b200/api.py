@@ -57,6 +57,8 @@ _SIGNATURES = [
                                         ctypes.POINTER(Plan)]),
     ("infini_attn_forward", ctypes.c_int, [_P, _P, _P, _P, _P, _P, ctypes.c_int, ctypes.c_int,
                                            ctypes.POINTER(Dims), _P, _P, _P, _P, ctypes.c_size_t, _P]),
+    ("infini_attn_state_update", ctypes.c_int, [_P, _P, _P, _P, ctypes.c_int, ctypes.c_int,
+                                                ctypes.POINTER(Dims), _P, _P, _P, ctypes.c_size_t, _P]),
     ("infini_attn_host_arena_bytes", ctypes.c_size_t, [ctypes.POINTER(Dims), ctypes.c_int, ctypes.c_int]),
     ("infini_attn_forward_host", ctypes.c_int, [_P, _P, _P, _P, _P, _P, ctypes.c_int, ctypes.c_int,
                                                 ctypes.POINTER(Dims), _P, _P, _P, _P,
@@ -199,6 +201,40 @@ def forward(q, k, v, beta, M_in, z_in, seg_len, rule, out=None, M_out=None, z_ou
     _check(lib.infini_attn_forward(*args, int(seg_len), _rule(rule), ctypes.byref(dims), *outs,
                                    ws_ptr, ws_n, _stream_handle(stream)))
     return out, M_out, z_out
+
+
+def state_update(k, v, M_in, z_in, seg_len, rule, M_out=None, z_out=None, workspace=None,
+                 stream=None):
+    """infini_attn_state_update on CUDA tensors: the state after the segments
+    of k, v from (M_in, z_in); returns (M_out, z_out).  ``workspace``: an
+    optional uint8 CUDA tensor of workspace_bytes(make_dims(B, H_kv, H_kv, L,
+    d_k, d_v, dtype), seg_len, rule) bytes or more."""
+    lib = load_library()
+    if k.dim() != 4 or v.dim() != 4:
+        raise ValueError("k and v must be [B, H_kv, L, d]")
+    B, H_kv, L, d_k = k.shape
+    d_v = v.shape[3]
+    if tuple(v.shape[:3]) != (B, H_kv, L) or v.dtype != k.dtype:
+        raise ValueError("v must match k in batch, heads, length and dtype")
+    if k.dtype not in DTYPES:
+        raise ValueError("k, v must be bfloat16 or float32")
+    dims = make_dims(B, H_kv, H_kv, L, d_k, d_v, k.dtype)
+    if M_out is None:
+        M_out = torch.empty((B, H_kv, d_k, d_v), dtype=torch.float32, device=k.device)
+    if z_out is None:
+        z_out = torch.empty((B, H_kv, d_k), dtype=torch.float32, device=k.device)
+    args = [_dev(k, "k"), _dev(v, "v"),
+            _dev(M_in, "M_in", torch.float32, (B, H_kv, d_k, d_v)),
+            _dev(z_in, "z_in", torch.float32, (B, H_kv, d_k))]
+    outs = [_dev(M_out, "M_out", torch.float32, (B, H_kv, d_k, d_v)),
+            _dev(z_out, "z_out", torch.float32, (B, H_kv, d_k))]
+    if workspace is not None:
+        ws_ptr, ws_n = _dev(workspace, "workspace", torch.uint8), workspace.numel()
+    else:
+        ws_ptr, ws_n = ctypes.c_void_p(0), 0
+    _check(lib.infini_attn_state_update(*args, int(seg_len), _rule(rule), ctypes.byref(dims), *outs,
+                                        ws_ptr, ws_n, _stream_handle(stream)))
+    return M_out, z_out
 
 
 def host_arena_bytes(dims, seg_len, rule):

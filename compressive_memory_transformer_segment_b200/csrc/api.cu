@@ -272,6 +272,72 @@ int infini_attn_forward(const void* q, const void* k, const void* v, const float
   return e == cudaSuccess ? INFINI_OK : INFINI_ERR_CUDA;
 }
 
+int infini_attn_state_update(const void* k, const void* v, const float* M_in, const float* z_in,
+                             int seg_len, int rule, const infini_dims_t* dims, float* M_out,
+                             float* z_out, void* workspace, size_t workspace_bytes, void* stream) {
+  Shape s;
+  int rc = check_shape(dims, seg_len, rule, &s);
+  if (rc != INFINI_OK) return rc;
+  if (!k || !v || !M_in || !z_in || !M_out || !z_out) return INFINI_ERR_ARG;
+  const void* ptrs[] = {k, v, M_in, z_in, M_out, z_out};
+  for (const void* p : ptrs)
+    if (!aligned16(p)) return INFINI_ERR_ALIGN;
+  if (workspace == nullptr && workspace_bytes != 0) return INFINI_ERR_ARG;
+  if (workspace != nullptr) {
+    if (workspace_bytes < s.ws_total || ((uintptr_t)workspace & (kAlign - 1)) != 0)
+      return INFINI_ERR_WORKSPACE;
+  }
+  const Range r_M = rng(M_out, s.M_bytes), r_z = rng(z_out, s.z_bytes);
+  const Range ins[] = {rng(k, s.k_bytes), rng(v, s.v_bytes), rng(M_in, s.M_bytes), rng(z_in, s.z_bytes)};
+  for (int i = 0; i < 4; ++i) {
+    if (overlap(r_M, ins[i]) && !(i == 2 && M_out == M_in)) return INFINI_ERR_ALIAS;
+    if (overlap(r_z, ins[i]) && !(i == 3 && z_out == z_in)) return INFINI_ERR_ALIAS;
+  }
+  if (overlap(r_M, r_z)) return INFINI_ERR_ALIAS;
+  if (workspace) {
+    const Range r_ws = rng(workspace, s.ws_total);
+    if (overlap(r_ws, r_M) || overlap(r_ws, r_z)) return INFINI_ERR_ALIAS;
+    for (int i = 0; i < 4; ++i)
+      if (overlap(r_ws, ins[i])) return INFINI_ERR_ALIAS;
+  }
+
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  unsigned int* status = status_ptr();
+  if (!status) return INFINI_ERR_CUDA;
+  char* ws = static_cast<char*>(workspace);
+  bool owned = false;
+  if (!ws) {
+    if (cudaMallocAsync(reinterpret_cast<void**>(&ws), s.ws_total, st) != cudaSuccess)
+      return INFINI_ERR_CUDA;
+    owned = true;
+  }
+  // The scan of infini_attn_forward alone: it reads k, v and the state, and
+  // writes the per-segment states to the workspace and (M_out, z_out).
+  Problem p;
+  p.q = nullptr; p.k = k; p.v = v; p.beta = nullptr; p.M_in = M_in;
+  p.out = nullptr; p.M_out = M_out; p.z_out = z_out;
+  p.B = s.B; p.H_q = s.H_q; p.H_kv = s.H_kv; p.L = s.L; p.d_k = s.d_k; p.d_v = s.d_v;
+  p.S = s.S; p.T = s.T; p.bf16 = s.bf16; p.delta = s.delta;
+  p.z_pref = reinterpret_cast<float*>(ws + s.ws_zpref);
+  p.M_pref = ws + s.ws_mpref;
+  p.M_pref_bf16 = s.path == INFINI_PATH_TCGEN05;
+  p.Gbuf = reinterpret_cast<float*>(ws + s.ws_g);
+  p.Bbuf = reinterpret_cast<float*>(ws + s.ws_b);
+  p.dz = reinterpret_cast<float*>(ws + s.ws_dz);
+  p.status = status;
+
+  cudaError_t e = cudaMemcpyAsync(p.z_pref, z_in, s.z_bytes, cudaMemcpyDeviceToDevice, st);
+  if (e == cudaSuccess)
+    e = timed(0, st, [&] {
+      return s.path == INFINI_PATH_TCGEN05 ? launch_tc_state_scan(p, st) : launch_simt_state_scan(p, st);
+    });
+  if (owned) {
+    cudaError_t f = cudaFreeAsync(ws, st);
+    if (e == cudaSuccess) e = f;
+  }
+  return e == cudaSuccess ? INFINI_OK : INFINI_ERR_CUDA;
+}
+
 size_t infini_attn_host_arena_bytes(const infini_dims_t* dims, int seg_len, int rule) {
   Shape s;
   if (check_shape(dims, seg_len, rule, &s) != INFINI_OK) return 0;

@@ -8,6 +8,18 @@ range of batch rows (whole rows keep every GQA group and every segment chain
 together), runs the forward on its own GPU, and results are assembled by
 concatenation.  The only collectives are for timing (max over ranks) and,
 when a caller wants the full result on one rank, a gather.
+
+Sequence parallelism for the linear rule.  Under the linear rule the memory
+after a run of segments is the memory before it plus a sum over the run's
+tokens ("Hugging Face Infini-Attention 再現分析", Memory Update: the
+outer-product contributions accumulate; z is the running sum of sigma(K)).
+So a sequence cut at segment boundaries into one contiguous run per rank
+needs one exchange: every rank computes its run's update from a zero state,
+the updates are all-gathered, each rank adds those of the ranks before it to
+the initial state (an exclusive prefix, in rank order, so every rank forms
+the same sums) and then runs the forward over its own segments from there.
+The delta rule's update depends on the memory it starts from, so it stays
+sequential in the segments and is sharded by batch rows only.
 """
 
 import torch
@@ -46,3 +58,75 @@ def max_over_ranks(value, device=None, group=None):
     if dist.is_available() and dist.is_initialized() and dist.get_world_size(group) > 1:
         dist.all_reduce(t, op=dist.ReduceOp.MAX, group=group)
     return float(t.item())
+
+
+def segment_range(L, S, world, rank):
+    """Token rows [l0, l1) of `rank`'s contiguous run of whole segments (a
+    near-equal split of the T = ceil(L / S) segments; only the last run may
+    end in the shorter final segment, and a run may be empty)."""
+    if S < 1 or L < 1:
+        raise ValueError("bad L/S")
+    T = -(-L // S)
+    s0, s1 = batch_range(T, world, rank)
+    return min(s0 * S, L), min(s1 * S, L)
+
+
+def local_state_update(k, v, seg_len, state_update, dtype=torch.float32):
+    """This rank's linear-rule update from a zero state, packed flat:
+    [dM (B*H_kv*d_k*d_v), dz (B*H_kv*d_k)] in the state's dtype (float32 for
+    the library).  `state_update` is the library call
+    (k, v, M_in, z_in, seg_len, rule) -> (M_out, z_out)."""
+    B, H_kv, L, d_k = k.shape
+    d_v = v.shape[3]
+    M0 = torch.zeros((B, H_kv, d_k, d_v), dtype=dtype, device=k.device)
+    z0 = torch.zeros((B, H_kv, d_k), dtype=dtype, device=k.device)
+    if L == 0:
+        return torch.cat([M0.flatten(), z0.flatten()])
+    dM, dz = state_update(k, v, M0, z0, seg_len, "linear")
+    return torch.cat([dM.flatten(), dz.flatten()])
+
+
+def prefix_states(updates, rank, M0, z0):
+    """(M_in, z_in) of `rank` and the final (M_T, z_T) from the gathered
+    per-rank updates (a list in rank order): M0 plus the updates of ranks
+    before `rank`, and plus all of them, added one rank at a time in float32."""
+    nM = M0.numel()
+    M_in, z_in = M0.clone(), z0.clone()
+    M_T, z_T = M0.clone(), z0.clone()
+    for r, u in enumerate(updates):
+        dM = u[:nM].view_as(M0)
+        dz = u[nM:].view_as(z0)
+        if r < rank:
+            M_in += dM
+            z_in += dz
+        M_T += dM
+        z_T += dz
+    return M_in, z_in, M_T, z_T
+
+
+def all_gather_flat(t, group=None):
+    """All-gather equal-size flat tensors, in rank order (one rank: [t])."""
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size(group) == 1:
+        return [t]
+    parts = [torch.empty_like(t) for _ in range(dist.get_world_size(group))]
+    dist.all_gather(parts, t.contiguous(), group=group)
+    return parts
+
+
+def sequence_parallel_forward(q, k, v, beta, M0, z0, seg_len, forward, state_update, group=None):
+    """Linear-rule forward of this rank's run of segments.
+
+    q, k, v: the rank's token rows [l0, l1) from segment_range (B, heads and d
+    as for the whole sequence); M0, z0: the state before token 0.  `forward`
+    and `state_update` are the library calls (api.forward, api.state_update).
+    Returns (out for the rank's rows, M_T, z_T) with the state after the whole
+    sequence on every rank.  One all-gather of B * H_kv * (d_k d_v + d_k)
+    floats per rank is the only exchange.
+    """
+    updates = all_gather_flat(local_state_update(k, v, seg_len, state_update, M0.dtype), group)
+    rank = dist.get_rank(group) if dist.is_available() and dist.is_initialized() else 0
+    M_in, z_in, M_T, z_T = prefix_states(updates, rank, M0, z0)
+    if q.shape[2] == 0:
+        return q.new_empty(q.shape[:3] + (v.shape[3],)), M_T, z_T
+    out, _, _ = forward(q, k, v, beta, M_in, z_in, seg_len, "linear")
+    return out, M_T, z_T

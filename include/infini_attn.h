@@ -155,6 +155,31 @@ INFINI_API int infini_attn_forward(const void* q, const void* k, const void* v, 
                         const infini_dims_t* dims, void* out, float* M_out, float* z_out,
                         void* workspace, size_t workspace_bytes, void* stream);
 
+/* The memory update alone: (M_out, z_out) = the state after the T segments
+ * of k, v starting from (M_in, z_in), by `rule`, exactly as
+ * infini_attn_forward computes them, without the attention output.
+ * ("Hugging Face Infini-Attention 再現分析", Memory Update and State Transfer;
+ * "Leave No Context Behind" explainer, "メモリの更新".)
+ *   k, v             device, layouts above, element type dims->dtype
+ *   M_in, z_in       device float32 state read by the first segment
+ *   seg_len, rule    as for infini_attn_forward
+ *   dims             as for infini_attn_forward; only B, H_kv, L, d_k, d_v
+ *                    and dtype matter (H_q must still be a multiple of H_kv,
+ *                    e.g. H_q = H_kv)
+ *   M_out, z_out     device float32; may equal M_in / z_in (in place)
+ *   workspace        as for infini_attn_forward, of
+ *                    infini_attn_workspace_bytes(dims, seg_len, rule) bytes
+ *   stream           cudaStream_t.
+ * Under the linear rule the update is a sum over tokens, so the state of a
+ * sequence cut at segment boundaries is M_0 plus the pieces' updates from a
+ * zero state, added in order: the exchange step of a sequence-parallel
+ * forward (one all-gather of every rank's update, then an exclusive prefix).
+ * Errors: those of infini_attn_forward. */
+INFINI_API int infini_attn_state_update(const void* k, const void* v, const float* M_in,
+                                        const float* z_in, int seg_len, int rule,
+                                        const infini_dims_t* dims, float* M_out, float* z_out,
+                                        void* workspace, size_t workspace_bytes, void* stream);
+
 /* Bytes of device arena infini_attn_forward_host needs: room for q, k, v,
  * beta, M, z, out and the workspace, each 256-byte aligned.  0 if invalid. */
 INFINI_API size_t infini_attn_host_arena_bytes(const infini_dims_t* dims, int seg_len, int rule);

@@ -7,6 +7,7 @@ import os
 import socket
 
 import numpy as np
+import pytest
 import torch
 import torch.distributed as dist
 import torch.multiprocessing as mp
@@ -70,3 +71,99 @@ def test_two_rank_gloo_sharding_matches_single_process():
         assert ok
         assert mx == 11.0
     assert results[0][2] == (0, 2) and results[1][2] == (2, 3)
+
+
+# ------------------------------------------- sequence parallelism (linear rule)
+
+def _oracle_forward(q, k, v, beta, M_in, z_in, S, rule):
+    out, M, z = oracle.infini_attention_forward(q.numpy(), k.numpy(), v.numpy(), beta.numpy(),
+                                                M_in.numpy(), z_in.numpy(), S, rule)
+    return torch.from_numpy(out), torch.from_numpy(M), torch.from_numpy(z)
+
+
+def _oracle_state_update(k, v, M_in, z_in, S, rule):
+    B, H_kv, L, d_k = k.shape
+    q = torch.zeros((B, H_kv, L, d_k), dtype=torch.float64)
+    beta = torch.zeros(H_kv, dtype=torch.float64)
+    _, M, z = _oracle_forward(q, k, v, beta, M_in, z_in, S, rule)
+    return M, z
+
+
+def _sp_problem():
+    # 7 segments of 16 rows, the last one 4 rows; GQA; a nonzero initial state.
+    rng = np.random.default_rng(9)
+    B, H_q, H_kv, L, d, S = 2, 4, 2, 100, 8, 16
+    q = rng.standard_normal((B, H_q, L, d))
+    k = rng.standard_normal((B, H_kv, L, d))
+    v = rng.standard_normal((B, H_kv, L, d))
+    beta = rng.uniform(-3, 3, H_q)
+    M0 = rng.standard_normal((B, H_kv, d, d))
+    z0 = rng.uniform(0.5, 2.0, (B, H_kv, d))
+    return q, k, v, beta, M0, z0, S
+
+
+def _sp_worker(rank, world, port, results):
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        q, k, v, beta, M0, z0, S = _sp_problem()
+        L = q.shape[2]
+        l0, l1 = shard.segment_range(L, S, world, rank)
+        t = torch.from_numpy
+        out, M_T, z_T = shard.sequence_parallel_forward(
+            t(q[:, :, l0:l1].copy()), t(k[:, :, l0:l1].copy()), t(v[:, :, l0:l1].copy()), t(beta),
+            t(M0), t(z0), S, forward=_oracle_forward, state_update=_oracle_state_update)
+        ref_out, ref_M, ref_z = oracle.infini_attention_forward(q, k, v, beta, M0, z0, S, "linear")
+        results[rank] = ((l0, l1),
+                         float(np.max(np.abs(out.numpy() - ref_out[:, :, l0:l1]), initial=0.0)),
+                         float(np.max(np.abs(M_T.numpy() - ref_M))),
+                         float(np.max(np.abs(z_T.numpy() - ref_z))))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_segment_range_partition():
+    for L, S in ((100, 16), (64, 64), (1, 5), (1000, 128), (2048, 1)):
+        T = -(-L // S)
+        for world in (1, 2, 3, 4, 8):
+            rs = [shard.segment_range(L, S, world, r) for r in range(world)]
+            assert rs[0][0] == 0 and rs[-1][1] == L
+            assert all(rs[i][1] == rs[i + 1][0] for i in range(world - 1))
+            # whole segments: every cut sits on a segment boundary
+            assert all(a % S == 0 for a, _ in rs if a < L)
+            counts = [-(-(b - a) // S) for a, b in rs]
+            assert sum(counts) == T and max(counts) - min(counts) <= 1
+
+
+def test_prefix_states_in_rank_order():
+    M0 = torch.full((1, 1, 2, 2), 1.0, dtype=torch.float64)
+    z0 = torch.full((1, 1, 2), 2.0, dtype=torch.float64)
+    ups = [torch.cat([torch.full((4,), float(10 ** r)), torch.full((2,), float(r))]).double()
+           for r in range(3)]
+    M_in, z_in, M_T, z_T = shard.prefix_states(ups, 2, M0, z0)
+    assert torch.all(M_in == 12.0) and torch.all(z_in == 3.0)
+    assert torch.all(M_T == 112.0) and torch.all(z_T == 5.0)
+    M_in, z_in, _, _ = shard.prefix_states(ups, 0, M0, z0)
+    assert torch.equal(M_in, M0) and torch.equal(z_in, z0)
+
+
+@pytest.mark.parametrize("world", [2, 3])
+def test_sequence_parallel_linear_rule_gloo(world):
+    """Sequence cut into per-rank runs of whole segments, one all-gather of
+    the runs' state updates, exclusive prefix, then each rank's own forward:
+    the rank's rows of `out` and the final state equal the single-process
+    forward (float64 oracle as the per-rank compute)."""
+    port = _free_port()
+    ctx = mp.get_context("spawn")
+    results = ctx.Manager().dict()
+    mp.start_processes(_sp_worker, args=(world, port, results), nprocs=world, join=True,
+                       start_method="spawn")
+    assert sorted(results.keys()) == list(range(world))
+    covered = 0
+    for r in range(world):
+        (l0, l1), e_out, e_M, e_z = results[r]
+        assert l0 == covered
+        covered = l1
+        assert e_out <= 1e-12 and e_M <= 1e-12 and e_z <= 1e-12, (r, e_out, e_M, e_z)
+    assert covered == 100
