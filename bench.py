@@ -447,6 +447,161 @@ def run_gpu(args, w):
     return 0
 
 
+def decode_bytes_per_segment(w):
+    """Algorithmic HBM bytes of decoding one full segment (S steps, pos =
+    0..S-1): per KV head the buffer rows 0..pos (keys and values), M and z,
+    the new k_t, v_t read and written into the buffer; per query head q_t
+    read, out_t written and beta."""
+    e = 2 if w.dtype == "bf16" else 4
+    d, S = w.d_k, w.seg_len
+    rows = S * (S + 1) // 2  # sum over pos of (pos + 1)
+    per_kv = rows * 2 * d * e + S * (d * d * 4 + d * 4 + 4 * d * e)
+    per_q = S * (2 * d * e + 4)
+    return w.B * (w.H_kv * per_kv + w.H_q * per_q)
+
+
+def run_decode(args, w):
+    """Streaming decode: one token per (batch row, head) per call, `steps`
+    full segments of the workload's shape (S calls each; the state update
+    runs once per segment).  Single GPU."""
+    import torch
+
+    from compressive_memory_transformer_segment_b200 import api
+
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    api.load_library()
+    S = w.seg_len
+    ws_ = w.with_(L=2 * S)
+    inp = synth.make_inputs(ws_)
+    tdt = torch.bfloat16 if w.dtype == "bf16" else torch.float32
+
+    def dev_tensor(x):
+        if w.dtype == "bf16":
+            return torch.from_numpy(np.ascontiguousarray(x).view(np.int16)).view(torch.bfloat16).to(dev)
+        return torch.from_numpy(np.ascontiguousarray(x, dtype=np.float32)).to(dev)
+
+    q, k, v = (dev_tensor(inp[n]) for n in ("q", "k", "v"))
+    beta = torch.from_numpy(inp["beta"]).to(dev)
+    # A prior state (the memory after the first segment), then the second
+    # segment's tokens, each [B, heads, d] contiguous.
+    M0, z0 = api.init_state(w.B, w.H_kv, w.d_k, w.d_v, device=dev)
+    M0, z0 = api.state_update(k[:, :, :S].contiguous(), v[:, :, :S].contiguous(), M0, z0, S, w.rule)
+    qt = q[:, :, S:].permute(2, 0, 1, 3).contiguous()
+    kt = k[:, :, S:].permute(2, 0, 1, 3).contiguous()
+    vt = v[:, :, S:].permute(2, 0, 1, 3).contiguous()
+    st = api.DecodeStream(w.B, w.H_q, w.H_kv, w.d_k, S, w.rule, dtype=tdt, device=dev, M=M0, z=z0)
+    out = torch.empty((w.B, w.H_q, w.d_v), dtype=tdt, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def segment(strm):
+        for t in range(S):
+            st.step(qt[t], kt[t], vt[t], beta, out=out, stream=strm)
+
+    for _ in range(args.warmup):
+        segment(stream)
+    api.sync_status(stream)
+    # Eager calls with per-kernel CUDA events: the decode kernels' device time.
+    api.set_kernel_timing(True)
+    api.kernel_times(reset=True)
+    torch.cuda.synchronize(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    segment(stream)
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    eager_ms = e0.elapsed_time(e1)
+    api.set_kernel_timing(False)
+    ktimes = api.kernel_times(reset=True)
+    api.sync_status(stream)
+    # The timed steps: one CUDA graph per segment (its S calls and the state
+    # update), replayed, so that host launch overhead is not measured.
+    graph, graph_note = torch.cuda.CUDAGraph(), "each timed step replays one CUDA graph of the segment's calls"
+    try:
+        cap = torch.cuda.Stream(dev)
+        cap.wait_stream(stream)
+        with torch.cuda.graph(graph, stream=cap):
+            segment(cap)
+        stream.wait_stream(cap)
+        run = graph.replay
+    except Exception as exc:  # capture refused: time eager calls instead
+        torch.cuda.synchronize(dev)
+        graph_note = f"graph capture failed ({type(exc).__name__}); eager calls timed"
+        st.pos = 0
+
+        def run():
+            segment(stream)
+    for _ in range(args.warmup):
+        run()
+    api.sync_status(stream)
+    torch.cuda.synchronize(dev)
+    with ClockSampler(0) as clocks:
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(args.steps):
+            run()
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+    elapsed_ms = e0.elapsed_time(e1)
+    api.sync_status(stream)
+    tokens = w.B * S * args.steps
+    value = tokens / (elapsed_ms / 1000.0)
+
+    # End to end: each token's q_t, k_t, v_t copied from pinned host memory
+    # and out_t copied back, inside the timed region (one segment).
+    hq, hk, hv = (x.cpu().pin_memory() for x in (qt, kt, vt))
+    hout = torch.empty((S,) + tuple(out.shape), dtype=tdt).pin_memory()
+    dq, dk, dv = torch.empty_like(qt[0]), torch.empty_like(kt[0]), torch.empty_like(vt[0])
+    torch.cuda.synchronize(dev)
+    e2, e3 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e2.record(stream)
+    for t in range(S):
+        dq.copy_(hq[t], non_blocking=True)
+        dk.copy_(hk[t], non_blocking=True)
+        dv.copy_(hv[t], non_blocking=True)
+        st.step(dq, dk, dv, beta, out=out, stream=stream)
+        hout[t].copy_(out, non_blocking=True)
+    e3.record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_value = w.B * S / (e2.elapsed_time(e3) / 1000.0)
+
+    peaks, peak_src = load_peaks()
+    dec_ms, dec_n = ktimes["attention"]
+    scan_ms, scan_n = ktimes["state_scan"]
+    seg_bytes = decode_bytes_per_segment(w)
+    achieved = seg_bytes / (dec_ms / 1000.0) / 1e9
+    plan = api.plan(api.make_dims(w.B, w.H_q, w.H_kv, S, w.d_k, w.d_v, tdt), S, w.rule)
+    line = {
+        "metric": "Infini-attention streaming decode tokens/s on 1 B200 (one token per call)",
+        "value": value, "unit": "tokens/s", "n_gpus": 1, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": elapsed_ms / args.steps,
+        "step": f"one segment: {S} decode calls of one token per (batch row, head), "
+                "then the segment's state update",
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": w.dtype,
+        "data": "synthetic (seeded Philox N(0,1) q/k/v, U(-r,r) beta)",
+        "config": {"workload": f"{w.name} decode", "B": w.B, "H_q": w.H_q, "H_kv": w.H_kv,
+                   "d": w.d_k, "seg_len": S, "rule": w.rule, "io_dtype": w.dtype,
+                   "l2": "buffers and state stay in L2 between calls (as in serving)"},
+        "clocks": clocks.summary(),
+        "e2e": {"value": e2e_value, "unit": "tokens/s", "note": "eager calls, per-token copies",
+                "h2d_bytes_per_step": sum(x.numel() * x.element_size() for x in (hq, hk, hv)),
+                "d2h_bytes_per_step": hout.numel() * hout.element_size(), "steps": 1},
+        "gpu_launches": (2 * S + plan["launches"] - 1) * args.steps,
+        "roofline": {"bound": "hbm", "kernel": "decode attention (partial + combine)",
+                     "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                     "frac": achieved / peaks["hbm_gbs"], "peak_source": f"{peak_src} copy",
+                     "traffic": None,
+                     "algorithmic_bytes_per_step": seg_bytes,
+                     "avg_call_us": dec_ms * 1000.0 / max(dec_n, 1)},
+        "kernel_ms": {"decode_per_segment": dec_ms, "state_update_per_segment": scan_ms},
+        "eager_tokens_per_s": w.B * S / (eager_ms / 1000.0),
+        "graph": graph_note,
+        "cpu_baseline": None,
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -463,6 +618,9 @@ def main():
                     help="seconds of oracle work for the cpu_baseline sample")
     ap.add_argument("--reference-budget", type=float, default=60.0,
                     help="total seconds of oracle work for --impl reference")
+    ap.add_argument("--decode", action="store_true",
+                    help="streaming decode (one token per call) of the workload's shape; "
+                         "a step is one full segment")
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "ours":
         args.warmup = 3
@@ -471,6 +629,8 @@ def main():
         w = w.with_(B=args.batch, name=f"{w.name}-B{args.batch}")
     if args.impl == "reference":
         return run_reference(args, w)
+    if args.decode:
+        return run_decode(args, w)
     return run_gpu(args, w)
 
 

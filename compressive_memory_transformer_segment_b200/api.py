@@ -59,6 +59,11 @@ _SIGNATURES = [
                                            ctypes.POINTER(Dims), _P, _P, _P, _P, ctypes.c_size_t, _P]),
     ("infini_attn_state_update", ctypes.c_int, [_P, _P, _P, _P, ctypes.c_int, ctypes.c_int,
                                                 ctypes.POINTER(Dims), _P, _P, _P, ctypes.c_size_t, _P]),
+    ("infini_attn_decode_workspace_bytes", ctypes.c_size_t, [ctypes.POINTER(Dims), ctypes.c_int,
+                                                              ctypes.c_int]),
+    ("infini_attn_decode_step", ctypes.c_int, [_P, _P, _P, _P, _P, _P, ctypes.c_int, _P, _P,
+                                               ctypes.c_int, ctypes.c_int, ctypes.POINTER(Dims), _P,
+                                               _P, ctypes.c_size_t, _P]),
     ("infini_attn_host_arena_bytes", ctypes.c_size_t, [ctypes.POINTER(Dims), ctypes.c_int, ctypes.c_int]),
     ("infini_attn_forward_host", ctypes.c_int, [_P, _P, _P, _P, _P, _P, ctypes.c_int, ctypes.c_int,
                                                 ctypes.POINTER(Dims), _P, _P, _P, _P,
@@ -235,6 +240,74 @@ def state_update(k, v, M_in, z_in, seg_len, rule, M_out=None, z_out=None, worksp
     _check(lib.infini_attn_state_update(*args, int(seg_len), _rule(rule), ctypes.byref(dims), *outs,
                                         ws_ptr, ws_n, _stream_handle(stream)))
     return M_out, z_out
+
+
+def decode_workspace_bytes(dims, seg_len, rule):
+    return int(load_library().infini_attn_decode_workspace_bytes(ctypes.byref(dims), int(seg_len),
+                                                                 _rule(rule)))
+
+
+def decode_step(q_t, k_t, v_t, beta, k_buf, v_buf, pos, M, z, seg_len, rule, out=None,
+                workspace=None, stream=None):
+    """infini_attn_decode_step on CUDA tensors: q_t [B, H_q, d], k_t, v_t
+    [B, H_kv, d], buffers [B, H_kv, seg_len, d]; (M, z) updated in place when
+    pos == seg_len - 1.  Returns out [B, H_q, d]."""
+    lib = load_library()
+    if q_t.dim() != 3 or k_t.dim() != 3 or v_t.dim() != 3 or k_buf.dim() != 4:
+        raise ValueError("q_t, k_t, v_t must be [B, heads, d] and the buffers [B, H_kv, S, d]")
+    B, H_q, d = q_t.shape
+    H_kv = k_t.shape[1]
+    if q_t.dtype not in DTYPES:
+        raise ValueError("dtype must be bfloat16 or float32")
+    dims = make_dims(B, H_q, H_kv, 1, d, d, q_t.dtype)
+    if out is None:
+        out = torch.empty_like(q_t)
+    buf = (B, H_kv, int(seg_len), d)
+    args = [_dev(q_t, "q_t", q_t.dtype, (B, H_q, d)), _dev(k_t, "k_t", q_t.dtype, (B, H_kv, d)),
+            _dev(v_t, "v_t", q_t.dtype, (B, H_kv, d)), _dev(beta, "beta", torch.float32, (H_q,)),
+            _dev(k_buf, "k_buf", q_t.dtype, buf), _dev(v_buf, "v_buf", q_t.dtype, buf), int(pos),
+            _dev(M, "M", torch.float32, (B, H_kv, d, d)), _dev(z, "z", torch.float32, (B, H_kv, d)),
+            int(seg_len), _rule(rule), ctypes.byref(dims), _dev(out, "out", q_t.dtype, (B, H_q, d))]
+    if workspace is not None:
+        ws_ptr, ws_n = _dev(workspace, "workspace", torch.uint8), workspace.numel()
+    else:
+        ws_ptr, ws_n = ctypes.c_void_p(0), 0
+    _check(lib.infini_attn_decode_step(*args, ws_ptr, ws_n, _stream_handle(stream)))
+    return out
+
+
+class DecodeStream:
+    """A stream decoded one token at a time: owns the segment buffers, the
+    memory state and the position (marshalling around decode_step)."""
+
+    def __init__(self, B, H_q, H_kv, d, seg_len, rule, dtype=torch.bfloat16, device=None,
+                 M=None, z=None):
+        device = torch.device("cuda") if device is None else device
+        self.seg_len, self.rule, self.pos = int(seg_len), rule, 0
+        self.k_buf = torch.zeros((B, H_kv, self.seg_len, d), dtype=dtype, device=device)
+        self.v_buf = torch.zeros_like(self.k_buf)
+        self.M = (torch.zeros((B, H_kv, d, d), dtype=torch.float32, device=device) if M is None
+                  else M.clone())
+        self.z = (torch.zeros((B, H_kv, d), dtype=torch.float32, device=device) if z is None
+                  else z.clone())
+        dims = make_dims(B, H_q, H_kv, 1, d, d, dtype)
+        self.workspace = torch.empty(decode_workspace_bytes(dims, self.seg_len, rule),
+                                     dtype=torch.uint8, device=device)
+
+    def step(self, q_t, k_t, v_t, beta, out=None, stream=None):
+        out = decode_step(q_t, k_t, v_t, beta, self.k_buf, self.v_buf, self.pos, self.M, self.z,
+                          self.seg_len, self.rule, out=out, workspace=self.workspace, stream=stream)
+        self.pos = (self.pos + 1) % self.seg_len
+        return out
+
+    def final_state(self, stream=None):
+        """(M, z) after every token so far, counting a partly filled segment
+        (the stream itself is left unchanged)."""
+        if self.pos == 0:
+            return self.M.clone(), self.z.clone()
+        n = self.pos
+        return state_update(self.k_buf[:, :, :n].contiguous(), self.v_buf[:, :, :n].contiguous(),
+                            self.M, self.z, n, self.rule, stream=stream)
 
 
 def host_arena_bytes(dims, seg_len, rule):

@@ -142,6 +142,32 @@ unsigned int* status_ptr() {
   return static_cast<unsigned int*>(p);
 }
 
+// The forward's state scan alone over (k, v) of shape `s`: (M_in, z_in) ->
+// (M_out, z_out), per-segment states in the workspace `ws` (laid out by
+// check_shape).
+cudaError_t run_state_scan(const Shape& s, const void* k, const void* v, const float* M_in,
+                           const float* z_in, float* M_out, float* z_out, char* ws,
+                           unsigned int* status, cudaStream_t st) {
+  Problem p;
+  p.q = nullptr; p.k = k; p.v = v; p.beta = nullptr; p.M_in = M_in;
+  p.out = nullptr; p.M_out = M_out; p.z_out = z_out;
+  p.B = s.B; p.H_q = s.H_q; p.H_kv = s.H_kv; p.L = s.L; p.d_k = s.d_k; p.d_v = s.d_v;
+  p.S = s.S; p.T = s.T; p.bf16 = s.bf16; p.delta = s.delta;
+  p.z_pref = reinterpret_cast<float*>(ws + s.ws_zpref);
+  p.M_pref = ws + s.ws_mpref;
+  p.M_pref_bf16 = s.path == INFINI_PATH_TCGEN05;
+  p.Gbuf = reinterpret_cast<float*>(ws + s.ws_g);
+  p.Bbuf = reinterpret_cast<float*>(ws + s.ws_b);
+  p.dz = reinterpret_cast<float*>(ws + s.ws_dz);
+  p.status = status;
+  cudaError_t e = cudaMemcpyAsync(p.z_pref, z_in, s.z_bytes, cudaMemcpyDeviceToDevice, st);
+  if (e == cudaSuccess)
+    e = timed(0, st, [&] {
+      return s.path == INFINI_PATH_TCGEN05 ? launch_tc_state_scan(p, st) : launch_simt_state_scan(p, st);
+    });
+  return e;
+}
+
 }  // namespace
 
 unsigned int* device_status_word() { return status_ptr(); }
@@ -313,24 +339,92 @@ int infini_attn_state_update(const void* k, const void* v, const float* M_in, co
   }
   // The scan of infini_attn_forward alone: it reads k, v and the state, and
   // writes the per-segment states to the workspace and (M_out, z_out).
-  Problem p;
-  p.q = nullptr; p.k = k; p.v = v; p.beta = nullptr; p.M_in = M_in;
-  p.out = nullptr; p.M_out = M_out; p.z_out = z_out;
-  p.B = s.B; p.H_q = s.H_q; p.H_kv = s.H_kv; p.L = s.L; p.d_k = s.d_k; p.d_v = s.d_v;
-  p.S = s.S; p.T = s.T; p.bf16 = s.bf16; p.delta = s.delta;
-  p.z_pref = reinterpret_cast<float*>(ws + s.ws_zpref);
-  p.M_pref = ws + s.ws_mpref;
-  p.M_pref_bf16 = s.path == INFINI_PATH_TCGEN05;
-  p.Gbuf = reinterpret_cast<float*>(ws + s.ws_g);
-  p.Bbuf = reinterpret_cast<float*>(ws + s.ws_b);
-  p.dz = reinterpret_cast<float*>(ws + s.ws_dz);
-  p.status = status;
+  cudaError_t e = run_state_scan(s, k, v, M_in, z_in, M_out, z_out, ws, status, st);
+  if (owned) {
+    cudaError_t f = cudaFreeAsync(ws, st);
+    if (e == cudaSuccess) e = f;
+  }
+  return e == cudaSuccess ? INFINI_OK : INFINI_ERR_CUDA;
+}
 
-  cudaError_t e = cudaMemcpyAsync(p.z_pref, z_in, s.z_bytes, cudaMemcpyDeviceToDevice, st);
-  if (e == cudaSuccess)
-    e = timed(0, st, [&] {
-      return s.path == INFINI_PATH_TCGEN05 ? launch_tc_state_scan(p, st) : launch_simt_state_scan(p, st);
-    });
+namespace {
+
+// Shape of the segment update a decode step runs when the segment fills: a
+// forward over one segment (L = S).  Also checks the decode arguments.
+int decode_shape(const infini_dims_t* dims, int seg_len, int rule, Shape* s, size_t* part_bytes) {
+  if (!dims) return INFINI_ERR_ARG;
+  infini_dims_t one = *dims;
+  one.L = seg_len;
+  int rc = check_shape(&one, seg_len, rule, s);
+  if (rc != INFINI_OK) return rc;
+  if (dims->d_k != dims->d_v) return INFINI_ERR_UNSUPPORTED;
+  *part_bytes = align_up((size_t)dims->B * dims->H_q * decode_splits(seg_len) * (dims->d_k + 2) * 4);
+  return INFINI_OK;
+}
+
+}  // namespace
+
+size_t infini_attn_decode_workspace_bytes(const infini_dims_t* dims, int seg_len, int rule) {
+  Shape s;
+  size_t part = 0;
+  if (decode_shape(dims, seg_len, rule, &s, &part) != INFINI_OK) return 0;
+  return part + s.ws_total;
+}
+
+int infini_attn_decode_step(const void* q_t, const void* k_t, const void* v_t, const float* beta,
+                            void* k_buf, void* v_buf, int pos, float* M, float* z, int seg_len,
+                            int rule, const infini_dims_t* dims, void* out_t, void* workspace,
+                            size_t workspace_bytes, void* stream) {
+  Shape s;
+  size_t part_bytes = 0;
+  int rc = decode_shape(dims, seg_len, rule, &s, &part_bytes);
+  if (rc != INFINI_OK) return rc;
+  if (pos < 0 || pos >= seg_len) return INFINI_ERR_ARG;
+  if (!q_t || !k_t || !v_t || !beta || !k_buf || !v_buf || !M || !z || !out_t) return INFINI_ERR_ARG;
+  const void* ptrs[] = {q_t, k_t, v_t, beta, k_buf, v_buf, M, z, out_t};
+  for (const void* p : ptrs)
+    if (!aligned16(p)) return INFINI_ERR_ALIGN;
+  const size_t total = part_bytes + s.ws_total;
+  if (workspace == nullptr && workspace_bytes != 0) return INFINI_ERR_ARG;
+  if (workspace != nullptr) {
+    if (workspace_bytes < total || ((uintptr_t)workspace & (kAlign - 1)) != 0) return INFINI_ERR_WORKSPACE;
+  }
+  // Per-step sizes: one token of q, k, v, out; the buffers hold S rows.
+  const size_t tok_q = (size_t)s.B * s.H_q * s.d_k * s.elem, tok_kv = (size_t)s.B * s.H_kv * s.d_k * s.elem;
+  const Range r_kb = rng(k_buf, s.k_bytes), r_vb = rng(v_buf, s.v_bytes), r_out = rng(out_t, tok_q);
+  const Range r_M = rng(M, s.M_bytes), r_z = rng(z, s.z_bytes);
+  const Range all[] = {rng(q_t, tok_q), rng(k_t, tok_kv), rng(v_t, tok_kv), rng(beta, s.beta_bytes),
+                       r_kb, r_vb, r_M, r_z, r_out};
+  for (int i = 0; i < 9; ++i)
+    for (int j = i + 1; j < 9; ++j)
+      if (j >= 4 && overlap(all[i], all[j])) return INFINI_ERR_ALIAS;  // j is written
+  if (workspace) {
+    const Range r_ws = rng(workspace, total);
+    for (int i = 0; i < 9; ++i)
+      if (overlap(r_ws, all[i])) return INFINI_ERR_ALIAS;
+  }
+
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  unsigned int* status = status_ptr();
+  if (!status) return INFINI_ERR_CUDA;
+  char* ws = static_cast<char*>(workspace);
+  bool owned = false;
+  if (!ws) {
+    if (cudaMallocAsync(reinterpret_cast<void**>(&ws), total, st) != cudaSuccess) return INFINI_ERR_CUDA;
+    owned = true;
+  }
+  DecodeProblem dp;
+  dp.q_t = q_t; dp.k_t = k_t; dp.v_t = v_t; dp.beta = beta;
+  dp.k_buf = k_buf; dp.v_buf = v_buf; dp.M = M; dp.z = z; dp.out_t = out_t;
+  dp.part = reinterpret_cast<float*>(ws);
+  dp.B = s.B; dp.H_q = s.H_q; dp.H_kv = s.H_kv; dp.d = s.d_k; dp.S = seg_len; dp.pos = pos;
+  dp.nsplit = decode_splits(seg_len);
+  dp.bf16 = s.bf16;
+  cudaError_t e = timed(1, st, [&] { return launch_decode_step(dp, st); });
+  // The token filled the segment: M_s, z_s from the whole buffer, in place
+  // (after the output above, which read M_{s-1}, z_{s-1}).
+  if (e == cudaSuccess && pos == seg_len - 1)
+    e = run_state_scan(s, k_buf, v_buf, M, z, M, z, ws + part_bytes, status, st);
   if (owned) {
     cudaError_t f = cudaFreeAsync(ws, st);
     if (e == cudaSuccess) e = f;

@@ -54,4 +54,24 @@ void tc_scan_workspace(int B, int H_kv, int T, int d, bool delta, size_t* g_byte
                        size_t* dz_bytes);
 cudaError_t launch_tc_state_scan(const Problem& p, cudaStream_t stream);
 
+// Streaming decode step (one new token per head; CUDA cores): attention of
+// q_t over rows 0..pos of the segment buffer (row pos taken from k_t, v_t and
+// written into the buffer), retrieval from (M, z), gate -> out_t.
+struct DecodeProblem {
+  const void* q_t;     // [B, H_q, d]
+  const void* k_t;     // [B, H_kv, d]
+  const void* v_t;     // [B, H_kv, d]
+  const float* beta;   // [H_q]
+  void* k_buf;         // [B, H_kv, S, d]
+  void* v_buf;         // [B, H_kv, S, d]
+  const float* M;      // [B, H_kv, d, d] f32 (M_{s-1})
+  const float* z;      // [B, H_kv, d] f32 (z_{s-1})
+  void* out_t;         // [B, H_q, d]
+  float* part;         // workspace: [B * H_q][nsplit][d + 2] f32
+  int B, H_q, H_kv, d, S, pos, nsplit;
+  bool bf16;
+};
+int decode_splits(int S);
+cudaError_t launch_decode_step(const DecodeProblem& p, cudaStream_t stream);
+
 }  // namespace infini

@@ -180,6 +180,54 @@ INFINI_API int infini_attn_state_update(const void* k, const void* v, const floa
                                         const infini_dims_t* dims, float* M_out, float* z_out,
                                         void* workspace, size_t workspace_bytes, void* stream);
 
+/* Streaming decode: the layer forward one token at a time.  The current
+ * segment's keys and values so far are kept by the caller in a rolling
+ * buffer of seg_len rows per KV head; (M, z) hold the memory of the segments
+ * before it.  Decoding a sequence token by token (pos = 0, 1, ..., S - 1,
+ * 0, 1, ...) gives the outputs and states infini_attn_forward gives for the
+ * whole sequence.  ("Hugging Face Infini-Attention 再現分析", State Transfer:
+ * a stream processed segment by segment keeps only the memory; "Leave No
+ * Context Behind" explainer, "実装上の流れ": read the memory, attend within the
+ * segment, mix, update with the segment's K/V.)
+ *
+ * Bytes of device workspace infini_attn_decode_step needs (0 if the sizes are
+ * invalid; dims->L is ignored). */
+INFINI_API size_t infini_attn_decode_workspace_bytes(const infini_dims_t* dims, int seg_len,
+                                                     int rule);
+
+/* One decode step.
+ *   q_t              device [B, H_q, d], element type dims->dtype: the new
+ *                    token's queries
+ *   k_t, v_t         device [B, H_kv, d]: its keys and values
+ *   beta             device float32 [H_q]
+ *   k_buf, v_buf     device [B, H_kv, seg_len, d]: rows 0..pos-1 hold the
+ *                    current segment's earlier tokens; the call writes k_t,
+ *                    v_t into row pos (rows after pos are not read)
+ *   pos              0 <= pos < seg_len: the token's row in its segment
+ *   M, z             device float32 [B, H_kv, d, d] and [B, H_kv, d]: the
+ *                    state before the current segment.  When pos ==
+ *                    seg_len - 1 the segment is complete and the call updates
+ *                    them in place by `rule` with the whole buffer (after the
+ *                    token's output); the next call starts a segment at pos 0.
+ *                    At the end of a stream whose last segment is shorter,
+ *                    infini_attn_state_update on the buffer's first pos + 1
+ *                    rows (made contiguous) gives the final state.
+ *   seg_len, rule    as for infini_attn_forward
+ *   dims             B, H_q, H_kv, d_k = d_v = d, dtype; dims->L is ignored
+ *   out_t            device [B, H_q, d], element type dims->dtype
+ *   workspace        device scratch of infini_attn_decode_workspace_bytes
+ *                    bytes, 256-byte aligned, or NULL with workspace_bytes
+ *                    == 0 (stream-ordered allocation, as for the forward)
+ *   stream           cudaStream_t.
+ * The written regions (k_buf, v_buf, M, z, out_t) may not overlap each other,
+ * the inputs or the workspace (INFINI_ERR_ALIAS); d_k != d_v is
+ * INFINI_ERR_UNSUPPORTED.  Other errors: those of infini_attn_forward. */
+INFINI_API int infini_attn_decode_step(const void* q_t, const void* k_t, const void* v_t,
+                                       const float* beta, void* k_buf, void* v_buf, int pos,
+                                       float* M, float* z, int seg_len, int rule,
+                                       const infini_dims_t* dims, void* out_t, void* workspace,
+                                       size_t workspace_bytes, void* stream);
+
 /* Bytes of device arena infini_attn_forward_host needs: room for q, k, v,
  * beta, M, z, out and the workspace, each 256-byte aligned.  0 if invalid. */
 INFINI_API size_t infini_attn_host_arena_bytes(const infini_dims_t* dims, int seg_len, int rule);

@@ -113,6 +113,54 @@ def test_forward_validates_on_host_before_any_cuda_call(lib):
     assert _fwd(lib, good, d_bad) == api.ERR_UNSUPPORTED
 
 
+def test_state_update_validates_on_host_before_any_cuda_call(lib):
+    P = ctypes.c_void_p
+    d = api.Dims(1, 2, 2, 128, 32, 32, 1)
+    MB = 1 << 20
+    k, v, M, z, Mo, zo = 1 * MB, 2 * MB, 3 * MB, 4 * MB, 5 * MB, 6 * MB
+
+    def call(k=k, v=v, M=M, z=z, Mo=Mo, zo=zo, seg=64, rule=0, ws=0, ws_n=0, dims=d):
+        return lib.infini_attn_state_update(P(k), P(v), P(M), P(z), seg, rule, ctypes.byref(dims),
+                                            P(Mo), P(zo), P(ws), ws_n, P(0))
+
+    assert call(k=0) == api.ERR_ARG
+    assert call(v=v + 8) == api.ERR_ALIGN
+    assert call(Mo=k + 1024) == api.ERR_ALIAS      # M_out inside k
+    assert call(zo=M + 16) == api.ERR_ALIAS        # z_out overlaps M_in
+    assert call(rule=7) == api.ERR_ARG
+    assert call(seg=0) == api.ERR_ARG
+    assert call(ws=10 * MB, ws_n=16) == api.ERR_WORKSPACE
+    assert call(dims=api.Dims(1, 2, 2, 128, 40, 32, 1)) == api.ERR_UNSUPPORTED
+
+
+def test_decode_step_validates_on_host_before_any_cuda_call(lib):
+    P = ctypes.c_void_p
+    d = api.Dims(1, 4, 2, 1, 32, 32, 1)
+    MB = 1 << 20
+    good = dict(q=1 * MB, k=2 * MB, v=3 * MB, beta=4 * MB, kb=5 * MB, vb=6 * MB, M=7 * MB, z=8 * MB,
+                out=9 * MB)
+
+    def call(pos=0, seg=16, rule=0, ws=0, ws_n=0, dims=d, **over):
+        a = dict(good, **over)
+        return lib.infini_attn_decode_step(P(a["q"]), P(a["k"]), P(a["v"]), P(a["beta"]), P(a["kb"]),
+                                           P(a["vb"]), pos, P(a["M"]), P(a["z"]), seg, rule,
+                                           ctypes.byref(dims), P(a["out"]), P(ws), ws_n, P(0))
+
+    assert lib.infini_attn_decode_workspace_bytes(ctypes.byref(d), 16, 0) > 0
+    assert lib.infini_attn_decode_workspace_bytes(ctypes.byref(api.Dims(1, 4, 2, 1, 32, 64, 1)),
+                                                  16, 0) == 0
+    assert call(pos=16) == api.ERR_ARG            # pos must be < seg_len
+    assert call(pos=-1) == api.ERR_ARG
+    assert call(q=0) == api.ERR_ARG
+    assert call(k=good["k"] + 4) == api.ERR_ALIGN
+    assert call(out=good["q"]) == api.ERR_ALIAS    # out over q_t
+    assert call(kb=good["vb"] + 64) == api.ERR_ALIAS
+    assert call(M=good["kb"] + 256) == api.ERR_ALIAS
+    assert call(ws=10 * MB, ws_n=16) == api.ERR_WORKSPACE
+    assert call(ws=good["M"], ws_n=1 << 22) == api.ERR_ALIAS
+    assert call(dims=api.Dims(1, 4, 2, 1, 32, 64, 1)) == api.ERR_UNSUPPORTED
+
+
 def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
     monkeypatch.setattr(api, "_lib", None)
     with pytest.raises(FileNotFoundError):
