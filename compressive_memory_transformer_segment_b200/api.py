@@ -291,7 +291,8 @@ class DecodeStream:
         self.z = (torch.zeros((B, H_kv, d), dtype=torch.float32, device=device) if z is None
                   else z.clone())
         dims = make_dims(B, H_q, H_kv, 1, d, d, dtype)
-        self.workspace = torch.empty(decode_workspace_bytes(dims, self.seg_len, rule),
+        # zero-filled: the step's ticket counters start at 0
+        self.workspace = torch.zeros(decode_workspace_bytes(dims, self.seg_len, rule),
                                      dtype=torch.uint8, device=device)
 
     def step(self, q_t, k_t, v_t, beta, out=None, stream=None):

@@ -351,14 +351,24 @@ namespace {
 
 // Shape of the segment update a decode step runs when the segment fills: a
 // forward over one segment (L = S).  Also checks the decode arguments.
-int decode_shape(const infini_dims_t* dims, int seg_len, int rule, Shape* s, size_t* part_bytes) {
+// Decode workspace: [tickets | attention partials | retrieval | scan].
+struct DecodeLayout {
+  size_t ctr, part, ret, scan, total;
+};
+
+int decode_shape(const infini_dims_t* dims, int seg_len, int rule, Shape* s, DecodeLayout* lay) {
   if (!dims) return INFINI_ERR_ARG;
   infini_dims_t one = *dims;
   one.L = seg_len;
   int rc = check_shape(&one, seg_len, rule, s);
   if (rc != INFINI_OK) return rc;
   if (dims->d_k != dims->d_v) return INFINI_ERR_UNSUPPORTED;
-  *part_bytes = align_up((size_t)dims->B * dims->H_q * decode_splits(seg_len) * (dims->d_k + 2) * 4);
+  const size_t BHq = (size_t)dims->B * dims->H_q, d = dims->d_k;
+  lay->ctr = 0;
+  lay->part = align_up((size_t)dims->B * dims->H_kv * decode_head_chunks(dims->H_q / dims->H_kv) * 4);
+  lay->ret = align_up(lay->part + BHq * decode_splits(seg_len) * (d + 2) * 4);
+  lay->scan = align_up(lay->ret + BHq * (d + 1) * 4);
+  lay->total = lay->scan + s->ws_total;
   return INFINI_OK;
 }
 
@@ -366,9 +376,9 @@ int decode_shape(const infini_dims_t* dims, int seg_len, int rule, Shape* s, siz
 
 size_t infini_attn_decode_workspace_bytes(const infini_dims_t* dims, int seg_len, int rule) {
   Shape s;
-  size_t part = 0;
-  if (decode_shape(dims, seg_len, rule, &s, &part) != INFINI_OK) return 0;
-  return part + s.ws_total;
+  DecodeLayout lay;
+  if (decode_shape(dims, seg_len, rule, &s, &lay) != INFINI_OK) return 0;
+  return lay.total;
 }
 
 int infini_attn_decode_step(const void* q_t, const void* k_t, const void* v_t, const float* beta,
@@ -376,15 +386,15 @@ int infini_attn_decode_step(const void* q_t, const void* k_t, const void* v_t, c
                             int rule, const infini_dims_t* dims, void* out_t, void* workspace,
                             size_t workspace_bytes, void* stream) {
   Shape s;
-  size_t part_bytes = 0;
-  int rc = decode_shape(dims, seg_len, rule, &s, &part_bytes);
+  DecodeLayout lay;
+  int rc = decode_shape(dims, seg_len, rule, &s, &lay);
   if (rc != INFINI_OK) return rc;
   if (pos < 0 || pos >= seg_len) return INFINI_ERR_ARG;
   if (!q_t || !k_t || !v_t || !beta || !k_buf || !v_buf || !M || !z || !out_t) return INFINI_ERR_ARG;
   const void* ptrs[] = {q_t, k_t, v_t, beta, k_buf, v_buf, M, z, out_t};
   for (const void* p : ptrs)
     if (!aligned16(p)) return INFINI_ERR_ALIGN;
-  const size_t total = part_bytes + s.ws_total;
+  const size_t total = lay.total;
   if (workspace == nullptr && workspace_bytes != 0) return INFINI_ERR_ARG;
   if (workspace != nullptr) {
     if (workspace_bytes < total || ((uintptr_t)workspace & (kAlign - 1)) != 0) return INFINI_ERR_WORKSPACE;
@@ -412,11 +422,17 @@ int infini_attn_decode_step(const void* q_t, const void* k_t, const void* v_t, c
   if (!ws) {
     if (cudaMallocAsync(reinterpret_cast<void**>(&ws), total, st) != cudaSuccess) return INFINI_ERR_CUDA;
     owned = true;
+    if (cudaMemsetAsync(ws + lay.ctr, 0, lay.part - lay.ctr, st) != cudaSuccess) {
+      cudaFreeAsync(ws, st);
+      return INFINI_ERR_CUDA;
+    }
   }
   DecodeProblem dp;
   dp.q_t = q_t; dp.k_t = k_t; dp.v_t = v_t; dp.beta = beta;
   dp.k_buf = k_buf; dp.v_buf = v_buf; dp.M = M; dp.z = z; dp.out_t = out_t;
-  dp.part = reinterpret_cast<float*>(ws);
+  dp.part = reinterpret_cast<float*>(ws + lay.part);
+  dp.ret = reinterpret_cast<float*>(ws + lay.ret);
+  dp.ctr = reinterpret_cast<unsigned int*>(ws + lay.ctr);
   dp.B = s.B; dp.H_q = s.H_q; dp.H_kv = s.H_kv; dp.d = s.d_k; dp.S = seg_len; dp.pos = pos;
   dp.nsplit = decode_splits(seg_len);
   dp.bf16 = s.bf16;
@@ -424,7 +440,7 @@ int infini_attn_decode_step(const void* q_t, const void* k_t, const void* v_t, c
   // The token filled the segment: M_s, z_s from the whole buffer, in place
   // (after the output above, which read M_{s-1}, z_{s-1}).
   if (e == cudaSuccess && pos == seg_len - 1)
-    e = run_state_scan(s, k_buf, v_buf, M, z, M, z, ws + part_bytes, status, st);
+    e = run_state_scan(s, k_buf, v_buf, M, z, M, z, ws + lay.scan, status, st);
   if (owned) {
     cudaError_t f = cudaFreeAsync(ws, st);
     if (e == cudaSuccess) e = f;

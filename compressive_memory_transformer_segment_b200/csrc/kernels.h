@@ -67,11 +67,14 @@ struct DecodeProblem {
   const float* M;      // [B, H_kv, d, d] f32 (M_{s-1})
   const float* z;      // [B, H_kv, d] f32 (z_{s-1})
   void* out_t;         // [B, H_q, d]
-  float* part;         // workspace: [B * H_q][nsplit][d + 2] f32
+  float* part;         // workspace: [B * H_q][nsplit][d + 2] f32 (attention partials)
+  float* ret;          // workspace: [B * H_q][d + 1] f32 (sigma(q) M, sigma(q).z)
+  unsigned int* ctr;   // workspace: [B * H_kv][head chunks] tickets, 0 between steps
   int B, H_q, H_kv, d, S, pos, nsplit;
   bool bf16;
 };
 int decode_splits(int S);
+int decode_head_chunks(int g);
 cudaError_t launch_decode_step(const DecodeProblem& p, cudaStream_t stream);
 
 }  // namespace infini

@@ -191,7 +191,9 @@ INFINI_API int infini_attn_state_update(const void* k, const void* v, const floa
  * segment, mix, update with the segment's K/V.)
  *
  * Bytes of device workspace infini_attn_decode_step needs (0 if the sizes are
- * invalid; dims->L is ignored). */
+ * invalid; dims->L is ignored).  The workspace starts with the step's ticket
+ * counters: a workspace must be zero-filled before its first decode step
+ * (each step leaves the counters at zero again); the rest is scratch. */
 INFINI_API size_t infini_attn_decode_workspace_bytes(const infini_dims_t* dims, int seg_len,
                                                      int rule);
 
@@ -216,8 +218,9 @@ INFINI_API size_t infini_attn_decode_workspace_bytes(const infini_dims_t* dims, 
  *   dims             B, H_q, H_kv, d_k = d_v = d, dtype; dims->L is ignored
  *   out_t            device [B, H_q, d], element type dims->dtype
  *   workspace        device scratch of infini_attn_decode_workspace_bytes
- *                    bytes, 256-byte aligned, or NULL with workspace_bytes
- *                    == 0 (stream-ordered allocation, as for the forward)
+ *                    bytes, 256-byte aligned, zero-filled before its first
+ *                    decode step (see above), or NULL with workspace_bytes
+ *                    == 0 (stream-ordered allocation, zeroed by the call)
  *   stream           cudaStream_t.
  * The written regions (k_buf, v_buf, M, z, out_t) may not overlap each other,
  * the inputs or the workspace (INFINI_ERR_ALIAS); d_k != d_v is
