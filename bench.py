@@ -460,6 +460,35 @@ def decode_bytes_per_segment(w):
     return w.B * (w.H_kv * per_kv + w.H_q * per_q)
 
 
+def run_decode_probe(args, w):
+    """Three eager decode calls of the workload's shape at one position (the
+    buffers hold N(0,1) rows), for a profiler capture of the decode kernel;
+    prints no result line."""
+    import torch
+
+    from compressive_memory_transformer_segment_b200 import api
+
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    tdt = torch.bfloat16 if w.dtype == "bf16" else torch.float32
+    st = api.DecodeStream(w.B, w.H_q, w.H_kv, w.d_k, w.seg_len, w.rule, dtype=tdt, device=dev)
+    gen = torch.Generator(device=dev).manual_seed(w.seed)
+    st.k_buf.normal_(generator=gen)
+    st.v_buf.normal_(generator=gen)
+    st.z.fill_(1.0)
+    q = torch.randn((w.B, w.H_q, w.d_k), generator=gen, device=dev).to(tdt)
+    k = torch.randn((w.B, w.H_kv, w.d_k), generator=gen, device=dev).to(tdt)
+    v = torch.randn((w.B, w.H_kv, w.d_k), generator=gen, device=dev).to(tdt)
+    beta = torch.zeros(w.H_q, device=dev)
+    pos = min(max(args.decode_probe, 0), w.seg_len - 2)
+    for _ in range(3):
+        st.pos = pos
+        st.step(q, k, v, beta)
+    api.sync_status()
+    torch.cuda.synchronize(dev)
+    return 0
+
+
 def run_decode(args, w):
     """Streaming decode: one token per (batch row, head) per call, `steps`
     full segments of the workload's shape (S calls each; the state update
@@ -618,6 +647,9 @@ def main():
                     help="seconds of oracle work for the cpu_baseline sample")
     ap.add_argument("--reference-budget", type=float, default=60.0,
                     help="total seconds of oracle work for --impl reference")
+    ap.add_argument("--decode-probe", type=int, default=None, metavar="POS",
+                    help="three eager decode calls at position POS, no result line "
+                         "(for a profiler capture of the decode kernel)")
     ap.add_argument("--decode", action="store_true",
                     help="streaming decode (one token per call) of the workload's shape; "
                          "a step is one full segment")
@@ -629,6 +661,8 @@ def main():
         w = w.with_(B=args.batch, name=f"{w.name}-B{args.batch}")
     if args.impl == "reference":
         return run_reference(args, w)
+    if args.decode_probe is not None:
+        return run_decode_probe(args, w)
     if args.decode:
         return run_decode(args, w)
     return run_gpu(args, w)
