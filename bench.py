@@ -174,7 +174,11 @@ class ClockSampler:
         self.samples = []
         self.thread = None
         self.proc = None
-        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_rank{gpu_index}.csv")
+        # Raw samples of the nvidia-smi fallback (INFINI_CLOCKS_DIR, else the
+        # temporary directory).
+        import tempfile
+        out_dir = os.environ.get("INFINI_CLOCKS_DIR", tempfile.gettempdir())
+        self.path = os.path.join(out_dir, f"clocks_rank{gpu_index}.csv")
 
     def _nvml_loop(self, pynvml, h):
         bits = {"hw_slowdown": 0x8, "hw_thermal_slowdown": 0x40, "sw_thermal_slowdown": 0x20,
