@@ -451,6 +451,91 @@ def run_gpu(args, w):
     return 0
 
 
+def run_seq_parallel(args, w):
+    """Sequence-parallel linear rule (strong scaling): the workload's sequence
+    is cut into one run of whole segments per rank (shard.segment_range); each
+    rank's timed step is its run's state update from zero, one all-gather of
+    the updates, the exclusive prefix and the forward over its run."""
+    import torch
+    import torch.distributed as dist
+
+    from compressive_memory_transformer_segment_b200 import api, shard
+
+    if w.rule != "linear":
+        raise SystemExit("--seq-parallel needs a linear-rule workload (the delta rule is sequential)")
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+    api.load_library()
+    l0, l1 = shard.segment_range(w.L, w.seg_len, world, rank)
+    # This rank's rows only, drawn with a seed of their own (the values differ
+    # from one draw of the whole sequence; the throughput does not depend on
+    # them), without the inserted key/value pair.
+    inp = synth.make_inputs(w.with_(L=l1 - l0, seed=w.seed + 104729 * (l0 // w.seg_len),
+                                    insert_pair=False))
+    tdt = torch.bfloat16 if w.dtype == "bf16" else torch.float32
+
+    def dev_tensor(x):
+        if w.dtype == "bf16":
+            return torch.from_numpy(np.ascontiguousarray(x).view(np.int16)).view(torch.bfloat16).to(dev)
+        return torch.from_numpy(np.ascontiguousarray(x, dtype=np.float32)).to(dev)
+
+    q, k, v = (dev_tensor(inp[n]) for n in ("q", "k", "v"))
+    beta = torch.from_numpy(inp["beta"]).to(dev)
+    M0, z0 = api.init_state(w.B, w.H_kv, w.d_k, w.d_v, device=dev)
+
+    def step():
+        return shard.sequence_parallel_forward(q, k, v, beta, M0, z0, w.seg_len,
+                                               forward=api.forward, state_update=api.state_update)
+
+    for _ in range(args.warmup):
+        step()
+    api.sync_status()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    stream = torch.cuda.current_stream(dev)
+    with ClockSampler(local) as clocks:
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(args.steps):
+            step()
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier()
+    api.sync_status()
+    max_ms = shard.max_over_ranks(e0.elapsed_time(e1), device=dev)
+    if world > 1:
+        dist.destroy_process_group()
+    if rank != 0:
+        return 0
+    tokens = w.B * w.L * args.steps
+    step_ms = max_ms / args.steps
+    peaks, _ = load_peaks()
+    flops = configs.algorithmic_flops(w)
+    print(json.dumps({
+        "metric": "Infini-attention fwd tokens/s, sequence-parallel linear rule",
+        "value": tokens / (max_ms / 1000.0), "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": step_ms,
+        "higher_is_better": True, "scaling": "strong", "vs_baseline": None, "dtype": w.dtype,
+        "data": "synthetic (seeded Philox N(0,1) q/k/v, U(-r,r) beta)",
+        "config": {"workload": w.name, "B": w.B, "H_q": w.H_q, "H_kv": w.H_kv, "L": w.L,
+                   "d": w.d_k, "seg_len": w.seg_len, "rule": w.rule,
+                   "parallelism": f"sp{world} (one run of whole segments per rank; one "
+                                  "all-gather of the runs' state updates)",
+                   "l2": "inputs larger than L2; steps timed back to back"},
+        "tc_peak_frac_step": (flops / (step_ms / 1000.0)) / (peaks["bf16_tflops"] * 1e12),
+        "clocks": clocks.summary(), "e2e": None, "cpu_baseline": None,
+    }), flush=True)
+    return 0
+
+
 def decode_bytes_per_segment(w):
     """Algorithmic HBM bytes of decoding one full segment (S steps, pos =
     0..S-1): per KV head the buffer rows 0..pos (keys and values), M and z,
@@ -654,6 +739,8 @@ def main():
     ap.add_argument("--decode-probe", type=int, default=None, metavar="POS",
                     help="three eager decode calls at position POS, no result line "
                          "(for a profiler capture of the decode kernel)")
+    ap.add_argument("--seq-parallel", action="store_true",
+                    help="sequence-parallel linear rule over the ranks (strong scaling)")
     ap.add_argument("--decode", action="store_true",
                     help="streaming decode (one token per call) of the workload's shape; "
                          "a step is one full segment")
@@ -669,6 +756,8 @@ def main():
         return run_decode_probe(args, w)
     if args.decode:
         return run_decode(args, w)
+    if args.seq_parallel:
+        return run_seq_parallel(args, w)
     return run_gpu(args, w)
 
 
