@@ -55,3 +55,24 @@ def test_make_head_matches_make_inputs():
             for h in range(H):
                 np.testing.assert_array_equal(synth.make_head(w, name, b, h), x[name][b, h])
     np.testing.assert_array_equal(synth.make_beta(w), x["beta"])
+
+
+def test_decode_bytes_per_segment_closed_form():
+    """The decode roofline's byte count (bench.py) against a sum over the
+    positions of one segment, written out call by call."""
+    import importlib.util
+    import os
+    spec = importlib.util.spec_from_file_location(
+        "bench_mod", os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "bench.py"))
+    bench = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(bench)
+    for name, over in (("8b-delta", {}), ("tiny", dict(dtype="bf16", d_k=64, d_v=64, seg_len=48))):
+        w = configs.WORKLOADS[name].with_(**over)
+        e = 2 if w.dtype == "bf16" else 4
+        d, S = w.d_k, w.seg_len
+        total = 0
+        for pos in range(S):
+            per_kv = (pos + 1) * 2 * d * e + d * d * 4 + d * 4 + 2 * d * e + 2 * d * e
+            per_q = d * e + d * e + 4
+            total += w.B * (w.H_kv * per_kv + w.H_q * per_q)
+        assert bench.decode_bytes_per_segment(w) == total
