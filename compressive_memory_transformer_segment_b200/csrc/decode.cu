@@ -17,8 +17,8 @@
 // Decode is bound by memory traffic and latency (each buffer row and M are
 // read once per step, a few flops per byte), so it runs on CUDA cores, in
 // ONE kernel per step: grid (row chunks + 1, B * H_kv, query-head chunks).
-//   - CTA x < chunks: up to 128 buffer rows of one KV head, read once for up
-//     to kG query heads of its group.  A warp takes 8 rows at a time (vector
+//   - CTA x < chunks: up to kRows (64) buffer rows of one KV head, read once
+//     for up to kG query heads of its group.  A warp takes 8 rows at a time (vector
 //     loads, lanes across d; the 8 x kG dot products and their 2^x are
 //     independent, so the latency of one row overlaps the next), keeping an
 //     online softmax per head; the CTA's partial (max, sum, acc[d]) per head

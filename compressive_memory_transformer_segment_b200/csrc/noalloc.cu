@@ -12,14 +12,21 @@
 // How.  The scratch the forward needs (the memory every segment reads, for
 // all segments) lives in one file-scope device array of fixed size,
 // kNoAllocScratchBytes.  Host code cannot use the array's name as a device
-// address, so the first call on each device looks its address up with
-// cudaGetSymbolAddress (with that device current) and keeps it; later calls
-// on that device reuse it.  The call then runs the regular forward with that
-// address as its workspace.  Nothing here allocates.
+// address, so every call looks the address up with cudaGetSymbolAddress
+// (with the caller's device current) and runs the regular forward with that
+// address as its workspace.  The lookup is repeated on every call rather
+// than cached: after cudaDeviceReset the module is loaded again, possibly at
+// another address, and a cached pointer would be stale.  Nothing here
+// allocates.
+//
+// First call per device.  CUDA loads a library's GPU code lazily by default
+// (CUDA_MODULE_LOADING=LAZY): the first call on a device loads the modules
+// this call uses, which commits device memory for their code and for the
+// 64 MiB array.  A caller that must never allocate makes one warm-up call
+// outside its no-allocation region (or runs with CUDA_MODULE_LOADING=EAGER);
+// later calls of the same shape commit nothing.
 #include <cuda_runtime.h>
 #include <stdint.h>
-
-#include <mutex>
 
 #include "infini_attn.h"
 
@@ -28,27 +35,14 @@ namespace {
 // 64 MiB: enough for the tiny, 200M-, 300M- and 8B-shaped workloads; a
 // 1M-token stream needs about 1.7 GiB and is rejected.
 constexpr size_t kNoAllocScratchBytes = size_t(64) << 20;
-constexpr int kMaxDevices = 64;
-
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
 
-std::mutex g_mu;
-void* g_scratch_addr[kMaxDevices];  // device address of g_noalloc_scratch, per device
-
-// Looks up (once per device) the device address of the static scratch array.
+// Device address of g_noalloc_scratch on the current device.
 cudaError_t scratch_address(void** out) {
-  int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
+  void* p = nullptr;
+  const cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
   if (e != cudaSuccess) return e;
-  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
-  std::lock_guard<std::mutex> lock(g_mu);
-  if (!g_scratch_addr[dev]) {
-    void* p = nullptr;
-    e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
-    if (e != cudaSuccess) return e;
-    g_scratch_addr[dev] = p;
-  }
-  *out = g_scratch_addr[dev];
+  *out = p;
   return cudaSuccess;
 }
 
