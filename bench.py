@@ -7,9 +7,12 @@ resident in HBM.  Prints one JSON line on rank 0.
   python bench.py [--gpus N] [--steps K] [--warmup W] [--config NAME] [--impl reference]
 
 Multi-GPU (launched by torchrun, one process per GPU): the work shards over
-independent (batch, KV head) chains with no data-path collective, so every
-rank runs its own full batch of the workload (weak scaling) and the value is
-all ranks' tokens over the slowest rank's device time.
+independent (batch, KV head) chains with no data-path collective.  By default
+every rank runs its own full batch of the workload (weak scaling) and the
+value is all ranks' tokens over the slowest rank's device time; with
+``--shard chains`` the workload's own chains are split into one (batch rows x
+KV heads) block per rank (strong scaling: the value is the workload's tokens
+over the slowest rank's device time).
 
 ``--impl reference`` times the float64 CPU oracle on a bounded sample of the
 same workload, on the host cores.
@@ -258,11 +261,17 @@ class ClockSampler:
                 "source": "nvml" if self.thread is not None else "nvidia-smi"}
 
 
-def config_dict(w, n_gpus, l2_note):
+def config_dict(w, n_gpus, l2_note, block=None):
     d = {"workload": w.name, "B": w.B, "H_q": w.H_q, "H_kv": w.H_kv, "L": w.L,
          "d_k": w.d_k, "d_v": w.d_v, "seg_len": w.seg_len, "T": w.T, "rule": w.rule,
          "io_dtype": w.dtype, "state_dtype": "f32", "tokens_per_step_per_gpu": w.tokens,
          "parallelism": f"dp{n_gpus} (independent (batch, KV head) chains, no collective)"}
+    if block is not None:
+        b0, b1, h0, h1 = block
+        d["tokens_per_step_per_gpu"] = None
+        d["parallelism"] = (f"chains{n_gpus} (the workload's (batch row, KV head) chains split "
+                            f"into one block per rank, no collective; rank 0: rows [{b0}, {b1}), "
+                            f"KV heads [{h0}, {h1}))")
     if l2_note:
         d["l2"] = l2_note
     return d
@@ -285,6 +294,16 @@ def run_gpu(args, w):
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
     api.load_library()
+    # --shard chains: this rank runs only its block of the workload's (batch
+    # row, KV head) chains (strong scaling); otherwise every rank runs the
+    # whole workload on inputs of its own (weak scaling).
+    w_job, block = w, None
+    if args.shard == "chains":
+        block = shard.chain_block(w.B, w.H_kv, world, rank)
+        g = w.H_q // w.H_kv
+        b0, b1, h0, h1 = block
+        w = w.with_(B=b1 - b0, H_kv=h1 - h0, H_q=(h1 - h0) * g)
+    job_tokens = w_job.tokens if block is not None else w.tokens * world
 
     def barrier():
         if world > 1:
@@ -358,7 +377,7 @@ def run_gpu(args, w):
     api.sync_status(stream)
 
     max_ms = shard.max_over_ranks(elapsed_ms, device=dev)
-    tokens = w.tokens * args.steps * world
+    tokens = job_tokens * args.steps
     value = tokens / (max_ms / 1000.0)
 
     # End to end through the C ABI with host buffers (pinned), copies inside.
@@ -369,7 +388,8 @@ def run_gpu(args, w):
             print(json.dumps({"metric": METRIC, "value": value, "unit": "tokens/s",
                               "ms_per_step": max_ms / args.steps,
                               "kernel_ms": {k: v[0] / max(v[1], 1) for k, v in ktimes.items()},
-                              "config": config_dict(w, world, l2_note), "note": "profiling run"}))
+                              "config": config_dict(w_job, world, l2_note, block),
+                              "note": "profiling run"}))
         return 0
     hq_p, hk_p, hv_p = (x.pin_memory() for x in (hq, hk, hv))
     hbeta = torch.from_numpy(inp["beta"]).pin_memory()
@@ -396,7 +416,7 @@ def run_gpu(args, w):
     e1.record(stream)
     torch.cuda.synchronize(dev)
     e2e_ms = shard.max_over_ranks(e0.elapsed_time(e1), device=dev)
-    e2e_value = w.tokens * e2e_steps * world / (e2e_ms / 1000.0)
+    e2e_value = job_tokens * e2e_steps / (e2e_ms / 1000.0)
     h2d = sum(x.numel() * x.element_size() for x in (hq_p, hk_p, hv_p, hbeta, hM0, hz0))
     d2h = sum(x.numel() * x.element_size() for x in (hout, hM1, hz1))
 
@@ -422,9 +442,10 @@ def run_gpu(args, w):
     line = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": step_ms,
-        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "higher_is_better": True, "scaling": "strong" if block is not None else "weak",
+        "vs_baseline": None,
         "dtype": w.dtype, "data": "synthetic (seeded Philox N(0,1) q/k/v, U(-r,r) beta)",
-        "config": config_dict(w, world, l2_note),
+        "config": config_dict(w_job, world, l2_note, block),
         "path": plan["path"],
         "tc_peak_frac_step": (flops / (step_ms / 1000.0)) / (peak * 1e12),
         # The step's algorithmic bytes (q, k, v read once, out written once,
@@ -444,7 +465,7 @@ def run_gpu(args, w):
         "kernel_ms": {"attention": att_ms / max(att_n, 1), "state_scan": scan_ms / max(scan_n, 1)},
     }
     if args.cpu_baseline:
-        v, desc, _ = oracle_sample(w, args.cpu_budget)
+        v, desc, _ = oracle_sample(w_job, args.cpu_budget)
         line["cpu_baseline"] = {"value": v, "unit": "tokens/s", "cores": host_cores(),
                                 "kind": "oracle", "sample": desc}
     print(json.dumps(line), flush=True)
@@ -491,7 +512,8 @@ def run_seq_parallel(args, w):
 
     def step():
         return shard.sequence_parallel_forward(q, k, v, beta, M0, z0, w.seg_len,
-                                               forward=api.forward, state_update=api.state_update)
+                                               forward=api.forward, state_update=api.state_update,
+                                               state_sum=api.state_sum)
 
     for _ in range(args.warmup):
         step()
@@ -739,6 +761,10 @@ def main():
     ap.add_argument("--decode-probe", type=int, default=None, metavar="POS",
                     help="three eager decode calls at position POS, no result line "
                          "(for a profiler capture of the decode kernel)")
+    ap.add_argument("--shard", choices=["replicas", "chains"], default="replicas",
+                    help="replicas: every rank runs the whole workload (weak scaling); chains: "
+                         "the workload's (batch row, KV head) chains are split, one block per "
+                         "rank (strong scaling)")
     ap.add_argument("--seq-parallel", action="store_true",
                     help="sequence-parallel linear rule over the ranks (strong scaling)")
     ap.add_argument("--decode", action="store_true",

@@ -59,6 +59,8 @@ _SIGNATURES = [
                                            ctypes.POINTER(Dims), _P, _P, _P, _P, ctypes.c_size_t, _P]),
     ("infini_attn_state_update", ctypes.c_int, [_P, _P, _P, _P, ctypes.c_int, ctypes.c_int,
                                                 ctypes.POINTER(Dims), _P, _P, _P, ctypes.c_size_t, _P]),
+    ("infini_attn_state_sum", ctypes.c_int, [_P, _P, _P, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                             ctypes.c_int, ctypes.c_int, _P, _P, _P]),
     ("infini_attn_decode_workspace_bytes", ctypes.c_size_t, [ctypes.POINTER(Dims), ctypes.c_int,
                                                               ctypes.c_int]),
     ("infini_attn_decode_step", ctypes.c_int, [_P, _P, _P, _P, _P, _P, ctypes.c_int, _P, _P,
@@ -118,6 +120,19 @@ def _stream_handle(stream):
     if stream is None:
         stream = torch.cuda.current_stream()
     return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _one_device(first, *tensors, stream=None):
+    """The library launches on the current CUDA device: every tensor (and the
+    stream, if given) must be on the device of ``first``, which the call then
+    makes current."""
+    dev = first.device
+    for t in tensors:
+        if isinstance(t, torch.Tensor) and t.device != dev:
+            raise ValueError(f"all tensors must be on {dev}; got one on {t.device}")
+    if stream is not None and stream.device != dev:
+        raise ValueError(f"the stream is on {stream.device}, the tensors on {dev}")
+    return torch.cuda.device(dev)
 
 
 def make_dims(B, H_q, H_kv, L, d_k, d_v, dtype):
@@ -203,8 +218,9 @@ def forward(q, k, v, beta, M_in, z_in, seg_len, rule, out=None, M_out=None, z_ou
         ws_ptr, ws_n = _dev(workspace, "workspace", torch.uint8), workspace.numel()
     else:
         ws_ptr, ws_n = ctypes.c_void_p(0), 0
-    _check(lib.infini_attn_forward(*args, int(seg_len), _rule(rule), ctypes.byref(dims), *outs,
-                                   ws_ptr, ws_n, _stream_handle(stream)))
+    with _one_device(q, k, v, beta, M_in, z_in, out, M_out, z_out, workspace, stream=stream):
+        _check(lib.infini_attn_forward(*args, int(seg_len), _rule(rule), ctypes.byref(dims), *outs,
+                                       ws_ptr, ws_n, _stream_handle(stream)))
     return out, M_out, z_out
 
 
@@ -237,8 +253,34 @@ def state_update(k, v, M_in, z_in, seg_len, rule, M_out=None, z_out=None, worksp
         ws_ptr, ws_n = _dev(workspace, "workspace", torch.uint8), workspace.numel()
     else:
         ws_ptr, ws_n = ctypes.c_void_p(0), 0
-    _check(lib.infini_attn_state_update(*args, int(seg_len), _rule(rule), ctypes.byref(dims), *outs,
-                                        ws_ptr, ws_n, _stream_handle(stream)))
+    with _one_device(k, v, M_in, z_in, M_out, z_out, workspace, stream=stream):
+        _check(lib.infini_attn_state_update(*args, int(seg_len), _rule(rule), ctypes.byref(dims),
+                                            *outs, ws_ptr, ws_n, _stream_handle(stream)))
+    return M_out, z_out
+
+
+def state_sum(M_base, z_base, parts, n_parts, M_out=None, z_out=None, stream=None):
+    """infini_attn_state_sum: (M_base + the first ``n_parts`` packed states of
+    ``parts`` (float32 CUDA tensor [n, B*H_kv*d_k*d_v + B*H_kv*d_k]), z_base
+    likewise), summed in part order; returns (M_out, z_out)."""
+    lib = load_library()
+    B, H_kv, d_k, d_v = M_base.shape
+    if M_out is None:
+        M_out = torch.empty_like(M_base)
+    if z_out is None:
+        z_out = torch.empty_like(z_base)
+    n_parts = int(n_parts)
+    width = B * H_kv * d_k * (d_v + 1)
+    if parts.dim() != 2 or parts.shape[1] != width or not 0 <= n_parts <= parts.shape[0]:
+        raise ValueError(f"parts must be [n >= n_parts, {width}]")
+    args = [_dev(M_base, "M_base", torch.float32, (B, H_kv, d_k, d_v)),
+            _dev(z_base, "z_base", torch.float32, (B, H_kv, d_k)),
+            _dev(parts, "parts", torch.float32) if n_parts > 0 else ctypes.c_void_p(0), n_parts,
+            B, H_kv, d_k, d_v,
+            _dev(M_out, "M_out", torch.float32, (B, H_kv, d_k, d_v)),
+            _dev(z_out, "z_out", torch.float32, (B, H_kv, d_k))]
+    with _one_device(M_base, z_base, parts, M_out, z_out, stream=stream):
+        _check(lib.infini_attn_state_sum(*args, _stream_handle(stream)))
     return M_out, z_out
 
 
@@ -272,7 +314,8 @@ def decode_step(q_t, k_t, v_t, beta, k_buf, v_buf, pos, M, z, seg_len, rule, out
         ws_ptr, ws_n = _dev(workspace, "workspace", torch.uint8), workspace.numel()
     else:
         ws_ptr, ws_n = ctypes.c_void_p(0), 0
-    _check(lib.infini_attn_decode_step(*args, ws_ptr, ws_n, _stream_handle(stream)))
+    with _one_device(q_t, k_t, v_t, beta, k_buf, v_buf, M, z, out, workspace, stream=stream):
+        _check(lib.infini_attn_decode_step(*args, ws_ptr, ws_n, _stream_handle(stream)))
     return out
 
 
@@ -385,8 +428,9 @@ def forward_noalloc(q, k, v, beta, M_in, z_in, seg_len, rule, out, M_out, z_out,
     outs = [_dev(out, "out", q.dtype, (B, H_q, L, d_v)),
             _dev(M_out, "M_out", torch.float32, (B, H_kv, d_k, d_v)),
             _dev(z_out, "z_out", torch.float32, (B, H_kv, d_k))]
-    _check(lib.infini_attn_forward_noalloc(*args, int(seg_len), _rule(rule), ctypes.byref(dims),
-                                           *outs, _stream_handle(stream)))
+    with _one_device(q, k, v, beta, M_in, z_in, out, M_out, z_out, stream=stream):
+        _check(lib.infini_attn_forward_noalloc(*args, int(seg_len), _rule(rule),
+                                               ctypes.byref(dims), *outs, _stream_handle(stream)))
     return out, M_out, z_out
 
 

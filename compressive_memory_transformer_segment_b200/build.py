@@ -36,14 +36,17 @@ def build(force=False, verbose=False, extra=()):
         return LIB
     objdir = os.path.join(PKG, "_build")
     os.makedirs(objdir, exist_ok=True)
-    objs = []
-    for src in srcs:
+    objs, procs = [], []
+    for src in srcs:  # one nvcc per source, in parallel
         obj = os.path.join(objdir, os.path.basename(src) + ".o")
         cmd = [NVCC, *FLAGS, *extra, "-I", INCLUDE, "-I", CSRC, "-c", src, "-o", obj]
         if verbose:
             print(" ".join(cmd), flush=True)
-        subprocess.run(cmd, check=True)
+        procs.append((cmd, subprocess.Popen(cmd)))
         objs.append(obj)
+    failed = [cmd for cmd, proc in procs if proc.wait() != 0]
+    if failed:
+        raise subprocess.CalledProcessError(1, failed[0])
     tmp = LIB + ".tmp"
     cmd = [NVCC, "-gencode", "arch=compute_100a,code=sm_100a", "-shared", "-Xcompiler", "-fPIC",
            *objs, "-o", tmp, "-lcudart_static", "-ldl", "-lrt", "-lpthread"]

@@ -168,6 +168,25 @@ cudaError_t run_state_scan(const Shape& s, const void* k, const void* v, const f
   return e;
 }
 
+// out[i] = base[i] + parts[0][i] + ... + parts[n - 1][i] over the packed
+// state [M | z]; each element summed in fp32 in part order.  (base and out
+// may be the same array: each element is read before it is written by the
+// same thread.)
+__global__ void __launch_bounds__(256) state_sum_kernel(const float* M_base, const float* z_base,
+                                                        const float* __restrict__ parts, int n_parts,
+                                                        size_t nM, size_t nz, float* M_out,
+                                                        float* z_out) {
+  const size_t n = nM + nz;
+  for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < n; i += (size_t)gridDim.x * blockDim.x) {
+    float acc = i < nM ? M_base[i] : z_base[i - nM];
+    for (int p = 0; p < n_parts; ++p) acc += parts[(size_t)p * n + i];
+    if (i < nM)
+      M_out[i] = acc;
+    else
+      z_out[i - nM] = acc;
+  }
+}
+
 }  // namespace
 
 unsigned int* device_status_word() { return status_ptr(); }
@@ -345,6 +364,34 @@ int infini_attn_state_update(const void* k, const void* v, const float* M_in, co
     if (e == cudaSuccess) e = f;
   }
   return e == cudaSuccess ? INFINI_OK : INFINI_ERR_CUDA;
+}
+
+int infini_attn_state_sum(const float* M_base, const float* z_base, const float* parts, int n_parts,
+                          int B, int H_kv, int d_k, int d_v, float* M_out, float* z_out,
+                          void* stream) {
+  if (!M_base || !z_base || !M_out || !z_out || n_parts < 0 || (n_parts > 0 && !parts))
+    return INFINI_ERR_ARG;
+  if (B < 1 || H_kv < 1 || d_k < 1 || d_v < 1) return INFINI_ERR_ARG;
+  const void* ptrs[] = {M_base, z_base, M_out, z_out, parts};
+  for (const void* p : ptrs)
+    if (p && !aligned16(p)) return INFINI_ERR_ALIGN;
+  const size_t nM = (size_t)B * H_kv * d_k * d_v, nz = (size_t)B * H_kv * d_k;
+  const Range r_M = rng(M_out, nM * 4), r_z = rng(z_out, nz * 4);
+  const Range r_bM = rng(M_base, nM * 4), r_bz = rng(z_base, nz * 4);
+  if (overlap(r_M, r_z)) return INFINI_ERR_ALIAS;
+  if (overlap(r_M, r_bM) && M_out != M_base) return INFINI_ERR_ALIAS;
+  if (overlap(r_z, r_bz) && z_out != z_base) return INFINI_ERR_ALIAS;
+  if (overlap(r_M, r_bz) || overlap(r_z, r_bM)) return INFINI_ERR_ALIAS;
+  if (n_parts > 0) {
+    const Range r_p = rng(parts, (size_t)n_parts * (nM + nz) * 4);
+    if (overlap(r_p, r_M) || overlap(r_p, r_z)) return INFINI_ERR_ALIAS;
+  }
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const size_t n = nM + nz;
+  const size_t blocks = (n + 255) / 256;
+  const unsigned grid = (unsigned)(blocks < 4096 ? blocks : 4096);
+  state_sum_kernel<<<grid, 256, 0, st>>>(M_base, z_base, parts, n_parts, nM, nz, M_out, z_out);
+  return cudaGetLastError() == cudaSuccess ? INFINI_OK : INFINI_ERR_CUDA;
 }
 
 namespace {

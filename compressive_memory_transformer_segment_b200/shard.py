@@ -3,11 +3,14 @@
 Each KV head's memory (and the query heads that read it) is independent of
 every other head and batch row: the method keeps one compressive memory per
 head ("Leave No Context Behind" explainer, section "メモリ構造").  So the work
-splits across ranks with no data-path exchange: a rank takes a contiguous
-range of batch rows (whole rows keep every GQA group and every segment chain
-together), runs the forward on its own GPU, and results are assembled by
-concatenation.  The only collectives are for timing (max over ranks) and,
-when a caller wants the full result on one rank, a gather.
+splits across ranks with no data-path exchange.  The (batch row, KV head)
+chains form a B x H_kv grid; a rank takes one rectangular block of it (a run
+of batch rows times a run of KV heads, with every query head of those KV
+heads' groups), runs the forward on its own GPU on contiguous copies of its
+block, and results are assembled by an all-gather.  Splitting along the KV
+heads comes first, so a single long stream (B = 1, the 1M-token shape) also
+splits.  The only collectives are for timing (max over ranks) and, when a
+caller wants the full result on one rank, the gather.
 
 Sequence parallelism for the linear rule.  Under the linear rule the memory
 after a run of segments is the memory before it plus a sum over the run's
@@ -17,9 +20,10 @@ So a sequence cut at segment boundaries into one contiguous run per rank
 needs one exchange: every rank computes its run's update from a zero state,
 the updates are all-gathered, each rank adds those of the ranks before it to
 the initial state (an exclusive prefix, in rank order, so every rank forms
-the same sums) and then runs the forward over its own segments from there.
-The delta rule's update depends on the memory it starts from, so it stays
-sequential in the segments and is sharded by batch rows only.
+the same sums; the library's infini_attn_state_sum does the additions) and
+then runs the forward over its own segments from there.  The delta rule's
+update depends on the memory it starts from, so it stays sequential in the
+segments and is sharded by chains only.
 """
 
 import torch
@@ -50,6 +54,62 @@ def gather_batch(local, B, world, group=None):
     parts = [torch.empty_like(pad) for _ in range(world)]
     dist.all_gather(parts, pad, group=group)
     return torch.cat([p[:n] for p, n in zip(parts, sizes)], dim=0)
+
+
+def split_factors(B, H_kv, world):
+    """(wb, wh) with wb * wh == world: ranks along the batch rows and along the
+    KV heads.  Each is at most its extent; splits that divide both extents
+    evenly come first, then the larger head split."""
+    best = None
+    for wh in range(min(world, H_kv), 0, -1):
+        if world % wh:
+            continue
+        wb = world // wh
+        if wb > B:
+            continue
+        key = (H_kv % wh == 0 and B % wb == 0, wh)
+        if best is None or key > best[0]:
+            best = (key, (wb, wh))
+    if best is None:
+        raise ValueError(f"{world} ranks cannot each take a block of {B} batch rows x {H_kv} KV heads")
+    return best[1]
+
+
+def chain_block(B, H_kv, world, rank):
+    """`rank`'s block of (batch row, KV head) chains: rows [b0, b1) and KV heads
+    [h0, h1) (near-equal splits; together the blocks tile the B x H_kv grid)."""
+    wb, wh = split_factors(B, H_kv, world)
+    if not 0 <= rank < world:
+        raise ValueError("bad rank")
+    rb, rh = divmod(rank, wh)
+    b0, b1 = batch_range(B, wb, rb)
+    h0, h1 = batch_range(H_kv, wh, rh)
+    return b0, b1, h0, h1
+
+
+def shard_chains(t, block, group_size=1):
+    """Contiguous copy of the block's part of a [B, heads, ...] tensor, where
+    each KV head owns `group_size` consecutive heads of `t` (the query heads of
+    its group for q, out and beta's broadcast; 1 for k, v, M and z)."""
+    b0, b1, h0, h1 = block
+    return t[b0:b1, h0 * group_size:h1 * group_size].contiguous()
+
+
+def gather_chains(local, B, H_kv, world, group_size=1, group=None):
+    """All-gather every rank's block (from shard_chains layout, possibly of
+    unequal sizes) into the full [B, H_kv * group_size, ...] tensor."""
+    blocks = [chain_block(B, H_kv, world, r) for r in range(world)]
+    nb = max(b1 - b0 for b0, b1, _, _ in blocks)
+    nh = max(h1 - h0 for _, _, h0, h1 in blocks) * group_size
+    rest = tuple(local.shape[2:])
+    pad = torch.zeros((nb, nh) + rest, dtype=local.dtype, device=local.device)
+    pad[: local.shape[0], : local.shape[1]] = local
+    parts = [torch.empty_like(pad) for _ in range(world)]
+    dist.all_gather(parts, pad, group=group)
+    full = torch.empty((B, H_kv * group_size) + rest, dtype=local.dtype, device=local.device)
+    for part, (b0, b1, h0, h1) in zip(parts, blocks):
+        full[b0:b1, h0 * group_size:h1 * group_size] = part[: b1 - b0, : (h1 - h0) * group_size]
+    return full
 
 
 def max_over_ranks(value, device=None, group=None):
@@ -86,46 +146,43 @@ def local_state_update(k, v, seg_len, state_update, dtype=torch.float32):
     return torch.cat([dM.flatten(), dz.flatten()])
 
 
-def prefix_states(updates, rank, M0, z0):
+def prefix_states(updates, rank, M0, z0, state_sum):
     """(M_in, z_in) of `rank` and the final (M_T, z_T) from the gathered
-    per-rank updates (a list in rank order): M0 plus the updates of ranks
-    before `rank`, and plus all of them, added one rank at a time in float32."""
-    nM = M0.numel()
-    M_in, z_in = M0.clone(), z0.clone()
-    M_T, z_T = M0.clone(), z0.clone()
-    for r, u in enumerate(updates):
-        dM = u[:nM].view_as(M0)
-        dz = u[nM:].view_as(z0)
-        if r < rank:
-            M_in += dM
-            z_in += dz
-        M_T += dM
-        z_T += dz
+    per-rank updates (`updates`: [world, packed], rank order): M0 plus the
+    updates of ranks before `rank`, and plus all of them.  `state_sum` is the
+    library call (M_base, z_base, parts, n_parts) -> (M, z), which adds the
+    parts in order (api.state_sum)."""
+    M_in, z_in = state_sum(M0, z0, updates, rank)
+    M_T, z_T = state_sum(M0, z0, updates, updates.shape[0])
     return M_in, z_in, M_T, z_T
 
 
 def all_gather_flat(t, group=None):
-    """All-gather equal-size flat tensors, in rank order (one rank: [t])."""
+    """All-gather equal-size flat tensors into one [world, n] tensor in rank
+    order (one rank: [1, n])."""
+    t = t.contiguous().view(1, -1)
     if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size(group) == 1:
-        return [t]
+        return t
     parts = [torch.empty_like(t) for _ in range(dist.get_world_size(group))]
-    dist.all_gather(parts, t.contiguous(), group=group)
-    return parts
+    dist.all_gather(parts, t, group=group)
+    return torch.cat(parts, dim=0)
 
 
-def sequence_parallel_forward(q, k, v, beta, M0, z0, seg_len, forward, state_update, group=None):
+def sequence_parallel_forward(q, k, v, beta, M0, z0, seg_len, forward, state_update, state_sum,
+                              group=None):
     """Linear-rule forward of this rank's run of segments.
 
     q, k, v: the rank's token rows [l0, l1) from segment_range (B, heads and d
-    as for the whole sequence); M0, z0: the state before token 0.  `forward`
-    and `state_update` are the library calls (api.forward, api.state_update).
-    Returns (out for the rank's rows, M_T, z_T) with the state after the whole
-    sequence on every rank.  One all-gather of B * H_kv * (d_k d_v + d_k)
-    floats per rank is the only exchange.
+    as for the whole sequence); M0, z0: the state before token 0.  `forward`,
+    `state_update` and `state_sum` are the library calls (api.forward,
+    api.state_update, api.state_sum).  Returns (out for the rank's rows, M_T,
+    z_T) with the state after the whole sequence on every rank.  One
+    all-gather of B * H_kv * (d_k d_v + d_k) floats per rank is the only
+    exchange.
     """
     updates = all_gather_flat(local_state_update(k, v, seg_len, state_update, M0.dtype), group)
     rank = dist.get_rank(group) if dist.is_available() and dist.is_initialized() else 0
-    M_in, z_in, M_T, z_T = prefix_states(updates, rank, M0, z0)
+    M_in, z_in, M_T, z_T = prefix_states(updates, rank, M0, z0, state_sum)
     if q.shape[2] == 0:
         return q.new_empty(q.shape[:3] + (v.shape[3],)), M_T, z_T
     out, _, _ = forward(q, k, v, beta, M_in, z_in, seg_len, "linear")

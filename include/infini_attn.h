@@ -180,6 +180,29 @@ INFINI_API int infini_attn_state_update(const void* k, const void* v, const floa
                                         const infini_dims_t* dims, float* M_out, float* z_out,
                                         void* workspace, size_t workspace_bytes, void* stream);
 
+/* Sum of memory states: the exchange step of the sequence-parallel linear
+ * rule, where the memory after a run of segments is the memory before it
+ * plus the run's own update from a zero state ("Hugging Face
+ * Infini-Attention 再現分析", Memory Update: the contributions accumulate).
+ *   M_out = M_base + M(parts[0]) + ... + M(parts[n_parts - 1]),
+ *   z_out = z_base + z(parts[0]) + ... + z(parts[n_parts - 1]),
+ * every element added in fp32 in that order (bitwise deterministic).
+ *   M_base, z_base   device float32 [B, H_kv, d_k, d_v] and [B, H_kv, d_k]
+ *   parts            device float32, n_parts consecutive packed states, each
+ *                    [M (B*H_kv*d_k*d_v floats) | z (B*H_kv*d_k floats)]
+ *                    (the updates of infini_attn_state_update, gathered in
+ *                    rank order); may be NULL when n_parts == 0
+ *   n_parts          >= 0 (0 copies the base)
+ *   M_out, z_out     device float32, shapes of M_base / z_base; may equal
+ *                    M_base / z_base (in place); no other overlap
+ *   stream           cudaStream_t; asynchronous.
+ * All pointers must be memory of the current device and 16-byte aligned.
+ * Errors: INFINI_ERR_ARG (NULL pointer, size < 1, n_parts < 0),
+ * INFINI_ERR_ALIGN, INFINI_ERR_ALIAS, INFINI_ERR_CUDA. */
+INFINI_API int infini_attn_state_sum(const float* M_base, const float* z_base, const float* parts,
+                                     int n_parts, int B, int H_kv, int d_k, int d_v, float* M_out,
+                                     float* z_out, void* stream);
+
 /* Streaming decode: the layer forward one token at a time.  The current
  * segment's keys and values so far are kept by the caller in a rolling
  * buffer of seg_len rows per KV head; (M, z) hold the memory of the segments
@@ -282,10 +305,18 @@ INFINI_API int infini_attn_kernel_times(double* ms, int* launches, int n_kinds, 
  *     (a 1M-token stream does; the tiny, 200M-, 300M- and 8B-shaped
  *     workloads fit).
  *   - The call allocates nothing: no cudaMalloc, cudaMallocAsync or
- *     allocating library routine.
- *   - The first call on each device looks up the array's device address
- *     (cudaGetSymbolAddress, with that device current); make that first call
- *     before any stream capture.
+ *     allocating library routine.  Every pointer must be memory of the
+ *     current device, and the stream must belong to it.
+ *   - Every call looks up the array's device address on the current device
+ *     (cudaGetSymbolAddress); the address is not cached, so the call stays
+ *     valid after cudaDeviceReset.
+ *   - First call per device: CUDA loads GPU code lazily by default
+ *     (CUDA_MODULE_LOADING=LAZY), so the first call on a device loads the
+ *     library's modules it uses, which commits device memory for their code
+ *     and for the 64 MiB array.  Make that first call as a warm-up, with the
+ *     same shape, outside any region where allocation is forbidden and before
+ *     any stream capture (or run the process with CUDA_MODULE_LOADING=EAGER).
+ *     Later calls of that shape commit no device memory.
  *   - All calls on a device share the one array and it keeps the last call's
  *     contents; nothing in it needs clearing (every byte read is written
  *     earlier in the same call).  Calls whose GPU work overlaps -- on two

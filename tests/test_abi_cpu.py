@@ -165,3 +165,29 @@ def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
     monkeypatch.setattr(api, "_lib", None)
     with pytest.raises(FileNotFoundError):
         api.load_library(str(tmp_path / "missing.so"))
+
+
+def test_state_sum_rejects_bad_arguments_on_the_host(lib):
+    """Argument checks of infini_attn_state_sum return before any CUDA call."""
+    P = ctypes.c_void_p
+    MB = 1 << 20
+    n_M, n_z = 2 * 3 * 8 * 8 * 4, 2 * 3 * 8 * 4
+    base = (P(MB), P(2 * MB))
+    assert lib.infini_attn_state_sum(P(0), P(2 * MB), P(0), 0, 2, 3, 8, 8, P(3 * MB), P(4 * MB),
+                                     P(0)) == api.ERR_ARG
+    assert lib.infini_attn_state_sum(*base, P(0), 2, 2, 3, 8, 8, P(3 * MB), P(4 * MB),
+                                     P(0)) == api.ERR_ARG  # parts NULL with n_parts > 0
+    assert lib.infini_attn_state_sum(*base, P(0), -1, 2, 3, 8, 8, P(3 * MB), P(4 * MB),
+                                     P(0)) == api.ERR_ARG
+    assert lib.infini_attn_state_sum(*base, P(0), 0, 0, 3, 8, 8, P(3 * MB), P(4 * MB),
+                                     P(0)) == api.ERR_ARG
+    assert lib.infini_attn_state_sum(*base, P(0), 0, 2, 3, 8, 8, P(3 * MB + 4), P(4 * MB),
+                                     P(0)) == api.ERR_ALIGN
+    # M_out overlapping z_out, or the parts, or another state's base
+    assert lib.infini_attn_state_sum(*base, P(0), 0, 2, 3, 8, 8, P(3 * MB), P(3 * MB + n_M - 16),
+                                     P(0)) == api.ERR_ALIAS
+    assert lib.infini_attn_state_sum(*base, P(5 * MB), 1, 2, 3, 8, 8, P(5 * MB + 64), P(4 * MB),
+                                     P(0)) == api.ERR_ALIAS
+    assert lib.infini_attn_state_sum(*base, P(0), 0, 2, 3, 8, 8, P(MB + 16), P(4 * MB),
+                                     P(0)) == api.ERR_ALIAS
+    assert n_z < n_M

@@ -73,6 +73,81 @@ def test_two_rank_gloo_sharding_matches_single_process():
     assert results[0][2] == (0, 2) and results[1][2] == (2, 3)
 
 
+# ------------------------------------------- (batch row, KV head) chain blocks
+
+def test_chain_blocks_tile_the_grid():
+    for B, H_kv in ((1, 32), (2, 8), (1, 4), (2, 3), (8, 12), (4, 16), (3, 5)):
+        for world in range(1, 17):
+            try:
+                blocks = [shard.chain_block(B, H_kv, world, r) for r in range(world)]
+            except ValueError:
+                assert world > B * H_kv or all(world % wh or world // wh > B
+                                               for wh in range(1, min(world, H_kv) + 1))
+                continue
+            seen = np.zeros((B, H_kv), dtype=int)
+            for b0, b1, h0, h1 in blocks:
+                assert b1 > b0 and h1 > h0
+                seen[b0:b1, h0:h1] += 1
+            assert np.all(seen == 1), (B, H_kv, world)
+    # One long stream (B = 1) splits over its KV heads; exact splits come first.
+    assert shard.split_factors(1, 32, 8) == (1, 8)
+    assert shard.split_factors(2, 8, 16) == (2, 8)
+    assert shard.split_factors(2, 3, 2) == (2, 1)
+
+
+_CHAIN_CASES = {"one_stream": (1, 8, 4), "two_rows": (2, 6, 3)}  # (B, H_q, H_kv)
+
+
+def _chain_worker(rank, world, port, case, results):
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        B, H_q, H_kv = _CHAIN_CASES[case]
+        L, d, S, g = 40, 8, 16, H_q // H_kv
+        rng = np.random.default_rng(11)  # same full problem on every rank
+        q = rng.standard_normal((B, H_q, L, d))
+        k = rng.standard_normal((B, H_kv, L, d))
+        v = rng.standard_normal((B, H_kv, L, d))
+        beta = rng.uniform(-2, 2, H_q)
+        M0 = rng.standard_normal((B, H_kv, d, d))
+        z0 = rng.uniform(0.5, 2.0, (B, H_kv, d))
+        block = shard.chain_block(B, H_kv, world, rank)
+        t = torch.from_numpy
+        h0, h1 = block[2], block[3]
+        out, M, z = oracle.infini_attention_forward(
+            shard.shard_chains(t(q), block, g).numpy(), shard.shard_chains(t(k), block).numpy(),
+            shard.shard_chains(t(v), block).numpy(), beta[h0 * g:h1 * g],
+            shard.shard_chains(t(M0), block).numpy(), shard.shard_chains(t(z0), block).numpy(),
+            S, "delta")
+        full = (shard.gather_chains(t(out), B, H_kv, world, g), shard.gather_chains(t(M), B, H_kv, world),
+                shard.gather_chains(t(z), B, H_kv, world))
+        ref = oracle.infini_attention_forward(q, k, v, beta, M0, z0, S, "delta")
+        results[rank] = (all(torch.equal(a, t(r)) for a, r in zip(full, ref)), block)
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("case,world", [("one_stream", 2), ("one_stream", 3), ("two_rows", 2),
+                                        ("two_rows", 3)])
+def test_chain_block_sharding_gloo(case, world):
+    """Every rank runs the layer (float64 oracle as the per-rank compute) on its
+    block of (batch row, KV head) chains, with the query heads of its groups;
+    the gathered output and final state equal the single-process forward
+    exactly."""
+    port = _free_port()
+    ctx = mp.get_context("spawn")
+    results = ctx.Manager().dict()
+    mp.start_processes(_chain_worker, args=(world, port, case, results), nprocs=world, join=True,
+                       start_method="spawn")
+    assert sorted(results.keys()) == list(range(world))
+    for r in range(world):
+        ok, block = results[r]
+        assert ok, (r, block)
+    if case == "one_stream":  # B = 1: the split is over KV heads
+        assert all(results[r][1][:2] == (0, 1) for r in range(world))
+
+
 # ------------------------------------------- sequence parallelism (linear rule)
 
 def _oracle_forward(q, k, v, beta, M_in, z_in, S, rule):
@@ -86,6 +161,17 @@ def _oracle_state_update(k, v, M_in, z_in, S, rule):
     q = torch.zeros((B, H_kv, L, d_k), dtype=torch.float64)
     beta = torch.zeros(H_kv, dtype=torch.float64)
     _, M, z = _oracle_forward(q, k, v, beta, M_in, z_in, S, rule)
+    return M, z
+
+
+def _host_state_sum(M_base, z_base, parts, n_parts):
+    """The sum the library's state_sum forms, on host tensors (test stand-in
+    for the CUDA call): base plus the first n_parts packed states, in order."""
+    nM = M_base.numel()
+    M, z = M_base.clone(), z_base.clone()
+    for p in range(n_parts):
+        M += parts[p, :nM].view_as(M)
+        z += parts[p, nM:].view_as(z)
     return M, z
 
 
@@ -113,7 +199,8 @@ def _sp_worker(rank, world, port, results):
         t = torch.from_numpy
         out, M_T, z_T = shard.sequence_parallel_forward(
             t(q[:, :, l0:l1].copy()), t(k[:, :, l0:l1].copy()), t(v[:, :, l0:l1].copy()), t(beta),
-            t(M0), t(z0), S, forward=_oracle_forward, state_update=_oracle_state_update)
+            t(M0), t(z0), S, forward=_oracle_forward, state_update=_oracle_state_update,
+            state_sum=_host_state_sum)
         ref_out, ref_M, ref_z = oracle.infini_attention_forward(q, k, v, beta, M0, z0, S, "linear")
         results[rank] = ((l0, l1),
                          float(np.max(np.abs(out.numpy() - ref_out[:, :, l0:l1]), initial=0.0)),
@@ -139,12 +226,12 @@ def test_segment_range_partition():
 def test_prefix_states_in_rank_order():
     M0 = torch.full((1, 1, 2, 2), 1.0, dtype=torch.float64)
     z0 = torch.full((1, 1, 2), 2.0, dtype=torch.float64)
-    ups = [torch.cat([torch.full((4,), float(10 ** r)), torch.full((2,), float(r))]).double()
-           for r in range(3)]
-    M_in, z_in, M_T, z_T = shard.prefix_states(ups, 2, M0, z0)
+    ups = torch.stack([torch.cat([torch.full((4,), float(10 ** r)), torch.full((2,), float(r))])
+                       for r in range(3)]).double()
+    M_in, z_in, M_T, z_T = shard.prefix_states(ups, 2, M0, z0, _host_state_sum)
     assert torch.all(M_in == 12.0) and torch.all(z_in == 3.0)
     assert torch.all(M_T == 112.0) and torch.all(z_T == 5.0)
-    M_in, z_in, _, _ = shard.prefix_states(ups, 0, M0, z0)
+    M_in, z_in, _, _ = shard.prefix_states(ups, 0, M0, z0, _host_state_sum)
     assert torch.equal(M_in, M0) and torch.equal(z_in, z0)
 
 

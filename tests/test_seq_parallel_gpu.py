@@ -90,11 +90,11 @@ def test_sequence_parallel_linear_rule(cuda_lib, name, over, world):
     q, k, v, beta, M0, z0 = _tensors(w, inp)
     runs = [shard.segment_range(w.L, w.seg_len, world, r) for r in range(world)]
     # each virtual rank's update of its run (the all-gather, stacked here)
-    updates = [shard.local_state_update(k[:, :, a:b].contiguous(), v[:, :, a:b].contiguous(),
-                                        w.seg_len, api.state_update) for a, b in runs]
+    updates = torch.stack([shard.local_state_update(k[:, :, a:b].contiguous(), v[:, :, a:b].contiguous(),
+                                                    w.seg_len, api.state_update) for a, b in runs])
     outs = []
     for r, (a, b) in enumerate(runs):
-        M_in, z_in, M_T, z_T = shard.prefix_states(updates, r, M0, z0)
+        M_in, z_in, M_T, z_T = shard.prefix_states(updates, r, M0, z0, api.state_sum)
         o, _, _ = api.forward(q[:, :, a:b].contiguous(), k[:, :, a:b].contiguous(),
                               v[:, :, a:b].contiguous(), beta, M_in, z_in, w.seg_len, "linear")
         outs.append(o)
@@ -105,3 +105,26 @@ def test_sequence_parallel_linear_rule(cuda_lib, name, over, world):
     assert err <= TOL_OUT[w.dtype], err
     em, ez = state_rel_errors(M_T.cpu().numpy(), z_T.cpu().numpy(), rM, rz)
     assert em <= TOL_STATE and ez <= TOL_STATE, (em, ez)
+
+
+def test_state_sum_adds_parts_in_order(cuda_lib):
+    """infini_attn_state_sum against the same fp32 additions done one part at a
+    time (bitwise: the library adds each element in part order), in place and
+    out of place, with zero parts copying the base."""
+    api = cuda_lib
+    g = torch.Generator(device="cuda").manual_seed(3)
+    B, H_kv, d_k, d_v, n = 2, 3, 64, 32, 5
+    M0 = torch.randn((B, H_kv, d_k, d_v), generator=g, device="cuda")
+    z0 = torch.rand((B, H_kv, d_k), generator=g, device="cuda")
+    parts = torch.randn((n, B * H_kv * d_k * (d_v + 1)), generator=g, device="cuda")
+    nM = M0.numel()
+    for k_ in (0, 1, 3, n):
+        M, z = api.state_sum(M0, z0, parts, k_)
+        rM, rz = M0.clone(), z0.clone()
+        for p in range(k_):
+            rM += parts[p, :nM].view_as(M0)
+            rz += parts[p, nM:].view_as(z0)
+        assert torch.equal(M, rM) and torch.equal(z, rz)
+    Mi, zi = M0.clone(), z0.clone()
+    api.state_sum(Mi, zi, parts, n, M_out=Mi, z_out=zi)
+    assert torch.equal(Mi, rM) and torch.equal(zi, rz)
