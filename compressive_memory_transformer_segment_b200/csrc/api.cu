@@ -142,6 +142,12 @@ unsigned int* status_ptr() {
   return static_cast<unsigned int*>(p);
 }
 
+// The state scan of the path `s` takes.
+cudaError_t launch_state_scan(const Shape& s, const Problem& p, cudaStream_t st) {
+  if (s.path != INFINI_PATH_TCGEN05) return launch_simt_state_scan(p, st);
+  return launch_tc_state_scan(p, st);
+}
+
 // The forward's state scan alone over (k, v) of shape `s`: (M_in, z_in) ->
 // (M_out, z_out), per-segment states in the workspace `ws` (laid out by
 // check_shape).
@@ -161,10 +167,7 @@ cudaError_t run_state_scan(const Shape& s, const void* k, const void* v, const f
   p.dz = reinterpret_cast<float*>(ws + s.ws_dz);
   p.status = status;
   cudaError_t e = cudaMemcpyAsync(p.z_pref, z_in, s.z_bytes, cudaMemcpyDeviceToDevice, st);
-  if (e == cudaSuccess)
-    e = timed(0, st, [&] {
-      return s.path == INFINI_PATH_TCGEN05 ? launch_tc_state_scan(p, st) : launch_simt_state_scan(p, st);
-    });
+  if (e == cudaSuccess) e = timed(0, st, [&] { return launch_state_scan(s, p, st); });
   return e;
 }
 
@@ -302,10 +305,7 @@ int infini_attn_forward(const void* q, const void* k, const void* v, const float
   p.status = status;
 
   cudaError_t e = cudaMemcpyAsync(p.z_pref, z_in, s.z_bytes, cudaMemcpyDeviceToDevice, st);
-  if (e == cudaSuccess)
-    e = timed(0, st, [&] {
-      return s.path == INFINI_PATH_TCGEN05 ? launch_tc_state_scan(p, st) : launch_simt_state_scan(p, st);
-    });
+  if (e == cudaSuccess) e = timed(0, st, [&] { return launch_state_scan(s, p, st); });
   if (e == cudaSuccess)
     e = timed(1, st, [&] {
       return s.path == INFINI_PATH_TCGEN05 ? launch_tc_attention(p, st) : launch_simt_attention(p, st);

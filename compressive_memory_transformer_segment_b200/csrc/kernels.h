@@ -36,8 +36,12 @@ cudaError_t launch_simt_state_scan(const Problem& p, cudaStream_t stream);
 cudaError_t launch_simt_attention(const Problem& p, cudaStream_t stream);
 
 // Tensor-core (tcgen05 / TMEM / TMA) segment attention: bf16 I/O,
-// d_k == d_v in {64, 128}, S a multiple of 128.  Reads bf16 M_pref.
+// d_k == d_v in {64, 128}, S a multiple of 128 (persistent kernel) or a
+// divisor of 128 with (128 / S) * d <= 256 (short-segment kernel).  Reads
+// bf16 M_pref.
 bool tc_attention_supported(int d_k, int d_v, int S, bool bf16);
+bool tc_small_attention_supported(int d_k, int d_v, int S, bool bf16);
+cudaError_t launch_tc_small_attention(const Problem& p, cudaStream_t stream);
 // Device address of the status word the kernels set (see common.cuh).
 unsigned int* device_status_word();
 

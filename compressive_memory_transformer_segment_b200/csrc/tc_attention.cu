@@ -12,32 +12,37 @@
 //
 // Persistent kernel, one CTA per SM.  A work item is a PAIR of query tiles
 // that read the same keys: two query heads of one KV group at the same tile
-// position, or (one query head per KV head) two neighbouring tiles of one
-// head.  The pair's two tiles ("slots" A and B) each have their own softmax
-// warpgroup and TMEM columns and take turns with the tensor core: while one
-// slot's softmax runs, the tensor core computes the other slot's P.V and next
-// scores.  Items are taken round-robin (item = CTA + k * grid), ordered by
-// (segment, batch row, KV head) group and, inside a group, heaviest first, so
-// the CTAs working at any moment share a few groups' keys in L2.
+// position.  The pair's two tiles ("slots" A and B) each have their own
+// softmax warpgroup and TMEM columns and take turns with the tensor core:
+// while one slot's softmax runs, the tensor core computes the other slot's
+// P.V and next scores.  Items are ordered by (segment, batch row, KV head)
+// group and, inside a group, heaviest first; they are handed out round-robin
+// in units of two, an item and its mirror image in the group's order
+// (heaviest with lightest), so that every unit costs the same and the CTAs,
+// which work on a few neighbouring groups at any moment, share those groups'
+// keys in L2.  (With one query head per KV head the one-tile-per-CTA kernel
+// runs instead.)
 //
 // Roles (384 threads, three warpgroups; the first gives registers to the
 // other two with setmaxnreg):
-//   warp 0      TMA producer: per item K_0, V_0, the next item's two Q
-//               tiles (double-buffered), K_1, V_1, ..., then M_{s-1}, through
-//               a ring of shared-memory slots.
-//   warp 1      allocates TMEM; one thread issues every tcgen05.mma with the
-//               operand descriptors precomputed per group of MMAs:
+//   warp 0      TMA producer: per item K_0, V_0, K_1, V_1, ..., M_{s-1}
+//               through a ring of shared-memory slots, and, early in the
+//               item, the next item's two query tiles (double-buffered), each
+//               with its z_{s-1} (a bulk copy on the tile's barrier).
+//   warp 1      allocates TMEM; one thread issues every tcgen05.mma:
 //               S_j = Q K_j^T, O += P_j V_j (P read from TMEM), and at the end
-//               of the item R = sigma(Q) M_{s-1} into the score columns.  A
-//               slot's P.V and next QK^T go back to back (16 MMAs at d = 128).
+//               of the item R' = (sigma(Q) c) M_{s-1} into O, then the next
+//               item's first S.  A slot's P.V and next QK^T go back to back.
 //   warps 2, 3  idle.
 //   warps 4..7  slot A, warps 8..11 slot B: one thread per query row.  Online
 //               softmax in base 2 on the scores in TMEM (the first tile's row
 //               max is the reference; it moves, and O is rescaled, only when
 //               a tile's sum exceeds 2^16); P (bf16) written over the scores;
-//               then sigma(Q) in place of Q with the fp32 retrieval
-//               denominator sigma(q).z, and the gated output stored from
-//               registers.
+//               the retrieval denominator sigma(q).z while the tensor core
+//               works on the first tile; at the end the retrieval rows
+//               sigma(Q) c in place of Q (the retrieval is folded into O, see
+//               the epilogue), the read-out of O, and one TMA store of the
+//               output tile staged in the query tile's buffer.
 // TMEM (512 columns): slot A S = [0, 128), O = [128, 128 + D);
 //                     slot B S = [256, 384), O = [384, 384 + D).
 #include <cuda.h>
@@ -54,8 +59,11 @@ using namespace tc;
 constexpr int kBM = 128;  // query rows per tile
 constexpr int kBN = 128;  // keys per K/V tile
 constexpr int kThreads = 384;
-constexpr int kRegsRoles = 120;   // per thread, warpgroup 0 (producer, MMA)
-constexpr int kRegsSoftmax = 192; // per thread, warpgroups 1 and 2
+// Registers per thread after setmaxnreg: 384 x 168 at launch =
+// 128 x kRegsRoles + 256 x kRegsSoftmax.
+constexpr int kRegsRoles = 104;    // warpgroup 0 (producer, MMA)
+constexpr int kRegsSoftmax = 200;  // warpgroups 1 and 2
+static_assert(128 * kRegsRoles + 256 * kRegsSoftmax <= kThreads * 168, "registers");
 constexpr uint32_t kTmemCols = 512;
 constexpr int kSmemLimit = 232448;  // opt-in dynamic shared memory per block
 
@@ -67,9 +75,9 @@ struct Smem {
   static constexpr int kQ = 0;
   static constexpr int kRingOff = 4 * kTile;
   static constexpr int kBar = kRingOff + kRing * kTile;
-  // ring full[kRing], ring empty[kRing], q_full[4] q_empty[4] (per Q
-  // tile), then two (one per slot) of each of s_full p_ready sq_ready r_full
-  // tmem_free z_ready, then drain.
+  // ring full[kRing], ring empty[kRing], q_full[4] q_empty[4] (per Q tile,
+  // with its z), then two (one per slot) of each of s_full p_ready sq_ready
+  // r_full tmem_free o_staged, then drain.
   static constexpr int kFull = 0;
   static constexpr int kEmpty = kRing;
   static constexpr int kQFull = 2 * kRing;
@@ -79,12 +87,13 @@ struct Smem {
   static constexpr int kSqReady = kPReady + 2;
   static constexpr int kRFull = kSqReady + 2;
   static constexpr int kTFree = kRFull + 2;
-  static constexpr int kZReady = kTFree + 2;
-  static constexpr int kDrain = kZReady + 2;
+  static constexpr int kOStaged = kTFree + 2;
+  static constexpr int kDrain = kOStaged + 2;
   static constexpr int kNumBars = kDrain + 1;
-  // z_{s-1} per slot, fp32 [2][D], read as float4: 128-byte aligned.
+  // z_{s-1} per query tile, fp32 [4][D] (copied in with the tile), read as
+  // float4: 128-byte aligned.
   static constexpr int kZ = (kBar + kNumBars * 8 + 127) / 128 * 128;
-  static constexpr int kTmemSlot = kZ + 2 * D * 4;
+  static constexpr int kTmemSlot = kZ + 4 * D * 4;
   static constexpr int kAbort = kTmemSlot + 4;
   // The dynamic shared memory base is 1024-byte aligned (checked at entry).
   static constexpr int kAlloc = kAbort + 4;
@@ -95,24 +104,41 @@ struct Smem {
 
 // One work item: a (segment, batch row, KV head) group and two query tiles
 // of it (slot x: query head h[x], tile qt[x], n[x] key tiles; n[x] = 0 for
-// an empty slot).
+// an empty slot).  Both slots read key tiles 0 .. n_max - 1.
 struct Item {
   int s, b, h_kv, seg0, seg_len;
   int h[2], qt[2], n[2];
   int n_max;
 };
 
+// n / d for 0 <= n < 2^31 as a multiply and a shift: m = ceil(2^(31 + l) / d),
+// l = ceil(log2 d) (exact there: the rounding error of m stays below one
+// step of n / d).
+struct FastDiv {
+  uint32_t m, sh;
+};
+__host__ __device__ inline FastDiv make_fastdiv(uint32_t d) {
+  uint32_t l = 0;
+  while ((1ull << l) < d) ++l;
+  return FastDiv{(uint32_t)(((1ull << (31 + l)) + d - 1) / d), 31 + l};
+}
+__device__ __forceinline__ int fdiv(int n, FastDiv f) {
+  return (int)(((unsigned long long)(uint32_t)n * f.m) >> f.sh);
+}
+
 struct Shape {
-  int B, H_q, H_kv, L, S, T, g, tps, per_group, items;
+  int B, H_q, H_kv, L, S, T, g, tps, per_group, upg, units;
+  FastDiv by_per_group, by_upg, by_H_kv, by_B;
 };
 
 __device__ __forceinline__ Item decode_item(int idx, const Shape& sh) {
   Item it;
-  const int group = idx / sh.per_group;
+  const int group = fdiv(idx, sh.by_per_group);
   const int p = idx - group * sh.per_group;
-  it.h_kv = group % sh.H_kv;
-  it.b = (group / sh.H_kv) % sh.B;
-  it.s = group / (sh.H_kv * sh.B);
+  const int gb = fdiv(group, sh.by_H_kv);  // group / H_kv
+  it.h_kv = group - gb * sh.H_kv;
+  it.s = fdiv(gb, sh.by_B);
+  it.b = gb - it.s * sh.B;
   it.seg0 = it.s * sh.S;
   it.seg_len = min(sh.S, sh.L - it.seg0);
   it.n_max = 0;
@@ -132,6 +158,31 @@ __device__ __forceinline__ Item decode_item(int idx, const Shape& sh) {
     it.n_max = max(it.n_max, it.n[x]);
   }
   return it;
+}
+
+// The CTA's k-th item.  Work is handed out in units, round-robin (unit =
+// CTA + (k / 2) * grid); a unit is the item at position r of its group and
+// the item at the mirrored position per_group - 1 - r (empty when the two
+// coincide).  Positions run from the heaviest item to the lightest, so every
+// unit holds about the same number of key tiles (tps + 1 when every tile is
+// full) and the CTAs finish together.
+__device__ __forceinline__ bool seq_valid(int k, const Shape& sh) {
+  return (int)blockIdx.x + (k >> 1) * (int)gridDim.x < sh.units;
+}
+
+__device__ __forceinline__ Item seq_item(int k, const Shape& sh) {
+  const int u = (int)blockIdx.x + (k >> 1) * (int)gridDim.x;
+  const int group = fdiv(u, sh.by_upg), r = u - group * sh.upg;
+  const int p = (k & 1) ? sh.per_group - 1 - r : r;
+  if ((k & 1) && p == r) {
+    Item it;
+    it.s = it.b = it.h_kv = it.seg0 = it.seg_len = 0;
+    it.h[0] = it.h[1] = it.qt[0] = it.qt[1] = 0;
+    it.n[0] = it.n[1] = 0;
+    it.n_max = 0;
+    return it;
+  }
+  return decode_item(group * sh.per_group + p, sh);
 }
 
 // Arrival of a whole warp on an mbarrier counted per warp: the warp's
@@ -166,6 +217,9 @@ __device__ __forceinline__ float row_max128(const uint32_t* a, const uint32_t* b
 // P = 2^(s * sl2 - m) for 64 scores (fp32 bit patterns), as 32 bf16 pairs;
 // returns the sum of the fp32 values.  Three pairs in four go to the MUFU
 // unit, one to the FMA pipe (exp2_poly2), which spreads 2^x over both.
+// MASKED (a diagonal tile, whose masked scores are -inf): masked keys get
+// exactly 0 on both pipes.
+template <bool MASKED>
 __device__ __forceinline__ float exp_pack64(const uint32_t* sv, float sl2, float m, uint32_t* packed) {
   const float2 sc2 = make_float2(sl2, sl2), nm2 = make_float2(-m, -m);
   float2 acc2[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
@@ -174,7 +228,7 @@ __device__ __forceinline__ float exp_pack64(const uint32_t* sv, float sl2, float
     const float2 xx = __ffma2_rn(make_float2(__uint_as_float(sv[2 * i]), __uint_as_float(sv[2 * i + 1])), sc2, nm2);
     float2 p;
     if ((i & 3) == 3) {
-      p = exp2_poly2(xx);
+      p = exp2_poly2<MASKED>(xx);
     } else {
       p.x = ex2_approx(xx.x);
       p.y = ex2_approx(xx.y);
@@ -185,12 +239,76 @@ __device__ __forceinline__ float exp_pack64(const uint32_t* sv, float sl2, float
   return (acc2[0].x + acc2[0].y) + (acc2[1].x + acc2[1].y);
 }
 
+// sigma(x) = x + 1 (x > 0), e^x (x <= 0) of a bf16 pair, in fp32; e^x as
+// 2^(x log2 e) on the MUFU unit or (POLY) on the FMA pipe.
+template <bool POLY>
+__device__ __forceinline__ float2 sigma2(uint32_t w) {
+  const float2 xv = make_float2(bf16lo_to_f32(w), bf16hi_to_f32(w));
+  const float2 xe = make_float2(xv.x * 1.4426950408889634f, xv.y * 1.4426950408889634f);
+  float2 e;
+  if (POLY) {
+    e = exp2_poly2<false>(xe);
+  } else {
+    e.x = ex2_approx(xe.x);
+    e.y = ex2_approx(xe.y);
+  }
+  return make_float2(xv.x > 0.f ? xv.x + 1.f : e.x, xv.y > 0.f ? xv.y + 1.f : e.y);
+}
+
+// The retrieval denominator of row r: sigma(q_r) . z_{s-1} in fp32 from the
+// unrounded sigma (q_r: row r of a 128-row query tile in shared memory; z in
+// shared memory, read as float4).  Loads go four 16-byte chunks at a time,
+// ahead of the arithmetic.
+template <int D>
+__device__ __forceinline__ float sigma_dot_z(const unsigned char* sQ, int r, const float* zs) {
+  float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll 2
+  for (int c8 = 0; c8 < D / 8; c8 += 4) {
+    uint4 v[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) v[i] = *reinterpret_cast<const uint4*>(sQ + sw128_offset(r, (c8 + i) * 8, kBM));
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const float4 za = reinterpret_cast<const float4*>(zs)[2 * (c8 + i)];
+      const float4 zb = reinterpret_cast<const float4*>(zs)[2 * (c8 + i) + 1];
+      const float2 s0 = sigma2<false>(v[i].x), s1 = sigma2<true>(v[i].y);
+      const float2 s2 = sigma2<false>(v[i].z), s3 = sigma2<true>(v[i].w);
+      acc[i] = fmaf(s0.y, za.y, fmaf(s0.x, za.x, acc[i]));
+      acc[i] = fmaf(s1.y, za.w, fmaf(s1.x, za.z, acc[i]));
+      acc[i] = fmaf(s2.y, zb.y, fmaf(s2.x, zb.x, acc[i]));
+      acc[i] = fmaf(s3.y, zb.w, fmaf(s3.x, zb.z, acc[i]));
+    }
+  }
+  return (acc[0] + acc[1]) + (acc[2] + acc[3]);
+}
+
+// Row r of the query tile replaced, in place, by bf16(sigma(q_r) * c), four
+// 16-byte chunks at a time.
+template <int D>
+__device__ __forceinline__ void sigma_scale_row(unsigned char* sQ, int r, float c) {
+#pragma unroll 2
+  for (int c8 = 0; c8 < D / 8; c8 += 4) {
+    uint4 v[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) v[i] = *reinterpret_cast<const uint4*>(sQ + sw128_offset(r, (c8 + i) * 8, kBM));
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const float2 s0 = sigma2<false>(v[i].x), s1 = sigma2<true>(v[i].y);
+      const float2 s2 = sigma2<false>(v[i].z), s3 = sigma2<true>(v[i].w);
+      v[i] = make_uint4(pack_bf16x2(s0.x * c, s0.y * c), pack_bf16x2(s1.x * c, s1.y * c),
+                        pack_bf16x2(s2.x * c, s2.y * c), pack_bf16x2(s3.x * c, s3.y * c));
+    }
+#pragma unroll
+    for (int i = 0; i < 4; ++i) *reinterpret_cast<uint4*>(sQ + sw128_offset(r, (c8 + i) * 8, kBM)) = v[i];
+  }
+}
+
 template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
 tc_attention(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
              const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_m,
-             const float* __restrict__ z_pref, const float* __restrict__ beta,
-             __nv_bfloat16* __restrict__ out, unsigned int* __restrict__ status, const Shape sh) {
+             const __grid_constant__ CUtensorMap tm_o, const float* __restrict__ z_pref,
+             const float* __restrict__ beta, unsigned int* __restrict__ status, const Shape sh) {
   using SM = Smem<D>;
   constexpr int kPanels = D / 64;
   constexpr uint32_t kTileBytes = SM::kTile;
@@ -216,7 +334,7 @@ tc_attention(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
   uint64_t* sq_ready = bars + SM::kSqReady;
   uint64_t* r_full = bars + SM::kRFull;
   uint64_t* tmem_free = bars + SM::kTFree;
-  uint64_t* z_ready = bars + SM::kZReady;
+  uint64_t* o_staged = bars + SM::kOStaged;
   uint64_t* drain = bars + SM::kDrain;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + SM::kTmemSlot);
   volatile int* abort = reinterpret_cast<volatile int*>(smem + SM::kAbort);
@@ -238,7 +356,7 @@ tc_attention(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
       mbar_init(sq_ready + x, 4);
       mbar_init(r_full + x, 1);
       mbar_init(tmem_free + x, 4);
-      mbar_init(z_ready + x, 4);
+      mbar_init(o_staged + x, 4);
     }
     mbar_init(drain, 1);
     *abort = 0;
@@ -249,6 +367,7 @@ tc_attention(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
     tma_prefetch_desc(&tm_k);
     tma_prefetch_desc(&tm_v);
     tma_prefetch_desc(&tm_m);
+    tma_prefetch_desc(&tm_o);
   }
   if (warp == 1) {
     tmem_alloc(tmem_slot, kTmemCols);
@@ -260,15 +379,15 @@ tc_attention(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
   const uint32_t tmem = *tmem_slot;
   const int BHkv = sh.B * sh.H_kv;
 
-  // 384 threads x 168 registers at launch = 4 x 32 x 120 + 8 x 32 x 192; each
-  // role's code sits under its own setmaxnreg.
+  // Each role's code sits under its own setmaxnreg (register split above).
   if (warp < 4) {
     asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsRoles));
   if (warp == 0) {
     {
       // ------------------------------------------------ TMA producer
       // The whole warp runs the loop and every wait (kept warp-uniform);
-      // lane 0 issues the copies.
+      // lane 0 issues the copies.  Ring entries per item: K_0 V_0 K_1 V_1
+      // ... M_{s-1}.
       uint32_t rc = 0;                // ring loads issued
       uint32_t qi[2] = {0u, 0u};      // Q loads issued per slot (tile = 2 * slot + count % 2)
       bool ok = true;
@@ -284,8 +403,11 @@ tc_attention(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
         ++rc;
         return true;
       };
-      // Query tiles of an item into the slots' next Q tiles (a tile is free
-      // once the retrieval two items back has read it).
+      // Query tiles of an item into the slots' next Q tiles, each with the
+      // item's z_{s-1} (D floats) in the tile's z buffer.  A tile is free
+      // once the output store of the item two back (which staged its output
+      // there) has read it; the softmax warps signal that after the first
+      // scores of the item in between.
       auto q_load = [&](const Item& nx) -> bool {
         for (int x = 0; x < 2; ++x) {
           if (nx.n[x] == 0) continue;
@@ -294,30 +416,34 @@ tc_attention(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
             return false;
           if (lane == 0) {
             unsigned char* dst = smem + SM::kQ + b * kTileBytes;
-            mbar_arrive_expect_tx(q_full + b, kTileBytes);
+            mbar_arrive_expect_tx(q_full + b, kTileBytes + D * 4);
             for (int p = 0; p < kPanels; ++p)
               tma_load_3d(dst + p * kBM * 128, &tm_q, q_full + b, p * 64, nx.seg0 + nx.qt[x] * kBM,
                           nx.b * sh.H_q + nx.h[x]);
+            bulk_load(smem + SM::kZ + b * D * 4,
+                      z_pref + (size_t)(nx.s * BHkv + nx.b * sh.H_kv + nx.h_kv) * D, D * 4, q_full + b);
           }
           ++qi[x];
         }
         return true;
       };
-      if (blockIdx.x < sh.items) ok = q_load(decode_item(blockIdx.x, sh));
-      for (int idx = blockIdx.x; ok && idx < sh.items; idx += gridDim.x) {
-        const Item it = decode_item(idx, sh);
+      if (seq_valid(0, sh)) ok = q_load(seq_item(0, sh));
+      for (int k = 0; ok && seq_valid(k, sh); ++k) {
+        const Item it = seq_item(k, sh);
+        const bool has_next = seq_valid(k + 1, sh);
         if (it.n_max == 0) {
-          // An empty item (past the end of a short last segment) still hands
-          // on the next item's query tiles.
-          if (idx + (int)gridDim.x < sh.items) ok = q_load(decode_item(idx + gridDim.x, sh));
+          // An empty item (past the end of a short last segment, or the
+          // missing half of a unit) still hands on the next item's query tiles.
+          if (has_next) ok = q_load(seq_item(k + 1, sh));
           continue;
         }
         const int bh_kv = it.b * sh.H_kv + it.h_kv;
         for (int j = 0; ok && j < it.n_max; ++j) {
           ok = ring_load(&tm_k, kBN, it.seg0 + j * kBN, bh_kv) &&
                ring_load(&tm_v, kBN, it.seg0 + j * kBN, bh_kv);
-          // The next item's query tiles, early in this item.
-          if (ok && j == 0 && idx + (int)gridDim.x < sh.items) ok = q_load(decode_item(idx + gridDim.x, sh));
+          // The next item's query tiles, after this item's second key tile
+          // (or its only one).
+          if (ok && j == min(1, it.n_max - 1) && has_next) ok = q_load(seq_item(k + 1, sh));
         }
         // M_{s-1} (D x D, panels of D rows).
         if (ok) ok = ring_load(&tm_m, D, 0, it.s * BHkv + bh_kv);
@@ -346,102 +472,128 @@ tc_attention(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
       const uint64_t dk0 = sw128_desc(smem_u32(ring), 16, 1024);
       const uint64_t dv0 = sw128_desc(smem_u32(ring), kBN * 128, 1024);
       const uint64_t dm0 = sw128_desc(smem_u32(ring), D * 128, 1024);
-      uint32_t rc = 0;
+      uint32_t base = 0;          // ring index of the current item's first entry
       uint32_t pc[2] = {0u, 0u};  // P tiles consumed per slot
       uint32_t ic[2] = {0u, 0u};  // items per slot
+      bool pre = false;           // this item's first scores were issued at the end of the last
       bool ok = true;
-      for (int idx = blockIdx.x; ok && idx < sh.items; idx += gridDim.x) {
-        const Item it = decode_item(idx, sh);
+      auto wait_entry = [&](uint32_t idx) -> bool {
+        return __all_sync(0xffffffffu, mbar_wait(full + idx % kRing, (idx / kRing) & 1u, abort, status));
+      };
+      // S = Q K^T for slot x into its score columns (query tile b, keys at
+      // ring index idx).
+      auto issue_qk = [&](int x, uint32_t b, uint32_t idx) {
+        const uint32_t tS = tmem + x * 256;
+        const uint64_t dq = dq0 + ((b * kTileBytes) >> 4);
+        const uint64_t dk = dk0 + (((idx % kRing) * kTileBytes) >> 4);
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk)
+          mma_ss(tS, dq + kmajor_step(kk, kBM), dk + kmajor_step(kk, kBN), idesc_qk, kk > 0 ? 1u : 0u);
+        tc_commit(s_full + x);
+      };
+      for (int k = 0; ok && seq_valid(k, sh); ++k) {
+        const Item it = seq_item(k, sh);
         if (it.n_max == 0) continue;
-        uint32_t ks = 0, kph = 0, vs = 0, vph = 0;
-        for (int j = 0; ok && j <= it.n_max; ++j) {
-          if (j > 0) {
-            vs = rc % kRing;
-            vph = (rc / kRing) & 1u;
-            ++rc;
-          }
-          if (j < it.n_max) {
-            ks = rc % kRing;
-            kph = (rc / kRing) & 1u;
-            ++rc;
-          }
-          const uint64_t dv = dv0 + ((vs * kTileBytes) >> 4);
-          const uint64_t dk = dk0 + ((ks * kTileBytes) >> 4);
-          bool v_ready = false, k_ready = false;
+        for (int i = 0; ok && i <= it.n_max; ++i) {
+          const uint32_t ki = base + 2 * i, vi = base + 2 * (i - 1) + 1;
 #pragma unroll
           for (int x = 0; x < 2; ++x) {
             const uint32_t tS = tmem + x * 256, tO = tS + 128;
-            if (j > 0 && j - 1 < it.n[x]) {
-              // O += P_{j-1} V_{j-1}
+            if (i > 0 && i - 1 < it.n[x]) {
+              // O (+)= P_{i-1} V_{i-1}
               if (!(ok = __all_sync(0xffffffffu, mbar_wait(p_ready + x, pc[x] & 1u, abort, status)))) break;
               ++pc[x];
-              if (!v_ready && !(ok = __all_sync(0xffffffffu, mbar_wait(full + vs, vph, abort, status)))) break;
-              v_ready = true;
+              // The first P.V of an item overwrites O: the epilogue of the
+              // slot's previous item must have read it.
+              if (i == 1 &&
+                  !(ok = __all_sync(0xffffffffu, mbar_wait(tmem_free + x, (ic[x] & 1u) ^ 1u, abort, status))))
+                break;
+              if ((x == 0 || it.n[0] < i) && !(ok = wait_entry(vi))) break;
               tc_fence_after();
               if (lane == 0) {
+                const uint64_t dv = dv0 + (((vi % kRing) * kTileBytes) >> 4);
                 // P of keys 0..63 sits in columns 0..31, of keys 64..127 in 64..95.
-                mma_ts(tO, tS, dv, idesc_pv, j > 1 ? 1u : 0u);
+                mma_ts(tO, tS, dv, idesc_pv, i > 1 ? 1u : 0u);
 #pragma unroll
                 for (int kk = 1; kk < kBN / 16; ++kk)
                   mma_ts(tO, tS + (kk < 4 ? kk * 8 : 64 + (kk - 4) * 8), dv + mnmajor_step(kk), idesc_pv, 1u);
+                // Both slots read the tile; release it after the last.
+                if (x == 1 || it.n[1] < i) tc_commit(empty + vi % kRing);
               }
             }
-            if (j < it.n[x]) {
-              // S_j = Q K_j^T
-              if (j == 0) {
-                // The previous item's epilogue has read this slot's TMEM.
-                if (!(ok = __all_sync(0xffffffffu, mbar_wait(tmem_free + x, (ic[x] & 1u) ^ 1u, abort, status)))) break;
-                if (!(ok = __all_sync(0xffffffffu, mbar_wait(q_full + 2 * x + (ic[x] & 1u), (ic[x] >> 1) & 1u,
-                                                             abort, status))))
-                  break;
-              }
-              const uint64_t dq = dq0 + (((2 * x + (ic[x] & 1u)) * kTileBytes) >> 4);
-              if (!k_ready && !(ok = __all_sync(0xffffffffu, mbar_wait(full + ks, kph, abort, status)))) break;
-              k_ready = true;
+            if (i < it.n[x] && !(i == 0 && pre)) {
+              // S_i = Q K_i^T
+              if (i == 0 && !(ok = __all_sync(0xffffffffu, mbar_wait(q_full + 2 * x + (ic[x] & 1u),
+                                                                      (ic[x] >> 1) & 1u, abort, status))))
+                break;
+              if ((x == 0 || it.n[0] <= i) && !(ok = wait_entry(ki))) break;
               tc_fence_after();
               if (lane == 0) {
-#pragma unroll
-                for (int kk = 0; kk < D / 16; ++kk)
-                  mma_ss(tS, dq + kmajor_step(kk, kBM), dk + kmajor_step(kk, kBN), idesc_qk,
-                         kk > 0 ? 1u : 0u);
-                tc_commit(s_full + x);
+                issue_qk(x, 2 * x + (ic[x] & 1u), ki);
+                if (x == 1 || it.n[1] <= i) tc_commit(empty + ki % kRing);
               }
             }
           }
           if (!ok) break;
-          if (lane == 0) {
-            if (j < it.n_max) tc_commit(empty + ks);
-            if (j > 0) tc_commit(empty + vs);
-          }
         }
         if (!ok) break;
-        // Retrieval R = sigma(Q) M_{s-1} into each slot's score columns.
-        const uint32_t ms = rc % kRing, mph = (rc / kRing) & 1u;
-        ++rc;
-        const uint64_t dm = dm0 + ((ms * kTileBytes) >> 4);
+        // Ring entries: M_{s-1} of this item, then the next item's.
+        const uint32_t mi = base + 2 * it.n_max;
+        const uint32_t next_base = mi + 1;
+        // Retrieval folded into O: O += R' = (rows of sigma(Q), scaled by the
+        // softmax warps) M_{s-1}, as soon as a slot's rows are in.  With the
+        // gate at exactly 1 the softmax part drops out and R' overwrites O
+        // instead.
+        const uint64_t dm = dm0 + (((mi % kRing) * kTileBytes) >> 4);
         bool m_ready = false;
 #pragma unroll
         for (int x = 0; x < 2; ++x) {
           if (it.n[x] == 0) continue;
+          const bool keep = gate_sigmoid(__ldg(beta + it.h[x])) != 1.f;
           if (!(ok = __all_sync(0xffffffffu, mbar_wait(sq_ready + x, ic[x] & 1u, abort, status)))) break;
-          if (!m_ready && !(ok = __all_sync(0xffffffffu, mbar_wait(full + ms, mph, abort, status)))) break;
+          if (!m_ready && !(ok = wait_entry(mi))) break;
           m_ready = true;
           tc_fence_after();
           if (lane == 0) {
-            const uint32_t tS = tmem + x * 256;
-            const uint32_t qb = 2 * x + (ic[x] & 1u);
-            const uint64_t dq = dq0 + ((qb * kTileBytes) >> 4);
+            const uint32_t tO = tmem + x * 256 + 128;
+            const uint64_t dq = dq0 + (((2 * x + (ic[x] & 1u)) * kTileBytes) >> 4);
 #pragma unroll
             for (int kk = 0; kk < D / 16; ++kk)
-              mma_ss(tS, dq + kmajor_step(kk, kBM), dm + mnmajor_step(kk), idesc_pv, kk > 0 ? 1u : 0u);
+              mma_ss(tO, dq + kmajor_step(kk, kBM), dm + mnmajor_step(kk), idesc_pv,
+                     (kk > 0 || keep) ? 1u : 0u);
             tc_commit(r_full + x);
-            tc_commit(q_empty + qb);
           }
         }
         if (!ok) break;
-        if (lane == 0) tc_commit(empty + ms);
-        for (int x = 0; x < 2; ++x)
-          if (it.n[x] > 0) ++ic[x];
+        if (lane == 0) tc_commit(empty + mi % kRing);
+        uint32_t icn[2];
+        for (int x = 0; x < 2; ++x) icn[x] = ic[x] + (it.n[x] > 0 ? 1u : 0u);
+        // The next item's first scores (a slot's score columns are free once
+        // its last P.V, issued above, has read them); the softmax warps find
+        // them ready when they are through with this item.
+        pre = false;
+        if (seq_valid(k + 1, sh)) {
+          const Item nx = seq_item(k + 1, sh);
+          if (nx.n_max > 0) {
+#pragma unroll
+            for (int x = 0; x < 2; ++x) {
+              if (nx.n[x] == 0) continue;
+              if (!(ok = __all_sync(0xffffffffu, mbar_wait(q_full + 2 * x + (icn[x] & 1u), (icn[x] >> 1) & 1u,
+                                                           abort, status))))
+                break;
+              if ((x == 0 || nx.n[0] == 0) && !(ok = wait_entry(next_base))) break;
+              tc_fence_after();
+              if (lane == 0) issue_qk(x, 2 * x + (icn[x] & 1u), next_base);
+            }
+            if (!ok) break;
+            // Both slots' first scores read K_0; release it.
+            if (lane == 0) tc_commit(empty + next_base % kRing);
+            pre = true;
+          }
+        }
+        ic[0] = icn[0];
+        ic[1] = icn[1];
+        base = next_base;
       }
       // Every MMA issued must be complete before TMEM is released.
       if (lane == 0) tc_commit(drain);
@@ -459,25 +611,24 @@ tc_attention(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
     // the .sync.aligned TMEM instructions are always executed by full warps.
     const int x = (warp - 4) >> 2;
     const int r = 32 * (warp & 3) + lane;
+    const bool leader = (warp & 3) == 0;  // stores the slot's output tiles
     const uint32_t lane_off = (uint32_t)(32 * (warp & 3)) << 16;
     const uint32_t tS = tmem + x * 256 + lane_off;
     const uint32_t tO = tS + 128;
-    float* zs = reinterpret_cast<float*>(smem + SM::kZ) + x * D;
     const float sl2 = rsqrtf((float)D) * 1.4426950408889634f;
     uint32_t sc = 0u, ic = 0u;
+    bool store_pending = false;  // (leader, lane 0) a store whose shared-memory reads may still run
+    uint32_t pend_b = 0;
     bool ok = true;
-    for (int idx = blockIdx.x; ok && idx < sh.items; idx += gridDim.x) {
-      const Item it = decode_item(idx, sh);
+    for (int k = 0; ok && seq_valid(k, sh); ++k) {
+      const Item it = seq_item(k, sh);
       const int n = it.n[x];
       if (n == 0) continue;
       const int qt = it.qt[x], h = it.h[x];
-      const int mslice = it.s * BHkv + it.b * sh.H_kv + it.h_kv;
-      // z_{s-1} to this slot's shared copy (every read of the previous
-      // item's copy precedes sq_ready, which the retrieval MMA waited for
-      // before r_full, which this warpgroup waited for before getting here).
-      if (r < D) zs[r] = __ldg(z_pref + (size_t)mslice * D + r);
-      warp_arrive(z_ready + x);
-      float m_run = -INFINITY, l_run = 0.f;
+      const uint32_t qb = 2 * x + (ic & 1u);
+      unsigned char* sQ = smem + SM::kQ + qb * kTileBytes;
+      const float* zs = reinterpret_cast<const float*>(smem + SM::kZ + qb * D * 4);
+      float m_run = -INFINITY, l_run = 0.f, den = 0.f;
       for (int j = 0; j < n; ++j) {
         ok = __all_sync(0xffffffffu, mbar_wait(s_full + x, sc & 1u, abort, status));
         ++sc;
@@ -487,11 +638,12 @@ tc_attention(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
 #pragma unroll
         for (int c = 0; c < 4; ++c) tmem_ld32(tS + c * 32, sv + c * 32);
         tmem_wait_ld();
-        if (j == qt) {
+        const bool diag = j == qt;
+        if (diag) {
           // Diagonal tile: key c is visible to row r iff c <= r.
 #pragma unroll
-          for (int i = 0; i < 128; ++i)
-            if (i > r) sv[i] = __float_as_uint(-INFINITY);
+          for (int c = 0; c < 128; ++c)
+            if (c > r) sv[c] = __float_as_uint(-INFINITY);
         }
         // The reference max: the row max of the item's first tile; later
         // tiles are exponentiated against it directly, and only if a row's
@@ -502,10 +654,21 @@ tc_attention(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
         // P (bf16 pairs) over the scores already read: keys 0..63 -> columns
         // 0..31, keys 64..127 -> columns 64..95.
         uint32_t packed[32];
-        float lsum = exp_pack64(sv, sl2, m_run, packed);
-        tmem_st32(tS, packed);
-        lsum += exp_pack64(sv + 64, sl2, m_run, packed);
-        tmem_st32(tS + 64, packed);
+        auto exp_row = [&](float ref) -> float {
+          float sum;
+          if (diag) {
+            sum = exp_pack64<true>(sv, sl2, ref, packed);
+            tmem_st32(tS, packed);
+            sum += exp_pack64<true>(sv + 64, sl2, ref, packed);
+          } else {
+            sum = exp_pack64<false>(sv, sl2, ref, packed);
+            tmem_st32(tS, packed);
+            sum += exp_pack64<false>(sv + 64, sl2, ref, packed);
+          }
+          tmem_st32(tS + 64, packed);
+          return sum;
+        };
+        float lsum = exp_row(m_run);
         const bool need = !(lsum <= 65536.f);
         if (__any_sync(0xffffffffu, need)) {
           const float mt = need ? sl2 * row_max128(sv, sv + 64) : m_run;
@@ -516,7 +679,7 @@ tc_attention(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
             tmem_ld16(tO + c * 16, raw);
             tmem_wait_ld();
 #pragma unroll
-            for (int i = 0; i < 16; ++i) raw[i] = __float_as_uint(__uint_as_float(raw[i]) * f);
+            for (int e = 0; e < 16; ++e) raw[e] = __float_as_uint(__uint_as_float(raw[e]) * f);
             tmem_st16(tO + c * 16, raw);
           }
           if (need) {
@@ -525,93 +688,89 @@ tc_attention(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
           }
           // Redo P against the (possibly new) reference (unchanged rows get
           // the same values again).
-          lsum = exp_pack64(sv, sl2, m_run, packed);
-          tmem_st32(tS, packed);
-          lsum += exp_pack64(sv + 64, sl2, m_run, packed);
-          tmem_st32(tS + 64, packed);
+          lsum = exp_row(m_run);
         }
         l_run += lsum;
         tmem_wait_st();
         tc_fence_before();
         warp_arrive(p_ready + x);
-      }
-      if (!ok) break;
-      // sigma(Q) in place of Q (every QK^T product of this slot is complete
-      // once its last score tile arrived) and the retrieval denominator
-      // sigma(q_r) . z_{s-1} in fp32 from the unrounded sigma.
-      ok = __all_sync(0xffffffffu, mbar_wait(z_ready + x, ic & 1u, abort, status));
-      if (!ok) break;
-      unsigned char* sQ = smem + SM::kQ + (2 * x + (ic & 1u)) * kTileBytes;
-      float den = 0.f;
-#pragma unroll 2
-      for (int c8 = 0; c8 < D / 8; ++c8) {
-        const uint32_t off = sw128_offset(r, c8 * 8, kBM);
-        const uint4 v = *reinterpret_cast<const uint4*>(sQ + off);
-        const float4 za = reinterpret_cast<const float4*>(zs)[2 * c8];
-        const float4 zb = reinterpret_cast<const float4*>(zs)[2 * c8 + 1];
-        const float zz[8] = {za.x, za.y, za.z, za.w, zb.x, zb.y, zb.z, zb.w};
-        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-        uint32_t o[4];
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          // sigma = x + 1 for x > 0, e^x otherwise; half of the 2^x on the
-          // FMA pipe (both are exact to well below bf16 rounding).
-          const float2 xv = make_float2(bf16lo_to_f32(w[i]), bf16hi_to_f32(w[i]));
-          const float2 xe = make_float2(xv.x * 1.4426950408889634f, xv.y * 1.4426950408889634f);
-          float2 e;
-          if (i & 1) {
-            e = exp2_poly2(xe);
-          } else {
-            e.x = ex2_approx(xe.x);
-            e.y = ex2_approx(xe.y);
+        if (j == 0) {
+          // While the tensor core works on: the previous output store of this
+          // slot has long read its buffer, which the producer may now refill;
+          // and the retrieval denominator sigma(q_r) . z_{s-1} (fp32).  (The
+          // tile and its z landed before the first scores; the wait makes
+          // the copy visible to this thread.)
+          if (store_pending && lane == 0) {
+            tma_store_wait_read();
+            mbar_arrive(q_empty + pend_b);
           }
-          const float a = xv.x > 0.f ? xv.x + 1.f : e.x;
-          const float b = xv.y > 0.f ? xv.y + 1.f : e.y;
-          den = fmaf(a, zz[2 * i], den);
-          den = fmaf(b, zz[2 * i + 1], den);
-          o[i] = pack_bf16x2(a, b);
+          store_pending = false;
+          ok = __all_sync(0xffffffffu, mbar_wait(q_full + qb, (ic >> 1) & 1u, abort, status));
+          if (!ok) break;
+          den = sigma_dot_z<D>(sQ, r, zs);
         }
-        *reinterpret_cast<uint4*>(sQ + off) = make_uint4(o[0], o[1], o[2], o[3]);
       }
+      if (!ok) break;
+      // out = (1 - g)/l * O + g/den * sigma(Q) M.  The retrieval enters O
+      // through its rows: R' = (sigma(q_r) c_r) M with c_r = g l / ((1 - g) den),
+      // so out = (1 - g)/l * (O + R').  With g == 1 (only the retrieval is
+      // left) R' overwrites O with c_r = 1/den.  A zero denominator (empty
+      // memory) gives a zero retrieval.
+      const float gm = gate_sigmoid(__ldg(beta + h));
+      float cr, so;
+      if (gm == 1.f) {
+        cr = den != 0.f ? 1.f / den : 0.f;
+        so = 1.f;
+      } else {
+        cr = den != 0.f ? gm * l_run / ((1.f - gm) * den) : 0.f;
+        so = (1.f - gm) / l_run;
+      }
+      // (Every QK^T of this slot is complete once its last score tile arrived.)
+      sigma_scale_row<D>(sQ, r, cr);
       fence_proxy_async();
       warp_arrive(sq_ready + x);
       ok = __all_sync(0xffffffffu, mbar_wait(r_full + x, ic & 1u, abort, status));
-      ++ic;
       if (!ok) break;
       tc_fence_after();
-      // out = (1 - g)/l * O + g/den * R: TMEM read out first (then the next
-      // item may use this slot's columns), stored row by row from registers.
-      const float gm = gate_sigmoid(__ldg(beta + h));
-      const float wo = (1.f - gm) / l_run;
-      const float wm = den != 0.f ? gm / den : 0.f;
-      const float2 wo2 = make_float2(wo, wo), wm2 = make_float2(wm, wm);
-      uint32_t w[D / 2];
+      // O read out (then the slot's next P.V may overwrite it), scaled to the
+      // output and staged as bf16 in the query tile, whose retrieval rows the
+      // tensor core has finished reading; 64 columns per TMEM wait, each
+      // chunk straight to the staging tile.
 #pragma unroll
-      for (int c = 0; c < D / 32; c += 2) {
-        // Two 32-column chunks of O and R per TMEM wait.
-        uint32_t o_raw[64], r_raw[64];
-        tmem_ld32(tO + c * 32, o_raw);
-        tmem_ld32(tS + c * 32, r_raw);
-        tmem_ld32(tO + c * 32 + 32, o_raw + 32);
-        tmem_ld32(tS + c * 32 + 32, r_raw + 32);
+      for (int c = 0; c < D; c += 64) {
+        uint32_t o_raw[64];
+        tmem_ld32(tO + c, o_raw);
+        tmem_ld32(tO + c + 32, o_raw + 32);
         tmem_wait_ld();
+        uint32_t w[32];
 #pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          const float2 a = make_float2(__uint_as_float(o_raw[2 * i]), __uint_as_float(o_raw[2 * i + 1]));
-          const float2 m = make_float2(__uint_as_float(r_raw[2 * i]), __uint_as_float(r_raw[2 * i + 1]));
-          const float2 y = __ffma2_rn(m, wm2, __fmul2_rn(a, wo2));
-          w[c * 16 + i] = pack_bf16x2(y.x, y.y);
-        }
+        for (int e = 0; e < 32; ++e)
+          w[e] = pack_bf16x2(__uint_as_float(o_raw[2 * e]) * so, __uint_as_float(o_raw[2 * e + 1]) * so);
+#pragma unroll
+        for (int e = 0; e < 8; ++e)
+          *reinterpret_cast<uint4*>(sQ + sw128_offset(r, c + e * 8, kBM)) =
+              make_uint4(w[4 * e], w[4 * e + 1], w[4 * e + 2], w[4 * e + 3]);
       }
       tc_fence_before();
       warp_arrive(tmem_free + x);
-      if (qt * kBM + r < it.seg_len) {
-        uint4* dst = reinterpret_cast<uint4*>(
-            out + ((size_t)(it.b * sh.H_q + h) * sh.L + it.seg0 + qt * kBM + r) * D);
-#pragma unroll
-        for (int i = 0; i < D / 8; ++i) dst[i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
+      fence_proxy_async();
+      warp_arrive(o_staged + x);
+      if (leader) {
+        // One TMA store of the tile (rows past the end of the sequence, in a
+        // short last segment, are clipped by the tensor bounds).
+        ok = __all_sync(0xffffffffu, mbar_wait(o_staged + x, ic & 1u, abort, status));
+        if (!ok) break;
+        if (lane == 0) {
+          for (int p = 0; p < kPanels; ++p)
+            tma_store_3d(&tm_o, sQ + p * kBM * 128, p * 64, it.seg0 + qt * kBM, it.b * sh.H_q + h);
+          tma_store_commit();
+        }
+        store_pending = true;
+        pend_b = qb;
       }
+      ++ic;
     }
+    if (leader && lane == 0) tma_store_wait_all();
   }
   tc_fence_before();
   __syncthreads();
@@ -642,7 +801,7 @@ EncodeTiledFn encode_fn() {
 }
 
 // 3-D bf16 map over [planes][rows][cols] (cols contiguous), box 64 x box_rows x 1,
-// 128-byte swizzle, out-of-range rows read as zero.
+// 128-byte swizzle, out-of-range rows read as zero (and are not written).
 bool make_map(CUtensorMap* m, const void* base, uint64_t cols, uint64_t rows, uint64_t planes,
               uint32_t box_rows) {
   EncodeTiledFn enc = encode_fn();
@@ -658,10 +817,11 @@ bool make_map(CUtensorMap* m, const void* base, uint64_t cols, uint64_t rows, ui
 
 template <int D>
 cudaError_t launch(const Problem& p, cudaStream_t stream) {
-  CUtensorMap tq, tk, tv, tm;
+  CUtensorMap tq, tk, tv, tm, to;
   const uint64_t BHq = (uint64_t)p.B * p.H_q, BHkv = (uint64_t)p.B * p.H_kv;
   if (!make_map(&tq, p.q, D, p.L, BHq, kBM) || !make_map(&tk, p.k, D, p.L, BHkv, kBN) ||
-      !make_map(&tv, p.v, D, p.L, BHkv, kBN) || !make_map(&tm, p.M_pref, D, D, (uint64_t)p.T * BHkv, D))
+      !make_map(&tv, p.v, D, p.L, BHkv, kBN) || !make_map(&tm, p.M_pref, D, D, (uint64_t)p.T * BHkv, D) ||
+      !make_map(&to, p.out, D, p.L, BHq, kBM))
     return cudaErrorInvalidValue;
   Shape sh;
   sh.B = p.B;
@@ -672,35 +832,42 @@ cudaError_t launch(const Problem& p, cudaStream_t stream) {
   sh.T = p.T;
   sh.g = p.H_q / p.H_kv;
   sh.tps = p.S / kBM;
-  sh.per_group = (sh.g * sh.tps + 1) / 2;
-  const long long items = (long long)p.T * BHkv * sh.per_group;
-  if (items > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
-  sh.items = (int)items;
-  if (sh.items == 0) return cudaSuccess;
+  sh.per_group = (sh.g * sh.tps + 1) / 2;  // items per group: pairs of its g * tps query tiles
+  sh.upg = (sh.per_group + 1) / 2;
+  sh.by_per_group = make_fastdiv((uint32_t)sh.per_group);
+  sh.by_upg = make_fastdiv((uint32_t)sh.upg);
+  sh.by_H_kv = make_fastdiv((uint32_t)sh.H_kv);
+  sh.by_B = make_fastdiv((uint32_t)sh.B);
+  const long long units = (long long)p.T * BHkv * sh.upg;
+  if ((long long)p.T * BHkv * sh.per_group > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
+  sh.units = (int)units;
+  if (sh.units == 0) return cudaSuccess;
   int dev = 0, sms = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
-  const int grid = sh.items < sms ? sh.items : sms;
+  const int grid = sh.units < sms ? sh.units : sms;
   const int smem = Smem<D>::kAlloc;
   auto kern = tc_attention<D>;
   e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
-  kern<<<grid, kThreads, smem, stream>>>(tq, tk, tv, tm, p.z_pref, p.beta,
-                                         static_cast<__nv_bfloat16*>(p.out), p.status, sh);
+  kern<<<grid, kThreads, smem, stream>>>(tq, tk, tv, tm, to, p.z_pref, p.beta, p.status, sh);
   return cudaGetLastError();
 }
 
 }  // namespace
 
 bool tc_attention_supported(int d_k, int d_v, int S, bool bf16) {
-  return bf16 && d_k == d_v && (d_k == 64 || d_k == 128) && S % kBM == 0;
+  return (bf16 && d_k == d_v && (d_k == 64 || d_k == 128) && S % kBM == 0) ||
+         tc_small_attention_supported(d_k, d_v, S, bf16);
 }
 
 cudaError_t launch_tc_attention(const Problem& p, cudaStream_t stream) {
-  // With one query head per KV head, a work item would pair tiles qt and
-  // qt - 1 of one head and one slot would idle for a tile of every item; the
-  // one-tile-per-CTA kernel (two CTAs per SM) is faster there.
+  // Segments shorter than a query tile: several segments per tile.
+  if (p.S < kBM) return launch_tc_small_attention(p, stream);
+  // With one query head per KV head, a work item would pair tiles of two
+  // heads that share no keys; the one-tile-per-CTA kernel (two CTAs per SM)
+  // runs there.
   if (p.H_q == p.H_kv) return launch_tc_attention_single(p, stream);
   if (p.d_k == 128) return launch<128>(p, stream);
   if (p.d_k == 64) return launch<64>(p, stream);

@@ -64,6 +64,20 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
+// Non-blocking test of whether the phase of `bar` with the given parity has
+// completed.
+__device__ __forceinline__ bool mbar_test(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
 // Waits until the phase of `bar` with the given parity has completed.  Gives
 // up after kWaitLimitNs, or as soon as another thread of the CTA has given up
 // (*abort != 0): it then sets the timeout bit of the device status word and
@@ -112,6 +126,21 @@ __device__ __forceinline__ void tma_store_commit() {
 
 __device__ __forceinline__ void tma_store_wait_read() {
   asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+}
+
+// Waits until every bulk store this thread committed has completed.
+__device__ __forceinline__ void tma_store_wait_all() {
+  asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
+}
+
+// Contiguous copy of `bytes` (a multiple of 16, both addresses 16-byte
+// aligned) from global to shared memory, completing on `bar`.
+__device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+          smem_u32(dst)),
+      "l"(src), "r"(bytes), "r"(smem_u32(bar))
+      : "memory");
 }
 
 // Pulls a tile into L2 ahead of its load (no shared memory, no barrier).
@@ -295,21 +324,25 @@ __device__ __forceinline__ float ex2_approx(float x) {
 // low mantissa bits), a degree-3 polynomial for 2^f (least-squares fit on
 // [-1/2, 1/2] weighted to the relative error; max relative error 7.6e-5), and
 // the scale by 2^n as an integer add of n << 23 to the exponent bits.  Inputs
-// are clamped to >= -125 so the exponent never underflows; results below
-// 2^-125 matter to nothing here.
+// are clamped to >= -125 so the exponent never underflows (results below
+// 2^-125 matter to nothing here); with EXACT_ZERO, inputs below -125 (a
+// masked score is -inf) give exactly 0, as the hardware 2^x does with
+// subnormal results flushed.
+template <bool EXACT_ZERO = true>
 __device__ __forceinline__ float2 exp2_poly2(float2 x) {
-  x.x = fmaxf(x.x, -125.f);
-  x.y = fmaxf(x.y, -125.f);
+  const float2 xc = make_float2(fmaxf(x.x, -125.f), fmaxf(x.y, -125.f));
   const float kRound = 12582912.f;
-  const float2 t = __fadd2_rn(x, make_float2(kRound, kRound));
+  const float2 t = __fadd2_rn(xc, make_float2(kRound, kRound));
   const float2 n = __fadd2_rn(t, make_float2(-kRound, -kRound));
-  const float2 f = __ffma2_rn(n, make_float2(-1.f, -1.f), x);
+  const float2 f = __ffma2_rn(n, make_float2(-1.f, -1.f), xc);
   float2 p = __ffma2_rn(make_float2(0.055186376f, 0.055186376f), f,
                         make_float2(0.24261236f, 0.24261236f));
   p = __ffma2_rn(p, f, make_float2(0.69325829f, 0.69325829f));
   p = __ffma2_rn(p, f, make_float2(0.99992794f, 0.99992794f));
-  return make_float2(__uint_as_float(__float_as_uint(p.x) + (__float_as_uint(t.x) << 23)),
-                     __uint_as_float(__float_as_uint(p.y) + (__float_as_uint(t.y) << 23)));
+  const float rx = __uint_as_float(__float_as_uint(p.x) + (__float_as_uint(t.x) << 23));
+  const float ry = __uint_as_float(__float_as_uint(p.y) + (__float_as_uint(t.y) << 23));
+  if (!EXACT_ZERO) return make_float2(rx, ry);
+  return make_float2(x.x < -125.f ? 0.f : rx, x.y < -125.f ? 0.f : ry);
 }
 
 // max(a, b, c) in one instruction (three-input fp32 max, sm_100).

@@ -263,6 +263,16 @@ TC_CASES = [
                                      H_kv=2, rule="delta")),
     ("tc_d128_gqa2_S256_ragged", dict(dtype="bf16", d_k=128, d_v=128, L=700, seg_len=256, B=2,
                                       H_q=4, H_kv=2)),
+    # Segments shorter than a query tile (several segments per tile, the
+    # short-segment kernel): a ragged last segment and a last tile that ends
+    # past the sequence; four segments per tile with GQA, where the last
+    # tile's later segments do not exist; d = 128.
+    ("tc_small_d64_S64_delta_ragged", dict(dtype="bf16", d_k=64, d_v=64, L=1000, seg_len=64, B=2,
+                                           H_q=3, H_kv=3, rule="delta")),
+    ("tc_small_d64_S32_gqa_ragged", dict(dtype="bf16", d_k=64, d_v=64, L=1030, seg_len=32, H_q=4,
+                                         H_kv=2)),
+    ("tc_small_d128_S64_delta", dict(dtype="bf16", d_k=128, d_v=128, L=384, seg_len=64, H_q=2,
+                                     H_kv=2, rule="delta")),
 ]
 
 
@@ -270,7 +280,8 @@ def test_path_selection(cuda_lib):
     api = cuda_lib
     for name, over, path in [("8b-delta", {}, "tcgen05"), ("1m-linear", {}, "tcgen05"),
                              ("300m-delta", {}, "tcgen05"), ("tiny", {}, "simt"),
-                             ("200m-linear", {}, "simt")]:
+                             ("200m-linear", {}, "tcgen05"), ("200m-delta", {}, "tcgen05"),
+                             ("200m-linear", {"seg_len": 63}, "simt")]:
         w = W[name].with_(**over)
         dims = api.make_dims(w.B, w.H_q, w.H_kv, w.L, w.d_k, w.d_v, 0 if w.dtype == "bf16" else 1)
         assert api.plan(dims, w.seg_len, w.rule)["path"] == path, name
@@ -295,23 +306,34 @@ def _scale_bf16_bits(bits, factor):
 # tile's row max by far more than 2^16 / 128 in 2^x terms, so the lazy softmax
 # reference moves mid-segment: in the low half of a tile (keys 0..63), in the
 # high half (64..127) and in both, with earlier tiles already accumulated in O.
+# With one query head per KV head the two halves of a work item take the even
+# and the odd key tiles, so spikes there also give the two halves row maxima
+# far apart when their softmax states are merged: 8x, 32x (scores ~2^7 apart
+# in 2^x terms, so the smaller half's weight would underflow fp32 if the
+# retrieval were folded into that half alone), and a spike inside tile 0.
+_LATER = (128 + 100, 256 + 10, 384 + 5, 384 + 120)
 SPIKE_CASES = [
     ("spike_d128_gqa", dict(dtype="bf16", d_k=128, d_v=128, L=1024, seg_len=512, H_q=4, H_kv=2,
-                            rule="delta")),
-    ("spike_d64_gqa", dict(dtype="bf16", d_k=64, d_v=64, L=1024, seg_len=512, H_q=4, H_kv=2)),
+                            rule="delta"), 8.0, _LATER),
+    ("spike_d64_gqa", dict(dtype="bf16", d_k=64, d_v=64, L=1024, seg_len=512, H_q=4, H_kv=2), 8.0,
+     _LATER),
     ("spike_d128_one_q_per_kv", dict(dtype="bf16", d_k=128, d_v=128, L=1024, seg_len=512, H_q=2,
-                                     H_kv=2)),
+                                     H_kv=2), 8.0, _LATER),
+    ("spike32_d64_one_q_per_kv_odd_tiles", dict(dtype="bf16", d_k=64, d_v=64, L=1024, seg_len=512,
+                                               H_q=2, H_kv=2), 32.0, (128 + 100, 384 + 5)),
+    ("spike_d128_one_q_per_kv_tile0", dict(dtype="bf16", d_k=128, d_v=128, L=1024, seg_len=512,
+                                           H_q=2, H_kv=2, rule="delta"), 8.0, (3, 77)),
 ]
 
 
-@pytest.mark.parametrize("name,over", SPIKE_CASES, ids=[c[0] for c in SPIKE_CASES])
-def test_tensor_core_path_softmax_reference_moves(cuda_lib, name, over):
+@pytest.mark.parametrize("name,over,factor,offsets", SPIKE_CASES, ids=[c[0] for c in SPIKE_CASES])
+def test_tensor_core_path_softmax_reference_moves(cuda_lib, name, over, factor, offsets):
     w = W["tiny"].with_(name=name, **over)
     inp = synth.make_inputs(w)
     for seg0 in range(0, w.L, w.seg_len):
-        for off in (128 + 100, 256 + 10, 384 + 5, 384 + 120):
+        for off in offsets:
             if seg0 + off < w.L:
-                inp["k"][:, :, seg0 + off, :] = _scale_bf16_bits(inp["k"][:, :, seg0 + off, :], 8.0)
+                inp["k"][:, :, seg0 + off, :] = _scale_bf16_bits(inp["k"][:, :, seg0 + off, :], factor)
     check_full(cuda_lib, w, inp)
 
 
@@ -329,13 +351,15 @@ def test_tensor_core_path_deterministic_and_workspace_independent(cuda_lib):
         np.testing.assert_array_equal(x, y)
 
 
-def test_tensor_core_path_gate_extremes(cuda_lib):
-    w = W["tiny"].with_(dtype="bf16", d_k=64, d_v=64, H_q=4, H_kv=2, L=512, seg_len=128)
+@pytest.mark.parametrize("seg_len", [128, 64])
+def test_tensor_core_path_gate_extremes(cuda_lib, seg_len):
+    w = W["tiny"].with_(dtype="bf16", d_k=64, d_v=64, H_q=4, H_kv=2, L=512, seg_len=seg_len)
     inp = synth.make_inputs(w)
     inp["beta"] = np.array([-np.inf, np.inf, -80.0, 80.0], np.float32)
     check_full(cuda_lib, w, inp)
     out, _, _ = gpu_forward(cuda_lib, inp, w)
-    assert np.all(out[:, 1, :128] == 0.0)
+    # beta = +inf: out is the retrieval alone, exactly 0 on the first segment
+    assert np.all(out[:, 1, :seg_len] == 0.0)
 
 
 def test_tensor_core_path_split_stream(cuda_lib):
