@@ -754,6 +754,8 @@ def main():
                     help="skip the host-buffer end-to-end measurement (profiling runs)")
     ap.add_argument("--batch", type=int, default=None,
                     help="override the workload's batch size (smaller profiling captures)")
+    ap.add_argument("--seq-len", type=int, default=None,
+                    help="override the workload's sequence length L (smaller profiling captures)")
     ap.add_argument("--cpu-budget", type=float, default=15.0,
                     help="seconds of oracle work for the cpu_baseline sample")
     ap.add_argument("--reference-budget", type=float, default=60.0,
@@ -776,6 +778,10 @@ def main():
     w = configs.WORKLOADS[args.config]
     if args.batch is not None:
         w = w.with_(B=args.batch, name=f"{w.name}-B{args.batch}")
+    if args.seq_len is not None:
+        if args.seq_len <= 0:
+            ap.error("--seq-len must be positive")
+        w = w.with_(L=args.seq_len, name=f"{w.name}-L{args.seq_len}")
     if args.impl == "reference":
         return run_reference(args, w)
     if args.decode_probe is not None:

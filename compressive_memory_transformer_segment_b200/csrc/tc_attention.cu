@@ -316,9 +316,12 @@ tc_attention(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
 
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   // The swizzled tiles need 1024-byte aligned addresses; the layout fills
-  // the opt-in maximum, leaving no room to realign.  (Every thread takes
-  // the same branch, before any barrier.)
-  if ((smem_u32(smem_raw) & 1023u) != 0) {
+  // the opt-in maximum, leaving no room to realign.  The MMA and copy issue
+  // relies on elect.sync picking lane 0 of a converged warp every time
+  // (commits and their MMAs from one thread).  Either failing, the CTA
+  // computes nothing (the decision is the same for every thread).
+  const bool misplaced = (smem_u32(smem_raw) & 1023u) != 0 || elected_lane() != 0;
+  if (__syncthreads_or(misplaced)) {
     if (threadIdx.x == 0) atomicOr(status, kStatusLayout);
     return;
   }
@@ -394,7 +397,7 @@ tc_attention(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
       auto ring_load = [&](const CUtensorMap* map, int rows_box, int row0, int plane) -> bool {
         const uint32_t slot = rc % kRing, ph = (rc / kRing) & 1u;
         if (!__all_sync(0xffffffffu, mbar_wait(empty + slot, ph ^ 1u, abort, status))) return false;
-        if (lane == 0) {
+        if (elect_one()) {
           unsigned char* dst = ring + slot * kTileBytes;
           mbar_arrive_expect_tx(full + slot, (uint32_t)rows_box * D * 2);
           for (int p = 0; p < kPanels; ++p)
@@ -414,7 +417,7 @@ tc_attention(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
           const uint32_t b = 2 * x + (qi[x] & 1u);
           if (!__all_sync(0xffffffffu, mbar_wait(q_empty + b, ((qi[x] >> 1) & 1u) ^ 1u, abort, status)))
             return false;
-          if (lane == 0) {
+          if (elect_one()) {
             unsigned char* dst = smem + SM::kQ + b * kTileBytes;
             mbar_arrive_expect_tx(q_full + b, kTileBytes + D * 4);
             for (int p = 0; p < kPanels; ++p)
@@ -510,7 +513,7 @@ tc_attention(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
                 break;
               if ((x == 0 || it.n[0] < i) && !(ok = wait_entry(vi))) break;
               tc_fence_after();
-              if (lane == 0) {
+              if (elect_one()) {
                 const uint64_t dv = dv0 + (((vi % kRing) * kTileBytes) >> 4);
                 // P of keys 0..63 sits in columns 0..31, of keys 64..127 in 64..95.
                 mma_ts(tO, tS, dv, idesc_pv, i > 1 ? 1u : 0u);
@@ -528,7 +531,7 @@ tc_attention(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
                 break;
               if ((x == 0 || it.n[0] <= i) && !(ok = wait_entry(ki))) break;
               tc_fence_after();
-              if (lane == 0) {
+              if (elect_one()) {
                 issue_qk(x, 2 * x + (ic[x] & 1u), ki);
                 if (x == 1 || it.n[1] <= i) tc_commit(empty + ki % kRing);
               }
@@ -554,7 +557,7 @@ tc_attention(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
           if (!m_ready && !(ok = wait_entry(mi))) break;
           m_ready = true;
           tc_fence_after();
-          if (lane == 0) {
+          if (elect_one()) {
             const uint32_t tO = tmem + x * 256 + 128;
             const uint64_t dq = dq0 + (((2 * x + (ic[x] & 1u)) * kTileBytes) >> 4);
 #pragma unroll
@@ -565,7 +568,7 @@ tc_attention(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
           }
         }
         if (!ok) break;
-        if (lane == 0) tc_commit(empty + mi % kRing);
+        if (elect_one()) tc_commit(empty + mi % kRing);
         uint32_t icn[2];
         for (int x = 0; x < 2; ++x) icn[x] = ic[x] + (it.n[x] > 0 ? 1u : 0u);
         // The next item's first scores (a slot's score columns are free once
@@ -583,11 +586,11 @@ tc_attention(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
                 break;
               if ((x == 0 || nx.n[0] == 0) && !(ok = wait_entry(next_base))) break;
               tc_fence_after();
-              if (lane == 0) issue_qk(x, 2 * x + (icn[x] & 1u), next_base);
+              if (elect_one()) issue_qk(x, 2 * x + (icn[x] & 1u), next_base);
             }
             if (!ok) break;
             // Both slots' first scores read K_0; release it.
-            if (lane == 0) tc_commit(empty + next_base % kRing);
+            if (elect_one()) tc_commit(empty + next_base % kRing);
             pre = true;
           }
         }
@@ -596,7 +599,7 @@ tc_attention(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
         base = next_base;
       }
       // Every MMA issued must be complete before TMEM is released.
-      if (lane == 0) tc_commit(drain);
+      if (elect_one()) tc_commit(drain);
       __syncwarp();
       mbar_wait(drain, 0, abort, status, false);
       __syncwarp();

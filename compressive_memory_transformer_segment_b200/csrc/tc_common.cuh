@@ -159,6 +159,35 @@ __device__ __forceinline__ void fence_proxy_async() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
+// One lane of a converged warp, chosen with elect.sync: true there, false in
+// the other lanes.  Single-thread work that the tensor core or the copy engine
+// carries out (tcgen05.mma, tcgen05.commit, TMA) is issued under it rather
+// than under a lane-index test: the compiler then knows that one thread of a
+// converged warp runs the block, and the issue of back-to-back MMAs runs at
+// the tensor core's rate (under `lane == 0` it ran at about half of it).
+// Every caller elects from the whole warp, converged; the elected lane is
+// the same each time (a commit covers the MMAs its own thread issued), which
+// elected_lane() lets a kernel check once.
+__device__ __forceinline__ bool elect_one() {
+  uint32_t pred = 0;
+  asm volatile(
+      "{\n\t.reg .pred P1;\n\t"
+      "elect.sync _|P1, 0xffffffff;\n\t"
+      "selp.b32 %0, 1, 0, P1;\n\t}"
+      : "=r"(pred));
+  return pred != 0;
+}
+
+// Lane index elect.sync picks in a converged warp.
+__device__ __forceinline__ uint32_t elected_lane() {
+  uint32_t l = 0;
+  asm volatile(
+      "{\n\t.reg .pred P1;\n\t"
+      "elect.sync %0|P1, 0xffffffff;\n\t}"
+      : "=r"(l));
+  return l;
+}
+
 __device__ __forceinline__ void named_barrier(int id, int threads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
 }
