@@ -87,6 +87,12 @@ tc_attention_single(const __grid_constant__ CUtensorMap tm_q, const __grid_const
   const int seg0 = s * S;
   const int seg_len = min(S, L - seg0);
   if (qt * kBM >= seg_len) return;  // past the end of a short last segment
+  // The MMA and copy issue relies on elect.sync picking lane 0 of a
+  // converged warp every time (commits and their MMAs from one thread).
+  if (__syncthreads_or(elected_lane() != 0)) {
+    if (threadIdx.x == 0) atomicOr(status, kStatusLayout);
+    return;
+  }
   const int n_kv = qt + 1;
   const int bh_kv = b * H_kv + h_kv;
   const int BH = B * H_kv;
@@ -154,7 +160,7 @@ tc_attention_single(const __grid_constant__ CUtensorMap tm_q, const __grid_const
       // ------------------------------------------------ TMA producer
       int issued_k = 0, issued_v = 0;
       bool ok = true;
-      if (lane == 0) {
+      if (elect_one()) {
         mbar_arrive_expect_tx(bar_q, kTileBytes);
         for (int p = 0; p < kPanels; ++p)
           tma_load_3d(sQ + p * kBM * 128, &tm_q, bar_q, p * 64, row_q, b * H_q + h);
@@ -162,14 +168,14 @@ tc_attention_single(const __grid_constant__ CUtensorMap tm_q, const __grid_const
       for (int j = 0; j < n_kv; ++j) {
         const uint32_t par = (j & 1) ^ 1;
         if (!(ok = __all_sync(0xffffffffu, mbar_wait(empty_k, par, abort, status)))) break;
-        if (lane == 0) {
+        if (elect_one()) {
           mbar_arrive_expect_tx(full_k, kTileBytes);
           for (int p = 0; p < kPanels; ++p)
             tma_load_3d(sK + p * kBN * 128, &tm_k, full_k, p * 64, seg0 + j * kBN, bh_kv);
         }
         issued_k = j + 1;
         if (!(ok = __all_sync(0xffffffffu, mbar_wait(empty_v, par, abort, status)))) break;
-        if (lane == 0) {
+        if (elect_one()) {
           mbar_arrive_expect_tx(full_v, kTileBytes);
           for (int p = 0; p < kPanels; ++p)
             tma_load_3d(sV + p * kBN * 128, &tm_v, full_v, p * 64, seg0 + j * kBN, bh_kv);
@@ -179,7 +185,7 @@ tc_attention_single(const __grid_constant__ CUtensorMap tm_q, const __grid_const
       // M_{s-1} goes into the K buffer once the last score tile is complete.
       bool m_issued = false;
       if (ok && (ok = __all_sync(0xffffffffu, mbar_wait(empty_k, (n_kv & 1) ^ 1, abort, status)))) {
-        if (lane == 0) {
+        if (elect_one()) {
           mbar_arrive_expect_tx(bar_m, D * D * 2);
           for (int p = 0; p < kPanels; ++p) tma_load_3d(sK + p * D * 128, &tm_m, bar_m, p * 64, 0, mslice);
         }
@@ -209,7 +215,7 @@ tc_attention_single(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         // read before these MMAs overwrite it: MMAs run in issue order).
         if (!(ok = __all_sync(0xffffffffu, mbar_wait(full_k, j & 1, abort, status)))) break;
         tc_fence_after();
-        if (lane == 0) {
+        if (elect_one()) {
 #pragma unroll
           for (int kk = 0; kk < D / 16; ++kk)
             mma_ss(tS, dq + kmajor_step(kk, kBM), dk + kmajor_step(kk, kBN), idesc_qk, kk > 0 ? 1u : 0u);
@@ -220,20 +226,20 @@ tc_attention_single(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         if (!(ok = __all_sync(0xffffffffu, mbar_wait(p_ready, j & 1, abort, status)))) break;
         if (!(ok = __all_sync(0xffffffffu, mbar_wait(full_v, j & 1, abort, status)))) break;
         tc_fence_after();
-        if (lane == 0) {
+        if (elect_one()) {
           mma_ts(tO, tS, dv, idesc_pv, j > 0 ? 1u : 0u);
 #pragma unroll
           for (int kk = 1; kk < kBN / 16; ++kk) mma_ts(tO, tS + kk * 8, dv + mnmajor_step(kk), idesc_pv, 1u);
           tc_commit(empty_v);
         }
       }
-      if (ok && lane == 0) tc_commit(o_done);
+      if (ok && elect_one()) tc_commit(o_done);
       // Retrieval R = sigma(Q) M_{s-1}, into the score columns.
       if (ok) ok = __all_sync(0xffffffffu, mbar_wait(bar_m, 0, abort, status));
       if (ok) ok = __all_sync(0xffffffffu, mbar_wait(sq_ready, 0, abort, status));
       if (ok) {
         tc_fence_after();
-        if (lane == 0) {
+        if (elect_one()) {
 #pragma unroll
           for (int kk = 0; kk < D / 16; ++kk)
             mma_ss(tS, dq + kmajor_step(kk, kBM), dm + mnmajor_step(kk), idesc_r, kk > 0 ? 1u : 0u);
@@ -241,7 +247,7 @@ tc_attention_single(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         }
       }
       // Every MMA issued must be complete before TMEM is released.
-      if (lane == 0) tc_commit(drain);
+      if (elect_one()) tc_commit(drain);
       __syncwarp();
       mbar_wait(drain, 0, abort, status, false);
       __syncwarp();

@@ -113,6 +113,12 @@ tc_small_attention(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
   volatile int* abort = reinterpret_cast<volatile int*>(smem + SM::kAbort);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  // The MMA and copy issue relies on elect.sync picking lane 0 of a
+  // converged warp every time (commits and their MMAs from one thread).
+  if (__syncthreads_or(elected_lane() != 0)) {
+    if (threadIdx.x == 0) atomicOr(status, kStatusLayout);
+    return;
+  }
 
   if (threadIdx.x == 0) {
     mbar_init(loaded, 1);
@@ -135,8 +141,9 @@ tc_small_attention(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
 
   if (warp == 0) {
     // ------------------------------------------------ loads, MMAs, store
-    // The whole warp runs the sequence and every wait; lane 0 issues.
-    if (lane == 0) {
+    // The whole warp runs the sequence and every wait; one elected lane
+    // issues.
+    if (elect_one()) {
       mbar_arrive_expect_tx(loaded, 3 * kTileBytes + SPT * D * D * 2 + SPT * D * 4);
       for (int p = 0; p < kPanels; ++p) {
         tma_load_3d(sQ + p * kBM * 128, &tm_q, loaded, p * 64, r0, bh);
@@ -158,7 +165,7 @@ tc_small_attention(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
     const uint32_t tS = tmem, tO = tmem + 128;
     if (ok) {
       tc_fence_after();
-      if (lane == 0) {
+      if (elect_one()) {
         // S = Q K^T (keys of the whole tile; the mask is applied in the softmax)
         constexpr uint32_t idesc_qk = idesc_bf16_f32(kBM, kBM, false, false);
         const uint64_t dq = sw128_desc(smem_u32(sQ), 16, 1024);
@@ -172,7 +179,7 @@ tc_small_attention(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
     }
     if (ok) {
       tc_fence_after();
-      if (lane == 0) {
+      if (elect_one()) {
         // O = P V, P read from TMEM (keys 0..63 in columns 0..31, 64..127 in 64..95)
         constexpr uint32_t idesc_pv = idesc_bf16_f32(kBM, D, false, true);
         const uint64_t dv = sw128_desc(smem_u32(sV), kBM * 128, 1024);
@@ -185,7 +192,7 @@ tc_small_attention(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
     }
     if (ok) {
       tc_fence_after();
-      if (lane == 0) {
+      if (elect_one()) {
         // O (+)= A_exp [M_{s0-1}; M_{s0}; ...]: overwrites O when the gate is
         // exactly 1 (only the retrieval is left).
         const bool keep = gate_sigmoid(__ldg(beta + h)) != 1.f;
@@ -207,7 +214,7 @@ tc_small_attention(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
     }
     // Every MMA issued must be complete before TMEM is released (o_full
     // follows all of them; a wait that was abandoned drains here).
-    if (!ok && lane == 0) tc_commit(o_full);
+    if (!ok && elect_one()) tc_commit(o_full);
     __syncwarp();
     mbar_wait(o_full, 0, abort, status, false);
     __syncwarp();

@@ -163,6 +163,12 @@ tc_segment_products(const __grid_constant__ CUtensorMap tm_k, const __grid_const
   volatile int* abort = reinterpret_cast<volatile int*>(smem + SM::kAbort);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  // The MMA and copy issue relies on elect.sync picking lane 0 of a
+  // converged warp every time (commits and their MMAs from one thread).
+  if (__syncthreads_or(elected_lane() != 0)) {
+    if (threadIdx.x == 0) atomicOr(status, kStatusLayout);
+    return;
+  }
 
   if (threadIdx.x == 0) {
     mbar_init(k_full, 1);
@@ -210,19 +216,19 @@ tc_segment_products(const __grid_constant__ CUtensorMap tm_k, const __grid_const
     {
       // ------------------------------------------------ TMA producer
       // The whole warp runs the loop and every wait (kept warp-uniform);
-      // lane 0 issues the copies.
+      // one elected lane issues the copies.
       int issued_k = 0, issued_v = 0;
       for (int blk = 0; blk < nblk; ++blk) {
         const uint32_t par = (blk & 1) ^ 1;
         if (!__all_sync(0xffffffffu, mbar_wait(k_empty, par, abort, status))) break;
-        if (lane == 0) {
+        if (elect_one()) {
           mbar_arrive_expect_tx(k_full, kTok * D * 2);
           for (int p = 0; p < D / 64; ++p)
             tma_load_3d(sK + p * kTok * 128, &tm_k, k_full, p * 64, seg0 + blk * kTok, bh);
         }
         issued_k = blk + 1;
         if (!__all_sync(0xffffffffu, mbar_wait(v_empty, par, abort, status))) break;
-        if (lane == 0) {
+        if (elect_one()) {
           mbar_arrive_expect_tx(v_full, kTok * D * 2);
           for (int p = 0; p < D / 64; ++p)
             tma_load_3d(sV + p * kTok * 128, &tm_v, v_full, p * 64, seg0 + blk * kTok, bh);
@@ -236,7 +242,7 @@ tc_segment_products(const __grid_constant__ CUtensorMap tm_k, const __grid_const
   } else if (warp == 1) {
     {
       // ------------------------------------------------ MMA issuer
-      // The whole warp runs the loop and every wait; lane 0 issues.
+      // The whole warp runs the loop and every wait; one elected lane issues.
       // All operands are MN-major [tokens][128] tiles (panels of 64 columns,
       // 16 KiB apart); one 16-token K step = 2048 bytes.
       const uint64_t skhi = sw128_desc(smem_u32(sSkHi), kTok * 128, 1024);
@@ -252,26 +258,27 @@ tc_segment_products(const __grid_constant__ CUtensorMap tm_k, const __grid_const
         if (!(ok = __all_sync(0xffffffffu, mbar_wait(op_ready, blk & 1, abort, status)))) break;
         if (!(ok = __all_sync(0xffffffffu, mbar_wait(v_full, blk & 1, abort, status)))) break;
         tc_fence_after();
-        if (lane != 0) continue;
+        if (elect_one()) {
 #pragma unroll
-        for (int kk = 0; kk < kTok / 16; ++kk) {
-          const uint32_t st = mnmajor_step(kk);
-          const uint32_t acc = (blk > 0 || kk > 0) ? 1u : 0u;
-          if (DELTA) {
-            mma_ss(tG, yhi + st, skhi + st, idesc_d, acc);
-            mma_ss(tG, ylo + st, skhi + st, idesc_d, 1u);
-            mma_ss(tG, yhi + st, sklo + st, idesc_d, 1u);
-            mma_ss(tB, skhi + st, vv + st, idesc_d, acc);
-            mma_ss(tB, sklo + st, vv + st, idesc_d, 1u);
-          } else {
-            mma_ss(tB, skhi + st, vv + st, idesc_ext, acc);
-            mma_ss(tB, sklo + st, vv + st, idesc_ext, 1u);
+          for (int kk = 0; kk < kTok / 16; ++kk) {
+            const uint32_t st = mnmajor_step(kk);
+            const uint32_t acc = (blk > 0 || kk > 0) ? 1u : 0u;
+            if (DELTA) {
+              mma_ss(tG, yhi + st, skhi + st, idesc_d, acc);
+              mma_ss(tG, ylo + st, skhi + st, idesc_d, 1u);
+              mma_ss(tG, yhi + st, sklo + st, idesc_d, 1u);
+              mma_ss(tB, skhi + st, vv + st, idesc_d, acc);
+              mma_ss(tB, sklo + st, vv + st, idesc_d, 1u);
+            } else {
+              mma_ss(tB, skhi + st, vv + st, idesc_ext, acc);
+              mma_ss(tB, sklo + st, vv + st, idesc_ext, 1u);
+            }
           }
+          tc_commit(op_free);
+          tc_commit(v_empty);
         }
-        tc_commit(op_free);
-        tc_commit(v_empty);
       }
-      if (lane == 0) tc_commit(done);
+      if (elect_one()) tc_commit(done);
       __syncwarp();
       mbar_wait(done, 0, abort, status, false);
       __syncwarp();
@@ -473,6 +480,12 @@ tc_pipe_products(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + SM::kTmemSlot);
   volatile int* abort = reinterpret_cast<volatile int*>(smem + SM::kAbort);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  // The MMA and copy issue relies on elect.sync picking lane 0 of a
+  // converged warp every time (commits and their MMAs from one thread).
+  if (__syncthreads_or(elected_lane() != 0)) {
+    if (threadIdx.x == 0) atomicOr(status, kStatusLayout);
+    return;
+  }
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < kStages; ++i) {
@@ -501,13 +514,13 @@ tc_pipe_products(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
   const uint32_t tG = tmem, tB = DELTA ? tmem + 128 : tmem;
 
   if (warp == 0) {
-    // ---------------------------------------------- TMA producer (whole warp waits, lane 0 issues)
+    // ---------------------------------------------- TMA producer (whole warp waits, one elected lane issues)
     int issued = 0;
     for (int b = 0; b < nblk; ++b) {
       const int st = b % kStages;
       const uint32_t ph = (uint32_t)(b / kStages) & 1u;
       if (!__all_sync(0xffffffffu, mbar_wait(empty + st, ph ^ 1u, abort, status))) break;
-      if (lane == 0) {
+      if (elect_one()) {
         unsigned char* dst = ring + st * SM::kStage;
         mbar_arrive_expect_tx(full + st, SM::kStage);
         for (int p = 0; p < D / 64; ++p) {
@@ -522,7 +535,7 @@ tc_pipe_products(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
       mbar_wait(full + b % kStages, (uint32_t)(b / kStages) & 1u, abort, status, false);
     __syncwarp();
   } else if (warp == 1) {
-    // ---------------------------------------------- MMA issuer (whole warp waits, lane 0 issues)
+    // ---------------------------------------------- MMA issuer (whole warp waits, one elected lane issues)
     constexpr uint32_t idesc = idesc_bf16_f32(128, D, true, true);
     const uint64_t dop = sw128_desc(smem_u32(op), SM::kPanel, 1024);
     const uint64_t dring = sw128_desc(smem_u32(ring + SM::kHalf), SM::kPanel, 1024);
@@ -532,7 +545,7 @@ tc_pipe_products(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
       if (!(ok = __all_sync(0xffffffffu, mbar_wait(op_full + ob, (uint32_t)(b >> 1) & 1u, abort, status)))) break;
       if (!(ok = __all_sync(0xffffffffu, mbar_wait(full + st, (uint32_t)(b / kStages) & 1u, abort, status)))) break;
       tc_fence_after();
-      if (lane == 0) {
+      if (elect_one()) {
         // Operand parts: sigma hi, sigma lo, (Y hi, Y lo).
         const uint64_t shi = dop + ((ob * SM::kOpParts * SM::kHalf) >> 4);
         const uint64_t slo = shi + (SM::kHalf >> 4);
@@ -555,7 +568,7 @@ tc_pipe_products(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
         tc_commit(empty + st);
       }
     }
-    if (lane == 0) tc_commit(acc_full);
+    if (elect_one()) tc_commit(acc_full);
     __syncwarp();
     mbar_wait(acc_full, 0, abort, status, false);
     __syncwarp();
