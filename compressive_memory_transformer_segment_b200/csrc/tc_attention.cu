@@ -255,51 +255,40 @@ __device__ __forceinline__ float2 sigma2(uint32_t w) {
   return make_float2(xv.x > 0.f ? xv.x + 1.f : e.x, xv.y > 0.f ? xv.y + 1.f : e.y);
 }
 
-// The retrieval denominator of row r: sigma(q_r) . z_{s-1} in fp32 from the
-// unrounded sigma (q_r: row r of a 128-row query tile in shared memory; z in
-// shared memory, read as float4).  Loads go four 16-byte chunks at a time,
-// ahead of the arithmetic.
+// sigma(q_r) of row r of a 128-row query tile in shared memory, into sg[D]
+// (fp32, unrounded), and the retrieval denominator sigma(q_r) . z_{s-1}
+// (z in shared memory, read as float4), in one pass over the row.
 template <int D>
-__device__ __forceinline__ float sigma_dot_z(const unsigned char* sQ, int r, const float* zs) {
+__device__ __forceinline__ float sigma_row(const unsigned char* sQ, int r, const float* zs, float* sg) {
   float acc[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll 2
-  for (int c8 = 0; c8 < D / 8; c8 += 4) {
-    uint4 v[4];
 #pragma unroll
-    for (int i = 0; i < 4; ++i) v[i] = *reinterpret_cast<const uint4*>(sQ + sw128_offset(r, (c8 + i) * 8, kBM));
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const float4 za = reinterpret_cast<const float4*>(zs)[2 * (c8 + i)];
-      const float4 zb = reinterpret_cast<const float4*>(zs)[2 * (c8 + i) + 1];
-      const float2 s0 = sigma2<false>(v[i].x), s1 = sigma2<true>(v[i].y);
-      const float2 s2 = sigma2<false>(v[i].z), s3 = sigma2<true>(v[i].w);
-      acc[i] = fmaf(s0.y, za.y, fmaf(s0.x, za.x, acc[i]));
-      acc[i] = fmaf(s1.y, za.w, fmaf(s1.x, za.z, acc[i]));
-      acc[i] = fmaf(s2.y, zb.y, fmaf(s2.x, zb.x, acc[i]));
-      acc[i] = fmaf(s3.y, zb.w, fmaf(s3.x, zb.z, acc[i]));
-    }
+  for (int c8 = 0; c8 < D / 8; ++c8) {
+    const uint4 v = *reinterpret_cast<const uint4*>(sQ + sw128_offset(r, c8 * 8, kBM));
+    const float4 za = reinterpret_cast<const float4*>(zs)[2 * c8];
+    const float4 zb = reinterpret_cast<const float4*>(zs)[2 * c8 + 1];
+    const float2 s0 = sigma2<false>(v.x), s1 = sigma2<true>(v.y);
+    const float2 s2 = sigma2<false>(v.z), s3 = sigma2<true>(v.w);
+    float* o = sg + c8 * 8;
+    o[0] = s0.x; o[1] = s0.y; o[2] = s1.x; o[3] = s1.y;
+    o[4] = s2.x; o[5] = s2.y; o[6] = s3.x; o[7] = s3.y;
+    float& a = acc[c8 & 3];
+    a = fmaf(s0.y, za.y, fmaf(s0.x, za.x, a));
+    a = fmaf(s1.y, za.w, fmaf(s1.x, za.z, a));
+    a = fmaf(s2.y, zb.y, fmaf(s2.x, zb.x, a));
+    a = fmaf(s3.y, zb.w, fmaf(s3.x, zb.z, a));
   }
   return (acc[0] + acc[1]) + (acc[2] + acc[3]);
 }
 
-// Row r of the query tile replaced, in place, by bf16(sigma(q_r) * c), four
-// 16-byte chunks at a time.
+// Row r of the query tile replaced, in place, by bf16(sg * c).
 template <int D>
-__device__ __forceinline__ void sigma_scale_row(unsigned char* sQ, int r, float c) {
-#pragma unroll 2
-  for (int c8 = 0; c8 < D / 8; c8 += 4) {
-    uint4 v[4];
+__device__ __forceinline__ void store_scaled_row(unsigned char* sQ, int r, const float* sg, float c) {
 #pragma unroll
-    for (int i = 0; i < 4; ++i) v[i] = *reinterpret_cast<const uint4*>(sQ + sw128_offset(r, (c8 + i) * 8, kBM));
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const float2 s0 = sigma2<false>(v[i].x), s1 = sigma2<true>(v[i].y);
-      const float2 s2 = sigma2<false>(v[i].z), s3 = sigma2<true>(v[i].w);
-      v[i] = make_uint4(pack_bf16x2(s0.x * c, s0.y * c), pack_bf16x2(s1.x * c, s1.y * c),
-                        pack_bf16x2(s2.x * c, s2.y * c), pack_bf16x2(s3.x * c, s3.y * c));
-    }
-#pragma unroll
-    for (int i = 0; i < 4; ++i) *reinterpret_cast<uint4*>(sQ + sw128_offset(r, (c8 + i) * 8, kBM)) = v[i];
+  for (int c8 = 0; c8 < D / 8; ++c8) {
+    const float* v = sg + c8 * 8;
+    *reinterpret_cast<uint4*>(sQ + sw128_offset(r, c8 * 8, kBM)) =
+        make_uint4(pack_bf16x2(v[0] * c, v[1] * c), pack_bf16x2(v[2] * c, v[3] * c),
+                   pack_bf16x2(v[4] * c, v[5] * c), pack_bf16x2(v[6] * c, v[7] * c));
   }
 }
 
@@ -631,7 +620,7 @@ tc_attention(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
       const uint32_t qb = 2 * x + (ic & 1u);
       unsigned char* sQ = smem + SM::kQ + qb * kTileBytes;
       const float* zs = reinterpret_cast<const float*>(smem + SM::kZ + qb * D * 4);
-      float m_run = -INFINITY, l_run = 0.f, den = 0.f;
+      float m_run = -INFINITY, l_run = 0.f;
       for (int j = 0; j < n; ++j) {
         ok = __all_sync(0xffffffffu, mbar_wait(s_full + x, sc & 1u, abort, status));
         ++sc;
@@ -698,22 +687,24 @@ tc_attention(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
         tc_fence_before();
         warp_arrive(p_ready + x);
         if (j == 0) {
-          // While the tensor core works on: the previous output store of this
-          // slot has long read its buffer, which the producer may now refill;
-          // and the retrieval denominator sigma(q_r) . z_{s-1} (fp32).  (The
-          // tile and its z landed before the first scores; the wait makes
-          // the copy visible to this thread.)
+          // The previous output store of this slot has long read its buffer,
+          // which the producer may now refill.
           if (store_pending && lane == 0) {
             tma_store_wait_read();
             mbar_arrive(q_empty + pend_b);
           }
           store_pending = false;
-          ok = __all_sync(0xffffffffu, mbar_wait(q_full + qb, (ic >> 1) & 1u, abort, status));
-          if (!ok) break;
-          den = sigma_dot_z<D>(sQ, r, zs);
         }
       }
       if (!ok) break;
+      // sigma(q_r) and the retrieval denominator sigma(q_r) . z_{s-1} (fp32),
+      // in one pass.  (The tile and its z landed before the first scores;
+      // the wait makes the copy visible to this thread.  Every QK^T of this
+      // slot is complete once its last score tile arrived.)
+      ok = __all_sync(0xffffffffu, mbar_wait(q_full + qb, (ic >> 1) & 1u, abort, status));
+      if (!ok) break;
+      float sg[D];
+      const float den = sigma_row<D>(sQ, r, zs, sg);
       // out = (1 - g)/l * O + g/den * sigma(Q) M.  The retrieval enters O
       // through its rows: R' = (sigma(q_r) c_r) M with c_r = g l / ((1 - g) den),
       // so out = (1 - g)/l * (O + R').  With g == 1 (only the retrieval is
@@ -728,8 +719,7 @@ tc_attention(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
         cr = den != 0.f ? gm * l_run / ((1.f - gm) * den) : 0.f;
         so = (1.f - gm) / l_run;
       }
-      // (Every QK^T of this slot is complete once its last score tile arrived.)
-      sigma_scale_row<D>(sQ, r, cr);
+      store_scaled_row<D>(sQ, r, sg, cr);
       fence_proxy_async();
       warp_arrive(sq_ready + x);
       ok = __all_sync(0xffffffffu, mbar_wait(r_full + x, ic & 1u, abort, status));
