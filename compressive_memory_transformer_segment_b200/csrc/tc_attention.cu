@@ -12,7 +12,8 @@
 //
 // Persistent kernel, one CTA per SM.  A work item is a PAIR of query tiles
 // that read the same keys: two query heads of one KV group at the same tile
-// position.  The pair's two tiles ("slots" A and B) each have their own
+// position, or, with one query head per KV head, tiles qt and qt - 1 of one
+// head (the second skips the first's diagonal key tile).  The pair's two tiles ("slots" A and B) each have their own
 // softmax warpgroup and TMEM columns and take turns with the tensor core:
 // while one slot's softmax runs, the tensor core computes the other slot's
 // P.V and next scores.  Items are ordered by (segment, batch row, KV head)
@@ -20,8 +21,8 @@
 // in units of two, an item and its mirror image in the group's order
 // (heaviest with lightest), so that every unit costs the same and the CTAs,
 // which work on a few neighbouring groups at any moment, share those groups'
-// keys in L2.  (With one query head per KV head the one-tile-per-CTA kernel
-// runs instead.)
+// keys in L2.  (With one query head per KV head and d = 64 the
+// one-tile-per-CTA kernel runs instead.)
 //
 // Roles (384 threads, three warpgroups; the first gives registers to the
 // other two with setmaxnreg):
@@ -858,10 +859,10 @@ bool tc_attention_supported(int d_k, int d_v, int S, bool bf16) {
 cudaError_t launch_tc_attention(const Problem& p, cudaStream_t stream) {
   // Segments shorter than a query tile: several segments per tile.
   if (p.S < kBM) return launch_tc_small_attention(p, stream);
-  // With one query head per KV head, a work item would pair tiles of two
-  // heads that share no keys; the one-tile-per-CTA kernel (two CTAs per SM)
-  // runs there.
-  if (p.H_q == p.H_kv) return launch_tc_attention_single(p, stream);
+  // With one query head per KV head a work item pairs query tiles qt and
+  // qt - 1 of one head (the second skips the first's last key tile).  At
+  // d = 64 the one-tile-per-CTA kernel (two CTAs per SM) is faster there.
+  if (p.H_q == p.H_kv && p.d_k == 64) return launch_tc_attention_single(p, stream);
   if (p.d_k == 128) return launch<128>(p, stream);
   if (p.d_k == 64) return launch<64>(p, stream);
   return cudaErrorInvalidValue;
