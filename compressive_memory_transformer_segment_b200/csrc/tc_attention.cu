@@ -536,54 +536,67 @@ tc_attention(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
         // Retrieval folded into O: O += R' = (rows of sigma(Q), scaled by the
         // softmax warps) M_{s-1}, as soon as a slot's rows are in.  With the
         // gate at exactly 1 the softmax part drops out and R' overwrites O
-        // instead.
+        // instead.  Then the next item's first scores (a slot's score columns
+        // are free once its last P.V, issued before, has read them), so the
+        // softmax warps find them ready when they are through with this item.
         const uint64_t dm = dm0 + (((mi % kRing) * kTileBytes) >> 4);
-        bool m_ready = false;
-#pragma unroll
-        for (int x = 0; x < 2; ++x) {
-          if (it.n[x] == 0) continue;
-          const bool keep = gate_sigmoid(__ldg(beta + it.h[x])) != 1.f;
-          if (!(ok = __all_sync(0xffffffffu, mbar_wait(sq_ready + x, ic[x] & 1u, abort, status)))) break;
-          if (!m_ready && !(ok = wait_entry(mi))) break;
+        uint32_t icn[2];
+        for (int x = 0; x < 2; ++x) icn[x] = ic[x] + (it.n[x] > 0 ? 1u : 0u);
+        Item nx;
+        const bool has_next = seq_valid(k + 1, sh);
+        if (has_next) nx = seq_item(k + 1, sh);
+        const bool next_busy = has_next && nx.n_max > 0;
+        bool m_ready = false, k0_ready = false;
+        auto retrieval = [&](int x) -> bool {
+          const uint32_t icx = x ? ic[1] : ic[0];
+          const int hx = x ? it.h[1] : it.h[0];
+          const bool keep = gate_sigmoid(__ldg(beta + hx)) != 1.f;
+          if (!__all_sync(0xffffffffu, mbar_wait(sq_ready + x, icx & 1u, abort, status))) return false;
+          if (!m_ready && !wait_entry(mi)) return false;
           m_ready = true;
           tc_fence_after();
           if (elect_one()) {
             const uint32_t tO = tmem + x * 256 + 128;
-            const uint64_t dq = dq0 + (((2 * x + (ic[x] & 1u)) * kTileBytes) >> 4);
+            const uint64_t dq = dq0 + (((2 * x + (icx & 1u)) * kTileBytes) >> 4);
 #pragma unroll
             for (int kk = 0; kk < D / 16; ++kk)
-              mma_ss(tO, dq + kmajor_step(kk, kBM), dm + mnmajor_step(kk), idesc_pv,
-                     (kk > 0 || keep) ? 1u : 0u);
+              mma_ss(tO, dq + kmajor_step(kk, kBM), dm + mnmajor_step(kk), idesc_pv, (kk > 0 || keep) ? 1u : 0u);
             tc_commit(r_full + x);
           }
+          return true;
+        };
+        auto first_scores = [&](int x) -> bool {
+          const uint32_t icnx = x ? icn[1] : icn[0];
+          if (!__all_sync(0xffffffffu, mbar_wait(q_full + 2 * x + (icnx & 1u), (icnx >> 1) & 1u, abort, status)))
+            return false;
+          if (!k0_ready && !wait_entry(next_base)) return false;
+          k0_ready = true;
+          tc_fence_after();
+          if (elect_one()) issue_qk(x, 2 * x + (icnx & 1u), next_base);
+          return true;
+        };
+        // With equal slots, each slot's next scores go right behind its R';
+        // otherwise (the second slot has one key tile less, one query head
+        // per KV head) both R' first, which measured faster there.
+        const bool interleave = it.n[0] == it.n[1];
+        const int nn0 = next_busy ? nx.n[0] : 0, nn1 = next_busy ? nx.n[1] : 0;
+#pragma unroll
+        for (int x = 0; x < 2; ++x) {
+          if ((x ? it.n[1] : it.n[0]) > 0 && !(ok = retrieval(x))) break;
+          if (interleave && (x ? nn1 : nn0) > 0 && !(ok = first_scores(x))) break;
+        }
+        if (ok && !interleave) {
+#pragma unroll
+          for (int x = 0; x < 2; ++x)
+            if ((x ? nn1 : nn0) > 0 && !(ok = first_scores(x))) break;
         }
         if (!ok) break;
-        if (elect_one()) tc_commit(empty + mi % kRing);
-        uint32_t icn[2];
-        for (int x = 0; x < 2; ++x) icn[x] = ic[x] + (it.n[x] > 0 ? 1u : 0u);
-        // The next item's first scores (a slot's score columns are free once
-        // its last P.V, issued above, has read them); the softmax warps find
-        // them ready when they are through with this item.
-        pre = false;
-        if (seq_valid(k + 1, sh)) {
-          const Item nx = seq_item(k + 1, sh);
-          if (nx.n_max > 0) {
-#pragma unroll
-            for (int x = 0; x < 2; ++x) {
-              if (nx.n[x] == 0) continue;
-              if (!(ok = __all_sync(0xffffffffu, mbar_wait(q_full + 2 * x + (icn[x] & 1u), (icn[x] >> 1) & 1u,
-                                                           abort, status))))
-                break;
-              if ((x == 0 || nx.n[0] == 0) && !(ok = wait_entry(next_base))) break;
-              tc_fence_after();
-              if (elect_one()) issue_qk(x, 2 * x + (icn[x] & 1u), next_base);
-            }
-            if (!ok) break;
-            // Both slots' first scores read K_0; release it.
-            if (elect_one()) tc_commit(empty + next_base % kRing);
-            pre = true;
-          }
+        if (elect_one()) {
+          tc_commit(empty + mi % kRing);
+          // Both slots' first scores read K_0 of the next item; release it.
+          if (next_busy) tc_commit(empty + next_base % kRing);
         }
+        pre = next_busy;
         ic[0] = icn[0];
         ic[1] = icn[1];
         base = next_base;
