@@ -241,19 +241,13 @@ __device__ __forceinline__ float exp_pack64(const uint32_t* sv, float sl2, float
 }
 
 // sigma(x) = x + 1 (x > 0), e^x (x <= 0) of a bf16 pair, in fp32; e^x as
-// 2^(x log2 e) on the MUFU unit or (POLY) on the FMA pipe.
-template <bool POLY>
+// 2^(x log2 e) on the MUFU unit (which measured faster here than sharing the
+// work with the FMA pipe: the end of an item has no MUFU-heavy softmax
+// running beside it).
 __device__ __forceinline__ float2 sigma2(uint32_t w) {
   const float2 xv = make_float2(bf16lo_to_f32(w), bf16hi_to_f32(w));
-  const float2 xe = make_float2(xv.x * 1.4426950408889634f, xv.y * 1.4426950408889634f);
-  float2 e;
-  if (POLY) {
-    e = exp2_poly2<false>(xe);
-  } else {
-    e.x = ex2_approx(xe.x);
-    e.y = ex2_approx(xe.y);
-  }
-  return make_float2(xv.x > 0.f ? xv.x + 1.f : e.x, xv.y > 0.f ? xv.y + 1.f : e.y);
+  const float ex = ex2_approx(xv.x * 1.4426950408889634f), ey = ex2_approx(xv.y * 1.4426950408889634f);
+  return make_float2(xv.x > 0.f ? xv.x + 1.f : ex, xv.y > 0.f ? xv.y + 1.f : ey);
 }
 
 // sigma(q_r) of row r of a 128-row query tile in shared memory, into sg[D]
@@ -267,8 +261,7 @@ __device__ __forceinline__ float sigma_row(const unsigned char* sQ, int r, const
     const uint4 v = *reinterpret_cast<const uint4*>(sQ + sw128_offset(r, c8 * 8, kBM));
     const float4 za = reinterpret_cast<const float4*>(zs)[2 * c8];
     const float4 zb = reinterpret_cast<const float4*>(zs)[2 * c8 + 1];
-    const float2 s0 = sigma2<false>(v.x), s1 = sigma2<true>(v.y);
-    const float2 s2 = sigma2<false>(v.z), s3 = sigma2<true>(v.w);
+    const float2 s0 = sigma2(v.x), s1 = sigma2(v.y), s2 = sigma2(v.z), s3 = sigma2(v.w);
     float* o = sg + c8 * 8;
     o[0] = s0.x; o[1] = s0.y; o[2] = s1.x; o[3] = s1.y;
     o[4] = s2.x; o[5] = s2.y; o[6] = s3.x; o[7] = s3.y;
@@ -628,9 +621,12 @@ tc_attention(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
     bool ok = true;
     for (int k = 0; ok && seq_valid(k, sh); ++k) {
       const Item it = seq_item(k, sh);
-      const int n = it.n[x];
+      // (selects, not it.n[x]: a struct indexed by a runtime value would live
+      // in local memory, which with almost all of L1 given to shared memory
+      // goes to L2)
+      const int n = x ? it.n[1] : it.n[0];
       if (n == 0) continue;
-      const int qt = it.qt[x], h = it.h[x];
+      const int qt = x ? it.qt[1] : it.qt[0], h = x ? it.h[1] : it.h[0];
       const uint32_t qb = 2 * x + (ic & 1u);
       unsigned char* sQ = smem + SM::kQ + qb * kTileBytes;
       const float* zs = reinterpret_cast<const float*>(smem + SM::kZ + qb * D * 4);
