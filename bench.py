@@ -42,14 +42,17 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # launch, from an ncu capture summarised under profiles/, valid only while the
 # kernel sources hash to what they were at capture time.
 ATTENTION_TRAFFIC = {
-    "8b-delta": {"bytes": 2 * (409.577728e6 + 230.632448e6),
-                 "note": "ncu capture at batch 1, scaled x2 to the batch-2 launch; the file's "
-                         "host dispatch to the one-tile kernel (H_q == H_kv) was added after "
-                         "the capture and the header comment rewritten; the paired kernel's "
-                         "device code is unchanged",
+    "8b-delta": {"bytes": 2 * (409.388544e6 + 231.382016e6),
+                 "note": "ncu capture at batch 1, scaled x2 to the batch-2 launch",
                  "profile": "profiles/tc_attention_8b-delta.md",
-                 "sha1": {"tc_attention.cu": "8054f13e63ddfd60411415ae0c937af5bf12fe6f",
-                          "tc_common.cuh": "a2612deb59163975e015c94465b32bea6a1a4f2d"}},
+                 "sha1": {"tc_attention.cu": "6370c59817bbe2487940b477ce95a2cbc7277627",
+                          "tc_common.cuh": "a896981e1b8e14dfabfd0f26a799d64c0af65a34"}},
+    "1m-linear": {"bytes": 16 * (1.754910e9 + 0.5212416e9),
+                  "note": "ncu capture of the same shape cut to 65,536 tokens, scaled x16 to the "
+                          "1,048,576-token launch (traffic grows with the tokens)",
+                  "profile": "profiles/tc_attention_1m-linear.md",
+                  "sha1": {"tc_attention.cu": "6370c59817bbe2487940b477ce95a2cbc7277627",
+                           "tc_common.cuh": "a896981e1b8e14dfabfd0f26a799d64c0af65a34"}},
 }
 
 
