@@ -719,7 +719,7 @@ tc_pipe_products(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
 
 // ---------------------------------------------------------------- sequential combine
 
-constexpr int kCB = 8;  // columns of M per combine CTA (delta)
+constexpr int kCB = 16;  // columns of M per combine CTA (delta)
 
 __device__ __forceinline__ void cp_async16(void* smem_dst, const void* gmem_src) {
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(smem_dst)), "l"(gmem_src)
@@ -731,9 +731,10 @@ __device__ __forceinline__ void cp_async_wait() {
   asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
 }
 
-// Delta rule: M_s = M_{s-1} - G_s M_{s-1} + B_s on columns [8 cb, 8 cb + 8).
-// Grid (B*H_kv, D/8), block 256 threads: thread -> (row k = tid % 128,
-// 4 columns); rows >= D idle for D = 64.  G_s is symmetric up to the
+// Delta rule: M_s = M_{s-1} - G_s M_{s-1} + B_s on columns [16 cb, 16 cb + 16).
+// Grid (B*H_kv, D/16), block 256 threads: thread -> (row k = tid % 128,
+// 8 columns); rows >= D idle for D = 64.  With 16 columns per CTA the grid
+// of the 8B shape (16 KV heads x 8) is one wave.  G_s is symmetric up to the
 // rounding of its bf16 pair products (the dropped lo*lo term, ~2^-16
 // relative), so row k of G_s M is read from column k of G_s, which makes
 // the shared-memory reads conflict-free; G_{s+1} streams in (cp.async)
@@ -746,18 +747,18 @@ __global__ void __launch_bounds__(256) combine_delta(const float* __restrict__ M
                                                      float* __restrict__ M_out, int T) {
   extern __shared__ __align__(16) float csm[];
   float* sG = csm;               // two G_s buffers [D][D]
-  float* sM = csm + 2 * D * D;   // M_{s-1}[:, 8 columns]
+  float* sM = csm + 2 * D * D;   // M_{s-1}[:, 16 columns]
   const int bh = blockIdx.x, c0 = blockIdx.y * kCB, BH = gridDim.x;
-  const int tid = threadIdx.x, k = tid & 127, cg = (tid >> 7) * 4;
+  const int tid = threadIdx.x, k = tid & 127, cg = (tid >> 7) * 8;
   const bool active = k < D;
   auto load_g = [&](int s, float* dst) {
     const float4* src = reinterpret_cast<const float4*>(Gbuf + ((size_t)s * BH + bh) * D * D);
     for (int e = tid; e < D * D / 4; e += 256) cp_async16(dst + 4 * e, src + e);
     cp_async_commit();
   };
-  float m[4];
+  float m[8];
 #pragma unroll
-  for (int i = 0; i < 4; ++i) m[i] = active ? M_in[((size_t)bh * D + k) * D + c0 + cg + i] : 0.f;
+  for (int i = 0; i < 8; ++i) m[i] = active ? M_in[((size_t)bh * D + k) * D + c0 + cg + i] : 0.f;
   load_g(0, sG);
   for (int s = 0; s < T; ++s) {
     const size_t slice = (size_t)s * BH + bh;
@@ -770,35 +771,48 @@ __global__ void __launch_bounds__(256) combine_delta(const float* __restrict__ M
     }
     // Publish M_{s-1} (bf16) for segment s's retrieval.
     if (active) {
-      uint2 w;
+      uint4 w;
       w.x = pack_bf16x2(m[0], m[1]);
       w.y = pack_bf16x2(m[2], m[3]);
-      *reinterpret_cast<uint2*>(M_pref + (slice * D + k) * D + c0 + cg) = w;
+      w.z = pack_bf16x2(m[4], m[5]);
+      w.w = pack_bf16x2(m[6], m[7]);
+      *reinterpret_cast<uint4*>(M_pref + (slice * D + k) * D + c0 + cg) = w;
       *reinterpret_cast<float4*>(sM + k * kCB + cg) = make_float4(m[0], m[1], m[2], m[3]);
+      *reinterpret_cast<float4*>(sM + k * kCB + cg + 4) = make_float4(m[4], m[5], m[6], m[7]);
     }
     __syncthreads();
     if (active) {
-      float acc[4] = {0.f, 0.f, 0.f, 0.f};
+      float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
 #pragma unroll 8
       for (int kk = 0; kk < D; ++kk) {
         const float gv = G[kk * D + k];
-        const float4 mv = *reinterpret_cast<const float4*>(sM + kk * kCB + cg);
-        acc[0] = fmaf(gv, mv.x, acc[0]);
-        acc[1] = fmaf(gv, mv.y, acc[1]);
-        acc[2] = fmaf(gv, mv.z, acc[2]);
-        acc[3] = fmaf(gv, mv.w, acc[3]);
+        const float4 ma = *reinterpret_cast<const float4*>(sM + kk * kCB + cg);
+        const float4 mb = *reinterpret_cast<const float4*>(sM + kk * kCB + cg + 4);
+        acc[0] = fmaf(gv, ma.x, acc[0]);
+        acc[1] = fmaf(gv, ma.y, acc[1]);
+        acc[2] = fmaf(gv, ma.z, acc[2]);
+        acc[3] = fmaf(gv, ma.w, acc[3]);
+        acc[4] = fmaf(gv, mb.x, acc[4]);
+        acc[5] = fmaf(gv, mb.y, acc[5]);
+        acc[6] = fmaf(gv, mb.z, acc[6]);
+        acc[7] = fmaf(gv, mb.w, acc[7]);
       }
-      const float4 bk = *reinterpret_cast<const float4*>(Bbuf + (slice * D + k) * D + c0 + cg);
-      m[0] = (m[0] - acc[0]) + bk.x;
-      m[1] = (m[1] - acc[1]) + bk.y;
-      m[2] = (m[2] - acc[2]) + bk.z;
-      m[3] = (m[3] - acc[3]) + bk.w;
+      const float4* bk = reinterpret_cast<const float4*>(Bbuf + (slice * D + k) * D + c0 + cg);
+      const float4 ba = bk[0], bb = bk[1];
+      m[0] = (m[0] - acc[0]) + ba.x;
+      m[1] = (m[1] - acc[1]) + ba.y;
+      m[2] = (m[2] - acc[2]) + ba.z;
+      m[3] = (m[3] - acc[3]) + ba.w;
+      m[4] = (m[4] - acc[4]) + bb.x;
+      m[5] = (m[5] - acc[5]) + bb.y;
+      m[6] = (m[6] - acc[6]) + bb.z;
+      m[7] = (m[7] - acc[7]) + bb.w;
     }
     __syncthreads();
   }
   if (active)
 #pragma unroll
-    for (int i = 0; i < 4; ++i) M_out[((size_t)bh * D + k) * D + c0 + cg + i] = m[i];
+    for (int i = 0; i < 8; ++i) M_out[((size_t)bh * D + k) * D + c0 + cg + i] = m[i];
 }
 
 // Linear rule: M_s = M_{s-1} + B_s, z_s = z_{s-1} + dz_s, element-parallel.
@@ -816,17 +830,27 @@ __global__ void __launch_bounds__(256) combine_linear(const float* __restrict__ 
   const int e = (blockIdx.y * 256 + threadIdx.x) * 4;  // element of the D x D matrix
   if (e < D * D) {
     float4 m = *reinterpret_cast<const float4*>(M_in + (size_t)bh * D * D + e);
-    for (int s = 0; s < T; ++s) {
-      const size_t slice = (size_t)s * BH + bh;
-      uint2 w;
-      w.x = pack_bf16x2(m.x, m.y);
-      w.y = pack_bf16x2(m.z, m.w);
-      *reinterpret_cast<uint2*>(M_pref + slice * D * D + e) = w;
-      const float4 b = *reinterpret_cast<const float4*>(Bbuf + slice * D * D + e);
-      m.x += b.x;
-      m.y += b.y;
-      m.z += b.z;
-      m.w += b.w;
+    // The products of kAhead segments are loaded before they are added, so
+    // that many loads are in flight per thread (the walk itself is serial).
+    constexpr int kAhead = 8;
+    for (int s0 = 0; s0 < T; s0 += kAhead) {
+      float4 b[kAhead];
+#pragma unroll
+      for (int i = 0; i < kAhead; ++i)
+        if (s0 + i < T)
+          b[i] = *reinterpret_cast<const float4*>(Bbuf + ((size_t)(s0 + i) * BH + bh) * D * D + e);
+#pragma unroll
+      for (int i = 0; i < kAhead; ++i) {
+        if (s0 + i >= T) break;
+        uint2 w;
+        w.x = pack_bf16x2(m.x, m.y);
+        w.y = pack_bf16x2(m.z, m.w);
+        *reinterpret_cast<uint2*>(M_pref + ((size_t)(s0 + i) * BH + bh) * D * D + e) = w;
+        m.x += b[i].x;
+        m.y += b[i].y;
+        m.z += b[i].z;
+        m.w += b[i].w;
+      }
     }
     *reinterpret_cast<float4*>(M_out + (size_t)bh * D * D + e) = m;
   }
