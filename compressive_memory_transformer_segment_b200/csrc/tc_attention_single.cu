@@ -263,26 +263,6 @@ tc_attention_single(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     const float sl2 = rsqrtf((float)D) * 1.4426950408889634f;
     float m_run = -INFINITY, l_run = 0.f;
     bool ok = true;
-    // The retrieval denominator sigma(q_r) . z_{s-1} in fp32, while the first
-    // score tile is being computed.
-    float den = 0.f;
-    ok = __all_sync(0xffffffffu, mbar_wait(bar_q, 0, abort, status));
-    if (ok) {
-      const float4* z4 = reinterpret_cast<const float4*>(z_pref + (size_t)mslice * D);
-#pragma unroll 4
-      for (int c8 = 0; c8 < D / 8; ++c8) {
-        const uint4 v = *reinterpret_cast<const uint4*>(sQ + sw128_offset(r, c8 * 8, kBM));
-        const float4 za = __ldg(z4 + 2 * c8), zb = __ldg(z4 + 2 * c8 + 1);
-        den = fmaf(elu1_fast(bf16lo_to_f32(v.x)), za.x, den);
-        den = fmaf(elu1_fast(bf16hi_to_f32(v.x)), za.y, den);
-        den = fmaf(elu1_fast(bf16lo_to_f32(v.y)), za.z, den);
-        den = fmaf(elu1_fast(bf16hi_to_f32(v.y)), za.w, den);
-        den = fmaf(elu1_fast(bf16lo_to_f32(v.z)), zb.x, den);
-        den = fmaf(elu1_fast(bf16hi_to_f32(v.z)), zb.y, den);
-        den = fmaf(elu1_fast(bf16lo_to_f32(v.w)), zb.z, den);
-        den = fmaf(elu1_fast(bf16hi_to_f32(v.w)), zb.w, den);
-      }
-    }
     for (int j = 0; ok && j < n_kv; ++j) {
       ok = __all_sync(0xffffffffu, mbar_wait(s_full, j & 1, abort, status));
       if (!ok) break;
@@ -400,18 +380,36 @@ tc_attention_single(const __grid_constant__ CUtensorMap tm_q, const __grid_const
       if (lane == 0) mbar_arrive(p_ready);
     }
     // sigma(Q) in place of Q (every QK^T product is complete once the last
-    // score tile arrived).
+    // score tile arrived), and in the same pass the retrieval denominator
+    // sigma(q_r) . z_{s-1} in fp32 from the unrounded sigma.  (The wait on
+    // the query tile's barrier makes its copy visible to this thread.)
+    float den = 0.f;
+    if (ok) ok = __all_sync(0xffffffffu, mbar_wait(bar_q, 0, abort, status));
     if (ok) {
+      const float4* z4 = reinterpret_cast<const float4*>(z_pref + (size_t)mslice * D);
+      float dacc[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll 4
       for (int c8 = 0; c8 < D / 8; ++c8) {
         const uint32_t off = sw128_offset(r, c8 * 8, kBM);
-        uint4 v = *reinterpret_cast<uint4*>(sQ + off);
-        uint32_t w[4] = {v.x, v.y, v.z, v.w};
+        const uint4 v = *reinterpret_cast<uint4*>(sQ + off);
+        const float4 za = __ldg(z4 + 2 * c8), zb = __ldg(z4 + 2 * c8 + 1);
+        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+        float sg[8];
 #pragma unroll
-        for (int i = 0; i < 4; ++i)
-          w[i] = pack_bf16x2(elu1_fast(bf16lo_to_f32(w[i])), elu1_fast(bf16hi_to_f32(w[i])));
-        *reinterpret_cast<uint4*>(sQ + off) = make_uint4(w[0], w[1], w[2], w[3]);
+        for (int i = 0; i < 4; ++i) {
+          sg[2 * i] = elu1_fast(bf16lo_to_f32(w[i]));
+          sg[2 * i + 1] = elu1_fast(bf16hi_to_f32(w[i]));
+        }
+        float& a = dacc[c8 & 3];
+        a = fmaf(sg[1], za.y, fmaf(sg[0], za.x, a));
+        a = fmaf(sg[3], za.w, fmaf(sg[2], za.z, a));
+        a = fmaf(sg[5], zb.y, fmaf(sg[4], zb.x, a));
+        a = fmaf(sg[7], zb.w, fmaf(sg[6], zb.z, a));
+        *reinterpret_cast<uint4*>(sQ + off) =
+            make_uint4(pack_bf16x2(sg[0], sg[1]), pack_bf16x2(sg[2], sg[3]), pack_bf16x2(sg[4], sg[5]),
+                       pack_bf16x2(sg[6], sg[7]));
       }
+      den = (dacc[0] + dacc[1]) + (dacc[2] + dacc[3]);
       fence_proxy_async();
       __syncwarp();
       if (lane == 0) mbar_arrive(sq_ready);
