@@ -103,39 +103,44 @@ int zsum_chunks(int S) { return S >= 256 * kZChunksMax ? kZChunksMax : (S >= 512
 
 // ---------------------------------------------------------------- segment products
 
-constexpr int kTok = 128;  // tokens per block
+// Tokens per block: 128, or 64 for segments of at most 64 tokens (half the
+// shared memory, so more CTAs fit on an SM when a segment is one block).
 constexpr int kThreads = 192;
-constexpr uint32_t kTmemCols = 256;
 
-template <int D, bool DELTA>
+template <int D, bool DELTA, int TOK>
 struct ProdSmem {
-  static constexpr int kK = 0;                                      // K block [128][D]
-  static constexpr int kV = kK + kTok * D * 2;                      // V block [128][D] (+ ones)
-  static constexpr int kVBytes = kTok * D * 2 + (DELTA ? 0 : kTok * 64 * 2);
-  static constexpr int kSkHi = kV + kVBytes;                        // [128 tok][128] (2 panels)
-  static constexpr int kSkLo = kSkHi + kTok * 128 * 2;
-  static constexpr int kYHi = kSkLo + kTok * 128 * 2;               // delta only
-  static constexpr int kYLo = kYHi + (DELTA ? kTok * 128 * 2 : 0);
-  static constexpr int kZ = kYLo + (DELTA ? kTok * 128 * 2 : 0);    // fp32 z_{s-1}
+  static constexpr int kK = 0;                                      // K block [TOK][D]
+  static constexpr int kV = kK + TOK * D * 2;                       // V block [TOK][D] (+ ones)
+  static constexpr int kVBytes = TOK * D * 2 + (DELTA ? 0 : TOK * 64 * 2);
+  static constexpr int kSkHi = kV + kVBytes;                        // [TOK tok][128] (2 panels)
+  static constexpr int kSkLo = kSkHi + TOK * 128 * 2;
+  static constexpr int kYHi = kSkLo + TOK * 128 * 2;                // delta only
+  static constexpr int kYLo = kYHi + (DELTA ? TOK * 128 * 2 : 0);
+  static constexpr int kZ = kYLo + (DELTA ? TOK * 128 * 2 : 0);     // fp32 z_{s-1}
   static constexpr int kBar = kZ + 128 * 4;
   // k_full k_empty v_full v_empty op_ready op_free done
   static constexpr int kNumBars = 7;
   static constexpr int kTmemSlot = kBar + kNumBars * 8;
   static constexpr int kAbort = kTmemSlot + 4;
   static constexpr int kAlloc = kAbort + 4 + 1024;
+  // TMEM: delta G [0, 128) and B [128, 128 + D); linear [B | dz] [0, D + 16).
+  static constexpr uint32_t kTmemCols = (DELTA || D + 16 > 128) ? 256 : 128;
 };
 
 // Grid (T, B*H_kv).  Roles: warp 0 TMA producer (K, V blocks), warp 1 TMEM
-// allocation + MMA issue, warps 2..5 one thread per token of the block (and,
-// at the end, per row of the products).
+// allocation + MMA issue, warps 2..5 one thread per token of the block (the
+// threads of rows 64..127 idle with 64-token blocks) and, at the end, one per
+// row of the products.
 // TMEM: delta G [0, D), B [128, 128 + D); linear [B | dz] [0, D + 16).
-template <int D, bool DELTA>
+template <int D, bool DELTA, int TOK>
 __global__ void __launch_bounds__(kThreads, 1)
 tc_segment_products(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                     const float* __restrict__ z_pref, float* __restrict__ Gbuf,
                     float* __restrict__ Bbuf, float* __restrict__ dz,
                     unsigned int* __restrict__ status, int L, int S) {
-  using SM = ProdSmem<D, DELTA>;
+  using SM = ProdSmem<D, DELTA, TOK>;
+  constexpr int kTok = TOK;
+  constexpr uint32_t kTmemCols = SM::kTmemCols;
   const int s = blockIdx.x, bh = blockIdx.y, BH = gridDim.y;
   const int seg0 = s * S, seg_len = min(S, L - seg0);
   const int nblk = (seg_len + kTok - 1) / kTok;
@@ -295,14 +300,16 @@ tc_segment_products(const __grid_constant__ CUtensorMap tm_k, const __grid_const
       }
       ok = __all_sync(0xffffffffu, mbar_wait(k_full, blk & 1, abort, status));
       if (!ok) break;
-      const bool valid = blk * kTok + t < seg_len;
+      // (with 64-token blocks the threads of rows 64..127 have no token)
+      const bool has_tok = t < kTok;
+      const bool valid = has_tok && blk * kTok + t < seg_len;
       // sigma(K) row t as hi/lo pairs (rows past the segment are 0), and
       // r_t = sigma(k_t) . z_{s-1} (delta).
       float r = 0.f;
 #pragma unroll 4
       for (int c8 = 0; c8 < D / 8; ++c8) {
         const uint32_t off = sw128_offset(t, 8 * c8, kTok);
-        const uint4 kv = *reinterpret_cast<const uint4*>(sK + off);
+        const uint4 kv = has_tok ? *reinterpret_cast<const uint4*>(sK + off) : make_uint4(0, 0, 0, 0);
         const uint32_t kw[4] = {kv.x, kv.y, kv.z, kv.w};
         float zc[8];
         if (DELTA) {
@@ -323,12 +330,14 @@ tc_segment_products(const __grid_constant__ CUtensorMap tm_k, const __grid_const
           hw[i] = pack_bf16x2(a, b);
           lw[i] = pack_bf16x2(a - bf16lo_to_f32(hw[i]), b - bf16hi_to_f32(hw[i]));
         }
-        *reinterpret_cast<uint4*>(sSkHi + off) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
-        *reinterpret_cast<uint4*>(sSkLo + off) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
+        if (has_tok) {
+          *reinterpret_cast<uint4*>(sSkHi + off) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+          *reinterpret_cast<uint4*>(sSkLo + off) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
+        }
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(k_empty);
-      if (DELTA) {
+      if (DELTA && has_tok) {
         // Y = sigma(K) / r (0 where r = 0), from the pair just written.
         const float w = r != 0.f ? 1.f / r : 0.f;
 #pragma unroll 4
@@ -898,11 +907,11 @@ bool make_map(CUtensorMap* m, const void* base, uint64_t cols, uint64_t rows, ui
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int D, bool DELTA>
+template <int D, bool DELTA, int TOK>
 cudaError_t launch_products(const Problem& p, const CUtensorMap& tk, const CUtensorMap& tv,
                             cudaStream_t stream) {
-  const int smem = ProdSmem<D, DELTA>::kAlloc;
-  auto kern = tc_segment_products<D, DELTA>;
+  const int smem = ProdSmem<D, DELTA, TOK>::kAlloc;
+  auto kern = tc_segment_products<D, DELTA, TOK>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
   kern<<<dim3(p.T, p.B * p.H_kv), kThreads, smem, stream>>>(tk, tv, p.z_pref, p.Gbuf, p.Bbuf, p.dz,
@@ -929,7 +938,10 @@ template <int D>
 cudaError_t launch(const Problem& p, cudaStream_t stream) {
   CUtensorMap tk, tv;
   const uint64_t BHkv = (uint64_t)p.B * p.H_kv;
-  if (!make_map(&tk, p.k, D, p.L, BHkv, kTok) || !make_map(&tv, p.v, D, p.L, BHkv, kTok))
+  // 64-token blocks when a segment fits in one (see ProdSmem).
+  const bool small = p.S <= 64;
+  const uint32_t tok = small ? 64 : 128;
+  if (!make_map(&tk, p.k, D, p.L, BHkv, tok) || !make_map(&tv, p.v, D, p.L, BHkv, tok))
     return cudaErrorInvalidValue;
   const unsigned BH = (unsigned)BHkv;
   __nv_bfloat16* Mp = static_cast<__nv_bfloat16*>(p.M_pref);
@@ -944,7 +956,7 @@ cudaError_t launch(const Problem& p, cudaStream_t stream) {
     if (D == 128)
       e = launch_pipe_products<true>(p, stream);
     else
-      e = launch_products<D, true>(p, tk, tv, stream);
+      e = small ? launch_products<D, true, 64>(p, tk, tv, stream) : launch_products<D, true, 128>(p, tk, tv, stream);
     if (e != cudaSuccess) return e;
     const int csmem = (2 * D * D + D * kCB) * (int)sizeof(float);
     e = cudaFuncSetAttribute(combine_delta<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, csmem);
@@ -956,7 +968,8 @@ cudaError_t launch(const Problem& p, cudaStream_t stream) {
   if (D == 128)
     e = launch_pipe_products<false>(p, stream);
   else
-    e = launch_products<D, false>(p, tk, tv, stream);
+    e = small ? launch_products<D, false, 64>(p, tk, tv, stream)
+              : launch_products<D, false, 128>(p, tk, tv, stream);
   if (e != cudaSuccess) return e;
   combine_linear<D><<<dim3(BH, (D * D + 1023) / 1024), 256, 0, stream>>>(
       p.M_in, p.Bbuf, p.dz, Mp, p.z_pref, p.M_out, p.z_out, p.T);

@@ -263,6 +263,16 @@ TC_CASES = [
                                      H_kv=2, rule="delta")),
     ("tc_d128_gqa2_S256_ragged", dict(dtype="bf16", d_k=128, d_v=128, L=700, seg_len=256, B=2,
                                       H_q=4, H_kv=2)),
+    # One query head per KV head at d = 128 (work items pair tiles qt and qt - 1
+    # of one head, so the second tile has one key tile less), several items
+    # per CTA and a ragged last segment.
+    ("tc_d128_mha_S512_ragged", dict(dtype="bf16", d_k=128, d_v=128, L=1500, seg_len=512, B=2,
+                                     H_q=3, H_kv=3, rule="delta")),
+    # Three query heads per KV head at d = 128: items whose two tiles sit at
+    # different positions (unequal key-tile counts) next to items with equal
+    # ones, so both orders of the end-of-item retrieval and next scores run.
+    ("tc_d128_gqa3_S384_ragged", dict(dtype="bf16", d_k=128, d_v=128, L=1000, seg_len=384, H_q=6,
+                                      H_kv=2)),
     # Segments shorter than a query tile (several segments per tile, the
     # short-segment kernel): a ragged last segment and a last tile that ends
     # past the sequence; four segments per tile with GQA, where the last
