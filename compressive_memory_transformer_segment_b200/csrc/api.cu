@@ -142,6 +142,13 @@ unsigned int* status_ptr() {
   return static_cast<unsigned int*>(p);
 }
 
+// Slot 0 of z_pref (z_in, read by segment 0): copied in for the SIMT scan;
+// the tensor-core scan writes it itself (one operation less per forward).
+cudaError_t seed_z(const Shape& s, const Problem& p, cudaStream_t st) {
+  if (s.path == INFINI_PATH_TCGEN05) return cudaSuccess;
+  return cudaMemcpyAsync(p.z_pref, p.z_in, s.z_bytes, cudaMemcpyDeviceToDevice, st);
+}
+
 // The state scan of the path `s` takes.
 cudaError_t launch_state_scan(const Shape& s, const Problem& p, cudaStream_t st) {
   if (s.path != INFINI_PATH_TCGEN05) return launch_simt_state_scan(p, st);
@@ -155,7 +162,7 @@ cudaError_t run_state_scan(const Shape& s, const void* k, const void* v, const f
                            const float* z_in, float* M_out, float* z_out, char* ws,
                            unsigned int* status, cudaStream_t st) {
   Problem p;
-  p.q = nullptr; p.k = k; p.v = v; p.beta = nullptr; p.M_in = M_in;
+  p.q = nullptr; p.k = k; p.v = v; p.beta = nullptr; p.M_in = M_in; p.z_in = z_in;
   p.out = nullptr; p.M_out = M_out; p.z_out = z_out;
   p.B = s.B; p.H_q = s.H_q; p.H_kv = s.H_kv; p.L = s.L; p.d_k = s.d_k; p.d_v = s.d_v;
   p.S = s.S; p.T = s.T; p.bf16 = s.bf16; p.delta = s.delta;
@@ -166,7 +173,7 @@ cudaError_t run_state_scan(const Shape& s, const void* k, const void* v, const f
   p.Bbuf = reinterpret_cast<float*>(ws + s.ws_b);
   p.dz = reinterpret_cast<float*>(ws + s.ws_dz);
   p.status = status;
-  cudaError_t e = cudaMemcpyAsync(p.z_pref, z_in, s.z_bytes, cudaMemcpyDeviceToDevice, st);
+  cudaError_t e = seed_z(s, p, st);
   if (e == cudaSuccess) e = timed(0, st, [&] { return launch_state_scan(s, p, st); });
   return e;
 }
@@ -292,7 +299,7 @@ int infini_attn_forward(const void* q, const void* k, const void* v, const float
     owned = true;
   }
   Problem p;
-  p.q = q; p.k = k; p.v = v; p.beta = beta; p.M_in = M_in;
+  p.q = q; p.k = k; p.v = v; p.beta = beta; p.M_in = M_in; p.z_in = z_in;
   p.out = out; p.M_out = M_out; p.z_out = z_out;
   p.B = s.B; p.H_q = s.H_q; p.H_kv = s.H_kv; p.L = s.L; p.d_k = s.d_k; p.d_v = s.d_v;
   p.S = s.S; p.T = s.T; p.bf16 = s.bf16; p.delta = s.delta;
@@ -304,7 +311,7 @@ int infini_attn_forward(const void* q, const void* k, const void* v, const float
   p.dz = reinterpret_cast<float*>(ws + s.ws_dz);
   p.status = status;
 
-  cudaError_t e = cudaMemcpyAsync(p.z_pref, z_in, s.z_bytes, cudaMemcpyDeviceToDevice, st);
+  cudaError_t e = seed_z(s, p, st);
   if (e == cudaSuccess) e = timed(0, st, [&] { return launch_state_scan(s, p, st); });
   if (e == cudaSuccess)
     e = timed(1, st, [&] {

@@ -14,6 +14,7 @@ struct Problem {
   const void* v;
   const float* beta;
   const float* M_in;
+  const float* z_in;   // the tensor-core scan seeds slot 0 of z_pref from it
   void* out;
   float* M_out;
   float* z_out;
@@ -21,7 +22,8 @@ struct Problem {
   bool bf16;
   bool delta;
   // Workspace views.
-  float* z_pref;       // [T][B*H_kv][d_k] f32: z_{s-1} read by segment s (slot 0 = z_in)
+  float* z_pref;       // [T][B*H_kv][d_k] f32: z_{s-1} read by segment s (slot 0 = z_in:
+                       // copied in before the SIMT scan, written by the tensor-core scan)
   void* M_pref;        // [T][B*H_kv][d_k][d_v]: M_{s-1} (f32 on the SIMT path, bf16 on tcgen05)
   bool M_pref_bf16;    // element type of M_pref
   // Tensor-core scan only: per (segment, KV head) products and column sums.

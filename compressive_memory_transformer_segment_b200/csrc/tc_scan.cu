@@ -83,12 +83,13 @@ __global__ void __launch_bounds__(256) zsum(const __nv_bfloat16* __restrict__ k,
 // z_{s-1} for s = 1..T-1 into z_pref (slot 0 already holds z_in) and z_T,
 // from the C chunk partials of every segment.  Grid (B*H_kv), block D threads.
 template <int D>
-__global__ void __launch_bounds__(128) zprefix(const float* __restrict__ dz, float* __restrict__ z_pref,
-                                               float* __restrict__ z_out, int T, int C) {
+__global__ void __launch_bounds__(128) zprefix(const float* __restrict__ dz, const float* z_in,
+                                               float* __restrict__ z_pref, float* z_out, int T, int C) {
   const int bh = blockIdx.x, c = threadIdx.x, BH = gridDim.x;
-  float z = z_pref[(size_t)bh * D + c];
+  // (z_out may be z_in: this thread reads its entry before it writes it)
+  float z = z_in[(size_t)bh * D + c];
   for (int s = 0; s < T; ++s) {
-    if (s > 0) z_pref[((size_t)s * BH + bh) * D + c] = z;
+    z_pref[((size_t)s * BH + bh) * D + c] = z;
     float seg = 0.f;
     for (int j = 0; j < C; ++j) seg += dz[((size_t)(s * C + j) * BH + bh) * D + c];
     z += seg;
@@ -832,9 +833,10 @@ __global__ void __launch_bounds__(256) combine_linear(const float* __restrict__ 
                                                       const float* __restrict__ Bbuf,
                                                       const float* __restrict__ dz,
                                                       __nv_bfloat16* __restrict__ M_pref,
+                                                      const float* z_in,
                                                       float* __restrict__ z_pref,
-                                                      float* __restrict__ M_out,
-                                                      float* __restrict__ z_out, int T) {
+                                                      float* __restrict__ M_out, float* z_out,
+                                                      int T) {
   const int bh = blockIdx.x, BH = gridDim.x;
   const int e = (blockIdx.y * 256 + threadIdx.x) * 4;  // element of the D x D matrix
   if (e < D * D) {
@@ -865,7 +867,9 @@ __global__ void __launch_bounds__(256) combine_linear(const float* __restrict__ 
   }
   if (blockIdx.y == 0 && threadIdx.x < D) {
     const int c = threadIdx.x;
-    float z = z_pref[(size_t)bh * D + c];  // slot 0 = z_in
+    // (z_out may be z_in: this thread reads its entry before it writes it)
+    float z = z_in[(size_t)bh * D + c];
+    z_pref[(size_t)bh * D + c] = z;  // slot 0, read by segment 0
     for (int s = 1; s < T; ++s) {
       z += dz[((size_t)(s - 1) * BH + bh) * D + c];
       z_pref[((size_t)s * BH + bh) * D + c] = z;
@@ -951,7 +955,7 @@ cudaError_t launch(const Problem& p, cudaStream_t stream) {
     zsum<D><<<dim3(p.T * C, BH), 256, 0, stream>>>(static_cast<const __nv_bfloat16*>(p.k), p.dz, p.L,
                                                    p.S, C);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    zprefix<D><<<BH, D, 0, stream>>>(p.dz, p.z_pref, p.z_out, p.T, C);
+    zprefix<D><<<BH, D, 0, stream>>>(p.dz, p.z_in, p.z_pref, p.z_out, p.T, C);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     if (D == 128)
       e = launch_pipe_products<true>(p, stream);
@@ -972,7 +976,7 @@ cudaError_t launch(const Problem& p, cudaStream_t stream) {
               : launch_products<D, false, 128>(p, tk, tv, stream);
   if (e != cudaSuccess) return e;
   combine_linear<D><<<dim3(BH, (D * D + 1023) / 1024), 256, 0, stream>>>(
-      p.M_in, p.Bbuf, p.dz, Mp, p.z_pref, p.M_out, p.z_out, p.T);
+      p.M_in, p.Bbuf, p.dz, Mp, p.z_in, p.z_pref, p.M_out, p.z_out, p.T);
   return cudaGetLastError();
 }
 
