@@ -431,10 +431,11 @@ constexpr int kLTok = 64;      // tokens per block
 template <bool DELTA>
 struct PipeSmem {
   static constexpr int kD = 128;
-  // Math warps: 16 for the linear rule (2 tokens per thread and block, to
-  // hide the latency of the sigma chain), 8 for the delta rule (its thread
-  // state needs the registers).
-  static constexpr int kMath = DELTA ? 8 : 16;
+  // Math warps: 16 (2 tokens per thread and block, to hide the latency of
+  // the sigma chain -- and, for the delta rule, of r_t's shuffle sum and
+  // 1/r_t; the parts go straight to the operand buffer, so the thread state
+  // fits in 76 registers).
+  static constexpr int kMath = 16;
   static constexpr int kThreads = 64 + 32 * kMath;
   static constexpr int kTL = 2 * kMath;                   // token lanes
   static constexpr int kTokPerThread = kLTok / kTL;
@@ -603,7 +604,11 @@ tc_pipe_products(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
       ok = __all_sync(0xffffffffu, mbar_wait(full + st, (uint32_t)(b / kStages) & 1u, abort, status));
       if (!ok) break;
       const unsigned char* kb = ring + st * SM::kStage;
-      uint4 hi4[kTPT], lo4[kTPT], yh4[kTPT], yl4[kTPT];
+      // The operand buffer is free once the MMAs of block b - 2 are done
+      // (long before, normally); the parts go straight into it.
+      ok = __all_sync(0xffffffffu, mbar_wait(op_empty + ob, ((uint32_t)(b >> 1) & 1u) ^ 1u, abort, status));
+      if (!ok) break;
+      unsigned char* hb = op + ob * SM::kOpParts * SM::kHalf;
 #pragma unroll
       for (int i = 0; i < kTPT; ++i) {
         const int t = tl + kTL * i;
@@ -620,8 +625,8 @@ tc_pipe_products(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
           hw[e] = pack_bf16x2(sg[2 * e], sg[2 * e + 1]);
           lw[e] = pack_bf16x2(sg[2 * e] - bf16lo_to_f32(hw[e]), sg[2 * e + 1] - bf16hi_to_f32(hw[e]));
         }
-        hi4[i] = make_uint4(hw[0], hw[1], hw[2], hw[3]);
-        lo4[i] = make_uint4(lw[0], lw[1], lw[2], lw[3]);
+        *reinterpret_cast<uint4*>(hb + off) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+        *reinterpret_cast<uint4*>(hb + SM::kHalf + off) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
         if (DELTA) {
           // r_t = sigma(k_t) . z_{s-1} over the token's 16 threads; Y = sigma / r.
           float r = 0.f;
@@ -637,8 +642,8 @@ tc_pipe_products(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
             yh[e] = pack_bf16x2(a, c);
             yl[e] = pack_bf16x2(a - bf16lo_to_f32(yh[e]), c - bf16hi_to_f32(yh[e]));
           }
-          yh4[i] = make_uint4(yh[0], yh[1], yh[2], yh[3]);
-          yl4[i] = make_uint4(yl[0], yl[1], yl[2], yl[3]);
+          *reinterpret_cast<uint4*>(hb + 2 * SM::kHalf + off) = make_uint4(yh[0], yh[1], yh[2], yh[3]);
+          *reinterpret_cast<uint4*>(hb + 3 * SM::kHalf + off) = make_uint4(yl[0], yl[1], yl[2], yl[3]);
         } else {
 #pragma unroll
           for (int e = 0; e < 8; ++e) acc[e] += sg[e];
@@ -647,20 +652,6 @@ tc_pipe_products(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
       // K of this block has been read.
       __syncwarp();
       if (lane == 0) mbar_arrive(empty + st);
-      // The operand buffer is free once the MMAs of block b - 2 are done.
-      ok = __all_sync(0xffffffffu, mbar_wait(op_empty + ob, ((uint32_t)(b >> 1) & 1u) ^ 1u, abort, status));
-      if (!ok) break;
-      unsigned char* hb = op + ob * SM::kOpParts * SM::kHalf;
-#pragma unroll
-      for (int i = 0; i < kTPT; ++i) {
-        const uint32_t off = sw128_offset(tl + kTL * i, 8 * cg, kLTok);
-        *reinterpret_cast<uint4*>(hb + off) = hi4[i];
-        *reinterpret_cast<uint4*>(hb + SM::kHalf + off) = lo4[i];
-        if (DELTA) {
-          *reinterpret_cast<uint4*>(hb + 2 * SM::kHalf + off) = yh4[i];
-          *reinterpret_cast<uint4*>(hb + 3 * SM::kHalf + off) = yl4[i];
-        }
-      }
       fence_proxy_async();
       __syncwarp();
       if (lane == 0) mbar_arrive(op_full + ob);
@@ -688,17 +679,21 @@ tc_pipe_products(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
       const int k = 32 * (warp & 3) + lane, half = (warp - 2) >> 2;
       const uint32_t lq = (uint32_t)(32 * (warp & 3)) << 16;
       if (DELTA) {
-        float* rowp = (half ? Bbuf : Gbuf) + (slice * D + k) * D;
-        const uint32_t ta = (half ? tB : tG) + lq;
+        // The delta rule's 16 math warps: four per lane quarter, each a
+        // quarter of the columns of G or of B.
+        constexpr int kCols = 8 * D / kLMath;  // columns per warp
+        const int quarter = (warp - 2) >> 2;     // 0..3
+        const int which = quarter >> 1, part = quarter & 1;
+        float* rowp = (which ? Bbuf : Gbuf) + (slice * D + k) * D + kCols * part;
+        const uint32_t ta = (which ? tB : tG) + lq + kCols * part;
 #pragma unroll
-        for (int c = 0; c < D / 64; ++c) {
-          uint32_t v[64];
-          tmem_ld32(ta + 64 * c, v);
-          tmem_ld32(ta + 64 * c + 32, v + 32);
+        for (int c = 0; c < kCols / 32; ++c) {
+          uint32_t v[32];
+          tmem_ld32(ta + 32 * c, v);
           tmem_wait_ld();
-          float4* dst = reinterpret_cast<float4*>(rowp + 64 * c);
+          float4* dst = reinterpret_cast<float4*>(rowp + 32 * c);
 #pragma unroll
-          for (int i = 0; i < 16; ++i)
+          for (int i = 0; i < 8; ++i)
             dst[i] = make_float4(__uint_as_float(v[4 * i]), __uint_as_float(v[4 * i + 1]),
                                  __uint_as_float(v[4 * i + 2]), __uint_as_float(v[4 * i + 3]));
         }
