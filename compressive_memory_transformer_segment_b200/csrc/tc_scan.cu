@@ -106,10 +106,12 @@ int zsum_chunks(int S) { return S >= 256 * kZChunksMax ? kZChunksMax : (S >= 512
 
 // Tokens per block: 128, or 64 for segments of at most 64 tokens (half the
 // shared memory, so more CTAs fit on an SM when a segment is one block).
-constexpr int kThreads = 192;
-
 template <int D, bool DELTA, int TOK>
 struct ProdSmem {
+  // Roles: warp 0 TMA, warp 1 MMA, then TOK / 16 math warps: two threads per
+  // token, each with half of the columns.
+  static constexpr int kMathWarps = TOK / 16;
+  static constexpr int kThreads = 64 + 32 * kMathWarps;
   static constexpr int kK = 0;                                      // K block [TOK][D]
   static constexpr int kV = kK + TOK * D * 2;                       // V block [TOK][D] (+ ones)
   static constexpr int kVBytes = TOK * D * 2 + (DELTA ? 0 : TOK * 64 * 2);
@@ -129,18 +131,19 @@ struct ProdSmem {
 };
 
 // Grid (T, B*H_kv).  Roles: warp 0 TMA producer (K, V blocks), warp 1 TMEM
-// allocation + MMA issue, warps 2..5 one thread per token of the block (the
-// threads of rows 64..127 idle with 64-token blocks) and, at the end, one per
-// row of the products.
+// allocation + MMA issue, warps 2.. two threads per token of the block (each
+// half of the columns) and, at the end, one per row of the products (the
+// warps of a TMEM lane quarter splitting the column chunks).
 // TMEM: delta G [0, D), B [128, 128 + D); linear [B | dz] [0, D + 16).
 template <int D, bool DELTA, int TOK>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(ProdSmem<D, DELTA, TOK>::kThreads, 1)
 tc_segment_products(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                     const float* __restrict__ z_pref, float* __restrict__ Gbuf,
                     float* __restrict__ Bbuf, float* __restrict__ dz,
                     unsigned int* __restrict__ status, int L, int S) {
   using SM = ProdSmem<D, DELTA, TOK>;
   constexpr int kTok = TOK;
+  constexpr int kThreads = SM::kThreads, kMathWarps = SM::kMathWarps;
   constexpr uint32_t kTmemCols = SM::kTmemCols;
   const int s = blockIdx.x, bh = blockIdx.y, BH = gridDim.y;
   const int seg0 = s * S, seg_len = min(S, L - seg0);
@@ -178,10 +181,10 @@ tc_segment_products(const __grid_constant__ CUtensorMap tm_k, const __grid_const
 
   if (threadIdx.x == 0) {
     mbar_init(k_full, 1);
-    mbar_init(k_empty, 4);   // one arrival per math warp
+    mbar_init(k_empty, kMathWarps);   // one arrival per math warp
     mbar_init(v_full, 1);
     mbar_init(v_empty, 1);
-    mbar_init(op_ready, 4);
+    mbar_init(op_ready, kMathWarps);
     mbar_init(op_free, 1);
     mbar_init(done, 1);
     *abort = 0;
@@ -291,7 +294,12 @@ tc_segment_products(const __grid_constant__ CUtensorMap tm_k, const __grid_const
     }
   } else {
     // -------------------------------------------------- math threads
-    const int t = 32 * (warp & 3) + lane;  // token of the block; later, row of the products
+    // Sigma phase: thread -> (token t, column half hp), the two threads of a
+    // token in adjacent lanes.  Products phase: thread -> TMEM lane (row of
+    // the products) and a share of the column chunks.
+    const int mt = threadIdx.x - 64;
+    const int t = mt >> 1, hp = mt & 1;
+    const int c8_0 = hp * (D / 16);
     const uint32_t lane_off = (uint32_t)(32 * (warp & 3)) << 16;
     bool ok = true;
     for (int blk = 0; blk < nblk; ++blk) {
@@ -301,14 +309,14 @@ tc_segment_products(const __grid_constant__ CUtensorMap tm_k, const __grid_const
       }
       ok = __all_sync(0xffffffffu, mbar_wait(k_full, blk & 1, abort, status));
       if (!ok) break;
-      // (with 64-token blocks the threads of rows 64..127 have no token)
-      const bool has_tok = t < kTok;
+      const bool has_tok = t < kTok;  // (always, with two threads per token)
       const bool valid = has_tok && blk * kTok + t < seg_len;
       // sigma(K) row t as hi/lo pairs (rows past the segment are 0), and
-      // r_t = sigma(k_t) . z_{s-1} (delta).
+      // r_t = sigma(k_t) . z_{s-1} (delta): each thread half the columns,
+      // the halves added across the lane pair.
       float r = 0.f;
 #pragma unroll 4
-      for (int c8 = 0; c8 < D / 8; ++c8) {
+      for (int c8 = c8_0; c8 < c8_0 + D / 16; ++c8) {
         const uint32_t off = sw128_offset(t, 8 * c8, kTok);
         const uint4 kv = has_tok ? *reinterpret_cast<const uint4*>(sK + off) : make_uint4(0, 0, 0, 0);
         const uint32_t kw[4] = {kv.x, kv.y, kv.z, kv.w};
@@ -336,13 +344,15 @@ tc_segment_products(const __grid_constant__ CUtensorMap tm_k, const __grid_const
           *reinterpret_cast<uint4*>(sSkLo + off) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
         }
       }
+      // (a + b == b + a: both threads of the token get the same r)
+      if (DELTA) r += __shfl_xor_sync(0xffffffffu, r, 1);
       __syncwarp();
       if (lane == 0) mbar_arrive(k_empty);
       if (DELTA && has_tok) {
         // Y = sigma(K) / r (0 where r = 0), from the pair just written.
         const float w = r != 0.f ? 1.f / r : 0.f;
 #pragma unroll 4
-        for (int c8 = 0; c8 < D / 8; ++c8) {
+        for (int c8 = c8_0; c8 < c8_0 + D / 16; ++c8) {
           const uint32_t off = sw128_offset(t, 8 * c8, kTok);
           const uint4 hv = *reinterpret_cast<const uint4*>(sSkHi + off);
           const uint4 lv = *reinterpret_cast<const uint4*>(sSkLo + off);
@@ -363,20 +373,24 @@ tc_segment_products(const __grid_constant__ CUtensorMap tm_k, const __grid_const
       __syncwarp();
       if (lane == 0) mbar_arrive(op_ready);
     }
-    // The segment's products, row t (t < D), to the workspace in fp32.
+    // The segment's products, row k (k < D), to the workspace in fp32: the
+    // warps of a TMEM lane quarter take turns with the 32-column chunks.
+    const int k = 32 * (warp & 3) + lane;
+    constexpr int kParts = kMathWarps / 4;
+    const int part = (warp - 2) >> 2;
     if (ok) ok = __all_sync(0xffffffffu, mbar_wait(done, 0, abort, status));
     if (ok) {
       tc_fence_after();
       if (DELTA) {
 #pragma unroll
-        for (int c = 0; c < D / 32; ++c) {
+        for (int c = part; c < D / 32; c += kParts) {
           uint32_t g[32], bb[32];
           tmem_ld32(tmem + lane_off + c * 32, g);
           tmem_ld32(tmem + 128 + lane_off + c * 32, bb);
           tmem_wait_ld();
-          if (t < D) {
-            float4* gd = reinterpret_cast<float4*>(Gbuf + (slice * D + t) * D + c * 32);
-            float4* bd = reinterpret_cast<float4*>(Bbuf + (slice * D + t) * D + c * 32);
+          if (k < D) {
+            float4* gd = reinterpret_cast<float4*>(Gbuf + (slice * D + k) * D + c * 32);
+            float4* bd = reinterpret_cast<float4*>(Bbuf + (slice * D + k) * D + c * 32);
 #pragma unroll
             for (int i = 0; i < 8; ++i) {
               gd[i] = make_float4(__uint_as_float(g[4 * i]), __uint_as_float(g[4 * i + 1]),
@@ -388,19 +402,19 @@ tc_segment_products(const __grid_constant__ CUtensorMap tm_k, const __grid_const
         }
       } else {
 #pragma unroll
-        for (int c = 0; c < D / 32 + 1; ++c) {
+        for (int c = part; c < D / 32 + 1; c += kParts) {
           uint32_t bb[32];
           tmem_ld32(tmem + lane_off + c * 32, bb);
           tmem_wait_ld();
-          if (t < D) {
+          if (k < D) {
             if (c < D / 32) {
-              float4* bd = reinterpret_cast<float4*>(Bbuf + (slice * D + t) * D + c * 32);
+              float4* bd = reinterpret_cast<float4*>(Bbuf + (slice * D + k) * D + c * 32);
 #pragma unroll
               for (int i = 0; i < 8; ++i)
                 bd[i] = make_float4(__uint_as_float(bb[4 * i]), __uint_as_float(bb[4 * i + 1]),
                                     __uint_as_float(bb[4 * i + 2]), __uint_as_float(bb[4 * i + 3]));
             } else {
-              dz[slice * D + t] = __uint_as_float(bb[0]);
+              dz[slice * D + k] = __uint_as_float(bb[0]);
             }
           }
         }
@@ -913,7 +927,7 @@ cudaError_t launch_products(const Problem& p, const CUtensorMap& tk, const CUten
   auto kern = tc_segment_products<D, DELTA, TOK>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
-  kern<<<dim3(p.T, p.B * p.H_kv), kThreads, smem, stream>>>(tk, tv, p.z_pref, p.Gbuf, p.Bbuf, p.dz,
+  kern<<<dim3(p.T, p.B * p.H_kv), ProdSmem<D, DELTA, TOK>::kThreads, smem, stream>>>(tk, tv, p.z_pref, p.Gbuf, p.Bbuf, p.dz,
                                                            p.status, p.L, p.S);
   return cudaGetLastError();
 }
