@@ -80,19 +80,35 @@ __global__ void __launch_bounds__(256) zsum(const __nv_bfloat16* __restrict__ k,
   }
 }
 
-// z_{s-1} for s = 1..T-1 into z_pref (slot 0 already holds z_in) and z_T,
-// from the C chunk partials of every segment.  Grid (B*H_kv), block D threads.
+// z_{s-1} for s = 0..T-1 into z_pref (slot 0 = z_in) and z_T, from the C
+// chunk partials of every segment.  Grid (B*H_kv), block D threads.  The
+// partials are loaded kAhead at a time before they are added, so that the
+// walk waits for one round of loads per kAhead partials, not for every one.
 template <int D>
 __global__ void __launch_bounds__(128) zprefix(const float* __restrict__ dz, const float* z_in,
                                                float* __restrict__ z_pref, float* z_out, int T, int C) {
   const int bh = blockIdx.x, c = threadIdx.x, BH = gridDim.x;
+  constexpr int kAhead = 16;
+  const int n = T * C;
   // (z_out may be z_in: this thread reads its entry before it writes it)
-  float z = z_in[(size_t)bh * D + c];
-  for (int s = 0; s < T; ++s) {
-    z_pref[((size_t)s * BH + bh) * D + c] = z;
-    float seg = 0.f;
-    for (int j = 0; j < C; ++j) seg += dz[((size_t)(s * C + j) * BH + bh) * D + c];
-    z += seg;
+  float z = z_in[(size_t)bh * D + c], seg = 0.f;
+  for (int i0 = 0; i0 < n; i0 += kAhead) {
+    float part[kAhead];
+#pragma unroll
+    for (int u = 0; u < kAhead; ++u)
+      part[u] = i0 + u < n ? dz[((size_t)(i0 + u) * BH + bh) * D + c] : 0.f;
+#pragma unroll
+    for (int u = 0; u < kAhead; ++u) {
+      const int i = i0 + u;
+      if (i >= n) break;
+      const int j = i % C;
+      if (j == 0) z_pref[((size_t)(i / C) * BH + bh) * D + c] = z;
+      seg += part[u];
+      if (j == C - 1) {
+        z += seg;
+        seg = 0.f;
+      }
+    }
   }
   z_out[(size_t)bh * D + c] = z;
 }
@@ -751,36 +767,51 @@ __device__ __forceinline__ void cp_async_wait() {
 }
 
 // Delta rule: M_s = M_{s-1} - G_s M_{s-1} + B_s on columns [16 cb, 16 cb + 16).
-// Grid (B*H_kv, D/16), block 256 threads: thread -> (row k = tid % 128,
-// 8 columns); rows >= D idle for D = 64.  With 16 columns per CTA the grid
-// of the 8B shape (16 KV heads x 8) is one wave.  G_s is symmetric up to the
-// rounding of its bf16 pair products (the dropped lo*lo term, ~2^-16
-// relative), so row k of G_s M is read from column k of G_s, which makes
-// the shared-memory reads conflict-free; G_{s+1} streams in (cp.async)
-// while G_s is used.  Plain block barriers only.
+// Grid (B*H_kv, D/16), block D threads (D/32 warps).  Thread tile: 4 rows x
+// 4 columns of M, lane -> (row group lane / 4 of the warp's 32 rows, column
+// group lane % 4), so that one 128-bit shared load of G and one of M_{s-1}
+// per kk feed 16 FMAs (8 fma.rn.f32x2), and a warp's loads per kk are two
+// shared-memory wavefronts: the loop is bound by the FMA pipe, not by
+// shared-memory bandwidth.  G_s is symmetric up to the rounding of its bf16
+// pair products (the dropped lo*lo term, ~2^-16 relative), so row k of
+// G_s M is read from column k of G_s: four consecutive rows of the tile are
+// one contiguous 16-byte piece.  G_{s+1} streams in (cp.async) and the B_{s+1}
+// tile is loaded into registers while step s runs.  Plain block barriers only.
 template <int D>
-__global__ void __launch_bounds__(256) combine_delta(const float* __restrict__ M_in,
-                                                     const float* __restrict__ Gbuf,
-                                                     const float* __restrict__ Bbuf,
-                                                     __nv_bfloat16* __restrict__ M_pref,
-                                                     float* __restrict__ M_out, int T) {
+__global__ void __launch_bounds__(D) combine_delta(const float* __restrict__ M_in,
+                                                   const float* __restrict__ Gbuf,
+                                                   const float* __restrict__ Bbuf,
+                                                   __nv_bfloat16* __restrict__ M_pref,
+                                                   float* __restrict__ M_out, int T) {
+  static_assert(kCB == 16 && D % 32 == 0, "combine_delta thread map");
   extern __shared__ __align__(16) float csm[];
   float* sG = csm;               // two G_s buffers [D][D]
   float* sM = csm + 2 * D * D;   // M_{s-1}[:, 16 columns]
   const int bh = blockIdx.x, c0 = blockIdx.y * kCB, BH = gridDim.x;
-  const int tid = threadIdx.x, k = tid & 127, cg = (tid >> 7) * 8;
-  const bool active = k < D;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int k0 = 32 * warp + 4 * (lane >> 2);  // first of the tile's 4 rows
+  const int c = 4 * (lane & 3);                // first of its 4 columns (in the CTA's 16)
   auto load_g = [&](int s, float* dst) {
     const float4* src = reinterpret_cast<const float4*>(Gbuf + ((size_t)s * BH + bh) * D * D);
-    for (int e = tid; e < D * D / 4; e += 256) cp_async16(dst + 4 * e, src + e);
+    for (int e = tid; e < D * D / 4; e += D) cp_async16(dst + 4 * e, src + e);
     cp_async_commit();
   };
-  float m[8];
+  auto load_b = [&](int s, float4* dst) {
+    const float* src = Bbuf + (((size_t)s * BH + bh) * D + k0) * D + c0 + c;
 #pragma unroll
-  for (int i = 0; i < 8; ++i) m[i] = active ? M_in[((size_t)bh * D + k) * D + c0 + cg + i] : 0.f;
+    for (int i = 0; i < 4; ++i) dst[i] = *reinterpret_cast<const float4*>(src + (size_t)i * D);
+  };
+  float4 m[4];  // M[k0 + i][c0 + c .. + 3]
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+    m[i] = *reinterpret_cast<const float4*>(M_in + ((size_t)bh * D + k0 + i) * D + c0 + c);
+  float4 bq[4];
   load_g(0, sG);
+  load_b(0, bq);
   for (int s = 0; s < T; ++s) {
     const size_t slice = (size_t)s * BH + bh;
+    float4 bn[4];
+    if (s + 1 < T) load_b(s + 1, bn);
     float* G = sG + (s & 1) * D * D;
     if (s + 1 < T) {
       load_g(s + 1, sG + ((s + 1) & 1) * D * D);
@@ -789,49 +820,45 @@ __global__ void __launch_bounds__(256) combine_delta(const float* __restrict__ M
       cp_async_wait<0>();
     }
     // Publish M_{s-1} (bf16) for segment s's retrieval.
-    if (active) {
-      uint4 w;
-      w.x = pack_bf16x2(m[0], m[1]);
-      w.y = pack_bf16x2(m[2], m[3]);
-      w.z = pack_bf16x2(m[4], m[5]);
-      w.w = pack_bf16x2(m[6], m[7]);
-      *reinterpret_cast<uint4*>(M_pref + (slice * D + k) * D + c0 + cg) = w;
-      *reinterpret_cast<float4*>(sM + k * kCB + cg) = make_float4(m[0], m[1], m[2], m[3]);
-      *reinterpret_cast<float4*>(sM + k * kCB + cg + 4) = make_float4(m[4], m[5], m[6], m[7]);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      uint2 w;
+      w.x = pack_bf16x2(m[i].x, m[i].y);
+      w.y = pack_bf16x2(m[i].z, m[i].w);
+      *reinterpret_cast<uint2*>(M_pref + (slice * D + k0 + i) * D + c0 + c) = w;
+      *reinterpret_cast<float4*>(sM + (k0 + i) * kCB + c) = m[i];
     }
     __syncthreads();
-    if (active) {
-      float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-#pragma unroll 8
-      for (int kk = 0; kk < D; ++kk) {
-        const float gv = G[kk * D + k];
-        const float4 ma = *reinterpret_cast<const float4*>(sM + kk * kCB + cg);
-        const float4 mb = *reinterpret_cast<const float4*>(sM + kk * kCB + cg + 4);
-        acc[0] = fmaf(gv, ma.x, acc[0]);
-        acc[1] = fmaf(gv, ma.y, acc[1]);
-        acc[2] = fmaf(gv, ma.z, acc[2]);
-        acc[3] = fmaf(gv, ma.w, acc[3]);
-        acc[4] = fmaf(gv, mb.x, acc[4]);
-        acc[5] = fmaf(gv, mb.y, acc[5]);
-        acc[6] = fmaf(gv, mb.z, acc[6]);
-        acc[7] = fmaf(gv, mb.w, acc[7]);
+    // (G_s M)[k0 + i][c .. c + 3] as column pairs.
+    float2 acc[4][2];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) acc[i][0] = acc[i][1] = make_float2(0.f, 0.f);
+#pragma unroll 4
+    for (int kk = 0; kk < D; ++kk) {
+      const float4 g = *reinterpret_cast<const float4*>(G + kk * D + k0);
+      const float4 mv = *reinterpret_cast<const float4*>(sM + kk * kCB + c);
+      const float2 mlo = make_float2(mv.x, mv.y), mhi = make_float2(mv.z, mv.w);
+      const float gr[4] = {g.x, g.y, g.z, g.w};
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const float2 g2 = make_float2(gr[i], gr[i]);
+        acc[i][0] = fma2(g2, mlo, acc[i][0]);
+        acc[i][1] = fma2(g2, mhi, acc[i][1]);
       }
-      const float4* bk = reinterpret_cast<const float4*>(Bbuf + (slice * D + k) * D + c0 + cg);
-      const float4 ba = bk[0], bb = bk[1];
-      m[0] = (m[0] - acc[0]) + ba.x;
-      m[1] = (m[1] - acc[1]) + ba.y;
-      m[2] = (m[2] - acc[2]) + ba.z;
-      m[3] = (m[3] - acc[3]) + ba.w;
-      m[4] = (m[4] - acc[4]) + bb.x;
-      m[5] = (m[5] - acc[5]) + bb.y;
-      m[6] = (m[6] - acc[6]) + bb.z;
-      m[7] = (m[7] - acc[7]) + bb.w;
+    }
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      m[i].x = (m[i].x - acc[i][0].x) + bq[i].x;
+      m[i].y = (m[i].y - acc[i][0].y) + bq[i].y;
+      m[i].z = (m[i].z - acc[i][1].x) + bq[i].z;
+      m[i].w = (m[i].w - acc[i][1].y) + bq[i].w;
+      bq[i] = bn[i];
     }
     __syncthreads();
   }
-  if (active)
 #pragma unroll
-    for (int i = 0; i < 8; ++i) M_out[((size_t)bh * D + k) * D + c0 + cg + i] = m[i];
+  for (int i = 0; i < 4; ++i)
+    *reinterpret_cast<float4*>(M_out + ((size_t)bh * D + k0 + i) * D + c0 + c) = m[i];
 }
 
 // Linear rule: M_s = M_{s-1} + B_s, z_s = z_{s-1} + dz_s, element-parallel.
@@ -974,7 +1001,7 @@ cudaError_t launch(const Problem& p, cudaStream_t stream) {
     const int csmem = (2 * D * D + D * kCB) * (int)sizeof(float);
     e = cudaFuncSetAttribute(combine_delta<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, csmem);
     if (e != cudaSuccess) return e;
-    combine_delta<D><<<dim3(BH, D / kCB), 256, csmem, stream>>>(p.M_in, p.Gbuf, p.Bbuf, Mp, p.M_out,
+    combine_delta<D><<<dim3(BH, D / kCB), D, csmem, stream>>>(p.M_in, p.Gbuf, p.Bbuf, Mp, p.M_out,
                                                                  p.T);
     return cudaGetLastError();
   }
