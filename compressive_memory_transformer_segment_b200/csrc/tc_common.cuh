@@ -392,19 +392,6 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   return *reinterpret_cast<uint32_t*>(&v);
 }
 
-// Two fp32 fused multiply-adds in one instruction (fma.rn.f32x2, sm_100):
-// each half is rounded exactly like fmaf, a.x * b.x + c.x and a.y * b.y + c.y.
-__device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c) {
-  uint64_t d, ua, ub, uc;
-  asm("mov.b64 %0, {%1, %2};" : "=l"(ua) : "f"(a.x), "f"(a.y));
-  asm("mov.b64 %0, {%1, %2};" : "=l"(ub) : "f"(b.x), "f"(b.y));
-  asm("mov.b64 %0, {%1, %2};" : "=l"(uc) : "f"(c.x), "f"(c.y));
-  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(ua), "l"(ub), "l"(uc));
-  float2 r;
-  asm("mov.b64 {%0, %1}, %2;" : "=f"(r.x), "=f"(r.y) : "l"(d));
-  return r;
-}
-
 // Byte offset of element (row, col) of a bf16 tile stored as described at the
 // top of this file (panels of `rows` x 128 B).
 __device__ __forceinline__ uint32_t sw128_offset(int row, int col, int rows) {

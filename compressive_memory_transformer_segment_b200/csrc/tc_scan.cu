@@ -29,6 +29,7 @@
 #include <cuda.h>
 
 #include "kernels.h"
+#include "packed_math.cuh"
 #include "tc_common.cuh"
 
 namespace infini {
@@ -453,7 +454,8 @@ tc_segment_products(const __grid_constant__ CUtensorMap tm_k, const __grid_const
 //           D = diag(sigma(K_s) z_{s-1}) (rows with r_t = 0 give zero rows).
 // A TMA ring of (K, V) blocks; sigma(K) (and Y) as bf16 hi/lo pairs in two
 // alternating operand buffers, so the math warps build block b+1 while the
-// tensor core multiplies block b; dz (linear) summed by the math threads.
+// tensor core multiplies block b; dz (linear) by the tensor core too, from
+// a constant operand whose first column is ones.
 // The linear rule is HBM-bound (each block brings 32 KiB of K and V); the
 // delta rule does 20 MMAs (128 x 128 x 16) per block.
 constexpr int kLTok = 64;      // tokens per block
@@ -476,15 +478,19 @@ struct PipeSmem {
   static constexpr int kOpParts = DELTA ? 4 : 2;          // sigma hi, lo (, Y hi, lo)
   static constexpr int kRing = 0;
   static constexpr int kOp = kRing + kStages * kStage;    // [2][parts]
-  static constexpr int kRed = kOp + 2 * kOpParts * kHalf; // dz partials fp32 [kTL][128]
-  static constexpr int kZ = kRed + (DELTA ? 0 : kTL * kD * 4);  // z_{s-1} fp32 [128] (delta)
+  // Linear rule: a constant [64 tokens][64] panel whose column 0 is 1.0, the
+  // B operand of the MMA that sums sigma(K) over the tokens (dz).
+  static constexpr int kOnes = kOp + 2 * kOpParts * kHalf;
+  static constexpr int kZ = kOnes + (DELTA ? 0 : kPanel);  // z_{s-1} fp32 [128] (delta)
   static constexpr int kBar = kZ + (DELTA ? kD * 4 : 0);
-  // full[kStages] empty[kStages] op_full[2] op_empty[2] acc_full red_ready
-  static constexpr int kNumBars = 2 * kStages + 6;
+  // full[kStages] empty[kStages] op_full[2] op_empty[2] acc_full
+  static constexpr int kNumBars = 2 * kStages + 5;
   static constexpr int kTmemSlot = kBar + kNumBars * 8;
   static constexpr int kAbort = kTmemSlot + 4;
   static constexpr int kAlloc = kAbort + 4 + 1024;
-  static constexpr uint32_t kTmemCols = DELTA ? 256 : 128;  // [G |] B
+  // TMEM: delta [G | B]; linear [B | dz (16 columns, column 0 used)].
+  static constexpr uint32_t kTmemCols = 256;
+  static_assert(kOnes % 1024 == 0, "ones panel alignment");
 };
 
 template <bool DELTA>
@@ -509,7 +515,7 @@ tc_pipe_products(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   unsigned char* ring = smem + SM::kRing;
   unsigned char* op = smem + SM::kOp;
-  float* red = reinterpret_cast<float*>(smem + SM::kRed);
+  unsigned char* ones = smem + SM::kOnes;
   float* zs = reinterpret_cast<float*>(smem + SM::kZ);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + SM::kBar);
   uint64_t* full = bars;
@@ -517,7 +523,6 @@ tc_pipe_products(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
   uint64_t* op_full = bars + 2 * kStages;
   uint64_t* op_empty = op_full + 2;
   uint64_t* acc_full = op_empty + 2;
-  uint64_t* red_ready = acc_full + 1;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + SM::kTmemSlot);
   volatile int* abort = reinterpret_cast<volatile int*>(smem + SM::kAbort);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -538,12 +543,22 @@ tc_pipe_products(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
       mbar_init(op_empty + i, 1);
     }
     mbar_init(acc_full, 1);
-    mbar_init(red_ready, kLMath);
     *abort = 0;
     fence_mbar_init();
   }
   if (DELTA)
     for (int i = threadIdx.x; i < D; i += kLThreads) zs[i] = z_pref[slice * D + i];
+  if (!DELTA) {
+    // Row t of the ones panel: its 16-byte chunk that holds logical column 0
+    // sits at chunk (t & 7) under the 128-byte swizzle.
+    for (int i = threadIdx.x; i < kLTok * 8; i += kLThreads) {
+      const int row = i / 8, chunk = i % 8;
+      uint4 v = make_uint4(0, 0, 0, 0);
+      if (chunk == (row & 7)) v.x = 0x3F80u;  // element (row, 0) = bf16(1.0)
+      *reinterpret_cast<uint4*>(ones + i * 16) = v;
+    }
+    fence_proxy_async();
+  }
   if (warp == 1) {
     tmem_alloc(tmem_slot, SM::kTmemCols);
     tmem_relinquish();
@@ -552,7 +567,7 @@ tc_pipe_products(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  const uint32_t tG = tmem, tB = DELTA ? tmem + 128 : tmem;
+  const uint32_t tG = tmem, tB = DELTA ? tmem + 128 : tmem, tDZ = tmem + 128;
 
   if (warp == 0) {
     // ---------------------------------------------- TMA producer (whole warp waits, one elected lane issues)
@@ -578,8 +593,10 @@ tc_pipe_products(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
   } else if (warp == 1) {
     // ---------------------------------------------- MMA issuer (whole warp waits, one elected lane issues)
     constexpr uint32_t idesc = idesc_bf16_f32(128, D, true, true);
+    constexpr uint32_t idesc_dz = idesc_bf16_f32(128, 16, true, true);
     const uint64_t dop = sw128_desc(smem_u32(op), SM::kPanel, 1024);
     const uint64_t dring = sw128_desc(smem_u32(ring + SM::kHalf), SM::kPanel, 1024);
+    const uint64_t dones = sw128_desc(smem_u32(ones), SM::kPanel, 1024);
     bool ok = true;
     for (int b = 0; ok && b < nblk; ++b) {
       const int st = b % kStages, ob = b & 1;
@@ -604,6 +621,10 @@ tc_pipe_products(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
           }
           mma_ss(tB, shi + stp, vv + stp, idesc, acc);
           mma_ss(tB, slo + stp, vv + stp, idesc, 1u);
+          if (!DELTA) {
+            mma_ss(tDZ, shi + stp, dones + stp, idesc_dz, acc);
+            mma_ss(tDZ, slo + stp, dones + stp, idesc_dz, 1u);
+          }
         }
         tc_commit(op_empty + ob);
         tc_commit(empty + st);
@@ -620,9 +641,6 @@ tc_pipe_products(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
     // one warp.
     const int mt = threadIdx.x - 64;
     const int cg = mt & 15, tl = mt >> 4;
-    float acc[8];
-#pragma unroll
-    for (int i = 0; i < 8; ++i) acc[i] = 0.f;
     float zc[8];
     if (DELTA) {
 #pragma unroll
@@ -644,16 +662,16 @@ tc_pipe_products(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
         const int t = tl + kTL * i;
         const bool valid = b * kLTok + t < seg_len;
         const uint32_t off = sw128_offset(t, 8 * cg, kLTok);
-        const uint4 kv = *reinterpret_cast<const uint4*>(kb + off);
+        uint4 kv = *reinterpret_cast<const uint4*>(kb + off);
+        // (rows past the segment: sigma = 0 exactly)
+        if (!valid) kv = make_uint4(0xFF7FFF7Fu, 0xFF7FFF7Fu, 0xFF7FFF7Fu, 0xFF7FFF7Fu);
         const uint32_t kw[4] = {kv.x, kv.y, kv.z, kv.w};
-        float sg[8];
+        float2 sg[4];
         uint32_t hw[4], lw[4];
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
-          sg[2 * e] = valid ? elu1_fast(bf16lo_to_f32(kw[e])) : 0.f;
-          sg[2 * e + 1] = valid ? elu1_fast(bf16hi_to_f32(kw[e])) : 0.f;
-          hw[e] = pack_bf16x2(sg[2 * e], sg[2 * e + 1]);
-          lw[e] = pack_bf16x2(sg[2 * e] - bf16lo_to_f32(hw[e]), sg[2 * e + 1] - bf16hi_to_f32(hw[e]));
+          sg[e] = pk::sigma_pair(kw[e]);
+          pk::split_pair(sg[e], hw[e], lw[e]);
         }
         *reinterpret_cast<uint4*>(hb + off) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
         *reinterpret_cast<uint4*>(hb + SM::kHalf + off) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
@@ -661,22 +679,18 @@ tc_pipe_products(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
           // r_t = sigma(k_t) . z_{s-1} over the token's 16 threads; Y = sigma / r.
           float r = 0.f;
 #pragma unroll
-          for (int e = 0; e < 8; ++e) r = fmaf(sg[e], zc[e], r);
+          for (int e = 0; e < 4; ++e) {
+            r = fmaf(sg[e].x, zc[2 * e], r);
+            r = fmaf(sg[e].y, zc[2 * e + 1], r);
+          }
 #pragma unroll
           for (int o = 8; o > 0; o >>= 1) r += __shfl_xor_sync(0xffffffffu, r, o);
           const float w = r != 0.f ? 1.f / r : 0.f;
           uint32_t yh[4], yl[4];
 #pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const float a = w * sg[2 * e], c = w * sg[2 * e + 1];
-            yh[e] = pack_bf16x2(a, c);
-            yl[e] = pack_bf16x2(a - bf16lo_to_f32(yh[e]), c - bf16hi_to_f32(yh[e]));
-          }
+          for (int e = 0; e < 4; ++e) pk::split_pair(pk::mul2(make_float2(w, w), sg[e]), yh[e], yl[e]);
           *reinterpret_cast<uint4*>(hb + 2 * SM::kHalf + off) = make_uint4(yh[0], yh[1], yh[2], yh[3]);
           *reinterpret_cast<uint4*>(hb + 3 * SM::kHalf + off) = make_uint4(yl[0], yl[1], yl[2], yl[3]);
-        } else {
-#pragma unroll
-          for (int e = 0; e < 8; ++e) acc[e] += sg[e];
         }
       }
       // K of this block has been read.
@@ -685,20 +699,6 @@ tc_pipe_products(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
       fence_proxy_async();
       __syncwarp();
       if (lane == 0) mbar_arrive(op_full + ob);
-    }
-    if (!DELTA) {
-      // dz: the token lanes' partial column sums, reduced in shared memory.
-#pragma unroll
-      for (int i = 0; i < 8; ++i) red[tl * D + 8 * cg + i] = acc[i];
-      __syncwarp();
-      if (lane == 0) mbar_arrive(red_ready);
-      if (ok) ok = __all_sync(0xffffffffu, mbar_wait(red_ready, 0, abort, status));
-      if (ok && mt < D) {
-        float sum = 0.f;
-#pragma unroll
-        for (int j = 0; j < kTL; ++j) sum += red[j * D + mt];
-        dz[slice * D + mt] = sum;
-      }
     }
     // The products: TMEM lane k = row k.  Linear: the kMath / 4 warps of a
     // lane quarter share the 128 columns of B; delta: one takes G, the
@@ -729,6 +729,13 @@ tc_pipe_products(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
         }
       } else {
         constexpr int kCols = 4 * D / kLMath;  // columns per warp
+        if (half == 0) {
+          // dz_k: column 0 of the ones-column accumulator.
+          uint32_t v[32];
+          tmem_ld32(tDZ + lq, v);
+          tmem_wait_ld();
+          dz[slice * D + k] = __uint_as_float(v[0]);
+        }
         const uint32_t ta = tB + lq + kCols * half;
         float4* dst = reinterpret_cast<float4*>(Bbuf + (slice * D + k) * D + kCols * half);
 #pragma unroll
@@ -842,8 +849,8 @@ __global__ void __launch_bounds__(D) combine_delta(const float* __restrict__ M_i
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
         const float2 g2 = make_float2(gr[i], gr[i]);
-        acc[i][0] = fma2(g2, mlo, acc[i][0]);
-        acc[i][1] = fma2(g2, mhi, acc[i][1]);
+        acc[i][0] = pk::fma2(g2, mlo, acc[i][0]);
+        acc[i][1] = pk::fma2(g2, mhi, acc[i][1]);
       }
     }
 #pragma unroll
