@@ -456,6 +456,10 @@ tc_segment_products(const __grid_constant__ CUtensorMap tm_k, const __grid_const
 // alternating operand buffers, so the math warps build block b+1 while the
 // tensor core multiplies block b; dz (linear) by the tensor core too, from
 // a constant operand whose first column is ones.
+// Persistent: one CTA per SM walks the (segment, KV head) items, with the
+// block counters running on across items, so the producer streams the next
+// item's blocks while the math warps write the last item's products out of
+// TMEM (the accumulator is handed back to the MMA warp through acc_empty).
 // The linear rule is HBM-bound (each block brings 32 KiB of K and V); the
 // delta rule does 20 MMAs (128 x 128 x 16) per block.
 constexpr int kLTok = 64;      // tokens per block
@@ -465,8 +469,7 @@ struct PipeSmem {
   static constexpr int kD = 128;
   // Math warps: 16 (2 tokens per thread and block, to hide the latency of
   // the sigma chain -- and, for the delta rule, of r_t's shuffle sum and
-  // 1/r_t; the parts go straight to the operand buffer, so the thread state
-  // fits in 76 registers).
+  // 1/r_t; the parts go straight to the operand buffer).
   static constexpr int kMath = 16;
   static constexpr int kThreads = 64 + 32 * kMath;
   static constexpr int kTL = 2 * kMath;                   // token lanes
@@ -481,10 +484,9 @@ struct PipeSmem {
   // Linear rule: a constant [64 tokens][64] panel whose column 0 is 1.0, the
   // B operand of the MMA that sums sigma(K) over the tokens (dz).
   static constexpr int kOnes = kOp + 2 * kOpParts * kHalf;
-  static constexpr int kZ = kOnes + (DELTA ? 0 : kPanel);  // z_{s-1} fp32 [128] (delta)
-  static constexpr int kBar = kZ + (DELTA ? kD * 4 : 0);
-  // full[kStages] empty[kStages] op_full[2] op_empty[2] acc_full
-  static constexpr int kNumBars = 2 * kStages + 5;
+  static constexpr int kBar = kOnes + (DELTA ? 0 : kPanel);
+  // full[kStages] empty[kStages] op_full[2] op_empty[2] acc_full acc_empty drain
+  static constexpr int kNumBars = 2 * kStages + 7;
   static constexpr int kTmemSlot = kBar + kNumBars * 8;
   static constexpr int kAbort = kTmemSlot + 4;
   static constexpr int kAlloc = kAbort + 4 + 1024;
@@ -497,18 +499,20 @@ template <bool DELTA>
 __global__ void __launch_bounds__(PipeSmem<DELTA>::kThreads, 1)
 tc_pipe_products(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                  const float* __restrict__ z_pref, float* __restrict__ Gbuf, float* __restrict__ Bbuf,
-                 float* __restrict__ dz, unsigned int* __restrict__ status, int L, int S) {
+                 float* __restrict__ dz, unsigned int* __restrict__ status, int L, int S, int T,
+                 int BH) {
   using SM = PipeSmem<DELTA>;
   constexpr int D = SM::kD;
   constexpr int kStages = SM::kStages;
   constexpr int kLMath = SM::kMath;
-  constexpr int kLThreads = SM::kThreads;
   constexpr int kTL = SM::kTL;
   constexpr int kTPT = SM::kTokPerThread;
-  const int s = blockIdx.x, bh = blockIdx.y, BH = gridDim.y;
-  const int seg0 = s * S, seg_len = min(S, L - seg0);
-  const int nblk = (seg_len + kLTok - 1) / kLTok;
-  const size_t slice = (size_t)s * BH + bh;
+  const int items = T * BH;
+  // Item -> (segment s = item % T, KV head bh = item / T).
+  auto item_blocks = [&](int item) {
+    const int seg_len = min(S, L - (item % T) * S);
+    return (seg_len + kLTok - 1) / kLTok;
+  };
 
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   unsigned char* smem = reinterpret_cast<unsigned char*>(
@@ -516,13 +520,14 @@ tc_pipe_products(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
   unsigned char* ring = smem + SM::kRing;
   unsigned char* op = smem + SM::kOp;
   unsigned char* ones = smem + SM::kOnes;
-  float* zs = reinterpret_cast<float*>(smem + SM::kZ);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + SM::kBar);
   uint64_t* full = bars;
   uint64_t* empty = bars + kStages;
   uint64_t* op_full = bars + 2 * kStages;
   uint64_t* op_empty = op_full + 2;
   uint64_t* acc_full = op_empty + 2;
+  uint64_t* acc_empty = acc_full + 1;
+  uint64_t* drain = acc_empty + 1;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + SM::kTmemSlot);
   volatile int* abort = reinterpret_cast<volatile int*>(smem + SM::kAbort);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -543,15 +548,15 @@ tc_pipe_products(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
       mbar_init(op_empty + i, 1);
     }
     mbar_init(acc_full, 1);
+    mbar_init(acc_empty, kLMath);
+    mbar_init(drain, 1);
     *abort = 0;
     fence_mbar_init();
   }
-  if (DELTA)
-    for (int i = threadIdx.x; i < D; i += kLThreads) zs[i] = z_pref[slice * D + i];
   if (!DELTA) {
     // Row t of the ones panel: its 16-byte chunk that holds logical column 0
     // sits at chunk (t & 7) under the 128-byte swizzle.
-    for (int i = threadIdx.x; i < kLTok * 8; i += kLThreads) {
+    for (int i = threadIdx.x; i < kLTok * 8; i += SM::kThreads) {
       const int row = i / 8, chunk = i % 8;
       uint4 v = make_uint4(0, 0, 0, 0);
       if (chunk == (row & 7)) v.x = 0x3F80u;  // element (row, 0) = bf16(1.0)
@@ -571,23 +576,26 @@ tc_pipe_products(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
 
   if (warp == 0) {
     // ---------------------------------------------- TMA producer (whole warp waits, one elected lane issues)
-    int issued = 0;
-    for (int b = 0; b < nblk; ++b) {
-      const int st = b % kStages;
-      const uint32_t ph = (uint32_t)(b / kStages) & 1u;
-      if (!__all_sync(0xffffffffu, mbar_wait(empty + st, ph ^ 1u, abort, status))) break;
-      if (elect_one()) {
-        unsigned char* dst = ring + st * SM::kStage;
-        mbar_arrive_expect_tx(full + st, SM::kStage);
-        for (int p = 0; p < D / 64; ++p) {
-          tma_load_3d(dst + p * SM::kPanel, &tm_k, full + st, p * 64, seg0 + b * kLTok, bh);
-          tma_load_3d(dst + SM::kHalf + p * SM::kPanel, &tm_v, full + st, p * 64, seg0 + b * kLTok, bh);
+    int gb = 0;  // blocks issued so far (all items)
+    bool ok = true;
+    for (int item = blockIdx.x; ok && item < items; item += gridDim.x) {
+      const int seg0 = (item % T) * S, bh = item / T, nblk = item_blocks(item);
+      for (int b = 0; b < nblk; ++b, ++gb) {
+        const int st = gb % kStages;
+        const uint32_t ph = (uint32_t)(gb / kStages) & 1u;
+        if (!(ok = __all_sync(0xffffffffu, mbar_wait(empty + st, ph ^ 1u, abort, status)))) break;
+        if (elect_one()) {
+          unsigned char* dst = ring + st * SM::kStage;
+          mbar_arrive_expect_tx(full + st, SM::kStage);
+          for (int p = 0; p < D / 64; ++p) {
+            tma_load_3d(dst + p * SM::kPanel, &tm_k, full + st, p * 64, seg0 + b * kLTok, bh);
+            tma_load_3d(dst + SM::kHalf + p * SM::kPanel, &tm_v, full + st, p * 64, seg0 + b * kLTok, bh);
+          }
         }
       }
-      issued = b + 1;
     }
     // Every copy issued must land before the CTA exits.
-    for (int b = max(0, issued - kStages); b < issued; ++b)
+    for (int b = max(0, gb - kStages); b < gb; ++b)
       mbar_wait(full + b % kStages, (uint32_t)(b / kStages) & 1u, abort, status, false);
     __syncwarp();
   } else if (warp == 1) {
@@ -598,121 +606,130 @@ tc_pipe_products(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
     const uint64_t dring = sw128_desc(smem_u32(ring + SM::kHalf), SM::kPanel, 1024);
     const uint64_t dones = sw128_desc(smem_u32(ones), SM::kPanel, 1024);
     bool ok = true;
-    for (int b = 0; ok && b < nblk; ++b) {
-      const int st = b % kStages, ob = b & 1;
-      if (!(ok = __all_sync(0xffffffffu, mbar_wait(op_full + ob, (uint32_t)(b >> 1) & 1u, abort, status)))) break;
-      if (!(ok = __all_sync(0xffffffffu, mbar_wait(full + st, (uint32_t)(b / kStages) & 1u, abort, status)))) break;
-      tc_fence_after();
-      if (elect_one()) {
-        // Operand parts: sigma hi, sigma lo, (Y hi, Y lo).
-        const uint64_t shi = dop + ((ob * SM::kOpParts * SM::kHalf) >> 4);
-        const uint64_t slo = shi + (SM::kHalf >> 4);
-        const uint64_t yhi = shi + ((2 * SM::kHalf) >> 4);
-        const uint64_t ylo = shi + ((3 * SM::kHalf) >> 4);
-        const uint64_t vv = dring + ((st * SM::kStage) >> 4);
+    int gb = 0, j = 0;  // blocks and items so far
+    for (int item = blockIdx.x; ok && item < items; item += gridDim.x, ++j) {
+      const int nblk = item_blocks(item);
+      // The accumulator is free once the math warps have read item j - 1's.
+      if (!(ok = __all_sync(0xffffffffu, mbar_wait(acc_empty, ((uint32_t)j & 1u) ^ 1u, abort, status)))) break;
+      for (int b = 0; b < nblk; ++b, ++gb) {
+        const int st = gb % kStages, ob = gb & 1;
+        if (!(ok = __all_sync(0xffffffffu, mbar_wait(op_full + ob, (uint32_t)(gb >> 1) & 1u, abort, status)))) break;
+        if (!(ok = __all_sync(0xffffffffu, mbar_wait(full + st, (uint32_t)(gb / kStages) & 1u, abort, status)))) break;
+        tc_fence_after();
+        if (elect_one()) {
+          // Operand parts: sigma hi, sigma lo, (Y hi, Y lo).
+          const uint64_t shi = dop + ((ob * SM::kOpParts * SM::kHalf) >> 4);
+          const uint64_t slo = shi + (SM::kHalf >> 4);
+          const uint64_t yhi = shi + ((2 * SM::kHalf) >> 4);
+          const uint64_t ylo = shi + ((3 * SM::kHalf) >> 4);
+          const uint64_t vv = dring + ((st * SM::kStage) >> 4);
 #pragma unroll
-        for (int kk = 0; kk < kLTok / 16; ++kk) {
-          const uint32_t stp = mnmajor_step(kk);
-          const uint32_t acc = (b > 0 || kk > 0) ? 1u : 0u;
-          if (DELTA) {
-            mma_ss(tG, yhi + stp, shi + stp, idesc, acc);
-            mma_ss(tG, ylo + stp, shi + stp, idesc, 1u);
-            mma_ss(tG, yhi + stp, slo + stp, idesc, 1u);
+          for (int kk = 0; kk < kLTok / 16; ++kk) {
+            const uint32_t stp = mnmajor_step(kk);
+            const uint32_t acc = (b > 0 || kk > 0) ? 1u : 0u;
+            if (DELTA) {
+              mma_ss(tG, yhi + stp, shi + stp, idesc, acc);
+              mma_ss(tG, ylo + stp, shi + stp, idesc, 1u);
+              mma_ss(tG, yhi + stp, slo + stp, idesc, 1u);
+            }
+            mma_ss(tB, shi + stp, vv + stp, idesc, acc);
+            mma_ss(tB, slo + stp, vv + stp, idesc, 1u);
+            if (!DELTA) {
+              mma_ss(tDZ, shi + stp, dones + stp, idesc_dz, acc);
+              mma_ss(tDZ, slo + stp, dones + stp, idesc_dz, 1u);
+            }
           }
-          mma_ss(tB, shi + stp, vv + stp, idesc, acc);
-          mma_ss(tB, slo + stp, vv + stp, idesc, 1u);
-          if (!DELTA) {
-            mma_ss(tDZ, shi + stp, dones + stp, idesc_dz, acc);
-            mma_ss(tDZ, slo + stp, dones + stp, idesc_dz, 1u);
-          }
+          tc_commit(op_empty + ob);
+          tc_commit(empty + st);
+          if (b == nblk - 1) tc_commit(acc_full);
         }
-        tc_commit(op_empty + ob);
-        tc_commit(empty + st);
       }
     }
-    if (elect_one()) tc_commit(acc_full);
+    // Every MMA issued must complete before the accumulator is released.
+    if (elect_one()) tc_commit(drain);
     __syncwarp();
-    mbar_wait(acc_full, 0, abort, status, false);
+    mbar_wait(drain, 0, abort, status, false);
     __syncwarp();
   } else {
     // ---------------------------------------------- math warps
     // Thread (column chunk cg of 8 columns, token lane tl): tokens tl,
     // tl + kTL, ...; the 16 threads of a token are lanes 0..15 or 16..31 of
-    // one warp.
+    // one warp.  Epilogue: TMEM lane k = row k of the products.
     const int mt = threadIdx.x - 64;
     const int cg = mt & 15, tl = mt >> 4;
-    float zc[8];
-    if (DELTA) {
-#pragma unroll
-      for (int i = 0; i < 8; ++i) zc[i] = zs[8 * cg + i];
-    }
+    const int k = 32 * (warp & 3) + lane, quarter = (warp - 2) >> 2;  // quarter 0..3
+    const uint32_t lq = (uint32_t)(32 * (warp & 3)) << 16;
     bool ok = true;
-    for (int b = 0; b < nblk; ++b) {
-      const int st = b % kStages, ob = b & 1;
-      ok = __all_sync(0xffffffffu, mbar_wait(full + st, (uint32_t)(b / kStages) & 1u, abort, status));
-      if (!ok) break;
-      const unsigned char* kb = ring + st * SM::kStage;
-      // The operand buffer is free once the MMAs of block b - 2 are done
-      // (long before, normally); the parts go straight into it.
-      ok = __all_sync(0xffffffffu, mbar_wait(op_empty + ob, ((uint32_t)(b >> 1) & 1u) ^ 1u, abort, status));
-      if (!ok) break;
-      unsigned char* hb = op + ob * SM::kOpParts * SM::kHalf;
+    int gb = 0, j = 0;
+    for (int item = blockIdx.x; ok && item < items; item += gridDim.x, ++j) {
+      const int s = item % T, bh = item / T, nblk = item_blocks(item);
+      const int seg_len = min(S, L - s * S);
+      const size_t slice = (size_t)s * BH + bh;
+      float zc[8];
+      if (DELTA) {
+        const float4 za = *reinterpret_cast<const float4*>(z_pref + slice * D + 8 * cg);
+        const float4 zb = *reinterpret_cast<const float4*>(z_pref + slice * D + 8 * cg + 4);
+        zc[0] = za.x; zc[1] = za.y; zc[2] = za.z; zc[3] = za.w;
+        zc[4] = zb.x; zc[5] = zb.y; zc[6] = zb.z; zc[7] = zb.w;
+      }
+      for (int b = 0; b < nblk; ++b, ++gb) {
+        const int st = gb % kStages, ob = gb & 1;
+        if (!(ok = __all_sync(0xffffffffu, mbar_wait(full + st, (uint32_t)(gb / kStages) & 1u, abort, status)))) break;
+        const unsigned char* kb = ring + st * SM::kStage;
+        // The operand buffer is free once the MMAs of block gb - 2 are done
+        // (long before, normally); the parts go straight into it.
+        if (!(ok = __all_sync(0xffffffffu, mbar_wait(op_empty + ob, ((uint32_t)(gb >> 1) & 1u) ^ 1u, abort, status)))) break;
+        unsigned char* hb = op + ob * SM::kOpParts * SM::kHalf;
 #pragma unroll
-      for (int i = 0; i < kTPT; ++i) {
-        const int t = tl + kTL * i;
-        const bool valid = b * kLTok + t < seg_len;
-        const uint32_t off = sw128_offset(t, 8 * cg, kLTok);
-        uint4 kv = *reinterpret_cast<const uint4*>(kb + off);
-        // (rows past the segment: sigma = 0 exactly)
-        if (!valid) kv = make_uint4(0xFF7FFF7Fu, 0xFF7FFF7Fu, 0xFF7FFF7Fu, 0xFF7FFF7Fu);
-        const uint32_t kw[4] = {kv.x, kv.y, kv.z, kv.w};
-        float2 sg[4];
-        uint32_t hw[4], lw[4];
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          sg[e] = pk::sigma_pair(kw[e]);
-          pk::split_pair(sg[e], hw[e], lw[e]);
-        }
-        *reinterpret_cast<uint4*>(hb + off) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
-        *reinterpret_cast<uint4*>(hb + SM::kHalf + off) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
-        if (DELTA) {
-          // r_t = sigma(k_t) . z_{s-1} over the token's 16 threads; Y = sigma / r.
-          float r = 0.f;
+        for (int i = 0; i < kTPT; ++i) {
+          const int t = tl + kTL * i;
+          const bool valid = b * kLTok + t < seg_len;
+          const uint32_t off = sw128_offset(t, 8 * cg, kLTok);
+          uint4 kv = *reinterpret_cast<const uint4*>(kb + off);
+          // (rows past the segment: sigma = 0 exactly)
+          if (!valid) kv = make_uint4(0xFF7FFF7Fu, 0xFF7FFF7Fu, 0xFF7FFF7Fu, 0xFF7FFF7Fu);
+          const uint32_t kw[4] = {kv.x, kv.y, kv.z, kv.w};
+          float2 sg[4];
+          uint32_t hw[4], lw[4];
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
-            r = fmaf(sg[e].x, zc[2 * e], r);
-            r = fmaf(sg[e].y, zc[2 * e + 1], r);
+            sg[e] = pk::sigma_pair(kw[e]);
+            pk::split_pair(sg[e], hw[e], lw[e]);
           }
+          *reinterpret_cast<uint4*>(hb + off) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+          *reinterpret_cast<uint4*>(hb + SM::kHalf + off) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
+          if (DELTA) {
+            // r_t = sigma(k_t) . z_{s-1} over the token's 16 threads; Y = sigma / r.
+            float r = 0.f;
 #pragma unroll
-          for (int o = 8; o > 0; o >>= 1) r += __shfl_xor_sync(0xffffffffu, r, o);
-          const float w = r != 0.f ? 1.f / r : 0.f;
-          uint32_t yh[4], yl[4];
+            for (int e = 0; e < 4; ++e) {
+              r = fmaf(sg[e].x, zc[2 * e], r);
+              r = fmaf(sg[e].y, zc[2 * e + 1], r);
+            }
 #pragma unroll
-          for (int e = 0; e < 4; ++e) pk::split_pair(pk::mul2(make_float2(w, w), sg[e]), yh[e], yl[e]);
-          *reinterpret_cast<uint4*>(hb + 2 * SM::kHalf + off) = make_uint4(yh[0], yh[1], yh[2], yh[3]);
-          *reinterpret_cast<uint4*>(hb + 3 * SM::kHalf + off) = make_uint4(yl[0], yl[1], yl[2], yl[3]);
+            for (int o = 8; o > 0; o >>= 1) r += __shfl_xor_sync(0xffffffffu, r, o);
+            const float w = r != 0.f ? 1.f / r : 0.f;
+            uint32_t yh[4], yl[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) pk::split_pair(pk::mul2(make_float2(w, w), sg[e]), yh[e], yl[e]);
+            *reinterpret_cast<uint4*>(hb + 2 * SM::kHalf + off) = make_uint4(yh[0], yh[1], yh[2], yh[3]);
+            *reinterpret_cast<uint4*>(hb + 3 * SM::kHalf + off) = make_uint4(yl[0], yl[1], yl[2], yl[3]);
+          }
         }
+        // K of this block has been read.
+        __syncwarp();
+        if (lane == 0) mbar_arrive(empty + st);
+        fence_proxy_async();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(op_full + ob);
       }
-      // K of this block has been read.
-      __syncwarp();
-      if (lane == 0) mbar_arrive(empty + st);
-      fence_proxy_async();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(op_full + ob);
-    }
-    // The products: TMEM lane k = row k.  Linear: the kMath / 4 warps of a
-    // lane quarter share the 128 columns of B; delta: one takes G, the
-    // other B.
-    if (ok) ok = __all_sync(0xffffffffu, mbar_wait(acc_full, 0, abort, status));
-    if (ok) {
+      if (!ok) break;
+      // The item's products out of TMEM.
+      if (!(ok = __all_sync(0xffffffffu, mbar_wait(acc_full, (uint32_t)j & 1u, abort, status)))) break;
       tc_fence_after();
-      const int k = 32 * (warp & 3) + lane, half = (warp - 2) >> 2;
-      const uint32_t lq = (uint32_t)(32 * (warp & 3)) << 16;
       if (DELTA) {
-        // The delta rule's 16 math warps: four per lane quarter, each a
-        // quarter of the columns of G or of B.
+        // Four warps per lane quarter, each a quarter of the columns of G or of B.
         constexpr int kCols = 8 * D / kLMath;  // columns per warp
-        const int quarter = (warp - 2) >> 2;     // 0..3
         const int which = quarter >> 1, part = quarter & 1;
         float* rowp = (which ? Bbuf : Gbuf) + (slice * D + k) * D + kCols * part;
         const uint32_t ta = (which ? tB : tG) + lq + kCols * part;
@@ -729,15 +746,15 @@ tc_pipe_products(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
         }
       } else {
         constexpr int kCols = 4 * D / kLMath;  // columns per warp
-        if (half == 0) {
+        if (quarter == 0) {
           // dz_k: column 0 of the ones-column accumulator.
           uint32_t v[32];
           tmem_ld32(tDZ + lq, v);
           tmem_wait_ld();
           dz[slice * D + k] = __uint_as_float(v[0]);
         }
-        const uint32_t ta = tB + lq + kCols * half;
-        float4* dst = reinterpret_cast<float4*>(Bbuf + (slice * D + k) * D + kCols * half);
+        const uint32_t ta = tB + lq + kCols * quarter;
+        float4* dst = reinterpret_cast<float4*>(Bbuf + (slice * D + k) * D + kCols * quarter);
 #pragma unroll
         for (int c = 0; c < kCols / 32; ++c) {
           uint32_t v[32];
@@ -749,6 +766,9 @@ tc_pipe_products(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
                                          __uint_as_float(v[4 * i + 2]), __uint_as_float(v[4 * i + 3]));
         }
       }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(acc_empty);
     }
   }
   tc_fence_before();
@@ -976,8 +996,13 @@ cudaError_t launch_pipe_products(const Problem& p, cudaStream_t stream) {
   auto kern = tc_pipe_products<DELTA>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
-  kern<<<dim3(p.T, (unsigned)BHkv), PipeSmem<DELTA>::kThreads, smem, stream>>>(
-      lk, lv, p.z_pref, p.Gbuf, p.Bbuf, p.dz, p.status, p.L, p.S);
+  int dev = 0, sms = 0;
+  if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
+  if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
+  const long items = (long)p.T * (long)BHkv;
+  const int grid = (int)(items < sms ? items : sms);  // persistent: one CTA per SM
+  kern<<<grid, PipeSmem<DELTA>::kThreads, smem, stream>>>(lk, lv, p.z_pref, p.Gbuf, p.Bbuf, p.dz,
+                                                         p.status, p.L, p.S, p.T, (int)BHkv);
   return cudaGetLastError();
 }
 
