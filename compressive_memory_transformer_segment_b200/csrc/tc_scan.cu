@@ -460,24 +460,28 @@ tc_segment_products(const __grid_constant__ CUtensorMap tm_k, const __grid_const
 // block counters running on across items, so the producer streams the next
 // item's blocks while the math warps write the last item's products out of
 // TMEM (the accumulator is handed back to the MMA warp through acc_empty).
-// The linear rule is HBM-bound (each block brings 32 KiB of K and V); the
-// delta rule does 20 MMAs (128 x 128 x 16) per block.
+// The linear rule is HBM-bound (each block brings 2 x 64 x d bf16 of K and
+// V); the delta rule does 20 MMAs (128 x d x 16) per block.  For d = 64 the
+// products' M = 128 operands (sigma(K)^T, Y^T) carry a zero upper half.
 constexpr int kLTok = 64;      // tokens per block
 
-template <bool DELTA>
+template <int D_, bool DELTA>
 struct PipeSmem {
-  static constexpr int kD = 128;
-  // Math warps: 16 (2 tokens per thread and block, to hide the latency of
-  // the sigma chain -- and, for the delta rule, of r_t's shuffle sum and
-  // 1/r_t; the parts go straight to the operand buffer).
-  static constexpr int kMath = 16;
+  static constexpr int kD = D_;
+  // Math warps: 2 tokens per thread and block, 8 columns per thread (16
+  // warps for d = 128, 8 for d = 64), to hide the latency of the sigma
+  // chain -- and, for the delta rule, of r_t's shuffle sum and 1/r_t; the
+  // parts go straight to the operand buffer.
+  static constexpr int kMath = kD / 8;
   static constexpr int kThreads = 64 + 32 * kMath;
-  static constexpr int kTL = 2 * kMath;                   // token lanes
+  static constexpr int kCG = kD / 8;                      // 8-column chunks per token
+  static constexpr int kTL = 32 * kMath / kCG;            // token lanes
   static constexpr int kTokPerThread = kLTok / kTL;
-  static constexpr int kStages = DELTA ? 2 : 4;          // K/V ring depth
+  static constexpr int kStages = DELTA ? 256 / kD : 512 / kD;  // K/V ring depth
   static constexpr int kPanel = kLTok * 128;              // 64 rows x 128 B
-  static constexpr int kHalf = kLTok * kD * 2;            // one 64 x 128 bf16 block
-  static constexpr int kStage = 2 * kHalf;                // K then V
+  static constexpr int kBlk = kLTok * kD * 2;             // one 64 x d bf16 block
+  static constexpr int kStage = 2 * kBlk;                 // K then V
+  static constexpr int kHalf = kLTok * 128 * 2;           // one 64 x 128 operand part
   static constexpr int kOpParts = DELTA ? 4 : 2;          // sigma hi, lo (, Y hi, lo)
   static constexpr int kRing = 0;
   static constexpr int kOp = kRing + kStages * kStage;    // [2][parts]
@@ -492,16 +496,16 @@ struct PipeSmem {
   static constexpr int kAlloc = kAbort + 4 + 1024;
   // TMEM: delta [G | B]; linear [B | dz (16 columns, column 0 used)].
   static constexpr uint32_t kTmemCols = 256;
-  static_assert(kOnes % 1024 == 0, "ones panel alignment");
+  static_assert(kOnes % 1024 == 0 && kTokPerThread * kTL == kLTok, "pipe layout");
 };
 
-template <bool DELTA>
-__global__ void __launch_bounds__(PipeSmem<DELTA>::kThreads, 1)
+template <int D_, bool DELTA>
+__global__ void __launch_bounds__(PipeSmem<D_, DELTA>::kThreads, 1)
 tc_pipe_products(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                  const float* __restrict__ z_pref, float* __restrict__ Gbuf, float* __restrict__ Bbuf,
                  float* __restrict__ dz, unsigned int* __restrict__ status, int L, int S, int T,
                  int BH) {
-  using SM = PipeSmem<DELTA>;
+  using SM = PipeSmem<D_, DELTA>;
   constexpr int D = SM::kD;
   constexpr int kStages = SM::kStages;
   constexpr int kLMath = SM::kMath;
@@ -553,6 +557,11 @@ tc_pipe_products(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
     *abort = 0;
     fence_mbar_init();
   }
+  if (D < 128) {
+    // The operand parts' upper panel (rows D..127 of sigma(K)^T, Y^T) stays 0.
+    for (int i = threadIdx.x; i < 2 * SM::kOpParts * SM::kHalf / 16; i += SM::kThreads)
+      *reinterpret_cast<uint4*>(op + i * 16) = make_uint4(0, 0, 0, 0);
+  }
   if (!DELTA) {
     // Row t of the ones panel: its 16-byte chunk that holds logical column 0
     // sits at chunk (t & 7) under the 128-byte swizzle.
@@ -562,8 +571,8 @@ tc_pipe_products(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
       if (chunk == (row & 7)) v.x = 0x3F80u;  // element (row, 0) = bf16(1.0)
       *reinterpret_cast<uint4*>(ones + i * 16) = v;
     }
-    fence_proxy_async();
   }
+  fence_proxy_async();
   if (warp == 1) {
     tmem_alloc(tmem_slot, SM::kTmemCols);
     tmem_relinquish();
@@ -589,7 +598,7 @@ tc_pipe_products(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
           mbar_arrive_expect_tx(full + st, SM::kStage);
           for (int p = 0; p < D / 64; ++p) {
             tma_load_3d(dst + p * SM::kPanel, &tm_k, full + st, p * 64, seg0 + b * kLTok, bh);
-            tma_load_3d(dst + SM::kHalf + p * SM::kPanel, &tm_v, full + st, p * 64, seg0 + b * kLTok, bh);
+            tma_load_3d(dst + SM::kBlk + p * SM::kPanel, &tm_v, full + st, p * 64, seg0 + b * kLTok, bh);
           }
         }
       }
@@ -603,7 +612,7 @@ tc_pipe_products(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
     constexpr uint32_t idesc = idesc_bf16_f32(128, D, true, true);
     constexpr uint32_t idesc_dz = idesc_bf16_f32(128, 16, true, true);
     const uint64_t dop = sw128_desc(smem_u32(op), SM::kPanel, 1024);
-    const uint64_t dring = sw128_desc(smem_u32(ring + SM::kHalf), SM::kPanel, 1024);
+    const uint64_t dring = sw128_desc(smem_u32(ring + SM::kBlk), SM::kPanel, 1024);
     const uint64_t dones = sw128_desc(smem_u32(ones), SM::kPanel, 1024);
     bool ok = true;
     int gb = 0, j = 0;  // blocks and items so far
@@ -653,11 +662,11 @@ tc_pipe_products(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
   } else {
     // ---------------------------------------------- math warps
     // Thread (column chunk cg of 8 columns, token lane tl): tokens tl,
-    // tl + kTL, ...; the 16 threads of a token are lanes 0..15 or 16..31 of
-    // one warp.  Epilogue: TMEM lane k = row k of the products.
+    // tl + kTL, ...; the D/8 threads of a token are consecutive lanes of one
+    // warp.  Epilogue: TMEM lane k = row k of the products.
     const int mt = threadIdx.x - 64;
-    const int cg = mt & 15, tl = mt >> 4;
-    const int k = 32 * (warp & 3) + lane, quarter = (warp - 2) >> 2;  // quarter 0..3
+    const int cg = mt % SM::kCG, tl = mt / SM::kCG;
+    const int k = 32 * (warp & 3) + lane, quarter = (warp - 2) >> 2;  // 0..kMath/4-1
     const uint32_t lq = (uint32_t)(32 * (warp & 3)) << 16;
     bool ok = true;
     int gb = 0, j = 0;
@@ -699,7 +708,7 @@ tc_pipe_products(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
           *reinterpret_cast<uint4*>(hb + off) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
           *reinterpret_cast<uint4*>(hb + SM::kHalf + off) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
           if (DELTA) {
-            // r_t = sigma(k_t) . z_{s-1} over the token's 16 threads; Y = sigma / r.
+            // r_t = sigma(k_t) . z_{s-1} over the token's D/8 threads; Y = sigma / r.
             float r = 0.f;
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
@@ -707,7 +716,7 @@ tc_pipe_products(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
               r = fmaf(sg[e].y, zc[2 * e + 1], r);
             }
 #pragma unroll
-            for (int o = 8; o > 0; o >>= 1) r += __shfl_xor_sync(0xffffffffu, r, o);
+            for (int o = SM::kCG / 2; o > 0; o >>= 1) r += __shfl_xor_sync(0xffffffffu, r, o);
             const float w = r != 0.f ? 1.f / r : 0.f;
             uint32_t yh[4], yl[4];
 #pragma unroll
@@ -727,43 +736,32 @@ tc_pipe_products(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
       // The item's products out of TMEM.
       if (!(ok = __all_sync(0xffffffffu, mbar_wait(acc_full, (uint32_t)j & 1u, abort, status)))) break;
       tc_fence_after();
-      if (DELTA) {
-        // Four warps per lane quarter, each a quarter of the columns of G or of B.
-        constexpr int kCols = 8 * D / kLMath;  // columns per warp
-        const int which = quarter >> 1, part = quarter & 1;
-        float* rowp = (which ? Bbuf : Gbuf) + (slice * D + k) * D + kCols * part;
-        const uint32_t ta = (which ? tB : tG) + lq + kCols * part;
-#pragma unroll
-        for (int c = 0; c < kCols / 32; ++c) {
-          uint32_t v[32];
-          tmem_ld32(ta + 32 * c, v);
-          tmem_wait_ld();
-          float4* dst = reinterpret_cast<float4*>(rowp + 32 * c);
-#pragma unroll
-          for (int i = 0; i < 8; ++i)
-            dst[i] = make_float4(__uint_as_float(v[4 * i]), __uint_as_float(v[4 * i + 1]),
-                                 __uint_as_float(v[4 * i + 2]), __uint_as_float(v[4 * i + 3]));
-        }
-      } else {
-        constexpr int kCols = 4 * D / kLMath;  // columns per warp
-        if (quarter == 0) {
+      // kMath / 4 warps per TMEM lane quarter share the row's columns: delta
+      // [G | B] (2D columns), linear B (D columns) and dz.  For D = 64 only
+      // lanes 0..63 hold rows.
+      constexpr int kParts = kLMath / 4;
+      constexpr int kCols = (DELTA ? 2 * D : D) / kParts;  // columns per warp
+      if (k < D) {
+        if (!DELTA && quarter == 0) {
           // dz_k: column 0 of the ones-column accumulator.
           uint32_t v[32];
           tmem_ld32(tDZ + lq, v);
           tmem_wait_ld();
           dz[slice * D + k] = __uint_as_float(v[0]);
         }
-        const uint32_t ta = tB + lq + kCols * quarter;
-        float4* dst = reinterpret_cast<float4*>(Bbuf + (slice * D + k) * D + kCols * quarter);
 #pragma unroll
         for (int c = 0; c < kCols / 32; ++c) {
+          const int col = kCols * quarter + 32 * c;  // of [G | B] or of B
+          const bool isB = !DELTA || col >= D;
+          const int cc = DELTA && col >= D ? col - D : col;
           uint32_t v[32];
-          tmem_ld32(ta + 32 * c, v);
+          tmem_ld32((isB ? tB : tG) + lq + cc, v);
           tmem_wait_ld();
+          float4* dst = reinterpret_cast<float4*>((isB ? Bbuf : Gbuf) + (slice * D + k) * D + cc);
 #pragma unroll
           for (int i = 0; i < 8; ++i)
-            dst[8 * c + i] = make_float4(__uint_as_float(v[4 * i]), __uint_as_float(v[4 * i + 1]),
-                                         __uint_as_float(v[4 * i + 2]), __uint_as_float(v[4 * i + 3]));
+            dst[i] = make_float4(__uint_as_float(v[4 * i]), __uint_as_float(v[4 * i + 1]),
+                                 __uint_as_float(v[4 * i + 2]), __uint_as_float(v[4 * i + 3]));
         }
       }
       tc_fence_before();
@@ -986,14 +984,14 @@ cudaError_t launch_products(const Problem& p, const CUtensorMap& tk, const CUten
   return cudaGetLastError();
 }
 
-template <bool DELTA>
+template <int D, bool DELTA>
 cudaError_t launch_pipe_products(const Problem& p, cudaStream_t stream) {
   CUtensorMap lk, lv;
   const uint64_t BHkv = (uint64_t)p.B * p.H_kv;
-  if (!make_map(&lk, p.k, 128, p.L, BHkv, kLTok) || !make_map(&lv, p.v, 128, p.L, BHkv, kLTok))
+  if (!make_map(&lk, p.k, D, p.L, BHkv, kLTok) || !make_map(&lv, p.v, D, p.L, BHkv, kLTok))
     return cudaErrorInvalidValue;
-  const int smem = PipeSmem<DELTA>::kAlloc;
-  auto kern = tc_pipe_products<DELTA>;
+  const int smem = PipeSmem<D, DELTA>::kAlloc;
+  auto kern = tc_pipe_products<D, DELTA>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
   int dev = 0, sms = 0;
@@ -1001,7 +999,7 @@ cudaError_t launch_pipe_products(const Problem& p, cudaStream_t stream) {
   if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
   const long items = (long)p.T * (long)BHkv;
   const int grid = (int)(items < sms ? items : sms);  // persistent: one CTA per SM
-  kern<<<grid, PipeSmem<DELTA>::kThreads, smem, stream>>>(lk, lv, p.z_pref, p.Gbuf, p.Bbuf, p.dz,
+  kern<<<grid, PipeSmem<D, DELTA>::kThreads, smem, stream>>>(lk, lv, p.z_pref, p.Gbuf, p.Bbuf, p.dz,
                                                          p.status, p.L, p.S, p.T, (int)BHkv);
   return cudaGetLastError();
 }
@@ -1025,10 +1023,7 @@ cudaError_t launch(const Problem& p, cudaStream_t stream) {
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     zprefix<D><<<BH, D, 0, stream>>>(p.dz, p.z_in, p.z_pref, p.z_out, p.T, C);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    if (D == 128)
-      e = launch_pipe_products<true>(p, stream);
-    else
-      e = small ? launch_products<D, true, 64>(p, tk, tv, stream) : launch_products<D, true, 128>(p, tk, tv, stream);
+    e = small ? launch_products<D, true, 64>(p, tk, tv, stream) : launch_pipe_products<D, true>(p, stream);
     if (e != cudaSuccess) return e;
     const int csmem = (2 * D * D + D * kCB) * (int)sizeof(float);
     e = cudaFuncSetAttribute(combine_delta<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, csmem);
@@ -1037,11 +1032,7 @@ cudaError_t launch(const Problem& p, cudaStream_t stream) {
                                                                  p.T);
     return cudaGetLastError();
   }
-  if (D == 128)
-    e = launch_pipe_products<false>(p, stream);
-  else
-    e = small ? launch_products<D, false, 64>(p, tk, tv, stream)
-              : launch_products<D, false, 128>(p, tk, tv, stream);
+  e = small ? launch_products<D, false, 64>(p, tk, tv, stream) : launch_pipe_products<D, false>(p, stream);
   if (e != cudaSuccess) return e;
   combine_linear<D><<<dim3(BH, (D * D + 1023) / 1024), 256, 0, stream>>>(
       p.M_in, p.Bbuf, p.dz, Mp, p.z_in, p.z_pref, p.M_out, p.z_out, p.T);

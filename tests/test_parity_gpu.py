@@ -283,6 +283,13 @@ TC_CASES = [
                                          H_kv=2)),
     ("tc_small_d128_S64_delta", dict(dtype="bf16", d_k=128, d_v=128, L=384, seg_len=64, H_q=2,
                                      H_kv=2, rule="delta")),
+    # More (segment, KV head) items than SMs: the persistent products kernel
+    # runs several items per CTA (block counters and the accumulator hand-off
+    # carry across items), with a ragged last segment.
+    ("tc_d64_S256_delta_items", dict(dtype="bf16", d_k=64, d_v=64, L=8292, seg_len=256, B=2,
+                                     H_q=3, H_kv=3, rule="delta")),
+    ("tc_d128_S128_linear_items", dict(dtype="bf16", d_k=128, d_v=128, L=6405, seg_len=128,
+                                       H_q=3, H_kv=3)),
 ]
 
 
