@@ -458,8 +458,13 @@ tc_segment_products(const __grid_constant__ CUtensorMap tm_k, const __grid_const
 // a constant operand whose first column is ones.
 // Persistent: one CTA per SM walks the (segment, KV head) items, with the
 // block counters running on across items, so the producer streams the next
-// item's blocks while the math warps write the last item's products out of
-// TMEM (the accumulator is handed back to the MMA warp through acc_empty).
+// items' blocks ahead.  Two TMEM accumulators alternate between items (an
+// accumulator goes back to the MMA warp through its acc_empty barrier); for
+// d = 64, whose items can be a single block, the math warps write item j's
+// products out of TMEM only after building the first block of item j + 1,
+// so that the tensor core works meanwhile.  (For d = 128 the epilogue
+// follows the item's last block: items are long there, and the 576-thread
+// CTA has no registers to spare inside the block loop.)
 // The linear rule is HBM-bound (each block brings 2 x 64 x d bf16 of K and
 // V); the delta rule does 20 MMAs (128 x d x 16) per block.  For d = 64 the
 // products' M = 128 operands (sigma(K)^T, Y^T) carry a zero upper half.
@@ -489,13 +494,15 @@ struct PipeSmem {
   // B operand of the MMA that sums sigma(K) over the tokens (dz).
   static constexpr int kOnes = kOp + 2 * kOpParts * kHalf;
   static constexpr int kBar = kOnes + (DELTA ? 0 : kPanel);
-  // full[kStages] empty[kStages] op_full[2] op_empty[2] acc_full acc_empty drain
-  static constexpr int kNumBars = 2 * kStages + 7;
+  // full[kStages] empty[kStages] op_full[2] op_empty[2] acc_full[2] acc_empty[2] drain
+  static constexpr int kNumBars = 2 * kStages + 9;
   static constexpr int kTmemSlot = kBar + kNumBars * 8;
   static constexpr int kAbort = kTmemSlot + 4;
   static constexpr int kAlloc = kAbort + 4 + 1024;
-  // TMEM: delta [G | B]; linear [B | dz (16 columns, column 0 used)].
-  static constexpr uint32_t kTmemCols = 256;
+  // TMEM: two accumulators of 256 columns, delta [G | B], linear [B | dz
+  // (16 columns, column 0 used)].
+  static constexpr uint32_t kAccCols = 256;
+  static constexpr uint32_t kTmemCols = 2 * kAccCols;
   static_assert(kOnes % 1024 == 0 && kTokPerThread * kTL == kLTok, "pipe layout");
 };
 
@@ -529,9 +536,9 @@ tc_pipe_products(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
   uint64_t* empty = bars + kStages;
   uint64_t* op_full = bars + 2 * kStages;
   uint64_t* op_empty = op_full + 2;
-  uint64_t* acc_full = op_empty + 2;
-  uint64_t* acc_empty = acc_full + 1;
-  uint64_t* drain = acc_empty + 1;
+  uint64_t* acc_full = op_empty + 2;    // [2]
+  uint64_t* acc_empty = acc_full + 2;   // [2]
+  uint64_t* drain = acc_empty + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + SM::kTmemSlot);
   volatile int* abort = reinterpret_cast<volatile int*>(smem + SM::kAbort);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -551,8 +558,10 @@ tc_pipe_products(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
       mbar_init(op_full + i, kLMath);
       mbar_init(op_empty + i, 1);
     }
-    mbar_init(acc_full, 1);
-    mbar_init(acc_empty, kLMath);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(acc_full + i, 1);
+      mbar_init(acc_empty + i, kLMath);
+    }
     mbar_init(drain, 1);
     *abort = 0;
     fence_mbar_init();
@@ -581,7 +590,10 @@ tc_pipe_products(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  const uint32_t tG = tmem, tB = DELTA ? tmem + 128 : tmem, tDZ = tmem + 128;
+  // Accumulator a: G at 0 and B at 128 (delta), B at 0 and dz at 128 (linear).
+  auto tG = [&](int a) { return tmem + a * SM::kAccCols; };
+  auto tB = [&](int a) { return tmem + a * SM::kAccCols + (DELTA ? 128 : 0); };
+  auto tDZ = [&](int a) { return tmem + a * SM::kAccCols + 128; };
 
   if (warp == 0) {
     // ---------------------------------------------- TMA producer (whole warp waits, one elected lane issues)
@@ -617,9 +629,9 @@ tc_pipe_products(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
     bool ok = true;
     int gb = 0, j = 0;  // blocks and items so far
     for (int item = blockIdx.x; ok && item < items; item += gridDim.x, ++j) {
-      const int nblk = item_blocks(item);
-      // The accumulator is free once the math warps have read item j - 1's.
-      if (!(ok = __all_sync(0xffffffffu, mbar_wait(acc_empty, ((uint32_t)j & 1u) ^ 1u, abort, status)))) break;
+      const int nblk = item_blocks(item), a = j & 1;
+      // Accumulator a is free once the math warps have read item j - 2's.
+      if (!(ok = __all_sync(0xffffffffu, mbar_wait(acc_empty + a, ((uint32_t)(j >> 1) & 1u) ^ 1u, abort, status)))) break;
       for (int b = 0; b < nblk; ++b, ++gb) {
         const int st = gb % kStages, ob = gb & 1;
         if (!(ok = __all_sync(0xffffffffu, mbar_wait(op_full + ob, (uint32_t)(gb >> 1) & 1u, abort, status)))) break;
@@ -637,20 +649,20 @@ tc_pipe_products(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
             const uint32_t stp = mnmajor_step(kk);
             const uint32_t acc = (b > 0 || kk > 0) ? 1u : 0u;
             if (DELTA) {
-              mma_ss(tG, yhi + stp, shi + stp, idesc, acc);
-              mma_ss(tG, ylo + stp, shi + stp, idesc, 1u);
-              mma_ss(tG, yhi + stp, slo + stp, idesc, 1u);
+              mma_ss(tG(a), yhi + stp, shi + stp, idesc, acc);
+              mma_ss(tG(a), ylo + stp, shi + stp, idesc, 1u);
+              mma_ss(tG(a), yhi + stp, slo + stp, idesc, 1u);
             }
-            mma_ss(tB, shi + stp, vv + stp, idesc, acc);
-            mma_ss(tB, slo + stp, vv + stp, idesc, 1u);
+            mma_ss(tB(a), shi + stp, vv + stp, idesc, acc);
+            mma_ss(tB(a), slo + stp, vv + stp, idesc, 1u);
             if (!DELTA) {
-              mma_ss(tDZ, shi + stp, dones + stp, idesc_dz, acc);
-              mma_ss(tDZ, slo + stp, dones + stp, idesc_dz, 1u);
+              mma_ss(tDZ(a), shi + stp, dones + stp, idesc_dz, acc);
+              mma_ss(tDZ(a), slo + stp, dones + stp, idesc_dz, 1u);
             }
           }
           tc_commit(op_empty + ob);
           tc_commit(empty + st);
-          if (b == nblk - 1) tc_commit(acc_full);
+          if (b == nblk - 1) tc_commit(acc_full + a);
         }
       }
     }
@@ -668,18 +680,71 @@ tc_pipe_products(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
     const int cg = mt % SM::kCG, tl = mt / SM::kCG;
     const int k = 32 * (warp & 3) + lane, quarter = (warp - 2) >> 2;  // 0..kMath/4-1
     const uint32_t lq = (uint32_t)(32 * (warp & 3)) << 16;
+    // Item jj's products (slice sl) out of accumulator jj & 1: kMath / 4
+    // warps per TMEM lane quarter share the row's columns, delta [G | B]
+    // (2D columns), linear B (D columns) and dz.  For D = 64 only lanes
+    // 0..63 hold rows.
+    auto epilogue = [&](int jj, size_t sl) -> bool {
+      const int a = jj & 1;
+      if (!__all_sync(0xffffffffu, mbar_wait(acc_full + a, (uint32_t)(jj >> 1) & 1u, abort, status)))
+        return false;
+      tc_fence_after();
+      constexpr int kParts = kLMath / 4;
+      constexpr int kCols = (DELTA ? 2 * D : D) / kParts;  // columns per warp
+      if (k < D) {
+        if (!DELTA && quarter == 0) {
+          // dz_k: column 0 of the ones-column accumulator.
+          uint32_t v[32];
+          tmem_ld32(tDZ(a) + lq, v);
+          tmem_wait_ld();
+          dz[sl * D + k] = __uint_as_float(v[0]);
+        }
+#pragma unroll
+        for (int c = 0; c < kCols / 32; ++c) {
+          const int col = kCols * quarter + 32 * c;  // of [G | B] or of B
+          const bool isB = !DELTA || col >= D;
+          const int cc = DELTA && col >= D ? col - D : col;
+          uint32_t v[32];
+          tmem_ld32((isB ? tB(a) : tG(a)) + lq + cc, v);
+          tmem_wait_ld();
+          float4* dst = reinterpret_cast<float4*>((isB ? Bbuf : Gbuf) + (sl * D + k) * D + cc);
+#pragma unroll
+          for (int i = 0; i < 8; ++i)
+            dst[i] = make_float4(__uint_as_float(v[4 * i]), __uint_as_float(v[4 * i + 1]),
+                                 __uint_as_float(v[4 * i + 2]), __uint_as_float(v[4 * i + 3]));
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(acc_empty + a);
+      return true;
+    };
+    auto load_z = [&](int item, float* zc) {
+      const size_t sl = (size_t)(item % T) * BH + item / T;
+      const float4 za = *reinterpret_cast<const float4*>(z_pref + sl * D + 8 * cg);
+      const float4 zb = *reinterpret_cast<const float4*>(z_pref + sl * D + 8 * cg + 4);
+      zc[0] = za.x; zc[1] = za.y; zc[2] = za.z; zc[3] = za.w;
+      zc[4] = zb.x; zc[5] = zb.y; zc[6] = zb.z; zc[7] = zb.w;
+    };
     bool ok = true;
     int gb = 0, j = 0;
+    size_t prev_slice = 0;  // item j - 1's slice, whose products are still in TMEM
+    // d = 64 (short items, registers to spare) writes item j's products
+    // after item j + 1's first block, and loads z_{s-1} one item ahead.
+    constexpr bool kLag = D < 128, kZAhead = D < 128;
+    float zc[8], zn[8];
+    if (DELTA && kZAhead && blockIdx.x < items) load_z(blockIdx.x, zn);
     for (int item = blockIdx.x; ok && item < items; item += gridDim.x, ++j) {
       const int s = item % T, bh = item / T, nblk = item_blocks(item);
       const int seg_len = min(S, L - s * S);
       const size_t slice = (size_t)s * BH + bh;
-      float zc[8];
-      if (DELTA) {
-        const float4 za = *reinterpret_cast<const float4*>(z_pref + slice * D + 8 * cg);
-        const float4 zb = *reinterpret_cast<const float4*>(z_pref + slice * D + 8 * cg + 4);
-        zc[0] = za.x; zc[1] = za.y; zc[2] = za.z; zc[3] = za.w;
-        zc[4] = zb.x; zc[5] = zb.y; zc[6] = zb.z; zc[7] = zb.w;
+      if (DELTA && kZAhead) {
+        // z_{s-1} of this item (loaded one item ahead), then the next item's.
+#pragma unroll
+        for (int i = 0; i < 8; ++i) zc[i] = zn[i];
+        if (item + (int)gridDim.x < items) load_z(item + gridDim.x, zn);
+      } else if (DELTA) {
+        load_z(item, zc);
       }
       for (int b = 0; b < nblk; ++b, ++gb) {
         const int st = gb % kStages, ob = gb & 1;
@@ -731,43 +796,13 @@ tc_pipe_products(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
         fence_proxy_async();
         __syncwarp();
         if (lane == 0) mbar_arrive(op_full + ob);
+        // With the tensor core fed, the previous item's products.
+        if (kLag && b == 0 && j > 0 && !(ok = epilogue(j - 1, prev_slice))) break;
       }
-      if (!ok) break;
-      // The item's products out of TMEM.
-      if (!(ok = __all_sync(0xffffffffu, mbar_wait(acc_full, (uint32_t)j & 1u, abort, status)))) break;
-      tc_fence_after();
-      // kMath / 4 warps per TMEM lane quarter share the row's columns: delta
-      // [G | B] (2D columns), linear B (D columns) and dz.  For D = 64 only
-      // lanes 0..63 hold rows.
-      constexpr int kParts = kLMath / 4;
-      constexpr int kCols = (DELTA ? 2 * D : D) / kParts;  // columns per warp
-      if (k < D) {
-        if (!DELTA && quarter == 0) {
-          // dz_k: column 0 of the ones-column accumulator.
-          uint32_t v[32];
-          tmem_ld32(tDZ + lq, v);
-          tmem_wait_ld();
-          dz[slice * D + k] = __uint_as_float(v[0]);
-        }
-#pragma unroll
-        for (int c = 0; c < kCols / 32; ++c) {
-          const int col = kCols * quarter + 32 * c;  // of [G | B] or of B
-          const bool isB = !DELTA || col >= D;
-          const int cc = DELTA && col >= D ? col - D : col;
-          uint32_t v[32];
-          tmem_ld32((isB ? tB : tG) + lq + cc, v);
-          tmem_wait_ld();
-          float4* dst = reinterpret_cast<float4*>((isB ? Bbuf : Gbuf) + (slice * D + k) * D + cc);
-#pragma unroll
-          for (int i = 0; i < 8; ++i)
-            dst[i] = make_float4(__uint_as_float(v[4 * i]), __uint_as_float(v[4 * i + 1]),
-                                 __uint_as_float(v[4 * i + 2]), __uint_as_float(v[4 * i + 3]));
-        }
-      }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(acc_empty);
+      if (!kLag && ok) ok = epilogue(j, slice);
+      prev_slice = slice;
     }
+    if (kLag && ok && j > 0) ok = epilogue(j - 1, prev_slice);
   }
   tc_fence_before();
   __syncthreads();
@@ -984,6 +1019,8 @@ cudaError_t launch_products(const Problem& p, const CUtensorMap& tk, const CUten
   return cudaGetLastError();
 }
 
+constexpr bool kSmallSegKernel = false;
+
 template <int D, bool DELTA>
 cudaError_t launch_pipe_products(const Problem& p, cudaStream_t stream) {
   CUtensorMap lk, lv;
@@ -1023,7 +1060,7 @@ cudaError_t launch(const Problem& p, cudaStream_t stream) {
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     zprefix<D><<<BH, D, 0, stream>>>(p.dz, p.z_in, p.z_pref, p.z_out, p.T, C);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    e = small ? launch_products<D, true, 64>(p, tk, tv, stream) : launch_pipe_products<D, true>(p, stream);
+    e = kSmallSegKernel && small ? launch_products<D, true, 64>(p, tk, tv, stream) : launch_pipe_products<D, true>(p, stream);
     if (e != cudaSuccess) return e;
     const int csmem = (2 * D * D + D * kCB) * (int)sizeof(float);
     e = cudaFuncSetAttribute(combine_delta<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, csmem);
@@ -1032,7 +1069,7 @@ cudaError_t launch(const Problem& p, cudaStream_t stream) {
                                                                  p.T);
     return cudaGetLastError();
   }
-  e = small ? launch_products<D, false, 64>(p, tk, tv, stream) : launch_pipe_products<D, false>(p, stream);
+  e = kSmallSegKernel && small ? launch_products<D, false, 64>(p, tk, tv, stream) : launch_pipe_products<D, false>(p, stream);
   if (e != cudaSuccess) return e;
   combine_linear<D><<<dim3(BH, (D * D + 1023) / 1024), 256, 0, stream>>>(
       p.M_in, p.Bbuf, p.dz, Mp, p.z_in, p.z_pref, p.M_out, p.z_out, p.T);
