@@ -13,9 +13,9 @@
 // z does not depend on M, so every segment's (G_s, B_s) can be formed at once:
 //   zsum / zprefix (delta only): dz_s = column sums of sigma(K_s), then the
 //       prefix z_{s-1} for every segment and z_T;
-//   tc_segment_products (tcgen05): one CTA per (segment, KV head) forms
-//       B_s (and dz_s through a constant ones column, linear rule) and, for
-//       the delta rule, G_s = Y^T sigma(K) with Y = D^-1 sigma(K);
+//   tc_pipe_products (tcgen05, persistent): for every (segment, KV head)
+//       item, B_s (and dz_s through a constant ones column, linear rule)
+//       and, for the delta rule, G_s = Y^T sigma(K) with Y = D^-1 sigma(K);
 //   combine_delta / combine_linear (fp32): walks the segments in order,
 //       publishing M_{s-1} (bf16, read by the attention kernel's retrieval)
 //       and z_{s-1}, and writes M_T, z_T.
@@ -119,334 +119,7 @@ constexpr int kZChunksMax = 8;
 // Row chunks per segment for zsum: about 256 rows each, at most kZChunksMax.
 int zsum_chunks(int S) { return S >= 256 * kZChunksMax ? kZChunksMax : (S >= 512 ? S / 256 : 1); }
 
-// ---------------------------------------------------------------- segment products
-
-// Tokens per block: 128, or 64 for segments of at most 64 tokens (half the
-// shared memory, so more CTAs fit on an SM when a segment is one block).
-template <int D, bool DELTA, int TOK>
-struct ProdSmem {
-  // Roles: warp 0 TMA, warp 1 MMA, then TOK / 16 math warps: two threads per
-  // token, each with half of the columns.
-  static constexpr int kMathWarps = TOK / 16;
-  static constexpr int kThreads = 64 + 32 * kMathWarps;
-  static constexpr int kK = 0;                                      // K block [TOK][D]
-  static constexpr int kV = kK + TOK * D * 2;                       // V block [TOK][D] (+ ones)
-  static constexpr int kVBytes = TOK * D * 2 + (DELTA ? 0 : TOK * 64 * 2);
-  static constexpr int kSkHi = kV + kVBytes;                        // [TOK tok][128] (2 panels)
-  static constexpr int kSkLo = kSkHi + TOK * 128 * 2;
-  static constexpr int kYHi = kSkLo + TOK * 128 * 2;                // delta only
-  static constexpr int kYLo = kYHi + (DELTA ? TOK * 128 * 2 : 0);
-  static constexpr int kZ = kYLo + (DELTA ? TOK * 128 * 2 : 0);     // fp32 z_{s-1}
-  static constexpr int kBar = kZ + 128 * 4;
-  // k_full k_empty v_full v_empty op_ready op_free done
-  static constexpr int kNumBars = 7;
-  static constexpr int kTmemSlot = kBar + kNumBars * 8;
-  static constexpr int kAbort = kTmemSlot + 4;
-  static constexpr int kAlloc = kAbort + 4 + 1024;
-  // TMEM: delta G [0, 128) and B [128, 128 + D); linear [B | dz] [0, D + 16).
-  static constexpr uint32_t kTmemCols = (DELTA || D + 16 > 128) ? 256 : 128;
-};
-
-// Grid (T, B*H_kv).  Roles: warp 0 TMA producer (K, V blocks), warp 1 TMEM
-// allocation + MMA issue, warps 2.. two threads per token of the block (each
-// half of the columns) and, at the end, one per row of the products (the
-// warps of a TMEM lane quarter splitting the column chunks).
-// TMEM: delta G [0, D), B [128, 128 + D); linear [B | dz] [0, D + 16).
-template <int D, bool DELTA, int TOK>
-__global__ void __launch_bounds__(ProdSmem<D, DELTA, TOK>::kThreads, 1)
-tc_segment_products(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
-                    const float* __restrict__ z_pref, float* __restrict__ Gbuf,
-                    float* __restrict__ Bbuf, float* __restrict__ dz,
-                    unsigned int* __restrict__ status, int L, int S) {
-  using SM = ProdSmem<D, DELTA, TOK>;
-  constexpr int kTok = TOK;
-  constexpr int kThreads = SM::kThreads, kMathWarps = SM::kMathWarps;
-  constexpr uint32_t kTmemCols = SM::kTmemCols;
-  const int s = blockIdx.x, bh = blockIdx.y, BH = gridDim.y;
-  const int seg0 = s * S, seg_len = min(S, L - seg0);
-  const int nblk = (seg_len + kTok - 1) / kTok;
-  const size_t slice = (size_t)s * BH + bh;
-
-  extern __shared__ __align__(1024) unsigned char smem_raw[];
-  unsigned char* smem = reinterpret_cast<unsigned char*>(
-      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  unsigned char* sK = smem + SM::kK;
-  unsigned char* sV = smem + SM::kV;
-  unsigned char* sSkHi = smem + SM::kSkHi;
-  unsigned char* sSkLo = smem + SM::kSkLo;
-  unsigned char* sYHi = smem + SM::kYHi;
-  unsigned char* sYLo = smem + SM::kYLo;
-  float* zs = reinterpret_cast<float*>(smem + SM::kZ);
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + SM::kBar);
-  uint64_t* k_full = bars + 0;
-  uint64_t* k_empty = bars + 1;
-  uint64_t* v_full = bars + 2;
-  uint64_t* v_empty = bars + 3;
-  uint64_t* op_ready = bars + 4;
-  uint64_t* op_free = bars + 5;
-  uint64_t* done = bars + 6;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + SM::kTmemSlot);
-  volatile int* abort = reinterpret_cast<volatile int*>(smem + SM::kAbort);
-
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  // The MMA and copy issue relies on elect.sync picking lane 0 of a
-  // converged warp every time (commits and their MMAs from one thread).
-  if (__syncthreads_or(elected_lane() != 0)) {
-    if (threadIdx.x == 0) atomicOr(status, kStatusLayout);
-    return;
-  }
-
-  if (threadIdx.x == 0) {
-    mbar_init(k_full, 1);
-    mbar_init(k_empty, kMathWarps);   // one arrival per math warp
-    mbar_init(v_full, 1);
-    mbar_init(v_empty, 1);
-    mbar_init(op_ready, kMathWarps);
-    mbar_init(op_free, 1);
-    mbar_init(done, 1);
-    *abort = 0;
-    fence_mbar_init();
-  }
-  if (warp == 1) {
-    tmem_alloc(tmem_slot, kTmemCols);
-    tmem_relinquish();
-    tc_fence_before();
-  }
-  // Constant operand parts: the ones column after V (linear rule) and, for
-  // D = 64, the zero upper halves of sigma(K) and Y (the products' M = 128).
-  for (int i = threadIdx.x; i < kTok * 64 * 2 / 16; i += kThreads) {
-    const int row = i / 8, chunk = i % 8;
-    if (!DELTA) {
-      uint4 v = make_uint4(0, 0, 0, 0);
-      if (chunk == (row & 7)) v.x = 0x3F80u;  // element (row, 0) = bf16(1.0)
-      *reinterpret_cast<uint4*>(sV + kTok * D * 2 + i * 16) = v;
-    }
-    if (D == 64) {
-      const uint4 zero = make_uint4(0, 0, 0, 0);
-      *reinterpret_cast<uint4*>(sSkHi + kTok * 128 + i * 16) = zero;
-      *reinterpret_cast<uint4*>(sSkLo + kTok * 128 + i * 16) = zero;
-      if (DELTA) {
-        *reinterpret_cast<uint4*>(sYHi + kTok * 128 + i * 16) = zero;
-        *reinterpret_cast<uint4*>(sYLo + kTok * 128 + i * 16) = zero;
-      }
-    }
-  }
-  if (DELTA)
-    for (int i = threadIdx.x; i < 128; i += kThreads) zs[i] = i < D ? z_pref[slice * D + i] : 0.f;
-  fence_proxy_async();
-  __syncthreads();
-  tc_fence_after();
-  const uint32_t tmem = *tmem_slot;
-
-  if (warp == 0) {
-    {
-      // ------------------------------------------------ TMA producer
-      // The whole warp runs the loop and every wait (kept warp-uniform);
-      // one elected lane issues the copies.
-      int issued_k = 0, issued_v = 0;
-      for (int blk = 0; blk < nblk; ++blk) {
-        const uint32_t par = (blk & 1) ^ 1;
-        if (!__all_sync(0xffffffffu, mbar_wait(k_empty, par, abort, status))) break;
-        if (elect_one()) {
-          mbar_arrive_expect_tx(k_full, kTok * D * 2);
-          for (int p = 0; p < D / 64; ++p)
-            tma_load_3d(sK + p * kTok * 128, &tm_k, k_full, p * 64, seg0 + blk * kTok, bh);
-        }
-        issued_k = blk + 1;
-        if (!__all_sync(0xffffffffu, mbar_wait(v_empty, par, abort, status))) break;
-        if (elect_one()) {
-          mbar_arrive_expect_tx(v_full, kTok * D * 2);
-          for (int p = 0; p < D / 64; ++p)
-            tma_load_3d(sV + p * kTok * 128, &tm_v, v_full, p * 64, seg0 + blk * kTok, bh);
-        }
-        issued_v = blk + 1;
-      }
-      if (issued_k > 0) mbar_wait(k_full, (issued_k - 1) & 1, abort, status, false);
-      if (issued_v > 0) mbar_wait(v_full, (issued_v - 1) & 1, abort, status, false);
-      __syncwarp();
-    }
-  } else if (warp == 1) {
-    {
-      // ------------------------------------------------ MMA issuer
-      // The whole warp runs the loop and every wait; one elected lane issues.
-      // All operands are MN-major [tokens][128] tiles (panels of 64 columns,
-      // 16 KiB apart); one 16-token K step = 2048 bytes.
-      const uint64_t skhi = sw128_desc(smem_u32(sSkHi), kTok * 128, 1024);
-      const uint64_t sklo = sw128_desc(smem_u32(sSkLo), kTok * 128, 1024);
-      const uint64_t yhi = sw128_desc(smem_u32(sYHi), kTok * 128, 1024);
-      const uint64_t ylo = sw128_desc(smem_u32(sYLo), kTok * 128, 1024);
-      const uint64_t vv = sw128_desc(smem_u32(sV), kTok * 128, 1024);
-      constexpr uint32_t idesc_d = idesc_bf16_f32(128, D, true, true);
-      constexpr uint32_t idesc_ext = idesc_bf16_f32(128, D + 16, true, true);
-      const uint32_t tG = tmem, tB = DELTA ? tmem + 128 : tmem;
-      bool ok = true;
-      for (int blk = 0; ok && blk < nblk; ++blk) {
-        if (!(ok = __all_sync(0xffffffffu, mbar_wait(op_ready, blk & 1, abort, status)))) break;
-        if (!(ok = __all_sync(0xffffffffu, mbar_wait(v_full, blk & 1, abort, status)))) break;
-        tc_fence_after();
-        if (elect_one()) {
-#pragma unroll
-          for (int kk = 0; kk < kTok / 16; ++kk) {
-            const uint32_t st = mnmajor_step(kk);
-            const uint32_t acc = (blk > 0 || kk > 0) ? 1u : 0u;
-            if (DELTA) {
-              mma_ss(tG, yhi + st, skhi + st, idesc_d, acc);
-              mma_ss(tG, ylo + st, skhi + st, idesc_d, 1u);
-              mma_ss(tG, yhi + st, sklo + st, idesc_d, 1u);
-              mma_ss(tB, skhi + st, vv + st, idesc_d, acc);
-              mma_ss(tB, sklo + st, vv + st, idesc_d, 1u);
-            } else {
-              mma_ss(tB, skhi + st, vv + st, idesc_ext, acc);
-              mma_ss(tB, sklo + st, vv + st, idesc_ext, 1u);
-            }
-          }
-          tc_commit(op_free);
-          tc_commit(v_empty);
-        }
-      }
-      if (elect_one()) tc_commit(done);
-      __syncwarp();
-      mbar_wait(done, 0, abort, status, false);
-      __syncwarp();
-    }
-  } else {
-    // -------------------------------------------------- math threads
-    // Sigma phase: thread -> (token t, column half hp), the two threads of a
-    // token in adjacent lanes.  Products phase: thread -> TMEM lane (row of
-    // the products) and a share of the column chunks.
-    const int mt = threadIdx.x - 64;
-    const int t = mt >> 1, hp = mt & 1;
-    const int c8_0 = hp * (D / 16);
-    const uint32_t lane_off = (uint32_t)(32 * (warp & 3)) << 16;
-    bool ok = true;
-    for (int blk = 0; blk < nblk; ++blk) {
-      if (blk > 0) {
-        ok = __all_sync(0xffffffffu, mbar_wait(op_free, (blk - 1) & 1, abort, status));
-        if (!ok) break;
-      }
-      ok = __all_sync(0xffffffffu, mbar_wait(k_full, blk & 1, abort, status));
-      if (!ok) break;
-      const bool has_tok = t < kTok;  // (always, with two threads per token)
-      const bool valid = has_tok && blk * kTok + t < seg_len;
-      // sigma(K) row t as hi/lo pairs (rows past the segment are 0), and
-      // r_t = sigma(k_t) . z_{s-1} (delta): each thread half the columns,
-      // the halves added across the lane pair.
-      float r = 0.f;
-#pragma unroll 4
-      for (int c8 = c8_0; c8 < c8_0 + D / 16; ++c8) {
-        const uint32_t off = sw128_offset(t, 8 * c8, kTok);
-        const uint4 kv = has_tok ? *reinterpret_cast<const uint4*>(sK + off) : make_uint4(0, 0, 0, 0);
-        const uint32_t kw[4] = {kv.x, kv.y, kv.z, kv.w};
-        float zc[8];
-        if (DELTA) {
-          const float4 za = *reinterpret_cast<const float4*>(zs + 8 * c8);
-          const float4 zb = *reinterpret_cast<const float4*>(zs + 8 * c8 + 4);
-          zc[0] = za.x; zc[1] = za.y; zc[2] = za.z; zc[3] = za.w;
-          zc[4] = zb.x; zc[5] = zb.y; zc[6] = zb.z; zc[7] = zb.w;
-        }
-        uint32_t hw[4], lw[4];
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const float a = valid ? elu1_fast(bf16lo_to_f32(kw[i])) : 0.f;
-          const float b = valid ? elu1_fast(bf16hi_to_f32(kw[i])) : 0.f;
-          if (DELTA) {
-            r = fmaf(a, zc[2 * i], r);
-            r = fmaf(b, zc[2 * i + 1], r);
-          }
-          hw[i] = pack_bf16x2(a, b);
-          lw[i] = pack_bf16x2(a - bf16lo_to_f32(hw[i]), b - bf16hi_to_f32(hw[i]));
-        }
-        if (has_tok) {
-          *reinterpret_cast<uint4*>(sSkHi + off) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
-          *reinterpret_cast<uint4*>(sSkLo + off) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
-        }
-      }
-      // (a + b == b + a: both threads of the token get the same r)
-      if (DELTA) r += __shfl_xor_sync(0xffffffffu, r, 1);
-      __syncwarp();
-      if (lane == 0) mbar_arrive(k_empty);
-      if (DELTA && has_tok) {
-        // Y = sigma(K) / r (0 where r = 0), from the pair just written.
-        const float w = r != 0.f ? 1.f / r : 0.f;
-#pragma unroll 4
-        for (int c8 = c8_0; c8 < c8_0 + D / 16; ++c8) {
-          const uint32_t off = sw128_offset(t, 8 * c8, kTok);
-          const uint4 hv = *reinterpret_cast<const uint4*>(sSkHi + off);
-          const uint4 lv = *reinterpret_cast<const uint4*>(sSkLo + off);
-          const uint32_t hh[4] = {hv.x, hv.y, hv.z, hv.w}, ll[4] = {lv.x, lv.y, lv.z, lv.w};
-          uint32_t hw[4], lw[4];
-#pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            const float a = w * (bf16lo_to_f32(hh[i]) + bf16lo_to_f32(ll[i]));
-            const float b = w * (bf16hi_to_f32(hh[i]) + bf16hi_to_f32(ll[i]));
-            hw[i] = pack_bf16x2(a, b);
-            lw[i] = pack_bf16x2(a - bf16lo_to_f32(hw[i]), b - bf16hi_to_f32(hw[i]));
-          }
-          *reinterpret_cast<uint4*>(sYHi + off) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
-          *reinterpret_cast<uint4*>(sYLo + off) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
-        }
-      }
-      fence_proxy_async();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(op_ready);
-    }
-    // The segment's products, row k (k < D), to the workspace in fp32: the
-    // warps of a TMEM lane quarter take turns with the 32-column chunks.
-    const int k = 32 * (warp & 3) + lane;
-    constexpr int kParts = kMathWarps / 4;
-    const int part = (warp - 2) >> 2;
-    if (ok) ok = __all_sync(0xffffffffu, mbar_wait(done, 0, abort, status));
-    if (ok) {
-      tc_fence_after();
-      if (DELTA) {
-#pragma unroll
-        for (int c = part; c < D / 32; c += kParts) {
-          uint32_t g[32], bb[32];
-          tmem_ld32(tmem + lane_off + c * 32, g);
-          tmem_ld32(tmem + 128 + lane_off + c * 32, bb);
-          tmem_wait_ld();
-          if (k < D) {
-            float4* gd = reinterpret_cast<float4*>(Gbuf + (slice * D + k) * D + c * 32);
-            float4* bd = reinterpret_cast<float4*>(Bbuf + (slice * D + k) * D + c * 32);
-#pragma unroll
-            for (int i = 0; i < 8; ++i) {
-              gd[i] = make_float4(__uint_as_float(g[4 * i]), __uint_as_float(g[4 * i + 1]),
-                                  __uint_as_float(g[4 * i + 2]), __uint_as_float(g[4 * i + 3]));
-              bd[i] = make_float4(__uint_as_float(bb[4 * i]), __uint_as_float(bb[4 * i + 1]),
-                                  __uint_as_float(bb[4 * i + 2]), __uint_as_float(bb[4 * i + 3]));
-            }
-          }
-        }
-      } else {
-#pragma unroll
-        for (int c = part; c < D / 32 + 1; c += kParts) {
-          uint32_t bb[32];
-          tmem_ld32(tmem + lane_off + c * 32, bb);
-          tmem_wait_ld();
-          if (k < D) {
-            if (c < D / 32) {
-              float4* bd = reinterpret_cast<float4*>(Bbuf + (slice * D + k) * D + c * 32);
-#pragma unroll
-              for (int i = 0; i < 8; ++i)
-                bd[i] = make_float4(__uint_as_float(bb[4 * i]), __uint_as_float(bb[4 * i + 1]),
-                                    __uint_as_float(bb[4 * i + 2]), __uint_as_float(bb[4 * i + 3]));
-            } else {
-              dz[slice * D + k] = __uint_as_float(bb[0]);
-            }
-          }
-        }
-      }
-    }
-  }
-  tc_fence_before();
-  __syncthreads();
-  if (warp == 1) {
-    tc_fence_after();
-    tmem_dealloc(tmem, kTmemCols);
-  }
-}
-
-// ---------------------------------------------------------------- pipelined products (d = 128)
+// ---------------------------------------------------------------- pipelined products
 
 // Per (segment, KV head), streamed in 64-token blocks:
 //   linear: B_s = sigma(K_s)^T V_s and dz_s = column sums of sigma(K_s);
@@ -1007,20 +680,6 @@ bool make_map(CUtensorMap* m, const void* base, uint64_t cols, uint64_t rows, ui
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int D, bool DELTA, int TOK>
-cudaError_t launch_products(const Problem& p, const CUtensorMap& tk, const CUtensorMap& tv,
-                            cudaStream_t stream) {
-  const int smem = ProdSmem<D, DELTA, TOK>::kAlloc;
-  auto kern = tc_segment_products<D, DELTA, TOK>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-  if (e != cudaSuccess) return e;
-  kern<<<dim3(p.T, p.B * p.H_kv), ProdSmem<D, DELTA, TOK>::kThreads, smem, stream>>>(tk, tv, p.z_pref, p.Gbuf, p.Bbuf, p.dz,
-                                                           p.status, p.L, p.S);
-  return cudaGetLastError();
-}
-
-constexpr bool kSmallSegKernel = false;
-
 template <int D, bool DELTA>
 cudaError_t launch_pipe_products(const Problem& p, cudaStream_t stream) {
   CUtensorMap lk, lv;
@@ -1043,14 +702,7 @@ cudaError_t launch_pipe_products(const Problem& p, cudaStream_t stream) {
 
 template <int D>
 cudaError_t launch(const Problem& p, cudaStream_t stream) {
-  CUtensorMap tk, tv;
-  const uint64_t BHkv = (uint64_t)p.B * p.H_kv;
-  // 64-token blocks when a segment fits in one (see ProdSmem).
-  const bool small = p.S <= 64;
-  const uint32_t tok = small ? 64 : 128;
-  if (!make_map(&tk, p.k, D, p.L, BHkv, tok) || !make_map(&tv, p.v, D, p.L, BHkv, tok))
-    return cudaErrorInvalidValue;
-  const unsigned BH = (unsigned)BHkv;
+  const unsigned BH = (unsigned)((uint64_t)p.B * p.H_kv);
   __nv_bfloat16* Mp = static_cast<__nv_bfloat16*>(p.M_pref);
   cudaError_t e;
   if (p.delta) {
@@ -1060,7 +712,7 @@ cudaError_t launch(const Problem& p, cudaStream_t stream) {
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     zprefix<D><<<BH, D, 0, stream>>>(p.dz, p.z_in, p.z_pref, p.z_out, p.T, C);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    e = kSmallSegKernel && small ? launch_products<D, true, 64>(p, tk, tv, stream) : launch_pipe_products<D, true>(p, stream);
+    e = launch_pipe_products<D, true>(p, stream);
     if (e != cudaSuccess) return e;
     const int csmem = (2 * D * D + D * kCB) * (int)sizeof(float);
     e = cudaFuncSetAttribute(combine_delta<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, csmem);
@@ -1069,7 +721,7 @@ cudaError_t launch(const Problem& p, cudaStream_t stream) {
                                                                  p.T);
     return cudaGetLastError();
   }
-  e = kSmallSegKernel && small ? launch_products<D, false, 64>(p, tk, tv, stream) : launch_pipe_products<D, false>(p, stream);
+  e = launch_pipe_products<D, false>(p, stream);
   if (e != cudaSuccess) return e;
   combine_linear<D><<<dim3(BH, (D * D + 1023) / 1024), 256, 0, stream>>>(
       p.M_in, p.Bbuf, p.dz, Mp, p.z_in, p.z_pref, p.M_out, p.z_out, p.T);
