@@ -12,20 +12,22 @@
 //           is 0 (Memory Retrieval; "Leave No Context Behind" explainer,
 //           "メモリの読み出し");
 //   out   = sg(beta_h) A_mem + (1 - sg(beta_h)) A_dot   (Integration).
-// A row sees at most S <= 64 keys, all in the tile, so the softmax is a
-// single pass (no running max).  The retrieval of every segment of the tile
-// is one MMA chain: row r of sigma(Q), scaled as below, sits in the column
+// A row sees at most S <= 64 keys, all in the tile and all in its
+// segment's block of the scores, so the softmax is a single pass over that
+// block (no running max); P is zero outside it.  The retrieval of every
+// segment of the tile is one MMA chain: row r of sigma(Q) sits in the column
 // block of its segment of an expanded A operand (zeros elsewhere), and the
-// spt memories M_{s-1} are stacked along K as the B operand; the result is
-// accumulated into the P.V accumulator O:
-//   O = P V + (sigma(Q) c) [M_{s0-1}; M_{s0}; ...],  c_r = g l_r / ((1 - g) den_r),
-//   out_r = (1 - g) / l_r * O_r
-// (with g == 1 the retrieval overwrites O instead: c_r = 1/den_r, out = O).
+// spt memories M_{s-1} are stacked along K as the B operand:
+//   R = sigma(Q)_exp [M_{s0-1}; M_{s0}; ...],   O = P V,
+//   out_r = g / den_r * R_r + (1 - g) / l_r * O_r   (0 for the first term
+//   where den_r = 0).
+// The retrieval operand needs only Q and z, so it is built (and R computed)
+// while the scores are on the tensor core; the softmax follows.
 //
 // Roles (160 threads): warp 0 allocates TMEM, lane 0 issues the TMA loads,
 // every tcgen05.mma and the output store; warps 1..4 one thread per query
 // row (warp w serves TMEM lanes 32 (w % 4) ..).  TMEM: S = [0, 128) (scores,
-// then P as bf16 pairs), O = [128, 128 + D).
+// then P as bf16 pairs), O = [128, 128 + D), R = [128 + D, 128 + 2D).
 #include <cuda.h>
 
 #include "kernels.h"
@@ -39,7 +41,8 @@ using namespace tc;
 
 constexpr int kBM = 128;  // query rows (and keys) per tile
 constexpr int kThreads = 160;
-constexpr uint32_t kTmemCols = 256;
+template <int D>
+constexpr uint32_t tmem_cols() { return 128 + 2 * D <= 256 ? 256 : 512; }
 
 // Arrival of a whole warp on an mbarrier counted per warp: the warp's
 // threads synchronise (ordering their prior writes and TMEM accesses, each
@@ -130,6 +133,7 @@ tc_small_attention(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
     *abort = 0;
     fence_mbar_init();
   }
+  constexpr uint32_t kTmemCols = tmem_cols<D>();
   if (warp == 0) {
     tmem_alloc(tmem_slot, kTmemCols);
     tmem_relinquish();
@@ -162,7 +166,7 @@ tc_small_attention(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
       }
     }
     bool ok = __all_sync(0xffffffffu, mbar_wait(loaded, 0, abort, status));
-    const uint32_t tS = tmem, tO = tmem + 128;
+    const uint32_t tS = tmem, tO = tmem + 128, tR = tmem + 128 + D;
     if (ok) {
       tc_fence_after();
       if (elect_one()) {
@@ -174,6 +178,19 @@ tc_small_attention(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
         for (int kk = 0; kk < D / 16; ++kk)
           mma_ss(tS, dq + kmajor_step(kk, kBM), dk + kmajor_step(kk, kBM), idesc_qk, kk > 0 ? 1u : 0u);
         tc_commit(s_full);
+      }
+      ok = __all_sync(0xffffffffu, mbar_wait(a_ready, 0, abort, status));
+    }
+    if (ok) {
+      tc_fence_after();
+      if (elect_one()) {
+        // R = A_exp [M_{s0-1}; M_{s0}; ...]
+        constexpr uint32_t idesc_r = idesc_bf16_f32(kBM, D, false, true);
+        const uint64_t da = sw128_desc(smem_u32(sA), 16, 1024);
+        const uint64_t dm = sw128_desc(smem_u32(sM), SM::kKx * 128, 1024);
+#pragma unroll
+        for (int kk = 0; kk < SM::kKx / 16; ++kk)
+          mma_ss(tR, da + kmajor_step(kk, kBM), dm + mnmajor_step(kk), idesc_r, kk > 0 ? 1u : 0u);
       }
       ok = __all_sync(0xffffffffu, mbar_wait(p_ready, 0, abort, status));
     }
@@ -187,21 +204,6 @@ tc_small_attention(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
         for (int kk = 0; kk < kBM / 16; ++kk)
           mma_ts(tO, tS + (kk < 4 ? kk * 8 : 64 + (kk - 4) * 8), dv + mnmajor_step(kk), idesc_pv,
                  kk > 0 ? 1u : 0u);
-      }
-      ok = __all_sync(0xffffffffu, mbar_wait(a_ready, 0, abort, status));
-    }
-    if (ok) {
-      tc_fence_after();
-      if (elect_one()) {
-        // O (+)= A_exp [M_{s0-1}; M_{s0}; ...]: overwrites O when the gate is
-        // exactly 1 (only the retrieval is left).
-        const bool keep = gate_sigmoid(__ldg(beta + h)) != 1.f;
-        constexpr uint32_t idesc_r = idesc_bf16_f32(kBM, D, false, true);
-        const uint64_t da = sw128_desc(smem_u32(sA), 16, 1024);
-        const uint64_t dm = sw128_desc(smem_u32(sM), SM::kKx * 128, 1024);
-#pragma unroll
-        for (int kk = 0; kk < SM::kKx / 16; ++kk)
-          mma_ss(tO, da + kmajor_step(kk, kBM), dm + mnmajor_step(kk), idesc_r, (kk > 0 || keep) ? 1u : 0u);
         tc_commit(o_full);
       }
       ok = __all_sync(0xffffffffu, mbar_wait(staged, 0, abort, status));
@@ -210,7 +212,7 @@ tc_small_attention(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
       // Rows past the end of the sequence are clipped by the tensor bounds.
       for (int p = 0; p < kPanels; ++p) tma_store_3d(&tm_o, sQ + p * kBM * 128, p * 64, r0, bh);
       tma_store_commit();
-      tma_store_wait_all();
+      tma_store_wait_read();  // (the shared-memory source is read; the writes land on their own)
     }
     // Every MMA issued must be complete before TMEM is released (o_full
     // follows all of them; a wait that was abandoned drains here).
@@ -222,105 +224,110 @@ tc_small_attention(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
     // ------------------------------------------------ one thread per row
     const int r = 32 * (warp & 3) + lane;  // row of the tile (= TMEM lane)
     const uint32_t lane_off = (uint32_t)(32 * (warp & 3)) << 16;
-    const uint32_t tS = tmem + lane_off, tO = tmem + 128 + lane_off;
+    const uint32_t tS = tmem + lane_off, tO = tmem + 128 + lane_off, tR = tmem + 128 + D + lane_off;
     const int seg = r / S;                  // the row's segment within the tile
     const float sl2 = rsqrtf((float)D) * 1.4426950408889634f;
-    // (The loads completed before the scores; the wait on their barrier makes
-    // the tiles and z visible to this thread.)
-    bool ok = __all_sync(0xffffffffu, mbar_wait(loaded, 0, abort, status)) &&
-              __all_sync(0xffffffffu, mbar_wait(s_full, 0, abort, status));
-    float l = 0.f;
+    // (The wait on the loads' barrier makes the tiles and z visible here.)
+    bool ok = __all_sync(0xffffffffu, mbar_wait(loaded, 0, abort, status));
+    float den = 0.f, l = 0.f;
     if (ok) {
-      tc_fence_after();
-      uint32_t sv[128];
-#pragma unroll
-      for (int c = 0; c < 4; ++c) tmem_ld32(tS + c * 32, sv + c * 32);
-      tmem_wait_ld();
-      // Visible keys: the row's own segment, up to the row itself.
-      float m = -INFINITY;
-#pragma unroll
-      for (int c = 0; c < 128; ++c) {
-        const bool vis = c / S == seg && c <= r;
-        const float x = vis ? __uint_as_float(sv[c]) * sl2 : -INFINITY;
-        sv[c] = __float_as_uint(x);
-        m = fmaxf(m, x);
-      }
-      uint32_t packed[32];
-#pragma unroll
-      for (int half = 0; half < 2; ++half) {
-#pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          const float a = ex2_approx(__uint_as_float(sv[half * 64 + 2 * i]) - m);
-          const float c2 = ex2_approx(__uint_as_float(sv[half * 64 + 2 * i + 1]) - m);
-          l += a + c2;
-          packed[i] = pack_bf16x2(a, c2);
-        }
-        tmem_st32(tS + half * 64, packed);
-      }
-      tmem_wait_st();
-      tc_fence_before();
-      warp_arrive(p_ready);
-      // The retrieval row: sigma(q_r) in its segment's column block of the
-      // expanded operand, scaled by c_r; zeros in the other blocks.
+      // The retrieval row: sigma(q_r) (bf16) in its segment's column block
+      // of the expanded operand, zeros in the other blocks; den_r =
+      // sigma(q_r) . z_{s-1} in fp32 on the way.
       const float* z = zs + seg * D;
-      float den = 0.f;
 #pragma unroll 4
       for (int c8 = 0; c8 < D / 8; ++c8) {
         const uint4 v = *reinterpret_cast<const uint4*>(sQ + sw128_offset(r, c8 * 8, kBM));
         const uint32_t wv[4] = {v.x, v.y, v.z, v.w};
+        uint32_t ow[4];
 #pragma unroll
-        for (int i = 0; i < 4; ++i)
-          den = fmaf(elu1_fast(bf16hi_to_f32(wv[i])), z[c8 * 8 + 2 * i + 1],
-                     fmaf(elu1_fast(bf16lo_to_f32(wv[i])), z[c8 * 8 + 2 * i], den));
-      }
-      const float gm = gate_sigmoid(__ldg(beta + h));
-      float cr;
-      if (gm == 1.f)
-        cr = den != 0.f ? 1.f / den : 0.f;
-      else
-        cr = den != 0.f ? gm * l / ((1.f - gm) * den) : 0.f;
-#pragma unroll
-      for (int blk = 0; blk < SPT; ++blk) {
-#pragma unroll 4
-        for (int c8 = 0; c8 < D / 8; ++c8) {
-          uint4 o = make_uint4(0u, 0u, 0u, 0u);
-          if (blk == seg) {
-            const uint4 v = *reinterpret_cast<const uint4*>(sQ + sw128_offset(r, c8 * 8, kBM));
-            const uint32_t wv[4] = {v.x, v.y, v.z, v.w};
-            uint32_t ow[4];
-#pragma unroll
-            for (int i = 0; i < 4; ++i)
-              ow[i] = pack_bf16x2(elu1_fast(bf16lo_to_f32(wv[i])) * cr, elu1_fast(bf16hi_to_f32(wv[i])) * cr);
-            o = make_uint4(ow[0], ow[1], ow[2], ow[3]);
-          }
-          *reinterpret_cast<uint4*>(sA + sw128_offset(r, blk * D + c8 * 8, kBM)) = o;
+        for (int i = 0; i < 4; ++i) {
+          const float a = elu1_fast(bf16lo_to_f32(wv[i])), c = elu1_fast(bf16hi_to_f32(wv[i]));
+          den = fmaf(c, z[c8 * 8 + 2 * i + 1], fmaf(a, z[c8 * 8 + 2 * i], den));
+          ow[i] = pack_bf16x2(a, c);
         }
+#pragma unroll
+        for (int blk = 0; blk < SPT; ++blk)
+          *reinterpret_cast<uint4*>(sA + sw128_offset(r, blk * D + c8 * 8, kBM)) =
+              blk == seg ? make_uint4(ow[0], ow[1], ow[2], ow[3]) : make_uint4(0u, 0u, 0u, 0u);
       }
       fence_proxy_async();
       warp_arrive(a_ready);
-      ok = __all_sync(0xffffffffu, mbar_wait(o_full, 0, abort, status));
-      if (ok) {
-        tc_fence_after();
-        const float w = gm == 1.f ? 1.f : (1.f - gm) / l;
-        // Output row, staged as bf16 in the query tile (whose reads by the
-        // tensor core and by this thread are done).
+      ok = __all_sync(0xffffffffu, mbar_wait(s_full, 0, abort, status));
+    }
+    if (ok) {
+      tc_fence_after();
+      // Scores of the row's own segment block: keys [seg S, seg S + S),
+      // visible up to the row itself.
+      uint32_t sv[S];
 #pragma unroll
-        for (int c = 0; c < D; c += 32) {
-          uint32_t o_raw[32];
-          tmem_ld32(tO + c, o_raw);
-          tmem_wait_ld();
-          uint32_t wv[16];
-#pragma unroll
-          for (int i = 0; i < 16; ++i)
-            wv[i] = pack_bf16x2(__uint_as_float(o_raw[2 * i]) * w, __uint_as_float(o_raw[2 * i + 1]) * w);
-#pragma unroll
-          for (int e = 0; e < 4; ++e)
-            *reinterpret_cast<uint4*>(sQ + sw128_offset(r, c + e * 8, kBM)) =
-                make_uint4(wv[4 * e], wv[4 * e + 1], wv[4 * e + 2], wv[4 * e + 3]);
-        }
-        fence_proxy_async();
-        warp_arrive(staged);
+      for (int c = 0; c < S; c += 32) {
+        if (S - c >= 32) tmem_ld32(tS + seg * S + c, sv + c);
+        else tmem_ld16(tS + seg * S + c, sv + c);
       }
+      tmem_wait_ld();
+      const int rr = r - seg * S;  // row within the segment
+      float m = -INFINITY;
+#pragma unroll
+      for (int c = 0; c < S; ++c) {
+        const float x = c <= rr ? __uint_as_float(sv[c]) * sl2 : -INFINITY;
+        sv[c] = __float_as_uint(x);
+        m = fmaxf(m, x);
+      }
+      uint32_t pk[S / 2];
+#pragma unroll
+      for (int i = 0; i < S / 2; ++i) {
+        const float a = ex2_approx(__uint_as_float(sv[2 * i]) - m);
+        const float c2 = ex2_approx(__uint_as_float(sv[2 * i + 1]) - m);
+        l += a + c2;
+        pk[i] = pack_bf16x2(a, c2);
+      }
+      // P in TMEM: key k of the tile in packed column (k / 64) * 64 +
+      // (k % 64) / 2; each 32-column half holds 64 keys, here the row's block
+      // and zeros.
+#pragma unroll
+      for (int half = 0; half < 2; ++half) {
+        uint32_t w32[32];
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          // packed word i of this half holds keys 64 half + 2i, +1
+          const int key = 64 * half + 2 * i;
+          const int blk = key / S, j = (key % S) / 2;
+          w32[i] = blk == seg ? pk[j] : 0u;
+        }
+        tmem_st32(tS + half * 64, w32);
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      warp_arrive(p_ready);
+      ok = __all_sync(0xffffffffu, mbar_wait(o_full, 0, abort, status));
+    }
+    if (ok) {
+      tc_fence_after();
+      const float gm = gate_sigmoid(__ldg(beta + h));
+      // out = g / den R + (1 - g) / l O (the retrieval term 0 where den = 0)
+      const float wr = den != 0.f ? gm / den : 0.f;
+      const float wo = (1.f - gm) / l;
+      // Output row, staged as bf16 in the query tile (whose reads by the
+      // tensor core and by this thread are done).
+#pragma unroll
+      for (int c = 0; c < D; c += 32) {
+        uint32_t o_raw[32], r_raw[32];
+        tmem_ld32(tO + c, o_raw);
+        tmem_ld32(tR + c, r_raw);
+        tmem_wait_ld();
+        uint32_t wv[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i)
+          wv[i] = pack_bf16x2(fmaf(wr, __uint_as_float(r_raw[2 * i]), wo * __uint_as_float(o_raw[2 * i])),
+                              fmaf(wr, __uint_as_float(r_raw[2 * i + 1]), wo * __uint_as_float(o_raw[2 * i + 1])));
+#pragma unroll
+        for (int e = 0; e < 4; ++e)
+          *reinterpret_cast<uint4*>(sQ + sw128_offset(r, c + e * 8, kBM)) =
+              make_uint4(wv[4 * e], wv[4 * e + 1], wv[4 * e + 2], wv[4 * e + 3]);
+      }
+      fence_proxy_async();
+      warp_arrive(staged);
     }
   }
   tc_fence_before();
