@@ -1,6 +1,7 @@
 // Paired fp32 arithmetic (add / mul / fma .f32x2, sm_100) and the ELU+1 map
-// on bf16 pairs, for the state-scan kernels.  Each half of a paired
-// instruction rounds exactly like the scalar fp32 instruction.
+// on bf16 pairs (the state-scan kernels and the short-segment attention).
+// Each half of a paired instruction rounds exactly like the scalar fp32
+// instruction.
 #pragma once
 
 #include <cuda_bf16.h>

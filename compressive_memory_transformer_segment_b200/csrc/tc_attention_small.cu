@@ -31,6 +31,7 @@
 #include <cuda.h>
 
 #include "kernels.h"
+#include "packed_math.cuh"
 #include "tc_common.cuh"
 
 namespace infini {
@@ -242,9 +243,9 @@ tc_small_attention(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
         uint32_t ow[4];
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
-          const float a = elu1_fast(bf16lo_to_f32(wv[i])), c = elu1_fast(bf16hi_to_f32(wv[i]));
-          den = fmaf(c, z[c8 * 8 + 2 * i + 1], fmaf(a, z[c8 * 8 + 2 * i], den));
-          ow[i] = pack_bf16x2(a, c);
+          const float2 sg = pk::sigma_pair(wv[i]);
+          den = fmaf(sg.y, z[c8 * 8 + 2 * i + 1], fmaf(sg.x, z[c8 * 8 + 2 * i], den));
+          ow[i] = pack_bf16x2(sg.x, sg.y);
         }
 #pragma unroll
         for (int blk = 0; blk < SPT; ++blk)
