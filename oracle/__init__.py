@@ -14,6 +14,10 @@ library routine, a closed form, brute force or an invariant):
   elu_plus_one, gate_sigmoid, local_causal_attention, memory_retrieval,
   memory_update (linear and delta), infini_attention_forward, scan_states,
   segment_output.
+The backward (``infini_backward``: elu_plus_one_grad, the vector-Jacobian
+products of each step and infini_attention_backward) is pinned in
+``tests/test_oracle_backward.py`` against central finite differences of the
+forward and closed forms of special cases.
 No function here is "parity unpinned".
 """
 
@@ -27,4 +31,12 @@ from .infini_oracle import (  # noqa: F401
     scan_states,
     segment_output,
     infini_attention_forward,
+)
+from .infini_backward import (  # noqa: F401
+    elu_plus_one_grad,
+    local_causal_attention_vjp,
+    memory_retrieval_vjp,
+    memory_update_vjp,
+    segment_output_vjp,
+    infini_attention_backward,
 )
