@@ -81,6 +81,11 @@ _SIGNATURES = [
                                                    ctypes.c_int, ctypes.POINTER(Dims), _P, _P, _P,
                                                    _P]),
     ("infini_attn_noalloc_scratch_limit", ctypes.c_size_t, []),
+    ("infini_attn_backward_workspace_bytes", ctypes.c_size_t, [ctypes.POINTER(Dims), ctypes.c_int,
+                                                                ctypes.c_int]),
+    ("infini_attn_backward", ctypes.c_int, [_P, _P, _P, _P, _P, _P, ctypes.c_int, ctypes.c_int,
+                                            ctypes.POINTER(Dims), _P, _P, _P, _P, _P, _P, _P, _P,
+                                            _P, _P, ctypes.c_size_t, _P]),
 ]
 
 
@@ -222,6 +227,49 @@ def forward(q, k, v, beta, M_in, z_in, seg_len, rule, out=None, M_out=None, z_ou
         _check(lib.infini_attn_forward(*args, int(seg_len), _rule(rule), ctypes.byref(dims), *outs,
                                        ws_ptr, ws_n, _stream_handle(stream)))
     return out, M_out, z_out
+
+
+def backward_workspace_bytes(dims, seg_len, rule):
+    """infini_attn_backward_workspace_bytes (0 for unsupported shapes)."""
+    return load_library().infini_attn_backward_workspace_bytes(ctypes.byref(dims), int(seg_len),
+                                                               _rule(rule))
+
+
+def backward(q, k, v, beta, M_in, z_in, seg_len, rule, dout, dM_out=None, dz_out=None,
+             workspace=None, stream=None):
+    """infini_attn_backward on CUDA tensors: the gradients of a loss with
+    respect to the forward's inputs, given its gradients with respect to
+    (out, M_out, z_out) (``dM_out`` / ``dz_out`` may be None for zero).
+    Returns (dq, dk, dv, dbeta, dM_in, dz_in), all float32."""
+    lib = load_library()
+    dims = _dims_from(q, k, v)
+    B, H_q, L, H_kv, d_k, d_v = dims.B, dims.H_q, dims.L, dims.H_kv, dims.d_k, dims.d_v
+    f32 = dict(dtype=torch.float32, device=q.device)
+    dq = torch.empty((B, H_q, L, d_k), **f32)
+    dk = torch.empty((B, H_kv, L, d_k), **f32)
+    dv = torch.empty((B, H_kv, L, d_v), **f32)
+    dbeta = torch.empty((H_q,), **f32)
+    dM_in = torch.empty((B, H_kv, d_k, d_v), **f32)
+    dz_in = torch.empty((B, H_kv, d_k), **f32)
+    args = [_dev(q, "q"), _dev(k, "k"), _dev(v, "v"),
+            _dev(beta, "beta", torch.float32, (H_q,)),
+            _dev(M_in, "M_in", torch.float32, (B, H_kv, d_k, d_v)),
+            _dev(z_in, "z_in", torch.float32, (B, H_kv, d_k))]
+    grads_in = [_dev(dout, "dout", q.dtype, (B, H_q, L, d_v)),
+                _dev(dM_out, "dM_out", torch.float32, (B, H_kv, d_k, d_v))
+                if dM_out is not None else ctypes.c_void_p(0),
+                _dev(dz_out, "dz_out", torch.float32, (B, H_kv, d_k))
+                if dz_out is not None else ctypes.c_void_p(0)]
+    outs = [_dev(t, n) for t, n in ((dq, "dq"), (dk, "dk"), (dv, "dv"), (dbeta, "dbeta"),
+                                     (dM_in, "dM_in"), (dz_in, "dz_in"))]
+    if workspace is not None:
+        ws_ptr, ws_n = _dev(workspace, "workspace", torch.uint8), workspace.numel()
+    else:
+        ws_ptr, ws_n = ctypes.c_void_p(0), 0
+    with _one_device(q, k, v, beta, M_in, z_in, dout, dM_out, dz_out, workspace, stream=stream):
+        _check(lib.infini_attn_backward(*args, int(seg_len), _rule(rule), ctypes.byref(dims),
+                                        *grads_in, *outs, ws_ptr, ws_n, _stream_handle(stream)))
+    return dq, dk, dv, dbeta, dM_in, dz_in
 
 
 def state_update(k, v, M_in, z_in, seg_len, rule, M_out=None, z_out=None, workspace=None,

@@ -502,6 +502,119 @@ int infini_attn_decode_step(const void* q_t, const void* k_t, const void* v_t, c
   return e == cudaSuccess ? INFINI_OK : INFINI_ERR_CUDA;
 }
 
+namespace {
+
+// Backward workspace: the forward's fp32 states (slot s = M_{s-1}, z_{s-1}),
+// a scratch M_T / z_T, and the per-query-head partials.
+struct BwdLayout {
+  size_t zf, Mf, Mscr, zscr, dKa, dVa, dMr, dzr, dbp, total;
+};
+
+int backward_layout(const infini_dims_t* dims, int seg_len, int rule, Shape* s, BwdLayout* lay) {
+  int rc = check_shape(dims, seg_len, rule, s);
+  if (rc != INFINI_OK) return rc;
+  if (!backward_supported(s->d_k, s->d_v, seg_len)) return INFINI_ERR_UNSUPPORTED;
+  const size_t d = s->d_k, T = s->T, L = s->L;
+  const size_t BHq = (size_t)s->B * s->H_q, BHkv = (size_t)s->B * s->H_kv;
+  lay->zf = kHeader;
+  lay->Mf = align_up(lay->zf + T * BHkv * d * 4);
+  lay->Mscr = align_up(lay->Mf + T * BHkv * d * d * 4);
+  lay->zscr = align_up(lay->Mscr + BHkv * d * d * 4);
+  lay->dKa = align_up(lay->zscr + BHkv * d * 4);
+  lay->dVa = align_up(lay->dKa + BHq * L * d * 4);
+  lay->dMr = align_up(lay->dVa + BHq * L * d * 4);
+  lay->dzr = align_up(lay->dMr + T * BHq * d * d * 4);
+  lay->dbp = align_up(lay->dzr + T * BHq * d * 4);
+  lay->total = align_up(lay->dbp + BHq * T * 4);
+  return INFINI_OK;
+}
+
+}  // namespace
+
+size_t infini_attn_backward_workspace_bytes(const infini_dims_t* dims, int seg_len, int rule) {
+  Shape s;
+  BwdLayout lay;
+  return backward_layout(dims, seg_len, rule, &s, &lay) == INFINI_OK ? lay.total : 0;
+}
+
+int infini_attn_backward(const void* q, const void* k, const void* v, const float* beta,
+                         const float* M_in, const float* z_in, int seg_len, int rule,
+                         const infini_dims_t* dims, const void* dout, const float* dM_out,
+                         const float* dz_out, float* dq, float* dk, float* dv, float* dbeta,
+                         float* dM_in, float* dz_in, void* workspace, size_t workspace_bytes,
+                         void* stream) {
+  Shape s;
+  BwdLayout lay;
+  int rc = backward_layout(dims, seg_len, rule, &s, &lay);
+  if (rc != INFINI_OK) return rc;
+  if (!q || !k || !v || !beta || !M_in || !z_in || !dout || !dq || !dk || !dv || !dbeta || !dM_in ||
+      !dz_in)
+    return INFINI_ERR_ARG;
+  const void* ptrs[] = {q, k, v, beta, M_in, z_in, dout, dM_out, dz_out, dq, dk, dv, dbeta, dM_in, dz_in};
+  for (const void* p : ptrs)
+    if (p && !aligned16(p)) return INFINI_ERR_ALIGN;
+  if (workspace == nullptr && workspace_bytes != 0) return INFINI_ERR_ARG;
+  if (workspace && (workspace_bytes < lay.total || ((uintptr_t)workspace & (kAlign - 1)) != 0))
+    return INFINI_ERR_WORKSPACE;
+  const size_t dq_bytes = (size_t)s.B * s.H_q * s.L * s.d_k * 4;
+  const size_t dkv_bytes = (size_t)s.B * s.H_kv * s.L * s.d_k * 4;
+  const Range outs[] = {rng(dq, dq_bytes), rng(dk, dkv_bytes), rng(dv, dkv_bytes),
+                        rng(dbeta, s.beta_bytes), rng(dM_in, s.M_bytes), rng(dz_in, s.z_bytes)};
+  const Range ins[] = {rng(q, s.q_bytes), rng(k, s.k_bytes), rng(v, s.v_bytes),
+                       rng(beta, s.beta_bytes), rng(M_in, s.M_bytes), rng(z_in, s.z_bytes),
+                       rng(dout, s.out_bytes), rng(dM_out, dM_out ? s.M_bytes : 0),
+                       rng(dz_out, dz_out ? s.z_bytes : 0)};
+  for (int i = 0; i < 6; ++i) {
+    for (int j = i + 1; j < 6; ++j)
+      if (overlap(outs[i], outs[j])) return INFINI_ERR_ALIAS;
+    for (const Range& r : ins)
+      if (overlap(outs[i], r)) return INFINI_ERR_ALIAS;
+    if (workspace && overlap(outs[i], rng(workspace, lay.total))) return INFINI_ERR_ALIAS;
+  }
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  unsigned int* status = status_ptr();
+  if (!status) return INFINI_ERR_CUDA;
+  char* ws = static_cast<char*>(workspace);
+  bool owned = false;
+  if (!ws) {
+    if (cudaMallocAsync(reinterpret_cast<void**>(&ws), lay.total, st) != cudaSuccess) return INFINI_ERR_CUDA;
+    owned = true;
+  }
+  // The forward's states M_{s-1}, z_{s-1} in fp32: the fp32 state scan, run again.
+  Problem p;
+  p.q = q; p.k = k; p.v = v; p.beta = beta; p.M_in = M_in; p.z_in = z_in;
+  p.out = nullptr;
+  p.M_out = reinterpret_cast<float*>(ws + lay.Mscr);
+  p.z_out = reinterpret_cast<float*>(ws + lay.zscr);
+  p.B = s.B; p.H_q = s.H_q; p.H_kv = s.H_kv; p.L = s.L; p.d_k = s.d_k; p.d_v = s.d_v;
+  p.S = s.S; p.T = s.T; p.bf16 = s.bf16; p.delta = s.delta;
+  p.z_pref = reinterpret_cast<float*>(ws + lay.zf);
+  p.M_pref = ws + lay.Mf;
+  p.M_pref_bf16 = false;
+  p.Gbuf = p.Bbuf = p.dz = nullptr;
+  p.status = status;
+  cudaError_t e = cudaMemcpyAsync(p.z_pref, z_in, s.z_bytes, cudaMemcpyDeviceToDevice, st);
+  if (e == cudaSuccess) e = timed(0, st, [&] { return launch_simt_state_scan(p, st); });
+  BackwardProblem bp;
+  bp.q = q; bp.k = k; bp.v = v; bp.beta = beta; bp.dout = dout; bp.dM_out = dM_out; bp.dz_out = dz_out;
+  bp.dq = dq; bp.dk = dk; bp.dv = dv; bp.dbeta = dbeta; bp.dM_in = dM_in; bp.dz_in = dz_in;
+  bp.Mf = reinterpret_cast<const float*>(ws + lay.Mf);
+  bp.zf = reinterpret_cast<const float*>(ws + lay.zf);
+  bp.dKa = reinterpret_cast<float*>(ws + lay.dKa);
+  bp.dVa = reinterpret_cast<float*>(ws + lay.dVa);
+  bp.dMr = reinterpret_cast<float*>(ws + lay.dMr);
+  bp.dzr = reinterpret_cast<float*>(ws + lay.dzr);
+  bp.dbp = reinterpret_cast<float*>(ws + lay.dbp);
+  bp.B = s.B; bp.H_q = s.H_q; bp.H_kv = s.H_kv; bp.L = s.L; bp.d = s.d_k; bp.S = s.S; bp.T = s.T;
+  bp.bf16 = s.bf16; bp.delta = s.delta;
+  if (e == cudaSuccess) e = timed(1, st, [&] { return launch_backward(bp, st); });
+  if (owned) {
+    cudaError_t f = cudaFreeAsync(ws, st);
+    if (e == cudaSuccess) e = f;
+  }
+  return e == cudaSuccess ? INFINI_OK : INFINI_ERR_CUDA;
+}
+
 size_t infini_attn_host_arena_bytes(const infini_dims_t* dims, int seg_len, int rule) {
   Shape s;
   if (check_shape(dims, seg_len, rule, &s) != INFINI_OK) return 0;

@@ -1,0 +1,453 @@
+// Backward of the Infini-attention forward (back-propagation through the
+// segments), fp32 CUDA-core kernels for short segments (S <= 64, the pages'
+// training rollout is 16 segments of 64: "Hugging Face Infini-Attention
+// 再現分析", "重み減衰とロールアウト"; BPTT through the memory: "Leave No
+// Context Behind" explainer, "限界").
+//
+// Given the gradients of a loss with respect to out, M_out and z_out, the
+// chain rule through the forward's steps (see the forward kernels) gives the
+// gradients with respect to q, k, v, beta, M_in and z_in:
+//   bwd_segment (per segment and query head): recomputes sigma(Q), the
+//     retrieval and the softmax, then
+//       dA_mem = g dout, dA_dot = (1 - g) dout, dbeta += sum(dout (A_mem -
+//       A_dot)) g (1 - g);
+//       retrieval: dnum = dA_mem / den, dden = -rowsum(dA_mem A_mem) / den
+//       (rows with den = 0 carry nothing), d sigma(Q) = dnum M^T + dden z^T,
+//       dM_{s-1} += sigma(Q)^T dnum, dz_{s-1} += sigma(Q)^T dden;
+//       attention: dV = P^T dA_dot, dP = dA_dot V^T, dS = P (dP - rowsum(dP P)),
+//       dQ = dS K / sqrt(d) + d sigma(Q) sigma'(Q), dK = dS^T Q / sqrt(d);
+//     writes dq, and per query head the attention's dK, dV and the
+//     retrieval's dM_{s-1}, dz_{s-1} to the workspace.
+//   bwd_scan (per KV head, segments in reverse): carries G_M = dL/dM_s and
+//     G_z = dL/dz_s from (dM_out, dz_out); per segment the update's VJP
+//       linear: d sigma(K) = V G_M^T + G_z, dV = sigma(K) G_M;
+//       delta:  r = sigma(K) z, R = sigma(K) M / r, U = V - R,
+//               dU = sigma(K) G_M, dV = dU, dN = -dU / r,
+//               dr = rowsum(dU R) / r, d sigma(K) = U G_M^T + dN M^T +
+//               dr z^T + G_z, G_M += sigma(K)^T dN, G_z += sigma(K)^T dr
+//       (rows with r = 0 carry no retrieval term),
+//     then adds the query heads' dM_{s-1}, dz_{s-1}; writes dk = d sigma(K)
+//     sigma'(K) + the heads' attention dK, dv likewise, and finally dM_in,
+//     dz_in.
+//   bwd_dbeta: the per-(segment, head) gate partials summed in a fixed order.
+// (M_{s-1}, z_{s-1}) come from the forward's fp32 state scan, run again.
+// Every sum runs in a fixed order: the results are bitwise reproducible.
+#include "common.cuh"
+#include "kernels.h"
+
+namespace infini {
+
+namespace {
+
+constexpr int kBwdThreads = 256;
+constexpr int kBwdMaxS = 64;
+
+__device__ __forceinline__ float elu1_grad(float x) { return x > 0.f ? 1.f : expf(x); }
+
+// Shared-memory plan of bwd_segment (floats): n x D tiles with row stride
+// D + 1 (rows and columns are both read across lanes without conflicts),
+// n x n tiles with stride kBwdMaxS + 1.
+template <int D>
+struct SegSmem {
+  static constexpr int kLd = D + 1;
+  static constexpr int kLp = kBwdMaxS + 1;
+  static constexpr int kTile = kBwdMaxS * kLd;
+  static constexpr int kQ = 0, kK = kQ + kTile, kV = kK + kTile, kDO = kV + kTile;
+  static constexpr int kM = kDO + kTile;            // [D][D + 1]
+  static constexpr int kX = kM + D * kLd;           // sigma(Q)
+  static constexpr int kAm = kX + kTile;            // A_mem, then dQ
+  static constexpr int kY = kAm + kTile;            // A_dot, then dnum
+  static constexpr int kP = kY + kTile;             // [n][n] softmax
+  static constexpr int kDS = kP + kBwdMaxS * kLp;   // [n][n] dP, then dS
+  static constexpr int kZ = kDS + kBwdMaxS * kLp;   // z_{s-1}
+  static constexpr int kDen = kZ + D;
+  static constexpr int kDden = kDen + kBwdMaxS;
+  static constexpr int kRs = kDden + kBwdMaxS;
+  static constexpr int kRed = kRs + kBwdMaxS;       // block reduction
+  static constexpr int kTotal = kRed + kBwdThreads / 32;
+};
+
+template <typename T, int D>
+__global__ void __launch_bounds__(kBwdThreads)
+bwd_segment(const T* __restrict__ q, const T* __restrict__ k, const T* __restrict__ v,
+            const float* __restrict__ beta, const T* __restrict__ dout,
+            const float* __restrict__ Mf, const float* __restrict__ zf,
+            float* __restrict__ dq, float* __restrict__ dKa, float* __restrict__ dVa,
+            float* __restrict__ dMr, float* __restrict__ dzr, float* __restrict__ dbp,
+            int H_q, int H_kv, int L, int S, int T_seg) {
+  using SM = SegSmem<D>;
+  constexpr int ld = SM::kLd, lp = SM::kLp;
+  extern __shared__ float sm[];
+  float *Q = sm + SM::kQ, *K = sm + SM::kK, *V = sm + SM::kV, *dO = sm + SM::kDO;
+  float *M = sm + SM::kM, *X = sm + SM::kX, *Am = sm + SM::kAm, *Y = sm + SM::kY;
+  float *P = sm + SM::kP, *dS = sm + SM::kDS, *z = sm + SM::kZ, *den = sm + SM::kDen;
+  float *dden = sm + SM::kDden, *rs = sm + SM::kRs, *red = sm + SM::kRed;
+  const int s = blockIdx.x, bh = blockIdx.y;  // bh = b * H_q + h
+  const int h = bh % H_q, b = bh / H_q;
+  const int bhkv = b * H_kv + h / (H_q / H_kv);
+  const int BHq = gridDim.y, BHkv = BHq / H_q * H_kv;
+  const int r0 = s * S, n = min(S, L - r0);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const float scale = rsqrtf((float)D);
+  const float g = gate_sigmoid(beta[h]);
+
+  // ---- loads (rows past the segment stay out of every sum: loops run to n)
+  const T* qs = q + ((size_t)bh * L + r0) * D;
+  const T* ks = k + ((size_t)bhkv * L + r0) * D;
+  const T* vs = v + ((size_t)bhkv * L + r0) * D;
+  const T* ds = dout + ((size_t)bh * L + r0) * D;
+  for (int e = tid; e < n * D; e += kBwdThreads) {
+    const int i = e / D, c = e % D;
+    Q[i * ld + c] = to_f32(qs[e]);
+    K[i * ld + c] = to_f32(ks[e]);
+    V[i * ld + c] = to_f32(vs[e]);
+    dO[i * ld + c] = to_f32(ds[e]);
+  }
+  const float* Ms = Mf + ((size_t)s * BHkv + bhkv) * D * D;
+  for (int e = tid; e < D * D; e += kBwdThreads) M[(e / D) * ld + e % D] = Ms[e];
+  for (int c = tid; c < D; c += kBwdThreads) z[c] = zf[((size_t)s * BHkv + bhkv) * D + c];
+  __syncthreads();
+  for (int e = tid; e < n * D; e += kBwdThreads) {
+    const int i = e / D, c = e % D;
+    X[i * ld + c] = elu1(Q[i * ld + c]);
+  }
+  __syncthreads();
+  // den_i = sigma(q_i) . z
+  for (int i = warp; i < n; i += kBwdThreads / 32) {
+    float a = 0.f;
+    for (int c = lane; c < D; c += 32) a = fmaf(X[i * ld + c], z[c], a);
+    a = warp_sum(a);
+    if (lane == 0) den[i] = a;
+  }
+  // scores, masked (key j <= row i)
+  for (int e = tid; e < n * n; e += kBwdThreads) {
+    const int i = e / n, j = e % n;
+    float a = 0.f;
+    for (int c = 0; c < D; ++c) a = fmaf(Q[i * ld + c], K[j * ld + c], a);
+    P[i * lp + j] = j <= i ? a * scale : -INFINITY;
+  }
+  __syncthreads();
+  // A_mem = sigma(Q) M / den (0 where den = 0); row softmax of the scores
+  for (int e = tid; e < n * D; e += kBwdThreads) {
+    const int i = e / D, c = e % D;
+    float a = 0.f;
+    for (int kk = 0; kk < D; ++kk) a = fmaf(X[i * ld + kk], M[kk * ld + c], a);
+    Am[i * ld + c] = den[i] != 0.f ? a / den[i] : 0.f;
+  }
+  for (int i = warp; i < n; i += kBwdThreads / 32) {
+    float m = -INFINITY;
+    for (int j = lane; j < n; j += 32) m = fmaxf(m, P[i * lp + j]);
+    m = warp_max(m);
+    float l = 0.f;
+    for (int j = lane; j < n; j += 32) {
+      const float p = expf(P[i * lp + j] - m);
+      P[i * lp + j] = p;
+      l += p;
+    }
+    l = warp_sum(l);
+    const float inv = 1.f / l;
+    for (int j = lane; j < n; j += 32) P[i * lp + j] *= inv;
+  }
+  __syncthreads();
+  // A_dot = P V, and the gate's partial sum(dout (A_mem - A_dot))
+  float part = 0.f;
+  for (int e = tid; e < n * D; e += kBwdThreads) {
+    const int i = e / D, c = e % D;
+    float a = 0.f;
+    for (int j = 0; j <= i; ++j) a = fmaf(P[i * lp + j], V[j * ld + c], a);
+    part = fmaf(dO[i * ld + c], Am[i * ld + c] - a, part);
+  }
+  part = warp_sum(part);
+  if (lane == 0) red[warp] = part;
+  // dden_i = -sum_c g dout A_mem / den
+  for (int i = warp; i < n; i += kBwdThreads / 32) {
+    float a = 0.f;
+    for (int c = lane; c < D; c += 32) a = fmaf(dO[i * ld + c], Am[i * ld + c], a);
+    a = warp_sum(a);
+    if (lane == 0) dden[i] = den[i] != 0.f ? -g * a / den[i] : 0.f;
+  }
+  // dnum = g dout / den
+  for (int e = tid; e < n * D; e += kBwdThreads) {
+    const int i = e / D, c = e % D;
+    Y[i * ld + c] = den[i] != 0.f ? g * dO[i * ld + c] / den[i] : 0.f;
+  }
+  __syncthreads();
+  if (tid == 0) {
+    float a = 0.f;
+    for (int w = 0; w < kBwdThreads / 32; ++w) a += red[w];
+    dbp[(size_t)bh * T_seg + s] = a * g * (1.f - g);
+  }
+  // Retrieval: dM_{s-1} += sigma(Q)^T dnum, dz_{s-1} += sigma(Q)^T dden
+  float* dMo = dMr + ((size_t)s * BHq + bh) * D * D;
+  for (int e = tid; e < D * D; e += kBwdThreads) {
+    const int kk = e / D, c = e % D;
+    float a = 0.f;
+    for (int i = 0; i < n; ++i) a = fmaf(X[i * ld + kk], Y[i * ld + c], a);
+    dMo[e] = a;
+  }
+  for (int kk = tid; kk < D; kk += kBwdThreads) {
+    float a = 0.f;
+    for (int i = 0; i < n; ++i) a = fmaf(X[i * ld + kk], dden[i], a);
+    dzr[((size_t)s * BHq + bh) * D + kk] = a;
+  }
+  // dQ (retrieval part) = (dnum M^T + dden z^T) sigma'(Q), into Am
+  for (int e = tid; e < n * D; e += kBwdThreads) {
+    const int i = e / D, kk = e % D;
+    float a = dden[i] * z[kk];
+    for (int c = 0; c < D; ++c) a = fmaf(Y[i * ld + c], M[kk * ld + c], a);
+    Am[i * ld + kk] = a * elu1_grad(Q[i * ld + kk]);
+  }
+  // Attention: dP = (1 - g) dout V^T (causal part only)
+  const float ga = 1.f - g;
+  for (int e = tid; e < n * n; e += kBwdThreads) {
+    const int i = e / n, j = e % n;
+    float a = 0.f;
+    if (j <= i)
+      for (int c = 0; c < D; ++c) a = fmaf(dO[i * ld + c], V[j * ld + c], a);
+    dS[i * lp + j] = ga * a;
+  }
+  // dV (attention) = P^T dA_dot
+  float* dVo = dVa + ((size_t)bh * L + r0) * D;
+  for (int e = tid; e < n * D; e += kBwdThreads) {
+    const int j = e / D, c = e % D;
+    float a = 0.f;
+    for (int i = j; i < n; ++i) a = fmaf(P[i * lp + j], dO[i * ld + c], a);
+    dVo[e] = ga * a;
+  }
+  __syncthreads();
+  // dS = P (dP - rowsum(dP P))
+  for (int i = warp; i < n; i += kBwdThreads / 32) {
+    float a = 0.f;
+    for (int j = lane; j <= i; j += 32) a = fmaf(dS[i * lp + j], P[i * lp + j], a);
+    a = warp_sum(a);
+    if (lane == 0) rs[i] = a;
+  }
+  __syncthreads();
+  for (int e = tid; e < n * n; e += kBwdThreads) {
+    const int i = e / n, j = e % n;
+    dS[i * lp + j] = j <= i ? P[i * lp + j] * (dS[i * lp + j] - rs[i]) : 0.f;
+  }
+  __syncthreads();
+  // dq = dS K / sqrt(d) + retrieval part; dK (attention) = dS^T Q / sqrt(d)
+  float* dqo = dq + ((size_t)bh * L + r0) * D;
+  float* dKo = dKa + ((size_t)bh * L + r0) * D;
+  for (int e = tid; e < n * D; e += kBwdThreads) {
+    const int i = e / D, c = e % D;
+    float a = 0.f;
+    for (int j = 0; j <= i; ++j) a = fmaf(dS[i * lp + j], K[j * ld + c], a);
+    dqo[e] = fmaf(a, scale, Am[i * ld + c]);
+    float bk = 0.f;
+    for (int r = i; r < n; ++r) bk = fmaf(dS[r * lp + i], Q[r * ld + c], bk);
+    dKo[e] = bk * scale;
+  }
+}
+
+// Shared-memory plan of bwd_scan (floats).
+template <int D>
+struct ScanBwdSmem {
+  static constexpr int kLd = D + 1;
+  static constexpr int kTile = kBwdMaxS * kLd;
+  static constexpr int kGM = 0;                    // [D][D + 1] dL/dM_s
+  static constexpr int kM = kGM + D * kLd;         // M_{s-1}
+  static constexpr int kSK = kM + D * kLd;         // sigma(K)
+  static constexpr int kV = kSK + kTile;
+  static constexpr int kX1 = kV + kTile;           // d sigma(K)
+  static constexpr int kX2 = kX1 + kTile;          // dV (= dU, delta)
+  static constexpr int kX3 = kX2 + kTile;          // R (delta)
+  static constexpr int kGz = kX3 + kTile;
+  static constexpr int kZ = kGz + D;
+  static constexpr int kR = kZ + D;                // r_t (delta)
+  static constexpr int kDr = kR + kBwdMaxS;        // dr_t (delta)
+  static constexpr int kTotal = kDr + kBwdMaxS;
+};
+
+template <typename T, int D, bool DELTA>
+__global__ void __launch_bounds__(kBwdThreads)
+bwd_scan(const T* __restrict__ k, const T* __restrict__ v, const float* __restrict__ Mf,
+         const float* __restrict__ zf, const float* __restrict__ dM_out,
+         const float* __restrict__ dz_out, const float* __restrict__ dKa,
+         const float* __restrict__ dVa, const float* __restrict__ dMr,
+         const float* __restrict__ dzr, float* __restrict__ dk, float* __restrict__ dv,
+         float* __restrict__ dM_in, float* __restrict__ dz_in, int H_q, int H_kv, int L, int S,
+         int T_seg) {
+  using SM = ScanBwdSmem<D>;
+  constexpr int ld = SM::kLd;
+  extern __shared__ float sm[];
+  float *GM = sm + SM::kGM, *M = sm + SM::kM, *sK = sm + SM::kSK, *V = sm + SM::kV;
+  float *X1 = sm + SM::kX1, *X2 = sm + SM::kX2, *X3 = sm + SM::kX3;
+  float *Gz = sm + SM::kGz, *z = sm + SM::kZ, *r = sm + SM::kR, *dr = sm + SM::kDr;
+  const int bhkv = blockIdx.x, BHkv = gridDim.x;
+  const int b = bhkv / H_kv, j = bhkv % H_kv, grp = H_q / H_kv;
+  const int BHq = BHkv / H_kv * H_q;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  for (int e = tid; e < D * D; e += kBwdThreads)
+    GM[(e / D) * ld + e % D] = dM_out ? dM_out[(size_t)bhkv * D * D + e] : 0.f;
+  for (int c = tid; c < D; c += kBwdThreads) Gz[c] = dz_out ? dz_out[(size_t)bhkv * D + c] : 0.f;
+  for (int s = T_seg - 1; s >= 0; --s) {
+    const int r0 = s * S, n = min(S, L - r0);
+    const T* ks = k + ((size_t)bhkv * L + r0) * D;
+    const T* vs = v + ((size_t)bhkv * L + r0) * D;
+    for (int e = tid; e < n * D; e += kBwdThreads) {
+      const int i = e / D, c = e % D;
+      sK[i * ld + c] = elu1(to_f32(ks[e]));
+      V[i * ld + c] = to_f32(vs[e]);
+    }
+    if (DELTA) {
+      const float* Ms = Mf + ((size_t)s * BHkv + bhkv) * D * D;
+      for (int e = tid; e < D * D; e += kBwdThreads) M[(e / D) * ld + e % D] = Ms[e];
+      for (int c = tid; c < D; c += kBwdThreads) z[c] = zf[((size_t)s * BHkv + bhkv) * D + c];
+    }
+    __syncthreads();
+    if (DELTA) {
+      // r_t = sigma(k_t) . z_{s-1}
+      for (int i = warp; i < n; i += kBwdThreads / 32) {
+        float a = 0.f;
+        for (int c = lane; c < D; c += 32) a = fmaf(sK[i * ld + c], z[c], a);
+        a = warp_sum(a);
+        if (lane == 0) r[i] = a;
+      }
+      __syncthreads();
+      // R = sigma(K) M / r (0 where r = 0); dU = sigma(K) G_M
+      for (int e = tid; e < n * D; e += kBwdThreads) {
+        const int i = e / D, c = e % D;
+        float a = 0.f, u = 0.f;
+        for (int kk = 0; kk < D; ++kk) {
+          a = fmaf(sK[i * ld + kk], M[kk * ld + c], a);
+          u = fmaf(sK[i * ld + kk], GM[kk * ld + c], u);
+        }
+        X3[i * ld + c] = r[i] != 0.f ? a / r[i] : 0.f;
+        X2[i * ld + c] = u;
+      }
+      __syncthreads();
+      // dr_t = rowsum(dU R) / r
+      for (int i = warp; i < n; i += kBwdThreads / 32) {
+        float a = 0.f;
+        for (int c = lane; c < D; c += 32) a = fmaf(X2[i * ld + c], X3[i * ld + c], a);
+        a = warp_sum(a);
+        if (lane == 0) dr[i] = r[i] != 0.f ? a / r[i] : 0.f;
+      }
+      __syncthreads();
+      // d sigma(K) = (V - R) G_M^T + dN M^T + dr z^T + G_z, dN = -dU / r
+      for (int e = tid; e < n * D; e += kBwdThreads) {
+        const int i = e / D, kk = e % D;
+        const float ir = r[i] != 0.f ? -1.f / r[i] : 0.f;
+        float a = fmaf(dr[i], z[kk], Gz[kk]);
+        for (int c = 0; c < D; ++c) {
+          a = fmaf(V[i * ld + c] - X3[i * ld + c], GM[kk * ld + c], a);
+          a = fmaf(X2[i * ld + c] * ir, M[kk * ld + c], a);
+        }
+        X1[i * ld + kk] = a;
+      }
+      __syncthreads();
+      // G_M += sigma(K)^T dN, G_z += sigma(K)^T dr
+      for (int e = tid; e < D * D; e += kBwdThreads) {
+        const int kk = e / D, c = e % D;
+        float a = 0.f;
+        for (int i = 0; i < n; ++i) {
+          const float ir = r[i] != 0.f ? -1.f / r[i] : 0.f;
+          a = fmaf(sK[i * ld + kk], X2[i * ld + c] * ir, a);
+        }
+        GM[kk * ld + c] += a;
+      }
+      for (int kk = tid; kk < D; kk += kBwdThreads) {
+        float a = 0.f;
+        for (int i = 0; i < n; ++i) a = fmaf(sK[i * ld + kk], dr[i], a);
+        Gz[kk] += a;
+      }
+    } else {
+      // d sigma(K) = V G_M^T + G_z, dV = sigma(K) G_M
+      for (int e = tid; e < n * D; e += kBwdThreads) {
+        const int i = e / D, c = e % D;
+        float a = Gz[c], u = 0.f;
+        for (int kk = 0; kk < D; ++kk) {
+          a = fmaf(V[i * ld + kk], GM[c * ld + kk], a);
+          u = fmaf(sK[i * ld + kk], GM[kk * ld + c], u);
+        }
+        X1[i * ld + c] = a;
+        X2[i * ld + c] = u;
+      }
+    }
+    __syncthreads();
+    // dk, dv of the segment: the update's part plus every query head's attention part.
+    for (int e = tid; e < n * D; e += kBwdThreads) {
+      const int i = e / D, c = e % D;
+      const float sk = sK[i * ld + c];
+      float a = X1[i * ld + c] * (sk > 1.f ? 1.f : sk);  // sigma'(k) = 1 or e^k = sigma(k)
+      float u = X2[i * ld + c];
+      for (int hh = 0; hh < grp; ++hh) {
+        const size_t row = ((size_t)(b * H_q + j * grp + hh) * L + r0 + i) * D + c;
+        a += dKa[row];
+        u += dVa[row];
+      }
+      const size_t o = ((size_t)bhkv * L + r0 + i) * D + c;
+      dk[o] = a;
+      dv[o] = u;
+    }
+    // The query heads' retrieval gradients with respect to (M_{s-1}, z_{s-1}).
+    for (int e = tid; e < D * D; e += kBwdThreads) {
+      float a = 0.f;
+      for (int hh = 0; hh < grp; ++hh)
+        a += dMr[((size_t)s * BHq + b * H_q + j * grp + hh) * D * D + e];
+      GM[(e / D) * ld + e % D] += a;
+    }
+    for (int c = tid; c < D; c += kBwdThreads) {
+      float a = 0.f;
+      for (int hh = 0; hh < grp; ++hh) a += dzr[((size_t)s * BHq + b * H_q + j * grp + hh) * D + c];
+      Gz[c] += a;
+    }
+    __syncthreads();
+  }
+  for (int e = tid; e < D * D; e += kBwdThreads)
+    dM_in[(size_t)bhkv * D * D + e] = GM[(e / D) * ld + e % D];
+  for (int c = tid; c < D; c += kBwdThreads) dz_in[(size_t)bhkv * D + c] = Gz[c];
+}
+
+// dbeta[h] = sum over batch rows and segments of the partials, in order.
+__global__ void __launch_bounds__(kBwdThreads)
+bwd_dbeta(const float* __restrict__ dbp, float* __restrict__ dbeta, int B, int H_q, int T_seg) {
+  for (int h = threadIdx.x; h < H_q; h += blockDim.x) {
+    float a = 0.f;
+    for (int b = 0; b < B; ++b)
+      for (int s = 0; s < T_seg; ++s) a += dbp[((size_t)b * H_q + h) * T_seg + s];
+    dbeta[h] = a;
+  }
+}
+
+template <typename T, int D>
+cudaError_t launch_bwd(const BackwardProblem& p, cudaStream_t st) {
+  const int BHq = p.B * p.H_q, BHkv = p.B * p.H_kv;
+  const size_t seg_smem = SegSmem<D>::kTotal * sizeof(float);
+  cudaError_t e = cudaFuncSetAttribute(bwd_segment<T, D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)seg_smem);
+  if (e != cudaSuccess) return e;
+  bwd_segment<T, D><<<dim3(p.T, BHq), kBwdThreads, seg_smem, st>>>(
+      static_cast<const T*>(p.q), static_cast<const T*>(p.k), static_cast<const T*>(p.v), p.beta,
+      static_cast<const T*>(p.dout), p.Mf, p.zf, p.dq, p.dKa, p.dVa, p.dMr, p.dzr, p.dbp, p.H_q,
+      p.H_kv, p.L, p.S, p.T);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  const size_t scan_smem = ScanBwdSmem<D>::kTotal * sizeof(float);
+  auto scan = p.delta ? bwd_scan<T, D, true> : bwd_scan<T, D, false>;
+  if ((e = cudaFuncSetAttribute(scan, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)scan_smem)) !=
+      cudaSuccess)
+    return e;
+  scan<<<BHkv, kBwdThreads, scan_smem, st>>>(
+      static_cast<const T*>(p.k), static_cast<const T*>(p.v), p.Mf, p.zf, p.dM_out, p.dz_out, p.dKa,
+      p.dVa, p.dMr, p.dzr, p.dk, p.dv, p.dM_in, p.dz_in, p.H_q, p.H_kv, p.L, p.S, p.T);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  bwd_dbeta<<<1, kBwdThreads, 0, st>>>(p.dbp, p.dbeta, p.B, p.H_q, p.T);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+bool backward_supported(int d_k, int d_v, int S) {
+  return d_k == d_v && (d_k == 32 || d_k == 64) && S >= 1 && S <= kBwdMaxS;
+}
+
+cudaError_t launch_backward(const BackwardProblem& p, cudaStream_t stream) {
+  if (p.d == 32) return p.bf16 ? launch_bwd<__nv_bfloat16, 32>(p, stream) : launch_bwd<float, 32>(p, stream);
+  if (p.d == 64) return p.bf16 ? launch_bwd<__nv_bfloat16, 64>(p, stream) : launch_bwd<float, 64>(p, stream);
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace infini

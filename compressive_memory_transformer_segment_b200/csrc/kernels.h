@@ -79,6 +79,38 @@ struct DecodeProblem {
   int B, H_q, H_kv, d, S, pos, nsplit;
   bool bf16;
 };
+// Backward through the segments (fp32 CUDA cores; S <= 64, d_k == d_v in
+// {32, 64}).  Mf / zf hold the forward's per-segment states M_{s-1}, z_{s-1}
+// in fp32 (from the SIMT state scan); the rest of the workspace holds the
+// per-query-head partials that the reverse scan sums in a fixed order.
+struct BackwardProblem {
+  const void* q;
+  const void* k;
+  const void* v;
+  const float* beta;
+  const void* dout;     // [B, H_q, L, d] in the I/O dtype
+  const float* dM_out;  // [B, H_kv, d, d] or NULL (zero)
+  const float* dz_out;  // [B, H_kv, d] or NULL (zero)
+  float* dq;            // [B, H_q, L, d]
+  float* dk;            // [B, H_kv, L, d]
+  float* dv;            // [B, H_kv, L, d]
+  float* dbeta;         // [H_q]
+  float* dM_in;         // [B, H_kv, d, d]
+  float* dz_in;         // [B, H_kv, d]
+  // workspace
+  const float* Mf;      // [T][B*H_kv][d][d]
+  const float* zf;      // [T][B*H_kv][d]
+  float* dKa;           // [B*H_q][L][d]  attention's dK per query head
+  float* dVa;           // [B*H_q][L][d]  attention's dV per query head
+  float* dMr;           // [T][B*H_q][d][d]  retrieval's dM_{s-1} per query head
+  float* dzr;           // [T][B*H_q][d]
+  float* dbp;           // [B*H_q][T]  gate partials
+  int B, H_q, H_kv, L, d, S, T;
+  bool bf16, delta;
+};
+bool backward_supported(int d_k, int d_v, int S);
+cudaError_t launch_backward(const BackwardProblem& p, cudaStream_t stream);
+
 int decode_splits(int S);
 int decode_head_chunks(int g);
 cudaError_t launch_decode_step(const DecodeProblem& p, cudaStream_t stream);

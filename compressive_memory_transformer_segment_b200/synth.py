@@ -16,7 +16,7 @@ import os
 
 import numpy as np
 
-_T_Q, _T_K, _T_V, _T_BETA, _T_PAIR = 1, 2, 3, 4, 5
+_T_Q, _T_K, _T_V, _T_BETA, _T_PAIR, _T_DOUT, _T_DSTATE, _T_STATE = 1, 2, 3, 4, 5, 6, 7, 8
 
 
 def _stream(seed, tensor, b=0, h=0):
@@ -141,3 +141,33 @@ def as_float64(x, dtype):
     if dtype == "bf16":
         return bf16_bits_to_f32(x).astype(np.float64)
     return np.asarray(x, dtype=np.float64)
+
+
+def make_output_grads(cfg, seed=None, scale=1.0):
+    """Seeded upstream gradients for the backward: dout [B, H_q, L, d_v]
+    (bf16 bits or float32, like the forward's output), and float32 dM_out
+    [B, H_kv, d_k, d_v], dz_out [B, H_kv, d_k], all i.i.d. N(0, scale^2)
+    (``scale`` a power of two keeps bf16 values exact)."""
+    seed = cfg.seed if seed is None else seed
+    bf16 = cfg.dtype == "bf16"
+    dout = np.zeros((cfg.B, cfg.H_q, cfg.L, cfg.d_v), dtype=np.uint16 if bf16 else np.float32)
+    for b in range(cfg.B):
+        for h in range(cfg.H_q):
+            x = _stream(seed, _T_DOUT, b, h).standard_normal((cfg.L, cfg.d_v), dtype=np.float32)
+            x *= np.float32(scale)
+            dout[b, h] = round_bf16_bits(x) if bf16 else x
+    g = _stream(seed, _T_DSTATE)
+    dM = g.standard_normal((cfg.B, cfg.H_kv, cfg.d_k, cfg.d_v), dtype=np.float32) * np.float32(scale)
+    dz = g.standard_normal((cfg.B, cfg.H_kv, cfg.d_k), dtype=np.float32) * np.float32(scale)
+    return dict(dout=dout, dM_out=dM, dz_out=dz)
+
+
+def make_state(cfg, seed=None):
+    """A seeded nonzero memory state to start from: M_in ~ N(0, 1/d_k) and
+    z_in ~ U(0.5, 1.5) (positive, as a sum of ELU+1 values is), float32."""
+    seed = cfg.seed if seed is None else seed
+    g = _stream(seed, _T_STATE)
+    M = g.standard_normal((cfg.B, cfg.H_kv, cfg.d_k, cfg.d_v), dtype=np.float32)
+    M *= np.float32(1.0 / np.sqrt(cfg.d_k))
+    z = g.uniform(0.5, 1.5, size=(cfg.B, cfg.H_kv, cfg.d_k)).astype(np.float32)
+    return M, z

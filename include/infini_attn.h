@@ -180,6 +180,48 @@ INFINI_API int infini_attn_state_update(const void* k, const void* v, const floa
                                         const infini_dims_t* dims, float* M_out, float* z_out,
                                         void* workspace, size_t workspace_bytes, void* stream);
 
+/* Bytes of device workspace infini_attn_backward needs for these sizes (the
+ * forward's per-segment states in fp32 and the per-query-head partials of
+ * the backward).  0 if the arguments are invalid or the shape is not one the
+ * backward supports. */
+INFINI_API size_t infini_attn_backward_workspace_bytes(const infini_dims_t* dims, int seg_len,
+                                                       int rule);
+
+/* Backward of infini_attn_forward through the segments (back-propagation
+ * through the memory, as training over a rollout of segments needs:
+ * "Hugging Face Infini-Attention 再現分析", "重み減衰とロールアウト";
+ * "Leave No Context Behind" explainer, "限界").  Given the gradients of a
+ * scalar loss with respect to the forward's outputs, writes its gradients
+ * with respect to the forward's inputs (the chain rule through every step of
+ * the forward; rows whose retrieval denominator is exactly 0 carry none).
+ *   q, k, v, beta,
+ *   M_in, z_in,
+ *   seg_len, rule,
+ *   dims             the forward's arguments, unchanged
+ *   dout             device [B, H_q, L, d_v], element type dims->dtype
+ *   dM_out, dz_out   device float32 [B, H_kv, d_k, d_v] and [B, H_kv, d_k],
+ *                    or NULL for a zero gradient
+ *   dq               device float32 [B, H_q, L, d_k]
+ *   dk, dv           device float32 [B, H_kv, L, d_k] / [B, H_kv, L, d_v]
+ *   dbeta            device float32 [H_q]
+ *   dM_in, dz_in     device float32, the shapes of M_in / z_in
+ *   workspace        device scratch of infini_attn_backward_workspace_bytes
+ *                    bytes, 256-byte aligned; or NULL with workspace_bytes == 0
+ *                    (taken with cudaMallocAsync on `stream`, freed after)
+ *   stream           cudaStream_t; asynchronous.
+ * Supported: d_k == d_v in {32, 64} and seg_len <= 64 (the short-segment
+ * training shapes); otherwise INFINI_ERR_UNSUPPORTED.  The outputs must not
+ * overlap each other, the inputs or the workspace (INFINI_ERR_ALIAS); all
+ * pointers 16-byte aligned (INFINI_ERR_ALIGN).  Every sum runs in a fixed
+ * order: repeated calls give bitwise identical gradients.  Other errors:
+ * INFINI_ERR_ARG, INFINI_ERR_WORKSPACE, INFINI_ERR_CUDA. */
+INFINI_API int infini_attn_backward(const void* q, const void* k, const void* v, const float* beta,
+                                    const float* M_in, const float* z_in, int seg_len, int rule,
+                                    const infini_dims_t* dims, const void* dout,
+                                    const float* dM_out, const float* dz_out, float* dq, float* dk,
+                                    float* dv, float* dbeta, float* dM_in, float* dz_in,
+                                    void* workspace, size_t workspace_bytes, void* stream);
+
 /* Sum of memory states: the exchange step of the sequence-parallel linear
  * rule, where the memory after a run of segments is the memory before it
  * plus the run's own update from a zero state ("Hugging Face
