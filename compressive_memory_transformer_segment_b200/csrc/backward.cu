@@ -44,6 +44,93 @@ constexpr int kBwdMaxS = 64;
 
 __device__ __forceinline__ float elu1_grad(float x) { return x > 0.f ? 1.f : expf(x); }
 
+// C = A B over kk < K for the calling thread's block of an NR x NC output
+// (NR, NC in {32, 64}): rows i = ti + 16u (u < NR/16), columns j = tj + 16v
+// (v < NC/16), thread (ti, tj) = (tid / 16, tid % 16) of 256.
+// A(i, kk) = A[i * lda + kk], or A[kk * lda + i] when TA; B(kk, j) =
+// B[kk * ldb + j], or B[j * ldb + kk] when TB.  Per kk, NR/16 + NC/16 shared
+// loads feed NR NC / 256 FMAs (16 for 64 x 64); a warp's loads of B touch 16
+// consecutive addresses (or stride ldb = d + 1), so no bank conflicts.  Rows
+// or columns past the operands' extent give values the caller does not
+// store.  acc is added to.
+template <int NR, int NC, bool TA, bool TB>
+__device__ __forceinline__ void mm_tile(const float* __restrict__ A, int lda,
+                                        const float* __restrict__ B, int ldb, int K,
+                                        float (&acc)[NR / 16][NC / 16]) {
+  const int ti = threadIdx.x >> 4, tj = threadIdx.x & 15;
+#pragma unroll 4
+  for (int kk = 0; kk < K; ++kk) {
+    float a[NR / 16], b[NC / 16];
+#pragma unroll
+    for (int u = 0; u < NR / 16; ++u) a[u] = TA ? A[kk * lda + ti + 16 * u] : A[(ti + 16 * u) * lda + kk];
+#pragma unroll
+    for (int v = 0; v < NC / 16; ++v) b[v] = TB ? B[(tj + 16 * v) * ldb + kk] : B[kk * ldb + tj + 16 * v];
+#pragma unroll
+    for (int u = 0; u < NR / 16; ++u)
+#pragma unroll
+      for (int v = 0; v < NC / 16; ++v) acc[u][v] = fmaf(a[u], b[v], acc[u][v]);
+  }
+}
+
+template <int NR, int NC>
+__device__ __forceinline__ void zero_tile(float (&acc)[NR / 16][NC / 16]) {
+#pragma unroll
+  for (int u = 0; u < NR / 16; ++u)
+#pragma unroll
+    for (int v = 0; v < NC / 16; ++v) acc[u][v] = 0.f;
+}
+
+// Calls f(i, j, value) for the thread's elements of an NR x NC tile result.
+template <int NR, int NC, typename F>
+__device__ __forceinline__ void for_tile(const float (&acc)[NR / 16][NC / 16], F&& f) {
+  const int ti = threadIdx.x >> 4, tj = threadIdx.x & 15;
+#pragma unroll
+  for (int u = 0; u < NR / 16; ++u)
+#pragma unroll
+    for (int v = 0; v < NC / 16; ++v) f(ti + 16 * u, tj + 16 * v, acc[u][v]);
+}
+
+// 16-byte pieces of a contiguous [rows][D] slice (element type T): the
+// thread's pieces of the first `count` elements are loaded into registers
+// first (all loads in flight together), then unpacked into a shared tile of
+// row stride ld.
+template <typename T, int D, int ROWS>
+struct TileLoad {
+  static constexpr int kVec = 16 / (int)sizeof(T);
+  static constexpr int kPer = (ROWS * D / kVec + kBwdThreads - 1) / kBwdThreads;
+  uint4 raw[kPer];
+  __device__ __forceinline__ void issue(const T* __restrict__ src, int count) {
+#pragma unroll
+    for (int u = 0; u < kPer; ++u) {
+      const int e = threadIdx.x + u * kBwdThreads;
+      raw[u] = e * kVec < count ? reinterpret_cast<const uint4*>(src)[e] : make_uint4(0, 0, 0, 0);
+    }
+  }
+  __device__ __forceinline__ void store(float* dst, int ld, int count) const {
+#pragma unroll
+    for (int u = 0; u < kPer; ++u) {
+      const int e = (threadIdx.x + u * kBwdThreads) * kVec;
+      if (e >= count) continue;
+      const T* x = reinterpret_cast<const T*>(&raw[u]);
+      const int i = e / D, c = e % D;  // kVec divides D: one row per piece
+#pragma unroll
+      for (int t = 0; t < kVec; ++t) dst[i * ld + c + t] = to_f32(x[t]);
+    }
+  }
+  // dst += the piece's values (fp32 sources only)
+  __device__ __forceinline__ void add(float* dst, int ld, int count) const {
+#pragma unroll
+    for (int u = 0; u < kPer; ++u) {
+      const int e = (threadIdx.x + u * kBwdThreads) * kVec;
+      if (e >= count) continue;
+      const float* x = reinterpret_cast<const float*>(&raw[u]);
+      const int i = e / D, c = e % D;
+#pragma unroll
+      for (int t = 0; t < kVec; ++t) dst[i * ld + c + t] += x[t];
+    }
+  }
+};
+
 // Shared-memory plan of bwd_segment (floats): n x D tiles with row stride
 // D + 1 (rows and columns are both read across lanes without conflicts),
 // n x n tiles with stride kBwdMaxS + 1.
@@ -96,16 +183,21 @@ bwd_segment(const T* __restrict__ q, const T* __restrict__ k, const T* __restric
   const T* ks = k + ((size_t)bhkv * L + r0) * D;
   const T* vs = v + ((size_t)bhkv * L + r0) * D;
   const T* ds = dout + ((size_t)bh * L + r0) * D;
-  for (int e = tid; e < n * D; e += kBwdThreads) {
-    const int i = e / D, c = e % D;
-    Q[i * ld + c] = to_f32(qs[e]);
-    K[i * ld + c] = to_f32(ks[e]);
-    V[i * ld + c] = to_f32(vs[e]);
-    dO[i * ld + c] = to_f32(ds[e]);
+  {
+    TileLoad<T, D, kBwdMaxS> lq, lk, lv, ld_o;
+    TileLoad<float, D, D> lm;
+    lq.issue(qs, n * D);
+    lk.issue(ks, n * D);
+    lv.issue(vs, n * D);
+    ld_o.issue(ds, n * D);
+    lm.issue(Mf + ((size_t)s * BHkv + bhkv) * D * D, D * D);
+    for (int c = tid; c < D; c += kBwdThreads) z[c] = zf[((size_t)s * BHkv + bhkv) * D + c];
+    lq.store(Q, ld, n * D);
+    lk.store(K, ld, n * D);
+    lv.store(V, ld, n * D);
+    ld_o.store(dO, ld, n * D);
+    lm.store(M, ld, D * D);
   }
-  const float* Ms = Mf + ((size_t)s * BHkv + bhkv) * D * D;
-  for (int e = tid; e < D * D; e += kBwdThreads) M[(e / D) * ld + e % D] = Ms[e];
-  for (int c = tid; c < D; c += kBwdThreads) z[c] = zf[((size_t)s * BHkv + bhkv) * D + c];
   __syncthreads();
   for (int e = tid; e < n * D; e += kBwdThreads) {
     const int i = e / D, c = e % D;
@@ -119,20 +211,25 @@ bwd_segment(const T* __restrict__ q, const T* __restrict__ k, const T* __restric
     a = warp_sum(a);
     if (lane == 0) den[i] = a;
   }
+  constexpr int N = kBwdMaxS;  // tile extent of the segment's rows
   // scores, masked (key j <= row i)
-  for (int e = tid; e < n * n; e += kBwdThreads) {
-    const int i = e / n, j = e % n;
-    float a = 0.f;
-    for (int c = 0; c < D; ++c) a = fmaf(Q[i * ld + c], K[j * ld + c], a);
-    P[i * lp + j] = j <= i ? a * scale : -INFINITY;
+  {
+    float acc[N / 16][N / 16];
+    zero_tile<N, N>(acc);
+    mm_tile<N, N, false, true>(Q, ld, K, ld, D, acc);
+    for_tile<N, N>(acc, [&](int i, int j, float x) {
+      if (i < n && j < n) P[i * lp + j] = j <= i ? x * scale : -INFINITY;
+    });
   }
   __syncthreads();
   // A_mem = sigma(Q) M / den (0 where den = 0); row softmax of the scores
-  for (int e = tid; e < n * D; e += kBwdThreads) {
-    const int i = e / D, c = e % D;
-    float a = 0.f;
-    for (int kk = 0; kk < D; ++kk) a = fmaf(X[i * ld + kk], M[kk * ld + c], a);
-    Am[i * ld + c] = den[i] != 0.f ? a / den[i] : 0.f;
+  {
+    float acc[N / 16][D / 16];
+    zero_tile<N, D>(acc);
+    mm_tile<N, D, false, false>(X, ld, M, ld, D, acc);
+    for_tile<N, D>(acc, [&](int i, int c, float x) {
+      if (i < n) Am[i * ld + c] = den[i] != 0.f ? x / den[i] : 0.f;
+    });
   }
   for (int i = warp; i < n; i += kBwdThreads / 32) {
     float m = -INFINITY;
@@ -149,13 +246,16 @@ bwd_segment(const T* __restrict__ q, const T* __restrict__ k, const T* __restric
     for (int j = lane; j < n; j += 32) P[i * lp + j] *= inv;
   }
   __syncthreads();
-  // A_dot = P V, and the gate's partial sum(dout (A_mem - A_dot))
+  // A_dot = P V (P is 0 right of the diagonal), and the gate's partial
+  // sum(dout (A_mem - A_dot))
   float part = 0.f;
-  for (int e = tid; e < n * D; e += kBwdThreads) {
-    const int i = e / D, c = e % D;
-    float a = 0.f;
-    for (int j = 0; j <= i; ++j) a = fmaf(P[i * lp + j], V[j * ld + c], a);
-    part = fmaf(dO[i * ld + c], Am[i * ld + c] - a, part);
+  {
+    float acc[N / 16][D / 16];
+    zero_tile<N, D>(acc);
+    mm_tile<N, D, false, false>(P, lp, V, ld, n, acc);
+    for_tile<N, D>(acc, [&](int i, int c, float x) {
+      if (i < n) part = fmaf(dO[i * ld + c], Am[i * ld + c] - x, part);
+    });
   }
   part = warp_sum(part);
   if (lane == 0) red[warp] = part;
@@ -178,12 +278,12 @@ bwd_segment(const T* __restrict__ q, const T* __restrict__ k, const T* __restric
     dbp[(size_t)bh * T_seg + s] = a * g * (1.f - g);
   }
   // Retrieval: dM_{s-1} += sigma(Q)^T dnum, dz_{s-1} += sigma(Q)^T dden
-  float* dMo = dMr + ((size_t)s * BHq + bh) * D * D;
-  for (int e = tid; e < D * D; e += kBwdThreads) {
-    const int kk = e / D, c = e % D;
-    float a = 0.f;
-    for (int i = 0; i < n; ++i) a = fmaf(X[i * ld + kk], Y[i * ld + c], a);
-    dMo[e] = a;
+  {
+    float* dMo = dMr + ((size_t)s * BHq + bh) * D * D;
+    float acc[D / 16][D / 16];
+    zero_tile<D, D>(acc);
+    mm_tile<D, D, true, false>(X, ld, Y, ld, n, acc);
+    for_tile<D, D>(acc, [&](int kk, int c, float x) { dMo[kk * D + c] = x; });
   }
   for (int kk = tid; kk < D; kk += kBwdThreads) {
     float a = 0.f;
@@ -191,28 +291,33 @@ bwd_segment(const T* __restrict__ q, const T* __restrict__ k, const T* __restric
     dzr[((size_t)s * BHq + bh) * D + kk] = a;
   }
   // dQ (retrieval part) = (dnum M^T + dden z^T) sigma'(Q), into Am
-  for (int e = tid; e < n * D; e += kBwdThreads) {
-    const int i = e / D, kk = e % D;
-    float a = dden[i] * z[kk];
-    for (int c = 0; c < D; ++c) a = fmaf(Y[i * ld + c], M[kk * ld + c], a);
-    Am[i * ld + kk] = a * elu1_grad(Q[i * ld + kk]);
+  {
+    float acc[N / 16][D / 16];
+    zero_tile<N, D>(acc);
+    mm_tile<N, D, false, true>(Y, ld, M, ld, D, acc);
+    for_tile<N, D>(acc, [&](int i, int kk, float x) {
+      if (i < n) Am[i * ld + kk] = fmaf(dden[i], z[kk], x) * elu1_grad(Q[i * ld + kk]);
+    });
   }
   // Attention: dP = (1 - g) dout V^T (causal part only)
   const float ga = 1.f - g;
-  for (int e = tid; e < n * n; e += kBwdThreads) {
-    const int i = e / n, j = e % n;
-    float a = 0.f;
-    if (j <= i)
-      for (int c = 0; c < D; ++c) a = fmaf(dO[i * ld + c], V[j * ld + c], a);
-    dS[i * lp + j] = ga * a;
+  {
+    float acc[N / 16][N / 16];
+    zero_tile<N, N>(acc);
+    mm_tile<N, N, false, true>(dO, ld, V, ld, D, acc);
+    for_tile<N, N>(acc, [&](int i, int j, float x) {
+      if (i < n && j < n) dS[i * lp + j] = j <= i ? ga * x : 0.f;
+    });
   }
   // dV (attention) = P^T dA_dot
-  float* dVo = dVa + ((size_t)bh * L + r0) * D;
-  for (int e = tid; e < n * D; e += kBwdThreads) {
-    const int j = e / D, c = e % D;
-    float a = 0.f;
-    for (int i = j; i < n; ++i) a = fmaf(P[i * lp + j], dO[i * ld + c], a);
-    dVo[e] = ga * a;
+  {
+    float* dVo = dVa + ((size_t)bh * L + r0) * D;
+    float acc[N / 16][D / 16];
+    zero_tile<N, D>(acc);
+    mm_tile<N, D, true, false>(P, lp, dO, ld, n, acc);
+    for_tile<N, D>(acc, [&](int j, int c, float x) {
+      if (j < n) dVo[j * D + c] = ga * x;
+    });
   }
   __syncthreads();
   // dS = P (dP - rowsum(dP P))
@@ -229,16 +334,23 @@ bwd_segment(const T* __restrict__ q, const T* __restrict__ k, const T* __restric
   }
   __syncthreads();
   // dq = dS K / sqrt(d) + retrieval part; dK (attention) = dS^T Q / sqrt(d)
-  float* dqo = dq + ((size_t)bh * L + r0) * D;
-  float* dKo = dKa + ((size_t)bh * L + r0) * D;
-  for (int e = tid; e < n * D; e += kBwdThreads) {
-    const int i = e / D, c = e % D;
-    float a = 0.f;
-    for (int j = 0; j <= i; ++j) a = fmaf(dS[i * lp + j], K[j * ld + c], a);
-    dqo[e] = fmaf(a, scale, Am[i * ld + c]);
-    float bk = 0.f;
-    for (int r = i; r < n; ++r) bk = fmaf(dS[r * lp + i], Q[r * ld + c], bk);
-    dKo[e] = bk * scale;
+  {
+    float* dqo = dq + ((size_t)bh * L + r0) * D;
+    float acc[N / 16][D / 16];
+    zero_tile<N, D>(acc);
+    mm_tile<N, D, false, false>(dS, lp, K, ld, n, acc);
+    for_tile<N, D>(acc, [&](int i, int c, float x) {
+      if (i < n) dqo[i * D + c] = fmaf(x, scale, Am[i * ld + c]);
+    });
+  }
+  {
+    float* dKo = dKa + ((size_t)bh * L + r0) * D;
+    float acc[N / 16][D / 16];
+    zero_tile<N, D>(acc);
+    mm_tile<N, D, true, false>(dS, lp, Q, ld, n, acc);
+    for_tile<N, D>(acc, [&](int j, int c, float x) {
+      if (j < n) dKo[j * D + c] = x * scale;
+    });
   }
 }
 
@@ -253,8 +365,9 @@ struct ScanBwdSmem {
   static constexpr int kV = kSK + kTile;
   static constexpr int kX1 = kV + kTile;           // d sigma(K)
   static constexpr int kX2 = kX1 + kTile;          // dV (= dU, delta)
-  static constexpr int kX3 = kX2 + kTile;          // R (delta)
-  static constexpr int kGz = kX3 + kTile;
+  static constexpr int kX3 = kX2 + kTile;          // R, then U = V - R (delta)
+  static constexpr int kX4 = kX3 + kTile;          // dN = -dU / r (delta)
+  static constexpr int kGz = kX4 + kTile;
   static constexpr int kZ = kGz + D;
   static constexpr int kR = kZ + D;                // r_t (delta)
   static constexpr int kDr = kR + kBwdMaxS;        // dr_t (delta)
@@ -274,7 +387,7 @@ bwd_scan(const T* __restrict__ k, const T* __restrict__ v, const float* __restri
   constexpr int ld = SM::kLd;
   extern __shared__ float sm[];
   float *GM = sm + SM::kGM, *M = sm + SM::kM, *sK = sm + SM::kSK, *V = sm + SM::kV;
-  float *X1 = sm + SM::kX1, *X2 = sm + SM::kX2, *X3 = sm + SM::kX3;
+  float *X1 = sm + SM::kX1, *X2 = sm + SM::kX2, *X3 = sm + SM::kX3, *X4 = sm + SM::kX4;
   float *Gz = sm + SM::kGz, *z = sm + SM::kZ, *r = sm + SM::kR, *dr = sm + SM::kDr;
   const int bhkv = blockIdx.x, BHkv = gridDim.x;
   const int b = bhkv / H_kv, j = bhkv % H_kv, grp = H_q / H_kv;
@@ -287,17 +400,26 @@ bwd_scan(const T* __restrict__ k, const T* __restrict__ v, const float* __restri
     const int r0 = s * S, n = min(S, L - r0);
     const T* ks = k + ((size_t)bhkv * L + r0) * D;
     const T* vs = v + ((size_t)bhkv * L + r0) * D;
-    for (int e = tid; e < n * D; e += kBwdThreads) {
-      const int i = e / D, c = e % D;
-      sK[i * ld + c] = elu1(to_f32(ks[e]));
-      V[i * ld + c] = to_f32(vs[e]);
-    }
-    if (DELTA) {
-      const float* Ms = Mf + ((size_t)s * BHkv + bhkv) * D * D;
-      for (int e = tid; e < D * D; e += kBwdThreads) M[(e / D) * ld + e % D] = Ms[e];
-      for (int c = tid; c < D; c += kBwdThreads) z[c] = zf[((size_t)s * BHkv + bhkv) * D + c];
+    {
+      TileLoad<T, D, kBwdMaxS> lk, lv;
+      TileLoad<float, D, D> lm;
+      lk.issue(ks, n * D);
+      lv.issue(vs, n * D);
+      if (DELTA) {
+        lm.issue(Mf + ((size_t)s * BHkv + bhkv) * D * D, D * D);
+        for (int c = tid; c < D; c += kBwdThreads) z[c] = zf[((size_t)s * BHkv + bhkv) * D + c];
+      }
+      lk.store(sK, ld, n * D);
+      lv.store(V, ld, n * D);
+      if (DELTA) lm.store(M, ld, D * D);
     }
     __syncthreads();
+    for (int e = tid; e < n * D; e += kBwdThreads) {
+      const int i = e / D, c = e % D;
+      sK[i * ld + c] = elu1(sK[i * ld + c]);
+    }
+    __syncthreads();
+    constexpr int N = kBwdMaxS;
     if (DELTA) {
       // r_t = sigma(k_t) . z_{s-1}
       for (int i = warp; i < n; i += kBwdThreads / 32) {
@@ -308,15 +430,18 @@ bwd_scan(const T* __restrict__ k, const T* __restrict__ v, const float* __restri
       }
       __syncthreads();
       // R = sigma(K) M / r (0 where r = 0); dU = sigma(K) G_M
-      for (int e = tid; e < n * D; e += kBwdThreads) {
-        const int i = e / D, c = e % D;
-        float a = 0.f, u = 0.f;
-        for (int kk = 0; kk < D; ++kk) {
-          a = fmaf(sK[i * ld + kk], M[kk * ld + c], a);
-          u = fmaf(sK[i * ld + kk], GM[kk * ld + c], u);
-        }
-        X3[i * ld + c] = r[i] != 0.f ? a / r[i] : 0.f;
-        X2[i * ld + c] = u;
+      {
+        float acc[N / 16][D / 16];
+        zero_tile<N, D>(acc);
+        mm_tile<N, D, false, false>(sK, ld, M, ld, D, acc);
+        for_tile<N, D>(acc, [&](int i, int c, float x) {
+          if (i < n) X3[i * ld + c] = r[i] != 0.f ? x / r[i] : 0.f;
+        });
+        zero_tile<N, D>(acc);
+        mm_tile<N, D, false, false>(sK, ld, GM, ld, D, acc);
+        for_tile<N, D>(acc, [&](int i, int c, float x) {
+          if (i < n) X2[i * ld + c] = x;
+        });
       }
       __syncthreads();
       // dr_t = rowsum(dU R) / r
@@ -327,27 +452,30 @@ bwd_scan(const T* __restrict__ k, const T* __restrict__ v, const float* __restri
         if (lane == 0) dr[i] = r[i] != 0.f ? a / r[i] : 0.f;
       }
       __syncthreads();
-      // d sigma(K) = (V - R) G_M^T + dN M^T + dr z^T + G_z, dN = -dU / r
+      // U = V - R (over R) and dN = -dU / r
       for (int e = tid; e < n * D; e += kBwdThreads) {
-        const int i = e / D, kk = e % D;
-        const float ir = r[i] != 0.f ? -1.f / r[i] : 0.f;
-        float a = fmaf(dr[i], z[kk], Gz[kk]);
-        for (int c = 0; c < D; ++c) {
-          a = fmaf(V[i * ld + c] - X3[i * ld + c], GM[kk * ld + c], a);
-          a = fmaf(X2[i * ld + c] * ir, M[kk * ld + c], a);
-        }
-        X1[i * ld + kk] = a;
+        const int i = e / D, c = e % D;
+        X3[i * ld + c] = V[i * ld + c] - X3[i * ld + c];
+        X4[i * ld + c] = r[i] != 0.f ? -X2[i * ld + c] / r[i] : 0.f;
+      }
+      __syncthreads();
+      // d sigma(K) = U G_M^T + dN M^T + dr z^T + G_z
+      {
+        float acc[N / 16][D / 16];
+        zero_tile<N, D>(acc);
+        mm_tile<N, D, false, true>(X3, ld, GM, ld, D, acc);
+        mm_tile<N, D, false, true>(X4, ld, M, ld, D, acc);
+        for_tile<N, D>(acc, [&](int i, int kk, float x) {
+          if (i < n) X1[i * ld + kk] = x + fmaf(dr[i], z[kk], Gz[kk]);
+        });
       }
       __syncthreads();
       // G_M += sigma(K)^T dN, G_z += sigma(K)^T dr
-      for (int e = tid; e < D * D; e += kBwdThreads) {
-        const int kk = e / D, c = e % D;
-        float a = 0.f;
-        for (int i = 0; i < n; ++i) {
-          const float ir = r[i] != 0.f ? -1.f / r[i] : 0.f;
-          a = fmaf(sK[i * ld + kk], X2[i * ld + c] * ir, a);
-        }
-        GM[kk * ld + c] += a;
+      {
+        float acc[D / 16][D / 16];
+        zero_tile<D, D>(acc);
+        mm_tile<D, D, true, false>(sK, ld, X4, ld, n, acc);
+        for_tile<D, D>(acc, [&](int kk, int c, float x) { GM[kk * ld + c] += x; });
       }
       for (int kk = tid; kk < D; kk += kBwdThreads) {
         float a = 0.f;
@@ -356,39 +484,45 @@ bwd_scan(const T* __restrict__ k, const T* __restrict__ v, const float* __restri
       }
     } else {
       // d sigma(K) = V G_M^T + G_z, dV = sigma(K) G_M
-      for (int e = tid; e < n * D; e += kBwdThreads) {
-        const int i = e / D, c = e % D;
-        float a = Gz[c], u = 0.f;
-        for (int kk = 0; kk < D; ++kk) {
-          a = fmaf(V[i * ld + kk], GM[c * ld + kk], a);
-          u = fmaf(sK[i * ld + kk], GM[kk * ld + c], u);
-        }
-        X1[i * ld + c] = a;
-        X2[i * ld + c] = u;
-      }
+      float acc[N / 16][D / 16];
+      zero_tile<N, D>(acc);
+      mm_tile<N, D, false, true>(V, ld, GM, ld, D, acc);
+      for_tile<N, D>(acc, [&](int i, int c, float x) {
+        if (i < n) X1[i * ld + c] = x + Gz[c];
+      });
+      zero_tile<N, D>(acc);
+      mm_tile<N, D, false, false>(sK, ld, GM, ld, D, acc);
+      for_tile<N, D>(acc, [&](int i, int c, float x) {
+        if (i < n) X2[i * ld + c] = x;
+      });
     }
     __syncthreads();
-    // dk, dv of the segment: the update's part plus every query head's attention part.
+    // dk, dv of the segment: the update's part (dk through sigma'(k) = 1 or
+    // e^k = sigma(k)) plus every query head's attention part, added in head
+    // order; and the heads' retrieval gradients with respect to M_{s-1}.
     for (int e = tid; e < n * D; e += kBwdThreads) {
       const int i = e / D, c = e % D;
       const float sk = sK[i * ld + c];
-      float a = X1[i * ld + c] * (sk > 1.f ? 1.f : sk);  // sigma'(k) = 1 or e^k = sigma(k)
-      float u = X2[i * ld + c];
-      for (int hh = 0; hh < grp; ++hh) {
-        const size_t row = ((size_t)(b * H_q + j * grp + hh) * L + r0 + i) * D + c;
-        a += dKa[row];
-        u += dVa[row];
-      }
-      const size_t o = ((size_t)bhkv * L + r0 + i) * D + c;
-      dk[o] = a;
-      dv[o] = u;
+      X1[i * ld + c] *= sk > 1.f ? 1.f : sk;
     }
-    // The query heads' retrieval gradients with respect to (M_{s-1}, z_{s-1}).
-    for (int e = tid; e < D * D; e += kBwdThreads) {
-      float a = 0.f;
-      for (int hh = 0; hh < grp; ++hh)
-        a += dMr[((size_t)s * BHq + b * H_q + j * grp + hh) * D * D + e];
-      GM[(e / D) * ld + e % D] += a;
+    __syncthreads();
+    for (int hh = 0; hh < grp; ++hh) {
+      const size_t head = (size_t)(b * H_q + j * grp + hh);
+      TileLoad<float, D, kBwdMaxS> la, lb;
+      TileLoad<float, D, D> lr;
+      la.issue(dKa + (head * L + r0) * D, n * D);
+      lb.issue(dVa + (head * L + r0) * D, n * D);
+      lr.issue(dMr + ((size_t)s * BHq + head) * D * D, D * D);
+      la.add(X1, ld, n * D);
+      lb.add(X2, ld, n * D);
+      lr.add(GM, ld, D * D);
+    }
+    __syncthreads();
+    for (int e = tid; e < n * D; e += kBwdThreads) {
+      const int i = e / D, c = e % D;
+      const size_t o = ((size_t)bhkv * L + r0 + i) * D + c;
+      dk[o] = X1[i * ld + c];
+      dv[o] = X2[i * ld + c];
     }
     for (int c = tid; c < D; c += kBwdThreads) {
       float a = 0.f;
