@@ -507,7 +507,8 @@ namespace {
 // Backward workspace: the forward's fp32 states (slot s = M_{s-1}, z_{s-1}),
 // a scratch M_T / z_T, and the per-query-head partials.
 struct BwdLayout {
-  size_t zf, Mf, Mscr, zscr, dKa, dVa, dMr, dzr, dbp, total;
+  size_t zf, Mf, Mscr, zscr, dKa, dVa, dMr, dzr, dbp, g, b, dz, total;
+  bool tc;  // the recompute runs the tensor-core scan (fp32 states out)
 };
 
 int backward_layout(const infini_dims_t* dims, int seg_len, int rule, Shape* s, BwdLayout* lay) {
@@ -525,7 +526,17 @@ int backward_layout(const infini_dims_t* dims, int seg_len, int rule, Shape* s, 
   lay->dMr = align_up(lay->dVa + BHq * L * d * 4);
   lay->dzr = align_up(lay->dMr + T * BHq * d * d * 4);
   lay->dbp = align_up(lay->dzr + T * BHq * d * 4);
-  lay->total = align_up(lay->dbp + BHq * T * 4);
+  lay->g = lay->b = lay->dz = align_up(lay->dbp + BHq * T * 4);
+  lay->tc = tc_scan_supported(s->d_k, s->d_v, s->bf16);
+  size_t end = lay->g;
+  if (lay->tc) {
+    size_t g = 0, b = 0, z = 0;
+    tc_scan_workspace(s->B, s->H_kv, s->T, s->d_k, s->delta, &g, &b, &z);
+    lay->b = align_up(lay->g + g);
+    lay->dz = align_up(lay->b + b);
+    end = align_up(lay->dz + z);
+  }
+  lay->total = end;
   return INFINI_OK;
 }
 
@@ -591,10 +602,17 @@ int infini_attn_backward(const void* q, const void* k, const void* v, const floa
   p.z_pref = reinterpret_cast<float*>(ws + lay.zf);
   p.M_pref = ws + lay.Mf;
   p.M_pref_bf16 = false;
-  p.Gbuf = p.Bbuf = p.dz = nullptr;
+  p.Gbuf = reinterpret_cast<float*>(ws + lay.g);
+  p.Bbuf = reinterpret_cast<float*>(ws + lay.b);
+  p.dz = reinterpret_cast<float*>(ws + lay.dz);
   p.status = status;
-  cudaError_t e = cudaMemcpyAsync(p.z_pref, z_in, s.z_bytes, cudaMemcpyDeviceToDevice, st);
-  if (e == cudaSuccess) e = timed(0, st, [&] { return launch_simt_state_scan(p, st); });
+  cudaError_t e = cudaSuccess;
+  if (lay.tc) {
+    e = timed(0, st, [&] { return launch_tc_state_scan(p, st); });
+  } else {
+    e = cudaMemcpyAsync(p.z_pref, z_in, s.z_bytes, cudaMemcpyDeviceToDevice, st);
+    if (e == cudaSuccess) e = timed(0, st, [&] { return launch_simt_state_scan(p, st); });
+  }
   BackwardProblem bp;
   bp.q = q; bp.k = k; bp.v = v; bp.beta = beta; bp.dout = dout; bp.dM_out = dM_out; bp.dz_out = dz_out;
   bp.dq = dq; bp.dk = dk; bp.dv = dv; bp.dbeta = dbeta; bp.dM_in = dM_in; bp.dz_in = dz_in;

@@ -52,8 +52,9 @@ cudaError_t launch_tc_attention(const Problem& p, cudaStream_t stream);
 cudaError_t launch_tc_attention_single(const Problem& p, cudaStream_t stream);
 
 // Tensor-core memory-state scan (both rules): bf16 I/O, d_k == d_v in
-// {64, 128}, any S.  Writes bf16 M_pref and fp32 z_pref; needs the Gbuf,
-// Bbuf and dz workspace regions sized by tc_scan_workspace.
+// {64, 128}, any S.  Writes M_pref (bf16, or fp32 when !M_pref_bf16) and
+// fp32 z_pref; needs the Gbuf, Bbuf and dz workspace regions sized by
+// tc_scan_workspace.
 bool tc_scan_supported(int d_k, int d_v, bool bf16);
 int tc_scan_launches(bool delta);
 void tc_scan_workspace(int B, int H_kv, int T, int d, bool delta, size_t* g_bytes, size_t* b_bytes,

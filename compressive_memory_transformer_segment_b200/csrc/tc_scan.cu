@@ -489,6 +489,18 @@ tc_pipe_products(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
 
 constexpr int kCB = 16;  // columns of M per combine CTA (delta)
 
+// Four consecutive elements of a published state M_{s-1}: bf16 for the
+// attention's retrieval, or fp32 (the backward's recompute of the states).
+__device__ __forceinline__ void store_state4(__nv_bfloat16* dst, float4 m) {
+  uint2 w;
+  w.x = pack_bf16x2(m.x, m.y);
+  w.y = pack_bf16x2(m.z, m.w);
+  *reinterpret_cast<uint2*>(dst) = w;
+}
+__device__ __forceinline__ void store_state4(float* dst, float4 m) {
+  *reinterpret_cast<float4*>(dst) = m;
+}
+
 __device__ __forceinline__ void cp_async16(void* smem_dst, const void* gmem_src) {
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(smem_dst)), "l"(gmem_src)
                : "memory");
@@ -510,11 +522,11 @@ __device__ __forceinline__ void cp_async_wait() {
 // G_s M is read from column k of G_s: four consecutive rows of the tile are
 // one contiguous 16-byte piece.  G_{s+1} streams in (cp.async) and the B_{s+1}
 // tile is loaded into registers while step s runs.  Plain block barriers only.
-template <int D>
+template <int D, typename MP>
 __global__ void __launch_bounds__(D) combine_delta(const float* __restrict__ M_in,
                                                    const float* __restrict__ Gbuf,
                                                    const float* __restrict__ Bbuf,
-                                                   __nv_bfloat16* __restrict__ M_pref,
+                                                   MP* __restrict__ M_pref,
                                                    float* __restrict__ M_out, int T) {
   static_assert(kCB == 16 && D % 32 == 0, "combine_delta thread map");
   extern __shared__ __align__(16) float csm[];
@@ -552,13 +564,10 @@ __global__ void __launch_bounds__(D) combine_delta(const float* __restrict__ M_i
     } else {
       cp_async_wait<0>();
     }
-    // Publish M_{s-1} (bf16) for segment s's retrieval.
+    // Publish M_{s-1} for segment s's retrieval.
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-      uint2 w;
-      w.x = pack_bf16x2(m[i].x, m[i].y);
-      w.y = pack_bf16x2(m[i].z, m[i].w);
-      *reinterpret_cast<uint2*>(M_pref + (slice * D + k0 + i) * D + c0 + c) = w;
+      store_state4(M_pref + (slice * D + k0 + i) * D + c0 + c, m[i]);
       *reinterpret_cast<float4*>(sM + (k0 + i) * kCB + c) = m[i];
     }
     __syncthreads();
@@ -597,11 +606,11 @@ __global__ void __launch_bounds__(D) combine_delta(const float* __restrict__ M_i
 // Linear rule: M_s = M_{s-1} + B_s, z_s = z_{s-1} + dz_s, element-parallel.
 // Grid (B*H_kv, ceil(D*D / 1024)), block 256 threads x 4 elements; block
 // (bh, 0) also carries z.
-template <int D>
+template <int D, typename MP>
 __global__ void __launch_bounds__(256) combine_linear(const float* __restrict__ M_in,
                                                       const float* __restrict__ Bbuf,
                                                       const float* __restrict__ dz,
-                                                      __nv_bfloat16* __restrict__ M_pref,
+                                                      MP* __restrict__ M_pref,
                                                       const float* z_in,
                                                       float* __restrict__ z_pref,
                                                       float* __restrict__ M_out, float* z_out,
@@ -622,10 +631,7 @@ __global__ void __launch_bounds__(256) combine_linear(const float* __restrict__ 
 #pragma unroll
       for (int i = 0; i < kAhead; ++i) {
         if (s0 + i >= T) break;
-        uint2 w;
-        w.x = pack_bf16x2(m.x, m.y);
-        w.y = pack_bf16x2(m.z, m.w);
-        *reinterpret_cast<uint2*>(M_pref + ((size_t)(s0 + i) * BH + bh) * D * D + e) = w;
+        store_state4(M_pref + ((size_t)(s0 + i) * BH + bh) * D * D + e, m);
         m.x += b[i].x;
         m.y += b[i].y;
         m.z += b[i].z;
@@ -700,10 +706,10 @@ cudaError_t launch_pipe_products(const Problem& p, cudaStream_t stream) {
   return cudaGetLastError();
 }
 
-template <int D>
+template <int D, typename MP>
 cudaError_t launch(const Problem& p, cudaStream_t stream) {
   const unsigned BH = (unsigned)((uint64_t)p.B * p.H_kv);
-  __nv_bfloat16* Mp = static_cast<__nv_bfloat16*>(p.M_pref);
+  MP* Mp = static_cast<MP*>(p.M_pref);
   cudaError_t e;
   if (p.delta) {
     const int C = zsum_chunks(p.S);
@@ -715,15 +721,15 @@ cudaError_t launch(const Problem& p, cudaStream_t stream) {
     e = launch_pipe_products<D, true>(p, stream);
     if (e != cudaSuccess) return e;
     const int csmem = (2 * D * D + D * kCB) * (int)sizeof(float);
-    e = cudaFuncSetAttribute(combine_delta<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, csmem);
+    e = cudaFuncSetAttribute(combine_delta<D, MP>, cudaFuncAttributeMaxDynamicSharedMemorySize, csmem);
     if (e != cudaSuccess) return e;
-    combine_delta<D><<<dim3(BH, D / kCB), D, csmem, stream>>>(p.M_in, p.Gbuf, p.Bbuf, Mp, p.M_out,
+    combine_delta<D, MP><<<dim3(BH, D / kCB), D, csmem, stream>>>(p.M_in, p.Gbuf, p.Bbuf, Mp, p.M_out,
                                                                  p.T);
     return cudaGetLastError();
   }
   e = launch_pipe_products<D, false>(p, stream);
   if (e != cudaSuccess) return e;
-  combine_linear<D><<<dim3(BH, (D * D + 1023) / 1024), 256, 0, stream>>>(
+  combine_linear<D, MP><<<dim3(BH, (D * D + 1023) / 1024), 256, 0, stream>>>(
       p.M_in, p.Bbuf, p.dz, Mp, p.z_in, p.z_pref, p.M_out, p.z_out, p.T);
   return cudaGetLastError();
 }
@@ -746,8 +752,13 @@ void tc_scan_workspace(int B, int H_kv, int T, int d, bool delta, size_t* g_byte
 }
 
 cudaError_t launch_tc_state_scan(const Problem& p, cudaStream_t stream) {
-  if (p.d_k == 128) return launch<128>(p, stream);
-  if (p.d_k == 64) return launch<64>(p, stream);
+  if (p.M_pref_bf16) {
+    if (p.d_k == 128) return launch<128, __nv_bfloat16>(p, stream);
+    if (p.d_k == 64) return launch<64, __nv_bfloat16>(p, stream);
+  } else {
+    if (p.d_k == 128) return launch<128, float>(p, stream);
+    if (p.d_k == 64) return launch<64, float>(p, stream);
+  }
   return cudaErrorInvalidValue;
 }
 
