@@ -745,6 +745,189 @@ def run_decode(args, w):
     return 0
 
 
+def backward_flops(w):
+    """Algorithmic fp32 flops of the backward kernels (the recompute of the
+    states excluded), per step: per (batch row, query head, segment of n
+    rows) the attention's six causal n x n x d products (scores and A_dot
+    recomputed, dP, dV, dQ, dK: 6 n (n + 1) d) and the retrieval's three
+    n x d x d products (A_mem recomputed, dM, d sigma(Q): 6 n d^2); per
+    (batch row, KV head, segment) the update's VJP: 2 products (linear) or
+    5 (delta) of n x d x d."""
+    d = w.d_k
+    per_kv = (4 if w.rule == "linear" else 10)
+    total = 0
+    for s in range(-(-w.L // w.seg_len)):
+        n = min(w.seg_len, w.L - s * w.seg_len)
+        total += w.B * w.H_q * (6 * n * (n + 1) * d + 6 * n * d * d)
+        total += w.B * w.H_kv * per_kv * n * d * d
+    return total
+
+
+def oracle_backward_sample(w, budget_s):
+    """Time the float64 oracle's backward on whole (batch row, KV head) chains
+    until about ``budget_s`` seconds have passed; token-equivalents/s as in
+    oracle_sample."""
+    import oracle  # the CPU baseline is the only product-adjacent use of the oracle
+
+    g = w.H_q // w.H_kv
+    beta = synth.make_beta(w).astype(np.float64)
+    grads = synth.make_output_grads(w)
+    one = w.with_(B=1, H_q=g, H_kv=1)
+    rows, used, elapsed = 0, [], 0.0
+    for b in range(w.B):
+        for j in range(w.H_kv):
+            kc = synth.as_float64(synth.make_head(w, "k", b, j), w.dtype)[None, None]
+            vc = synth.as_float64(synth.make_head(w, "v", b, j), w.dtype)[None, None]
+            heads = list(range(j * g, (j + 1) * g))
+            qc = np.stack([synth.as_float64(synth.make_head(w, "q", b, h), w.dtype)
+                           for h in heads])[None]
+            dout = synth.as_float64(grads["dout"][b, heads], w.dtype)[None]
+            t0 = time.perf_counter()
+            oracle.infini_attention_backward(
+                qc, kc, vc, beta[heads], np.zeros((1, 1, w.d_k, w.d_v)), np.zeros((1, 1, w.d_k)),
+                w.seg_len, w.rule, dout, grads["dM_out"][b:b + 1, j:j + 1].astype(np.float64),
+                grads["dz_out"][b:b + 1, j:j + 1].astype(np.float64))
+            elapsed += time.perf_counter() - t0
+            rows += w.L
+            used.append((b, j))
+            if elapsed >= budget_s:
+                break
+        if elapsed >= budget_s:
+            break
+    desc = (f"oracle backward (NumPy float64), {len(used)} whole (batch, KV head) chain(s) "
+            f"from {used[0]}, each with its {g} query head(s), {one.L} rows each, in "
+            f"{elapsed:.2f} s of compute (input generation untimed); token-equivalents = "
+            f"rows / H_kv")
+    return rows / w.H_kv / elapsed, desc
+
+
+def run_backward(args, w):
+    """The backward through the segments (gradients of every input given the
+    gradients of out, M_out, z_out) on one GPU; a step is one
+    infini_attn_backward over one batch, from the zero initial memory."""
+    import torch
+
+    from compressive_memory_transformer_segment_b200 import api
+
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    api.load_library()
+    inp = synth.make_inputs(w)
+    grads = synth.make_output_grads(w)
+    tdt = torch.bfloat16 if w.dtype == "bf16" else torch.float32
+
+    def host_tensor(x):
+        if w.dtype == "bf16":
+            return torch.from_numpy(np.ascontiguousarray(x).view(np.int16)).view(torch.bfloat16)
+        return torch.from_numpy(np.ascontiguousarray(x, dtype=np.float32))
+
+    hq, hk, hv, hd = (host_tensor(a) for a in (inp["q"], inp["k"], inp["v"], grads["dout"]))
+    q, k, v, dout = (t.to(dev) for t in (hq, hk, hv, hd))
+    beta = torch.from_numpy(inp["beta"]).to(dev)
+    M0, z0 = api.init_state(w.B, w.H_kv, w.d_k, w.d_v, device=dev)
+    dM = torch.from_numpy(grads["dM_out"]).to(dev)
+    dz = torch.from_numpy(grads["dz_out"]).to(dev)
+    dims = api.make_dims(w.B, w.H_q, w.H_kv, w.L, w.d_k, w.d_v, tdt)
+    nbytes = api.backward_workspace_bytes(dims, w.seg_len, w.rule)
+    if nbytes == 0:
+        print(json.dumps({"metric": "Infini-attention backward", "unsupported": w.name}))
+        return 1
+    ws = torch.empty(nbytes, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    in_bytes = sum(t.numel() * t.element_size() for t in (q, k, v, dout))
+    flush = torch.empty(2 * L2_BYTES, dtype=torch.uint8, device=dev) if in_bytes < 2 * L2_BYTES else None
+
+    def step():
+        return api.backward(q, k, v, beta, M0, z0, w.seg_len, w.rule, dout, dM, dz,
+                            workspace=ws, stream=stream)
+
+    for _ in range(args.warmup):
+        step()
+    api.sync_status(stream)
+    api.set_kernel_timing(True)
+    api.kernel_times(reset=True)
+    torch.cuda.synchronize(dev)
+    elapsed_ms = 0.0
+    with ClockSampler(0) as clocks:
+        for _ in range(args.steps):
+            if flush is not None:
+                flush.fill_(1)
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            step()
+            e1.record(stream)
+            torch.cuda.synchronize(dev)
+            elapsed_ms += e0.elapsed_time(e1)
+    api.set_kernel_timing(False)
+    ktimes = api.kernel_times(reset=True)
+    api.sync_status(stream)
+    tokens = w.B * w.L * args.steps
+    value = tokens / (elapsed_ms / 1000.0)
+
+    # End to end: inputs and upstream gradients copied from pinned host memory,
+    # the six gradients copied back, inside the timed region.
+    hp = [t.pin_memory() for t in (hq, hk, hv, hd)]
+    dev_in = [torch.empty_like(t, device=dev) for t in hp]
+    outs_h = None
+    e2e_steps = max(1, min(args.steps, 5))
+    torch.cuda.synchronize(dev)
+    e2, e3 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e2.record(stream)
+    for _ in range(e2e_steps):
+        for dst, src in zip(dev_in, hp):
+            dst.copy_(src, non_blocking=True)
+        res = api.backward(*dev_in[:3], beta, M0, z0, w.seg_len, w.rule, dev_in[3], dM, dz,
+                           workspace=ws, stream=stream)
+        if outs_h is None:
+            outs_h = [torch.empty(t.shape, dtype=t.dtype).pin_memory() for t in res]
+        for dst, src in zip(outs_h, res):
+            dst.copy_(src, non_blocking=True)
+    e3.record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_value = w.B * w.L * e2e_steps / (e2.elapsed_time(e3) / 1000.0)
+
+    scan_ms, scan_n = ktimes["state_scan"]
+    bwd_ms, bwd_n = ktimes["attention"]
+    flops = backward_flops(w)
+    sm_mhz = (clocks.summary() or {}).get("sm_max_mhz") or 1965
+    fp32_peak = 148 * 128 * 2 * sm_mhz * 1e6 / 1e12  # FMA lanes x 2 flop x max SM clock
+    achieved = flops / (bwd_ms / max(bwd_n, 1) / 1000.0) / 1e12
+    line = {
+        "metric": "Infini-attention backward tokens/s on 1 B200 (gradients through the segments)",
+        "value": value, "unit": "tokens/s", "n_gpus": 1, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": elapsed_ms / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": w.dtype,
+        "data": "synthetic (seeded Philox N(0,1) q/k/v and upstream gradients, U(-r,r) beta)",
+        "config": {"workload": f"{w.name} backward", "B": w.B, "H_q": w.H_q, "H_kv": w.H_kv,
+                   "L": w.L, "d_k": w.d_k, "d_v": w.d_v, "seg_len": w.seg_len,
+                   "rule": w.rule, "io_dtype": w.dtype, "grad_dtype": "f32",
+                   "l2": ("L2 flushed (256 MiB write) between timed steps; each step timed alone"
+                          if flush is not None else "inputs larger than L2")},
+        "clocks": clocks.summary(),
+        "e2e": {"value": e2e_value, "unit": "tokens/s",
+                "h2d_bytes_per_step": sum(t.numel() * t.element_size() for t in hp),
+                "d2h_bytes_per_step": sum(t.numel() * t.element_size() for t in outs_h),
+                "steps": e2e_steps},
+        "gpu_launches": None,
+        "roofline": {"bound": "alu", "kernel": "backward kernels (segment VJPs, reverse scan, gate)",
+                     "achieved": achieved, "peak": fp32_peak, "unit": "TFLOP/s",
+                     "frac": achieved / fp32_peak,
+                     "peak_source": "derived: 148 SMs x 128 fp32 FMA lanes x 2 flop x max SM clock",
+                     "traffic": None, "algorithmic_flops_per_step": flops,
+                     "avg_launch_ms": bwd_ms / max(bwd_n, 1)},
+        "kernel_ms": {"state_recompute": scan_ms / max(scan_n, 1),
+                      "backward": bwd_ms / max(bwd_n, 1)},
+    }
+    plan = api.plan(dims, w.seg_len, w.rule)
+    line["gpu_launches"] = (plan["launches"] - 1 + 3) * args.steps
+    if args.cpu_baseline:
+        v, desc = oracle_backward_sample(w, args.cpu_budget)
+        line["cpu_baseline"] = {"value": v, "unit": "tokens/s", "cores": host_cores(),
+                                "kind": "oracle", "sample": desc}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -772,6 +955,9 @@ def main():
                          "rank (strong scaling)")
     ap.add_argument("--seq-parallel", action="store_true",
                     help="sequence-parallel linear rule over the ranks (strong scaling)")
+    ap.add_argument("--backward", action="store_true",
+                    help="the backward through the segments (gradients of every input); "
+                         "short-segment shapes (seg_len <= 64, d in {32, 64})")
     ap.add_argument("--decode", action="store_true",
                     help="streaming decode (one token per call) of the workload's shape; "
                          "a step is one full segment")
@@ -791,6 +977,8 @@ def main():
         return run_decode_probe(args, w)
     if args.decode:
         return run_decode(args, w)
+    if args.backward:
+        return run_backward(args, w)
     if args.seq_parallel:
         return run_seq_parallel(args, w)
     return run_gpu(args, w)
