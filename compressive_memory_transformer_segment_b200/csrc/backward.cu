@@ -90,6 +90,83 @@ __device__ __forceinline__ void for_tile(const float (&acc)[NR / 16][NC / 16], F
     for (int v = 0; v < NC / 16; ++v) f(ti + 16 * u, tj + 16 * v, acc[u][v]);
 }
 
+// The 64 x 64 product with 128-bit shared loads, for K a multiple of 4 and
+// leading dimensions a multiple of 4 floats: per four kk, four float4 loads
+// of A and four of B feed 64 FMAs.  Thread (ti, tj) = (tid / 16, tid % 16):
+// its rows are ti + 16u (A row-major: a float4 runs along kk) or 4ti + u
+// (TA: a float4 runs along the rows), its columns 4tj + v (B row-major) or
+// tj + 16v (TB: a float4 runs along kk).  A warp's B loads are 16 distinct
+// 16-byte pieces in two wavefronts either way.
+template <bool TA, bool TB>
+__device__ __forceinline__ int vrow(int u) {
+  return TA ? 4 * (threadIdx.x >> 4) + u : (threadIdx.x >> 4) + 16 * u;
+}
+template <bool TA, bool TB>
+__device__ __forceinline__ int vcol(int v) {
+  return TB ? (threadIdx.x & 15) + 16 * v : 4 * (threadIdx.x & 15) + v;
+}
+
+template <bool TA, bool TB>
+__device__ __forceinline__ void mm_tile_v(const float* __restrict__ A, int lda,
+                                          const float* __restrict__ B, int ldb, int K,
+                                          float (&acc)[4][4]) {
+  const int ti = threadIdx.x >> 4, tj = threadIdx.x & 15;
+#pragma unroll 2
+  for (int k4 = 0; k4 < K; k4 += 4) {
+    float a[4][4], b[4][4];  // a[u][t] = A(row u, k4 + t), b[t][v] = B(k4 + t, col v)
+#pragma unroll
+    for (int x = 0; x < 4; ++x) {
+      if (TA) {  // A[(k4 + x) * lda + 4ti .. + 3]: rows 4ti + u at kk = k4 + x
+        const float4 f = *reinterpret_cast<const float4*>(A + (k4 + x) * lda + 4 * ti);
+        a[0][x] = f.x; a[1][x] = f.y; a[2][x] = f.z; a[3][x] = f.w;
+      } else {   // A[(ti + 16x) * lda + k4 .. + 3]: row ti + 16x
+        const float4 f = *reinterpret_cast<const float4*>(A + (ti + 16 * x) * lda + k4);
+        a[x][0] = f.x; a[x][1] = f.y; a[x][2] = f.z; a[x][3] = f.w;
+      }
+      if (TB) {  // B[(tj + 16x) * ldb + k4 .. + 3]: column tj + 16x
+        const float4 f = *reinterpret_cast<const float4*>(B + (tj + 16 * x) * ldb + k4);
+        b[0][x] = f.x; b[1][x] = f.y; b[2][x] = f.z; b[3][x] = f.w;
+      } else {   // B[(k4 + x) * ldb + 4tj .. + 3]: columns 4tj + v at kk = k4 + x
+        const float4 f = *reinterpret_cast<const float4*>(B + (k4 + x) * ldb + 4 * tj);
+        b[x][0] = f.x; b[x][1] = f.y; b[x][2] = f.z; b[x][3] = f.w;
+      }
+    }
+#pragma unroll
+    for (int t = 0; t < 4; ++t)
+#pragma unroll
+      for (int u = 0; u < 4; ++u)
+#pragma unroll
+        for (int v = 0; v < 4; ++v) acc[u][v] = fmaf(a[u][t], b[t][v], acc[u][v]);
+  }
+}
+
+// C = A B (NR x NC, over kk < K) handed to f(i, j, value) element by element:
+// the 128-bit path where it applies (64 x 64, K % 4 == 0), else mm_tile.
+// With a second pair (A2, B2) the two products are summed (same shapes).
+template <int NR, int NC, bool TA, bool TB, typename F>
+__device__ __forceinline__ void product(const float* __restrict__ A, int lda,
+                                        const float* __restrict__ B, int ldb, int K, F&& f,
+                                        const float* __restrict__ A2 = nullptr,
+                                        const float* __restrict__ B2 = nullptr, int lda2 = 0,
+                                        int ldb2 = 0) {
+  if (NR == 64 && NC == 64 && (K & 3) == 0) {
+    float acc[4][4];
+    zero_tile<64, 64>(acc);
+    mm_tile_v<TA, TB>(A, lda, B, ldb, K, acc);
+    if (A2) mm_tile_v<TA, TB>(A2, lda2, B2, ldb2, K, acc);
+#pragma unroll
+    for (int u = 0; u < 4; ++u)
+#pragma unroll
+      for (int v = 0; v < 4; ++v) f(vrow<TA, TB>(u), vcol<TA, TB>(v), acc[u][v]);
+    return;
+  }
+  float acc[NR / 16][NC / 16];
+  zero_tile<NR, NC>(acc);
+  mm_tile<NR, NC, TA, TB>(A, lda, B, ldb, K, acc);
+  if (A2) mm_tile<NR, NC, TA, TB>(A2, lda2, B2, ldb2, K, acc);
+  for_tile<NR, NC>(acc, f);
+}
+
 // 16-byte pieces of a contiguous [rows][D] slice (element type T): the
 // thread's pieces of the first `count` elements are loaded into registers
 // first (all loads in flight together), then unpacked into a shared tile of
@@ -132,12 +209,13 @@ struct TileLoad {
 };
 
 // Shared-memory plan of bwd_segment (floats): n x D tiles with row stride
-// D + 1 (rows and columns are both read across lanes without conflicts),
-// n x n tiles with stride kBwdMaxS + 1.
+// D + 4, n x n tiles with stride kBwdMaxS + 4 (16-byte aligned rows for the
+// 128-bit loads; rows and columns are both read across lanes at most two
+// wavefronts deep).
 template <int D>
 struct SegSmem {
-  static constexpr int kLd = D + 1;
-  static constexpr int kLp = kBwdMaxS + 1;
+  static constexpr int kLd = D + 4;
+  static constexpr int kLp = kBwdMaxS + 4;
   static constexpr int kTile = kBwdMaxS * kLd;
   static constexpr int kQ = 0, kK = kQ + kTile, kV = kK + kTile, kDO = kV + kTile;
   static constexpr int kM = kDO + kTile;            // [D][D + 1]
@@ -164,7 +242,7 @@ bwd_segment(const T* __restrict__ q, const T* __restrict__ k, const T* __restric
             int H_q, int H_kv, int L, int S, int T_seg) {
   using SM = SegSmem<D>;
   constexpr int ld = SM::kLd, lp = SM::kLp;
-  extern __shared__ float sm[];
+  extern __shared__ __align__(16) float sm[];
   float *Q = sm + SM::kQ, *K = sm + SM::kK, *V = sm + SM::kV, *dO = sm + SM::kDO;
   float *M = sm + SM::kM, *X = sm + SM::kX, *Am = sm + SM::kAm, *Y = sm + SM::kY;
   float *P = sm + SM::kP, *dS = sm + SM::kDS, *z = sm + SM::kZ, *den = sm + SM::kDen;
@@ -214,20 +292,14 @@ bwd_segment(const T* __restrict__ q, const T* __restrict__ k, const T* __restric
   constexpr int N = kBwdMaxS;  // tile extent of the segment's rows
   // scores, masked (key j <= row i)
   {
-    float acc[N / 16][N / 16];
-    zero_tile<N, N>(acc);
-    mm_tile<N, N, false, true>(Q, ld, K, ld, D, acc);
-    for_tile<N, N>(acc, [&](int i, int j, float x) {
+    product<N, N, false, true>(Q, ld, K, ld, D, [&](int i, int j, float x) {
       if (i < n && j < n) P[i * lp + j] = j <= i ? x * scale : -INFINITY;
     });
   }
   __syncthreads();
   // A_mem = sigma(Q) M / den (0 where den = 0); row softmax of the scores
   {
-    float acc[N / 16][D / 16];
-    zero_tile<N, D>(acc);
-    mm_tile<N, D, false, false>(X, ld, M, ld, D, acc);
-    for_tile<N, D>(acc, [&](int i, int c, float x) {
+    product<N, D, false, false>(X, ld, M, ld, D, [&](int i, int c, float x) {
       if (i < n) Am[i * ld + c] = den[i] != 0.f ? x / den[i] : 0.f;
     });
   }
@@ -250,10 +322,7 @@ bwd_segment(const T* __restrict__ q, const T* __restrict__ k, const T* __restric
   // sum(dout (A_mem - A_dot))
   float part = 0.f;
   {
-    float acc[N / 16][D / 16];
-    zero_tile<N, D>(acc);
-    mm_tile<N, D, false, false>(P, lp, V, ld, n, acc);
-    for_tile<N, D>(acc, [&](int i, int c, float x) {
+    product<N, D, false, false>(P, lp, V, ld, n, [&](int i, int c, float x) {
       if (i < n) part = fmaf(dO[i * ld + c], Am[i * ld + c] - x, part);
     });
   }
@@ -280,10 +349,7 @@ bwd_segment(const T* __restrict__ q, const T* __restrict__ k, const T* __restric
   // Retrieval: dM_{s-1} += sigma(Q)^T dnum, dz_{s-1} += sigma(Q)^T dden
   {
     float* dMo = dMr + ((size_t)s * BHq + bh) * D * D;
-    float acc[D / 16][D / 16];
-    zero_tile<D, D>(acc);
-    mm_tile<D, D, true, false>(X, ld, Y, ld, n, acc);
-    for_tile<D, D>(acc, [&](int kk, int c, float x) { dMo[kk * D + c] = x; });
+    product<D, D, true, false>(X, ld, Y, ld, n, [&](int kk, int c, float x) { dMo[kk * D + c] = x; });
   }
   for (int kk = tid; kk < D; kk += kBwdThreads) {
     float a = 0.f;
@@ -292,30 +358,21 @@ bwd_segment(const T* __restrict__ q, const T* __restrict__ k, const T* __restric
   }
   // dQ (retrieval part) = (dnum M^T + dden z^T) sigma'(Q), into Am
   {
-    float acc[N / 16][D / 16];
-    zero_tile<N, D>(acc);
-    mm_tile<N, D, false, true>(Y, ld, M, ld, D, acc);
-    for_tile<N, D>(acc, [&](int i, int kk, float x) {
+    product<N, D, false, true>(Y, ld, M, ld, D, [&](int i, int kk, float x) {
       if (i < n) Am[i * ld + kk] = fmaf(dden[i], z[kk], x) * elu1_grad(Q[i * ld + kk]);
     });
   }
   // Attention: dP = (1 - g) dout V^T (causal part only)
   const float ga = 1.f - g;
   {
-    float acc[N / 16][N / 16];
-    zero_tile<N, N>(acc);
-    mm_tile<N, N, false, true>(dO, ld, V, ld, D, acc);
-    for_tile<N, N>(acc, [&](int i, int j, float x) {
+    product<N, N, false, true>(dO, ld, V, ld, D, [&](int i, int j, float x) {
       if (i < n && j < n) dS[i * lp + j] = j <= i ? ga * x : 0.f;
     });
   }
   // dV (attention) = P^T dA_dot
   {
     float* dVo = dVa + ((size_t)bh * L + r0) * D;
-    float acc[N / 16][D / 16];
-    zero_tile<N, D>(acc);
-    mm_tile<N, D, true, false>(P, lp, dO, ld, n, acc);
-    for_tile<N, D>(acc, [&](int j, int c, float x) {
+    product<N, D, true, false>(P, lp, dO, ld, n, [&](int j, int c, float x) {
       if (j < n) dVo[j * D + c] = ga * x;
     });
   }
@@ -336,19 +393,13 @@ bwd_segment(const T* __restrict__ q, const T* __restrict__ k, const T* __restric
   // dq = dS K / sqrt(d) + retrieval part; dK (attention) = dS^T Q / sqrt(d)
   {
     float* dqo = dq + ((size_t)bh * L + r0) * D;
-    float acc[N / 16][D / 16];
-    zero_tile<N, D>(acc);
-    mm_tile<N, D, false, false>(dS, lp, K, ld, n, acc);
-    for_tile<N, D>(acc, [&](int i, int c, float x) {
+    product<N, D, false, false>(dS, lp, K, ld, n, [&](int i, int c, float x) {
       if (i < n) dqo[i * D + c] = fmaf(x, scale, Am[i * ld + c]);
     });
   }
   {
     float* dKo = dKa + ((size_t)bh * L + r0) * D;
-    float acc[N / 16][D / 16];
-    zero_tile<N, D>(acc);
-    mm_tile<N, D, true, false>(dS, lp, Q, ld, n, acc);
-    for_tile<N, D>(acc, [&](int j, int c, float x) {
+    product<N, D, true, false>(dS, lp, Q, ld, n, [&](int j, int c, float x) {
       if (j < n) dKo[j * D + c] = x * scale;
     });
   }
@@ -357,7 +408,7 @@ bwd_segment(const T* __restrict__ q, const T* __restrict__ k, const T* __restric
 // Shared-memory plan of bwd_scan (floats).
 template <int D>
 struct ScanBwdSmem {
-  static constexpr int kLd = D + 1;
+  static constexpr int kLd = D + 4;
   static constexpr int kTile = kBwdMaxS * kLd;
   static constexpr int kGM = 0;                    // [D][D + 1] dL/dM_s
   static constexpr int kM = kGM + D * kLd;         // M_{s-1}
@@ -385,7 +436,7 @@ bwd_scan(const T* __restrict__ k, const T* __restrict__ v, const float* __restri
          int T_seg) {
   using SM = ScanBwdSmem<D>;
   constexpr int ld = SM::kLd;
-  extern __shared__ float sm[];
+  extern __shared__ __align__(16) float sm[];
   float *GM = sm + SM::kGM, *M = sm + SM::kM, *sK = sm + SM::kSK, *V = sm + SM::kV;
   float *X1 = sm + SM::kX1, *X2 = sm + SM::kX2, *X3 = sm + SM::kX3, *X4 = sm + SM::kX4;
   float *Gz = sm + SM::kGz, *z = sm + SM::kZ, *r = sm + SM::kR, *dr = sm + SM::kDr;
@@ -431,15 +482,10 @@ bwd_scan(const T* __restrict__ k, const T* __restrict__ v, const float* __restri
       __syncthreads();
       // R = sigma(K) M / r (0 where r = 0); dU = sigma(K) G_M
       {
-        float acc[N / 16][D / 16];
-        zero_tile<N, D>(acc);
-        mm_tile<N, D, false, false>(sK, ld, M, ld, D, acc);
-        for_tile<N, D>(acc, [&](int i, int c, float x) {
+        product<N, D, false, false>(sK, ld, M, ld, D, [&](int i, int c, float x) {
           if (i < n) X3[i * ld + c] = r[i] != 0.f ? x / r[i] : 0.f;
         });
-        zero_tile<N, D>(acc);
-        mm_tile<N, D, false, false>(sK, ld, GM, ld, D, acc);
-        for_tile<N, D>(acc, [&](int i, int c, float x) {
+        product<N, D, false, false>(sK, ld, GM, ld, D, [&](int i, int c, float x) {
           if (i < n) X2[i * ld + c] = x;
         });
       }
@@ -461,21 +507,14 @@ bwd_scan(const T* __restrict__ k, const T* __restrict__ v, const float* __restri
       __syncthreads();
       // d sigma(K) = U G_M^T + dN M^T + dr z^T + G_z
       {
-        float acc[N / 16][D / 16];
-        zero_tile<N, D>(acc);
-        mm_tile<N, D, false, true>(X3, ld, GM, ld, D, acc);
-        mm_tile<N, D, false, true>(X4, ld, M, ld, D, acc);
-        for_tile<N, D>(acc, [&](int i, int kk, float x) {
+        product<N, D, false, true>(X3, ld, GM, ld, D, [&](int i, int kk, float x) {
           if (i < n) X1[i * ld + kk] = x + fmaf(dr[i], z[kk], Gz[kk]);
-        });
+        }, X4, M, ld, ld);
       }
       __syncthreads();
       // G_M += sigma(K)^T dN, G_z += sigma(K)^T dr
       {
-        float acc[D / 16][D / 16];
-        zero_tile<D, D>(acc);
-        mm_tile<D, D, true, false>(sK, ld, X4, ld, n, acc);
-        for_tile<D, D>(acc, [&](int kk, int c, float x) { GM[kk * ld + c] += x; });
+        product<D, D, true, false>(sK, ld, X4, ld, n, [&](int kk, int c, float x) { GM[kk * ld + c] += x; });
       }
       for (int kk = tid; kk < D; kk += kBwdThreads) {
         float a = 0.f;
@@ -484,15 +523,10 @@ bwd_scan(const T* __restrict__ k, const T* __restrict__ v, const float* __restri
       }
     } else {
       // d sigma(K) = V G_M^T + G_z, dV = sigma(K) G_M
-      float acc[N / 16][D / 16];
-      zero_tile<N, D>(acc);
-      mm_tile<N, D, false, true>(V, ld, GM, ld, D, acc);
-      for_tile<N, D>(acc, [&](int i, int c, float x) {
+      product<N, D, false, true>(V, ld, GM, ld, D, [&](int i, int c, float x) {
         if (i < n) X1[i * ld + c] = x + Gz[c];
       });
-      zero_tile<N, D>(acc);
-      mm_tile<N, D, false, false>(sK, ld, GM, ld, D, acc);
-      for_tile<N, D>(acc, [&](int i, int c, float x) {
+      product<N, D, false, false>(sK, ld, GM, ld, D, [&](int i, int c, float x) {
         if (i < n) X2[i * ld + c] = x;
       });
     }
