@@ -39,14 +39,16 @@ namespace infini {
 
 namespace {
 
-constexpr int kBwdThreads = 256;
+constexpr int kBwdThreads = 256;  // reverse scan, gate sum; one product group
+constexpr int kSegThreads = 512;  // bwd_segment: two product groups
 constexpr int kBwdMaxS = 64;
 
 __device__ __forceinline__ float elu1_grad(float x) { return x > 0.f ? 1.f : expf(x); }
 
 // C = A B over kk < K for the calling thread's block of an NR x NC output
 // (NR, NC in {32, 64}): rows i = ti + 16u (u < NR/16), columns j = tj + 16v
-// (v < NC/16), thread (ti, tj) = (tid / 16, tid % 16) of 256.
+// (v < NC/16), thread (ti, tj) = (t / 16, t % 16) of a group of 256 threads
+// (t = tid % 256; a 512-thread CTA runs two products at once).
 // A(i, kk) = A[i * lda + kk], or A[kk * lda + i] when TA; B(kk, j) =
 // B[kk * ldb + j], or B[j * ldb + kk] when TB.  Per kk, NR/16 + NC/16 shared
 // loads feed NR NC / 256 FMAs (16 for 64 x 64); a warp's loads of B touch 16
@@ -57,7 +59,7 @@ template <int NR, int NC, bool TA, bool TB>
 __device__ __forceinline__ void mm_tile(const float* __restrict__ A, int lda,
                                         const float* __restrict__ B, int ldb, int K,
                                         float (&acc)[NR / 16][NC / 16]) {
-  const int ti = threadIdx.x >> 4, tj = threadIdx.x & 15;
+  const int ti = (threadIdx.x & 255) >> 4, tj = threadIdx.x & 15;
 #pragma unroll 4
   for (int kk = 0; kk < K; ++kk) {
     float a[NR / 16], b[NC / 16];
@@ -83,7 +85,7 @@ __device__ __forceinline__ void zero_tile(float (&acc)[NR / 16][NC / 16]) {
 // Calls f(i, j, value) for the thread's elements of an NR x NC tile result.
 template <int NR, int NC, typename F>
 __device__ __forceinline__ void for_tile(const float (&acc)[NR / 16][NC / 16], F&& f) {
-  const int ti = threadIdx.x >> 4, tj = threadIdx.x & 15;
+  const int ti = (threadIdx.x & 255) >> 4, tj = threadIdx.x & 15;
 #pragma unroll
   for (int u = 0; u < NR / 16; ++u)
 #pragma unroll
@@ -99,7 +101,7 @@ __device__ __forceinline__ void for_tile(const float (&acc)[NR / 16][NC / 16], F
 // 16-byte pieces in two wavefronts either way.
 template <bool TA, bool TB>
 __device__ __forceinline__ int vrow(int u) {
-  return TA ? 4 * (threadIdx.x >> 4) + u : (threadIdx.x >> 4) + 16 * u;
+  return TA ? 4 * ((threadIdx.x & 255) >> 4) + u : ((threadIdx.x & 255) >> 4) + 16 * u;
 }
 template <bool TA, bool TB>
 __device__ __forceinline__ int vcol(int v) {
@@ -110,7 +112,7 @@ template <bool TA, bool TB>
 __device__ __forceinline__ void mm_tile_v(const float* __restrict__ A, int lda,
                                           const float* __restrict__ B, int ldb, int K,
                                           float (&acc)[4][4]) {
-  const int ti = threadIdx.x >> 4, tj = threadIdx.x & 15;
+  const int ti = (threadIdx.x & 255) >> 4, tj = threadIdx.x & 15;
 #pragma unroll 2
   for (int k4 = 0; k4 < K; k4 += 4) {
     float a[4][4], b[4][4];  // a[u][t] = A(row u, k4 + t), b[t][v] = B(k4 + t, col v)
@@ -171,22 +173,22 @@ __device__ __forceinline__ void product(const float* __restrict__ A, int lda,
 // thread's pieces of the first `count` elements are loaded into registers
 // first (all loads in flight together), then unpacked into a shared tile of
 // row stride ld.
-template <typename T, int D, int ROWS>
+template <typename T, int D, int ROWS, int NT = kBwdThreads>
 struct TileLoad {
   static constexpr int kVec = 16 / (int)sizeof(T);
-  static constexpr int kPer = (ROWS * D / kVec + kBwdThreads - 1) / kBwdThreads;
+  static constexpr int kPer = (ROWS * D / kVec + NT - 1) / NT;
   uint4 raw[kPer];
   __device__ __forceinline__ void issue(const T* __restrict__ src, int count) {
 #pragma unroll
     for (int u = 0; u < kPer; ++u) {
-      const int e = threadIdx.x + u * kBwdThreads;
+      const int e = threadIdx.x + u * NT;
       raw[u] = e * kVec < count ? reinterpret_cast<const uint4*>(src)[e] : make_uint4(0, 0, 0, 0);
     }
   }
   __device__ __forceinline__ void store(float* dst, int ld, int count) const {
 #pragma unroll
     for (int u = 0; u < kPer; ++u) {
-      const int e = (threadIdx.x + u * kBwdThreads) * kVec;
+      const int e = (threadIdx.x + u * NT) * kVec;
       if (e >= count) continue;
       const T* x = reinterpret_cast<const T*>(&raw[u]);
       const int i = e / D, c = e % D;  // kVec divides D: one row per piece
@@ -198,7 +200,7 @@ struct TileLoad {
   __device__ __forceinline__ void add(float* dst, int ld, int count) const {
 #pragma unroll
     for (int u = 0; u < kPer; ++u) {
-      const int e = (threadIdx.x + u * kBwdThreads) * kVec;
+      const int e = (threadIdx.x + u * NT) * kVec;
       if (e >= count) continue;
       const float* x = reinterpret_cast<const float*>(&raw[u]);
       const int i = e / D, c = e % D;
@@ -229,11 +231,14 @@ struct SegSmem {
   static constexpr int kDden = kDen + kBwdMaxS;
   static constexpr int kRs = kDden + kBwdMaxS;
   static constexpr int kRed = kRs + kBwdMaxS;       // block reduction
-  static constexpr int kTotal = kRed + kBwdThreads / 32;
+  static constexpr int kTotal = kRed + kSegThreads / 32;
 };
 
+// Thread groups: threads 0..255 (group 0) and 256..511 (group 1) run
+// independent products of a phase side by side; row reductions use all 16
+// warps.
 template <typename T, int D>
-__global__ void __launch_bounds__(kBwdThreads)
+__global__ void __launch_bounds__(kSegThreads)
 bwd_segment(const T* __restrict__ q, const T* __restrict__ k, const T* __restrict__ v,
             const float* __restrict__ beta, const T* __restrict__ dout,
             const float* __restrict__ Mf, const float* __restrict__ zf,
@@ -242,6 +247,7 @@ bwd_segment(const T* __restrict__ q, const T* __restrict__ k, const T* __restric
             int H_q, int H_kv, int L, int S, int T_seg) {
   using SM = SegSmem<D>;
   constexpr int ld = SM::kLd, lp = SM::kLp;
+  constexpr int kWarps = kSegThreads / 32;
   extern __shared__ __align__(16) float sm[];
   float *Q = sm + SM::kQ, *K = sm + SM::kK, *V = sm + SM::kV, *dO = sm + SM::kDO;
   float *M = sm + SM::kM, *X = sm + SM::kX, *Am = sm + SM::kAm, *Y = sm + SM::kY;
@@ -253,8 +259,11 @@ bwd_segment(const T* __restrict__ q, const T* __restrict__ k, const T* __restric
   const int BHq = gridDim.y, BHkv = BHq / H_q * H_kv;
   const int r0 = s * S, n = min(S, L - r0);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int grp = tid >> 8, gt = tid & 255;
   const float scale = rsqrtf((float)D);
   const float g = gate_sigmoid(beta[h]);
+  const float ga = 1.f - g;
+  constexpr int N = kBwdMaxS;  // tile extent of the segment's rows
 
   // ---- loads (rows past the segment stay out of every sum: loops run to n)
   const T* qs = q + ((size_t)bh * L + r0) * D;
@@ -262,14 +271,14 @@ bwd_segment(const T* __restrict__ q, const T* __restrict__ k, const T* __restric
   const T* vs = v + ((size_t)bhkv * L + r0) * D;
   const T* ds = dout + ((size_t)bh * L + r0) * D;
   {
-    TileLoad<T, D, kBwdMaxS> lq, lk, lv, ld_o;
-    TileLoad<float, D, D> lm;
+    TileLoad<T, D, kBwdMaxS, kSegThreads> lq, lk, lv, ld_o;
+    TileLoad<float, D, D, kSegThreads> lm;
     lq.issue(qs, n * D);
     lk.issue(ks, n * D);
     lv.issue(vs, n * D);
     ld_o.issue(ds, n * D);
     lm.issue(Mf + ((size_t)s * BHkv + bhkv) * D * D, D * D);
-    for (int c = tid; c < D; c += kBwdThreads) z[c] = zf[((size_t)s * BHkv + bhkv) * D + c];
+    for (int c = tid; c < D; c += kSegThreads) z[c] = zf[((size_t)s * BHkv + bhkv) * D + c];
     lq.store(Q, ld, n * D);
     lk.store(K, ld, n * D);
     lv.store(V, ld, n * D);
@@ -277,33 +286,33 @@ bwd_segment(const T* __restrict__ q, const T* __restrict__ k, const T* __restric
     lm.store(M, ld, D * D);
   }
   __syncthreads();
-  for (int e = tid; e < n * D; e += kBwdThreads) {
+  for (int e = tid; e < n * D; e += kSegThreads) {
     const int i = e / D, c = e % D;
     X[i * ld + c] = elu1(Q[i * ld + c]);
   }
   __syncthreads();
   // den_i = sigma(q_i) . z
-  for (int i = warp; i < n; i += kBwdThreads / 32) {
+  for (int i = warp; i < n; i += kWarps) {
     float a = 0.f;
     for (int c = lane; c < D; c += 32) a = fmaf(X[i * ld + c], z[c], a);
     a = warp_sum(a);
     if (lane == 0) den[i] = a;
   }
-  constexpr int N = kBwdMaxS;  // tile extent of the segment's rows
-  // scores, masked (key j <= row i)
-  {
+  __syncthreads();
+  if (grp == 0) {
+    // scores, masked (key j <= row i)
     product<N, N, false, true>(Q, ld, K, ld, D, [&](int i, int j, float x) {
       if (i < n && j < n) P[i * lp + j] = j <= i ? x * scale : -INFINITY;
     });
-  }
-  __syncthreads();
-  // A_mem = sigma(Q) M / den (0 where den = 0); row softmax of the scores
-  {
+  } else {
+    // A_mem = sigma(Q) M / den (0 where den = 0)
     product<N, D, false, false>(X, ld, M, ld, D, [&](int i, int c, float x) {
       if (i < n) Am[i * ld + c] = den[i] != 0.f ? x / den[i] : 0.f;
     });
   }
-  for (int i = warp; i < n; i += kBwdThreads / 32) {
+  __syncthreads();
+  // row softmax of the scores
+  for (int i = warp; i < n; i += kWarps) {
     float m = -INFINITY;
     for (int j = lane; j < n; j += 32) m = fmaxf(m, P[i * lp + j]);
     m = warp_max(m);
@@ -318,86 +327,80 @@ bwd_segment(const T* __restrict__ q, const T* __restrict__ k, const T* __restric
     for (int j = lane; j < n; j += 32) P[i * lp + j] *= inv;
   }
   __syncthreads();
-  // A_dot = P V (P is 0 right of the diagonal), and the gate's partial
-  // sum(dout (A_mem - A_dot))
-  float part = 0.f;
-  {
+  if (grp == 0) {
+    // A_dot = P V (P is 0 right of the diagonal), and the gate's partial
+    // sum(dout (A_mem - A_dot))
+    float part = 0.f;
     product<N, D, false, false>(P, lp, V, ld, n, [&](int i, int c, float x) {
       if (i < n) part = fmaf(dO[i * ld + c], Am[i * ld + c] - x, part);
     });
-  }
-  part = warp_sum(part);
-  if (lane == 0) red[warp] = part;
-  // dden_i = -sum_c g dout A_mem / den
-  for (int i = warp; i < n; i += kBwdThreads / 32) {
-    float a = 0.f;
-    for (int c = lane; c < D; c += 32) a = fmaf(dO[i * ld + c], Am[i * ld + c], a);
-    a = warp_sum(a);
-    if (lane == 0) dden[i] = den[i] != 0.f ? -g * a / den[i] : 0.f;
-  }
-  // dnum = g dout / den
-  for (int e = tid; e < n * D; e += kBwdThreads) {
-    const int i = e / D, c = e % D;
-    Y[i * ld + c] = den[i] != 0.f ? g * dO[i * ld + c] / den[i] : 0.f;
+    part = warp_sum(part);
+    if (lane == 0) red[warp] = part;
+  } else {
+    // dden_i = -sum_c g dout A_mem / den; dnum = g dout / den
+    for (int i = warp - kWarps / 2; i < n; i += kWarps / 2) {
+      float a = 0.f;
+      for (int c = lane; c < D; c += 32) a = fmaf(dO[i * ld + c], Am[i * ld + c], a);
+      a = warp_sum(a);
+      if (lane == 0) dden[i] = den[i] != 0.f ? -g * a / den[i] : 0.f;
+    }
+    for (int e = gt; e < n * D; e += 256) {
+      const int i = e / D, c = e % D;
+      Y[i * ld + c] = den[i] != 0.f ? g * dO[i * ld + c] / den[i] : 0.f;
+    }
   }
   __syncthreads();
   if (tid == 0) {
     float a = 0.f;
-    for (int w = 0; w < kBwdThreads / 32; ++w) a += red[w];
+    for (int w = 0; w < kWarps / 2; ++w) a += red[w];
     dbp[(size_t)bh * T_seg + s] = a * g * (1.f - g);
   }
-  // Retrieval: dM_{s-1} += sigma(Q)^T dnum, dz_{s-1} += sigma(Q)^T dden
-  {
+  if (grp == 0) {
+    // Retrieval: dM_{s-1} += sigma(Q)^T dnum; dQ (retrieval part) =
+    // (dnum M^T + dden z^T) sigma'(Q), into Am
     float* dMo = dMr + ((size_t)s * BHq + bh) * D * D;
     product<D, D, true, false>(X, ld, Y, ld, n, [&](int kk, int c, float x) { dMo[kk * D + c] = x; });
-  }
-  for (int kk = tid; kk < D; kk += kBwdThreads) {
-    float a = 0.f;
-    for (int i = 0; i < n; ++i) a = fmaf(X[i * ld + kk], dden[i], a);
-    dzr[((size_t)s * BHq + bh) * D + kk] = a;
-  }
-  // dQ (retrieval part) = (dnum M^T + dden z^T) sigma'(Q), into Am
-  {
     product<N, D, false, true>(Y, ld, M, ld, D, [&](int i, int kk, float x) {
       if (i < n) Am[i * ld + kk] = fmaf(dden[i], z[kk], x) * elu1_grad(Q[i * ld + kk]);
     });
-  }
-  // Attention: dP = (1 - g) dout V^T (causal part only)
-  const float ga = 1.f - g;
-  {
+  } else {
+    // Attention: dP = (1 - g) dout V^T (causal part only); dV = P^T dA_dot;
+    // dz_{s-1} += sigma(Q)^T dden
     product<N, N, false, true>(dO, ld, V, ld, D, [&](int i, int j, float x) {
       if (i < n && j < n) dS[i * lp + j] = j <= i ? ga * x : 0.f;
     });
-  }
-  // dV (attention) = P^T dA_dot
-  {
     float* dVo = dVa + ((size_t)bh * L + r0) * D;
     product<N, D, true, false>(P, lp, dO, ld, n, [&](int j, int c, float x) {
       if (j < n) dVo[j * D + c] = ga * x;
     });
+    for (int kk = gt; kk < D; kk += 256) {
+      float a = 0.f;
+      for (int i = 0; i < n; ++i) a = fmaf(X[i * ld + kk], dden[i], a);
+      dzr[((size_t)s * BHq + bh) * D + kk] = a;
+    }
   }
   __syncthreads();
   // dS = P (dP - rowsum(dP P))
-  for (int i = warp; i < n; i += kBwdThreads / 32) {
+  for (int i = warp; i < n; i += kWarps) {
     float a = 0.f;
     for (int j = lane; j <= i; j += 32) a = fmaf(dS[i * lp + j], P[i * lp + j], a);
     a = warp_sum(a);
     if (lane == 0) rs[i] = a;
   }
   __syncthreads();
-  for (int e = tid; e < n * n; e += kBwdThreads) {
+  for (int e = tid; e < n * n; e += kSegThreads) {
     const int i = e / n, j = e % n;
     dS[i * lp + j] = j <= i ? P[i * lp + j] * (dS[i * lp + j] - rs[i]) : 0.f;
   }
   __syncthreads();
-  // dq = dS K / sqrt(d) + retrieval part; dK (attention) = dS^T Q / sqrt(d)
-  {
+  if (grp == 0) {
+    // dq = dS K / sqrt(d) + retrieval part
     float* dqo = dq + ((size_t)bh * L + r0) * D;
     product<N, D, false, false>(dS, lp, K, ld, n, [&](int i, int c, float x) {
       if (i < n) dqo[i * D + c] = fmaf(x, scale, Am[i * ld + c]);
     });
-  }
-  {
+  } else {
+    // dK (attention) = dS^T Q / sqrt(d)
     float* dKo = dKa + ((size_t)bh * L + r0) * D;
     product<N, D, true, false>(dS, lp, Q, ld, n, [&](int j, int c, float x) {
       if (j < n) dKo[j * D + c] = x * scale;
@@ -588,7 +591,7 @@ cudaError_t launch_bwd(const BackwardProblem& p, cudaStream_t st) {
   cudaError_t e = cudaFuncSetAttribute(bwd_segment<T, D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)seg_smem);
   if (e != cudaSuccess) return e;
-  bwd_segment<T, D><<<dim3(p.T, BHq), kBwdThreads, seg_smem, st>>>(
+  bwd_segment<T, D><<<dim3(p.T, BHq), kSegThreads, seg_smem, st>>>(
       static_cast<const T*>(p.q), static_cast<const T*>(p.k), static_cast<const T*>(p.v), p.beta,
       static_cast<const T*>(p.dout), p.Mf, p.zf, p.dq, p.dKa, p.dVa, p.dMr, p.dzr, p.dbp, p.H_q,
       p.H_kv, p.L, p.S, p.T);
