@@ -421,15 +421,19 @@ struct ScanBwdSmem {
   static constexpr int kX2 = kX1 + kTile;          // dV (= dU, delta)
   static constexpr int kX3 = kX2 + kTile;          // R, then U = V - R (delta)
   static constexpr int kX4 = kX3 + kTile;          // dN = -dU / r (delta)
-  static constexpr int kGz = kX4 + kTile;
+  static constexpr int kX5 = kX4 + kTile;          // sigma(K)^T dN (delta)
+  static constexpr int kGz = kX5 + kTile;
   static constexpr int kZ = kGz + D;
   static constexpr int kR = kZ + D;                // r_t (delta)
   static constexpr int kDr = kR + kBwdMaxS;        // dr_t (delta)
   static constexpr int kTotal = kDr + kBwdMaxS;
 };
 
+// 512 threads: two 256-thread groups run the independent products of a
+// phase side by side; the next segment's K, V (and M_{s-1}) are in flight in
+// registers while the current one is processed.
 template <typename T, int D, bool DELTA>
-__global__ void __launch_bounds__(kBwdThreads)
+__global__ void __launch_bounds__(kSegThreads)
 bwd_scan(const T* __restrict__ k, const T* __restrict__ v, const float* __restrict__ Mf,
          const float* __restrict__ zf, const float* __restrict__ dM_out,
          const float* __restrict__ dz_out, const float* __restrict__ dKa,
@@ -439,62 +443,67 @@ bwd_scan(const T* __restrict__ k, const T* __restrict__ v, const float* __restri
          int T_seg) {
   using SM = ScanBwdSmem<D>;
   constexpr int ld = SM::kLd;
+  constexpr int NT = kSegThreads, kWarps = NT / 32;
   extern __shared__ __align__(16) float sm[];
   float *GM = sm + SM::kGM, *M = sm + SM::kM, *sK = sm + SM::kSK, *V = sm + SM::kV;
   float *X1 = sm + SM::kX1, *X2 = sm + SM::kX2, *X3 = sm + SM::kX3, *X4 = sm + SM::kX4;
+  float *X5 = sm + SM::kX5;
   float *Gz = sm + SM::kGz, *z = sm + SM::kZ, *r = sm + SM::kR, *dr = sm + SM::kDr;
   const int bhkv = blockIdx.x, BHkv = gridDim.x;
   const int b = bhkv / H_kv, j = bhkv % H_kv, grp = H_q / H_kv;
   const int BHq = BHkv / H_kv * H_q;
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  for (int e = tid; e < D * D; e += kBwdThreads)
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, half = tid >> 8;
+  constexpr int N = kBwdMaxS;
+  for (int e = tid; e < D * D; e += NT)
     GM[(e / D) * ld + e % D] = dM_out ? dM_out[(size_t)bhkv * D * D + e] : 0.f;
-  for (int c = tid; c < D; c += kBwdThreads) Gz[c] = dz_out ? dz_out[(size_t)bhkv * D + c] : 0.f;
+  for (int c = tid; c < D; c += NT) Gz[c] = dz_out ? dz_out[(size_t)bhkv * D + c] : 0.f;
+  TileLoad<T, D, kBwdMaxS, NT> lk, lv;
+  TileLoad<float, D, D, NT> lm;
+  auto issue = [&](int s) {
+    const int r0 = s * S, n = min(S, L - r0);
+    lk.issue(k + ((size_t)bhkv * L + r0) * D, n * D);
+    lv.issue(v + ((size_t)bhkv * L + r0) * D, n * D);
+    if (DELTA) lm.issue(Mf + ((size_t)s * BHkv + bhkv) * D * D, D * D);
+  };
+  issue(T_seg - 1);
   for (int s = T_seg - 1; s >= 0; --s) {
     const int r0 = s * S, n = min(S, L - r0);
-    const T* ks = k + ((size_t)bhkv * L + r0) * D;
-    const T* vs = v + ((size_t)bhkv * L + r0) * D;
-    {
-      TileLoad<T, D, kBwdMaxS> lk, lv;
-      TileLoad<float, D, D> lm;
-      lk.issue(ks, n * D);
-      lv.issue(vs, n * D);
-      if (DELTA) {
-        lm.issue(Mf + ((size_t)s * BHkv + bhkv) * D * D, D * D);
-        for (int c = tid; c < D; c += kBwdThreads) z[c] = zf[((size_t)s * BHkv + bhkv) * D + c];
-      }
-      lk.store(sK, ld, n * D);
-      lv.store(V, ld, n * D);
-      if (DELTA) lm.store(M, ld, D * D);
+    lk.store(sK, ld, n * D);
+    lv.store(V, ld, n * D);
+    if (DELTA) {
+      lm.store(M, ld, D * D);
+      for (int c = tid; c < D; c += NT) z[c] = zf[((size_t)s * BHkv + bhkv) * D + c];
     }
     __syncthreads();
-    for (int e = tid; e < n * D; e += kBwdThreads) {
+    if (s > 0) issue(s - 1);
+    for (int e = tid; e < n * D; e += NT) {
       const int i = e / D, c = e % D;
       sK[i * ld + c] = elu1(sK[i * ld + c]);
     }
     __syncthreads();
-    constexpr int N = kBwdMaxS;
     if (DELTA) {
       // r_t = sigma(k_t) . z_{s-1}
-      for (int i = warp; i < n; i += kBwdThreads / 32) {
+      for (int i = warp; i < n; i += kWarps) {
         float a = 0.f;
         for (int c = lane; c < D; c += 32) a = fmaf(sK[i * ld + c], z[c], a);
         a = warp_sum(a);
         if (lane == 0) r[i] = a;
       }
       __syncthreads();
-      // R = sigma(K) M / r (0 where r = 0); dU = sigma(K) G_M
-      {
+      if (half == 0) {
+        // R = sigma(K) M / r (0 where r = 0)
         product<N, D, false, false>(sK, ld, M, ld, D, [&](int i, int c, float x) {
           if (i < n) X3[i * ld + c] = r[i] != 0.f ? x / r[i] : 0.f;
         });
+      } else {
+        // dU = sigma(K) G_M
         product<N, D, false, false>(sK, ld, GM, ld, D, [&](int i, int c, float x) {
           if (i < n) X2[i * ld + c] = x;
         });
       }
       __syncthreads();
       // dr_t = rowsum(dU R) / r
-      for (int i = warp; i < n; i += kBwdThreads / 32) {
+      for (int i = warp; i < n; i += kWarps) {
         float a = 0.f;
         for (int c = lane; c < D; c += 32) a = fmaf(X2[i * ld + c], X3[i * ld + c], a);
         a = warp_sum(a);
@@ -502,42 +511,50 @@ bwd_scan(const T* __restrict__ k, const T* __restrict__ v, const float* __restri
       }
       __syncthreads();
       // U = V - R (over R) and dN = -dU / r
-      for (int e = tid; e < n * D; e += kBwdThreads) {
+      for (int e = tid; e < n * D; e += NT) {
         const int i = e / D, c = e % D;
         X3[i * ld + c] = V[i * ld + c] - X3[i * ld + c];
         X4[i * ld + c] = r[i] != 0.f ? -X2[i * ld + c] / r[i] : 0.f;
       }
       __syncthreads();
-      // d sigma(K) = U G_M^T + dN M^T + dr z^T + G_z
-      {
+      if (half == 0) {
+        // d sigma(K) = U G_M^T + dN M^T + dr z^T + G_z
         product<N, D, false, true>(X3, ld, GM, ld, D, [&](int i, int kk, float x) {
           if (i < n) X1[i * ld + kk] = x + fmaf(dr[i], z[kk], Gz[kk]);
         }, X4, M, ld, ld);
+      } else {
+        // sigma(K)^T dN (added to G_M below, once G_M has been read)
+        product<D, D, true, false>(sK, ld, X4, ld, n, [&](int kk, int c, float x) { X5[kk * ld + c] = x; });
       }
       __syncthreads();
       // G_M += sigma(K)^T dN, G_z += sigma(K)^T dr
-      {
-        product<D, D, true, false>(sK, ld, X4, ld, n, [&](int kk, int c, float x) { GM[kk * ld + c] += x; });
+      for (int e = tid; e < D * D; e += NT) {
+        const int kk = e / D, c = e % D;
+        GM[kk * ld + c] += X5[kk * ld + c];
       }
-      for (int kk = tid; kk < D; kk += kBwdThreads) {
+      for (int kk = tid; kk < D; kk += NT) {
         float a = 0.f;
         for (int i = 0; i < n; ++i) a = fmaf(sK[i * ld + kk], dr[i], a);
         Gz[kk] += a;
       }
     } else {
-      // d sigma(K) = V G_M^T + G_z, dV = sigma(K) G_M
-      product<N, D, false, true>(V, ld, GM, ld, D, [&](int i, int c, float x) {
-        if (i < n) X1[i * ld + c] = x + Gz[c];
-      });
-      product<N, D, false, false>(sK, ld, GM, ld, D, [&](int i, int c, float x) {
-        if (i < n) X2[i * ld + c] = x;
-      });
+      if (half == 0) {
+        // d sigma(K) = V G_M^T + G_z
+        product<N, D, false, true>(V, ld, GM, ld, D, [&](int i, int c, float x) {
+          if (i < n) X1[i * ld + c] = x + Gz[c];
+        });
+      } else {
+        // dV = sigma(K) G_M
+        product<N, D, false, false>(sK, ld, GM, ld, D, [&](int i, int c, float x) {
+          if (i < n) X2[i * ld + c] = x;
+        });
+      }
     }
     __syncthreads();
     // dk, dv of the segment: the update's part (dk through sigma'(k) = 1 or
     // e^k = sigma(k)) plus every query head's attention part, added in head
     // order; and the heads' retrieval gradients with respect to M_{s-1}.
-    for (int e = tid; e < n * D; e += kBwdThreads) {
+    for (int e = tid; e < n * D; e += NT) {
       const int i = e / D, c = e % D;
       const float sk = sK[i * ld + c];
       X1[i * ld + c] *= sk > 1.f ? 1.f : sk;
@@ -545,8 +562,8 @@ bwd_scan(const T* __restrict__ k, const T* __restrict__ v, const float* __restri
     __syncthreads();
     for (int hh = 0; hh < grp; ++hh) {
       const size_t head = (size_t)(b * H_q + j * grp + hh);
-      TileLoad<float, D, kBwdMaxS> la, lb;
-      TileLoad<float, D, D> lr;
+      TileLoad<float, D, kBwdMaxS, NT> la, lb;
+      TileLoad<float, D, D, NT> lr;
       la.issue(dKa + (head * L + r0) * D, n * D);
       lb.issue(dVa + (head * L + r0) * D, n * D);
       lr.issue(dMr + ((size_t)s * BHq + head) * D * D, D * D);
@@ -555,22 +572,22 @@ bwd_scan(const T* __restrict__ k, const T* __restrict__ v, const float* __restri
       lr.add(GM, ld, D * D);
     }
     __syncthreads();
-    for (int e = tid; e < n * D; e += kBwdThreads) {
+    for (int e = tid; e < n * D; e += NT) {
       const int i = e / D, c = e % D;
       const size_t o = ((size_t)bhkv * L + r0 + i) * D + c;
       dk[o] = X1[i * ld + c];
       dv[o] = X2[i * ld + c];
     }
-    for (int c = tid; c < D; c += kBwdThreads) {
+    for (int c = tid; c < D; c += NT) {
       float a = 0.f;
       for (int hh = 0; hh < grp; ++hh) a += dzr[((size_t)s * BHq + b * H_q + j * grp + hh) * D + c];
       Gz[c] += a;
     }
     __syncthreads();
   }
-  for (int e = tid; e < D * D; e += kBwdThreads)
+  for (int e = tid; e < D * D; e += NT)
     dM_in[(size_t)bhkv * D * D + e] = GM[(e / D) * ld + e % D];
-  for (int c = tid; c < D; c += kBwdThreads) dz_in[(size_t)bhkv * D + c] = Gz[c];
+  for (int c = tid; c < D; c += NT) dz_in[(size_t)bhkv * D + c] = Gz[c];
 }
 
 // dbeta[h] = sum over batch rows and segments of the partials, in order.
@@ -601,7 +618,7 @@ cudaError_t launch_bwd(const BackwardProblem& p, cudaStream_t st) {
   if ((e = cudaFuncSetAttribute(scan, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)scan_smem)) !=
       cudaSuccess)
     return e;
-  scan<<<BHkv, kBwdThreads, scan_smem, st>>>(
+  scan<<<BHkv, kSegThreads, scan_smem, st>>>(
       static_cast<const T*>(p.k), static_cast<const T*>(p.v), p.Mf, p.zf, p.dM_out, p.dz_out, p.dKa,
       p.dVa, p.dMr, p.dzr, p.dk, p.dv, p.dM_in, p.dz_in, p.H_q, p.H_kv, p.L, p.S, p.T);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
