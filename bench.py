@@ -350,33 +350,42 @@ def run_gpu(args, w):
         step()
     api.sync_status(stream)
 
-    api.set_kernel_timing(True)
-    api.kernel_times(reset=True)
-    barrier()
-    torch.cuda.synchronize(dev)
-    with ClockSampler(local) as clocks:
-        if flush is None:
+    def timed_pass(n, flush_each):
+        """Device time of n steps (each alone after an L2 flush, or back to back)."""
+        if not flush_each:
             e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             e0.record(stream)
-            for _ in range(args.steps):
+            for _ in range(n):
                 step()
             e1.record(stream)
             torch.cuda.synchronize(dev)
-            elapsed_ms = e0.elapsed_time(e1)
-        else:
-            elapsed_ms = 0.0
-            for _ in range(args.steps):
-                flush.fill_(1)
-                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-                e0.record(stream)
-                step()
-                e1.record(stream)
-                torch.cuda.synchronize(dev)
-                elapsed_ms += e0.elapsed_time(e1)
-    barrier()
-    torch.cuda.synchronize(dev)
+            return e0.elapsed_time(e1)
+        total = 0.0
+        for _ in range(n):
+            flush.fill_(1)
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            step()
+            e1.record(stream)
+            torch.cuda.synchronize(dev)
+            total += e0.elapsed_time(e1)
+        return total
+
+    # Per-kernel device times come from a separate pass with events around the
+    # state scan and the attention: those events sit between the kernels and
+    # would add their own gaps to the timed steps.
+    api.set_kernel_timing(True)
+    api.kernel_times(reset=True)
+    timed_pass(args.steps, flush is not None)
     api.set_kernel_timing(False)
     ktimes = api.kernel_times(reset=True)
+    api.sync_status(stream)
+    barrier()
+    torch.cuda.synchronize(dev)
+    with ClockSampler(local) as clocks:
+        elapsed_ms = timed_pass(args.steps, flush is not None)
+    barrier()
+    torch.cuda.synchronize(dev)
     api.sync_status(stream)
 
     max_ms = shard.max_over_ranks(elapsed_ms, device=dev)
@@ -844,12 +853,10 @@ def run_backward(args, w):
     for _ in range(args.warmup):
         step()
     api.sync_status(stream)
-    api.set_kernel_timing(True)
-    api.kernel_times(reset=True)
-    torch.cuda.synchronize(dev)
-    elapsed_ms = 0.0
-    with ClockSampler(0) as clocks:
-        for _ in range(args.steps):
+
+    def timed_pass(n):
+        total = 0.0
+        for _ in range(n):
             if flush is not None:
                 flush.fill_(1)
             e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -857,9 +864,18 @@ def run_backward(args, w):
             step()
             e1.record(stream)
             torch.cuda.synchronize(dev)
-            elapsed_ms += e0.elapsed_time(e1)
+            total += e0.elapsed_time(e1)
+        return total
+
+    # Per-kernel times from a separate pass (their events would add gaps).
+    api.set_kernel_timing(True)
+    api.kernel_times(reset=True)
+    timed_pass(args.steps)
     api.set_kernel_timing(False)
     ktimes = api.kernel_times(reset=True)
+    torch.cuda.synchronize(dev)
+    with ClockSampler(0) as clocks:
+        elapsed_ms = timed_pass(args.steps)
     api.sync_status(stream)
     tokens = w.B * w.L * args.steps
     value = tokens / (elapsed_ms / 1000.0)

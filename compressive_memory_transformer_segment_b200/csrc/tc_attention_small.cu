@@ -32,6 +32,7 @@
 
 #include "kernels.h"
 #include "packed_math.cuh"
+#include "pdl.cuh"
 #include "tc_common.cuh"
 
 namespace infini {
@@ -143,6 +144,8 @@ tc_small_attention(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  pdl_trigger();
+  pdl_wait();  // (nothing above touched global memory)
 
   if (warp == 0) {
     // ------------------------------------------------ loads, MMAs, store
@@ -388,9 +391,8 @@ cudaError_t launch(const Problem& p, cudaStream_t stream) {
   auto kern = tc_small_attention<D, SPT>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
-  kern<<<(unsigned)grid, kThreads, smem, stream>>>(tq, tk, tv, tm, to, p.z_pref, p.beta, p.status, p.B,
-                                                   p.H_q, p.H_kv, p.L, p.T);
-  return cudaGetLastError();
+  return launch_pdl(true, kern, dim3((unsigned)grid), dim3(kThreads), smem, stream, tq, tk, tv, tm, to,
+                    (const float*)p.z_pref, p.beta, p.status, p.B, p.H_q, p.H_kv, p.L, p.T);
 }
 
 }  // namespace

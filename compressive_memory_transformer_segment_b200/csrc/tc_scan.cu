@@ -30,6 +30,7 @@
 
 #include "kernels.h"
 #include "packed_math.cuh"
+#include "pdl.cuh"
 #include "tc_common.cuh"
 
 namespace infini {
@@ -52,6 +53,8 @@ __global__ void __launch_bounds__(256) zsum(const __nv_bfloat16* __restrict__ k,
   constexpr int kCG = D / 8;      // 16-byte column groups per row
   constexpr int kNT = 256 / kCG;  // token lanes
   __shared__ float part[kNT * D];
+  pdl_trigger();
+  pdl_wait();
   const int s = blockIdx.x / C, c = blockIdx.x % C, bh = blockIdx.y, tid = threadIdx.x;
   const int cg = tid % kCG, tg = tid / kCG;
   const int chunk = (S + C - 1) / C;
@@ -91,6 +94,8 @@ __global__ void __launch_bounds__(128) zprefix(const float* __restrict__ dz, con
   const int bh = blockIdx.x, c = threadIdx.x, BH = gridDim.x;
   constexpr int kAhead = 16;
   const int n = T * C;
+  pdl_trigger();
+  pdl_wait();
   // (z_out may be z_in: this thread reads its entry before it writes it)
   float z = z_in[(size_t)bh * D + c], seg = 0.f;
   for (int i0 = 0; i0 < n; i0 += kAhead) {
@@ -263,6 +268,8 @@ tc_pipe_products(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  pdl_trigger();
+  pdl_wait();  // (nothing above touched global memory)
   // Accumulator a: G at 0 and B at 128 (delta), B at 0 and dz at 128 (linear).
   auto tG = [&](int a) { return tmem + a * SM::kAccCols; };
   auto tB = [&](int a) { return tmem + a * SM::kAccCols + (DELTA ? 128 : 0); };
@@ -530,6 +537,9 @@ __global__ void __launch_bounds__(D) combine_delta(const float* __restrict__ M_i
                                                    float* __restrict__ M_out, int T) {
   static_assert(kCB == 16 && D % 32 == 0, "combine_delta thread map");
   extern __shared__ __align__(16) float csm[];
+  // (The successor may launch only once the walk is done: CTAs parked in
+  // pdl_wait beside this latency-bound walk were measured to slow it.)
+  pdl_wait();
   float* sG = csm;               // two G_s buffers [D][D]
   float* sM = csm + 2 * D * D;   // M_{s-1}[:, 16 columns]
   const int bh = blockIdx.x, c0 = blockIdx.y * kCB, BH = gridDim.x;
@@ -598,6 +608,7 @@ __global__ void __launch_bounds__(D) combine_delta(const float* __restrict__ M_i
     }
     __syncthreads();
   }
+  pdl_trigger();
 #pragma unroll
   for (int i = 0; i < 4; ++i)
     *reinterpret_cast<float4*>(M_out + ((size_t)bh * D + k0 + i) * D + c0 + c) = m[i];
@@ -615,6 +626,8 @@ __global__ void __launch_bounds__(256) combine_linear(const float* __restrict__ 
                                                       float* __restrict__ z_pref,
                                                       float* __restrict__ M_out, float* z_out,
                                                       int T) {
+  pdl_trigger();
+  pdl_wait();
   const int bh = blockIdx.x, BH = gridDim.x;
   const int e = (blockIdx.y * 256 + threadIdx.x) * 4;  // element of the D x D matrix
   if (e < D * D) {
@@ -701,11 +714,15 @@ cudaError_t launch_pipe_products(const Problem& p, cudaStream_t stream) {
   if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
   const long items = (long)p.T * (long)BHkv;
   const int grid = (int)(items < sms ? items : sms);  // persistent: one CTA per SM
-  kern<<<grid, PipeSmem<D, DELTA>::kThreads, smem, stream>>>(lk, lv, p.z_pref, p.Gbuf, p.Bbuf, p.dz,
-                                                         p.status, p.L, p.S, p.T, (int)BHkv);
-  return cudaGetLastError();
+  return launch_pdl(!DELTA, kern, dim3(grid), dim3(PipeSmem<D, DELTA>::kThreads), smem, stream, lk, lv,
+                    (const float*)p.z_pref, p.Gbuf, p.Bbuf, p.dz, p.status, p.L, p.S, p.T, (int)BHkv);
 }
 
+// Launch chain.  The linear rule's kernels (products, combine) and the
+// attention after them are launched with programmatic dependent launch: the
+// next kernel's launch and prologue overlap the previous one's tail (200M
+// shape: 56 -> 52 us per forward).  The delta rule's chain is launched
+// plainly: with every link dependent, the forward took 129 us against 116.
 template <int D, typename MP>
 cudaError_t launch(const Problem& p, cudaStream_t stream) {
   const unsigned BH = (unsigned)((uint64_t)p.B * p.H_kv);
@@ -713,25 +730,25 @@ cudaError_t launch(const Problem& p, cudaStream_t stream) {
   cudaError_t e;
   if (p.delta) {
     const int C = zsum_chunks(p.S);
-    zsum<D><<<dim3(p.T * C, BH), 256, 0, stream>>>(static_cast<const __nv_bfloat16*>(p.k), p.dz, p.L,
-                                                   p.S, C);
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    zprefix<D><<<BH, D, 0, stream>>>(p.dz, p.z_in, p.z_pref, p.z_out, p.T, C);
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    if ((e = launch_pdl(false, zsum<D>, dim3(p.T * C, BH), dim3(256), 0, stream,
+                        static_cast<const __nv_bfloat16*>(p.k), p.dz, p.L, p.S, C)) != cudaSuccess)
+      return e;
+    if ((e = launch_pdl(false, zprefix<D>, dim3(BH), dim3(D), 0, stream, (const float*)p.dz, p.z_in, p.z_pref,
+                        p.z_out, p.T, C)) != cudaSuccess)
+      return e;
     e = launch_pipe_products<D, true>(p, stream);
     if (e != cudaSuccess) return e;
     const int csmem = (2 * D * D + D * kCB) * (int)sizeof(float);
     e = cudaFuncSetAttribute(combine_delta<D, MP>, cudaFuncAttributeMaxDynamicSharedMemorySize, csmem);
     if (e != cudaSuccess) return e;
-    combine_delta<D, MP><<<dim3(BH, D / kCB), D, csmem, stream>>>(p.M_in, p.Gbuf, p.Bbuf, Mp, p.M_out,
-                                                                 p.T);
-    return cudaGetLastError();
+    return launch_pdl(false, combine_delta<D, MP>, dim3(BH, D / kCB), dim3(D), csmem, stream, p.M_in,
+                      (const float*)p.Gbuf, (const float*)p.Bbuf, Mp, p.M_out, p.T);
   }
   e = launch_pipe_products<D, false>(p, stream);
   if (e != cudaSuccess) return e;
-  combine_linear<D, MP><<<dim3(BH, (D * D + 1023) / 1024), 256, 0, stream>>>(
-      p.M_in, p.Bbuf, p.dz, Mp, p.z_in, p.z_pref, p.M_out, p.z_out, p.T);
-  return cudaGetLastError();
+  return launch_pdl(true, combine_linear<D, MP>, dim3(BH, (D * D + 1023) / 1024), dim3(256), 0, stream,
+                    p.M_in, (const float*)p.Bbuf, (const float*)p.dz, Mp, p.z_in, p.z_pref, p.M_out,
+                    p.z_out, p.T);
 }
 
 }  // namespace
