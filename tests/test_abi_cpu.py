@@ -191,3 +191,24 @@ def test_state_sum_rejects_bad_arguments_on_the_host(lib):
     assert lib.infini_attn_state_sum(*base, P(0), 0, 2, 3, 8, 8, P(MB + 16), P(4 * MB),
                                      P(0)) == api.ERR_ALIAS
     assert n_z < n_M
+
+
+def test_backward_workspace_and_host_checks(lib):
+    """The backward's sizing and argument checks run on the host: supported
+    shapes (seg_len <= 64, d_k = d_v in {32, 64}) get a workspace that holds
+    at least the fp32 states of every segment; others get 0, and the call
+    returns INFINI_ERR_UNSUPPORTED (or INFINI_ERR_ARG for NULL pointers)
+    before touching a GPU."""
+    w = configs.WORKLOADS["200m-delta"]
+    d = dims_of(w)
+    nbytes = api.backward_workspace_bytes(d, w.seg_len, w.rule)
+    assert nbytes >= w.T * w.B * w.H_kv * w.d_k * w.d_k * 4
+    for over in (dict(d_k=128, d_v=128), dict(d_k=64, d_v=32)):
+        dd = dims_of(w.with_(**over))
+        assert api.backward_workspace_bytes(dd, w.seg_len, w.rule) == 0
+    assert api.backward_workspace_bytes(d, 65, w.rule) == 0
+    null = ctypes.c_void_p(0)
+    args = [null] * 6 + [w.seg_len, 1, ctypes.byref(d)] + [null] * 9 + [null, 0, null]
+    assert lib.infini_attn_backward(*args) == -1  # INFINI_ERR_ARG
+    args[6] = 128
+    assert lib.infini_attn_backward(*args) == -2  # INFINI_ERR_UNSUPPORTED
