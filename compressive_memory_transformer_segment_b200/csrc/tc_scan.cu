@@ -273,7 +273,13 @@ tc_pipe_products(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
   // Accumulator a: G at 0 and B at 128 (delta), B at 0 and dz at 128 (linear).
   auto tG = [&](int a) { return tmem + a * SM::kAccCols; };
   auto tB = [&](int a) { return tmem + a * SM::kAccCols + (DELTA ? 128 : 0); };
-  auto tDZ = [&](int a) { return tmem + a * SM::kAccCols + 128; };
+  // d = 64, linear rule: V's panel and the ones panel form one N = 80 operand
+  // (the descriptor's panel stride reaches from the ring stage to the ones
+  // panel), so dz lands in columns 64.. of the B accumulator with no MMAs of
+  // its own; d = 128 keeps the separate N = 16 dz MMAs (its three panels
+  // would need one stride).
+  constexpr bool kFusedDz = !DELTA && D_ == 64;
+  auto tDZ = [&](int a) { return tmem + a * SM::kAccCols + (kFusedDz ? 64 : 128); };
 
   if (warp == 0) {
     // ---------------------------------------------- TMA producer (whole warp waits, one elected lane issues)
@@ -303,6 +309,7 @@ tc_pipe_products(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
     // ---------------------------------------------- MMA issuer (whole warp waits, one elected lane issues)
     constexpr uint32_t idesc = idesc_bf16_f32(128, D, true, true);
     constexpr uint32_t idesc_dz = idesc_bf16_f32(128, 16, true, true);
+    constexpr uint32_t idesc_vz = idesc_bf16_f32(128, D + 16, true, true);  // [V | ones]
     const uint64_t dop = sw128_desc(smem_u32(op), SM::kPanel, 1024);
     const uint64_t dring = sw128_desc(smem_u32(ring + SM::kBlk), SM::kPanel, 1024);
     const uint64_t dones = sw128_desc(smem_u32(ones), SM::kPanel, 1024);
@@ -324,6 +331,10 @@ tc_pipe_products(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
           const uint64_t yhi = shi + ((2 * SM::kHalf) >> 4);
           const uint64_t ylo = shi + ((3 * SM::kHalf) >> 4);
           const uint64_t vv = dring + ((st * SM::kStage) >> 4);
+          // [V | ones]: V's panel, then the ones panel as the second one.
+          const uint32_t v_off = SM::kRing + st * SM::kStage + SM::kBlk;
+          const uint64_t vz = sw128_desc(smem_u32(ring + st * SM::kStage + SM::kBlk),
+                                         (uint32_t)SM::kOnes - v_off, 1024);
 #pragma unroll
           for (int kk = 0; kk < kLTok / 16; ++kk) {
             const uint32_t stp = mnmajor_step(kk);
@@ -333,9 +344,14 @@ tc_pipe_products(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
               mma_ss(tG(a), ylo + stp, shi + stp, idesc, 1u);
               mma_ss(tG(a), yhi + stp, slo + stp, idesc, 1u);
             }
-            mma_ss(tB(a), shi + stp, vv + stp, idesc, acc);
-            mma_ss(tB(a), slo + stp, vv + stp, idesc, 1u);
-            if (!DELTA) {
+            if (kFusedDz) {
+              mma_ss(tB(a), shi + stp, vz + stp, idesc_vz, acc);
+              mma_ss(tB(a), slo + stp, vz + stp, idesc_vz, 1u);
+            } else {
+              mma_ss(tB(a), shi + stp, vv + stp, idesc, acc);
+              mma_ss(tB(a), slo + stp, vv + stp, idesc, 1u);
+            }
+            if (!DELTA && !kFusedDz) {
               mma_ss(tDZ(a), shi + stp, dones + stp, idesc_dz, acc);
               mma_ss(tDZ(a), slo + stp, dones + stp, idesc_dz, 1u);
             }
