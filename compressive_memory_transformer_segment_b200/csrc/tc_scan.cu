@@ -85,28 +85,60 @@ __global__ void __launch_bounds__(256) zsum(const __nv_bfloat16* __restrict__ k,
 }
 
 // z_{s-1} for s = 0..T-1 into z_pref (slot 0 = z_in) and z_T, from the C
-// chunk partials of every segment.  Grid (B*H_kv), block D threads.  The
-// partials are loaded kAhead at a time before they are added, so that the
-// walk waits for one round of loads per kAhead partials, not for every one.
+// chunk partials of every segment.  Grid (B*H_kv), block 1024 threads: column
+// c of z and a group g of kSG = 1024 / D contiguous segment ranges per
+// thread.  Each group sums its range (the partials loaded kAhead at a time,
+// so that a range costs about one memory round trip), the groups' totals are
+// added in group order through shared memory, and each group then walks its
+// range again from that offset, writing z_{s-1} at every segment start.
 template <int D>
-__global__ void __launch_bounds__(128) zprefix(const float* __restrict__ dz, const float* z_in,
-                                               float* __restrict__ z_pref, float* z_out, int T, int C) {
-  const int bh = blockIdx.x, c = threadIdx.x, BH = gridDim.x;
+__global__ void __launch_bounds__(1024) zprefix(const float* __restrict__ dz, const float* z_in,
+                                                float* __restrict__ z_pref, float* z_out, int T,
+                                                int C) {
+  constexpr int kSG = 1024 / D;
   constexpr int kAhead = 16;
-  const int n = T * C;
+  __shared__ float tot[kSG][D];
   pdl_trigger();
   pdl_wait();
-  // (z_out may be z_in: this thread reads its entry before it writes it)
-  float z = z_in[(size_t)bh * D + c], seg = 0.f;
-  for (int i0 = 0; i0 < n; i0 += kAhead) {
+  const int bh = blockIdx.x, c = threadIdx.x % D, g = threadIdx.x / D, BH = gridDim.x;
+  const int per = (T + kSG - 1) / kSG;
+  const int s0 = min(T, g * per), s1 = min(T, s0 + per);
+  const int i0 = s0 * C, i1 = s1 * C;
+  auto part_at = [&](int i) { return dz[((size_t)i * BH + bh) * D + c]; };
+  // (z_out may be z_in: every thread reads its entry before the barrier, and
+  // only the last group writes z_out, after it)
+  const float zin = z_in[(size_t)bh * D + c];
+  // The range's total, segment by segment in order.
+  float total = 0.f, seg = 0.f;
+  for (int b0 = i0; b0 < i1; b0 += kAhead) {
     float part[kAhead];
 #pragma unroll
-    for (int u = 0; u < kAhead; ++u)
-      part[u] = i0 + u < n ? dz[((size_t)(i0 + u) * BH + bh) * D + c] : 0.f;
+    for (int u = 0; u < kAhead; ++u) part[u] = b0 + u < i1 ? part_at(b0 + u) : 0.f;
 #pragma unroll
     for (int u = 0; u < kAhead; ++u) {
-      const int i = i0 + u;
-      if (i >= n) break;
+      const int i = b0 + u;
+      if (i >= i1) break;
+      seg += part[u];
+      if (i % C == C - 1) {
+        total += seg;
+        seg = 0.f;
+      }
+    }
+  }
+  tot[g][c] = total;
+  __syncthreads();
+  float z = zin;
+  for (int h = 0; h < g; ++h) z += tot[h][c];
+  // The walk over the range from its offset.
+  seg = 0.f;
+  for (int b0 = i0; b0 < i1; b0 += kAhead) {
+    float part[kAhead];
+#pragma unroll
+    for (int u = 0; u < kAhead; ++u) part[u] = b0 + u < i1 ? part_at(b0 + u) : 0.f;
+#pragma unroll
+    for (int u = 0; u < kAhead; ++u) {
+      const int i = b0 + u;
+      if (i >= i1) break;
       const int j = i % C;
       if (j == 0) z_pref[((size_t)(i / C) * BH + bh) * D + c] = z;
       seg += part[u];
@@ -116,7 +148,7 @@ __global__ void __launch_bounds__(128) zprefix(const float* __restrict__ dz, con
       }
     }
   }
-  z_out[(size_t)bh * D + c] = z;
+  if (g == kSG - 1) z_out[(size_t)bh * D + c] = z;
 }
 
 constexpr int kZChunksMax = 8;
@@ -755,7 +787,7 @@ cudaError_t launch(const Problem& p, cudaStream_t stream) {
     if ((e = launch_pdl(false, zsum<D>, dim3(p.T * C, BH), dim3(256), 0, stream,
                         static_cast<const __nv_bfloat16*>(p.k), p.dz, p.L, p.S, C)) != cudaSuccess)
       return e;
-    if ((e = launch_pdl(false, zprefix<D>, dim3(BH), dim3(D), 0, stream, (const float*)p.dz, p.z_in, p.z_pref,
+    if ((e = launch_pdl(false, zprefix<D>, dim3(BH), dim3(1024), 0, stream, (const float*)p.dz, p.z_in, p.z_pref,
                         p.z_out, p.T, C)) != cudaSuccess)
       return e;
     e = launch_pipe_products<D, true>(p, stream);
