@@ -124,3 +124,26 @@ def test_backward_unsupported_shapes(cuda_lib):
     with pytest.raises(api.InfiniError) as exc:
         run_gpu(api, w, inp, grads, inp["M_in"], inp["z_in"])
     assert exc.value.status == -2  # INFINI_ERR_UNSUPPORTED
+
+
+def test_backward_ignores_workspace_contents(cuda_lib):
+    """A workspace full of NaN gives the same gradients as a fresh one: every
+    byte the backward reads there is written earlier in the same call."""
+    api = cuda_lib
+    w = W["tiny"].with_(name="ws_nan", dtype="bf16", d_k=64, d_v=64, rule="delta", H_q=4, H_kv=2,
+                        L=300)
+    inp = synth.make_inputs(w)
+    grads = synth.make_output_grads(w)
+    M_in, z_in = synth.make_state(w)
+    ref = run_gpu(api, w, inp, grads, M_in, z_in)
+    q, k, v = (to_torch(inp[n], w.dtype) for n in ("q", "k", "v"))
+    dims = api.make_dims(w.B, w.H_q, w.H_kv, w.L, w.d_k, w.d_v, q.dtype)
+    nbytes = api.backward_workspace_bytes(dims, w.seg_len, w.rule)
+    ws = torch.full((nbytes // 4,), float("nan"), dtype=torch.float32, device="cuda").view(torch.uint8)
+    got = api.backward(q, k, v, torch.from_numpy(inp["beta"]).cuda(), torch.from_numpy(M_in).cuda(),
+                       torch.from_numpy(z_in).cuda(), w.seg_len, w.rule, to_torch(grads["dout"], w.dtype),
+                       torch.from_numpy(grads["dM_out"]).cuda(), torch.from_numpy(grads["dz_out"]).cuda(),
+                       workspace=ws)
+    api.sync_status()
+    for name, g, r in zip(NAMES, got, ref):
+        assert np.array_equal(g.cpu().numpy().astype(np.float64), r), name
