@@ -16,7 +16,8 @@ import os
 
 import numpy as np
 
-_T_Q, _T_K, _T_V, _T_BETA, _T_PAIR, _T_DOUT, _T_DSTATE, _T_STATE = 1, 2, 3, 4, 5, 6, 7, 8
+(_T_Q, _T_K, _T_V, _T_BETA, _T_PAIR, _T_DOUT, _T_DSTATE, _T_STATE, _T_X, _T_W,
+ _T_BIAS) = 1, 2, 3, 4, 5, 6, 7, 8, 9, 10, 11
 
 
 def _stream(seed, tensor, b=0, h=0):
@@ -171,3 +172,43 @@ def make_state(cfg, seed=None):
     M *= np.float32(1.0 / np.sqrt(cfg.d_k))
     z = g.uniform(0.5, 1.5, size=(cfg.B, cfg.H_kv, cfg.d_k)).astype(np.float32)
     return M, z
+
+
+_X_ROWS = 4096  # rows of x per Philox stream (any chunk regenerates alone)
+
+
+def make_projection_inputs(cfg, d_model=None, seed=None, bias=True, threads=None):
+    """Inputs of the Q/K/V projection prologue for a workload.
+
+    Returns a dict with
+      x    : uint16 bf16 bits [B, L, d_model], i.i.d. N(0, 1)
+      w    : uint16 bf16 bits [(H_q + 2 H_kv) d, d_model], N(0, 1/d_model)
+             (query rows, then key rows, then value rows)
+      bias : float32 [(H_q + 2 H_kv) d], N(0, 0.1^2), or None
+    d_model defaults to H_q * d_k (the model width of the pages' Llama
+    shapes).  Needs d_k == d_v.
+    """
+    seed = cfg.seed if seed is None else seed
+    if cfg.d_k != cfg.d_v:
+        raise ValueError("the fused projection needs d_k == d_v")
+    dm = cfg.H_q * cfg.d_k if d_model is None else d_model
+    n_out = (cfg.H_q + 2 * cfg.H_kv) * cfg.d_k
+    x = np.empty((cfg.B, cfg.L, dm), dtype=np.uint16)
+    jobs = [(b, r0) for b in range(cfg.B) for r0 in range(0, cfg.L, _X_ROWS)]
+
+    def work(job):
+        b, r0 = job
+        n = min(_X_ROWS, cfg.L - r0)
+        g = _stream(seed, _T_X, b, r0 // _X_ROWS)
+        x[b, r0:r0 + n] = round_bf16_bits(g.standard_normal((n, dm), dtype=np.float32))
+
+    nt = threads or min(32, os.cpu_count() or 1)
+    with ThreadPoolExecutor(max_workers=nt) as ex:
+        list(ex.map(work, jobs))
+    wf = _stream(seed, _T_W).standard_normal((n_out, dm), dtype=np.float32)
+    wf *= np.float32(1.0 / np.sqrt(dm))
+    res = dict(x=x, w=round_bf16_bits(wf), bias=None)
+    if bias:
+        res["bias"] = (_stream(seed, _T_BIAS).standard_normal(n_out, dtype=np.float32)
+                       * np.float32(0.1))
+    return res

@@ -18,6 +18,10 @@ The backward (``infini_backward``: elu_plus_one_grad, the vector-Jacobian
 products of each step and infini_attention_backward) is pinned in
 ``tests/test_oracle_backward.py`` against central finite differences of the
 forward and closed forms of special cases.
+The prologue (``infini_projection``: rope_angles, rope_tables, apply_rope,
+qkv_projection, qkv_project_rope) is pinned in
+``tests/test_oracle_projection.py`` against brute-force loops, the complex
+form of the rotation and its invariants.
 No function here is "parity unpinned".
 """
 
@@ -39,4 +43,11 @@ from .infini_backward import (  # noqa: F401
     memory_update_vjp,
     segment_output_vjp,
     infini_attention_backward,
+)
+from .infini_projection import (  # noqa: F401
+    rope_angles,
+    rope_tables,
+    apply_rope,
+    qkv_projection,
+    qkv_project_rope,
 )
