@@ -944,6 +944,155 @@ def run_backward(args, w):
     return 0
 
 
+def oracle_projection_sample(w, pin, budget_s):
+    """Time the float64 oracle's projection prologue on blocks of 256 token
+    rows of batch row 0 until about ``budget_s`` seconds have passed."""
+    import oracle  # the CPU baseline is the only product-adjacent use of the oracle
+
+    d = w.d_k
+    wf = synth.bf16_bits_to_f32(pin["w"]).astype(np.float64)
+    bf = pin["bias"].astype(np.float64)
+    c64, s64 = oracle.rope_tables(w.L, d)
+    rows, elapsed = 0, 0.0
+    while elapsed < budget_s and rows < w.L:
+        n = min(256, w.L - rows)
+        xr = synth.bf16_bits_to_f32(pin["x"][0:1, rows:rows + n]).astype(np.float64)
+        t0 = time.perf_counter()
+        oracle.qkv_project_rope(xr, wf, bf, c64[rows:rows + n], s64[rows:rows + n], w.H_q,
+                                w.H_kv, d)
+        elapsed += time.perf_counter() - t0
+        rows += n
+    desc = (f"oracle (NumPy float64 matmul + rotation), {rows} token rows of batch row 0 in "
+            f"blocks of 256, {elapsed:.2f} s of compute (tables and conversion untimed)")
+    return rows / elapsed, desc
+
+
+def run_projection(args, w):
+    """The Q/K/V projection prologue: y = x W^T + bias, rotary embedding of the
+    query and key heads, bf16 heads in the attention's layout.  A step is one
+    infini_attn_qkv_project over the workload's tokens (d_model = H_q d)."""
+    import torch
+
+    from compressive_memory_transformer_segment_b200 import api
+
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    api.load_library()
+    d, H_q, H_kv = w.d_k, w.H_q, w.H_kv
+    dm = H_q * d
+    n_out = (H_q + 2 * H_kv) * d
+    pin = synth.make_projection_inputs(w)
+
+    def host_bf16(a):
+        return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16)
+
+    hx = host_bf16(pin["x"])
+    x = hx.to(dev)
+    W = host_bf16(pin["w"]).to(dev)
+    bias = torch.from_numpy(pin["bias"]).to(dev)
+    cos, sin = api.rope_tables(w.L, d, device=dev)
+    q = torch.empty((w.B, H_q, w.L, d), dtype=torch.bfloat16, device=dev)
+    k = torch.empty((w.B, H_kv, w.L, d), dtype=torch.bfloat16, device=dev)
+    v = torch.empty((w.B, H_kv, w.L, d), dtype=torch.bfloat16, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    in_bytes = x.numel() * 2 + W.numel() * 2
+    flush = torch.empty(2 * L2_BYTES, dtype=torch.uint8, device=dev) if in_bytes < 2 * L2_BYTES else None
+
+    def step():
+        api.qkv_project(x, W, bias, cos, sin, H_q, H_kv, d, q=q, k=k, v=v, stream=stream)
+
+    bias_bf16 = bias.to(torch.bfloat16)
+
+    def torch_step():
+        # The unfused library route, for context: cuBLAS GEMM with bias, then
+        # the rotation and the head layout in PyTorch ops.
+        y = torch.nn.functional.linear(x, W, bias_bf16)
+        yq, yk, yv = y.split([H_q * d, H_kv * d, H_kv * d], dim=-1)
+        out = []
+        for part, H, rot in ((yq, H_q, True), (yk, H_kv, True), (yv, H_kv, False)):
+            t = part.view(w.B, w.L, H, d).transpose(1, 2)
+            if rot:
+                t1, t2 = t[..., : d // 2].float(), t[..., d // 2:].float()
+                t = torch.cat([t1 * cos - t2 * sin, t2 * cos + t1 * sin], dim=-1).to(torch.bfloat16)
+            out.append(t.contiguous())
+        return out
+
+    def timed(fn, n):
+        total = 0.0
+        for _ in range(n):
+            if flush is not None:
+                flush.fill_(1)
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            fn()
+            e1.record(stream)
+            torch.cuda.synchronize(dev)
+            total += e0.elapsed_time(e1)
+        return total
+
+    for _ in range(args.warmup):
+        step()
+        torch_step()
+    api.sync_status(stream)
+    torch.cuda.synchronize(dev)
+    with ClockSampler(0) as clocks:
+        elapsed_ms = timed(step, args.steps)
+    api.sync_status(stream)
+    torch_ms = timed(torch_step, args.steps)
+    tokens = w.B * w.L * args.steps
+    value = tokens / (elapsed_ms / 1000.0)
+
+    # End to end: x from pinned host memory in, q / k / v back to pinned host
+    # memory, inside the timed region (weights and tables stay resident).
+    hxp = hx.pin_memory()
+    outs_h = [torch.empty(t.shape, dtype=t.dtype).pin_memory() for t in (q, k, v)]
+    e2e_steps = max(1, min(args.steps, 3))
+    torch.cuda.synchronize(dev)
+    e2, e3 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e2.record(stream)
+    for _ in range(e2e_steps):
+        x.copy_(hxp, non_blocking=True)
+        step()
+        for dst, src in zip(outs_h, (q, k, v)):
+            dst.copy_(src, non_blocking=True)
+    e3.record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_value = w.B * w.L * e2e_steps / (e2.elapsed_time(e3) / 1000.0)
+
+    peaks, peak_src = load_peaks()
+    peak = peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
+    flops = 2.0 * w.B * w.L * n_out * dm
+    achieved = flops / (elapsed_ms / args.steps / 1000.0) / 1e12
+    line = {
+        "metric": "Q/K/V projection + rotary embedding tokens/s on 1 B200",
+        "value": value, "unit": "tokens/s", "n_gpus": 1, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": elapsed_ms / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded Philox N(0,1) x, N(0,1/d_model) weights, N(0,0.01) bias)",
+        "config": {"workload": f"{w.name} projection prologue", "B": w.B, "L": w.L,
+                   "d_model": dm, "H_q": H_q, "H_kv": H_kv, "d": d, "n_out": n_out,
+                   "rope": "rotate-half, base 10000, positions 0..L-1",
+                   "l2": ("L2 flushed (256 MiB write) between timed steps; each step timed alone"
+                          if flush is not None else "inputs larger than L2")},
+        "clocks": clocks.summary(),
+        "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": hx.numel() * 2,
+                "d2h_bytes_per_step": sum(t.numel() * 2 for t in outs_h), "steps": e2e_steps},
+        "gpu_launches": args.steps,
+        "roofline": {"bound": "tensor", "kernel": "qkv_rope", "achieved": achieved, "peak": peak,
+                     "unit": "TFLOP/s", "frac": achieved / peak,
+                     "peak_source": f"{peak_src} bf16 (burst)", "traffic": None,
+                     "algorithmic_flops_per_step": flops,
+                     "avg_launch_ms": elapsed_ms / args.steps},
+        "library_route_ms": torch_ms / args.steps,
+    }
+    if args.cpu_baseline:
+        v_cpu, desc = oracle_projection_sample(w, pin, args.cpu_budget)
+        line["cpu_baseline"] = {"value": v_cpu, "unit": "tokens/s", "cores": host_cores(),
+                                "kind": "oracle", "sample": desc}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -977,6 +1126,9 @@ def main():
     ap.add_argument("--decode", action="store_true",
                     help="streaming decode (one token per call) of the workload's shape; "
                          "a step is one full segment")
+    ap.add_argument("--projection", action="store_true",
+                    help="the Q/K/V projection + rotary embedding prologue of the workload's "
+                         "shape (d_model = H_q d)")
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "ours":
         args.warmup = 3
@@ -995,6 +1147,8 @@ def main():
         return run_decode(args, w)
     if args.backward:
         return run_backward(args, w)
+    if args.projection:
+        return run_projection(args, w)
     if args.seq_parallel:
         return run_seq_parallel(args, w)
     return run_gpu(args, w)

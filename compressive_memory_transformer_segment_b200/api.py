@@ -83,6 +83,10 @@ _SIGNATURES = [
     ("infini_attn_noalloc_scratch_limit", ctypes.c_size_t, []),
     ("infini_attn_backward_workspace_bytes", ctypes.c_size_t, [ctypes.POINTER(Dims), ctypes.c_int,
                                                                 ctypes.c_int]),
+    ("infini_attn_qkv_project", ctypes.c_int, [_P, _P, _P, _P, _P, ctypes.POINTER(Dims), ctypes.c_int,
+                                               _P, _P, _P, _P]),
+    ("infini_attn_rope_tables", ctypes.c_int, [_P, _P, ctypes.c_int, ctypes.c_int, ctypes.c_double,
+                                               _P]),
     ("infini_attn_backward", ctypes.c_int, [_P, _P, _P, _P, _P, _P, ctypes.c_int, ctypes.c_int,
                                             ctypes.POINTER(Dims), _P, _P, _P, _P, _P, _P, _P, _P,
                                             _P, _P, ctypes.c_size_t, _P]),
@@ -330,6 +334,52 @@ def state_sum(M_base, z_base, parts, n_parts, M_out=None, z_out=None, stream=Non
     with _one_device(M_base, z_base, parts, M_out, z_out, stream=stream):
         _check(lib.infini_attn_state_sum(*args, _stream_handle(stream)))
     return M_out, z_out
+
+
+def rope_tables(n_pos, d, base=10000.0, device=None, stream=None):
+    """infini_attn_rope_tables: float32 (cos, sin) [n_pos, d/2] on the GPU."""
+    device = device or torch.device("cuda", torch.cuda.current_device())
+    cos = torch.empty((n_pos, d // 2), dtype=torch.float32, device=device)
+    sin = torch.empty((n_pos, d // 2), dtype=torch.float32, device=device)
+    with _one_device(cos, sin, stream=stream):
+        _check(load_library().infini_attn_rope_tables(
+            ctypes.c_void_p(cos.data_ptr()), ctypes.c_void_p(sin.data_ptr()), int(n_pos), int(d),
+            float(base), _stream_handle(stream)))
+    return cos, sin
+
+
+def qkv_project(x, w_qkv, bias, rope_cos, rope_sin, H_q, H_kv, d, q=None, k=None, v=None,
+                stream=None):
+    """infini_attn_qkv_project: x bf16 [B, L, d_model], w_qkv bf16
+    [(H_q + 2 H_kv) d, d_model], bias float32 [(H_q + 2 H_kv) d] or None,
+    rope_cos / rope_sin float32 [L, d/2] or None; returns bf16 (q, k, v) in
+    the [B, H, L, d] layout of ``forward``."""
+    lib = load_library()
+    if x.dim() != 3:
+        raise ValueError("x must be [B, L, d_model]")
+    B, L, dm = x.shape
+    n_out = (H_q + 2 * H_kv) * d
+    if q is None:
+        q = torch.empty((B, H_q, L, d), dtype=torch.bfloat16, device=x.device)
+    if k is None:
+        k = torch.empty((B, H_kv, L, d), dtype=torch.bfloat16, device=x.device)
+    if v is None:
+        v = torch.empty((B, H_kv, L, d), dtype=torch.bfloat16, device=x.device)
+    if (rope_cos is None) != (rope_sin is None):
+        raise ValueError("give both rotary tables or neither")
+    rot = [ctypes.c_void_p(0), ctypes.c_void_p(0)]
+    if rope_cos is not None:
+        rot = [_dev(rope_cos, "rope_cos", torch.float32, (L, d // 2)),
+               _dev(rope_sin, "rope_sin", torch.float32, (L, d // 2))]
+    dims = make_dims(B, H_q, H_kv, L, d, d, torch.bfloat16)
+    args = [_dev(x, "x", torch.bfloat16), _dev(w_qkv, "w_qkv", torch.bfloat16, (n_out, dm)),
+            _dev(bias, "bias", torch.float32, (n_out,)) if bias is not None else ctypes.c_void_p(0),
+            *rot, ctypes.byref(dims), int(dm),
+            _dev(q, "q", torch.bfloat16, (B, H_q, L, d)), _dev(k, "k", torch.bfloat16, (B, H_kv, L, d)),
+            _dev(v, "v", torch.bfloat16, (B, H_kv, L, d))]
+    with _one_device(x, w_qkv, bias, rope_cos, rope_sin, q, k, v, stream=stream):
+        _check(lib.infini_attn_qkv_project(*args, _stream_handle(stream)))
+    return q, k, v
 
 
 def decode_workspace_bytes(dims, seg_len, rule):

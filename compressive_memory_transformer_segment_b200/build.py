@@ -15,7 +15,8 @@ LIB = os.path.join(PKG, "libinfini_attn.so")
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 
 SOURCES = ["api.cu", "simt.cu", "tc_attention.cu", "tc_attention_single.cu", "tc_attention_small.cu",
-           "tc_scan.cu", "selftest.cu", "noalloc.cu", "decode.cu", "backward.cu"]
+           "tc_scan.cu", "selftest.cu", "noalloc.cu", "decode.cu", "backward.cu",
+           "qkv_rope.cu"]
 FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",
     "-O3", "-lineinfo", "-std=c++17",

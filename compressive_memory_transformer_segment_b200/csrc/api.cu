@@ -715,6 +715,70 @@ int infini_attn_kernel_times(double* ms, int* launches, int n_kinds, int reset) 
   return INFINI_OK;
 }
 
+int infini_attn_qkv_project(const void* x, const void* w_qkv, const float* bias,
+                            const float* rope_cos, const float* rope_sin, const infini_dims_t* dims,
+                            int d_model, void* q, void* k, void* v, void* stream) {
+  if (!dims || !x || !w_qkv || !q || !k || !v) return INFINI_ERR_ARG;
+  if ((rope_cos == nullptr) != (rope_sin == nullptr)) return INFINI_ERR_ARG;
+  if (dims->B < 1 || dims->H_q < 1 || dims->H_kv < 1 || dims->L < 1 || d_model < 1 ||
+      dims->d_k < 1 || dims->d_v < 1)
+    return INFINI_ERR_ARG;
+  if (dims->dtype != INFINI_DTYPE_BF16 && dims->dtype != INFINI_DTYPE_F32) return INFINI_ERR_ARG;
+  if (!qkv_projection_supported(dims->d_k, dims->d_v, d_model, dims->dtype == INFINI_DTYPE_BF16))
+    return INFINI_ERR_UNSUPPORTED;
+  const long long rows = (long long)dims->B * dims->L;
+  if (rows > 0x7fffffffLL) return INFINI_ERR_UNSUPPORTED;
+  const int d = dims->d_k;
+  const size_t N = (size_t)(dims->H_q + 2 * dims->H_kv) * d;
+  const void* ptrs[] = {x, w_qkv, bias, rope_cos, rope_sin, q, k, v};
+  for (const void* p : ptrs)
+    if (p && !aligned16(p)) return INFINI_ERR_ALIGN;
+  const Range ins[] = {rng(x, (size_t)rows * d_model * 2), rng(w_qkv, N * d_model * 2),
+                       rng(bias, bias ? N * 4 : 0), rng(rope_cos, rope_cos ? (size_t)dims->L * d / 2 * 4 : 0),
+                       rng(rope_sin, rope_sin ? (size_t)dims->L * d / 2 * 4 : 0)};
+  const Range outs[] = {rng(q, (size_t)rows * dims->H_q * d * 2),
+                        rng(k, (size_t)rows * dims->H_kv * d * 2),
+                        rng(v, (size_t)rows * dims->H_kv * d * 2)};
+  for (int i = 0; i < 3; ++i) {
+    for (const Range& r : ins)
+      if (overlap(outs[i], r)) return INFINI_ERR_ALIAS;
+    for (int j = i + 1; j < 3; ++j)
+      if (overlap(outs[i], outs[j])) return INFINI_ERR_ALIAS;
+  }
+  unsigned int* status = status_ptr();
+  if (!status) return INFINI_ERR_CUDA;
+  ProjectionProblem p;
+  p.x = x;
+  p.w = w_qkv;
+  p.bias = bias;
+  p.rope_cos = rope_cos;
+  p.rope_sin = rope_sin;
+  p.q = q;
+  p.k = k;
+  p.v = v;
+  p.B = dims->B;
+  p.H_q = dims->H_q;
+  p.H_kv = dims->H_kv;
+  p.L = dims->L;
+  p.d = d;
+  p.d_model = d_model;
+  p.status = status;
+  return launch_qkv_projection(p, static_cast<cudaStream_t>(stream)) == cudaSuccess ? INFINI_OK
+                                                                                    : INFINI_ERR_CUDA;
+}
+
+int infini_attn_rope_tables(float* cos_out, float* sin_out, int n_pos, int d, double base,
+                            void* stream) {
+  if (!cos_out || !sin_out || n_pos < 1 || d < 2 || d % 2 != 0 || !(base > 0.0))
+    return INFINI_ERR_ARG;
+  const size_t n = (size_t)n_pos * (d / 2) * 4;
+  if (overlap(rng(cos_out, n), rng(sin_out, n))) return INFINI_ERR_ALIAS;
+  return launch_rope_tables(cos_out, sin_out, n_pos, d, base, static_cast<cudaStream_t>(stream)) ==
+                 cudaSuccess
+             ? INFINI_OK
+             : INFINI_ERR_CUDA;
+}
+
 int infini_attn_sync_status(void* stream) {
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (cudaStreamSynchronize(st) != cudaSuccess) return INFINI_ERR_CUDA;

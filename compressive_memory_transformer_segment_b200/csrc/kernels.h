@@ -112,6 +112,26 @@ struct BackwardProblem {
 bool backward_supported(int d_k, int d_v, int S);
 cudaError_t launch_backward(const BackwardProblem& p, cudaStream_t stream);
 
+// Q/K/V projections with rotary embedding (tcgen05 GEMM with the bias, the
+// rotation and the head split in its epilogue): bf16, d in {64, 128},
+// d_model >= 64 and a multiple of 8.
+struct ProjectionProblem {
+  const void* x;         // [B * L][d_model] bf16
+  const void* w;         // [(H_q + 2 H_kv) d][d_model] bf16
+  const float* bias;     // [(H_q + 2 H_kv) d] or null
+  const float* rope_cos; // [L][d / 2] or null (no rotation)
+  const float* rope_sin;
+  void* q;               // [B, H_q, L, d] bf16
+  void* k;               // [B, H_kv, L, d]
+  void* v;               // [B, H_kv, L, d]
+  int B, H_q, H_kv, L, d, d_model;
+  unsigned int* status;
+};
+bool qkv_projection_supported(int d_k, int d_v, int d_model, bool bf16);
+cudaError_t launch_qkv_projection(const ProjectionProblem& p, cudaStream_t stream);
+cudaError_t launch_rope_tables(float* cos_out, float* sin_out, int n_pos, int d, double base,
+                               cudaStream_t stream);
+
 int decode_splits(int S);
 int decode_head_chunks(int g);
 cudaError_t launch_decode_step(const DecodeProblem& p, cudaStream_t stream);

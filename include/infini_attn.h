@@ -245,6 +245,52 @@ INFINI_API int infini_attn_state_sum(const float* M_base, const float* z_base, c
                                      int n_parts, int B, int H_kv, int d_k, int d_v, float* M_out,
                                      float* z_out, void* stream);
 
+/* Q/K/V projections with rotary position embedding: the prologue that
+ * produces the heads the layer consumes.  The memory reuses the attention's
+ * own Q, K and V ("Leave No Context Behind" explainer, "メモリ構造"); they
+ * come from linear layers over the layer input ("Как работает
+ * Infini-attention", section 9).  For every token row r = b L + t of x:
+ *   y_r = x_r W^T + bias   (fp32 accumulation over d_model)
+ * y's columns are H_q query heads, then H_kv key heads, then H_kv value heads
+ * of d columns each.  Query and key heads are rotated (rotary embedding,
+ * rotate-half pairing: for i < d/2, with c = rope_cos[t][i], s = rope_sin[t][i],
+ *   y'_i = y_i c - y_{i+d/2} s,  y'_{i+d/2} = y_{i+d/2} c + y_i s);
+ * value heads are not.  Results are rounded to bf16.
+ *   x          device bf16 [B, L, d_model] (row-major, rows contiguous)
+ *   w_qkv      device bf16 [(H_q + 2 H_kv) d, d_model]: W_q's rows, then
+ *              W_k's, then W_v's (the layout of a linear layer's weight)
+ *   bias       device float32 [(H_q + 2 H_kv) d], or NULL for none
+ *   rope_cos, rope_sin
+ *              device float32 [L, d/2] (row t rotates token t of every batch
+ *              row; see infini_attn_rope_tables), or both NULL for no rotation
+ *   dims       B, H_q, H_kv, L; d = d_k = d_v; dtype must be BF16
+ *   d_model    input width
+ *   q, k, v    device bf16 outputs [B, H_q, L, d], [B, H_kv, L, d],
+ *              [B, H_kv, L, d]: the inputs of infini_attn_forward
+ *   stream     cudaStream_t; asynchronous.
+ * Supported: d_k == d_v in {64, 128}, d_model >= 64 and a multiple of 8,
+ * dtype BF16 (otherwise INFINI_ERR_UNSUPPORTED).  The outputs must not
+ * overlap each other or any input (INFINI_ERR_ALIAS); all pointers 16-byte
+ * aligned (INFINI_ERR_ALIGN); one of rope_cos / rope_sin NULL without the
+ * other, a NULL x / w_qkv / output, or a size < 1 is INFINI_ERR_ARG.  A kernel
+ * that gives up a bounded wait sets the device status word (see
+ * infini_attn_sync_status).  Other errors: INFINI_ERR_CUDA. */
+INFINI_API int infini_attn_qkv_project(const void* x, const void* w_qkv, const float* bias,
+                                       const float* rope_cos, const float* rope_sin,
+                                       const infini_dims_t* dims, int d_model, void* q, void* k,
+                                       void* v, void* stream);
+
+/* Rotary embedding tables for infini_attn_qkv_project:
+ *   cos_out[p][i] = cos(p base^(-2i/d)),  sin_out[p][i] = sin(p base^(-2i/d))
+ * for p = 0..n_pos-1, i < d/2, computed in fp64 and rounded to float32
+ * (RoFormer's frequencies; a reading, the pages name no position encoding).
+ *   cos_out, sin_out   device float32 [n_pos, d/2], not overlapping
+ *   n_pos >= 1, d >= 2 even, base > 0; stream: cudaStream_t.
+ * Errors: INFINI_ERR_ARG (NULL, bad size or base), INFINI_ERR_ALIAS,
+ * INFINI_ERR_CUDA. */
+INFINI_API int infini_attn_rope_tables(float* cos_out, float* sin_out, int n_pos, int d,
+                                       double base, void* stream);
+
 /* Streaming decode: the layer forward one token at a time.  The current
  * segment's keys and values so far are kept by the caller in a rolling
  * buffer of seg_len rows per KV head; (M, z) hold the memory of the segments

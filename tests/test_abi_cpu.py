@@ -212,3 +212,36 @@ def test_backward_workspace_and_host_checks(lib):
     assert lib.infini_attn_backward(*args) == -1  # INFINI_ERR_ARG
     args[6] = 128
     assert lib.infini_attn_backward(*args) == -2  # INFINI_ERR_UNSUPPORTED
+
+
+def test_qkv_project_and_rope_tables_check_arguments_on_the_host(lib):
+    """The projection prologue's and the rotary tables' argument checks
+    return before any CUDA call."""
+    P = ctypes.c_void_p
+    MB = 1 << 20
+    d = api.make_dims(2, 4, 2, 256, 64, 64, 0)
+    x, w, bias, cs, sn = P(1 * MB), P(8 * MB), P(12 * MB), P(13 * MB), P(14 * MB)
+    q, k, v = P(20 * MB), P(24 * MB), P(28 * MB)
+
+    def call(*a, dims=d, dm=256):
+        a = list(a) if a else [x, w, bias, cs, sn]
+        return lib.infini_attn_qkv_project(*a, ctypes.byref(dims), dm, q, k, v, P(0))
+
+    assert call(P(0), w, bias, cs, sn) == api.ERR_ARG
+    assert call(x, w, bias, cs, P(0)) == api.ERR_ARG         # one table without the other
+    assert call(dm=0) == api.ERR_ARG
+    assert call(dims=api.make_dims(2, 4, 2, 256, 128, 64, 0)) == api.ERR_UNSUPPORTED
+    assert call(dims=api.make_dims(2, 4, 2, 256, 32, 32, 0)) == api.ERR_UNSUPPORTED
+    assert call(dims=api.make_dims(2, 4, 2, 256, 64, 64, 1)) == api.ERR_UNSUPPORTED  # f32
+    assert call(dm=60) == api.ERR_UNSUPPORTED
+    assert call(dm=260) == api.ERR_UNSUPPORTED
+    assert call(P(1 * MB + 8), w, bias, cs, sn) == api.ERR_ALIGN
+    # q [2, 4, 256, 64] bf16 = 256 KB from 20 MB: an input there overlaps it.
+    assert call(x, w, bias, P(20 * MB + 4096), sn) == api.ERR_ALIAS
+    assert lib.infini_attn_qkv_project(x, w, bias, cs, sn, ctypes.byref(d), 256, q, P(20 * MB + 64),
+                                       v, P(0)) == api.ERR_ALIAS
+    assert lib.infini_attn_rope_tables(P(0), P(MB), 16, 64, 10000.0, P(0)) == api.ERR_ARG
+    assert lib.infini_attn_rope_tables(P(MB), P(2 * MB), 0, 64, 10000.0, P(0)) == api.ERR_ARG
+    assert lib.infini_attn_rope_tables(P(MB), P(2 * MB), 16, 63, 10000.0, P(0)) == api.ERR_ARG
+    assert lib.infini_attn_rope_tables(P(MB), P(2 * MB), 16, 64, 0.0, P(0)) == api.ERR_ARG
+    assert lib.infini_attn_rope_tables(P(MB), P(MB + 256), 16, 64, 1e4, P(0)) == api.ERR_ALIAS
