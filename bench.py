@@ -56,11 +56,22 @@ ATTENTION_TRAFFIC = {
 }
 
 
-def attention_traffic(name):
+# The same for the projection prologue's qkv_rope launch.
+PROJECTION_TRAFFIC = {
+    "8b-delta": {"bytes": 2 * (862.808320e6 + 389.649664e6),
+                 "note": "ncu capture at batch 1, scaled x2 to the batch-2 launch (traffic grows "
+                         "with the token rows)",
+                 "profile": "profiles/qkv_rope_8b-projection.md",
+                 "sha1": {"qkv_rope.cu": "e66e05c97c9799a33c647c83133a18d55ef0d0ab",
+                          "tc_common.cuh": "a896981e1b8e14dfabfd0f26a799d64c0af65a34"}},
+}
+
+
+def attention_traffic(name, table=None):
     """Recorded per-launch traffic for this workload, or None if the kernel
     changed since the counters were taken (or none were taken)."""
     import hashlib
-    rec = ATTENTION_TRAFFIC.get(name)
+    rec = (ATTENTION_TRAFFIC if table is None else table).get(name)
     if rec is None:
         return None
     csrc = os.path.join(ROOT, "compressive_memory_transformer_segment_b200", "csrc")
@@ -1044,24 +1055,29 @@ def run_projection(args, w):
 
     # End to end: x from pinned host memory in, q / k / v back to pinned host
     # memory, inside the timed region (weights and tables stay resident).
-    hxp = hx.pin_memory()
-    outs_h = [torch.empty(t.shape, dtype=t.dtype).pin_memory() for t in (q, k, v)]
-    e2e_steps = max(1, min(args.steps, 3))
-    torch.cuda.synchronize(dev)
-    e2, e3 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e2.record(stream)
-    for _ in range(e2e_steps):
-        x.copy_(hxp, non_blocking=True)
-        step()
-        for dst, src in zip(outs_h, (q, k, v)):
-            dst.copy_(src, non_blocking=True)
-    e3.record(stream)
-    torch.cuda.synchronize(dev)
-    e2e_value = w.B * w.L * e2e_steps / (e2.elapsed_time(e3) / 1000.0)
+    e2e = None
+    if args.e2e:
+        hxp = hx.pin_memory()
+        outs_h = [torch.empty(t.shape, dtype=t.dtype).pin_memory() for t in (q, k, v)]
+        e2e_steps = max(1, min(args.steps, 3))
+        torch.cuda.synchronize(dev)
+        e2, e3 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e2.record(stream)
+        for _ in range(e2e_steps):
+            x.copy_(hxp, non_blocking=True)
+            step()
+            for dst, src in zip(outs_h, (q, k, v)):
+                dst.copy_(src, non_blocking=True)
+        e3.record(stream)
+        torch.cuda.synchronize(dev)
+        e2e = {"value": w.B * w.L * e2e_steps / (e2.elapsed_time(e3) / 1000.0), "unit": "tokens/s",
+               "h2d_bytes_per_step": hx.numel() * 2,
+               "d2h_bytes_per_step": sum(t.numel() * 2 for t in outs_h), "steps": e2e_steps}
 
     peaks, peak_src = load_peaks()
     peak = peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
     flops = 2.0 * w.B * w.L * n_out * dm
+    traffic = attention_traffic(w.name, PROJECTION_TRAFFIC)
     achieved = flops / (elapsed_ms / args.steps / 1000.0) / 1e12
     line = {
         "metric": "Q/K/V projection + rotary embedding tokens/s on 1 B200",
@@ -1075,12 +1091,14 @@ def run_projection(args, w):
                    "l2": ("L2 flushed (256 MiB write) between timed steps; each step timed alone"
                           if flush is not None else "inputs larger than L2")},
         "clocks": clocks.summary(),
-        "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": hx.numel() * 2,
-                "d2h_bytes_per_step": sum(t.numel() * 2 for t in outs_h), "steps": e2e_steps},
+        "e2e": e2e,
         "gpu_launches": args.steps,
         "roofline": {"bound": "tensor", "kernel": "qkv_rope", "achieved": achieved, "peak": peak,
                      "unit": "TFLOP/s", "frac": achieved / peak,
-                     "peak_source": f"{peak_src} bf16 (burst)", "traffic": None,
+                     "peak_source": f"{peak_src} bf16 (burst)",
+                     "traffic": traffic["bytes"] if traffic else None,
+                     "traffic_note": (f"{traffic['note']}; {traffic['profile']}" if traffic
+                                      else "no capture of this kernel source for this workload"),
                      "algorithmic_flops_per_step": flops,
                      "avg_launch_ms": elapsed_ms / args.steps},
         "library_route_ms": torch_ms / args.steps,
