@@ -80,6 +80,9 @@ CASES = [
     ("d128_gqa", dict(B=1, H_q=8, H_kv=2, L=300, d_k=128, d_v=128), 512, False, True),
     ("d64_padded_col_tile_partial_k", dict(B=1, H_q=3, H_kv=1, L=130, d_k=64, d_v=64), 200, True, False),
     ("d128_fewer_rows_than_a_tile", dict(B=1, H_q=2, H_kv=1, L=20, d_k=128, d_v=128), 64, True, True),
+    # Many row tiles (1183, eight waves on 148 SMs), the last one ragged,
+    # tiles straddling the two batch rows.
+    ("d64_many_row_tiles_ragged", dict(B=2, H_q=2, H_kv=1, L=75700, d_k=64, d_v=64), 64, True, True),
 ]
 
 
