@@ -245,3 +245,22 @@ def test_qkv_project_and_rope_tables_check_arguments_on_the_host(lib):
     assert lib.infini_attn_rope_tables(P(MB), P(2 * MB), 16, 63, 10000.0, P(0)) == api.ERR_ARG
     assert lib.infini_attn_rope_tables(P(MB), P(2 * MB), 16, 64, 0.0, P(0)) == api.ERR_ARG
     assert lib.infini_attn_rope_tables(P(MB), P(MB + 256), 16, 64, 1e4, P(0)) == api.ERR_ALIAS
+
+
+def test_plain_c_program_uses_the_boundary(tmp_path):
+    """The header compiles as C99 and a C program linked against the library
+    gets the documented answers from the host-side calls (no GPU needed)."""
+    import shutil
+    import subprocess
+
+    cc = shutil.which("gcc") or shutil.which("cc")
+    if cc is None:
+        pytest.skip("no C compiler")
+    lib_dir = os.path.dirname(api.LIB_PATH)
+    exe = tmp_path / "c_abi_check"
+    subprocess.run([cc, "-std=c99", "-Wall", "-Wextra", "-Werror", "-I", os.path.join(ROOT, "include"),
+                    os.path.join(ROOT, "tests", "c_abi_check.c"), api.LIB_PATH,
+                    f"-Wl,-rpath,{lib_dir}", "-o", str(exe)], check=True)
+    res = subprocess.run([str(exe)], capture_output=True, text=True, timeout=120)
+    assert res.returncode == 0, res.stderr
+    assert res.stdout.strip() == "c-abi ok"
