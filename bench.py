@@ -749,7 +749,9 @@ def run_decode(args, w):
         "e2e": {"value": e2e_value, "unit": "tokens/s", "note": "eager calls, per-token copies",
                 "h2d_bytes_per_step": sum(x.numel() * x.element_size() for x in (hq, hk, hv)),
                 "d2h_bytes_per_step": hout.numel() * hout.element_size(), "steps": 1},
-        "gpu_launches": (2 * S + plan["launches"] - 1) * args.steps,
+        # one decode kernel per call, plus the state update's scan kernels
+        # once per segment
+        "gpu_launches": (S + plan["launches"] - 1) * args.steps,
         "roofline": {"bound": "hbm", "kernel": "decode attention (partial + combine)",
                      "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                      "frac": achieved / peaks["hbm_gbs"], "peak_source": f"{peak_src} copy",
