@@ -69,9 +69,37 @@ __device__ __forceinline__ void copy_vec(const T* src, T* dst) {
   *reinterpret_cast<V*>(dst) = *reinterpret_cast<const V*>(src);
 }
 
+// Sums each of v[0..31] over the 32 lanes of the warp; afterwards every lane
+// holds all 32 totals.  Recursive halving (each exchange sends half of the
+// values still held, so that lane L ends with the total of value L: 31
+// shuffles) and a broadcast back (32 shuffles), against 32 x 5 shuffles for
+// 32 separate butterfly sums: the shuffle unit, not the arithmetic, bounds
+// the step's 32 dot products per warp.
+__device__ __forceinline__ void warp_sum32(float (&v)[32], int lane) {
+  float w[32];
+#pragma unroll
+  for (int i = 0; i < 32; ++i) w[i] = v[i];
+#pragma unroll
+  for (int lvl = 0; lvl < 5; ++lvl) {
+    const int o = 16 >> lvl;  // lanes exchanged with, and values kept
+    const bool upper = (lane & o) != 0;
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      if (i < o) {
+        const float send = upper ? w[i] : w[i + o];
+        const float keep = upper ? w[i + o] : w[i];
+        w[i] = keep + __shfl_xor_sync(0xffffffffu, send, o);
+      }
+    }
+  }
+#pragma unroll
+  for (int i = 0; i < 32; ++i) v[i] = __shfl_sync(0xffffffffu, w[0], i);
+}
+
 template <typename T, int D>
 __global__ void __launch_bounds__(kThreads, 2)
 decode_step_kernel(DecodeProblem p) {
+  static_assert(kNB * kG == 32, "one score per lane after the reduce-scatter");
   constexpr int E = D / 32;  // elements of d per lane
   __shared__ float qs[kG][D];
   __shared__ float red[kWarps][kG][D + 2];
@@ -147,13 +175,18 @@ decode_step_kernel(DecodeProblem p) {
           for (int e = 0; e < E; ++e) t = fmaf(qr[hh][e], elem<T, E>(kx[rr], e), t);
           s[rr][hh] = t;
         }
+      {
+        float sv[32];
 #pragma unroll
-      for (int rr = 0; rr < kNB; ++rr)
+        for (int rr = 0; rr < kNB; ++rr)
 #pragma unroll
-        for (int hh = 0; hh < kG; ++hh) {
-          const float t = warp_sum(s[rr][hh]);
-          s[rr][hh] = i0 + rr < nr ? t : -INFINITY;
-        }
+          for (int hh = 0; hh < kG; ++hh) sv[rr * kG + hh] = s[rr][hh];
+        warp_sum32(sv, lane);
+#pragma unroll
+        for (int rr = 0; rr < kNB; ++rr)
+#pragma unroll
+          for (int hh = 0; hh < kG; ++hh) s[rr][hh] = i0 + rr < nr ? sv[rr * kG + hh] : -INFINITY;
+      }
 #pragma unroll
       for (int hh = 0; hh < kG; ++hh) {
         float bm = s[0][hh];
@@ -265,6 +298,20 @@ decode_step_kernel(DecodeProblem p) {
   __syncthreads();
   if (!last) return;
   __threadfence();  // every other CTA's writes of this group are visible
+  // The retrieval terms and the gates of this thread's output column, loaded
+  // now so that they arrive during the merge of the partials.
+  float r_num[kG], r_den[kG], gate[kG];
+  {
+    const int e = threadIdx.x % D;
+#pragma unroll
+    for (int hh = 0; hh < kG; ++hh) {
+      const bool ok = hh < ng && threadIdx.x < D;
+      const float* rt = p.ret + (size_t)(b * p.H_q + hq0 + (ok ? hh : 0)) * (D + 1);
+      r_num[hh] = ok ? __ldcg(rt + e) : 0.f;
+      r_den[hh] = ok ? __ldcg(rt + D) : 0.f;
+      gate[hh] = ok ? p.beta[hq0 + hh] : 0.f;
+    }
+  }
   // Column e of every head of the CTA is merged by kParts threads, each over
   // every kParts-th chunk, four chunks at a time for all heads (independent
   // loads in flight) with a running max; then the parts are combined.
@@ -342,10 +389,8 @@ decode_step_kernel(DecodeProblem p) {
         }
         const int h = hq0 + hh;
         const float a_dot = a2 / l2;
-        const float* rt = p.ret + (size_t)(b * p.H_q + h) * (D + 1);
-        const float den = __ldcg(rt + D);
-        const float a_mem = den != 0.f ? __ldcg(rt + e) / den : 0.f;
-        const float gm = gate_sigmoid(p.beta[h]);
+        const float a_mem = r_den[hh] != 0.f ? r_num[hh] / r_den[hh] : 0.f;
+        const float gm = gate_sigmoid(gate[hh]);
         static_cast<T*>(p.out_t)[(size_t)(b * p.H_q + h) * D + e] =
             from_f32<T>(gm * a_mem + (1.f - gm) * a_dot);
       }
