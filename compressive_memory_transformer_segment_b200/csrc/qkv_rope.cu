@@ -49,7 +49,8 @@ struct ProjSmem {
   static constexpr uint32_t kBar = kB + kStages * kBBytes;
   // full[kStages] empty[kStages] acc_full[2] acc_empty[2] drain
   static constexpr uint32_t kNumBars = 2 * kStages + 5;
-  static constexpr uint32_t kTmemSlot = kBar + kNumBars * 8;
+  static constexpr uint32_t kBias = kBar + kNumBars * 8;        // the tile's bias [kBN] f32
+  static constexpr uint32_t kTmemSlot = kBias + kBN * 4;
   static constexpr uint32_t kAbort = kTmemSlot + 4;
   static constexpr uint32_t kAlloc = kAbort + 4 + 1024;  // + room to align the base
   static_assert(kB % 1024 == 0 && kBar % 1024 == 0, "tiles must be 1024-byte aligned");
@@ -64,6 +65,7 @@ struct ProjArgs {
   const float* rsin;
   unsigned int* status;
   int rows;            // B * L
+  int n_out;           // (H_q + 2 H_kv) d
   int L, H_q, H_kv;
   int kslices;         // ceil(d_model / 64)
   int n_tiles, tiles;
@@ -78,6 +80,21 @@ __device__ __forceinline__ void load16f(const float* p, float* r) {
     r[4 * i + 2] = v.z;
     r[4 * i + 3] = v.w;
   }
+}
+
+// Barrier `id` over `threads` threads (whole warps) that also returns whether
+// any of them passed pred = true.
+__device__ __forceinline__ bool named_barrier_or(int id, int threads, bool pred) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 q, %1, 0;\n\t"
+      "bar.red.or.pred p, %2, %3, q;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(r)
+      : "r"((uint32_t)pred), "r"(id), "r"(threads)
+      : "memory");
+  return r != 0;
 }
 
 __device__ __forceinline__ void store16bf(__nv_bfloat16* dst, const float* x) {
@@ -203,63 +220,73 @@ qkv_rope(const __grid_constant__ CUtensorMap tx, const __grid_constant__ CUtenso
   } else {
     // ---------------------------------------------- epilogue warps
     // Warp w reads TMEM lanes 32 (w % 4) .. + 31: row 32 (w % 4) + lane of
-    // the tile.
+    // the tile.  Chunk-major: the rotation's cos / sin of a 16-column chunk
+    // are loaded once per row and serve every query and key head of the
+    // tile; the tile's bias sits in shared memory.  (Head-major order with
+    // the bias and the tables read per head left two dependent global loads
+    // in every step and made the epilogue, not the MMAs, the bound when the
+    // contraction is short.)
     const int quarter = warp & 3;
     const uint32_t lq = (uint32_t)(32 * quarter) << 16;
     const int H_tot = a.H_q + 2 * a.H_kv;
+    float* sbias = reinterpret_cast<float*>(smem + ProjSmem::kBias);
+    const int et = threadIdx.x - 64;  // 0..127 over the four epilogue warps
     int j = 0;
     for (int t = blockIdx.x; t < a.tiles; t += gridDim.x, ++j) {
       const int acc = j & 1;
-      if (!__all_sync(0xffffffffu, mbar_wait(acc_full + acc, (uint32_t)(j >> 1) & 1u, abort, a.status)))
-        break;
-      tc_fence_after();
       const int m0 = (t / a.n_tiles) * kBM, n0 = (t % a.n_tiles) * kBN;
+      const bool ok = __all_sync(0xffffffffu,
+                                 mbar_wait(acc_full + acc, (uint32_t)(j >> 1) & 1u, abort, a.status));
+      // The four epilogue warps leave together if any wait gave up (so that
+      // none is left at a barrier); otherwise the previous tile's bias
+      // readers are done, and this tile's bias is staged.
+      if (named_barrier_or(1, 128, !ok)) break;
+      for (int i = et; i < kBN; i += 128)
+        sbias[i] = (a.bias != nullptr && n0 + i < a.n_out) ? __ldg(a.bias + n0 + i) : 0.f;
+      named_barrier(1, 128);
+      tc_fence_after();
       const int r = m0 + 32 * quarter + lane;
       const bool valid = r < a.rows;
       const int b = valid ? r / a.L : 0, tok = valid ? r - b * a.L : 0;
       const uint32_t tacc = tmem + (uint32_t)(acc * kBN) + lq;
-#pragma unroll 1
-      for (int hh = 0; hh < kBN / D; ++hh) {
-        const int gh = n0 / D + hh;  // head index over [q heads | k heads | v heads]
-        if (gh >= H_tot) break;      // the last tile's padding columns
-        __nv_bfloat16* base;
-        int h, H;
-        if (gh < a.H_q) {
-          base = a.q, h = gh, H = a.H_q;
-        } else if (gh < a.H_q + a.H_kv) {
-          base = a.k, h = gh - a.H_q, H = a.H_kv;
+      const int nh = min(kBN / D, H_tot - n0 / D);  // heads in this tile
+      const bool tile_rot = a.rcos != nullptr && n0 / D < a.H_q + a.H_kv;
+#pragma unroll
+      for (int c = 0; c < kHalf; c += 16) {
+        float cs[16], sn[16];
+        if (tile_rot && valid) {
+          load16f(a.rcos + (size_t)tok * kHalf + c, cs);
+          load16f(a.rsin + (size_t)tok * kHalf + c, sn);
         } else {
-          base = a.v, h = gh - a.H_q - a.H_kv, H = a.H_kv;
+#pragma unroll
+          for (int i = 0; i < 16; ++i) cs[i] = 1.f, sn[i] = 0.f;
         }
-        const bool rot = a.rcos != nullptr && gh < a.H_q + a.H_kv;
-        __nv_bfloat16* dst = base + (((size_t)b * H + h) * a.L + tok) * D;
-        const float* bias = a.bias ? a.bias + (size_t)n0 + hh * D : nullptr;
 #pragma unroll 1
-        for (int c = 0; c < kHalf; c += 16) {
+        for (int hh = 0; hh < nh; ++hh) {
+          const int gh = n0 / D + hh;  // head index over [q heads | k heads | v heads]
+          __nv_bfloat16* base;
+          int head, heads;
+          if (gh < a.H_q) {
+            base = a.q, head = gh, heads = a.H_q;
+          } else if (gh < a.H_q + a.H_kv) {
+            base = a.k, head = gh - a.H_q, heads = a.H_kv;
+          } else {
+            base = a.v, head = gh - a.H_q - a.H_kv, heads = a.H_kv;
+          }
+          const bool rot = a.rcos != nullptr && gh < a.H_q + a.H_kv;
+          __nv_bfloat16* dst = base + (((size_t)b * heads + head) * a.L + tok) * D;
           uint32_t ulo[16], uhi[16];
           tmem_ld16(tacc + (uint32_t)(hh * D + c), ulo);
           tmem_ld16(tacc + (uint32_t)(hh * D + kHalf + c), uhi);
           tmem_wait_ld();
           float xl[16], xh[16];
+          const float* bl = sbias + hh * D + c;
 #pragma unroll
           for (int i = 0; i < 16; ++i) {
-            xl[i] = __uint_as_float(ulo[i]);
-            xh[i] = __uint_as_float(uhi[i]);
+            xl[i] = __uint_as_float(ulo[i]) + bl[i];
+            xh[i] = __uint_as_float(uhi[i]) + bl[kHalf + i];
           }
-          if (bias) {
-            float bl[16], bh[16];
-            load16f(bias + c, bl);
-            load16f(bias + kHalf + c, bh);
-#pragma unroll
-            for (int i = 0; i < 16; ++i) {
-              xl[i] += bl[i];
-              xh[i] += bh[i];
-            }
-          }
-          if (rot && valid) {
-            float cs[16], sn[16];
-            load16f(a.rcos + (size_t)tok * kHalf + c, cs);
-            load16f(a.rsin + (size_t)tok * kHalf + c, sn);
+          if (rot) {
 #pragma unroll
             for (int i = 0; i < 16; ++i) {
               const float l = xl[i], u = xh[i];
@@ -354,6 +381,7 @@ cudaError_t launch(const ProjectionProblem& p, cudaStream_t stream) {
   a.rsin = p.rope_sin;
   a.status = p.status;
   a.rows = (int)rows;
+  a.n_out = (int)N;
   a.L = p.L;
   a.H_q = p.H_q;
   a.H_kv = p.H_kv;
