@@ -58,11 +58,11 @@ ATTENTION_TRAFFIC = {
 
 # The same for the projection prologue's qkv_rope launch.
 PROJECTION_TRAFFIC = {
-    "8b-delta": {"bytes": 2 * (862.808320e6 + 389.649664e6),
+    "8b-delta": {"bytes": 2 * (792.638720e6 + 388.922880e6),
                  "note": "ncu capture at batch 1, scaled x2 to the batch-2 launch (traffic grows "
                          "with the token rows)",
                  "profile": "profiles/qkv_rope_8b-projection.md",
-                 "sha1": {"qkv_rope.cu": "e66e05c97c9799a33c647c83133a18d55ef0d0ab",
+                 "sha1": {"qkv_rope.cu": "6f1d6c92e520d53cb8aa0da4741bfc9c36993ebb",
                           "tc_common.cuh": "a896981e1b8e14dfabfd0f26a799d64c0af65a34"}},
 }
 
