@@ -1119,6 +1119,93 @@ def run_projection(args, w):
     return 0
 
 
+def run_layer(args, w):
+    """The whole layer from its input: the Q/K/V projection prologue with the
+    rotary embedding, then the forward (attention, retrieval, gate, memory
+    update) on the heads it wrote, both through the C ABI on one stream.  A
+    step is one pass over the workload's tokens (d_model = H_q d)."""
+    import torch
+
+    from compressive_memory_transformer_segment_b200 import api
+
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    api.load_library()
+    d, H_q, H_kv = w.d_k, w.H_q, w.H_kv
+    dm = H_q * d
+    n_out = (H_q + 2 * H_kv) * d
+    pin = synth.make_projection_inputs(w)
+
+    def host_bf16(a):
+        return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16)
+
+    x = host_bf16(pin["x"]).to(dev)
+    W = host_bf16(pin["w"]).to(dev)
+    bias = torch.from_numpy(pin["bias"]).to(dev)
+    cos, sin = api.rope_tables(w.L, d, device=dev)
+    q = torch.empty((w.B, H_q, w.L, d), dtype=torch.bfloat16, device=dev)
+    k = torch.empty((w.B, H_kv, w.L, d), dtype=torch.bfloat16, device=dev)
+    v = torch.empty((w.B, H_kv, w.L, d), dtype=torch.bfloat16, device=dev)
+    beta = torch.from_numpy(synth.make_beta(w)).to(dev)
+    M0, z0 = api.init_state(w.B, H_kv, d, d, device=dev)
+    dims = api.make_dims(w.B, H_q, H_kv, w.L, d, d, torch.bfloat16)
+    plan = api.plan(dims, w.seg_len, w.rule)
+    ws = torch.empty(plan["workspace_bytes"], dtype=torch.uint8, device=dev)
+    out = torch.empty((w.B, H_q, w.L, d), dtype=torch.bfloat16, device=dev)
+    M1, z1 = torch.empty_like(M0), torch.empty_like(z0)
+    stream = torch.cuda.current_stream(dev)
+    flush = torch.empty(2 * L2_BYTES, dtype=torch.uint8, device=dev) if x.numel() * 2 < 2 * L2_BYTES else None
+
+    def step():
+        api.qkv_project(x, W, bias, cos, sin, H_q, H_kv, d, q=q, k=k, v=v, stream=stream)
+        api.forward(q, k, v, beta, M0, z0, w.seg_len, w.rule, out=out, M_out=M1, z_out=z1,
+                    workspace=ws, stream=stream)
+
+    for _ in range(args.warmup):
+        step()
+    api.sync_status(stream)
+    torch.cuda.synchronize(dev)
+    total = 0.0
+    with ClockSampler(0) as clocks:
+        for _ in range(args.steps):
+            if flush is not None:
+                flush.fill_(1)
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            step()
+            e1.record(stream)
+            torch.cuda.synchronize(dev)
+            total += e0.elapsed_time(e1)
+    api.sync_status(stream)
+    ms = total / args.steps
+    peaks, peak_src = load_peaks()
+    peak = peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
+    flops = 2.0 * w.B * w.L * n_out * dm + configs.algorithmic_flops(w)
+    achieved = flops / (ms / 1000.0) / 1e12
+    line = {
+        "metric": "Infini-attention layer (Q/K/V projection + rotary embedding + forward) tokens/s "
+                  "on 1 B200",
+        "value": w.B * w.L / (ms / 1000.0), "unit": "tokens/s", "n_gpus": 1, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded Philox N(0,1) x, N(0,1/d_model) weights, U(-r,r) beta)",
+        "config": {"workload": f"{w.name} layer", "B": w.B, "L": w.L, "d_model": dm, "H_q": H_q,
+                   "H_kv": H_kv, "d": d, "seg_len": w.seg_len, "rule": w.rule,
+                   "l2": ("L2 flushed (256 MiB write) between timed steps"
+                          if flush is not None else "inputs larger than L2")},
+        "clocks": clocks.summary(),
+        "e2e": None,
+        "gpu_launches": (1 + plan["launches"]) * args.steps,
+        "roofline": {"bound": "tensor", "kernel": "whole layer (projection GEMM + attention + scan)",
+                     "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
+                     "peak_source": f"{peak_src} bf16 (burst)", "traffic": None,
+                     "algorithmic_flops_per_step": flops},
+        "cpu_baseline": None,
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -1155,6 +1242,9 @@ def main():
     ap.add_argument("--projection", action="store_true",
                     help="the Q/K/V projection + rotary embedding prologue of the workload's "
                          "shape (d_model = H_q d)")
+    ap.add_argument("--layer", action="store_true",
+                    help="the whole layer from its input: the projection prologue, then the "
+                         "forward on the heads it wrote")
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "ours":
         args.warmup = 3
@@ -1175,6 +1265,8 @@ def main():
         return run_backward(args, w)
     if args.projection:
         return run_projection(args, w)
+    if args.layer:
+        return run_layer(args, w)
     if args.seq_parallel:
         return run_seq_parallel(args, w)
     return run_gpu(args, w)

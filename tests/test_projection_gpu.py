@@ -143,3 +143,35 @@ def test_projection_rejects_unsupported_shapes(cuda_lib):
     with pytest.raises(api.InfiniError) as exc:
         api.qkv_project(x, wq, None, None, None, 2, 1, 32)
     assert exc.value.status == api.ERR_UNSUPPORTED
+
+
+def test_projection_then_forward_matches_the_oracle_chain(cuda_lib):
+    """The prologue feeds the layer: x -> (q, k, v) -> forward on the GPU
+    against the oracle's projection (rounded to bf16, the prologue's output
+    type) followed by the oracle's forward.  A bf16 rounding tie resolved
+    differently on the two sides moves an output by far less than the bf16
+    output tolerance."""
+    api = cuda_lib
+    w = W["tiny"].with_(name="chain", dtype="bf16", B=1, H_q=4, H_kv=2, L=320, d_k=64, d_v=64,
+                        seg_len=128, rule="delta")
+    inp = synth.make_projection_inputs(w, 256)
+    x, wq = to_torch(inp["x"], "bf16"), to_torch(inp["w"], "bf16")
+    b_t = torch.from_numpy(inp["bias"]).cuda()
+    cos, sin = api.rope_tables(w.L, 64)
+    q, k, v = api.qkv_project(x, wq, b_t, cos, sin, w.H_q, w.H_kv, 64)
+    beta = torch.from_numpy(synth.make_beta(w)).cuda()
+    M0, z0 = api.init_state(w.B, w.H_kv, 64, 64)
+    out, M, z = api.forward(q, k, v, beta, M0, z0, w.seg_len, w.rule)
+    api.sync_status()
+    c64, s64 = oracle.rope_tables(w.L, 64)
+    rq, rk, rv = oracle.qkv_project_rope(synth.as_float64(inp["x"], "bf16"),
+                                         synth.as_float64(inp["w"], "bf16"),
+                                         inp["bias"].astype(np.float64), c64, s64, w.H_q, w.H_kv, 64)
+    rq, rk, rv = (synth.as_float64(synth.round_bf16_bits(t.astype(np.float32)), "bf16")
+                  for t in (rq, rk, rv))
+    ro, rM, rz = oracle.infini_attention_forward(
+        rq, rk, rv, synth.make_beta(w).astype(np.float64), np.zeros((w.B, w.H_kv, 64, 64)),
+        np.zeros((w.B, w.H_kv, 64)), w.seg_len, w.rule)
+    assert float(np.max(np.abs(out.float().cpu().numpy() - ro))) <= 2e-2
+    scale = float(np.max(np.abs(rM)))
+    assert float(np.max(np.abs(M.cpu().numpy() - rM))) <= 1e-3 * scale
