@@ -76,3 +76,23 @@ def test_decode_bytes_per_segment_closed_form():
             per_q = d * e + d * e + 4
             total += w.B * (w.H_kv * per_kv + w.H_q * per_q)
         assert bench.decode_bytes_per_segment(w) == total
+
+
+def test_bench_reference_arm_runs_on_the_host():
+    """`bench.py --impl reference` (the float64 oracle on the host cores)
+    prints one JSON line in the bench's format, with no GPU."""
+    import json
+    import os
+    import subprocess
+    import sys
+
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    res = subprocess.run([sys.executable, os.path.join(root, "bench.py"), "--impl", "reference",
+                          "--config", "tiny", "--steps", "1", "--warmup", "1",
+                          "--reference-budget", "1"],
+                         capture_output=True, text=True, timeout=300, cwd=root)
+    assert res.returncode == 0, res.stderr[-2000:]
+    line = json.loads(res.stdout.strip().splitlines()[-1])
+    assert line["impl"] == "reference" and line["value"] > 0
+    assert line["unit"] == "tokens/s" and line["e2e"]["h2d_bytes_per_step"] == 0
+    assert line["cpu_baseline"]["kind"] == "oracle"
